@@ -1,0 +1,141 @@
+"""Seeded synthetic jagged batches for SLA HSTU attention.
+
+This module only draws inputs: sequence lengths, candidate counts and the
+bf16 tensors q, k, v, dout.  It holds none of the attention arithmetic; the
+oracle (test infrastructure) and the CUDA library both consume what it
+returns, so the two are fed bit-identical inputs.
+
+Shapes follow the workloads the ULTRA-HSTU pages describe: user histories of
+3K-16K events ("Bending the Scaling Law Curve in Large-Scale Recommendation
+Systems", section 5.1.1; 16K production sequences, section 1), a contextual
+prefix at the start and candidate targets at the end (section 3, "Input";
+TorchEasyRec "ULTRA HSTU" docs), 4 heads of 128 (TorchEasyRec example config,
+embedding_dim 512 / num_heads 4 / attention_dim 128).  The industrial logs and
+KuaiRand the pages measure on are not available; these draws stand in for
+them.
+
+Recipe (fixed): lengths from ``numpy.random.default_rng(1000 + index)``;
+tensors from ``torch.Generator('cpu').manual_seed(1000 + index)`` drawn as
+fp32 N(0, 1) in the order q, k, v, dout, then rounded to bf16.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Optional
+
+import numpy as np
+import torch
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    index: int                 # 1-based; seeds derive from it
+    name: str
+    B: int
+    H: int
+    d: int
+    K1: int
+    K2: int
+    contextual_len: int
+    num_targets: int
+    alpha: float
+    N: float
+    fwd_only: bool = False
+    description: str = ""
+
+    @property
+    def seed(self) -> int:
+        return 1000 + self.index
+
+
+WORKLOADS = {
+    "tiny": Workload(1, "tiny", B=4, H=2, d=32, K1=32, K2=16, contextual_len=4,
+                     num_targets=8, alpha=1.0 / math.sqrt(32), N=256.0,
+                     description="4 seqs, L~U{32..256}, 2x32 heads"),
+    "mid": Workload(2, "mid", B=32, H=4, d=128, K1=256, K2=64, contextual_len=16,
+                    num_targets=16, alpha=1.0 / math.sqrt(128), N=4096.0,
+                    description="32 seqs, L~U{1024..4096}, 4x128 heads"),
+    "hist16k": Workload(3, "hist16k", B=8, H=4, d=128, K1=1024, K2=128,
+                        contextual_len=32, num_targets=64,
+                        alpha=1.0 / math.sqrt(128), N=16384.0,
+                        description="8 seqs: 4x16384 + 4x16384*U(0.25,1), total<=98304"),
+    "infer": Workload(4, "infer", B=64, H=4, d=128, K1=512, K2=128,
+                      contextual_len=32, num_targets=512,
+                      alpha=1.0 / math.sqrt(128), N=8704.0, fwd_only=True,
+                      description="64 seqs of 8192 history + 512 candidates"),
+    "stu": Workload(5, "stu", B=16, H=4, d=128, K1=1024, K2=128,
+                    contextual_len=32, num_targets=64,
+                    alpha=1.0 / math.sqrt(128), N=16384.0,
+                    description="6-layer STU stack, L~U{4096..16384}"),
+}
+
+HIST16K_TOKEN_BUDGET = 96 * 1024
+
+
+def draw_lengths(w: Workload) -> np.ndarray:
+    """Total per-sequence lengths (contextual prefix and candidates included)."""
+    rng = np.random.default_rng(w.seed)
+    if w.name == "tiny":
+        return rng.integers(32, 256, size=w.B, endpoint=True).astype(np.int64)
+    if w.name == "mid":
+        return rng.integers(1024, 4096, size=w.B, endpoint=True).astype(np.int64)
+    if w.name == "hist16k":
+        pinned = np.full(4, 16384, dtype=np.int64)
+        while True:  # redraw the free half until the batch fits the token budget
+            free = np.floor(16384 * rng.uniform(0.25, 1.0, size=4)).astype(np.int64)
+            if pinned.sum() + free.sum() <= HIST16K_TOKEN_BUDGET:
+                return np.concatenate([pinned, free])
+    if w.name == "infer":
+        return np.full(w.B, 8192 + 512, dtype=np.int64)
+    if w.name == "stu":
+        return rng.integers(4096, 16384, size=w.B, endpoint=True).astype(np.int64)
+    raise KeyError(w.name)
+
+
+def offsets_from_lengths(lengths) -> np.ndarray:
+    lengths = np.asarray(lengths, dtype=np.int64)
+    return np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64)
+
+
+def draw_tensors(T: int, H: int, d: int, seed: int, n: int = 4):
+    """n bf16 tensors [T, H, d] ~ N(0,1) in the order q, k, v, dout."""
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    return [torch.randn((T, H, d), generator=g, dtype=torch.float32).to(torch.bfloat16)
+            for _ in range(n)]
+
+
+@dataclasses.dataclass
+class Batch:
+    workload: Workload
+    lengths: np.ndarray          # [B] int64
+    seq_offsets: np.ndarray      # [B+1] int64
+    num_targets: np.ndarray      # [B] int64
+    q: torch.Tensor              # bf16 [T, H, d] (CPU)
+    k: torch.Tensor
+    v: torch.Tensor
+    dout: Optional[torch.Tensor]
+
+    @property
+    def T(self) -> int:
+        return int(self.seq_offsets[-1])
+
+
+def make_batch(w: Workload, lengths=None, num_targets=None, seed: Optional[int] = None,
+               with_dout: bool = True) -> Batch:
+    """Draw the workload's batch.  ``lengths``/``num_targets``/``seed`` override
+    the workload's own draw (used for small parity and edge cases)."""
+    lengths = draw_lengths(w) if lengths is None else np.asarray(lengths, dtype=np.int64)
+    if num_targets is None:
+        nt = np.minimum(np.full(len(lengths), w.num_targets, dtype=np.int64), lengths)
+    else:
+        nt = np.broadcast_to(np.asarray(num_targets, dtype=np.int64), lengths.shape).copy()
+    offs = offsets_from_lengths(lengths)
+    T = int(offs[-1])
+    ts = draw_tensors(T, w.H, w.d, w.seed if seed is None else seed, n=4 if with_dout else 3)
+    return Batch(w, lengths, offs, nt, ts[0], ts[1], ts[2], ts[3] if with_dout else None)
+
+
+def with_params(w: Workload, **kw) -> Workload:
+    """A copy of a workload with some fields changed (edge cases)."""
+    return dataclasses.replace(w, **kw)
