@@ -1,0 +1,392 @@
+#!/usr/bin/env python
+"""SLA HSTU attention fwd+bwd throughput on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload hist16k]
+    python bench.py --impl reference ...        # the CPU oracle as the reference arm
+
+A step is one forward and one backward pass (work list, attention kernels,
+dq conversion) over one synthetic jagged batch.  The metric is TFLOP/s counted
+over unmasked (row, key) pairs: 4d FLOPs per pair per head forward, 10d
+backward.  Inputs (q, k, v, dout: 4 x 403 MB for the 16K workload) exceed the
+126 MB L2, so no flush is needed between steps.  N > 1 runs one process per
+GPU (torchrun), each on its own batch of the same shape (weak scaling, no
+collective on the data path); time is the max over ranks.
+
+Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_hstu_attention_b200 import flops as F  # noqa: E402
+from workloads import WORKLOADS, make_batch  # noqa: E402
+
+METRIC = "SLA HSTU attn fwd+bwd TFLOP/s (unmasked pairs), % of B200 BF16 peak"
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0}
+KERNEL_SOURCES = {"fwd": "sparse_hstu_attention_b200/csrc/fwd_mma.cu",
+                  "bwd": "sparse_hstu_attention_b200/csrc/bwd_mma.cu"}
+KERNEL_NAMES = {"fwd": "fwd_mma_kernel", "bwd": "bwd_mma_kernel"}
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def _sha1(path):
+    with open(os.path.join(ROOT, path), "rb") as f:
+        return hashlib.sha1(f.read()).hexdigest()
+
+
+def _traffic(which, workload):
+    """DRAM bytes per launch from a committed ncu capture, if the kernel source
+    is unchanged since it was taken."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(f"{KERNEL_NAMES[which]}/{workload}")
+    if not e or e.get("source_sha1") != _sha1(KERNEL_SOURCES[which]):
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while active."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.file = None
+
+    def __enter__(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.dev)], stdout=self.file,
+                stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.file is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.file.seek(0)
+        rows = [l.strip().split(", ") for l in self.file if l.strip()]
+        os.unlink(self.file.name)
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                smax.append(float(r[2]))
+                power.append(float(r[3]))
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        pmax = max(power) if power else 0
+        loaded = [s for s, p in zip(sm, power) if p >= 0.5 * pmax] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": pmax}
+
+
+def _setup_dist(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and args.impl == "ours":
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def _sample_cost_flops(p, rows, d, H, row_pairs, key_pairs):
+    """Metric-equivalent FLOPs of an oracle sample: forward on the sampled rows
+    plus the backward split evenly between the sampled rows (dq) and the same
+    tokens taken as keys (dk, dv)."""
+    rp = float(row_pairs[rows].sum())
+    kp = float(key_pairs[rows].sum())
+    return H * d * (4.0 * rp + 10.0 * 0.5 * (rp + kp)), rp
+
+
+def _oracle_sample(batch, n_tokens, seed):
+    import oracle
+    p = oracle.Problem.from_batch(batch)
+    rng = np.random.default_rng(seed)
+    rows = np.sort(rng.choice(batch.T, size=min(n_tokens, batch.T), replace=False))
+    t0 = time.perf_counter()
+    p.fwd(batch.q, batch.k, batch.v, rows=rows)
+    p.bwd_dq(batch.q, batch.k, batch.v, batch.dout, rows=rows)
+    p.bwd_dkv(batch.q, batch.k, batch.v, batch.dout, keys=rows)
+    return time.perf_counter() - t0, rows
+
+
+def _pair_tables(batch):
+    w = batch.workload
+    return F.pairs_per_token(batch.lengths, batch.num_targets, w.contextual_len, w.K1, w.K2)
+
+
+def cpu_baseline(batch, target_s=15.0):
+    """The oracle, as it stands, on a bounded random sample of the workload's tokens."""
+    w = batch.workload
+    rp, kp = _pair_tables(batch)
+    n = 64
+    t, _ = _oracle_sample(batch, n, seed=7)
+    n = int(min(batch.T, max(64, n * target_s / max(t, 1e-3))))
+    t, rows = _oracle_sample(batch, n, seed=8)
+    fl, _ = _sample_cost_flops(None, rows, w.d, w.H, rp, kp)
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    cores = int(os.environ.get("OMP_NUM_THREADS", cores))
+    return {"value": fl / t / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"{len(rows)} random tokens of the {w.name} batch: forward and dq for them "
+                      f"as rows, dk/dv for them as keys; fp64 C loops; {t:.1f} s",
+            "seconds": t}
+
+
+def run_reference(args):
+    """The oracle timed on the host cores as the reference arm (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = WORKLOADS[args.workload]
+    batch = make_batch(w)
+    rp, kp = _pair_tables(batch)
+    per_step_s = max(0.5, min(10.0, 150.0 / (args.steps + args.warmup)))
+    t, _ = _oracle_sample(batch, 64, seed=1)
+    n = int(min(batch.T, max(16, 64 * per_step_s / max(t, 1e-3))))
+    total_t, total_fl = 0.0, 0.0
+    for s in range(args.warmup + args.steps):
+        t, rows = _oracle_sample(batch, n, seed=100 + s)
+        if s >= args.warmup:
+            fl, _ = _sample_cost_flops(None, rows, w.d, w.H, rp, kp)
+            total_t += t
+            total_fl += fl
+    value = total_fl / total_t / 1e12
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    cores = int(os.environ.get("OMP_NUM_THREADS", cores))
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "impl": "reference",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total_t / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": _config(w, batch),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{n} random tokens per step of the {w.name} batch"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def _config(w, batch):
+    pairs = F.total_pairs(batch.lengths, batch.num_targets, w.contextual_len, w.K1, w.K2)
+    in_bytes = 4 * batch.T * w.H * w.d * 2
+    return {"workload": w.name, "B": int(len(batch.lengths)), "T": int(batch.T), "H": w.H,
+            "d": w.d, "K1": w.K1, "K2": w.K2, "contextual_len": w.contextual_len,
+            "num_targets": w.num_targets, "N": w.N, "alpha": w.alpha,
+            "lengths": [int(x) for x in batch.lengths], "pairs_per_head": pairs,
+            "l2": f"inputs {in_bytes / 1e6:.0f} MB > 126 MB L2; no flush"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="hist16k", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import sparse_hstu_attention_b200 as sla
+
+    world, rank, local = _setup_dist(args)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = WORKLOADS[args.workload]
+    batch = make_batch(w, seed=w.seed + 7919 * rank)
+    T, H, d = batch.T, w.H, w.d
+    pairs = F.total_pairs(batch.lengths, batch.num_targets, w.contextual_len, w.K1, w.K2)
+    fl_f, fl_b = F.fwd_flops(pairs, H, d), (0.0 if w.fwd_only else F.bwd_flops(pairs, H, d))
+
+    offs = torch.tensor(batch.seq_offsets, dtype=torch.int32, device=dev)
+    nts = torch.tensor(batch.num_targets, dtype=torch.int32, device=dev)
+    q, k, v = (t.to(dev) for t in (batch.q, batch.k, batch.v))
+    dout = batch.dout.to(dev)
+    out = torch.empty_like(q)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    ws_f = torch.empty(sla.hstu_sla_workspace_bytes(0, T, len(batch.lengths), H, d),
+                       dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(sla.hstu_sla_workspace_bytes(1, T, len(batch.lengths), H, d),
+                       dtype=torch.uint8, device=dev)
+    kw = dict(contextual_len=w.contextual_len, K1=w.K1, K2=w.K2, alpha=w.alpha, N=w.N,
+              max_seq_len=int(batch.lengths.max()))
+    stream = torch.cuda.current_stream()
+
+    def new_events(n):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        for e in evs:
+            e.record(stream)  # force creation of the underlying cudaEvent
+        return evs
+
+    K = args.steps
+    fb, fe, bb, be = new_events(K), new_events(K), new_events(K), new_events(K)
+
+    def step(i=None, e2e=None):
+        evf = (fb[i], fe[i]) if i is not None else None
+        evb = (bb[i], be[i]) if i is not None else None
+        sla.hstu_sla_fwd(q, k, v, offs, nts, out=out, workspace=ws_f, events=evf, **kw)
+        if not w.fwd_only:
+            sla.hstu_sla_bwd(dout, q, k, v, offs, nts, dq=dq, dk=dk, dv=dv, workspace=ws_b,
+                             events=evb, **kw)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    status = max(sla.hstu_sla_get_error(ws_f), 0 if w.fwd_only else sla.hstu_sla_get_error(ws_b))
+    if status != 0:
+        raise RuntimeError(f"device status {status}")
+
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        t_start.record(stream)
+        for i in range(K):
+            step(i)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+    ms = t_start.elapsed_time(t_end)
+    if world > 1:
+        tt = torch.tensor([ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        ms = float(tt.item())
+    ms_step = ms / K
+    value = world * (fl_f + fl_b) / (ms_step * 1e-3) / 1e12
+    fwd_ms = sum(fb[i].elapsed_time(fe[i]) for i in range(K)) / K
+    bwd_ms = 0.0 if w.fwd_only else sum(bb[i].elapsed_time(be[i]) for i in range(K)) / K
+
+    # end to end through the public API from pinned host buffers
+    hq, hk, hv, hdo = (t.pin_memory() for t in (batch.q, batch.k, batch.v, batch.dout))
+    hoffs = torch.tensor(batch.seq_offsets, dtype=torch.int32).pin_memory()
+    hnts = torch.tensor(batch.num_targets, dtype=torch.int32).pin_memory()
+    hout = [torch.empty(q.shape, dtype=torch.bfloat16).pin_memory() for _ in range(4)]
+    ins = [(q, hq), (k, hk), (v, hv), (dout, hdo), (offs, hoffs), (nts, hnts)]
+    outs = [(hout[0], out), (hout[1], dq), (hout[2], dk), (hout[3], dv)]
+    if w.fwd_only:
+        ins, outs = ins[:3] + ins[4:], outs[:1]
+    h2d = sum(h.numel() * h.element_size() for _, h in ins)
+    d2h = sum(h.numel() * h.element_size() for h, _ in outs)
+
+    def e2e_step():
+        for dst, src in ins:
+            dst.copy_(src, non_blocking=True)
+        step()
+        for dst, src in outs:
+            dst.copy_(src, non_blocking=True)
+
+    E = max(1, args.e2e_steps)
+    e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(E):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / E
+    if world > 1:
+        tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+
+    if rank != 0:
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+        return
+
+    peaks, peak_src = _peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    dom = "bwd" if bwd_ms > fwd_ms else "fwd"
+    dom_ms = bwd_ms if dom == "bwd" else fwd_ms
+    dom_fl = fl_b if dom == "bwd" else fl_f
+    achieved = dom_fl / (dom_ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16, jagged lengths drawn per workload recipe)",
+        "config": _config(w, batch),
+        "pct_of_peak": 100.0 * value / world / peak,
+        "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
+        "fwd_tflops": fl_f / (fwd_ms * 1e-3) / 1e12 if fwd_ms else None,
+        "bwd_tflops": fl_b / (bwd_ms * 1e-3) / 1e12 if bwd_ms else None,
+        "roofline": {"bound": "tensor", "kernel": KERNEL_NAMES[dom], "achieved": achieved,
+                     "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_source": f"bf16_tflops (burst) of {peak_src}",
+                     "traffic": _traffic(dom, w.name),
+                     "algorithmic_flops_per_launch": dom_fl},
+        "e2e": {"value": world * (fl_f + fl_b) / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": K * (2 if w.fwd_only else 5),
+        "clocks": clocks.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(batch)
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

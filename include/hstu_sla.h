@@ -1,0 +1,153 @@
+/*
+ * hstu_sla.h -- C ABI of the B200 (sm_100a) SLA HSTU attention library.
+ *
+ * The operation is HSTU's pointwise-SiLU attention ("Bending the Scaling Law
+ * Curve in Large-Scale Recommendation Systems", section 3, Eq. 3; HSTU notes
+ * "Actions Speak Louder than Words", section 2.4, Eq. 2) under the
+ * Semi-Local Attention mask (same paper, section 4.2.1, Eq. 7), over a jagged
+ * batch.  Per sequence b of length L (contextual prefix first, num_targets
+ * candidates last, Lh = L - num_targets history tokens) and per head:
+ *
+ *     out_i = (1/N) * sum_j M(i,j) * SiLU(alpha * q_i . k_j) * v_j
+ *
+ * with K2eff = max(K2, contextual_len) (TorchEasyRec "ULTRA HSTU" docs,
+ * Semi-Local Attention bullet) and 0-based positions i, j in the sequence:
+ *     history row i < Lh:   M = [j <= i] and ([i - j < K1] or [j < K2eff])
+ *     candidate row i >= Lh: M = ([j < Lh] and ([Lh - j < K1] or [j < K2eff]))
+ *                                or [j == i]
+ * (candidates see the history and themselves, never each other: HSTU notes,
+ * section 2.6, M-FALCON mask figure).  K1 and K2 are taken literally: K1 = 0
+ * means no local window; "full causal" is K1 >= max length.
+ *
+ * The backward produces dq, dk, dv of  L = sum(out * dout)  (the attention
+ * step of Listing 1's attention_backward(dattn, q, k, v)).
+ *
+ * Conventions for every entry point:
+ *  - Pointers named "device" are CUDA device pointers; the caller owns every
+ *    buffer (the library allocates nothing and keeps no state between calls).
+ *  - Tensors are bf16 [T, H, d] with the H*d values of one token contiguous
+ *    (head h at element offset h*d) and a per-token row stride in ELEMENTS,
+ *    so q/k/v may be strided views into a fused projection buffer.  Row
+ *    strides must be multiples of 8 elements and base pointers 16-byte
+ *    aligned.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream).  They return HSTU_SLA_OK or a negative code; no C++
+ *    exception crosses the ABI.  Argument errors are detected on the host and
+ *    nothing is launched.  Errors in the device-resident offsets/targets are
+ *    detected on the device: the kernels then skip all work and the error is
+ *    reported by hstu_sla_get_error().  Kernels never trap.
+ *  - Supported head_dim d: 32, 64, 128.  max_seq_len bounds every length.
+ */
+#ifndef HSTU_SLA_H_
+#define HSTU_SLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st* hstu_stream_t; /* identical to cudaStream_t */
+
+enum {
+  HSTU_SLA_OK = 0,
+  HSTU_SLA_ERR_INVALID_ARG = -1,  /* null pointer, bad size, misalignment */
+  HSTU_SLA_ERR_UNSUPPORTED = -2,  /* head_dim or device not supported */
+  HSTU_SLA_ERR_CUDA = -3,         /* a CUDA runtime call failed */
+  HSTU_SLA_ERR_BAD_INPUT = -4,    /* device-side check of offsets/targets failed */
+  HSTU_SLA_ERR_WORKSPACE = -5,    /* workspace missing, too small or misaligned */
+  HSTU_SLA_ERR_TIMEOUT = -6       /* a bounded device-side wait gave up */
+};
+
+/* Forward problem.  All integer fields are host values. */
+typedef struct {
+  int32_t B;                    /* number of sequences, >= 1 */
+  int32_t H;                    /* heads, >= 1 */
+  int32_t d;                    /* head_dim: 32, 64 or 128 */
+  int64_t total_tokens;         /* T = seq_offsets[B] (host copy, for sizing) */
+  int32_t max_seq_len;          /* >= every sequence length (device-checked) */
+  const int32_t* seq_offsets;   /* device [B+1], offsets[0] = 0, non-decreasing */
+  const int32_t* num_targets;   /* device [B], 0 <= num_targets[b] <= len_b; NULL = all 0 */
+  int32_t contextual_len;       /* >= 0; K2eff = max(K2, contextual_len) */
+  int32_t K1;                   /* local window (keys incl. self), >= 0 */
+  int32_t K2;                   /* global prefix, >= 0 */
+  float alpha;                  /* scale inside SiLU */
+  float N;                      /* normaliser, > 0 */
+  const void* q;                /* device bf16 [T, H, d] */
+  const void* k;
+  const void* v;
+  int64_t q_row_stride;         /* elements between consecutive tokens (>= H*d) */
+  int64_t k_row_stride;
+  int64_t v_row_stride;
+  void* out;                    /* device bf16 [T, H, d], written by hstu_sla_fwd */
+  int64_t out_row_stride;
+  /* Optional timing hooks: cudaEvent_t handles recorded on `stream` just
+   * before and just after the main attention kernel (not the work-list or
+   * conversion kernels).  NULL = not recorded. */
+  void* event_begin;
+  void* event_end;
+} hstu_sla_fwd_params;
+
+/* Backward problem: the forward problem plus dout and the three gradients. */
+typedef struct {
+  hstu_sla_fwd_params fwd;      /* fwd.out and fwd.out_row_stride are ignored */
+  const void* dout;             /* device bf16 [T, H, d] */
+  int64_t dout_row_stride;
+  void* dq;                     /* device bf16 [T, H, d], written */
+  void* dk;
+  void* dv;
+  int64_t dq_row_stride;
+  int64_t dk_row_stride;
+  int64_t dv_row_stride;
+} hstu_sla_bwd_params;
+
+#define HSTU_SLA_WS_FWD 0
+#define HSTU_SLA_WS_BWD 1
+
+/* Bytes of device workspace hstu_sla_fwd (which = HSTU_SLA_WS_FWD) or
+ * hstu_sla_bwd (HSTU_SLA_WS_BWD) needs for a batch of total_tokens tokens in
+ * B sequences.  The workspace must be 256-byte aligned; the backward one holds
+ * an fp32 dq accumulator of T*H*d floats.  Returns 0 on invalid arguments. */
+size_t hstu_sla_workspace_bytes(int which, int64_t total_tokens, int32_t B, int32_t H,
+                                int32_t d);
+
+/* Forward: writes p->out.  Enqueues a work-list kernel (validates offsets and
+ * targets on the device, enumerates the non-empty query tiles) and the
+ * attention kernel; nothing returns to the host. */
+int hstu_sla_fwd(const hstu_sla_fwd_params* p, void* workspace, size_t workspace_bytes,
+                 hstu_stream_t stream);
+
+/* Backward: writes p->dq, p->dk, p->dv (bf16).  Key-tile-parallel: dk/dv are
+ * accumulated on chip without atomics; dq is reduced in the fp32 workspace and
+ * converted at the end. */
+int hstu_sla_bwd(const hstu_sla_bwd_params* p, void* workspace, size_t workspace_bytes,
+                 hstu_stream_t stream);
+
+/* Test hook: the number of visible keys of every token as the forward
+ * kernels enumerate them (row_counts, device int64 [T]) and the number of
+ * query rows that see every token as a key, as the backward kernels
+ * enumerate them (key_counts, device int64 [T]).  Either may be NULL.
+ * Counts are per head (identical for all heads). */
+int hstu_sla_count_pairs(const hstu_sla_fwd_params* p, int64_t* row_counts,
+                         int64_t* key_counts, void* workspace, size_t workspace_bytes,
+                         hstu_stream_t stream);
+
+/* Synchronises `stream` and returns the device-side status recorded in
+ * `workspace` by the last call that used it (HSTU_SLA_OK, HSTU_SLA_ERR_BAD_INPUT
+ * or HSTU_SLA_ERR_TIMEOUT), or HSTU_SLA_ERR_CUDA.  The status is cleared by the
+ * next hstu_sla_fwd / hstu_sla_bwd / hstu_sla_count_pairs call. */
+int hstu_sla_get_error(const void* workspace, hstu_stream_t stream);
+
+/* Static message for a status code. */
+const char* hstu_sla_strerror(int code);
+
+/* Library ABI version (major * 100 + minor). */
+int hstu_sla_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HSTU_SLA_H_ */

@@ -61,10 +61,11 @@ def _load():
             lib.oracle_sla_visible.argtypes = [i64] * 7 + [ctypes.c_int]
             lib.oracle_sla_visible.restype = ctypes.c_int
             lib.oracle_sla_row_counts.argtypes = [vp, vp]
+            lib.oracle_sla_key_counts.argtypes = [vp, vp]
             lib.oracle_sla_fwd_rows.argtypes = [vp, vp, vp, vp, vp, i64, vp]
             lib.oracle_sla_bwd_dq_rows.argtypes = [vp, vp, vp, vp, vp, vp, i64, vp]
             lib.oracle_sla_bwd_dkv_keys.argtypes = [vp, vp, vp, vp, vp, vp, i64, vp, vp]
-            for f in ("oracle_sla_row_counts", "oracle_sla_fwd_rows",
+            for f in ("oracle_sla_row_counts", "oracle_sla_key_counts", "oracle_sla_fwd_rows",
                       "oracle_sla_bwd_dq_rows", "oracle_sla_bwd_dkv_keys"):
                 getattr(lib, f).restype = None
             _lib = lib
@@ -111,6 +112,11 @@ class Problem:
     def row_counts(self) -> np.ndarray:
         out = np.zeros(self.T, np.int64)
         _load().oracle_sla_row_counts(ctypes.byref(self._cfg), out.ctypes.data)
+        return out
+
+    def key_counts(self) -> np.ndarray:
+        out = np.zeros(self.T, np.int64)
+        _load().oracle_sla_key_counts(ctypes.byref(self._cfg), out.ctypes.data)
         return out
 
     def fwd(self, q, k, v, rows=None) -> np.ndarray:

@@ -116,6 +116,19 @@ void oracle_sla_row_counts(const oracle_cfg* c, int64_t* counts) {
   }
 }
 
+/* Number of rows that see every token as a key (the same for every head): [T]. */
+void oracle_sla_key_counts(const oracle_cfg* c, int64_t* counts) {
+  int64_t T = c->offsets[c->B];
+#pragma omp parallel for schedule(dynamic, 64)
+  for (int64_t t = 0; t < T; ++t) {
+    int b = seq_of(c->offsets, c->B, t);
+    int64_t s0 = c->offsets[b], L = c->offsets[b + 1] - s0, j = t - s0, n = 0;
+    for (int64_t i = 0; i < L; ++i)
+      n += oracle_sla_visible(L, nt_of(c, b), c->contextual_len, c->K1, c->K2, i, j, c->flags);
+    counts[t] = n;
+  }
+}
+
 /* out[r, h, :] = (1/N) sum_j M(i,j) SiLU(alpha q_i.k_j) v_j for the tokens rows[r]. */
 void oracle_sla_fwd_rows(const oracle_cfg* c, const double* q, const double* k,
                          const double* v, const int64_t* rows, int64_t n_rows,

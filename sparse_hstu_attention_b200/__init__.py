@@ -1,0 +1,201 @@
+"""SLA HSTU attention on B200 (sm_100a).
+
+A thin binding over the C ABI of ``libhstu_sla.so`` (include/hstu_sla.h):
+every step of the attention runs in the library's CUDA kernels; this module
+only checks tensor shapes, allocates outputs / workspace with PyTorch and
+marshals pointers.  There is no CPU or PyTorch fallback: if the library is
+missing, the calls raise.
+
+    out = hstu_sla_fwd(q, k, v, seq_offsets, num_targets, contextual_len=32,
+                       K1=1024, K2=128, alpha=128 ** -0.5, N=16384.0)
+    dq, dk, dv = hstu_sla_bwd(dout, q, k, v, seq_offsets, num_targets, ...)
+
+q, k, v, dout: CUDA bf16 tensors [T, H, d] whose last two dims are dense
+(row stride free, so views into a fused [T, 4*H*d] projection work);
+seq_offsets: CUDA int32 [B+1]; num_targets: CUDA int32 [B] or None.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional
+
+import torch
+
+from . import _abi
+from ._abi import LibraryMissing  # noqa: F401
+
+__all__ = ["hstu_sla_fwd", "hstu_sla_bwd", "hstu_sla_workspace_bytes", "hstu_sla_count_pairs",
+           "hstu_sla_get_error", "hstu_sla_strerror", "SLAError", "SLAAttention",
+           "sla_attention"]
+
+
+class SLAError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {hstu_sla_strerror(code)} (status {code})")
+
+
+def hstu_sla_strerror(code: int) -> str:
+    return _abi.strerror(code)
+
+
+def _check(code: int, where: str):
+    if code != _abi.OK:
+        raise SLAError(code, where)
+
+
+def _stream_ptr(stream) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return int(s.cuda_stream)
+
+
+def _row_stride(t: torch.Tensor, name: str, H: int, d: int) -> int:
+    if t.dtype != torch.bfloat16 or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA bfloat16 tensor")
+    if t.dim() != 3 or t.shape[1] != H or t.shape[2] != d:
+        raise ValueError(f"{name} must be [T, {H}, {d}], got {tuple(t.shape)}")
+    if t.stride(2) != 1 or t.stride(1) != d:
+        raise ValueError(f"{name}: heads and head_dim must be dense (stride (*, {d}, 1))")
+    return t.stride(0)
+
+
+def hstu_sla_workspace_bytes(which: int, total_tokens: int, B: int, H: int, d: int) -> int:
+    return int(_abi.load().hstu_sla_workspace_bytes(which, total_tokens, B, H, d))
+
+
+def _fwd_params(q, k, v, seq_offsets, num_targets, contextual_len, K1, K2, alpha, N,
+                max_seq_len, events=None) -> _abi.FwdParams:
+    T, H, d = q.shape
+    if seq_offsets.dtype != torch.int32 or not seq_offsets.is_cuda:
+        raise TypeError("seq_offsets must be a CUDA int32 tensor [B+1]")
+    if num_targets is not None and (num_targets.dtype != torch.int32 or not num_targets.is_cuda):
+        raise TypeError("num_targets must be a CUDA int32 tensor [B] or None")
+    B = seq_offsets.numel() - 1
+    p = _abi.FwdParams()
+    p.B, p.H, p.d = B, H, d
+    p.total_tokens = T
+    p.max_seq_len = T if max_seq_len is None else int(max_seq_len)
+    p.seq_offsets = seq_offsets.data_ptr()
+    p.num_targets = num_targets.data_ptr() if num_targets is not None else None
+    p.contextual_len, p.K1, p.K2 = int(contextual_len), int(K1), int(K2)
+    p.alpha, p.N = float(alpha), float(N)
+    p.q, p.k, p.v = q.data_ptr(), k.data_ptr(), v.data_ptr()
+    p.q_row_stride = _row_stride(q, "q", H, d)
+    p.k_row_stride = _row_stride(k, "k", H, d)
+    p.v_row_stride = _row_stride(v, "v", H, d)
+    if k.shape[0] != T or v.shape[0] != T:
+        raise ValueError("q, k, v must have the same number of tokens")
+    if events is not None:
+        p.event_begin = events[0].cuda_event
+        p.event_end = events[1].cuda_event
+    return p
+
+
+def _workspace(which, T, B, H, d, device, workspace):
+    need = hstu_sla_workspace_bytes(which, T, B, H, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=device)
+    if workspace.numel() < need:
+        raise ValueError(f"workspace too small: {workspace.numel()} < {need} bytes")
+    return workspace
+
+
+def hstu_sla_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, seq_offsets: torch.Tensor,
+                 num_targets: Optional[torch.Tensor], *, contextual_len: int, K1: int, K2: int,
+                 alpha: float, N: float, max_seq_len: Optional[int] = None,
+                 out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                 stream=None, events=None) -> torch.Tensor:
+    """SLA HSTU attention forward; returns out [T, H, d] (bf16).  `events`: an
+    optional pair of torch.cuda.Event recorded around the attention kernel."""
+    lib = _abi.load()
+    p = _fwd_params(q, k, v, seq_offsets, num_targets, contextual_len, K1, K2, alpha, N,
+                    max_seq_len, events)
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
+    p.out = out.data_ptr()
+    p.out_row_stride = _row_stride(out, "out", p.H, p.d)
+    ws = _workspace(_abi.WS_FWD, p.total_tokens, p.B, p.H, p.d, q.device, workspace)
+    _check(lib.hstu_sla_fwd(ctypes.byref(p), ws.data_ptr(), ws.numel(), _stream_ptr(stream)),
+           "hstu_sla_fwd")
+    return out
+
+
+def hstu_sla_bwd(dout: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                 seq_offsets: torch.Tensor, num_targets: Optional[torch.Tensor], *,
+                 contextual_len: int, K1: int, K2: int, alpha: float, N: float,
+                 max_seq_len: Optional[int] = None, dq: Optional[torch.Tensor] = None,
+                 dk: Optional[torch.Tensor] = None, dv: Optional[torch.Tensor] = None,
+                 workspace: Optional[torch.Tensor] = None, stream=None, events=None):
+    """SLA HSTU attention backward; returns (dq, dk, dv) [T, H, d] (bf16)."""
+    lib = _abi.load()
+    p = _abi.BwdParams()
+    p.fwd = _fwd_params(q, k, v, seq_offsets, num_targets, contextual_len, K1, K2, alpha, N,
+                        max_seq_len, events)
+    H, d = p.fwd.H, p.fwd.d
+    dq = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device) if dq is None else dq
+    dk = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device) if dk is None else dk
+    dv = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device) if dv is None else dv
+    p.dout, p.dout_row_stride = dout.data_ptr(), _row_stride(dout, "dout", H, d)
+    p.dq, p.dq_row_stride = dq.data_ptr(), _row_stride(dq, "dq", H, d)
+    p.dk, p.dk_row_stride = dk.data_ptr(), _row_stride(dk, "dk", H, d)
+    p.dv, p.dv_row_stride = dv.data_ptr(), _row_stride(dv, "dv", H, d)
+    ws = _workspace(_abi.WS_BWD, p.fwd.total_tokens, p.fwd.B, H, d, q.device, workspace)
+    _check(lib.hstu_sla_bwd(ctypes.byref(p), ws.data_ptr(), ws.numel(), _stream_ptr(stream)),
+           "hstu_sla_bwd")
+    return dq, dk, dv
+
+
+def hstu_sla_count_pairs(q, k, v, seq_offsets, num_targets, *, contextual_len, K1, K2,
+                         max_seq_len=None, stream=None):
+    """Per-token visible-key counts (forward enumeration) and per-token
+    seeing-row counts (backward enumeration), int64 [T] each."""
+    lib = _abi.load()
+    p = _fwd_params(q, k, v, seq_offsets, num_targets, contextual_len, K1, K2, 1.0, 1.0,
+                    max_seq_len)
+    T = p.total_tokens
+    rows = torch.empty(T, dtype=torch.int64, device=q.device)
+    keys = torch.empty(T, dtype=torch.int64, device=q.device)
+    ws = _workspace(_abi.WS_FWD, T, p.B, p.H, p.d, q.device, None)
+    _check(lib.hstu_sla_count_pairs(ctypes.byref(p), rows.data_ptr(), keys.data_ptr(),
+                                    ws.data_ptr(), ws.numel(), _stream_ptr(stream)),
+           "hstu_sla_count_pairs")
+    status = lib.hstu_sla_get_error(ws.data_ptr(), _stream_ptr(stream))
+    _check(status, "hstu_sla_count_pairs (device)")
+    return rows, keys
+
+
+def hstu_sla_get_error(workspace: torch.Tensor, stream=None) -> int:
+    """Synchronise and return the device-side status stored in `workspace`."""
+    return int(_abi.load().hstu_sla_get_error(workspace.data_ptr(), _stream_ptr(stream)))
+
+
+class SLAAttention(torch.autograd.Function):
+    """Autograd wrapper: forward and backward both run in the CUDA library."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, seq_offsets, num_targets, contextual_len, K1, K2, alpha, N,
+                max_seq_len):
+        out = hstu_sla_fwd(q, k, v, seq_offsets, num_targets, contextual_len=contextual_len,
+                           K1=K1, K2=K2, alpha=alpha, N=N, max_seq_len=max_seq_len)
+        ctx.save_for_backward(q, k, v, seq_offsets,
+                              num_targets if num_targets is not None else seq_offsets[:0])
+        ctx.has_targets = num_targets is not None
+        ctx.cfg = (contextual_len, K1, K2, alpha, N, max_seq_len)
+        return out
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, offs, nts = ctx.saved_tensors
+        c, K1, K2, alpha, N, msl = ctx.cfg
+        if dout.stride(2) != 1 or dout.stride(1) != dout.shape[2]:
+            dout = dout.contiguous()
+        dq, dk, dv = hstu_sla_bwd(dout, q, k, v, offs, nts if ctx.has_targets else None,
+                                  contextual_len=c, K1=K1, K2=K2, alpha=alpha, N=N,
+                                  max_seq_len=msl)
+        return dq, dk, dv, None, None, None, None, None, None, None, None
+
+
+def sla_attention(q, k, v, seq_offsets, num_targets=None, *, contextual_len=0, K1, K2, alpha,
+                  N, max_seq_len=None):
+    return SLAAttention.apply(q, k, v, seq_offsets, num_targets, contextual_len, K1, K2, alpha,
+                              N, max_seq_len)

@@ -1,0 +1,180 @@
+// C ABI of the SLA HSTU attention library: host-side argument checks,
+// workspace carving and kernel launches.  See include/hstu_sla.h.
+#include <math.h>
+#include <string.h>
+
+#include "sla_common.cuh"
+
+using namespace hstu;
+
+namespace {
+
+constexpr int kAbiVersion = 100;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+int check_tensor(const void* p, int64_t rs, const hstu_sla_fwd_params* f) {
+  if (p == nullptr) return HSTU_SLA_ERR_INVALID_ARG;
+  if (!aligned16(p)) return HSTU_SLA_ERR_INVALID_ARG;
+  if (rs < (int64_t)f->H * f->d || (rs % 8) != 0) return HSTU_SLA_ERR_INVALID_ARG;
+  return HSTU_SLA_OK;
+}
+
+int check_common(const hstu_sla_fwd_params* f) {
+  if (f == nullptr) return HSTU_SLA_ERR_INVALID_ARG;
+  if (f->B < 1 || f->H < 1 || f->total_tokens < 0 || f->max_seq_len < 0)
+    return HSTU_SLA_ERR_INVALID_ARG;
+  if (f->total_tokens > INT32_MAX) return HSTU_SLA_ERR_UNSUPPORTED;
+  if (f->d != 32 && f->d != 64 && f->d != 128) return HSTU_SLA_ERR_UNSUPPORTED;
+  if (f->K1 < 0 || f->K2 < 0 || f->contextual_len < 0) return HSTU_SLA_ERR_INVALID_ARG;
+  if (!(f->N > 0.f) || !isfinite(f->N) || !isfinite(f->alpha)) return HSTU_SLA_ERR_INVALID_ARG;
+  if (f->seq_offsets == nullptr) return HSTU_SLA_ERR_INVALID_ARG;
+  int e;
+  if ((e = check_tensor(f->q, f->q_row_stride, f))) return e;
+  if ((e = check_tensor(f->k, f->k_row_stride, f))) return e;
+  if ((e = check_tensor(f->v, f->v_row_stride, f))) return e;
+  return HSTU_SLA_OK;
+}
+
+int check_ws(void* ws, size_t bytes, size_t need) {
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255) != 0) return HSTU_SLA_ERR_WORKSPACE;
+  if (bytes < need) return HSTU_SLA_ERR_WORKSPACE;
+  return HSTU_SLA_OK;
+}
+
+AttnArgs make_args(const hstu_sla_fwd_params* f, void* ws) {
+  AttnArgs a;
+  memset(&a, 0, sizeof(a));
+  a.offs = f->seq_offsets;
+  a.nts = f->num_targets;
+  a.ws = reinterpret_cast<WsHeader*>(ws);
+  a.items = reinterpret_cast<const int2*>(static_cast<char*>(ws) + ws_items_offset());
+  a.B = f->B;
+  a.H = f->H;
+  a.K1 = f->K1;
+  a.K2e = f->K2 > f->contextual_len ? f->K2 : f->contextual_len;
+  a.max_seq_len = f->max_seq_len;
+  a.T = f->total_tokens;
+  a.alpha = f->alpha;
+  a.inv_n = 1.0f / f->N;
+  a.q = static_cast<const bf16*>(f->q);
+  a.k = static_cast<const bf16*>(f->k);
+  a.v = static_cast<const bf16*>(f->v);
+  a.q_rs = f->q_row_stride;
+  a.k_rs = f->k_row_stride;
+  a.v_rs = f->v_row_stride;
+  return a;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? HSTU_SLA_OK : HSTU_SLA_ERR_CUDA; }
+
+cudaError_t record(void* ev, cudaStream_t st) {
+  return ev ? cudaEventRecord(reinterpret_cast<cudaEvent_t>(ev), st) : cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t hstu_sla_workspace_bytes(int which, int64_t total_tokens, int32_t B, int32_t H,
+                                int32_t d) {
+  if (total_tokens < 0 || B < 1 || H < 1 || d < 1) return 0;
+  if (which == HSTU_SLA_WS_FWD) return ws_dq_offset(total_tokens, B);
+  if (which == HSTU_SLA_WS_BWD)
+    return ws_dq_offset(total_tokens, B) + align256(sizeof(float) * (size_t)total_tokens * H * d);
+  return 0;
+}
+
+int hstu_sla_fwd(const hstu_sla_fwd_params* p, void* workspace, size_t workspace_bytes,
+                 hstu_stream_t stream) {
+  int e = check_common(p);
+  if (e) return e;
+  if ((e = check_tensor(p->out, p->out_row_stride, p))) return e;
+  if ((e = check_ws(workspace, workspace_bytes,
+                    hstu_sla_workspace_bytes(HSTU_SLA_WS_FWD, p->total_tokens, p->B, p->H, p->d))))
+    return e;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  AttnArgs a = make_args(p, workspace);
+  a.out = static_cast<bf16*>(p->out);
+  a.o_rs = p->out_row_stride;
+  cudaError_t ce = launch_worklist(a, 64, 0, st);
+  if (ce == cudaSuccess) ce = record(p->event_begin, st);
+  if (ce == cudaSuccess) ce = launch_fwd_mma(a, p->d, st);
+  if (ce == cudaSuccess) ce = record(p->event_end, st);
+  return cuda_status(ce);
+}
+
+int hstu_sla_bwd(const hstu_sla_bwd_params* p, void* workspace, size_t workspace_bytes,
+                 hstu_stream_t stream) {
+  if (p == nullptr) return HSTU_SLA_ERR_INVALID_ARG;
+  const hstu_sla_fwd_params* f = &p->fwd;
+  int e = check_common(f);
+  if (e) return e;
+  if ((e = check_tensor(p->dout, p->dout_row_stride, f))) return e;
+  if ((e = check_tensor(p->dq, p->dq_row_stride, f))) return e;
+  if ((e = check_tensor(p->dk, p->dk_row_stride, f))) return e;
+  if ((e = check_tensor(p->dv, p->dv_row_stride, f))) return e;
+  if ((e = check_ws(workspace, workspace_bytes,
+                    hstu_sla_workspace_bytes(HSTU_SLA_WS_BWD, f->total_tokens, f->B, f->H, f->d))))
+    return e;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  AttnArgs a = make_args(f, workspace);
+  a.dout = static_cast<const bf16*>(p->dout);
+  a.dq = static_cast<bf16*>(p->dq);
+  a.dk = static_cast<bf16*>(p->dk);
+  a.dv = static_cast<bf16*>(p->dv);
+  a.do_rs = p->dout_row_stride;
+  a.dq_rs = p->dq_row_stride;
+  a.dk_rs = p->dk_row_stride;
+  a.dv_rs = p->dv_row_stride;
+  a.dq_acc = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                      ws_dq_offset(f->total_tokens, f->B));
+  cudaError_t ce = cudaMemsetAsync(a.dq_acc, 0, sizeof(float) * (size_t)f->total_tokens * f->H * f->d, st);
+  if (ce == cudaSuccess) ce = launch_worklist(a, 64, 1, st);
+  if (ce == cudaSuccess) ce = record(f->event_begin, st);
+  if (ce == cudaSuccess) ce = launch_bwd_mma(a, f->d, st);
+  if (ce == cudaSuccess) ce = record(f->event_end, st);
+  if (ce == cudaSuccess) ce = launch_dq_convert(a, f->d, st);
+  return cuda_status(ce);
+}
+
+int hstu_sla_count_pairs(const hstu_sla_fwd_params* p, int64_t* row_counts, int64_t* key_counts,
+                         void* workspace, size_t workspace_bytes, hstu_stream_t stream) {
+  int e = check_common(p);
+  if (e) return e;
+  if ((e = check_ws(workspace, workspace_bytes,
+                    hstu_sla_workspace_bytes(HSTU_SLA_WS_FWD, p->total_tokens, p->B, p->H, p->d))))
+    return e;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  AttnArgs a = make_args(p, workspace);
+  cudaError_t ce = launch_worklist(a, 64, 0, st);
+  if (ce == cudaSuccess) ce = launch_count_pairs(a, 64, 64, row_counts, key_counts, st);
+  return cuda_status(ce);
+}
+
+int hstu_sla_get_error(const void* workspace, hstu_stream_t stream) {
+  if (workspace == nullptr) return HSTU_SLA_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int32_t status = 0;
+  cudaError_t ce = cudaMemcpyAsync(&status, workspace, sizeof(status), cudaMemcpyDeviceToHost, st);
+  if (ce == cudaSuccess) ce = cudaStreamSynchronize(st);
+  if (ce != cudaSuccess) return HSTU_SLA_ERR_CUDA;
+  return status;
+}
+
+const char* hstu_sla_strerror(int code) {
+  switch (code) {
+    case HSTU_SLA_OK: return "ok";
+    case HSTU_SLA_ERR_INVALID_ARG: return "invalid argument (null pointer, bad size or misalignment)";
+    case HSTU_SLA_ERR_UNSUPPORTED: return "unsupported configuration (head_dim or device)";
+    case HSTU_SLA_ERR_CUDA: return "CUDA runtime error";
+    case HSTU_SLA_ERR_BAD_INPUT: return "invalid seq_offsets / num_targets detected on the device";
+    case HSTU_SLA_ERR_WORKSPACE: return "workspace missing, too small or not 256-byte aligned";
+    case HSTU_SLA_ERR_TIMEOUT: return "a bounded device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int hstu_sla_version(void) { return kAbiVersion; }
+
+}  // extern "C"

@@ -1,0 +1,230 @@
+// Shared device-side definitions of the SLA HSTU attention library: the
+// kernel argument block, the workspace layout, the mask predicate and the
+// tile enumeration that every kernel (work list, forward, backward, pair
+// count) uses, so that all of them agree on which (query tile, key tile)
+// pairs are non-empty.
+//
+// Mask ("Bending the Scaling Law Curve in Large-Scale Recommendation
+// Systems", section 4.2.1, Eq. 7, read with a K1-token window that includes
+// self; K2eff = max(K2, contextual_len) from the TorchEasyRec "ULTRA HSTU"
+// docs; candidates as in the M-FALCON mask figure of the HSTU notes):
+//   history row i < Lh:    j <= i  and (i - j < K1  or  j < K2eff)
+//   candidate row i >= Lh: j == i  or (j < Lh and (Lh - j < K1 or j < K2eff))
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/hstu_sla.h"
+
+namespace hstu {
+
+using bf16 = __nv_bfloat16;
+
+// ---------------------------------------------------------------- workspace
+// [0, 256)            WsHeader
+// [256, ...)          int2 items[max_items]   (sequence, tile) pairs
+// [align256, ...)     float dq_acc[T * H * d] (backward only)
+struct WsHeader {
+  int32_t status;       // HSTU_SLA_OK or a negative code
+  int32_t n_items;      // items written by the work-list kernel
+  int32_t n_items_pre;  // backward: leading items that hold prefix key tiles
+  int32_t sched;        // dynamic tile scheduler counter (persistent kernels)
+  int32_t pad[60];
+};
+static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
+
+constexpr int kMinTile = 64;  // smallest tile any kernel enumerates with
+
+__host__ __device__ inline int64_t max_items(int64_t T, int B) {
+  return (T + kMinTile - 1) / kMinTile + B;
+}
+__host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+__host__ __device__ inline size_t ws_items_offset() { return sizeof(WsHeader); }
+__host__ __device__ inline size_t ws_dq_offset(int64_t T, int B) {
+  return align256(ws_items_offset() + sizeof(int2) * size_t(max_items(T, B)));
+}
+
+// ------------------------------------------------------------ kernel args
+struct AttnArgs {
+  const int32_t* offs;   // [B+1]
+  const int32_t* nts;    // [B] or null
+  const int2* items;     // work list
+  WsHeader* ws;          // status / counts
+  int B, H, K1, K2e, max_seq_len;
+  int64_t T;
+  float alpha, inv_n;
+  const bf16* q;
+  const bf16* k;
+  const bf16* v;
+  const bf16* dout;
+  bf16* out;
+  bf16* dq;
+  bf16* dk;
+  bf16* dv;
+  float* dq_acc;
+  int64_t q_rs, k_rs, v_rs, do_rs, o_rs, dq_rs, dk_rs, dv_rs;
+};
+
+__host__ __device__ inline int cdiv(int a, int b) { return (a + b - 1) / b; }
+__host__ __device__ __forceinline__ int imin(int a, int b) { return a < b ? a : b; }
+__host__ __device__ __forceinline__ int imax(int a, int b) { return a > b ? a : b; }
+
+struct SeqGeom {
+  int s0;  // first token of the sequence
+  int L;   // length
+  int Lh;  // history length (L - num_targets)
+};
+
+__device__ __forceinline__ SeqGeom seq_geom(const AttnArgs& a, int b) {
+  SeqGeom g;
+  g.s0 = a.offs[b];
+  g.L = a.offs[b + 1] - g.s0;
+  g.Lh = g.L - (a.nts ? a.nts[b] : 0);
+  return g;
+}
+
+// Mask predicate for 0 <= i, j.
+__host__ __device__ __forceinline__ bool sla_visible(int i, int j, int L, int Lh, int K1, int K2e) {
+  if (i < Lh) return j <= i && (i - j < K1 || j < K2e);
+  if (i >= L) return false;
+  return j == i || (j < Lh && (Lh - j < K1 || j < K2e));
+}
+
+// The same predicate as three intervals per row, for inner loops:
+// visible(j) = j < pre || (lo <= j && j < hi) || j == self.
+struct RowMask {
+  int pre, lo, hi, self;
+  __host__ __device__ __forceinline__ bool operator()(int j) const {
+    return j < pre || (j >= lo && j < hi) || j == self;
+  }
+};
+
+__host__ __device__ __forceinline__ RowMask row_mask(int i, int L, int Lh, int K1, int K2e) {
+  RowMask m;
+  if (i < Lh) {
+    m.pre = imin(K2e, i + 1);
+    m.lo = imax(0, i - K1 + 1);
+    m.hi = K1 > 0 ? i + 1 : 0;
+    m.self = -1;
+  } else if (i < L) {
+    m.pre = imin(K2e, Lh);
+    m.lo = imax(0, Lh - K1 + 1);
+    m.hi = K1 > 0 ? Lh : 0;
+    m.self = i;
+  } else {
+    m.pre = 0; m.lo = 0; m.hi = 0; m.self = -1;
+  }
+  return m;
+}
+
+// Up to three disjoint, increasing tile-index intervals [lo, hi).
+struct Spans {
+  int lo[3], hi[3], n;
+  __host__ __device__ void clear() { n = 0; }
+  // Pushes must come in non-decreasing order of lo; overlapping or touching
+  // intervals merge.
+  __host__ __device__ void push(int l, int h) {
+    if (l >= h) return;
+    if (n > 0 && l <= hi[n - 1]) {
+      if (h > hi[n - 1]) hi[n - 1] = h;
+      return;
+    }
+    lo[n] = l; hi[n] = h; ++n;
+  }
+  __host__ __device__ int count() const {
+    int c = 0;
+    for (int s = 0; s < n; ++s) c += hi[s] - lo[s];
+    return c;
+  }
+  // Tile index of the n-th element (0 <= e < count()).
+  __host__ __device__ int at(int e) const {
+    for (int s = 0; s < n; ++s) {
+      int w = hi[s] - lo[s];
+      if (e < w) return lo[s] + e;
+      e -= w;
+    }
+    return -1;
+  }
+};
+
+// Key tiles (width BN) that hold a visible key for some row of the query
+// rows [r0, r1) of one sequence: the global prefix, the local band (which for
+// candidate rows is the band ending at Lh) and the candidates' own diagonal.
+__host__ __device__ inline Spans q_tile_key_tiles(int r0, int r1, int Lh, int K1, int K2e,
+                                                  int BN) {
+  Spans s;
+  s.clear();
+  int hist_end = r1 < Lh ? r1 : Lh;        // prefix keys are history keys
+  int pre_hi = K2e < hist_end ? K2e : hist_end;
+  s.push(0, cdiv(pre_hi, BN));
+  if (K1 > 0) {
+    int blo, bhi;
+    if (r0 < Lh) {
+      blo = r0 - K1 + 1;
+      bhi = r1 < Lh ? r1 : Lh;
+    } else {
+      blo = Lh - K1 + 1;
+      bhi = Lh;
+    }
+    if (blo < 0) blo = 0;
+    if (blo < bhi) s.push(blo / BN, cdiv(bhi, BN));
+  }
+  if (r1 > Lh) {
+    int dlo = r0 > Lh ? r0 : Lh;
+    s.push(dlo / BN, cdiv(r1, BN));
+  }
+  return s;
+}
+
+// Query tiles (height BM) that hold a row seeing some key of the key tile
+// [j0, j1) of one sequence of length L.
+__host__ __device__ inline Spans k_tile_q_tiles(int j0, int j1, int L, int Lh, int K1, int K2e,
+                                                int BM) {
+  Spans s;
+  s.clear();
+  int pre_end = K2e < Lh ? K2e : Lh;
+  if (j0 < pre_end) {  // a prefix key of the history: every later row sees it
+    s.push(j0 / BM, cdiv(L, BM));
+    return s;
+  }
+  if (K1 > 0 && j0 < Lh) {
+    int jh = j1 < Lh ? j1 : Lh;  // last history key + 1
+    int rhi = jh - 1 + K1;       // history rows i <= j + K1 - 1
+    if (rhi > Lh) rhi = Lh;
+    s.push(j0 / BM, cdiv(rhi, BM));
+    if (jh - 1 >= Lh - K1 + 1) s.push(Lh / BM, cdiv(L, BM));  // candidates' band
+  }
+  if (j1 > Lh) {  // candidate keys: only the candidate itself
+    int dlo = j0 > Lh ? j0 : Lh;
+    s.push(dlo / BM, cdiv(j1, BM));
+  }
+  return s;
+}
+
+// True if every (row, key) pair of rows [r0, r1) x keys [j0, j1) is visible,
+// so the mask need not be evaluated.
+__host__ __device__ __forceinline__ bool tile_full(int r0, int r1, int j0, int j1, int Lh, int K1,
+                                          int K2e) {
+  return r1 <= Lh && j1 <= r0 + 1 && (j1 <= K2e || j0 >= r1 - K1);
+}
+
+__device__ __forceinline__ void set_status(WsHeader* ws, int code) {
+  atomicCAS(&ws->status, 0, code);
+}
+
+__device__ __forceinline__ int load_status(const WsHeader* ws) {
+  return *((volatile const int32_t*)&ws->status);
+}
+
+// ------------------------------------------------------------ host launchers
+// (defined in the .cu files; return cudaError_t of the launch)
+cudaError_t launch_worklist(const AttnArgs& a, int tile, int backward, cudaStream_t st);
+cudaError_t launch_count_pairs(const AttnArgs& a, int BM, int BN, int64_t* row_counts,
+                               int64_t* key_counts, cudaStream_t st);
+cudaError_t launch_dq_convert(const AttnArgs& a, int d, cudaStream_t st);
+cudaError_t launch_fwd_mma(const AttnArgs& a, int d, cudaStream_t st);
+cudaError_t launch_bwd_mma(const AttnArgs& a, int d, cudaStream_t st);
+
+}  // namespace hstu

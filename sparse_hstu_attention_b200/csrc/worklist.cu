@@ -1,0 +1,193 @@
+// Work-list construction, device-side input validation, the pair-count test
+// hook and the dq fp32 -> bf16 conversion.
+//
+// The work list is built on the device from seq_offsets / num_targets, so a
+// call never waits on the host.  Forward items are (sequence, query tile);
+// backward items are (sequence, key tile) with the prefix key tiles first:
+// a prefix key is seen by every later row of its sequence, so those items are
+// the longest and start first (a longest-first order without a sort).
+#include "sla_common.cuh"
+
+namespace hstu {
+
+namespace {
+
+constexpr int kWlThreads = 1024;
+
+// Block-wide exclusive scan of one int per thread; returns the block total.
+__device__ int block_exclusive_scan(int v, int* out, int* smem) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) smem[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < (kWlThreads / 32) ? smem[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    smem[lane] = w;  // inclusive warp sums
+  }
+  __syncthreads();
+  int base = warp > 0 ? smem[warp - 1] : 0;
+  *out = base + x - v;
+  int total = smem[kWlThreads / 32 - 1];
+  __syncthreads();
+  return total;
+}
+
+// One block.  backward = 0: items (b, query tile) in sequence order.
+// backward = 1: first every (b, key tile) whose key tile starts inside the
+// history prefix [0, min(K2eff, Lh)), then all other key tiles.
+__global__ void __launch_bounds__(kWlThreads) worklist_kernel(AttnArgs a, int tile, int backward) {
+  __shared__ int s_scan[32];
+  __shared__ int s_bad;
+  int2* items = const_cast<int2*>(a.items);
+  if (threadIdx.x == 0) s_bad = 0;
+  __syncthreads();
+  // validation of the device-resident offsets and targets
+  for (int b = threadIdx.x; b <= a.B; b += blockDim.x) {
+    int o = a.offs[b];
+    bool bad = false;
+    if (b == 0) bad |= (o != 0);
+    if (b == a.B) bad |= ((int64_t)o != a.T);
+    if (b < a.B) {
+      int len = a.offs[b + 1] - o;
+      int nt = a.nts ? a.nts[b] : 0;
+      bad |= (len < 0) | (len > a.max_seq_len) | (nt < 0) | (nt > len);
+    }
+    if (bad) s_bad = 1;
+  }
+  __syncthreads();
+  if (s_bad) {
+    if (threadIdx.x == 0) {
+      a.ws->status = HSTU_SLA_ERR_BAD_INPUT;
+      a.ws->n_items = 0;
+      a.ws->n_items_pre = 0;
+      a.ws->sched = 0;
+    }
+    return;
+  }
+  // pass 0 counts prefix items (backward) and writes them; pass 1 the rest.
+  int written = 0, n_pre = 0;
+  for (int pass = backward ? 0 : 1; pass < 2; ++pass) {
+    for (int c0 = 0; c0 < a.B; c0 += kWlThreads) {
+      int b = c0 + threadIdx.x;
+      int cnt = 0, first = 0;
+      if (b < a.B) {
+        int L = a.offs[b + 1] - a.offs[b];
+        int Lh = L - (a.nts ? a.nts[b] : 0);
+        int ntile = cdiv(L, tile);
+        int npre = 0;
+        if (backward) {
+          int pre_end = a.K2e < Lh ? a.K2e : Lh;
+          npre = cdiv(pre_end, tile);
+          if (npre > ntile) npre = ntile;
+        }
+        if (pass == 0) { cnt = npre; first = 0; }
+        else { cnt = ntile - npre; first = npre; }
+      }
+      int off;
+      int total = block_exclusive_scan(cnt, &off, s_scan);
+      for (int e = 0; e < cnt; ++e) items[written + off + e] = make_int2(b, first + e);
+      written += total;
+    }
+    if (pass == 0) n_pre = written;
+  }
+  if (threadIdx.x == 0) {
+    a.ws->status = HSTU_SLA_OK;
+    a.ws->n_items = written;
+    a.ws->n_items_pre = n_pre;
+    a.ws->sched = 0;
+  }
+}
+
+// Per token: number of visible keys found by walking the forward enumeration
+// (row_counts), and number of rows that see it found by walking the backward
+// enumeration (key_counts).
+__global__ void count_pairs_kernel(AttnArgs a, int BM, int BN, int64_t* row_counts,
+                                   int64_t* key_counts) {
+  if (load_status(a.ws) != 0) return;
+  int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (t >= a.T) return;
+  int lo = 0, hi = a.B - 1;  // sequence of token t
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (a.offs[mid] <= t) lo = mid; else hi = mid - 1;
+  }
+  SeqGeom g = seq_geom(a, lo);
+  int p = int(t - g.s0);
+  if (row_counts) {
+    int r0 = (p / BM) * BM, r1 = imin(r0 + BM, g.L);
+    Spans s = q_tile_key_tiles(r0, r1, g.Lh, a.K1, a.K2e, BN);
+    int64_t n = 0;
+    for (int e = 0; e < s.count(); ++e) {
+      int kt = s.at(e);
+      for (int j = kt * BN; j < imin(kt * BN + BN, g.L); ++j)
+        n += sla_visible(p, j, g.L, g.Lh, a.K1, a.K2e);
+    }
+    row_counts[t] = n;
+  }
+  if (key_counts) {
+    int j0 = (p / BN) * BN, j1 = imin(j0 + BN, g.L);
+    Spans s = k_tile_q_tiles(j0, j1, g.L, g.Lh, a.K1, a.K2e, BM);
+    int64_t n = 0;
+    for (int e = 0; e < s.count(); ++e) {
+      int qt = s.at(e);
+      for (int i = qt * BM; i < imin(qt * BM + BM, g.L); ++i)
+        n += sla_visible(i, p, g.L, g.Lh, a.K1, a.K2e);
+    }
+    key_counts[t] = n;
+  }
+}
+
+// dq[t, h, :] (bf16, strided) = dq_acc[t, h, :] (fp32, dense), 8 values a thread.
+template <int D>
+__global__ void dq_convert_kernel(AttnArgs a) {
+  if (load_status(a.ws) != 0) return;
+  const int64_t chunks = a.T * a.H * (D / 8);
+  for (int64_t c = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; c < chunks;
+       c += (int64_t)gridDim.x * blockDim.x) {
+    int64_t e = c * 8;
+    int64_t t = e / (a.H * D);
+    int64_t hc = e - t * (a.H * D);
+    const float4* src = reinterpret_cast<const float4*>(a.dq_acc + e);
+    float4 x = src[0], y = src[1];
+    __nv_bfloat162 o[4] = {__floats2bfloat162_rn(x.x, x.y), __floats2bfloat162_rn(x.z, x.w),
+                           __floats2bfloat162_rn(y.x, y.y), __floats2bfloat162_rn(y.z, y.w)};
+    *reinterpret_cast<uint4*>(a.dq + t * a.dq_rs + hc) = *reinterpret_cast<uint4*>(o);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_worklist(const AttnArgs& a, int tile, int backward, cudaStream_t st) {
+  worklist_kernel<<<1, kWlThreads, 0, st>>>(a, tile, backward);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_count_pairs(const AttnArgs& a, int BM, int BN, int64_t* row_counts,
+                               int64_t* key_counts, cudaStream_t st) {
+  if (a.T == 0) return cudaSuccess;
+  int threads = 256;
+  int64_t blocks = (a.T + threads - 1) / threads;
+  count_pairs_kernel<<<(unsigned)blocks, threads, 0, st>>>(a, BM, BN, row_counts, key_counts);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dq_convert(const AttnArgs& a, int d, cudaStream_t st) {
+  if (a.T == 0) return cudaSuccess;
+  int threads = 256, blocks = 148 * 8;
+  if (d == 32) dq_convert_kernel<32><<<blocks, threads, 0, st>>>(a);
+  else if (d == 64) dq_convert_kernel<64><<<blocks, threads, 0, st>>>(a);
+  else dq_convert_kernel<128><<<blocks, threads, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace hstu

@@ -1,0 +1,111 @@
+"""The C-ABI library: it loads without a GPU, exports every symbol the header
+declares, and rejects bad arguments on the host before touching CUDA."""
+import ctypes
+
+import pytest
+
+import sparse_hstu_attention_b200 as sla
+from sparse_hstu_attention_b200 import _abi
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from sparse_hstu_attention_b200 import build
+    build.build()
+    return _abi.load()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _abi.declared_functions()
+    assert {"hstu_sla_fwd", "hstu_sla_bwd", "hstu_sla_workspace_bytes",
+            "hstu_sla_count_pairs", "hstu_sla_get_error", "hstu_sla_strerror"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_version_and_messages(lib):
+    assert lib.hstu_sla_version() >= 100
+    for code in (0, -1, -2, -3, -4, -5, -6):
+        assert sla.hstu_sla_strerror(code)
+    assert "unknown" in sla.hstu_sla_strerror(-99)
+
+
+def test_workspace_sizes(lib):
+    f = lib.hstu_sla_workspace_bytes
+    assert f(_abi.WS_FWD, 0, 1, 1, 32) >= 256
+    fwd = f(_abi.WS_FWD, 100_000, 8, 4, 128)
+    bwd = f(_abi.WS_BWD, 100_000, 8, 4, 128)
+    assert fwd % 256 == 0 and bwd % 256 == 0
+    assert bwd - fwd >= 100_000 * 4 * 128 * 4   # the fp32 dq accumulator
+    assert f(7, 10, 1, 1, 32) == 0
+    assert f(_abi.WS_FWD, -1, 1, 1, 32) == 0
+
+
+FAKE = 0x10000  # never dereferenced: every case below fails a host check first
+
+
+def _params(**kw):
+    p = _abi.FwdParams()
+    p.B, p.H, p.d, p.total_tokens, p.max_seq_len = 2, 4, 128, 100, 100
+    p.seq_offsets = FAKE
+    p.contextual_len, p.K1, p.K2, p.alpha, p.N = 0, 8, 4, 0.1, 10.0
+    p.q = p.k = p.v = p.out = FAKE
+    p.q_row_stride = p.k_row_stride = p.v_row_stride = p.out_row_stride = 512
+    for k, v in kw.items():
+        setattr(p, k, v)
+    return p
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("d", 48, _abi.ERR_UNSUPPORTED),
+    ("d", 256, _abi.ERR_UNSUPPORTED),
+    ("B", 0, _abi.ERR_INVALID_ARG),
+    ("H", 0, _abi.ERR_INVALID_ARG),
+    ("K1", -1, _abi.ERR_INVALID_ARG),
+    ("K2", -3, _abi.ERR_INVALID_ARG),
+    ("contextual_len", -1, _abi.ERR_INVALID_ARG),
+    ("N", 0.0, _abi.ERR_INVALID_ARG),
+    ("N", float("nan"), _abi.ERR_INVALID_ARG),
+    ("alpha", float("inf"), _abi.ERR_INVALID_ARG),
+    ("q", None, _abi.ERR_INVALID_ARG),
+    ("v", FAKE + 8, _abi.ERR_INVALID_ARG),          # not 16-byte aligned
+    ("k_row_stride", 500, _abi.ERR_INVALID_ARG),    # < H*d
+    ("q_row_stride", 516, _abi.ERR_INVALID_ARG),    # not a multiple of 8
+    ("seq_offsets", None, _abi.ERR_INVALID_ARG),
+    ("out", None, _abi.ERR_INVALID_ARG),
+    ("total_tokens", 1 << 40, _abi.ERR_UNSUPPORTED),
+])
+def test_fwd_host_validation(lib, field, value, code):
+    p = _params(**{field: value})
+    assert lib.hstu_sla_fwd(ctypes.byref(p), FAKE * 256, 1 << 30, None) == code
+
+
+def test_workspace_validation(lib):
+    p = _params()
+    need = lib.hstu_sla_workspace_bytes(_abi.WS_FWD, 100, 2, 4, 128)
+    assert lib.hstu_sla_fwd(ctypes.byref(p), None, need, None) == _abi.ERR_WORKSPACE
+    assert lib.hstu_sla_fwd(ctypes.byref(p), FAKE * 256 + 16, need, None) == _abi.ERR_WORKSPACE
+    assert lib.hstu_sla_fwd(ctypes.byref(p), FAKE * 256, need - 1, None) == _abi.ERR_WORKSPACE
+
+
+def test_bwd_host_validation(lib):
+    b = _abi.BwdParams()
+    b.fwd = _params()
+    b.dout = b.dq = b.dk = b.dv = FAKE
+    b.dout_row_stride = b.dq_row_stride = b.dk_row_stride = b.dv_row_stride = 512
+    b.dk = None
+    assert lib.hstu_sla_bwd(ctypes.byref(b), FAKE * 256, 1 << 40, None) == _abi.ERR_INVALID_ARG
+    b.dk = FAKE
+    b.dv_row_stride = 4
+    assert lib.hstu_sla_bwd(ctypes.byref(b), FAKE * 256, 1 << 40, None) == _abi.ERR_INVALID_ARG
+    b.dv_row_stride = 512
+    need = lib.hstu_sla_workspace_bytes(_abi.WS_BWD, 100, 2, 4, 128)
+    assert lib.hstu_sla_bwd(ctypes.byref(b), FAKE * 256, need - 256, None) == _abi.ERR_WORKSPACE
+    assert lib.hstu_sla_bwd(None, FAKE * 256, need, None) == _abi.ERR_INVALID_ARG
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(_abi, "_lib", None)
+    monkeypatch.setattr(_abi, "LIB_PATH", str(tmp_path / "absent.so"))
+    with pytest.raises(_abi.LibraryMissing):
+        _abi.load()

@@ -1,0 +1,171 @@
+"""GPU parity: the CUDA library (through its C ABI) against the oracle on the
+same seeded bf16 inputs.  Floating point: max|gpu - ref| <= 2e-2 * max|ref|
+per tensor (out, dq, dk, dv).  Pair counts: exact."""
+import numpy as np
+import pytest
+import torch
+
+import sparse_hstu_attention_b200 as sla
+from workloads import WORKLOADS, make_batch, with_params
+
+from parity import (TOL, assert_close, gpu_bwd, gpu_fwd, oracle_problem, sample_tokens,
+                    to_gpu)
+
+pytestmark = pytest.mark.gpu
+
+
+def _edge_batch(lengths, nt, H=2, d=128, K1=40, K2=10, ctx=3, seed=5, alpha=None, N=300.0):
+    w = with_params(WORKLOADS["tiny"], H=H, d=d, K1=K1, K2=K2, contextual_len=ctx,
+                    num_targets=nt, alpha=alpha if alpha is not None else d ** -0.5, N=N)
+    lengths = np.array(lengths, dtype=np.int64)
+    return make_batch(w, lengths=lengths, num_targets=np.minimum(nt, lengths), seed=seed)
+
+
+def _full_check(batch, strided=False, fwd=True, bwd=True):
+    g = to_gpu(batch, strided=strided)
+    p = oracle_problem(batch)
+    if fwd:
+        out = gpu_fwd(batch, g)
+        assert_close("out", out, p.fwd(batch.q, batch.k, batch.v))
+    if bwd:
+        dq, dk, dv = gpu_bwd(batch, g)
+        rq, rk, rv = p.bwd(batch.q, batch.k, batch.v, batch.dout)
+        assert_close("dq", dq, rq)
+        assert_close("dk", dk, rk)
+        assert_close("dv", dv, rv)
+
+
+def _count_check(batch):
+    g = to_gpu(batch)
+    w = batch.workload
+    rows, keys = sla.hstu_sla_count_pairs(g["q"], g["k"], g["v"], g["offs"], g["nts"],
+                                          contextual_len=w.contextual_len, K1=w.K1, K2=w.K2,
+                                          max_seq_len=int(batch.lengths.max()))
+    p = oracle_problem(batch)
+    np.testing.assert_array_equal(rows.cpu().numpy(), p.row_counts())
+    np.testing.assert_array_equal(keys.cpu().numpy(), p.key_counts())
+
+
+def test_tiny_workload_full():
+    b = make_batch(WORKLOADS["tiny"])
+    _full_check(b)
+    _count_check(b)
+
+
+EDGE = {
+    "ragged": dict(lengths=[1, 2, 17, 64, 65, 127, 128, 129, 300], nt=8),
+    "all_candidates": dict(lengths=[5, 70, 130], nt=200),
+    "no_candidates": dict(lengths=[190, 33], nt=0),
+    "prefix_only_K1_0": dict(lengths=[150, 257], nt=6, K1=0),
+    "window_K1_1": dict(lengths=[150, 97], nt=5, K1=1, K2=0, ctx=0),
+    "pure_window": dict(lengths=[300, 64], nt=0, K1=50, K2=0, ctx=0),
+    "full_causal": dict(lengths=[260, 31], nt=4, K1=100000, K2=0, ctx=0),
+    "nothing_but_self": dict(lengths=[140], nt=20, K1=0, K2=0, ctx=0),
+    "empty_sequences": dict(lengths=[0, 90, 0, 0, 200, 0], nt=7),
+    "contextual_longer_than_seq": dict(lengths=[40, 300], nt=5, ctx=64, K2=2),
+    "d64": dict(lengths=[200, 77], nt=9, d=64, H=3),
+    "d32": dict(lengths=[200, 77], nt=9, d=32, H=4),
+    "big_window_prefix": dict(lengths=[700], nt=64, K1=300, K2=130, ctx=32),
+}
+
+
+@pytest.mark.parametrize("name", sorted(EDGE))
+def test_edge_cases(name):
+    b = _edge_batch(**EDGE[name])
+    _full_check(b)
+    _count_check(b)
+
+
+def test_strided_fused_projection_views():
+    b = _edge_batch(lengths=[150, 260, 9], nt=12)
+    _full_check(b, strided=True)
+
+
+def test_repeat_calls_are_consistent():
+    """Forward is deterministic; backward dq sums in fp32 atomics (order may vary)."""
+    b = _edge_batch(lengths=[300, 200], nt=10)
+    g = to_gpu(b)
+    o1, o2 = gpu_fwd(b, g), gpu_fwd(b, g)
+    assert torch.equal(o1, o2)
+    d1, d2 = gpu_bwd(b, g), gpu_bwd(b, g)
+    assert torch.equal(d1[1], d2[1]) and torch.equal(d1[2], d2[2])  # dk, dv: no atomics
+    assert (d1[0].float() - d2[0].float()).abs().max().item() <= 1e-2 * d1[0].float().abs().max().item()
+
+
+@pytest.mark.parametrize("wname", ["mid", "hist16k"])
+def test_full_size_sampled(wname):
+    """The bench workloads at full size, checked on sampled rows (forward, dq)
+    and sampled keys (dk, dv) that the oracle computes one by one."""
+    b = make_batch(WORKLOADS[wname])
+    g = to_gpu(b)
+    out = gpu_fwd(b, g)
+    dq, dk, dv = gpu_bwd(b, g)
+    p = oracle_problem(b)
+    rows = sample_tokens(b, 160, seed=1)
+    keys = sample_tokens(b, 160, seed=2)
+    assert_close("out", out[rows], p.fwd(b.q, b.k, b.v, rows=rows))
+    assert_close("dq", dq[rows], p.bwd_dq(b.q, b.k, b.v, b.dout, rows=rows))
+    rk, rv = p.bwd_dkv(b.q, b.k, b.v, b.dout, keys=keys)
+    assert_close("dk", dk[keys], rk)
+    assert_close("dv", dv[keys], rv)
+    for t in (out, dq, dk, dv):
+        assert torch.isfinite(t.float()).all()
+
+
+def test_inference_workload_sampled():
+    b = make_batch(WORKLOADS["infer"], with_dout=False)
+    g = to_gpu(b)
+    out = gpu_fwd(b, g)
+    p = oracle_problem(b)
+    rows = sample_tokens(b, 96, seed=3)
+    assert_close("out", out[rows], p.fwd(b.q, b.k, b.v, rows=rows))
+    assert torch.isfinite(out.float()).all()
+
+
+@pytest.mark.parametrize("wname", ["mid", "hist16k"])
+def test_full_size_pair_counts(wname):
+    _count_check(make_batch(WORKLOADS[wname], with_dout=False))
+
+
+@pytest.mark.parametrize("bad", ["non_monotone", "targets_exceed_length", "last_offset",
+                                 "too_long"])
+def test_device_detected_bad_input(bad):
+    """Corrupted offsets / targets are caught on the device: the kernels skip all
+    work and the status reads ERR_BAD_INPUT; the context stays usable."""
+    b = _edge_batch(lengths=[100, 100, 100], nt=4)
+    g = to_gpu(b)
+    offs, nts = g["offs"].clone(), g["nts"].clone()
+    msl = 100
+    if bad == "non_monotone":
+        offs[1] = 250
+    elif bad == "targets_exceed_length":
+        nts[2] = 101
+    elif bad == "last_offset":
+        offs[3] = 299
+    else:
+        msl = 99
+    ws = torch.zeros(sla.hstu_sla_workspace_bytes(1, b.T, 3, b.q.shape[1], b.q.shape[2]),
+                     dtype=torch.uint8, device="cuda")
+    kw = dict(contextual_len=3, K1=40, K2=10, alpha=0.1, N=300.0, max_seq_len=msl)
+    sla.hstu_sla_fwd(g["q"], g["k"], g["v"], offs, nts, workspace=ws, **kw)
+    assert sla.hstu_sla_get_error(ws) == -4
+    sla.hstu_sla_bwd(g["dout"], g["q"], g["k"], g["v"], offs, nts, workspace=ws, **kw)
+    assert sla.hstu_sla_get_error(ws) == -4
+    # the same workspace with good inputs clears the status
+    sla.hstu_sla_fwd(g["q"], g["k"], g["v"], g["offs"], g["nts"], workspace=ws,
+                     **dict(kw, max_seq_len=100))
+    assert sla.hstu_sla_get_error(ws) == 0
+
+
+def test_autograd_wrapper():
+    b = _edge_batch(lengths=[120, 64], nt=6)
+    g = to_gpu(b)
+    q, k, v = (g[n].clone().requires_grad_(True) for n in ("q", "k", "v"))
+    out = sla.sla_attention(q, k, v, g["offs"], g["nts"], contextual_len=3, K1=40, K2=10,
+                            alpha=128 ** -0.5, N=300.0, max_seq_len=120)
+    out.backward(g["dout"])
+    p = oracle_problem(b)
+    rq, rk, rv = p.bwd(b.q, b.k, b.v, b.dout)
+    assert_close("dq", q.grad, rq)
+    assert_close("dk", k.grad, rk)
+    assert_close("dv", v.grad, rv)

@@ -127,6 +127,13 @@ def test_row_counts_closed_form(L, nt, ctx, K1, K2):
     np.testing.assert_array_equal(p.row_counts(), _closed_form_counts(L, nt, ctx, K1, K2))
 
 
+def test_key_counts_are_column_sums():
+    for (L, nt, ctx, K1, K2) in _count_cases()[:30]:
+        p = oracle.Problem([0, L], [nt], 1, 1, ctx, K1, K2, 1.0, 1.0)
+        np.testing.assert_array_equal(p.key_counts(),
+                                      _dense_mask_textbook(L, nt, ctx, K1, K2).sum(axis=0))
+
+
 def test_mask_matches_textbook_pieces():
     for (L, nt, ctx, K1, K2) in _count_cases()[:40]:
         np.testing.assert_array_equal(oracle.mask_matrix(L, nt, ctx, K1, K2),
