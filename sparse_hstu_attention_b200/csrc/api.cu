@@ -97,9 +97,9 @@ int hstu_sla_fwd(const hstu_sla_fwd_params* p, void* workspace, size_t workspace
   AttnArgs a = make_args(p, workspace);
   a.out = static_cast<bf16*>(p->out);
   a.o_rs = p->out_row_stride;
-  cudaError_t ce = launch_worklist(a, 64, 0, st);
+  cudaError_t ce = launch_worklist(a, kFwdBM, 0, st);
   if (ce == cudaSuccess) ce = record(p->event_begin, st);
-  if (ce == cudaSuccess) ce = launch_fwd_mma(a, p->d, st);
+  if (ce == cudaSuccess) ce = launch_fwd_tc(a, p->d, st);
   if (ce == cudaSuccess) ce = record(p->event_end, st);
   return cuda_status(ce);
 }
@@ -130,7 +130,7 @@ int hstu_sla_bwd(const hstu_sla_bwd_params* p, void* workspace, size_t workspace
   a.dq_acc = reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                       ws_dq_offset(f->total_tokens, f->B));
   cudaError_t ce = cudaMemsetAsync(a.dq_acc, 0, sizeof(float) * (size_t)f->total_tokens * f->H * f->d, st);
-  if (ce == cudaSuccess) ce = launch_worklist(a, 64, 1, st);
+  if (ce == cudaSuccess) ce = launch_worklist(a, kBwdBN, 1, st);
   if (ce == cudaSuccess) ce = record(f->event_begin, st);
   if (ce == cudaSuccess) ce = launch_bwd_mma(a, f->d, st);
   if (ce == cudaSuccess) ce = record(f->event_end, st);
@@ -147,8 +147,9 @@ int hstu_sla_count_pairs(const hstu_sla_fwd_params* p, int64_t* row_counts, int6
     return e;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   AttnArgs a = make_args(p, workspace);
-  cudaError_t ce = launch_worklist(a, 64, 0, st);
-  if (ce == cudaSuccess) ce = launch_count_pairs(a, 64, 64, row_counts, key_counts, st);
+  cudaError_t ce = launch_worklist(a, kFwdBM, 0, st);
+  if (ce == cudaSuccess)
+    ce = launch_count_pairs(a, kFwdBM, kFwdBN, kBwdBM, kBwdBN, row_counts, key_counts, st);
   return cuda_status(ce);
 }
 

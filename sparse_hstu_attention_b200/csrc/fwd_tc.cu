@@ -1,0 +1,411 @@
+// SLA HSTU attention forward on the 5th-generation tensor cores (tcgen05).
+//
+//   out_i = (1/N) sum_j M(i,j) SiLU(alpha q_i.k_j) v_j
+// ("Bending the Scaling Law Curve in Large-Scale Recommendation Systems",
+// section 3, Eq. 3, under the Semi-Local Attention mask of section 4.2.1,
+// Eq. 7; candidates per the M-FALCON mask of the HSTU notes.)
+//
+// Persistent, warp-specialised: one CTA per SM walks (head, 128-row query
+// tile) work units.  Per unit only the key tiles that the SLA mask leaves
+// non-empty are visited (global prefix, local band, candidates' diagonal).
+//   warp 0      TMA producer: Q tile, then K and V tiles (128 keys) into a
+//               2-stage ring; 128B-swizzled boxes of 64 head-dim columns.
+//   warp 1      allocates TMEM; one lane issues UMMA: S = Q K^T into one of
+//               two TMEM S buffers (M=128, N=128, K=d), then O += P V with P
+//               read from TMEM (M=128, N=d, K=128) into the O accumulator.
+//   warps 2..9  pointwise: TMEM -> registers, P = SiLU(alpha S) (masked only
+//               on partial tiles) as bf16 back into TMEM; after the last key
+//               tile, the epilogue: O * (1/N) -> bf16 -> global, rows past the
+//               sequence end not written.  Two warps share each 32-lane TMEM
+//               quarter, splitting its columns.
+// TMEM columns: S0 [0,128) S1 [128,256) O [256,256+d) P0 [384,448) P1 [448,512).
+// SiLU(x) = h + h tanh(h), h = x/2: one MUFU op per score; 1/N applied once.
+// Every wait is bounded; on a timeout the kernel records HSTU_SLA_ERR_TIMEOUT,
+// drains what it issued and frees TMEM.
+#include <cudaTypedefs.h>
+
+#include "sm100.cuh"
+
+namespace hstu {
+namespace {
+
+using namespace sm100;
+
+constexpr int kBM = 128, kBN = 128, kStages = 2, kPwWarps = 8;
+constexpr int kThreads = 64 + 32 * kPwWarps;
+constexpr uint32_t kColS0 = 0, kColO = 256, kColP0 = 384, kTmemCols = 512;
+
+template <int D>
+struct Cfg {
+  static constexpr int SW = D >= 64 ? 128 : 64;   // swizzle span (bytes) = one box row
+  static constexpr int BOXW = SW / 2;             // bf16 elements per box row
+  static constexpr int NB = D / BOXW;             // boxes per tile
+  static constexpr int BLK = 128 * SW;            // bytes per box (128 rows)
+  static constexpr int TILE = 128 * D * 2;        // bytes per Q / K / V tile
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = TILE;
+  static constexpr int OFF_V = TILE * (1 + kStages);
+  static constexpr int OFF_BAR = TILE * (1 + 2 * kStages);
+  static constexpr int SMEM = OFF_BAR + 256 + 1024;  // barriers + 1 KB alignment slack
+  static constexpr uint32_t SWZ = SW == 128 ? kSwizzle128B : kSwizzle64B;
+  static constexpr uint32_t SBO = 8 * SW;             // stride of 8-row groups
+  static constexpr uint32_t IDESC_S = idesc_bf16(128, kBN, false, false);
+  static constexpr uint32_t IDESC_O = idesc_bf16(128, D, false, true);
+  static constexpr int COLS_PER_PW = kBN / (kPwWarps / 4);  // S columns per pointwise warp
+};
+
+// Barrier slots (8 bytes each) after the tiles.
+enum {
+  BAR_Q_FULL = 0, BAR_Q_EMPTY, BAR_K_FULL, BAR_K_EMPTY = BAR_K_FULL + kStages,
+  BAR_V_FULL = BAR_K_EMPTY + kStages, BAR_V_EMPTY = BAR_V_FULL + kStages,
+  BAR_S_FULL = BAR_V_EMPTY + kStages, BAR_P_FULL = BAR_S_FULL + 2, BAR_O_FULL = BAR_P_FULL + 2,
+  BAR_O_EMPTY, BAR_DRAIN, BAR_COUNT
+};
+
+struct Unit {
+  int h, s0, L, Lh, r0, r1;
+  Spans sp;
+  int ntiles;
+};
+
+__device__ __forceinline__ Unit unit_at(const AttnArgs& a, int n_items, int u) {
+  Unit w;
+  w.h = u / n_items;
+  const int2 it = a.items[u - w.h * n_items];
+  const SeqGeom g = seq_geom(a, it.x);
+  w.s0 = g.s0; w.L = g.L; w.Lh = g.Lh;
+  w.r0 = it.y * kBM;
+  w.r1 = imin(w.r0 + kBM, g.L);
+  w.sp = q_tile_key_tiles(w.r0, w.r1, g.Lh, a.K1, a.K2e, kBN);
+  w.ntiles = w.sp.count();
+  return w;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                  const __grid_constant__ CUtensorMap tmv, const AttnArgs a) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* base_ptr = smem_raw + (base - raw);
+  const uint32_t sQ = base + C::OFF_Q, sK = base + C::OFF_K, sV = base + C::OFF_V;
+  const uint32_t bar0 = base + C::OFF_BAR;
+  auto bar = [&](int i) { return bar0 + 8u * i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + C::OFF_BAR + 8 * BAR_COUNT);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (load_status(a.ws) != 0) return;  // device-side input check failed
+  const int n_items = a.ws->n_items;
+  const int total = n_items * a.H;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(BAR_Q_FULL), 1);
+    mbar_init(bar(BAR_Q_EMPTY), 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar(BAR_K_FULL + s), 1);
+      mbar_init(bar(BAR_K_EMPTY + s), 1);
+      mbar_init(bar(BAR_V_FULL + s), 1);
+      mbar_init(bar(BAR_V_EMPTY + s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(BAR_S_FULL + b), 1);
+      mbar_init(bar(BAR_P_FULL + b), 32 * kPwWarps);
+    }
+    mbar_init(bar(BAR_O_FULL), 1);
+    mbar_init(bar(BAR_O_EMPTY), 32 * kPwWarps);
+    mbar_init(bar(BAR_DRAIN), 1);
+    fence_barrier_init();
+    prefetch_tmap(&tmq);
+    prefetch_tmap(&tmk);
+    prefetch_tmap(&tmv);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t qn = 0, kv = 0, kn = 0, vn = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+        const Unit w = unit_at(a, n_items, u);
+        if (w.ntiles == 0) continue;
+        ok = mbar_wait(bar(BAR_Q_EMPTY), (qn & 1) ^ 1, a.ws);
+        if (!ok) break;
+        mbar_expect_tx(bar(BAR_Q_FULL), C::TILE);
+        for (int b = 0; b < C::NB; ++b)
+          tma_load_2d(sQ + b * C::BLK, &tmq, bar(BAR_Q_FULL), w.h * D + b * C::BOXW, w.s0 + w.r0);
+        ++qn;
+        for (int n = 0; n < w.ntiles && ok; ++n) {
+          const int y = w.s0 + w.sp.at(n) * kBN;
+          const int s = kv % kStages;
+          const uint32_t ph = (kv / kStages) & 1;
+          ok = mbar_wait(bar(BAR_K_EMPTY + s), ph ^ 1, a.ws);
+          if (!ok) break;
+          mbar_expect_tx(bar(BAR_K_FULL + s), C::TILE);
+          for (int b = 0; b < C::NB; ++b)
+            tma_load_2d(sK + s * C::TILE + b * C::BLK, &tmk, bar(BAR_K_FULL + s),
+                        w.h * D + b * C::BOXW, y);
+          ++kn;
+          ok = mbar_wait(bar(BAR_V_EMPTY + s), ph ^ 1, a.ws);
+          if (!ok) break;
+          mbar_expect_tx(bar(BAR_V_FULL + s), C::TILE);
+          for (int b = 0; b < C::NB; ++b)
+            tma_load_2d(sV + s * C::TILE + b * C::BLK, &tmv, bar(BAR_V_FULL + s),
+                        w.h * D + b * C::BOXW, y);
+          ++vn;
+          ++kv;
+        }
+      }
+      // If any role gave up, every load this thread issued must still land
+      // before the CTA exits (each barrier has at most its last armed phase
+      // outstanding).
+      if (load_status(a.ws) != 0) {
+        if (qn > 0) drain_wait(bar(BAR_Q_FULL), (qn - 1) & 1);
+        for (int s = 0; s < kStages; ++s) {
+          const uint32_t k_armed = kn / kStages + (s < (int)(kn % kStages) ? 1u : 0u);
+          const uint32_t v_armed = vn / kStages + (s < (int)(vn % kStages) ? 1u : 0u);
+          if (k_armed > 0) drain_wait(bar(BAR_K_FULL + s), (k_armed - 1) & 1);
+          if (v_armed > 0) drain_wait(bar(BAR_V_FULL + s), (v_armed - 1) & 1);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      uint32_t qn = 0, kv = 0, tc = 0, on = 0;
+      bool ok = true;
+      auto q_desc = [&](int ks) {
+        const int byte = ks * 32;  // 16 bf16 per k-step
+        return smem_desc(sQ + (byte / C::SW) * C::BLK + (byte % C::SW), 16, C::SBO, C::SWZ);
+      };
+      auto k_desc = [&](int s, int ks) {
+        const int byte = ks * 32;
+        return smem_desc(sK + s * C::TILE + (byte / C::SW) * C::BLK + (byte % C::SW), 16, C::SBO,
+                         C::SWZ);
+      };
+      auto v_desc = [&](int s, int ks) {  // V tile as MN-major B: 16 keys per k-step
+        return smem_desc(sV + s * C::TILE + ks * 16 * C::SW, C::BLK, C::SBO, C::SWZ);
+      };
+      // O += P(tile m) V(tile m); kvm / tcm: that tile's ring / S-buffer counters.
+      auto pv = [&](uint32_t kvm, uint32_t tcm, bool first) -> bool {
+        const uint32_t b = tcm & 1;
+        if (!mbar_wait(bar(BAR_P_FULL + b), (tcm >> 1) & 1, a.ws)) return false;
+        const int s = kvm % kStages;
+        if (!mbar_wait(bar(BAR_V_FULL + s), (kvm / kStages) & 1, a.ws)) return false;
+        if (first && !mbar_wait(bar(BAR_O_EMPTY), (on & 1) ^ 1, a.ws)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < kBN / 16; ++ks)
+          mma_ts(tmem + kColO, tmem + kColP0 + b * 64 + ks * 8, v_desc(s, ks), C::IDESC_O,
+                 (!first || ks > 0) ? 1u : 0u);
+        tc_commit(bar(BAR_V_EMPTY + s));
+        return true;
+      };
+      for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+        const Unit w = unit_at(a, n_items, u);
+        if (w.ntiles == 0) continue;
+        ok = mbar_wait(bar(BAR_Q_FULL), qn & 1, a.ws);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t kv0 = kv, tc0 = tc;
+        for (int n = 0; n < w.ntiles; ++n) {
+          const int s = kv % kStages;
+          ok = mbar_wait(bar(BAR_K_FULL + s), (kv / kStages) & 1, a.ws);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t b = tc & 1;
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks)
+            mma_ss(tmem + kColS0 + b * 128, q_desc(ks), k_desc(s, ks), C::IDESC_S,
+                   ks > 0 ? 1u : 0u);
+          tc_commit(bar(BAR_S_FULL + b));
+          tc_commit(bar(BAR_K_EMPTY + s));
+          if (n > 0) {
+            ok = pv(kv - 1, tc - 1, n == 1);
+            if (!ok) break;
+          }
+          ++kv;
+          ++tc;
+        }
+        if (!ok) break;
+        ok = pv(kv0 + w.ntiles - 1, tc0 + w.ntiles - 1, w.ntiles == 1);
+        if (!ok) break;
+        tc_commit(bar(BAR_Q_EMPTY));
+        tc_commit(bar(BAR_O_FULL));
+        ++qn;
+        ++on;
+      }
+      // Every MMA issued must finish before TMEM is released.
+      tc_commit(bar(BAR_DRAIN));
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try_wait(bar(BAR_DRAIN), 0) && globaltimer() - t0 < kWaitLimitNs) {}
+    }
+  } else {
+    // ----------------------------------------------- pointwise and epilogue
+    const int pw = warp - 2;               // 0..7
+    const int quarter = warp & 3;          // TMEM lanes [32*quarter, +32)
+    const int half = pw >> 2;              // which column half of the tile
+    const int row = quarter * 32 + lane;   // row of the 128-row tile
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    const float half_alpha = 0.5f * a.alpha;
+    uint32_t tc = 0, on = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+      const Unit w = unit_at(a, n_items, u);
+      const int i = w.r0 + row;  // row within the sequence
+      bf16* orow = a.out + (int64_t)(w.s0 + i) * a.o_rs + w.h * D;
+      if (w.ntiles == 0) {  // no visible key anywhere in the tile
+        if (i < w.r1) {
+          const uint4 z = make_uint4(0, 0, 0, 0);
+          for (int c = half; c < D / 32; c += 2)
+#pragma unroll
+            for (int v = 0; v < 4; ++v) reinterpret_cast<uint4*>(orow + c * 32)[v] = z;
+        }
+        continue;
+      }
+      const RowMask m = row_mask(i, w.L, w.Lh, a.K1, a.K2e);
+      for (int n = 0; n < w.ntiles; ++n) {
+        const uint32_t b = tc & 1;
+        ok = mbar_wait(bar(BAR_S_FULL + b), (tc >> 1) & 1, a.ws);
+        if (!ok) break;
+        tc_fence_after();
+        const int j0 = w.sp.at(n) * kBN;
+        const bool full = tile_full(w.r0, w.r1, j0, imin(j0 + kBN, w.L), w.Lh, a.K1, a.K2e);
+#pragma unroll
+        for (int c = 0; c < C::COLS_PER_PW / 32; ++c) {
+          const int col = half * C::COLS_PER_PW + c * 32;
+          uint32_t r[32];
+          tmem_ld32(lane_base + kColS0 + b * 128 + col, r);
+          tmem_ld_wait(r);
+          uint32_t p[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float h0 = __uint_as_float(r[2 * e]) * half_alpha;
+            const float h1 = __uint_as_float(r[2 * e + 1]) * half_alpha;
+            float p0 = fmaf(h0, tanh_approx(h0), h0);
+            float p1 = fmaf(h1, tanh_approx(h1), h1);
+            if (!full) {
+              const int j = j0 + col + 2 * e;
+              p0 = m(j) ? p0 : 0.f;
+              p1 = m(j + 1) ? p1 : 0.f;
+            }
+            p[e] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(lane_base + kColP0 + b * 64 + col / 2, p);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar(BAR_P_FULL + b));
+        ++tc;
+      }
+      if (!ok) break;
+      // epilogue
+      ok = mbar_wait(bar(BAR_O_FULL), on & 1, a.ws);
+      if (!ok) break;
+      tc_fence_after();
+      // 32-column chunks of O alternate between the two warps of a quarter
+      for (int c = half; c < D / 32; c += 2) {
+        uint32_t r[32];
+        tmem_ld32(lane_base + kColO + c * 32, r);
+        tmem_ld_wait(r);
+        if (i < w.r1) {
+          uint32_t o[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            o[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * a.inv_n,
+                               __uint_as_float(r[2 * e + 1]) * a.inv_n);
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            dst[v] = make_uint4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(BAR_O_EMPTY));
+      ++on;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D map over a [T, H*D] bf16 matrix with row stride rs elements; boxes of
+// box_w columns x 128 rows, swizzled to match the UMMA descriptors.
+bool make_map(CUtensorMap* m, const void* ptr, int64_t T, int HD, int64_t rs, int box_w,
+              bool sw128) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)HD, (cuuint64_t)T};
+  cuuint64_t strides[1] = {(cuuint64_t)(rs * 2)};
+  cuuint32_t box[2] = {(cuuint32_t)box_w, 128u};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  sw128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+template <int D>
+cudaError_t launch_d(const AttnArgs& a, cudaStream_t st) {
+  using C = Cfg<D>;
+  CUtensorMap mq, mk, mv;
+  const int HD = a.H * D;
+  if (!make_map(&mq, a.q, a.T, HD, a.q_rs, C::BOXW, C::SW == 128) ||
+      !make_map(&mk, a.k, a.T, HD, a.k_rs, C::BOXW, C::SW == 128) ||
+      !make_map(&mv, a.v, a.T, HD, a.v_rs, C::BOXW, C::SW == 128))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  const int64_t units = max_items(a.T, a.B) * a.H;
+  const int grid = (int)(units < num_sms() ? units : num_sms());
+  fwd_tc_kernel<D><<<grid, kThreads, C::SMEM, st>>>(mq, mk, mv, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_tc(const AttnArgs& a, int d, cudaStream_t st) {
+  if (a.T == 0) return cudaSuccess;
+  if (d == 32) return launch_d<32>(a, st);
+  if (d == 64) return launch_d<64>(a, st);
+  return launch_d<128>(a, st);
+}
+
+}  // namespace hstu

@@ -37,6 +37,11 @@ static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 
 constexpr int kMinTile = 64;  // smallest tile any kernel enumerates with
 
+// Tile shapes of the kernels the entry points launch (the pair-count hook
+// walks the same enumeration).
+constexpr int kFwdBM = 128, kFwdBN = 128;  // tcgen05 forward
+constexpr int kBwdBM = 64, kBwdBN = 64;    // backward
+
 __host__ __device__ inline int64_t max_items(int64_t T, int B) {
   return (T + kMinTile - 1) / kMinTile + B;
 }
@@ -221,10 +226,11 @@ __device__ __forceinline__ int load_status(const WsHeader* ws) {
 // ------------------------------------------------------------ host launchers
 // (defined in the .cu files; return cudaError_t of the launch)
 cudaError_t launch_worklist(const AttnArgs& a, int tile, int backward, cudaStream_t st);
-cudaError_t launch_count_pairs(const AttnArgs& a, int BM, int BN, int64_t* row_counts,
-                               int64_t* key_counts, cudaStream_t st);
+cudaError_t launch_count_pairs(const AttnArgs& a, int BMf, int BNf, int BMb, int BNb,
+                               int64_t* row_counts, int64_t* key_counts, cudaStream_t st);
 cudaError_t launch_dq_convert(const AttnArgs& a, int d, cudaStream_t st);
 cudaError_t launch_fwd_mma(const AttnArgs& a, int d, cudaStream_t st);
+cudaError_t launch_fwd_tc(const AttnArgs& a, int d, cudaStream_t st);
 cudaError_t launch_bwd_mma(const AttnArgs& a, int d, cudaStream_t st);
 
 }  // namespace hstu

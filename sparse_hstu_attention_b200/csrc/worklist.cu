@@ -111,8 +111,8 @@ __global__ void __launch_bounds__(kWlThreads) worklist_kernel(AttnArgs a, int ti
 // Per token: number of visible keys found by walking the forward enumeration
 // (row_counts), and number of rows that see it found by walking the backward
 // enumeration (key_counts).
-__global__ void count_pairs_kernel(AttnArgs a, int BM, int BN, int64_t* row_counts,
-                                   int64_t* key_counts) {
+__global__ void count_pairs_kernel(AttnArgs a, int BMf, int BNf, int BMb, int BNb,
+                                   int64_t* row_counts, int64_t* key_counts) {
   if (load_status(a.ws) != 0) return;
   int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   if (t >= a.T) return;
@@ -124,23 +124,23 @@ __global__ void count_pairs_kernel(AttnArgs a, int BM, int BN, int64_t* row_coun
   SeqGeom g = seq_geom(a, lo);
   int p = int(t - g.s0);
   if (row_counts) {
-    int r0 = (p / BM) * BM, r1 = imin(r0 + BM, g.L);
-    Spans s = q_tile_key_tiles(r0, r1, g.Lh, a.K1, a.K2e, BN);
+    int r0 = (p / BMf) * BMf, r1 = imin(r0 + BMf, g.L);
+    Spans s = q_tile_key_tiles(r0, r1, g.Lh, a.K1, a.K2e, BNf);
     int64_t n = 0;
     for (int e = 0; e < s.count(); ++e) {
       int kt = s.at(e);
-      for (int j = kt * BN; j < imin(kt * BN + BN, g.L); ++j)
+      for (int j = kt * BNf; j < imin(kt * BNf + BNf, g.L); ++j)
         n += sla_visible(p, j, g.L, g.Lh, a.K1, a.K2e);
     }
     row_counts[t] = n;
   }
   if (key_counts) {
-    int j0 = (p / BN) * BN, j1 = imin(j0 + BN, g.L);
-    Spans s = k_tile_q_tiles(j0, j1, g.L, g.Lh, a.K1, a.K2e, BM);
+    int j0 = (p / BNb) * BNb, j1 = imin(j0 + BNb, g.L);
+    Spans s = k_tile_q_tiles(j0, j1, g.L, g.Lh, a.K1, a.K2e, BMb);
     int64_t n = 0;
     for (int e = 0; e < s.count(); ++e) {
       int qt = s.at(e);
-      for (int i = qt * BM; i < imin(qt * BM + BM, g.L); ++i)
+      for (int i = qt * BMb; i < imin(qt * BMb + BMb, g.L); ++i)
         n += sla_visible(i, p, g.L, g.Lh, a.K1, a.K2e);
     }
     key_counts[t] = n;
@@ -172,12 +172,13 @@ cudaError_t launch_worklist(const AttnArgs& a, int tile, int backward, cudaStrea
   return cudaGetLastError();
 }
 
-cudaError_t launch_count_pairs(const AttnArgs& a, int BM, int BN, int64_t* row_counts,
-                               int64_t* key_counts, cudaStream_t st) {
+cudaError_t launch_count_pairs(const AttnArgs& a, int BMf, int BNf, int BMb, int BNb,
+                               int64_t* row_counts, int64_t* key_counts, cudaStream_t st) {
   if (a.T == 0) return cudaSuccess;
   int threads = 256;
   int64_t blocks = (a.T + threads - 1) / threads;
-  count_pairs_kernel<<<(unsigned)blocks, threads, 0, st>>>(a, BM, BN, row_counts, key_counts);
+  count_pairs_kernel<<<(unsigned)blocks, threads, 0, st>>>(a, BMf, BNf, BMb, BNb, row_counts,
+                                                           key_counts);
   return cudaGetLastError();
 }
 
