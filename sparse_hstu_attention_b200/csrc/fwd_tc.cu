@@ -275,7 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const RowMask m = row_mask(i, w.L, w.Lh, a.K1, a.K2e);
       for (int n = 0; n < w.ntiles; ++n) {
         const uint32_t b = tc & 1;
-        ok = mbar_wait(bar(BAR_S_FULL + b), (tc >> 1) & 1, a.ws);
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(BAR_S_FULL + b), (tc >> 1) & 1, a.ws));
         if (!ok) break;
         tc_fence_after();
         const int j0 = w.sp.at(n) * kBN;
@@ -309,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
       // epilogue
-      ok = mbar_wait(bar(BAR_O_FULL), on & 1, a.ws);
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(BAR_O_FULL), on & 1, a.ws));
       if (!ok) break;
       tc_fence_after();
       // 32-column chunks of O alternate between the two warps of a quarter
