@@ -37,9 +37,10 @@ from workloads import WORKLOADS, make_batch  # noqa: E402
 
 METRIC = "SLA HSTU attn fwd+bwd TFLOP/s (unmasked pairs), % of B200 BF16 peak"
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0}
-KERNEL_SOURCES = {"fwd": "sparse_hstu_attention_b200/csrc/fwd_mma.cu",
-                  "bwd": "sparse_hstu_attention_b200/csrc/bwd_mma.cu"}
-KERNEL_NAMES = {"fwd": "fwd_mma_kernel", "bwd": "bwd_mma_kernel"}
+KERNEL_SOURCES = {"fwd": "sparse_hstu_attention_b200/csrc/fwd_tc.cu",
+                  "bwd": "sparse_hstu_attention_b200/csrc/bwd_tc.cu"}
+KERNEL_NAMES = {"fwd": "fwd_tc_kernel", "bwd": "bwd_tc_kernel (KV pass + Q pass)"}
+LAUNCHES_PER_STEP = {"fwd": 2, "bwd": 4}  # work list(s) + attention kernel(s)
 
 
 def _peaks():
@@ -52,7 +53,10 @@ def _peaks():
 
 
 def _sha1(path):
-    with open(os.path.join(ROOT, path), "rb") as f:
+    p = os.path.join(ROOT, path)
+    if not os.path.exists(p):
+        return None
+    with open(p, "rb") as f:
         return hashlib.sha1(f.read()).hexdigest()
 
 
@@ -377,7 +381,8 @@ def main():
                      "algorithmic_flops_per_launch": dom_fl},
         "e2e": {"value": world * (fl_f + fl_b) / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": K * (2 if w.fwd_only else 5),
+        "gpu_launches": K * (LAUNCHES_PER_STEP["fwd"] +
+                             (0 if w.fwd_only else LAUNCHES_PER_STEP["bwd"])),
         "clocks": clocks.summary(),
     }
     if world == 1 and not args.no_cpu_baseline:

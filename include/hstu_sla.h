@@ -108,8 +108,9 @@ typedef struct {
 
 /* Bytes of device workspace hstu_sla_fwd (which = HSTU_SLA_WS_FWD) or
  * hstu_sla_bwd (HSTU_SLA_WS_BWD) needs for a batch of total_tokens tokens in
- * B sequences.  The workspace must be 256-byte aligned; the backward one holds
- * an fp32 dq accumulator of T*H*d floats.  Returns 0 on invalid arguments. */
+ * B sequences: a status word and the device-built work lists, about
+ * 16 * (total_tokens / 64 + B) bytes (H and d do not change it).  The
+ * workspace must be 256-byte aligned.  Returns 0 on invalid arguments. */
 size_t hstu_sla_workspace_bytes(int which, int64_t total_tokens, int32_t B, int32_t H,
                                 int32_t d);
 
@@ -119,9 +120,9 @@ size_t hstu_sla_workspace_bytes(int which, int64_t total_tokens, int32_t B, int3
 int hstu_sla_fwd(const hstu_sla_fwd_params* p, void* workspace, size_t workspace_bytes,
                  hstu_stream_t stream);
 
-/* Backward: writes p->dq, p->dk, p->dv (bf16).  Key-tile-parallel: dk/dv are
- * accumulated on chip without atomics; dq is reduced in the fp32 workspace and
- * converted at the end. */
+/* Backward: writes p->dq, p->dk, p->dv (bf16).  Two passes, no atomics, a
+ * deterministic result: a key-tile pass accumulates dk/dv on chip, a
+ * query-tile pass recomputes the scores and accumulates dq on chip. */
 int hstu_sla_bwd(const hstu_sla_bwd_params* p, void* workspace, size_t workspace_bytes,
                  hstu_stream_t stream);
 

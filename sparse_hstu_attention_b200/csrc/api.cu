@@ -49,6 +49,8 @@ AttnArgs make_args(const hstu_sla_fwd_params* f, void* ws) {
   a.nts = f->num_targets;
   a.ws = reinterpret_cast<WsHeader*>(ws);
   a.items = reinterpret_cast<const int2*>(static_cast<char*>(ws) + ws_items_offset());
+  a.items2 = reinterpret_cast<const int2*>(static_cast<char*>(ws) +
+                                           ws_items2_offset(f->total_tokens, f->B));
   a.B = f->B;
   a.H = f->H;
   a.K1 = f->K1;
@@ -79,9 +81,7 @@ extern "C" {
 size_t hstu_sla_workspace_bytes(int which, int64_t total_tokens, int32_t B, int32_t H,
                                 int32_t d) {
   if (total_tokens < 0 || B < 1 || H < 1 || d < 1) return 0;
-  if (which == HSTU_SLA_WS_FWD) return ws_dq_offset(total_tokens, B);
-  if (which == HSTU_SLA_WS_BWD)
-    return ws_dq_offset(total_tokens, B) + align256(sizeof(float) * (size_t)total_tokens * H * d);
+  if (which == HSTU_SLA_WS_FWD || which == HSTU_SLA_WS_BWD) return ws_bytes(total_tokens, B);
   return 0;
 }
 
@@ -127,14 +127,12 @@ int hstu_sla_bwd(const hstu_sla_bwd_params* p, void* workspace, size_t workspace
   a.dq_rs = p->dq_row_stride;
   a.dk_rs = p->dk_row_stride;
   a.dv_rs = p->dv_row_stride;
-  a.dq_acc = reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                      ws_dq_offset(f->total_tokens, f->B));
-  cudaError_t ce = cudaMemsetAsync(a.dq_acc, 0, sizeof(float) * (size_t)f->total_tokens * f->H * f->d, st);
-  if (ce == cudaSuccess) ce = launch_worklist(a, kBwdBN, 1, st);
+  cudaError_t ce = launch_worklist(a, kQpBM, 0, st);
+  if (ce == cudaSuccess) ce = launch_worklist(a, kKvBN, 1, st);
   if (ce == cudaSuccess) ce = record(f->event_begin, st);
-  if (ce == cudaSuccess) ce = launch_bwd_mma(a, f->d, st);
+  if (ce == cudaSuccess) ce = launch_bwd_tc(a, f->d, /*kv_pass=*/true, st);
+  if (ce == cudaSuccess) ce = launch_bwd_tc(a, f->d, /*kv_pass=*/false, st);
   if (ce == cudaSuccess) ce = record(f->event_end, st);
-  if (ce == cudaSuccess) ce = launch_dq_convert(a, f->d, st);
   return cuda_status(ce);
 }
 
@@ -149,7 +147,7 @@ int hstu_sla_count_pairs(const hstu_sla_fwd_params* p, int64_t* row_counts, int6
   AttnArgs a = make_args(p, workspace);
   cudaError_t ce = launch_worklist(a, kFwdBM, 0, st);
   if (ce == cudaSuccess)
-    ce = launch_count_pairs(a, kFwdBM, kFwdBN, kBwdBM, kBwdBN, row_counts, key_counts, st);
+    ce = launch_count_pairs(a, kFwdBM, kFwdBN, kKvBM, kKvBN, row_counts, key_counts, st);
   return cuda_status(ce);
 }
 

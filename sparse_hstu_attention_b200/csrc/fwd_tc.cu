@@ -27,6 +27,11 @@
 #include "sm100.cuh"
 
 namespace hstu {
+
+bool make_tma_2d(CUtensorMap* m, const void* ptr, int64_t T, int HD, int64_t rs, int box_w,
+                 int box_h, bool sw128);
+int device_sm_count();
+
 namespace {
 
 using namespace sm100;
@@ -279,7 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         const int j0 = w.sp.at(n) * kBN;
-        const bool full = tile_full(w.r0, w.r1, j0, imin(j0 + kBN, w.L), w.Lh, a.K1, a.K2e);
+        const bool full = tile_full(w.r0, w.r0 + kBM, j0, j0 + kBN, w.Lh, a.K1, a.K2e);
 #pragma unroll
         for (int c = 0; c < C::COLS_PER_PW / 32; ++c) {
           const int col = half * C::COLS_PER_PW + c * 32;
@@ -344,57 +349,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (fn == nullptr) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
-// 2-D map over a [T, H*D] bf16 matrix with row stride rs elements; boxes of
-// box_w columns x 128 rows, swizzled to match the UMMA descriptors.
-bool make_map(CUtensorMap* m, const void* ptr, int64_t T, int HD, int64_t rs, int box_w,
-              bool sw128) {
-  auto fn = encode_fn();
-  if (fn == nullptr) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)HD, (cuuint64_t)T};
-  cuuint64_t strides[1] = {(cuuint64_t)(rs * 2)};
-  cuuint32_t box[2] = {(cuuint32_t)box_w, 128u};
-  cuuint32_t estr[2] = {1u, 1u};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  sw128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
-int num_sms() {
-  int dev = 0, n = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n > 0 ? n : 148;
-}
-
 template <int D>
 cudaError_t launch_d(const AttnArgs& a, cudaStream_t st) {
   using C = Cfg<D>;
   CUtensorMap mq, mk, mv;
   const int HD = a.H * D;
-  if (!make_map(&mq, a.q, a.T, HD, a.q_rs, C::BOXW, C::SW == 128) ||
-      !make_map(&mk, a.k, a.T, HD, a.k_rs, C::BOXW, C::SW == 128) ||
-      !make_map(&mv, a.v, a.T, HD, a.v_rs, C::BOXW, C::SW == 128))
+  if (!make_tma_2d(&mq, a.q, a.T, HD, a.q_rs, C::BOXW, kBM, C::SW == 128) ||
+      !make_tma_2d(&mk, a.k, a.T, HD, a.k_rs, C::BOXW, kBN, C::SW == 128) ||
+      !make_tma_2d(&mv, a.v, a.T, HD, a.v_rs, C::BOXW, kBN, C::SW == 128))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   const int64_t units = max_items(a.T, a.B) * a.H;
-  const int grid = (int)(units < num_sms() ? units : num_sms());
+  const int sms = device_sm_count();
+  const int grid = (int)(units < sms ? units : sms);
   fwd_tc_kernel<D><<<grid, kThreads, C::SMEM, st>>>(mq, mk, mv, a);
   return cudaGetLastError();
 }

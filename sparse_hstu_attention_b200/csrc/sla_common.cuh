@@ -24,14 +24,17 @@ using bf16 = __nv_bfloat16;
 
 // ---------------------------------------------------------------- workspace
 // [0, 256)            WsHeader
-// [256, ...)          int2 items[max_items]   (sequence, tile) pairs
-// [align256, ...)     float dq_acc[T * H * d] (backward only)
+// [256, ...)          int2 items[max_items]   list 0: (sequence, query tile)
+// [align256, ...)     int2 items2[max_items]  list 1: (sequence, key tile),
+//                                             prefix key tiles first
 struct WsHeader {
-  int32_t status;       // HSTU_SLA_OK or a negative code
-  int32_t n_items;      // items written by the work-list kernel
-  int32_t n_items_pre;  // backward: leading items that hold prefix key tiles
-  int32_t sched;        // dynamic tile scheduler counter (persistent kernels)
-  int32_t pad[60];
+  int32_t status;        // HSTU_SLA_OK or a negative code
+  int32_t n_items;       // entries of list 0
+  int32_t n_items2;      // entries of list 1
+  int32_t n_items2_pre;  // leading entries of list 1 that hold prefix key tiles
+  int32_t sched;         // dynamic scheduler counter over list 0 units
+  int32_t sched2;        // dynamic scheduler counter over list 1 units
+  int32_t pad[58];
 };
 static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 
@@ -39,23 +42,28 @@ constexpr int kMinTile = 64;  // smallest tile any kernel enumerates with
 
 // Tile shapes of the kernels the entry points launch (the pair-count hook
 // walks the same enumeration).
-constexpr int kFwdBM = 128, kFwdBN = 128;  // tcgen05 forward
-constexpr int kBwdBM = 64, kBwdBN = 64;    // backward
+constexpr int kFwdBM = 128, kFwdBN = 128;  // forward: query tile x key tile
+constexpr int kKvBN = 128, kKvBM = 64;     // backward KV pass: key tile x streamed rows
+constexpr int kQpBM = 128, kQpBN = 64;     // backward Q pass: query tile x streamed keys
 
 __host__ __device__ inline int64_t max_items(int64_t T, int B) {
   return (T + kMinTile - 1) / kMinTile + B;
 }
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 __host__ __device__ inline size_t ws_items_offset() { return sizeof(WsHeader); }
-__host__ __device__ inline size_t ws_dq_offset(int64_t T, int B) {
+__host__ __device__ inline size_t ws_items2_offset(int64_t T, int B) {
   return align256(ws_items_offset() + sizeof(int2) * size_t(max_items(T, B)));
+}
+__host__ __device__ inline size_t ws_bytes(int64_t T, int B) {
+  return align256(ws_items2_offset(T, B) + sizeof(int2) * size_t(max_items(T, B)));
 }
 
 // ------------------------------------------------------------ kernel args
 struct AttnArgs {
   const int32_t* offs;   // [B+1]
   const int32_t* nts;    // [B] or null
-  const int2* items;     // work list
+  const int2* items;     // work list 0 (query tiles)
+  const int2* items2;    // work list 1 (key tiles)
   WsHeader* ws;          // status / counts
   int B, H, K1, K2e, max_seq_len;
   int64_t T;
@@ -68,7 +76,6 @@ struct AttnArgs {
   bf16* dq;
   bf16* dk;
   bf16* dv;
-  float* dq_acc;
   int64_t q_rs, k_rs, v_rs, do_rs, o_rs, dq_rs, dk_rs, dv_rs;
 };
 
@@ -208,11 +215,43 @@ __host__ __device__ inline Spans k_tile_q_tiles(int j0, int j1, int L, int Lh, i
   return s;
 }
 
-// True if every (row, key) pair of rows [r0, r1) x keys [j0, j1) is visible,
-// so the mask need not be evaluated.
+// True if every (row, key) pair of rows [r0, r1) x keys [j0, j1) lies inside
+// the sequence and is visible, so the mask need not be evaluated.  Callers pass
+// the UNCLIPPED tile ends (r0 + BM, j0 + BN): a tile that runs past the
+// sequence end is never full, so rows / keys past the end are always masked.
 __host__ __device__ __forceinline__ bool tile_full(int r0, int r1, int j0, int j1, int Lh, int K1,
-                                          int K2e) {
+                                                   int K2e) {
   return r1 <= Lh && j1 <= r0 + 1 && (j1 <= K2e || j0 >= r1 - K1);
+}
+
+// The visible rows of key j as intervals, for inner loops of the key-major
+// backward: visible(i) = (lo <= i < hi) || (tlo <= i < thi) || i == self.
+struct KeyMask {
+  int lo, hi, tlo, thi, self;
+  __host__ __device__ __forceinline__ bool operator()(int i) const {
+    return (i >= lo && i < hi) || (i >= tlo && i < thi) || i == self;
+  }
+};
+
+__host__ __device__ __forceinline__ KeyMask key_mask(int j, int L, int Lh, int K1, int K2e) {
+  KeyMask m;
+  m.lo = m.hi = m.tlo = m.thi = 0;
+  m.self = -1;
+  if (j >= L || j < 0) return m;
+  if (j >= Lh) {          // a candidate key: seen by that candidate only
+    m.self = j;
+  } else if (j < K2e) {   // a prefix key: every row from j on
+    m.lo = j;
+    m.hi = L;
+  } else {                // history rows of its window; candidates if in theirs
+    m.lo = j;
+    m.hi = imin(j + K1, Lh);
+    if (Lh - j < K1) {
+      m.tlo = Lh;
+      m.thi = L;
+    }
+  }
+  return m;
 }
 
 __device__ __forceinline__ void set_status(WsHeader* ws, int code) {
@@ -225,12 +264,12 @@ __device__ __forceinline__ int load_status(const WsHeader* ws) {
 
 // ------------------------------------------------------------ host launchers
 // (defined in the .cu files; return cudaError_t of the launch)
-cudaError_t launch_worklist(const AttnArgs& a, int tile, int backward, cudaStream_t st);
+// list 0: (sequence, query tile of `tile` rows); list 1: (sequence, key tile
+// of `tile` keys), prefix key tiles first.
+cudaError_t launch_worklist(const AttnArgs& a, int tile, int list, cudaStream_t st);
 cudaError_t launch_count_pairs(const AttnArgs& a, int BMf, int BNf, int BMb, int BNb,
                                int64_t* row_counts, int64_t* key_counts, cudaStream_t st);
-cudaError_t launch_dq_convert(const AttnArgs& a, int d, cudaStream_t st);
-cudaError_t launch_fwd_mma(const AttnArgs& a, int d, cudaStream_t st);
 cudaError_t launch_fwd_tc(const AttnArgs& a, int d, cudaStream_t st);
-cudaError_t launch_bwd_mma(const AttnArgs& a, int d, cudaStream_t st);
+cudaError_t launch_bwd_tc(const AttnArgs& a, int d, bool kv_pass, cudaStream_t st);
 
 }  // namespace hstu

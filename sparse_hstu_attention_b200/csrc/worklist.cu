@@ -1,5 +1,5 @@
-// Work-list construction, device-side input validation, the pair-count test
-// hook and the dq fp32 -> bf16 conversion.
+// Work-list construction, device-side input validation and the pair-count
+// test hook.
 //
 // The work list is built on the device from seq_offsets / num_targets, so a
 // call never waits on the host.  Forward items are (sequence, query tile);
@@ -42,13 +42,14 @@ __device__ int block_exclusive_scan(int v, int* out, int* smem) {
   return total;
 }
 
-// One block.  backward = 0: items (b, query tile) in sequence order.
-// backward = 1: first every (b, key tile) whose key tile starts inside the
-// history prefix [0, min(K2eff, Lh)), then all other key tiles.
-__global__ void __launch_bounds__(kWlThreads) worklist_kernel(AttnArgs a, int tile, int backward) {
+// One block.  list 0: items (b, query tile) in sequence order.  list 1:
+// first every (b, key tile) whose key tile starts inside the history prefix
+// [0, min(K2eff, Lh)), then all other key tiles.
+__global__ void __launch_bounds__(kWlThreads) worklist_kernel(AttnArgs a, int tile, int list) {
   __shared__ int s_scan[32];
   __shared__ int s_bad;
-  int2* items = const_cast<int2*>(a.items);
+  const int backward = list;
+  int2* items = const_cast<int2*>(list ? a.items2 : a.items);
   if (threadIdx.x == 0) s_bad = 0;
   __syncthreads();
   // validation of the device-resident offsets and targets
@@ -69,8 +70,10 @@ __global__ void __launch_bounds__(kWlThreads) worklist_kernel(AttnArgs a, int ti
     if (threadIdx.x == 0) {
       a.ws->status = HSTU_SLA_ERR_BAD_INPUT;
       a.ws->n_items = 0;
-      a.ws->n_items_pre = 0;
+      a.ws->n_items2 = 0;
+      a.ws->n_items2_pre = 0;
       a.ws->sched = 0;
+      a.ws->sched2 = 0;
     }
     return;
   }
@@ -101,10 +104,15 @@ __global__ void __launch_bounds__(kWlThreads) worklist_kernel(AttnArgs a, int ti
     if (pass == 0) n_pre = written;
   }
   if (threadIdx.x == 0) {
-    a.ws->status = HSTU_SLA_OK;
-    a.ws->n_items = written;
-    a.ws->n_items_pre = n_pre;
-    a.ws->sched = 0;
+    if (list) {
+      a.ws->n_items2 = written;
+      a.ws->n_items2_pre = n_pre;
+      a.ws->sched2 = 0;
+    } else {
+      a.ws->status = HSTU_SLA_OK;  // list 0 is always built first
+      a.ws->n_items = written;
+      a.ws->sched = 0;
+    }
   }
 }
 
@@ -147,28 +155,10 @@ __global__ void count_pairs_kernel(AttnArgs a, int BMf, int BNf, int BMb, int BN
   }
 }
 
-// dq[t, h, :] (bf16, strided) = dq_acc[t, h, :] (fp32, dense), 8 values a thread.
-template <int D>
-__global__ void dq_convert_kernel(AttnArgs a) {
-  if (load_status(a.ws) != 0) return;
-  const int64_t chunks = a.T * a.H * (D / 8);
-  for (int64_t c = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; c < chunks;
-       c += (int64_t)gridDim.x * blockDim.x) {
-    int64_t e = c * 8;
-    int64_t t = e / (a.H * D);
-    int64_t hc = e - t * (a.H * D);
-    const float4* src = reinterpret_cast<const float4*>(a.dq_acc + e);
-    float4 x = src[0], y = src[1];
-    __nv_bfloat162 o[4] = {__floats2bfloat162_rn(x.x, x.y), __floats2bfloat162_rn(x.z, x.w),
-                           __floats2bfloat162_rn(y.x, y.y), __floats2bfloat162_rn(y.z, y.w)};
-    *reinterpret_cast<uint4*>(a.dq + t * a.dq_rs + hc) = *reinterpret_cast<uint4*>(o);
-  }
-}
-
 }  // namespace
 
-cudaError_t launch_worklist(const AttnArgs& a, int tile, int backward, cudaStream_t st) {
-  worklist_kernel<<<1, kWlThreads, 0, st>>>(a, tile, backward);
+cudaError_t launch_worklist(const AttnArgs& a, int tile, int list, cudaStream_t st) {
+  worklist_kernel<<<1, kWlThreads, 0, st>>>(a, tile, list);
   return cudaGetLastError();
 }
 
@@ -179,15 +169,6 @@ cudaError_t launch_count_pairs(const AttnArgs& a, int BMf, int BNf, int BMb, int
   int64_t blocks = (a.T + threads - 1) / threads;
   count_pairs_kernel<<<(unsigned)blocks, threads, 0, st>>>(a, BMf, BNf, BMb, BNb, row_counts,
                                                            key_counts);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_dq_convert(const AttnArgs& a, int d, cudaStream_t st) {
-  if (a.T == 0) return cudaSuccess;
-  int threads = 256, blocks = 148 * 8;
-  if (d == 32) dq_convert_kernel<32><<<blocks, threads, 0, st>>>(a);
-  else if (d == 64) dq_convert_kernel<64><<<blocks, threads, 0, st>>>(a);
-  else dq_convert_kernel<128><<<blocks, threads, 0, st>>>(a);
   return cudaGetLastError();
 }
 

@@ -5,8 +5,10 @@
 //   - every visible (row, key) pair lies in an enumerated (query tile, key tile)
 //     pair, from the query side (forward) and from the key side (backward);
 //   - no enumerated (query tile, key tile) pair is empty, from either side;
-//   - tile_full() is only true when every pair in the tile is visible;
-//   - the per-row interval form row_mask() equals the predicate.
+//   - tile_full() on an unclipped tile is only true when every pair of the
+//     tile lies inside the sequence and is visible;
+//   - the per-row and per-key interval forms row_mask() / key_mask() equal the
+//     predicate.
 // Prints "OK <cases>" or the first failure.
 #include <cstdio>
 #include <cstdlib>
@@ -30,6 +32,7 @@ static int check(int L, int nt, int K1, int K2e, int BM, int BN) {
     RowMask m = row_mask(i, L, Lh, K1, K2e);
     for (int j = 0; j < L; ++j) {
       bool v = vis(i, j, L, Lh, K1, K2e);
+      if (v != key_mask(j, L, Lh, K1, K2e)(i)) { printf("key_mask mismatch L=%d nt=%d K1=%d K2e=%d i=%d j=%d\n", L, nt, K1, K2e, i, j); return 1; }
       if (v != m(j)) { printf("row_mask mismatch L=%d nt=%d K1=%d K2e=%d i=%d j=%d\n", L, nt, K1, K2e, i, j); return 1; }
       if (v) qk[size_t(i / BM) * nk + j / BN] = 1;
     }
@@ -42,10 +45,11 @@ static int check(int L, int nt, int K1, int K2e, int BM, int BN) {
       if (kt < 0 || kt >= nk) { printf("fwd tile out of range\n"); return 1; }
       if (fwd[size_t(qt) * nk + kt]) { printf("fwd tile twice\n"); return 1; }
       fwd[size_t(qt) * nk + kt] = 1;
-      int j0 = kt * BN, j1 = j0 + BN < L ? j0 + BN : L;
-      if (tile_full(r0, r1, j0, j1, Lh, K1, K2e))
-        for (int i = r0; i < r1; ++i)
-          for (int j = j0; j < j1; ++j)
+      int j0 = kt * BN;
+      // full means: the whole unclipped tile is inside the sequence and visible
+      if (tile_full(r0, r0 + BM, j0, j0 + BN, Lh, K1, K2e))
+        for (int i = r0; i < r0 + BM; ++i)
+          for (int j = j0; j < j0 + BN; ++j)
             if (!vis(i, j, L, Lh, K1, K2e)) { printf("tile_full wrong L=%d nt=%d K1=%d K2e=%d r0=%d j0=%d BM=%d BN=%d\n", L, nt, K1, K2e, r0, j0, BM, BN); return 1; }
     }
   }
@@ -80,6 +84,7 @@ int main(int argc, char** argv) {
   const int tiles[][2] = {{64, 64}, {128, 128}, {128, 64}, {64, 128}};
   for (int c = 0; c < n; ++c) {
     int L = 1 + rng() % 700;
+    if (rng() % 6 == 0) L = 64 * (1 + rng() % 8) + (rng() % 2 ? 1 : 0);
     int nt = (rng() % 4 == 0) ? 0 : rng() % (L + 1);
     if (rng() % 8 == 0) nt = L;
     int K1 = rng() % 5 == 0 ? 0 : rng() % 400;
