@@ -126,6 +126,29 @@ int hstu_sla_fwd(const hstu_sla_fwd_params* p, void* workspace, size_t workspace
 int hstu_sla_bwd(const hstu_sla_bwd_params* p, void* workspace, size_t workspace_bytes,
                  hstu_stream_t stream);
 
+/* Forward without a caller-provided workspace, for callers that may not
+ * allocate device memory: inference engines and plugin hosts that plan all
+ * device memory before running and forbid allocation inside their launch
+ * path, and latency-critical loops that cannot afford cudaMalloc/cudaFree
+ * (which may synchronise the device).  The pages have no counterpart: this is
+ * an interface convenience, not part of the method.
+ *
+ * Same arguments, outputs and kernels as hstu_sla_fwd; the work lists and
+ * status word go to a 2 MiB array in the library's own device memory, which
+ * every GPU that loads the library keeps until the process exits.  Batches
+ * need ceil(total_tokens / 64) + B <= 131,040 (about 8.3 million tokens);
+ * larger ones return HSTU_SLA_ERR_WORKSPACE without launching anything.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress), so make that first call before any stream capture.
+ *  - Every call on a device reuses the same array: calls that overlap on the
+ *    GPU (other streams, other host threads) race and must be serialised by
+ *    the caller.  Each call rewrites the status and work lists it reads, so
+ *    nothing carries over from the previous call.
+ *  - Device-detected input errors are not reported (hstu_sla_get_error needs
+ *    a workspace pointer); out is then left unwritten.
+ * Allocates nothing: no cudaMalloc, no cudaFree. */
+int hstu_sla_fwd_noalloc(const hstu_sla_fwd_params* p, hstu_stream_t stream);
+
 /* Test hook: the number of visible keys of every token as the forward
  * kernels enumerate them (row_counts, device int64 [T]) and the number of
  * query rows that see every token as a key, as the backward kernels

@@ -24,7 +24,7 @@ import torch
 from . import _abi
 from ._abi import LibraryMissing  # noqa: F401
 
-__all__ = ["hstu_sla_fwd", "hstu_sla_bwd", "hstu_sla_workspace_bytes", "hstu_sla_count_pairs",
+__all__ = ["hstu_sla_fwd", "hstu_sla_fwd_noalloc", "hstu_sla_bwd", "hstu_sla_workspace_bytes", "hstu_sla_count_pairs",
            "hstu_sla_get_error", "hstu_sla_strerror", "SLAError", "SLAAttention",
            "sla_attention"]
 
@@ -117,6 +117,25 @@ def hstu_sla_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, seq_offsets:
     ws = _workspace(_abi.WS_FWD, p.total_tokens, p.B, p.H, p.d, q.device, workspace)
     _check(lib.hstu_sla_fwd(ctypes.byref(p), ws.data_ptr(), ws.numel(), _stream_ptr(stream)),
            "hstu_sla_fwd")
+    return out
+
+
+def hstu_sla_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                         seq_offsets: torch.Tensor, num_targets: Optional[torch.Tensor], *,
+                         contextual_len: int, K1: int, K2: int, alpha: float, N: float,
+                         max_seq_len: Optional[int] = None, out: Optional[torch.Tensor] = None,
+                         stream=None) -> torch.Tensor:
+    """The forward through the C entry point that allocates no workspace (for
+    callers whose runtime forbids device allocation in the launch path).  The
+    library keeps one 2 MiB scratch array per device; overlapping calls race."""
+    lib = _abi.load()
+    p = _fwd_params(q, k, v, seq_offsets, num_targets, contextual_len, K1, K2, alpha, N,
+                    max_seq_len)
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
+    p.out = out.data_ptr()
+    p.out_row_stride = _row_stride(out, "out", p.H, p.d)
+    _check(lib.hstu_sla_fwd_noalloc(ctypes.byref(p), _stream_ptr(stream)), "hstu_sla_fwd_noalloc")
     return out
 
 

@@ -70,6 +70,8 @@ def load():
     lib.hstu_sla_fwd.restype = ctypes.c_int
     lib.hstu_sla_bwd.argtypes = [ctypes.POINTER(BwdParams), vp, sz, vp]
     lib.hstu_sla_bwd.restype = ctypes.c_int
+    lib.hstu_sla_fwd_noalloc.argtypes = [ctypes.POINTER(FwdParams), vp]
+    lib.hstu_sla_fwd_noalloc.restype = ctypes.c_int
     lib.hstu_sla_count_pairs.argtypes = [ctypes.POINTER(FwdParams), vp, vp, vp, sz, vp]
     lib.hstu_sla_count_pairs.restype = ctypes.c_int
     lib.hstu_sla_get_error.argtypes = [vp, vp]
