@@ -24,8 +24,9 @@
 //   warp 0      scheduler + TMA producer (resident tiles once per unit,
 //               streamed tiles through a 4-stage ring)
 //   warp 1      TMEM allocation; one lane issues every UMMA
-//   warps 2..9  pointwise (P, dS into TMEM, aliasing the fp32 scores they
-//               replace) and the epilogue (accumulators -> bf16 -> global)
+//   warps 2..17 pointwise (P, dS into TMEM, aliasing the fp32 scores they
+//               replace) and the epilogue (accumulators -> bf16 -> global);
+//               four warps per 32-lane TMEM quarter hide TMEM latency
 // TMEM columns: X1 (scores) [0,64) [64,128), X2 (dP) [128,192) [192,256),
 // ACC1 [256,256+d), ACC2 [384,384+d).
 #include <cudaTypedefs.h>
@@ -42,7 +43,7 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kRes = 128, kStr = 64, kStages = 4, kPwWarps = 8;
+constexpr int kRes = 128, kStr = 64, kStages = 4, kPwWarps = 16;
 constexpr int kThreads = 64 + 32 * kPwWarps;
 constexpr uint32_t kColX1 = 0, kColX2 = 128, kColAcc1 = 256, kColAcc2 = 384, kTmemCols = 512;
 
@@ -127,14 +128,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(B_X_FULL + b), 1);
-      mbar_init(bar(B_OP_FULL + b), 32 * kPwWarps);
+      mbar_init(bar(B_OP_FULL + b), kPwWarps);  // one arrive per pointwise warp
       mbar_init(bar(B_U_FULL + b), 1);
-      mbar_init(bar(B_U_EMPTY + b), 1 + 32 * kPwWarps);
+      mbar_init(bar(B_U_EMPTY + b), 1 + kPwWarps);  // MMA warp + pointwise warps
     }
     mbar_init(bar(B_ACC_FULL), 1);
-    mbar_init(bar(B_ACC_EMPTY), 32 * kPwWarps);
+    mbar_init(bar(B_ACC_EMPTY), kPwWarps);
     mbar_init(bar(B_DRAIN), 1);
-    mbar_init(bar(B_PW_SYNC), 32 * kPwWarps);
+    mbar_init(bar(B_PW_SYNC), kPwWarps);
     fence_barrier_init();
     prefetch_tmap(&tma1);
     prefetch_tmap(&tma2);
@@ -152,33 +153,41 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------- scheduler + producer
-    if (lane == 0) {
-      uint32_t k = 0, an = 0, bn = 0;
-      bool ok = true;
-      for (;;) {
-        const uint32_t slot = k & 1;
-        ok = mbar_wait(bar(B_U_EMPTY + slot), ((k >> 1) & 1) ^ 1, a.ws);
-        if (!ok) break;
-        int u = atomicAdd(sched, 1);
+    // The whole warp walks the schedule (warp-uniform values); lane 0 takes
+    // units from the counter, arms barriers and issues the copies.
+    uint32_t k = 0, an = 0, bn = 0;
+    bool ok = true;
+    for (;;) {
+      const uint32_t slot = k & 1;
+      ok = warp_wait(bar(B_U_EMPTY + slot), ((k >> 1) & 1) ^ 1, a.ws);
+      if (!ok) break;
+      int u = 0;
+      if (lane == 0) {
+        u = atomicAdd(sched, 1);
         if (u >= total) u = -1;
         s_unit[slot] = u;
         mbar_arrive(bar(B_U_FULL + slot));
-        ++k;
-        if (u < 0) break;
-        const BUnit w = bunit_at<KV>(a, items, u);
-        if (w.nsteps == 0) continue;
-        ok = mbar_wait(bar(B_A_EMPTY), (an & 1) ^ 1, a.ws);
-        if (!ok) break;
+      }
+      u = __shfl_sync(0xffffffffu, u, 0);
+      ++k;
+      if (u < 0) break;
+      const BUnit w = bunit_at<KV>(a, items, u);
+      if (w.nsteps == 0) continue;
+      ok = warp_wait(bar(B_A_EMPTY), (an & 1) ^ 1, a.ws);
+      if (!ok) break;
+      if (lane == 0) {
         mbar_expect_tx(bar(B_A_FULL), 2 * C::RTILE);
         for (int b = 0; b < C::NB; ++b) {
           tma_load_2d(sA1 + b * C::RBLK, &tma1, bar(B_A_FULL), w.h * D + b * C::BOXW, w.s0 + w.t0);
           tma_load_2d(sA2 + b * C::RBLK, &tma2, bar(B_A_FULL), w.h * D + b * C::BOXW, w.s0 + w.t0);
         }
-        ++an;
-        for (int n = 0; n < w.nsteps; ++n) {
-          const int s = bn % kStages;
-          ok = mbar_wait(bar(B_B_EMPTY + s), ((bn / kStages) & 1) ^ 1, a.ws);
-          if (!ok) break;
+      }
+      ++an;
+      for (int n = 0; n < w.nsteps; ++n) {
+        const int s = bn % kStages;
+        ok = warp_wait(bar(B_B_EMPTY + s), ((bn / kStages) & 1) ^ 1, a.ws);
+        if (!ok) break;
+        if (lane == 0) {
           mbar_expect_tx(bar(B_B_FULL + s), 2 * C::STILE);
           const int y = w.s0 + w.sp.at(n) * kStr;
           for (int b = 0; b < C::NB; ++b) {
@@ -187,104 +196,122 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_2d(sB2 + s * C::STILE + b * C::SBLK, &tmb2, bar(B_B_FULL + s),
                         w.h * D + b * C::BOXW, y);
           }
-          ++bn;
         }
-        if (!ok) break;
+        ++bn;
       }
-      if (load_status(a.ws) != 0) {  // drain copies in flight before exiting
-        if (an > 0) drain_wait(bar(B_A_FULL), (an - 1) & 1);
-        for (int s = 0; s < kStages; ++s) {
-          const uint32_t armed = bn / kStages + (s < (int)(bn % kStages) ? 1u : 0u);
-          if (armed > 0) drain_wait(bar(B_B_FULL + s), (armed - 1) & 1);
-        }
+      if (!ok) break;
+    }
+    if (lane == 0 && load_status(a.ws) != 0) {  // drain copies in flight before exiting
+      if (an > 0) drain_wait(bar(B_A_FULL), (an - 1) & 1);
+      for (int s = 0; s < kStages; ++s) {
+        const uint32_t armed = bn / kStages + (s < (int)(bn % kStages) ? 1u : 0u);
+        if (armed > 0) drain_wait(bar(B_B_FULL + s), (armed - 1) & 1);
       }
     }
   } else if (warp == 1) {
     // --------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      uint32_t k = 0, an = 0, bn = 0, xc = 0, accn = 0;
-      bool ok = true;
-      auto kdesc = [&](uint32_t tile, int blk, int ks) {  // K-major operand, k-step ks
-        const int byte = ks * 32;
-        return smem_desc(tile + (byte / C::SW) * blk + (byte % C::SW), 16, C::SBO, C::SWZ);
-      };
-      auto mndesc = [&](uint32_t tile, int ks) {  // streamed tile as MN-major B, 16 rows a step
-        return smem_desc(tile + ks * 16 * C::SW, C::SBLK, C::SBO, C::SWZ);
-      };
-      auto acc = [&](uint32_t bm, uint32_t xm, bool first) -> bool {
-        const uint32_t b = xm & 1;
-        if (!mbar_wait(bar(B_OP_FULL + b), (xm >> 1) & 1, a.ws)) return false;
-        if (first && !mbar_wait(bar(B_ACC_EMPTY), (accn & 1) ^ 1, a.ws)) return false;
-        tc_fence_after();
-        const int s = bm % kStages;
-        const uint32_t b1 = sB1 + s * C::STILE, b2 = sB2 + s * C::STILE;
+    // Whole warp, warp-uniform descriptors; lane 0 issues every UMMA / commit.
+    uint32_t k = 0, an = 0, bn = 0, xc = 0, accn = 0;
+    bool ok = true;
+    // Descriptor bases; offsets only add to the start-address field.
+    const uint64_t dA1 = smem_desc(sA1, 16, C::SBO, C::SWZ);
+    const uint64_t dA2 = smem_desc(sA2, 16, C::SBO, C::SWZ);
+    const uint64_t dB1 = smem_desc(sB1, 16, C::SBO, C::SWZ);
+    const uint64_t dB2 = smem_desc(sB2, 16, C::SBO, C::SWZ);
+    const uint64_t mB1 = smem_desc(sB1, C::SBLK, C::SBO, C::SWZ);  // MN-major views
+    const uint64_t mB2 = smem_desc(sB2, C::SBLK, C::SBO, C::SWZ);
+    auto koff = [](int ks, int blk) -> uint32_t {  // k-step ks of a K-major tile, 16-byte units
+      return (uint32_t)((((ks * 32) / C::SW) * blk + (ks * 32) % C::SW) >> 4);
+    };
+    auto acc = [&](uint32_t bm, uint32_t xm, bool first) -> bool {
+      const uint32_t b = xm & 1;
+      if (!warp_wait(bar(B_OP_FULL + b), (xm >> 1) & 1, a.ws)) return false;
+      if (first && !warp_wait(bar(B_ACC_EMPTY), (accn & 1) ^ 1, a.ws)) return false;
+      tc_fence_after();
+      const int s = bm % kStages;
+      if (lane == 0) {
+        const uint32_t so = (uint32_t)(s * C::STILE) >> 4;
 #pragma unroll
         for (int ks = 0; ks < kStr / 16; ++ks) {
           const uint32_t accum = (!first || ks > 0) ? 1u : 0u;
+          const uint32_t ko = so + ((uint32_t)(ks * 16 * C::SW) >> 4);
           if (KV) {
-            mma_ts(tmem + kColAcc1, tmem + kColX1 + b * 64 + ks * 8, mndesc(b2, ks), C::IDESC_ACC,
+            mma_ts(tmem + kColAcc1, tmem + kColX1 + b * 64 + ks * 8, mB2 + ko, C::IDESC_ACC,
                    accum);  // dV += P^T dO
-            mma_ts(tmem + kColAcc2, tmem + kColX2 + b * 64 + ks * 8, mndesc(b1, ks), C::IDESC_ACC,
+            mma_ts(tmem + kColAcc2, tmem + kColX2 + b * 64 + ks * 8, mB1 + ko, C::IDESC_ACC,
                    accum);  // dK += dS^T Q
           } else {
-            mma_ts(tmem + kColAcc1, tmem + kColX2 + b * 64 + ks * 8, mndesc(b1, ks), C::IDESC_ACC,
+            mma_ts(tmem + kColAcc1, tmem + kColX2 + b * 64 + ks * 8, mB1 + ko, C::IDESC_ACC,
                    accum);  // dQ += dS K
           }
         }
         tc_commit(bar(B_B_EMPTY + s));
-        return true;
-      };
-      for (;;) {
-        const uint32_t slot = k & 1;
-        ok = mbar_wait(bar(B_U_FULL + slot), (k >> 1) & 1, a.ws);
-        if (!ok) break;
-        const int u = s_unit[slot];
-        mbar_arrive(bar(B_U_EMPTY + slot));
-        ++k;
-        if (u < 0) break;
-        const BUnit w = bunit_at<KV>(a, items, u);
-        if (w.nsteps == 0) continue;
-        ok = mbar_wait(bar(B_A_FULL), an & 1, a.ws);
+      }
+      __syncwarp();
+      return true;
+    };
+    for (;;) {
+      const uint32_t slot = k & 1;
+      ok = warp_wait(bar(B_U_FULL + slot), (k >> 1) & 1, a.ws);
+      if (!ok) break;
+      const int u = s_unit[slot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_U_EMPTY + slot));
+      ++k;
+      if (u < 0) break;
+      const BUnit w = bunit_at<KV>(a, items, u);
+      if (w.nsteps == 0) continue;
+      ok = warp_wait(bar(B_A_FULL), an & 1, a.ws);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t bn0 = bn, xc0 = xc;
+      for (int n = 0; n < w.nsteps; ++n) {
+        const int s = bn % kStages;
+        ok = warp_wait(bar(B_B_FULL + s), (bn / kStages) & 1, a.ws);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t bn0 = bn, xc0 = xc;
-        for (int n = 0; n < w.nsteps; ++n) {
-          const int s = bn % kStages;
-          ok = mbar_wait(bar(B_B_FULL + s), (bn / kStages) & 1, a.ws);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t b = xc & 1;
+        const uint32_t b = xc & 1;
+        if (lane == 0) {
+          const uint32_t so = (uint32_t)(s * C::STILE) >> 4;
 #pragma unroll
           for (int ks = 0; ks < D / 16; ++ks) {
-            mma_ss(tmem + kColX1 + b * 64, kdesc(sA1, C::RBLK, ks),
-                   kdesc(sB1 + s * C::STILE, C::SBLK, ks), C::IDESC_X, ks > 0 ? 1u : 0u);
-            mma_ss(tmem + kColX2 + b * 64, kdesc(sA2, C::RBLK, ks),
-                   kdesc(sB2 + s * C::STILE, C::SBLK, ks), C::IDESC_X, ks > 0 ? 1u : 0u);
+            mma_ss(tmem + kColX1 + b * 64, dA1 + koff(ks, C::RBLK), dB1 + so + koff(ks, C::SBLK),
+                   C::IDESC_X, ks > 0 ? 1u : 0u);
+            mma_ss(tmem + kColX2 + b * 64, dA2 + koff(ks, C::RBLK), dB2 + so + koff(ks, C::SBLK),
+                   C::IDESC_X, ks > 0 ? 1u : 0u);
           }
           tc_commit(bar(B_X_FULL + b));
-          if (n > 0) {
-            ok = acc(bn - 1, xc - 1, n == 1);
-            if (!ok) break;
-          }
-          ++bn;
-          ++xc;
+          if (n + 1 == w.nsteps) tc_commit(bar(B_A_EMPTY));  // last use of the resident tiles
         }
-        if (!ok) break;
-        ok = acc(bn0 + w.nsteps - 1, xc0 + w.nsteps - 1, w.nsteps == 1);
-        if (!ok) break;
-        tc_commit(bar(B_A_EMPTY));
-        tc_commit(bar(B_ACC_FULL));
-        ++an;
-        ++accn;
+        __syncwarp();
+        if (n > 0) {
+          ok = acc(bn - 1, xc - 1, n == 1);
+          if (!ok) break;
+        }
+        ++bn;
+        ++xc;
       }
+      if (!ok) break;
+      ok = acc(bn0 + w.nsteps - 1, xc0 + w.nsteps - 1, w.nsteps == 1);
+      if (!ok) break;
+      if (lane == 0) tc_commit(bar(B_ACC_FULL));
+      __syncwarp();
+      ++an;
+      ++accn;
+    }
+    if (lane == 0) {
       tc_commit(bar(B_DRAIN));
       drain_wait(bar(B_DRAIN), 0);
     }
+    __syncwarp();
   } else {
     // ------------------------------------------------ pointwise + epilogue
+    // Four warps share each 32-lane TMEM quarter; warp `chunk` of a quarter
+    // owns streamed columns [16 chunk, +16) of every step and accumulator
+    // columns [32 chunk, +32) in the epilogue.
     const int pw = warp - 2;
     const int quarter = warp & 3;
-    const int half = pw >> 2;
+    const int chunk = pw >> 2;            // 0..3
     const int row = quarter * 32 + lane;  // resident row of this thread
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     const float half_alpha = 0.5f * a.alpha;
@@ -292,29 +319,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float sc2 = a.alpha * a.inv_n;                 // ACC2: dK
     bf16* out1 = KV ? a.dv : a.dq;
     const int64_t rs1 = KV ? a.dv_rs : a.dq_rs;
+    const int col = chunk * 16;
+    const bool has_acc = chunk < D / 32;
     uint32_t k = 0, xc = 0, accn = 0;
     bool ok = true;
     for (;;) {
       const uint32_t slot = k & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_U_FULL + slot), (k >> 1) & 1, a.ws));
+      ok = warp_wait(bar(B_U_FULL + slot), (k >> 1) & 1, a.ws);
       if (!ok) break;
       const int u = s_unit[slot];
-      mbar_arrive(bar(B_U_EMPTY + slot));
+      warp_arrive(bar(B_U_EMPTY + slot));
       ++k;
       if (u < 0) break;
       const BUnit w = bunit_at<KV>(a, items, u);
       const int r = w.t0 + row;  // this thread's resident position in the sequence
-      bf16* o1 = out1 + (int64_t)(w.s0 + r) * rs1 + w.h * D;
-      bf16* o2 = a.dk + (int64_t)(w.s0 + r) * a.dk_rs + w.h * D;
+      bf16* o1 = out1 + (int64_t)(w.s0 + r) * rs1 + w.h * D + chunk * 32;
+      bf16* o2 = a.dk + (int64_t)(w.s0 + r) * a.dk_rs + w.h * D + chunk * 32;
       if (w.nsteps == 0) {
-        if (r < w.t1) {
+        if (has_acc && r < w.t1) {
           const uint4 z = make_uint4(0, 0, 0, 0);
-          for (int c = half; c < D / 32; c += 2)
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              reinterpret_cast<uint4*>(o1 + c * 32)[v] = z;
-              if (KV) reinterpret_cast<uint4*>(o2 + c * 32)[v] = z;
-            }
+          for (int v = 0; v < 4; ++v) {
+            reinterpret_cast<uint4*>(o1)[v] = z;
+            if (KV) reinterpret_cast<uint4*>(o2)[v] = z;
+          }
         }
         continue;
       }
@@ -322,69 +350,67 @@ __global__ void __launch_bounds__(kThreads, 1)
       const RowMask rm = row_mask(r, w.L, w.Lh, a.K1, a.K2e);
       for (int n = 0; n < w.nsteps; ++n) {
         const uint32_t b = xc & 1;
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(B_X_FULL + b), (xc >> 1) & 1, a.ws));
+        ok = warp_wait(bar(B_X_FULL + b), (xc >> 1) & 1, a.ws);
         if (!ok) break;
         tc_fence_after();
         const int c0 = w.sp.at(n) * kStr;  // first streamed position of this step
         const bool full = KV ? tile_full(c0, c0 + kStr, w.t0, w.t0 + kRes, w.Lh, a.K1, a.K2e)
                              : tile_full(w.t0, w.t0 + kRes, c0, c0 + kStr, w.Lh, a.K1, a.K2e);
-        const int col = half * 32;
-        uint32_t xs[32], xd[32];
-        tmem_ld32(lane_base + kColX1 + b * 64 + col, xs);
-        tmem_ld32(lane_base + kColX2 + b * 64 + col, xd);
-        tmem_ld_wait(xs);
-        tmem_ld_wait(xd);
+        uint32_t xs[16], xd[16];
+        tmem_ld16(lane_base + kColX1 + b * 64 + col, xs);
+        tmem_ld16(lane_base + kColX2 + b * 64 + col, xd);
+        tmem_ld_wait2(xs, xd);
         // every score is in registers before P / dS overwrite them (a bounded
         // group barrier over the pointwise warps, one phase per step)
-        mbar_arrive(bar(B_PW_SYNC));
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(B_PW_SYNC), xc & 1, a.ws));
+        warp_arrive(bar(B_PW_SYNC));
+        ok = warp_wait(bar(B_PW_SYNC), xc & 1, a.ws);
         if (!ok) break;
-        uint32_t pp[16], dd[16];
+        // P = SiLU(x) and dS = dP SiLU'(x) for x = alpha S, with h = x/2 and
+        // t = tanh(h): SiLU = h + h t, SiLU' = (1 + t)/2 (1 + h - h t).
+        // Fully visible tiles skip the mask; others clear invisible entries
+        // by one bit test against this thread's 32-position visibility mask.
+        uint32_t pp[8], dd[8];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          float pv[2], dv[2];
+        for (int e = 0; e < 8; ++e)
+          bwd_pair(xs[2 * e], xs[2 * e + 1], xd[2 * e], xd[2 * e + 1], half_alpha, pp[e], dd[e]);
+        if (!full) {
+          const uint32_t bits =
+              KV ? key_mask_bits(km, c0 + col) : row_mask_bits(rm, c0 + col);
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            const float hx = __uint_as_float(xs[2 * e + q]) * half_alpha;
-            const float t = tanh_approx(hx);
-            const float silu = fmaf(hx, t, hx);
-            const float dsilu = fmaf(0.5f, t, 0.5f) * (1.f + fmaf(-hx, t, hx));
-            const float dsv = __uint_as_float(xd[2 * e + q]) * dsilu;
-            bool vis = true;
-            if (!full) {
-              const int c = c0 + col + 2 * e + q;
-              vis = KV ? km(c) : rm(c);
-            }
-            pv[q] = vis ? silu : 0.f;
-            dv[q] = vis ? dsv : 0.f;
+          for (int e = 0; e < 8; ++e) {
+            pp[e] = mask_pair(pp[e], bits, e);
+            dd[e] = mask_pair(dd[e], bits, e);
           }
-          pp[e] = pack_bf16x2(pv[0], pv[1]);
-          dd[e] = pack_bf16x2(dv[0], dv[1]);
         }
-        if (KV) tmem_st16(lane_base + kColX1 + b * 64 + half * 16, pp);
-        tmem_st16(lane_base + kColX2 + b * 64 + half * 16, dd);
+        if (KV) tmem_st8(lane_base + kColX1 + b * 64 + col / 2, pp);
+        tmem_st8(lane_base + kColX2 + b * 64 + col / 2, dd);
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(bar(B_OP_FULL + b));
+        warp_arrive(bar(B_OP_FULL + b));
         ++xc;
       }
       if (!ok) break;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_ACC_FULL), accn & 1, a.ws));
+      ok = warp_wait(bar(B_ACC_FULL), accn & 1, a.ws);
       if (!ok) break;
       tc_fence_after();
-      for (int c = half; c < D / 32; c += 2) {
+      if (has_acc) {
 #pragma unroll
         for (int which = 0; which < (KV ? 2 : 1); ++which) {
-          uint32_t v[32];
-          tmem_ld32(lane_base + (which ? kColAcc2 : kColAcc1) + c * 32, v);
-          tmem_ld_wait(v);
+          uint32_t v0[16], v1[16];
+          const uint32_t cbase = lane_base + (which ? kColAcc2 : kColAcc1) + chunk * 32;
+          tmem_ld16(cbase, v0);
+          tmem_ld16(cbase + 16, v1);
+          tmem_ld_wait2(v0, v1);
           if (r < w.t1) {
             const float sc = which ? sc2 : sc1;
             uint32_t o[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-              o[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * sc, __uint_as_float(v[2 * e + 1]) * sc);
-            uint4* dst = reinterpret_cast<uint4*>((which ? o2 : o1) + c * 32);
+            for (int e = 0; e < 8; ++e) {
+              o[e] = pack_bf16x2(__uint_as_float(v0[2 * e]) * sc, __uint_as_float(v0[2 * e + 1]) * sc);
+              o[8 + e] =
+                  pack_bf16x2(__uint_as_float(v1[2 * e]) * sc, __uint_as_float(v1[2 * e + 1]) * sc);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(which ? o2 : o1);
 #pragma unroll
             for (int q = 0; q < 4; ++q)
               dst[q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
@@ -392,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(bar(B_ACC_EMPTY));
+      warp_arrive(bar(B_ACC_EMPTY));
       ++accn;
     }
   }

@@ -131,6 +131,30 @@ __host__ __device__ __forceinline__ RowMask row_mask(int i, int L, int Lh, int K
   return m;
 }
 
+// Bit e set iff position base + e lies in [lo, hi), for e in [0, 32).
+__host__ __device__ __forceinline__ uint32_t range_bits(int lo, int hi, int base) {
+  const int a = lo - base < 0 ? 0 : lo - base;
+  const int b = hi - base > 32 ? 32 : hi - base;
+  if (a >= b) return 0u;
+  const uint32_t upto_b = b >= 32 ? 0xFFFFFFFFu : ((1u << b) - 1u);
+  return upto_b & ~((1u << a) - 1u);
+}
+
+// Visibility of keys [base, base + 32) for one row / of rows [base, base + 32)
+// for one key, one bit each: the interval forms above turned into a bitmask,
+// so the per-element test in inner loops is a single bit test.
+__host__ __device__ __forceinline__ uint32_t row_mask_bits(const RowMask& m, int base) {
+  uint32_t bits = range_bits(0, m.pre, base) | range_bits(m.lo, m.hi, base);
+  if (m.self >= base && m.self < base + 32) bits |= 1u << (m.self - base);
+  return bits;
+}
+
+// Zero the bf16 halves of a packed pair whose bits (2e, 2e+1) of `bits` are clear.
+__host__ __device__ __forceinline__ uint32_t mask_pair(uint32_t p2, uint32_t bits, int e) {
+  const uint32_t lo = (bits >> (2 * e)) & 1u, hi = (bits >> (2 * e + 1)) & 1u;
+  return p2 & ((0u - lo) & 0x0000FFFFu | (0u - hi) & 0xFFFF0000u);
+}
+
 // Up to three disjoint, increasing tile-index intervals [lo, hi).
 struct Spans {
   int lo[3], hi[3], n;
@@ -252,6 +276,12 @@ __host__ __device__ __forceinline__ KeyMask key_mask(int j, int L, int Lh, int K
     }
   }
   return m;
+}
+
+__host__ __device__ __forceinline__ uint32_t key_mask_bits(const KeyMask& m, int base) {
+  uint32_t bits = range_bits(m.lo, m.hi, base) | range_bits(m.tlo, m.thi, base);
+  if (m.self >= base && m.self < base + 32) bits |= 1u << (m.self - base);
+  return bits;
 }
 
 __device__ __forceinline__ void set_status(WsHeader* ws, int code) {

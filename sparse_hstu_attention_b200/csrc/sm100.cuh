@@ -71,6 +71,18 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, WsHeade
   }
 }
 
+// Arrive once for the whole warp (barriers counting warps): every lane's
+// prior work is ordered before lane 0's arrive by the warp synchronisation.
+__device__ __forceinline__ void warp_arrive(uint32_t bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
+// mbar_wait by every lane of a warp, with a warp-uniform result.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, WsHeader* ws) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, ws));
+}
+
 // Bounded wait that ignores the error status: used only to drain copies
 // already in flight before a CTA that gave up exits.
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
@@ -166,6 +178,43 @@ __device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[32]) {
                :
                : "memory");
 }
+// 32 lanes x 16 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                 "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                 "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+               :
+               : "memory");
+}
+// One wait for two outstanding loads of 16 columns.
+__device__ __forceinline__ void tmem_ld_wait2(uint32_t (&r)[16], uint32_t (&s)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                 "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                 "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(s[0]), "+r"(s[1]),
+                 "+r"(s[2]), "+r"(s[3]), "+r"(s[4]), "+r"(s[5]), "+r"(s[6]), "+r"(s[7]),
+                 "+r"(s[8]), "+r"(s[9]), "+r"(s[10]), "+r"(s[11]), "+r"(s[12]), "+r"(s[13]),
+                 "+r"(s[14]), "+r"(s[15])
+               :
+               : "memory");
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(
+                   taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+               "r"(r[7])
+               : "memory");
+}
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
@@ -203,10 +252,40 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// SiLU on a bf16 pair given h = x/2:  SiLU(x) = h + h tanh(h), evaluated with
+// the packed bf16 MUFU tanh and one packed bf16 FMA (the result is a bf16
+// operand for the next MMA either way).
+__device__ __forceinline__ uint32_t silu_half_bf16x2(uint32_t h2) {
+  uint32_t t2, p2;
+  asm("tanh.approx.bf16x2 %0, %1;" : "=r"(t2) : "r"(h2));
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(p2) : "r"(h2), "r"(t2), "r"(h2));
+  return p2;
+}
+
 __device__ __forceinline__ float tanh_approx(float x) {
   float y;
   asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Backward pointwise for two scores s (raw fp32 bits) and their dP: packed
+// bf16 P = SiLU(alpha s) and dS = dP SiLU'(alpha s), with h = alpha s / 2,
+// t = tanh(h): SiLU = h + h t and SiLU' = (1 + t)/2 (1 + h - h t).
+__device__ __forceinline__ void bwd_pair(uint32_t s0, uint32_t s1, uint32_t d0, uint32_t d1,
+                                         float half_alpha, uint32_t& p2, uint32_t& ds2) {
+  const float h0 = __uint_as_float(s0) * half_alpha, h1 = __uint_as_float(s1) * half_alpha;
+  const float t0 = tanh_approx(h0), t1 = tanh_approx(h1);
+  const float g0 = fmaf(0.5f, t0, 0.5f) * (1.f + fmaf(-h0, t0, h0));
+  const float g1 = fmaf(0.5f, t1, 0.5f) * (1.f + fmaf(-h1, t1, h1));
+  p2 = pack_bf16x2(fmaf(h0, t0, h0), fmaf(h1, t1, h1));
+  ds2 = pack_bf16x2(__uint_as_float(d0) * g0, __uint_as_float(d1) * g1);
+}
+
+// SiLU of two fp32 scores (raw bits) packed as bf16x2, with h = alpha s / 2:
+// SiLU(alpha s) = h + h tanh(h).
+__device__ __forceinline__ uint32_t silu_pair(uint32_t s0, uint32_t s1, float half_alpha) {
+  const float h0 = __uint_as_float(s0) * half_alpha, h1 = __uint_as_float(s1) * half_alpha;
+  return pack_bf16x2(fmaf(h0, tanh_approx(h0), h0), fmaf(h1, tanh_approx(h1), h1));
 }
 
 }  // namespace sm100

@@ -7,8 +7,8 @@
 //   - no enumerated (query tile, key tile) pair is empty, from either side;
 //   - tile_full() on an unclipped tile is only true when every pair of the
 //     tile lies inside the sequence and is visible;
-//   - the per-row and per-key interval forms row_mask() / key_mask() equal the
-//     predicate.
+//   - the per-row and per-key interval forms row_mask() / key_mask() and
+//     their 32-bit bitmask forms equal the predicate.
 // Prints "OK <cases>" or the first failure.
 #include <cstdio>
 #include <cstdlib>
@@ -30,6 +30,14 @@ static int check(int L, int nt, int K1, int K2e, int BM, int BN) {
   std::vector<char> qk(size_t(nq) * nk, 0), fwd(size_t(nq) * nk, 0), bwd(size_t(nq) * nk, 0);
   for (int i = 0; i < L; ++i) {
     RowMask m = row_mask(i, L, Lh, K1, K2e);
+    for (int base = 0; base < L + 32; base += 16) {
+      const uint32_t rb = row_mask_bits(m, base);
+      const uint32_t kb = key_mask_bits(key_mask(i, L, Lh, K1, K2e), base);
+      for (int e = 0; e < 32; ++e) {
+        if (((rb >> e) & 1u) != (uint32_t)vis(i, base + e, L, Lh, K1, K2e)) { printf("row_mask_bits mismatch L=%d i=%d base=%d e=%d\n", L, i, base, e); return 1; }
+        if (((kb >> e) & 1u) != (uint32_t)vis(base + e, i, L, Lh, K1, K2e)) { printf("key_mask_bits mismatch L=%d j=%d base=%d e=%d\n", L, i, base, e); return 1; }
+      }
+    }
     for (int j = 0; j < L; ++j) {
       bool v = vis(i, j, L, Lh, K1, K2e);
       if (v != key_mask(j, L, Lh, K1, K2e)(i)) { printf("key_mask mismatch L=%d nt=%d K1=%d K2e=%d i=%d j=%d\n", L, nt, K1, K2e, i, j); return 1; }
