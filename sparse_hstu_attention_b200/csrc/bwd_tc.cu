@@ -71,7 +71,8 @@ struct BCfg {
 enum {
   B_A_FULL = 0, B_A_EMPTY, B_B_FULL, B_B_EMPTY = B_B_FULL + kStages,
   B_X_FULL = B_B_EMPTY + kStages, B_OP_FULL = B_X_FULL + 2, B_ACC_FULL = B_OP_FULL + 2,
-  B_ACC_EMPTY, B_U_FULL, B_U_EMPTY = B_U_FULL + 2, B_DRAIN = B_U_EMPTY + 2, B_PW_SYNC, B_COUNT
+  B_ACC_EMPTY, B_U_FULL, B_U_EMPTY = B_U_FULL + 2, B_DRAIN = B_U_EMPTY + 2, B_PW_SYNC,
+  B_COUNT = B_PW_SYNC + 2
 };
 
 struct BUnit {
@@ -128,14 +129,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(B_X_FULL + b), 1);
-      mbar_init(bar(B_OP_FULL + b), kPwWarps);  // one arrive per pointwise warp
+      mbar_init(bar(B_OP_FULL + b), kPwWarps / 2);  // one arrive per warp of group b
+      mbar_init(bar(B_PW_SYNC + b), kPwWarps / 2);
       mbar_init(bar(B_U_FULL + b), 1);
       mbar_init(bar(B_U_EMPTY + b), 1 + kPwWarps);  // MMA warp + pointwise warps
     }
     mbar_init(bar(B_ACC_FULL), 1);
     mbar_init(bar(B_ACC_EMPTY), kPwWarps);
     mbar_init(bar(B_DRAIN), 1);
-    mbar_init(bar(B_PW_SYNC), kPwWarps);
     fence_barrier_init();
     prefetch_tmap(&tma1);
     prefetch_tmap(&tma2);
@@ -306,12 +307,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------ pointwise + epilogue
-    // Four warps share each 32-lane TMEM quarter; warp `chunk` of a quarter
-    // owns streamed columns [16 chunk, +16) of every step and accumulator
-    // columns [32 chunk, +32) in the epilogue.
+    // Two groups of eight warps take alternate steps (group g owns X buffer
+    // g), so one group's TMEM latency overlaps the other's arithmetic; the two
+    // warps of a group on one 32-lane TMEM quarter split the step's 64
+    // streamed columns in halves.  The epilogue uses all sixteen warps: warp
+    // `chunk` of a quarter writes accumulator columns [32 chunk, +32).
     const int pw = warp - 2;
+    const int grp = pw >> 3;              // X buffer / step parity of this warp
     const int quarter = warp & 3;
     const int chunk = pw >> 2;            // 0..3
+    const int half = chunk & 1;           // streamed-column half within the group
     const int row = quarter * 32 + lane;  // resident row of this thread
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     const float half_alpha = 0.5f * a.alpha;
@@ -319,7 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float sc2 = a.alpha * a.inv_n;                 // ACC2: dK
     bf16* out1 = KV ? a.dv : a.dq;
     const int64_t rs1 = KV ? a.dv_rs : a.dq_rs;
-    const int col = chunk * 16;
+    const int col = half * 32;
     const bool has_acc = chunk < D / 32;
     uint32_t k = 0, xc = 0, accn = 0;
     bool ok = true;
@@ -348,46 +353,52 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const KeyMask km = key_mask(r, w.L, w.Lh, a.K1, a.K2e);
       const RowMask rm = row_mask(r, w.L, w.Lh, a.K1, a.K2e);
-      for (int n = 0; n < w.nsteps; ++n) {
+      for (int n = 0; n < w.nsteps; ++n, ++xc) {
         const uint32_t b = xc & 1;
+        if ((int)b != grp) continue;  // the other group's step
         ok = warp_wait(bar(B_X_FULL + b), (xc >> 1) & 1, a.ws);
         if (!ok) break;
         tc_fence_after();
         const int c0 = w.sp.at(n) * kStr;  // first streamed position of this step
         const bool full = KV ? tile_full(c0, c0 + kStr, w.t0, w.t0 + kRes, w.Lh, a.K1, a.K2e)
                              : tile_full(w.t0, w.t0 + kRes, c0, c0 + kStr, w.Lh, a.K1, a.K2e);
-        uint32_t xs[16], xd[16];
-        tmem_ld16(lane_base + kColX1 + b * 64 + col, xs);
-        tmem_ld16(lane_base + kColX2 + b * 64 + col, xd);
-        tmem_ld_wait2(xs, xd);
-        // every score is in registers before P / dS overwrite them (a bounded
-        // group barrier over the pointwise warps, one phase per step)
-        warp_arrive(bar(B_PW_SYNC));
-        ok = warp_wait(bar(B_PW_SYNC), xc & 1, a.ws);
+        uint32_t xs0[16], xs1[16], xd0[16], xd1[16];
+        tmem_ld16(lane_base + kColX1 + b * 64 + col, xs0);
+        tmem_ld16(lane_base + kColX1 + b * 64 + col + 16, xs1);
+        tmem_ld16(lane_base + kColX2 + b * 64 + col, xd0);
+        tmem_ld16(lane_base + kColX2 + b * 64 + col + 16, xd1);
+        tmem_ld_wait2(xs0, xs1);
+        tmem_ld_wait2(xd0, xd1);
+        // every score of the group is in registers before P / dS overwrite
+        // them (a bounded barrier over the group's warps, one phase per step)
+        warp_arrive(bar(B_PW_SYNC + b));
+        ok = warp_wait(bar(B_PW_SYNC + b), (xc >> 1) & 1, a.ws);
         if (!ok) break;
         // P = SiLU(x) and dS = dP SiLU'(x) for x = alpha S, with h = x/2 and
         // t = tanh(h): SiLU = h + h t, SiLU' = (1 + t)/2 (1 + h - h t).
         // Fully visible tiles skip the mask; others clear invisible entries
         // by one bit test against this thread's 32-position visibility mask.
-        uint32_t pp[8], dd[8];
+        const uint32_t bits =
+            full ? 0xFFFFFFFFu : (KV ? key_mask_bits(km, c0 + col) : row_mask_bits(rm, c0 + col));
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-          bwd_pair(xs[2 * e], xs[2 * e + 1], xd[2 * e], xd[2 * e + 1], half_alpha, pp[e], dd[e]);
-        if (!full) {
-          const uint32_t bits =
-              KV ? key_mask_bits(km, c0 + col) : row_mask_bits(rm, c0 + col);
+        for (int sub = 0; sub < 2; ++sub) {
+          const uint32_t* xs = sub ? xs1 : xs0;
+          const uint32_t* xd = sub ? xd1 : xd0;
+          uint32_t pp[8], dd[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            pp[e] = mask_pair(pp[e], bits, e);
-            dd[e] = mask_pair(dd[e], bits, e);
+            bwd_pair(xs[2 * e], xs[2 * e + 1], xd[2 * e], xd[2 * e + 1], half_alpha, pp[e], dd[e]);
+            if (!full) {
+              pp[e] = mask_pair(pp[e], bits, 8 * sub + e);
+              dd[e] = mask_pair(dd[e], bits, 8 * sub + e);
+            }
           }
+          if (KV) tmem_st8(lane_base + kColX1 + b * 64 + col / 2 + 8 * sub, pp);
+          tmem_st8(lane_base + kColX2 + b * 64 + col / 2 + 8 * sub, dd);
         }
-        if (KV) tmem_st8(lane_base + kColX1 + b * 64 + col / 2, pp);
-        tmem_st8(lane_base + kColX2 + b * 64 + col / 2, dd);
         tmem_st_wait();
         tc_fence_before();
         warp_arrive(bar(B_OP_FULL + b));
-        ++xc;
       }
       if (!ok) break;
       ok = warp_wait(bar(B_ACC_FULL), accn & 1, a.ws);

@@ -125,7 +125,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(BAR_S_FULL + b), 1);
-      mbar_init(bar(BAR_P_FULL + b), kPwWarps);  // one arrive per pointwise warp
+      mbar_init(bar(BAR_P_FULL + b), kPwWarps / 2);  // one arrive per warp of group b
     }
     mbar_init(bar(BAR_O_FULL), 1);
     mbar_init(bar(BAR_O_EMPTY), kPwWarps);
@@ -278,15 +278,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ----------------------------------------------- pointwise and epilogue
-    // Four warps share each 32-lane TMEM quarter; warp `chunk` of a quarter
-    // owns S columns [32 chunk, 32 chunk + 32) and O columns [32 chunk, +32).
+    // Two groups of eight warps take alternate S tiles (group g owns S buffer
+    // g), so one group's TMEM load / store latency overlaps the other's
+    // arithmetic.  Within a group, the two warps on a 32-lane TMEM quarter
+    // split the tile's 128 columns in halves.  The epilogue uses all sixteen:
+    // warp `chunk` of a quarter writes O columns [32 chunk, +32).
     const int pw = warp - 2;               // 0..15
+    const int grp = pw >> 3;               // S buffer / tile parity of this warp
     const int quarter = warp & 3;          // TMEM lanes [32*quarter, +32)
     const int chunk = pw >> 2;             // 0..3
+    const int half = chunk & 1;            // column half within the group
     const int row = quarter * 32 + lane;   // row of the 128-row tile
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     const float half_alpha = 0.5f * a.alpha;
-    const int col = chunk * C::COLS_PER_PW;
     const bool has_o = chunk < D / 32;     // this warp writes an O chunk
     uint32_t tc = 0, on = 0;
     bool ok = true;
@@ -303,39 +307,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         continue;
       }
       const RowMask m = row_mask(i, w.L, w.Lh, a.K1, a.K2e);
-      for (int n = 0; n < w.ntiles; ++n) {
+      for (int n = 0; n < w.ntiles; ++n, ++tc) {
         const uint32_t b = tc & 1;
+        if ((int)b != grp) continue;  // the other group's tile
         ok = warp_wait(bar(BAR_S_FULL + b), (tc >> 1) & 1, a.ws);
         if (!ok) break;
         tc_fence_after();
-        uint32_t c0[16], c1[16];
-        tmem_ld16(lane_base + kColS0 + b * 128 + col, c0);
-        tmem_ld16(lane_base + kColS0 + b * 128 + col + 16, c1);
-        tmem_ld_wait2(c0, c1);
         const int j0 = w.sp.at(n) * kBN;
+        const bool full = tile_full(w.r0, w.r0 + kBM, j0, j0 + kBN, w.Lh, a.K1, a.K2e);
         // P = SiLU(alpha S) = h + h tanh(h) with h = alpha S / 2.  Tiles that
         // are entirely visible skip the mask; the others clear invisible
         // entries with one bit test each against this row's 32-key bitmask.
-        uint32_t p[16];
-        if (tile_full(w.r0, w.r0 + kBM, j0, j0 + kBN, w.Lh, a.K1, a.K2e)) {
+#pragma unroll
+        for (int sub = 0; sub < 2; ++sub) {
+          const int col = half * 64 + sub * 32;
+          uint32_t c0[16], c1[16];
+          tmem_ld16(lane_base + kColS0 + b * 128 + col, c0);
+          tmem_ld16(lane_base + kColS0 + b * 128 + col + 16, c1);
+          tmem_ld_wait2(c0, c1);
+          uint32_t p[16];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             p[e] = silu_pair(c0[2 * e], c0[2 * e + 1], half_alpha);
             p[8 + e] = silu_pair(c1[2 * e], c1[2 * e + 1], half_alpha);
           }
-        } else {
-          const uint32_t bits = row_mask_bits(m, j0 + col);
+          if (!full) {
+            const uint32_t bits = row_mask_bits(m, j0 + col);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            p[e] = mask_pair(silu_pair(c0[2 * e], c0[2 * e + 1], half_alpha), bits, e);
-            p[8 + e] = mask_pair(silu_pair(c1[2 * e], c1[2 * e + 1], half_alpha), bits, 8 + e);
+            for (int e = 0; e < 16; ++e) p[e] = mask_pair(p[e], bits, e);
           }
+          tmem_st16(lane_base + kColP0 + b * 64 + col / 2, p);
         }
-        tmem_st16(lane_base + kColP0 + b * 64 + col / 2, p);
         tmem_st_wait();
         tc_fence_before();
         warp_arrive(bar(BAR_P_FULL + b));
-        ++tc;
       }
       if (!ok) break;
       // epilogue
