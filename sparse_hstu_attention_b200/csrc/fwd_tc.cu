@@ -8,8 +8,9 @@
 // Persistent, warp-specialised: one CTA per SM walks (head, 128-row query
 // tile) work units.  Per unit only the key tiles that the SLA mask leaves
 // non-empty are visited (global prefix, local band, candidates' diagonal).
-//   warp 0      TMA producer: Q tile, then K and V tiles (128 keys) into a
-//               2-stage ring; 128B-swizzled boxes of 64 head-dim columns.
+//   warp 0      TMA producer: Q tiles into two alternating buffers, K and V
+//               tiles (128 keys) into a 2-stage ring; 128B-swizzled boxes
+//               of 64 head-dim columns.
 //   warp 1      allocates TMEM; one lane issues UMMA: S = Q K^T into one of
 //               two TMEM S buffers (M=128, N=128, K=d), then O += P V with P
 //               read from TMEM (M=128, N=d, K=128) into the O accumulator.
@@ -53,10 +54,10 @@ struct Cfg {
   static constexpr int NB = D / BOXW;             // boxes per tile
   static constexpr int BLK = 128 * SW;            // bytes per box (128 rows)
   static constexpr int TILE = 128 * D * 2;        // bytes per Q / K / V tile
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = TILE;
-  static constexpr int OFF_V = TILE * (1 + kStages);
-  static constexpr int OFF_BAR = TILE * (1 + 2 * kStages);
+  static constexpr int OFF_Q = 0;                      // two Q buffers
+  static constexpr int OFF_K = 2 * TILE;
+  static constexpr int OFF_V = TILE * (2 + kStages);
+  static constexpr int OFF_BAR = TILE * (2 + 2 * kStages);
   static_assert(OFF_BAR + 256 + 1024 <= 232448, "shared memory budget");
   static constexpr int SMEM = OFF_BAR + 256 + 1024;  // barriers + 1 KB alignment slack
   static constexpr uint32_t SWZ = SW == 128 ? kSwizzle128B : kSwizzle64B;
@@ -69,7 +70,7 @@ struct Cfg {
 // Barrier slots (8 bytes each) after the tiles.
 constexpr int kMaxStages = 4;
 enum {
-  BAR_Q_FULL = 0, BAR_Q_EMPTY, BAR_K_FULL, BAR_K_EMPTY = BAR_K_FULL + kMaxStages,
+  BAR_Q_FULL = 0, BAR_Q_EMPTY = 2, BAR_K_FULL = 4, BAR_K_EMPTY = BAR_K_FULL + kMaxStages,
   BAR_V_FULL = BAR_K_EMPTY + kMaxStages, BAR_V_EMPTY = BAR_V_FULL + kMaxStages,
   BAR_S_FULL = BAR_V_EMPTY + kMaxStages, BAR_P_FULL = BAR_S_FULL + 2, BAR_O_FULL = BAR_P_FULL + 2,
   BAR_O_EMPTY, BAR_DRAIN, BAR_COUNT
@@ -115,8 +116,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int total = n_items * a.H;
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(BAR_Q_FULL), 1);
-    mbar_init(bar(BAR_Q_EMPTY), 1);
+    for (int qb = 0; qb < 2; ++qb) {
+      mbar_init(bar(BAR_Q_FULL + qb), 1);
+      mbar_init(bar(BAR_Q_EMPTY + qb), 1);
+    }
     for (int s = 0; s < kStages; ++s) {
       mbar_init(bar(BAR_K_FULL + s), 1);
       mbar_init(bar(BAR_K_EMPTY + s), 1);
@@ -153,12 +156,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
       const Unit w = unit_at(a, n_items, u);
       if (w.ntiles == 0) continue;
-      ok = warp_wait(bar(BAR_Q_EMPTY), (qn & 1) ^ 1, a.ws);
+      // Q tiles alternate between two buffers, so the next unit's Q is loaded
+      // while the current unit still runs.
+      const uint32_t qb = qn & 1;
+      ok = warp_wait(bar(BAR_Q_EMPTY + qb), ((qn >> 1) & 1) ^ 1, a.ws);
       if (!ok) break;
       if (lane == 0) {
-        mbar_expect_tx(bar(BAR_Q_FULL), C::TILE);
+        mbar_expect_tx(bar(BAR_Q_FULL + qb), C::TILE);
         for (int b = 0; b < C::NB; ++b)
-          tma_load_2d(sQ + b * C::BLK, &tmq, bar(BAR_Q_FULL), w.h * D + b * C::BOXW, w.s0 + w.r0);
+          tma_load_2d(sQ + qb * C::TILE + b * C::BLK, &tmq, bar(BAR_Q_FULL + qb),
+                      w.h * D + b * C::BOXW, w.s0 + w.r0);
       }
       ++qn;
       for (int n = 0; n < w.ntiles && ok; ++n) {
@@ -189,7 +196,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // If any role gave up, every load issued must still land before the CTA
     // exits (each barrier has at most its last armed phase outstanding).
     if (lane == 0 && load_status(a.ws) != 0) {
-      if (qn > 0) drain_wait(bar(BAR_Q_FULL), (qn - 1) & 1);
+      for (uint32_t qb = 0; qb < 2; ++qb) {
+        const uint32_t armed = qn / 2 + (qb < (qn & 1) ? 1u : 0u);
+        if (armed > 0) drain_wait(bar(BAR_Q_FULL + qb), (armed - 1) & 1);
+      }
       for (int s = 0; s < kStages; ++s) {
         const uint32_t k_armed = kn / kStages + (s < (int)(kn % kStages) ? 1u : 0u);
         const uint32_t v_armed = vn / kStages + (s < (int)(vn % kStages) ? 1u : 0u);
@@ -234,7 +244,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
       const Unit w = unit_at(a, n_items, u);
       if (w.ntiles == 0) continue;
-      ok = warp_wait(bar(BAR_Q_FULL), qn & 1, a.ws);
+      const uint32_t qb = qn & 1;
+      ok = warp_wait(bar(BAR_Q_FULL + qb), (qn >> 1) & 1, a.ws);
       if (!ok) break;
       tc_fence_after();
       const uint32_t kv0 = kv, tc0 = tc;
@@ -248,11 +259,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t dk = dK + ((uint32_t)(s * C::TILE) >> 4);
 #pragma unroll
           for (int ks = 0; ks < D / 16; ++ks)
-            mma_ss(tmem + kColS0 + b * 128, dQ + (kstep(ks) >> 4), dk + (kstep(ks) >> 4),
+            mma_ss(tmem + kColS0 + b * 128, dQ + ((qb * C::TILE + kstep(ks)) >> 4),
+                   dk + (kstep(ks) >> 4),
                    C::IDESC_S, ks > 0 ? 1u : 0u);
           tc_commit(bar(BAR_S_FULL + b));
           tc_commit(bar(BAR_K_EMPTY + s));
-          if (n + 1 == w.ntiles) tc_commit(bar(BAR_Q_EMPTY));  // last use of this Q tile
+          if (n + 1 == w.ntiles) tc_commit(bar(BAR_Q_EMPTY + qb));  // last use of this Q tile
         }
         __syncwarp();
         if (n > 0) {
