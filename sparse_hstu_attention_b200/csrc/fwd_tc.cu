@@ -8,19 +8,28 @@
 // Persistent, warp-specialised: one CTA per SM walks (head, 128-row query
 // tile) work units.  Per unit only the key tiles that the SLA mask leaves
 // non-empty are visited (global prefix, local band, candidates' diagonal).
-//   warp 0      TMA producer: Q tiles into two alternating buffers, K and V
-//               tiles (128 keys) into a 2-stage ring; 128B-swizzled boxes
-//               of 64 head-dim columns.
-//   warp 1      allocates TMEM; one lane issues UMMA: S = Q K^T into one of
-//               two TMEM S buffers (M=128, N=128, K=d), then O += P V with P
-//               read from TMEM (M=128, N=d, K=128) into the O accumulator.
-//   warps 2..17 pointwise: TMEM -> registers, P = SiLU(alpha S) (masked only
-//               on partial tiles) as bf16 back into TMEM; after the last key
-//               tile, the epilogue: O * (1/N) -> bf16 -> global, rows past the
-//               sequence end not written.  Four warps share each 32-lane TMEM
-//               quarter, one per 32-column chunk, so TMEM load/store latency
-//               is hidden across warps.
-// TMEM columns: S0 [0,128) S1 [128,256) O [256,256+d) P0 [384,448) P1 [448,512).
+//   warp 0      decodes each unit once into a 4-slot shared-memory ring that
+//               the other roles read, and loads Q tiles (two alternating
+//               buffers) and K tiles (ring) by TMA, 128B-swizzled boxes of
+//               64 head-dim columns.
+//   warp 1      allocates TMEM; one lane issues UMMA: S = Q K^T (M=128,
+//               N=128, K=d) into one of three TMEM score buffers, and
+//               O += P V (M=128, N=d, K=128) with P read from TMEM.  S runs
+//               two key tiles ahead of P V, so the pointwise stage of a tile
+//               has two tile periods of tensor work to hide behind.
+//   warp 2      loads V tiles into their own ring, so a K load never queues
+//               behind a V slot that is still being read.
+//   warps 3..18 pointwise: two groups of eight take alternate key tiles;
+//               TMEM -> registers, P = SiLU(alpha S) (masked only on partial
+//               tiles) as bf16 written back over the scores it replaces;
+//               after a unit's last key tile all sixteen run the epilogue:
+//               O * (1/N) -> bf16 -> global, rows past the sequence end not
+//               written.
+// TMEM columns: score buffers [0,128) [128,256) [256,384), O [384,384+d).
+// P of score columns [32c, 32c+32) lives in columns [32c, 32c+16) of the
+// same buffer; the P V MMA for keys [16k, 16k+16) reads 8 columns there.
+// A score buffer is rewritten only by an S MMA issued after the P V MMA that
+// read it (tcgen05.mma from one thread executes in issue order).
 // SiLU(x) = h + h tanh(h), h = x/2: one MUFU op per score; 1/N applied once.
 // Every wait is bounded; on a timeout the kernel records HSTU_SLA_ERR_TIMEOUT,
 // drains what it issued and frees TMEM.
@@ -38,61 +47,61 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kBM = 128, kBN = 128, kPwWarps = 16;
-constexpr int kThreads = 64 + 32 * kPwWarps;
-constexpr uint32_t kColS0 = 0, kColO = 256, kColP0 = 384, kTmemCols = 512;
-
-// K/V ring depth: as deep as 227 KB of shared memory allows.
-template <int D>
-constexpr int fwd_stages() { return D == 128 ? 2 : 4; }
+constexpr int kBM = 128, kBN = 128, kPwWarps = 16, kSBufs = 3, kUSlots = 4;
+constexpr int kPwWarp0 = 3;                         // first pointwise warp
+constexpr int kThreads = 32 * (kPwWarp0 + kPwWarps);
+constexpr uint32_t kColS = 0, kColO = 384, kTmemCols = 512;
 
 template <int D>
 struct Cfg {
-  static constexpr int kStages = fwd_stages<D>();
+  // Ring depths, as deep as 227 KB of shared memory allows.  A K slot is
+  // free again once the S MMA that read it has completed, which the score
+  // buffer's S_FULL barrier already signals; that reuse needs kKSt <= 3 (a
+  // buffer's next S cannot complete before the load that waits on it).
+  static constexpr int kKSt = D == 128 ? 2 : 3;
+  static constexpr int kVSt = D == 128 ? 3 : 4;
   static constexpr int SW = D >= 64 ? 128 : 64;   // swizzle span (bytes) = one box row
   static constexpr int BOXW = SW / 2;             // bf16 elements per box row
   static constexpr int NB = D / BOXW;             // boxes per tile
   static constexpr int BLK = 128 * SW;            // bytes per box (128 rows)
   static constexpr int TILE = 128 * D * 2;        // bytes per Q / K / V tile
-  static constexpr int OFF_Q = 0;                      // two Q buffers
+  static constexpr int OFF_Q = 0;                 // two Q buffers
   static constexpr int OFF_K = 2 * TILE;
-  static constexpr int OFF_V = TILE * (2 + kStages);
-  static constexpr int OFF_BAR = TILE * (2 + 2 * kStages);
-  static_assert(OFF_BAR + 256 + 1024 <= 232448, "shared memory budget");
-  static constexpr int SMEM = OFF_BAR + 256 + 1024;  // barriers + 1 KB alignment slack
+  static constexpr int OFF_V = (2 + kKSt) * TILE;
+  static constexpr int OFF_BAR = (2 + kKSt + kVSt) * TILE;
+  static constexpr int OFF_UNIT = OFF_BAR + 512;
+  static constexpr int OFF_SLOT = OFF_UNIT + kUSlots * (int)sizeof(UnitRec);
+  static constexpr int SMEM = OFF_SLOT + 16 + 1024;  // + 1 KB alignment slack
+  static_assert(SMEM <= 232448, "shared memory budget");
   static constexpr uint32_t SWZ = SW == 128 ? kSwizzle128B : kSwizzle64B;
   static constexpr uint32_t SBO = 8 * SW;             // stride of 8-row groups
   static constexpr uint32_t IDESC_S = idesc_bf16(128, kBN, false, false);
   static constexpr uint32_t IDESC_O = idesc_bf16(128, D, false, true);
-  static constexpr int COLS_PER_PW = kBN / (kPwWarps / 4);  // S columns per pointwise warp (32)
 };
 
 // Barrier slots (8 bytes each) after the tiles.
-constexpr int kMaxStages = 4;
+constexpr int kMaxSt = 4;
 enum {
-  BAR_Q_FULL = 0, BAR_Q_EMPTY = 2, BAR_K_FULL = 4, BAR_K_EMPTY = BAR_K_FULL + kMaxStages,
-  BAR_V_FULL = BAR_K_EMPTY + kMaxStages, BAR_V_EMPTY = BAR_V_FULL + kMaxStages,
-  BAR_S_FULL = BAR_V_EMPTY + kMaxStages, BAR_P_FULL = BAR_S_FULL + 2, BAR_O_FULL = BAR_P_FULL + 2,
-  BAR_O_EMPTY, BAR_DRAIN, BAR_COUNT
+  BAR_Q_FULL = 0, BAR_Q_EMPTY = 2, BAR_K_FULL = 4, BAR_V_FULL = BAR_K_FULL + kMaxSt, BAR_V_EMPTY = BAR_V_FULL + kMaxSt,
+  BAR_S_FULL = BAR_V_EMPTY + kMaxSt, BAR_P_FULL = BAR_S_FULL + kSBufs,
+  BAR_O_FULL = BAR_P_FULL + kSBufs, BAR_O_EMPTY, BAR_U_FULL, BAR_U_EMPTY = BAR_U_FULL + kUSlots,
+  BAR_DRAIN = BAR_U_EMPTY + kUSlots, BAR_COUNT
 };
+static_assert(8 * BAR_COUNT <= 512, "barrier area");
 
-struct Unit {
-  int h, s0, L, Lh, r0, r1;
-  Spans sp;
-  int ntiles;
-};
-
-__device__ __forceinline__ Unit unit_at(const AttnArgs& a, int n_items, int u) {
-  Unit w;
-  w.h = u / n_items;
-  const int2 it = a.items[u - w.h * n_items];
+// Unit u of the static schedule: head u / n_items, query tile
+// items[u % n_items]; the key tiles it meets.  u >= total ends the schedule.
+__device__ void decode_unit(const AttnArgs& a, int n_items, int total, int u, UnitRec* r) {
+  if (u >= total) {
+    r->nsteps = -1;
+    return;
+  }
+  const int h = u / n_items;
+  const int2 it = a.items[u - h * n_items];
   const SeqGeom g = seq_geom(a, it.x);
-  w.s0 = g.s0; w.L = g.L; w.Lh = g.Lh;
-  w.r0 = it.y * kBM;
-  w.r1 = imin(w.r0 + kBM, g.L);
-  w.sp = q_tile_key_tiles(w.r0, w.r1, g.Lh, a.K1, a.K2e, kBN);
-  w.ntiles = w.sp.count();
-  return w;
+  const int t0 = it.y * kBM;
+  const int t1 = imin(t0 + kBM, g.L);
+  unit_rec_fill(r, h, g.s0, g.L, g.Lh, t0, t1, q_tile_key_tiles(t0, t1, g.Lh, a.K1, a.K2e, kBN));
 }
 
 template <int D>
@@ -100,7 +109,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv, const AttnArgs a) {
   using C = Cfg<D>;
-  constexpr int kStages = C::kStages;
+  constexpr int kKSt = C::kKSt, kVSt = C::kVSt;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -108,7 +117,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sQ = base + C::OFF_Q, sK = base + C::OFF_K, sV = base + C::OFF_V;
   const uint32_t bar0 = base + C::OFF_BAR;
   auto bar = [&](int i) { return bar0 + 8u * i; };
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + C::OFF_BAR + 8 * BAR_COUNT);
+  UnitRec* ring = reinterpret_cast<UnitRec*>(base_ptr + C::OFF_UNIT);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + C::OFF_SLOT);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (load_status(a.ws) != 0) return;  // device-side input check failed
@@ -120,18 +130,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(BAR_Q_FULL + qb), 1);
       mbar_init(bar(BAR_Q_EMPTY + qb), 1);
     }
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kKSt; ++s) {
       mbar_init(bar(BAR_K_FULL + s), 1);
-      mbar_init(bar(BAR_K_EMPTY + s), 1);
+    }
+    for (int s = 0; s < kVSt; ++s) {
       mbar_init(bar(BAR_V_FULL + s), 1);
       mbar_init(bar(BAR_V_EMPTY + s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kSBufs; ++b) {
       mbar_init(bar(BAR_S_FULL + b), 1);
-      mbar_init(bar(BAR_P_FULL + b), kPwWarps / 2);  // one arrive per warp of group b
+      mbar_init(bar(BAR_P_FULL + b), kPwWarps / 2);  // one arrive per warp of the tile's group
     }
     mbar_init(bar(BAR_O_FULL), 1);
     mbar_init(bar(BAR_O_EMPTY), kPwWarps);
+    for (int s = 0; s < kUSlots; ++s) {
+      mbar_init(bar(BAR_U_FULL + s), 1);
+      mbar_init(bar(BAR_U_EMPTY + s), kPwWarps + 2);  // MMA, V loader, pointwise warps
+    }
     mbar_init(bar(BAR_DRAIN), 1);
     fence_barrier_init();
     prefetch_tmap(&tmq);
@@ -148,14 +163,33 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    // The whole warp walks the schedule (so every value stays warp-uniform);
-    // lane 0 arms the barriers and issues the copies.
-    uint32_t qn = 0, kv = 0, kn = 0, vn = 0;
+    // ------------------------------------------- unit decoder, Q and K loads
+    // The whole warp walks the schedule (every value stays warp-uniform);
+    // lane 0 decodes units, arms the barriers and issues the copies.  Unit
+    // kk + 1 is decoded right after unit kk's first K load is issued, so its
+    // global reads overlap the copies in flight.
+    uint32_t qn = 0, kn = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
-      const Unit w = unit_at(a, n_items, u);
-      if (w.ntiles == 0) continue;
+    auto publish = [&](int kk) -> bool {
+      const int slot = kk % kUSlots;
+      if (!warp_wait(bar(BAR_U_EMPTY + slot), ((kk / kUSlots) & 1) ^ 1, a.ws)) return false;
+      if (lane == 0) {
+        decode_unit(a, n_items, total, blockIdx.x + kk * gridDim.x, &ring[slot]);
+        mbar_arrive(bar(BAR_U_FULL + slot));
+      }
+      __syncwarp();
+      return true;
+    };
+    ok = publish(0);
+    for (int kk = 0; ok; ++kk) {
+      const UnitRec* r = &ring[kk % kUSlots];
+      const int nt = r->nsteps;
+      if (nt < 0) break;
+      if (nt == 0) {
+        ok = publish(kk + 1);
+        continue;
+      }
+      const int h = r->h, s0 = r->s0;
       // Q tiles alternate between two buffers, so the next unit's Q is loaded
       // while the current unit still runs.
       const uint32_t qb = qn & 1;
@@ -165,32 +199,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_expect_tx(bar(BAR_Q_FULL + qb), C::TILE);
         for (int b = 0; b < C::NB; ++b)
           tma_load_2d(sQ + qb * C::TILE + b * C::BLK, &tmq, bar(BAR_Q_FULL + qb),
-                      w.h * D + b * C::BOXW, w.s0 + w.r0);
+                      h * D + b * C::BOXW, s0 + r->t0);
       }
       ++qn;
-      for (int n = 0; n < w.ntiles && ok; ++n) {
-        const int y = w.s0 + w.sp.at(n) * kBN;
-        const int s = kv % kStages;
-        const uint32_t ph = (kv / kStages) & 1;
-        ok = warp_wait(bar(BAR_K_EMPTY + s), ph ^ 1, a.ws);
-        if (!ok) break;
+      SpanCursor c;
+      c.begin(r);
+      for (int n = 0; n < nt && ok; ++n, c.next(r)) {
+        // the slot's previous tile, kn - kKSt, must have been read by its S MMA
+        const int s = kn % kKSt;
+        if (kn >= (uint32_t)kKSt) {
+          const uint32_t prev = kn - kKSt;
+          ok = warp_wait(bar(BAR_S_FULL + prev % kSBufs), (prev / kSBufs) & 1, a.ws);
+          if (!ok) break;
+        }
         if (lane == 0) {
           mbar_expect_tx(bar(BAR_K_FULL + s), C::TILE);
           for (int b = 0; b < C::NB; ++b)
             tma_load_2d(sK + s * C::TILE + b * C::BLK, &tmk, bar(BAR_K_FULL + s),
-                        w.h * D + b * C::BOXW, y);
+                        h * D + b * C::BOXW, s0 + c.j * kBN);
         }
         ++kn;
-        ok = warp_wait(bar(BAR_V_EMPTY + s), ph ^ 1, a.ws);
-        if (!ok) break;
-        if (lane == 0) {
-          mbar_expect_tx(bar(BAR_V_FULL + s), C::TILE);
-          for (int b = 0; b < C::NB; ++b)
-            tma_load_2d(sV + s * C::TILE + b * C::BLK, &tmv, bar(BAR_V_FULL + s),
-                        w.h * D + b * C::BOXW, y);
-        }
-        ++vn;
-        ++kv;
+        if (n == 0) ok = publish(kk + 1);
       }
     }
     // If any role gave up, every load issued must still land before the CTA
@@ -200,103 +229,157 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t armed = qn / 2 + (qb < (qn & 1) ? 1u : 0u);
         if (armed > 0) drain_wait(bar(BAR_Q_FULL + qb), (armed - 1) & 1);
       }
-      for (int s = 0; s < kStages; ++s) {
-        const uint32_t k_armed = kn / kStages + (s < (int)(kn % kStages) ? 1u : 0u);
-        const uint32_t v_armed = vn / kStages + (s < (int)(vn % kStages) ? 1u : 0u);
-        if (k_armed > 0) drain_wait(bar(BAR_K_FULL + s), (k_armed - 1) & 1);
-        if (v_armed > 0) drain_wait(bar(BAR_V_FULL + s), (v_armed - 1) & 1);
+      for (int s = 0; s < kKSt; ++s) {
+        const uint32_t armed = kn / kKSt + (s < (int)(kn % kKSt) ? 1u : 0u);
+        if (armed > 0) drain_wait(bar(BAR_K_FULL + s), (armed - 1) & 1);
+      }
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------- V loads
+    uint32_t vn = 0;
+    bool ok = true;
+    for (int kk = 0; ok; ++kk) {
+      const int slot = kk % kUSlots;
+      ok = warp_wait(bar(BAR_U_FULL + slot), (kk / kUSlots) & 1, a.ws);
+      if (!ok) break;
+      const UnitRec* r = &ring[slot];
+      const int nt = r->nsteps, h = r->h, s0 = r->s0;
+      SpanCursor c;
+      c.begin(r);
+      for (int n = 0; n < nt && ok; ++n, c.next(r)) {
+        const int s = vn % kVSt;
+        ok = warp_wait(bar(BAR_V_EMPTY + s), ((vn / kVSt) & 1) ^ 1, a.ws);
+        if (!ok) break;
+        if (lane == 0) {
+          mbar_expect_tx(bar(BAR_V_FULL + s), C::TILE);
+          for (int b = 0; b < C::NB; ++b)
+            tma_load_2d(sV + s * C::TILE + b * C::BLK, &tmv, bar(BAR_V_FULL + s),
+                        h * D + b * C::BOXW, s0 + c.j * kBN);
+        }
+        ++vn;
+      }
+      warp_arrive(bar(BAR_U_EMPTY + slot));
+      if (nt < 0) break;
+    }
+    if (lane == 0 && load_status(a.ws) != 0) {
+      for (int s = 0; s < kVSt; ++s) {
+        const uint32_t armed = vn / kVSt + (s < (int)(vn % kVSt) ? 1u : 0u);
+        if (armed > 0) drain_wait(bar(BAR_V_FULL + s), (armed - 1) & 1);
       }
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------- MMA issuer
-    // The whole warp runs the loop with warp-uniform descriptors; lane 0
-    // issues every UMMA and commit (a commit tracks the issuing thread's MMAs).
-    uint32_t qn = 0, kv = 0, tc = 0, on = 0;
-    bool ok = true;
-    // Descriptor bases; a k-step / stage only adds to the start-address field
-    // (smem addresses stay below 2^18, so the 14-bit field never carries).
-    const uint64_t dQ = smem_desc(sQ, 16, C::SBO, C::SWZ);
-    const uint64_t dK = smem_desc(sK, 16, C::SBO, C::SWZ);
-    const uint64_t dV = smem_desc(sV, C::BLK, C::SBO, C::SWZ);
-    auto kstep = [](int ks) -> uint32_t {  // byte offset of k-step ks in a K-major tile
-      return (uint32_t)(((ks * 32) / C::SW) * C::BLK + (ks * 32) % C::SW);
-    };
-    // O += P(tile m) V(tile m); kvm / tcm: that tile's ring / S-buffer counters.
-    auto pv = [&](uint32_t kvm, uint32_t tcm, bool first) -> bool {
-      const uint32_t b = tcm & 1;
-      if (!warp_wait(bar(BAR_P_FULL + b), (tcm >> 1) & 1, a.ws)) return false;
-      const int s = kvm % kStages;
-      if (!warp_wait(bar(BAR_V_FULL + s), (kvm / kStages) & 1, a.ws)) return false;
-      if (first && !warp_wait(bar(BAR_O_EMPTY), (on & 1) ^ 1, a.ws)) return false;
-      tc_fence_after();
-      if (lane == 0) {
+    // One lane runs this role alone: a tcgen05.mma costs its issuing thread
+    // about as long as the tensor pipe takes to execute it, so every wait and
+    // commit here is kept single-threaded and per tile there are only two
+    // commits (S_FULL, which also frees the K slot, and V_EMPTY).
+    // Tiles are numbered across units: tile t uses score buffer t % 3, K slot
+    // t % kKSt and V slot t % kVSt; its P V is issued once S of tile t + 2 is
+    // issued (or earlier, see below), so P V of a unit's last tiles overlaps
+    // S of the next unit's first.
+    if (lane == 0) {
+      uint32_t qn = 0, tc = 0, pvc = 0, on = 0;
+      uint32_t pend = 0;  // 2 bits per tile in [pvc, tc): first / last of its unit
+      bool ok = true;
+      // Descriptor bases; a k-step / stage only adds to the start-address field
+      // (smem addresses stay below 2^18, so the 14-bit field never carries).
+      const uint64_t dQ = smem_desc(sQ, 16, C::SBO, C::SWZ);
+      const uint64_t dK = smem_desc(sK, 16, C::SBO, C::SWZ);
+      const uint64_t dV = smem_desc(sV, C::BLK, C::SBO, C::SWZ);
+      auto kstep = [](int ks) -> uint32_t {  // byte offset of k-step ks in a K-major tile
+        return (uint32_t)(((ks * 32) / C::SW) * C::BLK + (ks * 32) % C::SW);
+      };
+      auto pv = [&]() -> bool {  // O += P V for tile pvc
+        const uint32_t f = pend & 3u;
+        pend >>= 2;
+        const bool first = (f & 1u) != 0, last = (f & 2u) != 0;
+        const uint32_t b = pvc % kSBufs;
+        const int s = pvc % kVSt;
+        if (!mbar_wait(bar(BAR_P_FULL + b), (pvc / kSBufs) & 1, a.ws)) return false;
+        if (!mbar_wait(bar(BAR_V_FULL + s), (pvc / kVSt) & 1, a.ws)) return false;
+        if (first && !mbar_wait(bar(BAR_O_EMPTY), (on & 1) ^ 1, a.ws)) return false;
+        tc_fence_after();
         const uint64_t dv = dV + ((uint32_t)(s * C::TILE) >> 4);
 #pragma unroll
         for (int ks = 0; ks < kBN / 16; ++ks)
-          mma_ts(tmem + kColO, tmem + kColP0 + b * 64 + ks * 8,
+          mma_ts(tmem + kColO, tmem + kColS + b * 128 + (ks >> 1) * 32 + (ks & 1) * 8,
                  dv + ((uint32_t)(ks * 16 * C::SW) >> 4), C::IDESC_O,
-                 (!first || ks > 0) ? 1u : 0u);
+                 (first && ks == 0) ? 0u : 1u);
         tc_commit(bar(BAR_V_EMPTY + s));
-      }
-      __syncwarp();
-      return true;
-    };
-    for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
-      const Unit w = unit_at(a, n_items, u);
-      if (w.ntiles == 0) continue;
-      const uint32_t qb = qn & 1;
-      ok = warp_wait(bar(BAR_Q_FULL + qb), (qn >> 1) & 1, a.ws);
-      if (!ok) break;
-      tc_fence_after();
-      const uint32_t kv0 = kv, tc0 = tc;
-      for (int n = 0; n < w.ntiles; ++n) {
-        const int s = kv % kStages;
-        ok = warp_wait(bar(BAR_K_FULL + s), (kv / kStages) & 1, a.ws);
+        if (last) {
+          tc_commit(bar(BAR_O_FULL));
+          ++on;
+        }
+        ++pvc;
+        return true;
+      };
+      // P V may be deferred into the next unit only when that unit is already
+      // published and not empty: pending P V then belong to the last two
+      // non-empty units, and nothing the producer waits on (the release of
+      // the ring slot four units back, which follows that unit's epilogue)
+      // depends on them.
+      auto flush = [&]() -> bool {
+        while (pvc != tc)
+          if (!pv()) return false;
+        return true;
+      };
+      for (int kk = 0; ok; ++kk) {
+        const int slot = kk % kUSlots;
+        const uint32_t uph = (kk / kUSlots) & 1;
+        if (pvc != tc && !mbar_try_wait(bar(BAR_U_FULL + slot), uph)) {
+          ok = flush();
+          if (!ok) break;
+        }
+        ok = mbar_wait(bar(BAR_U_FULL + slot), uph, a.ws);
+        if (!ok) break;
+        const int nt = ring[slot].nsteps;
+        mbar_arrive(bar(BAR_U_EMPTY + slot));
+        if (nt <= 0) {
+          ok = flush();
+          if (nt < 0) break;
+          continue;
+        }
+        const uint32_t qb = qn & 1;
+        ok = mbar_wait(bar(BAR_Q_FULL + qb), (qn >> 1) & 1, a.ws);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t b = tc & 1;
-        if (lane == 0) {
+        for (int n = 0; n < nt; ++n) {
+          const int s = tc % kKSt;
+          ok = mbar_wait(bar(BAR_K_FULL + s), (tc / kKSt) & 1, a.ws);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t b = tc % kSBufs;
           const uint64_t dk = dK + ((uint32_t)(s * C::TILE) >> 4);
 #pragma unroll
           for (int ks = 0; ks < D / 16; ++ks)
-            mma_ss(tmem + kColS0 + b * 128, dQ + ((qb * C::TILE + kstep(ks)) >> 4),
-                   dk + (kstep(ks) >> 4),
-                   C::IDESC_S, ks > 0 ? 1u : 0u);
+            mma_ss(tmem + kColS + b * 128, dQ + ((qb * C::TILE + kstep(ks)) >> 4),
+                   dk + (kstep(ks) >> 4), C::IDESC_S, ks > 0 ? 1u : 0u);
           tc_commit(bar(BAR_S_FULL + b));
-          tc_commit(bar(BAR_K_EMPTY + s));
-          if (n + 1 == w.ntiles) tc_commit(bar(BAR_Q_EMPTY + qb));  // last use of this Q tile
+          if (n + 1 == nt) tc_commit(bar(BAR_Q_EMPTY + qb));  // last use of this Q tile
+          pend |= ((n == 0 ? 1u : 0u) | (n + 1 == nt ? 2u : 0u)) << (2 * (tc - pvc));
+          ++tc;
+          if (tc - pvc > 2) {
+            ok = pv();
+            if (!ok) break;
+          }
         }
-        __syncwarp();
-        if (n > 0) {
-          ok = pv(kv - 1, tc - 1, n == 1);
-          if (!ok) break;
-        }
-        ++kv;
-        ++tc;
+        ++qn;
       }
-      if (!ok) break;
-      ok = pv(kv0 + w.ntiles - 1, tc0 + w.ntiles - 1, w.ntiles == 1);
-      if (!ok) break;
-      if (lane == 0) tc_commit(bar(BAR_O_FULL));
-      __syncwarp();
-      ++qn;
-      ++on;
-    }
-    // Every MMA issued must finish before TMEM is released.
-    if (lane == 0) {
+      if (ok) flush();
+      // Every MMA issued must finish before TMEM is released.
       tc_commit(bar(BAR_DRAIN));
       drain_wait(bar(BAR_DRAIN), 0);
     }
     __syncwarp();
   } else {
     // ----------------------------------------------- pointwise and epilogue
-    // Two groups of eight warps take alternate S tiles (group g owns S buffer
-    // g), so one group's TMEM load / store latency overlaps the other's
-    // arithmetic.  Within a group, the two warps on a 32-lane TMEM quarter
-    // split the tile's 128 columns in halves.  The epilogue uses all sixteen:
-    // warp `chunk` of a quarter writes O columns [32 chunk, +32).
-    const int pw = warp - 2;               // 0..15
-    const int grp = pw >> 3;               // S buffer / tile parity of this warp
+    // Two groups of eight warps take alternate key tiles, so one group's TMEM
+    // load / store latency overlaps the other's arithmetic.  Within a group,
+    // the two warps on a 32-lane TMEM quarter split the tile's 128 columns in
+    // halves.  The epilogue uses all sixteen: warp `chunk` of a quarter writes
+    // O columns [32 chunk, +32).
+    const int pw = warp - kPwWarp0;        // 0..15
+    const int grp = pw >> 3;               // tile parity of this warp
     const int quarter = warp & 3;          // TMEM lanes [32*quarter, +32)
     const int chunk = pw >> 2;             // 0..3
     const int half = chunk & 1;            // column half within the group
@@ -306,36 +389,49 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool has_o = chunk < D / 32;     // this warp writes an O chunk
     uint32_t tc = 0, on = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
-      const Unit w = unit_at(a, n_items, u);
-      const int i = w.r0 + row;  // row within the sequence
-      bf16* orow = a.out + (int64_t)(w.s0 + i) * a.o_rs + w.h * D + chunk * 32;
-      if (w.ntiles == 0) {  // no visible key anywhere in the tile
-        if (has_o && i < w.r1) {
+    for (int kk = 0; ok; ++kk) {
+      const int slot = kk % kUSlots;
+      ok = warp_wait(bar(BAR_U_FULL + slot), (kk / kUSlots) & 1, a.ws);
+      if (!ok) break;
+      const UnitRec* r = &ring[slot];
+      const int nt = r->nsteps;
+      if (nt < 0) {
+        warp_arrive(bar(BAR_U_EMPTY + slot));
+        break;
+      }
+      const int h = r->h, s0 = r->s0, Lh = r->Lh, t0 = r->t0, t1 = r->t1;
+      const int i = t0 + row;  // row within the sequence
+      bf16* orow = a.out + (int64_t)(s0 + i) * a.o_rs + h * D + chunk * 32;
+      if (nt == 0) {  // no visible key anywhere in the tile
+        if (has_o && i < t1) {
           const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
           for (int v = 0; v < 4; ++v) reinterpret_cast<uint4*>(orow)[v] = z;
         }
+        warp_arrive(bar(BAR_U_EMPTY + slot));
         continue;
       }
-      const RowMask m = row_mask(i, w.L, w.Lh, a.K1, a.K2e);
-      for (int n = 0; n < w.ntiles; ++n, ++tc) {
-        const uint32_t b = tc & 1;
-        if ((int)b != grp) continue;  // the other group's tile
-        ok = warp_wait(bar(BAR_S_FULL + b), (tc >> 1) & 1, a.ws);
+      const RowMask m = row_mask(i, r->L, Lh, a.K1, a.K2e);
+      SpanCursor c;
+      c.begin(r);
+      for (int n = 0; n < nt; ++n, ++tc, c.next(r)) {
+        if ((int)(tc & 1) != grp) continue;  // the other group's tile
+        const uint32_t b = tc % kSBufs;
+        ok = warp_wait(bar(BAR_S_FULL + b), (tc / kSBufs) & 1, a.ws);
         if (!ok) break;
         tc_fence_after();
-        const int j0 = w.sp.at(n) * kBN;
-        const bool full = tile_full(w.r0, w.r0 + kBM, j0, j0 + kBN, w.Lh, a.K1, a.K2e);
+        const int j0 = c.j * kBN;
+        const bool full = tile_full(t0, t0 + kBM, j0, j0 + kBN, Lh, a.K1, a.K2e);
         // P = SiLU(alpha S) = h + h tanh(h) with h = alpha S / 2.  Tiles that
         // are entirely visible skip the mask; the others clear invisible
         // entries with one bit test each against this row's 32-key bitmask.
 #pragma unroll
         for (int sub = 0; sub < 2; ++sub) {
           const int col = half * 64 + sub * 32;
+          const uint32_t taddr = lane_base + kColS + b * 128 + col;
           uint32_t c0[16], c1[16];
-          tmem_ld16(lane_base + kColS0 + b * 128 + col, c0);
-          tmem_ld16(lane_base + kColS0 + b * 128 + col + 16, c1);
+          tmem_ld16(taddr, c0);
+          tmem_ld16(taddr + 16, c1);
           tmem_ld_wait2(c0, c1);
           uint32_t p[16];
 #pragma unroll
@@ -348,7 +444,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 16; ++e) p[e] = mask_pair(p[e], bits, e);
           }
-          tmem_st16(lane_base + kColP0 + b * 64 + col / 2, p);
+          tmem_st16(taddr, p);  // over the first half of the scores just read
         }
         tmem_st_wait();
         tc_fence_before();
@@ -364,7 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld16(lane_base + kColO + chunk * 32, r0);
         tmem_ld16(lane_base + kColO + chunk * 32 + 16, r1);
         tmem_ld_wait2(r0, r1);
-        if (i < w.r1) {
+        if (i < t1) {
           uint32_t o[16];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
@@ -382,6 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       warp_arrive(bar(BAR_O_EMPTY));
       ++on;
+      warp_arrive(bar(BAR_U_EMPTY + slot));
     }
   }
 

@@ -284,6 +284,45 @@ __host__ __device__ __forceinline__ uint32_t key_mask_bits(const KeyMask& m, int
   return bits;
 }
 
+// One work unit as the producer warp decodes it once and hands it to the other
+// roles through a shared-memory ring: the sequence geometry, the resident
+// tile's rows [t0, t1) and the streamed tiles it meets, as up to three spans
+// of tile indices.  nsteps = -1 marks the end of the CTA's schedule.
+struct UnitRec {
+  int h, s0, L, Lh, t0, t1, nsteps, nsp;
+  int lo[3], hi[3];
+  int pad[2];
+};
+static_assert(sizeof(UnitRec) == 64, "unit record size");
+
+__device__ __forceinline__ void unit_rec_fill(UnitRec* r, int h, int s0, int L, int Lh, int t0,
+                                              int t1, const Spans& sp) {
+  r->h = h; r->s0 = s0; r->L = L; r->Lh = Lh; r->t0 = t0; r->t1 = t1;
+  r->nsteps = sp.count();
+  r->nsp = sp.n;
+  for (int s = 0; s < 3; ++s) {
+    r->lo[s] = s < sp.n ? sp.lo[s] : 0;
+    r->hi[s] = s < sp.n ? sp.hi[s] : 0;
+  }
+}
+
+// Walks the streamed tiles of a unit record in order, one step at a time.
+struct SpanCursor {
+  int s, j, hi;
+  __device__ __forceinline__ void begin(const UnitRec* r) {
+    s = 0;
+    j = r->lo[0];
+    hi = r->hi[0];
+  }
+  __device__ __forceinline__ void next(const UnitRec* r) {
+    if (++j == hi && s + 1 < r->nsp) {
+      ++s;
+      j = r->lo[s];
+      hi = r->hi[s];
+    }
+  }
+};
+
 __device__ __forceinline__ void set_status(WsHeader* ws, int code) {
   atomicCAS(&ws->status, 0, code);
 }
