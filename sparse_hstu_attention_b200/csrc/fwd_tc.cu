@@ -85,7 +85,7 @@ enum {
   BAR_Q_FULL = 0, BAR_Q_EMPTY = 2, BAR_K_FULL = 4, BAR_V_FULL = BAR_K_FULL + kMaxSt, BAR_V_EMPTY = BAR_V_FULL + kMaxSt,
   BAR_S_FULL = BAR_V_EMPTY + kMaxSt, BAR_P_FULL = BAR_S_FULL + kSBufs,
   BAR_O_FULL = BAR_P_FULL + kSBufs, BAR_O_EMPTY, BAR_U_FULL, BAR_U_EMPTY = BAR_U_FULL + kUSlots,
-  BAR_DRAIN = BAR_U_EMPTY + kUSlots, BAR_COUNT
+  BAR_DRAIN = BAR_U_EMPTY + kUSlots, BAR_OST, BAR_COUNT = BAR_OST + 2
 };
 static_assert(8 * BAR_COUNT <= 512, "barrier area");
 
@@ -107,7 +107,8 @@ __device__ void decode_unit(const AttnArgs& a, int n_items, int total, int u, Un
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
-                  const __grid_constant__ CUtensorMap tmv, const AttnArgs a) {
+                  const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
+                  const AttnArgs a) {
   using C = Cfg<D>;
   constexpr int kKSt = C::kKSt, kVSt = C::kVSt;
   extern __shared__ uint8_t smem_raw[];
@@ -128,7 +129,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int qb = 0; qb < 2; ++qb) {
       mbar_init(bar(BAR_Q_FULL + qb), 1);
-      mbar_init(bar(BAR_Q_EMPTY + qb), 1);
+      mbar_init(bar(BAR_Q_EMPTY + qb), 1 + C::NB);  // last S commit + one per O box stored
     }
     for (int s = 0; s < kKSt; ++s) {
       mbar_init(bar(BAR_K_FULL + s), 1);
@@ -148,10 +149,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(BAR_U_EMPTY + s), kPwWarps + 2);  // MMA, V loader, pointwise warps
     }
     mbar_init(bar(BAR_DRAIN), 1);
+    for (int b = 0; b < C::NB; ++b) mbar_init(bar(BAR_OST + b), 4 * (C::BOXW / 32));
     fence_barrier_init();
     prefetch_tmap(&tmq);
     prefetch_tmap(&tmk);
     prefetch_tmap(&tmv);
+    prefetch_tmap(&tmo);
   }
   if (warp == 1) {
     tmem_alloc(smem_addr(tmem_slot), kTmemCols);
@@ -275,8 +278,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // commits (S_FULL, which also frees the K slot, and V_EMPTY).
     // Tiles are numbered across units: tile t uses score buffer t % 3, K slot
     // t % kKSt and V slot t % kVSt; its P V is issued once S of tile t + 2 is
-    // issued (or earlier, see below), so P V of a unit's last tiles overlaps
-    // S of the next unit's first.
+    // issued, or earlier while the lane waits for a copy, so P V of a unit's
+    // last tiles overlaps S of the next unit's first.
     if (lane == 0) {
       uint32_t qn = 0, tc = 0, pvc = 0, on = 0;
       uint32_t pend = 0;  // 2 bits per tile in [pvc, tc): first / last of its unit
@@ -289,15 +292,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto kstep = [](int ks) -> uint32_t {  // byte offset of k-step ks in a K-major tile
         return (uint32_t)(((ks * 32) / C::SW) * C::BLK + (ks * 32) % C::SW);
       };
-      auto pv = [&]() -> bool {  // O += P V for tile pvc
+      // O += P V for tile pvc, its operands known to be ready.
+      auto pv_issue = [&]() {
         const uint32_t f = pend & 3u;
         pend >>= 2;
         const bool first = (f & 1u) != 0, last = (f & 2u) != 0;
         const uint32_t b = pvc % kSBufs;
         const int s = pvc % kVSt;
-        if (!mbar_wait(bar(BAR_P_FULL + b), (pvc / kSBufs) & 1, a.ws)) return false;
-        if (!mbar_wait(bar(BAR_V_FULL + s), (pvc / kVSt) & 1, a.ws)) return false;
-        if (first && !mbar_wait(bar(BAR_O_EMPTY), (on & 1) ^ 1, a.ws)) return false;
         tc_fence_after();
         const uint64_t dv = dV + ((uint32_t)(s * C::TILE) >> 4);
 #pragma unroll
@@ -311,41 +312,57 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++on;
         }
         ++pvc;
+      };
+      auto pv_ready = [&]() -> bool {  // P, V (and O, for a unit's first) of tile pvc
+        return mbar_test_wait(bar(BAR_P_FULL + pvc % kSBufs), (pvc / kSBufs) & 1) &&
+               mbar_test_wait(bar(BAR_V_FULL + pvc % kVSt), (pvc / kVSt) & 1) &&
+               ((pend & 1u) == 0 || mbar_test_wait(bar(BAR_O_EMPTY), (on & 1) ^ 1));
+      };
+      auto pv = [&]() -> bool {  // blocking form
+        if (!mbar_wait(bar(BAR_P_FULL + pvc % kSBufs), (pvc / kSBufs) & 1, a.ws)) return false;
+        if (!mbar_wait(bar(BAR_V_FULL + pvc % kVSt), (pvc / kVSt) & 1, a.ws)) return false;
+        if ((pend & 1u) && !mbar_wait(bar(BAR_O_EMPTY), (on & 1) ^ 1, a.ws)) return false;
+        pv_issue();
         return true;
       };
-      // P V may be deferred into the next unit only when that unit is already
-      // published and not empty: pending P V then belong to the last two
-      // non-empty units, and nothing the producer waits on (the release of
-      // the ring slot four units back, which follows that unit's epilogue)
-      // depends on them.
-      auto flush = [&]() -> bool {
-        while (pvc != tc)
-          if (!pv()) return false;
-        return true;
+      // Waits for a load / the next unit while issuing every deferred P V as
+      // soon as its operands are ready.  What these waits depend on (the
+      // producer's next copies, which may wait for a unit's epilogue to free
+      // its Q buffer or ring slot) can depend on deferred P V, so they must
+      // never sit behind such a wait.
+      auto wait_issuing = [&](uint32_t b, uint32_t parity) -> bool {
+        if (mbar_test_wait(b, parity)) return true;
+        const uint64_t t0 = globaltimer();
+        for (uint32_t it = 1;; ++it) {
+          if (mbar_test_wait(b, parity)) return true;
+          if (pvc != tc && pv_ready()) {
+            pv_issue();
+            continue;
+          }
+          if ((it & 255u) == 0) {
+            if (load_status(a.ws) != 0) return false;
+            if (globaltimer() - t0 > kWaitLimitNs) {
+              set_status(a.ws, HSTU_SLA_ERR_TIMEOUT);
+              return false;
+            }
+          }
+        }
       };
       for (int kk = 0; ok; ++kk) {
         const int slot = kk % kUSlots;
-        const uint32_t uph = (kk / kUSlots) & 1;
-        if (pvc != tc && !mbar_try_wait(bar(BAR_U_FULL + slot), uph)) {
-          ok = flush();
-          if (!ok) break;
-        }
-        ok = mbar_wait(bar(BAR_U_FULL + slot), uph, a.ws);
+        ok = wait_issuing(bar(BAR_U_FULL + slot), (kk / kUSlots) & 1);
         if (!ok) break;
         const int nt = ring[slot].nsteps;
         mbar_arrive(bar(BAR_U_EMPTY + slot));
-        if (nt <= 0) {
-          ok = flush();
-          if (nt < 0) break;
-          continue;
-        }
+        if (nt < 0) break;
+        if (nt == 0) continue;
         const uint32_t qb = qn & 1;
-        ok = mbar_wait(bar(BAR_Q_FULL + qb), (qn >> 1) & 1, a.ws);
+        ok = wait_issuing(bar(BAR_Q_FULL + qb), (qn >> 1) & 1);
         if (!ok) break;
         tc_fence_after();
         for (int n = 0; n < nt; ++n) {
           const int s = tc % kKSt;
-          ok = mbar_wait(bar(BAR_K_FULL + s), (tc / kKSt) & 1, a.ws);
+          ok = wait_issuing(bar(BAR_K_FULL + s), (tc / kKSt) & 1);
           if (!ok) break;
           tc_fence_after();
           const uint32_t b = tc % kSBufs;
@@ -355,9 +372,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_ss(tmem + kColS + b * 128, dQ + ((qb * C::TILE + kstep(ks)) >> 4),
                    dk + (kstep(ks) >> 4), C::IDESC_S, ks > 0 ? 1u : 0u);
           tc_commit(bar(BAR_S_FULL + b));
-          if (n + 1 == nt) tc_commit(bar(BAR_Q_EMPTY + qb));  // last use of this Q tile
+          if (n + 1 == nt) tc_commit(bar(BAR_Q_EMPTY + qb));  // last S read of this Q tile
           pend |= ((n == 0 ? 1u : 0u) | (n + 1 == nt ? 2u : 0u)) << (2 * (tc - pvc));
           ++tc;
+          // the score buffer of tile tc (next S) is free once P V of tc - 3
+          // is issued: keep at most two tiles' P V pending
           if (tc - pvc > 2) {
             ok = pv();
             if (!ok) break;
@@ -365,7 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ++qn;
       }
-      if (ok) flush();
+      while (ok && pvc != tc) ok = pv();
       // Every MMA issued must finish before TMEM is released.
       tc_commit(bar(BAR_DRAIN));
       drain_wait(bar(BAR_DRAIN), 0);
@@ -387,7 +406,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     const float half_alpha = 0.5f * a.alpha;
     const bool has_o = chunk < D / 32;     // this warp writes an O chunk
-    uint32_t tc = 0, on = 0;
+    // Epilogue store: a tile that lies inside its sequence is staged as bf16
+    // in the unit's Q buffer (no S MMA reads it any more) in the swizzled
+    // layout of a TMA box and stored by one thread per box; that thread
+    // releases the Q buffer once the store has read it.  Tiles that run past
+    // the sequence end are written row by row, rows past the end skipped.
+    const int box = (chunk * 32) / C::BOXW;          // O box of this warp's chunk
+    const int box_c0 = ((chunk * 32) % C::BOXW) / 8;  // its first 16-byte chunk in a box row
+    const bool box_leader = has_o && quarter == 0 && (chunk * 32) % C::BOXW == 0;
+    const uint32_t swz = C::SW == 128 ? (uint32_t)(row & 7) : (uint32_t)((row >> 1) & 3);
+    uint32_t tc = 0, on = 0, qn = 0;
     bool ok = true;
     for (int kk = 0; ok; ++kk) {
       const int slot = kk % kUSlots;
@@ -455,31 +483,61 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = warp_wait(bar(BAR_O_FULL), on & 1, a.ws);
       if (!ok) break;
       tc_fence_after();
+      const uint32_t qb = qn & 1;
+      const bool whole = t1 - t0 == kBM;
+      uint32_t o[16];
       if (has_o) {
         uint32_t r0[16], r1[16];
         tmem_ld16(lane_base + kColO + chunk * 32, r0);
         tmem_ld16(lane_base + kColO + chunk * 32 + 16, r1);
         tmem_ld_wait2(r0, r1);
-        if (i < t1) {
-          uint32_t o[16];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            o[e] = pack_bf16x2(__uint_as_float(r0[2 * e]) * a.inv_n,
-                               __uint_as_float(r0[2 * e + 1]) * a.inv_n);
-            o[8 + e] = pack_bf16x2(__uint_as_float(r1[2 * e]) * a.inv_n,
-                                   __uint_as_float(r1[2 * e + 1]) * a.inv_n);
-          }
+        for (int e = 0; e < 8; ++e) {
+          o[e] = pack_bf16x2(__uint_as_float(r0[2 * e]) * a.inv_n,
+                             __uint_as_float(r0[2 * e + 1]) * a.inv_n);
+          o[8 + e] = pack_bf16x2(__uint_as_float(r1[2 * e]) * a.inv_n,
+                                 __uint_as_float(r1[2 * e + 1]) * a.inv_n);
+        }
+      }
+      // O is in registers: the next unit's P V may overwrite it
+      tc_fence_before();
+      warp_arrive(bar(BAR_O_EMPTY));
+      if (has_o) {
+        if (whole) {
+          const uint32_t rowaddr = sQ + qb * C::TILE + box * C::BLK + row * C::SW;
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            st_shared_v4(rowaddr + ((((uint32_t)(box_c0 + v)) ^ swz) << 4), o[4 * v],
+                         o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+          fence_proxy_async_smem();  // staged rows visible to the TMA store
+        } else if (i < t1) {
           uint4* dst = reinterpret_cast<uint4*>(orow);
 #pragma unroll
           for (int v = 0; v < 4; ++v)
             dst[v] = make_uint4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
         }
+        warp_arrive(bar(BAR_OST + box));
+        if (box_leader) {
+          ok = mbar_wait(bar(BAR_OST + box), qn & 1, a.ws) && ok;
+          if (lane == 0 && ok) {
+            if (whole) {
+              tma_store_2d(&tmo, sQ + qb * C::TILE + box * C::BLK, h * D + box * C::BOXW,
+                           s0 + t0);
+              bulk_commit_group();
+              bulk_wait_read_all();
+            }
+            mbar_arrive(bar(BAR_Q_EMPTY + qb));
+          }
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+        }
       }
-      tc_fence_before();
-      warp_arrive(bar(BAR_O_EMPTY));
       ++on;
+      ++qn;
       warp_arrive(bar(BAR_U_EMPTY + slot));
     }
+    // stores still in flight must complete before the CTA exits
+    if (box_leader && lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -494,11 +552,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int D>
 cudaError_t launch_d(const AttnArgs& a, cudaStream_t st) {
   using C = Cfg<D>;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   const int HD = a.H * D;
   if (!make_tma_2d(&mq, a.q, a.T, HD, a.q_rs, C::BOXW, kBM, C::SW == 128) ||
       !make_tma_2d(&mk, a.k, a.T, HD, a.k_rs, C::BOXW, kBN, C::SW == 128) ||
-      !make_tma_2d(&mv, a.v, a.T, HD, a.v_rs, C::BOXW, kBN, C::SW == 128))
+      !make_tma_2d(&mv, a.v, a.T, HD, a.v_rs, C::BOXW, kBN, C::SW == 128) ||
+      !make_tma_2d(&mo, a.out, a.T, HD, a.o_rs, C::BOXW, kBM, C::SW == 128))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -506,7 +565,7 @@ cudaError_t launch_d(const AttnArgs& a, cudaStream_t st) {
   const int64_t units = max_items(a.T, a.B) * a.H;
   const int sms = device_sm_count();
   const int grid = (int)(units < sms ? units : sms);
-  fwd_tc_kernel<D><<<grid, kThreads, C::SMEM, st>>>(mq, mk, mv, a);
+  fwd_tc_kernel<D><<<grid, kThreads, C::SMEM, st>>>(mq, mk, mv, mo, a);
   return cudaGetLastError();
 }
 
