@@ -404,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int half = chunk & 1;            // column half within the group
     const int row = quarter * 32 + lane;   // row of the 128-row tile
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-    const float half_alpha = 0.5f * a.alpha;
+    const uint64_t half_alpha2 = f2s(0.5f * a.alpha);
     const bool has_o = chunk < D / 32;     // this warp writes an O chunk
     // Epilogue store: a tile that lies inside its sequence is staged as bf16
     // in the unit's Q buffer (no S MMA reads it any more) in the swizzled
@@ -464,8 +464,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t p[16];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            p[e] = silu_pair(c0[2 * e], c0[2 * e + 1], half_alpha);
-            p[8 + e] = silu_pair(c1[2 * e], c1[2 * e + 1], half_alpha);
+            p[e] = silu_pair(c0[2 * e], c0[2 * e + 1], half_alpha2);
+            p[8 + e] = silu_pair(c1[2 * e], c1[2 * e + 1], half_alpha2);
           }
           if (!full) {
             const uint32_t bits = row_mask_bits(m, j0 + col);

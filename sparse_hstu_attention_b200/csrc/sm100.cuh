@@ -310,24 +310,57 @@ __device__ __forceinline__ float tanh_approx(float x) {
   return y;
 }
 
-// Backward pointwise for two scores s (raw fp32 bits) and their dP: packed
-// bf16 P = SiLU(alpha s) and dS = dP SiLU'(alpha s), with h = alpha s / 2,
-// t = tanh(h): SiLU = h + h t and SiLU' = (1 + t)/2 (1 + h - h t).
+// Packed fp32 pairs (one 64-bit register, low half first) and the sm_100
+// paired FMA-pipe instructions: one issue slot for two lanes of arithmetic.
+__device__ __forceinline__ uint64_t f2(uint32_t lo_bits, uint32_t hi_bits) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo_bits), "r"(hi_bits));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2s(float v) { return f2(__float_as_uint(v), __float_as_uint(v)); }
+__device__ __forceinline__ float f2_lo(uint64_t v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float f2_hi(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_tanh(uint64_t h) {
+  return f2(__float_as_uint(tanh_approx(f2_lo(h))), __float_as_uint(tanh_approx(f2_hi(h))));
+}
+__device__ __forceinline__ uint32_t f2_bf16(uint64_t v) { return pack_bf16x2(f2_lo(v), f2_hi(v)); }
+
+// Backward pointwise for two scores s (raw fp32 bits) and their dP, with
+// h = alpha s / 2, t = tanh(h) and u = 1 + t:
+//   P = SiLU(alpha s) = h u,   SiLU'(alpha s) = (u / 2) (1 + 2h - P),
+// returning packed bf16 P and dS2 = dP u (1 + 2h - P) = 2 dP SiLU'(alpha s)
+// (the factor 1/2 is applied with alpha / N when dS is consumed).
 __device__ __forceinline__ void bwd_pair(uint32_t s0, uint32_t s1, uint32_t d0, uint32_t d1,
-                                         float half_alpha, uint32_t& p2, uint32_t& ds2) {
-  const float h0 = __uint_as_float(s0) * half_alpha, h1 = __uint_as_float(s1) * half_alpha;
-  const float t0 = tanh_approx(h0), t1 = tanh_approx(h1);
-  const float g0 = fmaf(0.5f, t0, 0.5f) * (1.f + fmaf(-h0, t0, h0));
-  const float g1 = fmaf(0.5f, t1, 0.5f) * (1.f + fmaf(-h1, t1, h1));
-  p2 = pack_bf16x2(fmaf(h0, t0, h0), fmaf(h1, t1, h1));
-  ds2 = pack_bf16x2(__uint_as_float(d0) * g0, __uint_as_float(d1) * g1);
+                                         uint64_t half_alpha2, uint32_t& p2, uint32_t& ds2) {
+  const uint64_t h = f2_mul(f2(s0, s1), half_alpha2);
+  const uint64_t u = f2_add(f2_tanh(h), f2s(1.f));
+  const uint64_t p = f2_mul(h, u);
+  const uint64_t w = f2_fma(p, f2s(-1.f), f2_fma(h, f2s(2.f), f2s(1.f)));  // 1 + 2h - P
+  const uint64_t ds = f2_mul(f2(d0, d1), f2_mul(u, w));
+  p2 = f2_bf16(p);
+  ds2 = f2_bf16(ds);
 }
 
 // SiLU of two fp32 scores (raw bits) packed as bf16x2, with h = alpha s / 2:
 // SiLU(alpha s) = h + h tanh(h).
-__device__ __forceinline__ uint32_t silu_pair(uint32_t s0, uint32_t s1, float half_alpha) {
-  const float h0 = __uint_as_float(s0) * half_alpha, h1 = __uint_as_float(s1) * half_alpha;
-  return pack_bf16x2(fmaf(h0, tanh_approx(h0), h0), fmaf(h1, tanh_approx(h1), h1));
+__device__ __forceinline__ uint32_t silu_pair(uint32_t s0, uint32_t s1, uint64_t half_alpha2) {
+  const uint64_t h = f2_mul(f2(s0, s1), half_alpha2);
+  return f2_bf16(f2_fma(h, f2_tanh(h), h));
 }
 
 }  // namespace sm100
