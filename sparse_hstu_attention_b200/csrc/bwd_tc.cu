@@ -49,12 +49,15 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kRes = 128, kStr = 64, kStages = 4, kPwWarps = 16, kUSlots = 4, kPwWarp0 = 2;
+constexpr int kRes = 128, kStr = 64, kMaxSt = 4, kPwWarps = 16, kUSlots = 4, kPwWarp0 = 2;
 constexpr int kThreads = 32 * (kPwWarp0 + kPwWarps);
 constexpr uint32_t kColX1 = 0, kColX2 = 128, kColAcc1 = 256, kColAcc2 = 384, kTmemCols = 512;
 
 template <int D>
 struct BCfg {
+  // Streamed-tile ring depth (a slot is freed by a commit after the
+  // accumulating MMAs of its step).
+  static constexpr int kSt = D == 128 ? 3 : 4;
   static constexpr int SW = D >= 64 ? 128 : 64;
   static constexpr int BOXW = SW / 2;
   static constexpr int NB = D / BOXW;      // boxes per tile row
@@ -62,12 +65,13 @@ struct BCfg {
   static constexpr int STILE = kStr * D * 2;
   static constexpr int RBLK = kRes * SW;
   static constexpr int SBLK = kStr * SW;
-  static constexpr int OFF_A1 = 0;
-  static constexpr int OFF_A2 = RTILE;
-  static constexpr int OFF_B1 = 2 * RTILE;
-  static constexpr int OFF_B2 = 2 * RTILE + kStages * STILE;
-  static constexpr int OFF_ST = 2 * RTILE + 2 * kStages * STILE;  // epilogue staging tile
-  static constexpr int OFF_BAR = OFF_ST + RTILE;
+  // Two resident buffers (tiles A1, A2 each), so the next unit's resident
+  // tiles load while the current unit runs; a finished unit's buffer also
+  // stages its epilogue (ACC1 over A1, ACC2 over A2) for the TMA stores.
+  static constexpr int ABUF = 2 * RTILE;
+  static constexpr int OFF_B1 = 2 * ABUF;
+  static constexpr int OFF_B2 = OFF_B1 + kSt * STILE;
+  static constexpr int OFF_BAR = OFF_B2 + kSt * STILE;
   static constexpr int OFF_UNIT = OFF_BAR + 512;
   static constexpr int OFF_SLOT = OFF_UNIT + kUSlots * (int)sizeof(UnitRec);
   static constexpr int SMEM = OFF_SLOT + 16 + 1024;
@@ -79,10 +83,11 @@ struct BCfg {
 };
 
 enum {
-  B_A_FULL = 0, B_A_EMPTY, B_B_FULL, B_B_EMPTY = B_B_FULL + kStages,
-  B_X_FULL = B_B_EMPTY + kStages, B_OP_FULL = B_X_FULL + 2, B_ACC_FULL = B_OP_FULL + 2,
-  B_ACC_EMPTY, B_U_FULL, B_U_EMPTY = B_U_FULL + kUSlots, B_DRAIN = B_U_EMPTY + kUSlots,
-  B_OST, B_SFREE = B_OST + 2, B_COUNT = B_SFREE + 2
+  B_A_FULL = 0, B_A_EMPTY = 2, B_B_FULL = 4, B_B_EMPTY = B_B_FULL + kMaxSt,
+  B_X_FULL = B_B_EMPTY + kMaxSt,
+  B_OP_FULL = B_X_FULL + 2, B_ACC_FULL = B_OP_FULL + 2, B_ACC_EMPTY, B_U_FULL,
+  B_U_EMPTY = B_U_FULL + kUSlots, B_DRAIN = B_U_EMPTY + kUSlots, B_OST,  // OST: accumulator x box
+  B_COUNT = B_OST + 4
 };
 static_assert(8 * B_COUNT <= 512, "barrier area");
 
@@ -112,12 +117,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                   const __grid_constant__ CUtensorMap tmo1, const __grid_constant__ CUtensorMap tmo2,
                   const AttnArgs a) {
   using C = BCfg<D>;
+  constexpr int kSt = C::kSt;
+  constexpr int kNacc = KV ? 2 : 1;  // accumulators: dV, dK or dQ
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* base_ptr = smem_raw + (base - raw);
-  const uint32_t sA1 = base + C::OFF_A1, sA2 = base + C::OFF_A2;
-  const uint32_t sB1 = base + C::OFF_B1, sB2 = base + C::OFF_B2, sST = base + C::OFF_ST;
+  const uint32_t sA = base;  // resident buffer ab: A1 at sA + ab * ABUF, A2 RTILE further
+  const uint32_t sB1 = base + C::OFF_B1, sB2 = base + C::OFF_B2;
   const uint32_t bar0 = base + C::OFF_BAR;
   auto bar = [&](int i) { return bar0 + 8u * i; };
   UnitRec* ring = reinterpret_cast<UnitRec*>(base_ptr + C::OFF_UNIT);
@@ -130,9 +137,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   int* sched = KV ? &a.ws->sched2 : &a.ws->sched;
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(B_A_FULL), 1);
-    mbar_init(bar(B_A_EMPTY), 1);
-    for (int s = 0; s < kStages; ++s) {
+    for (int ab = 0; ab < 2; ++ab) {
+      mbar_init(bar(B_A_FULL + ab), 1);
+      mbar_init(bar(B_A_EMPTY + ab), 1 + C::NB);  // last X commit + one per box stored
+    }
+    for (int s = 0; s < kSt; ++s) {
       mbar_init(bar(B_B_FULL + s), 1);
       mbar_init(bar(B_B_EMPTY + s), 1);
     }
@@ -147,10 +156,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(B_U_EMPTY + s), 1 + kPwWarps);  // MMA lane + pointwise warps
     }
     mbar_init(bar(B_DRAIN), 1);
-    for (int b = 0; b < C::NB; ++b) {
-      mbar_init(bar(B_OST + b), 4 * (C::BOXW / 32));  // warps staging one box
-      mbar_init(bar(B_SFREE + b), 1);
-    }
+    for (int w = 0; w < kNacc; ++w)
+      for (int b = 0; b < C::NB; ++b)
+        mbar_init(bar(B_OST + 2 * w + b), 4 * (C::BOXW / 32));  // warps staging one box
     fence_barrier_init();
     prefetch_tmap(&tma1);
     prefetch_tmap(&tma2);
@@ -189,21 +197,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (nt < 0) break;
       if (nt == 0) continue;
       const int h = r->h, s0 = r->s0;
-      ok = warp_wait(bar(B_A_EMPTY), (an & 1) ^ 1, a.ws);
+      // resident buffer an % 2: free once the unit two back is done with it
+      const uint32_t ab = an & 1;
+      ok = warp_wait(bar(B_A_EMPTY + ab), ((an >> 1) & 1) ^ 1, a.ws);
       if (!ok) break;
       if (lane == 0) {
-        mbar_expect_tx(bar(B_A_FULL), 2 * C::RTILE);
+        const uint32_t a1 = sA + ab * C::ABUF, fb = bar(B_A_FULL + ab);
+        mbar_expect_tx(fb, 2 * C::RTILE);
         for (int b = 0; b < C::NB; ++b) {
-          tma_load_2d(sA1 + b * C::RBLK, &tma1, bar(B_A_FULL), h * D + b * C::BOXW, s0 + r->t0);
-          tma_load_2d(sA2 + b * C::RBLK, &tma2, bar(B_A_FULL), h * D + b * C::BOXW, s0 + r->t0);
+          tma_load_2d(a1 + b * C::RBLK, &tma1, fb, h * D + b * C::BOXW, s0 + r->t0);
+          tma_load_2d(a1 + C::RTILE + b * C::RBLK, &tma2, fb, h * D + b * C::BOXW, s0 + r->t0);
         }
       }
       ++an;
       SpanCursor c;
       c.begin(r);
       for (int n = 0; n < nt && ok; ++n, c.next(r)) {
-        const int s = bn % kStages;
-        ok = warp_wait(bar(B_B_EMPTY + s), ((bn / kStages) & 1) ^ 1, a.ws);
+        const int s = bn % kSt;
+        ok = warp_wait(bar(B_B_EMPTY + s), ((bn / kSt) & 1) ^ 1, a.ws);
         if (!ok) break;
         if (lane == 0) {
           mbar_expect_tx(bar(B_B_FULL + s), 2 * C::STILE);
@@ -219,9 +230,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     if (lane == 0 && load_status(a.ws) != 0) {  // drain copies in flight before exiting
-      if (an > 0) drain_wait(bar(B_A_FULL), (an - 1) & 1);
-      for (int s = 0; s < kStages; ++s) {
-        const uint32_t armed = bn / kStages + (s < (int)(bn % kStages) ? 1u : 0u);
+      for (uint32_t ab = 0; ab < 2; ++ab) {
+        const uint32_t armed = an / 2 + (ab < (an & 1) ? 1u : 0u);
+        if (armed > 0) drain_wait(bar(B_A_FULL + ab), (armed - 1) & 1);
+      }
+      for (int s = 0; s < kSt; ++s) {
+        const uint32_t armed = bn / kSt + (s < (int)(bn % kSt) ? 1u : 0u);
         if (armed > 0) drain_wait(bar(B_B_FULL + s), (armed - 1) & 1);
       }
     }
@@ -236,8 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t an = 0, bn = 0, xc = 0, accn = 0;
       bool ok = true;
       // Descriptor bases; offsets only add to the start-address field.
-      const uint64_t dA1 = smem_desc(sA1, 16, C::SBO, C::SWZ);
-      const uint64_t dA2 = smem_desc(sA2, 16, C::SBO, C::SWZ);
+      const uint64_t dA = smem_desc(sA, 16, C::SBO, C::SWZ);
       const uint64_t dB1 = smem_desc(sB1, 16, C::SBO, C::SWZ);
       const uint64_t dB2 = smem_desc(sB2, 16, C::SBO, C::SWZ);
       const uint64_t mB1 = smem_desc(sB1, C::SBLK, C::SBO, C::SWZ);  // MN-major views
@@ -251,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(bar(B_OP_FULL + b), (xm >> 1) & 1, a.ws)) return false;
         if (first && !mbar_wait(bar(B_ACC_EMPTY), (accn & 1) ^ 1, a.ws)) return false;
         tc_fence_after();
-        const int s = bm % kStages;
+        const int s = bm % kSt;
         const uint32_t so = (uint32_t)(s * C::STILE) >> 4;
 #pragma unroll
         for (int ks = 0; ks < kStr / 16; ++ks) {
@@ -276,13 +289,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(bar(B_U_EMPTY + slot));
         if (nt < 0) break;
         if (nt == 0) continue;
-        ok = mbar_wait(bar(B_A_FULL), an & 1, a.ws);
+        const uint32_t ab = an & 1;
+        ok = mbar_wait(bar(B_A_FULL + ab), (an >> 1) & 1, a.ws);
         if (!ok) break;
         tc_fence_after();
+        const uint64_t dA1 = dA + ((ab * C::ABUF) >> 4), dA2 = dA1 + (C::RTILE >> 4);
         const uint32_t bn0 = bn, xc0 = xc;
         for (int n = 0; n < nt; ++n) {
-          const int s = bn % kStages;
-          ok = mbar_wait(bar(B_B_FULL + s), (bn / kStages) & 1, a.ws);
+          const int s = bn % kSt;
+          ok = mbar_wait(bar(B_B_FULL + s), (bn / kSt) & 1, a.ws);
           if (!ok) break;
           tc_fence_after();
           const uint32_t b = xc & 1;
@@ -295,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                    C::IDESC_X, ks > 0 ? 1u : 0u);
           }
           tc_commit(bar(B_X_FULL + b));
-          if (n + 1 == nt) tc_commit(bar(B_A_EMPTY));  // last use of the resident tiles
+          if (n + 1 == nt) tc_commit(bar(B_A_EMPTY + ab));  // last use of the resident tiles
           if (n > 0) {
             ok = acc(bn - 1, xc - 1, n == 1);
             if (!ok) break;
@@ -342,7 +357,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int box_c0 = ((chunk * 32) % C::BOXW) / 8;
     const bool box_leader = has_acc && quarter == 0 && (chunk * 32) % C::BOXW == 0;
     const uint32_t swz = C::SW == 128 ? (uint32_t)(row & 7) : (uint32_t)((row >> 1) & 3);
-    uint32_t xc = 0, accn = 0, ep = 0;
+    uint32_t xc = 0, accn = 0, an = 0;
+    // Box leaders: resident buffer whose epilogue stores were issued but not
+    // yet released.  The wait for the stores to read it is deferred past this
+    // warp's next step (the producer reuses the buffer only two units on).
+    int pend_ab = -1;
+    auto release = [&]() {
+      if (pend_ab >= 0) {
+        if (lane == 0) {
+          bulk_wait_read_all();
+          mbar_arrive(bar(B_A_EMPTY + pend_ab));
+        }
+        __syncwarp();
+        pend_ab = -1;
+      }
+    };
     bool ok = true;
     for (int kk = 0; ok; ++kk) {
       const int slot = kk % kUSlots;
@@ -416,6 +445,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_st_wait();
         tc_fence_before();
         warp_arrive(bar(B_OP_FULL + b));
+        release();
       }
       if (!ok) break;
       // ---------------------------------------------------------- epilogue
@@ -423,8 +453,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const bool whole = t1 - t0 == kRes;
+      // This unit's resident buffer: its last X MMA is complete (ACC_FULL
+      // follows it), and it is reloaded only after the stores below read it.
+      const uint32_t ab = an & 1;
 #pragma unroll 1
-      for (int which = 0; which < (KV ? 2 : 1); ++which) {
+      for (int which = 0; which < kNacc; ++which) {
         uint32_t o[16];
         if (has_acc) {
           uint32_t x0[16], x1[16];
@@ -440,50 +473,54 @@ __global__ void __launch_bounds__(kThreads, 1)
                 pack_bf16x2(__uint_as_float(x1[2 * e]) * sc, __uint_as_float(x1[2 * e + 1]) * sc);
           }
         }
-        if (which + 1 == (KV ? 2 : 1)) {
-          // every accumulator is in registers or stored: the next unit may start
+        if (which + 1 == kNacc) {
+          // every accumulator is in registers or staged: the next unit may start
           tc_fence_before();
           warp_arrive(bar(B_ACC_EMPTY));
           ++accn;
         }
         if (!has_acc) continue;
         if (whole) {
-          // the staging box is free once the previous store has read it
-          ok = warp_wait(bar(B_SFREE + box), (ep & 1) ^ 1, a.ws);
-          if (!ok) break;
-          const uint32_t rowaddr = sST + box * C::RBLK + row * C::SW;
+          const uint32_t rowaddr = sA + ab * C::ABUF + which * C::RTILE + box * C::RBLK + row * C::SW;
 #pragma unroll
           for (int q = 0; q < 4; ++q)
             st_shared_v4(rowaddr + ((((uint32_t)(box_c0 + q)) ^ swz) << 4), o[4 * q], o[4 * q + 1],
                          o[4 * q + 2], o[4 * q + 3]);
-          fence_proxy_async_smem();
+          fence_proxy_async_smem();  // staged rows visible to the TMA store
         } else if (rr < t1) {
           uint4* dst = reinterpret_cast<uint4*>(which ? o2 : o1);
 #pragma unroll
           for (int q = 0; q < 4; ++q)
             dst[q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
         }
-        warp_arrive(bar(B_OST + box));
-        if (box_leader) {
-          ok = mbar_wait(bar(B_OST + box), ep & 1, a.ws) && ok;
-          if (lane == 0 && ok) {
-            if (whole) {
-              tma_store_2d(which ? &tmo2 : &tmo1, sST + box * C::RBLK, h * D + box * C::BOXW,
-                           s0 + t0);
-              bulk_commit_group();
-              bulk_wait_read_all();
-            }
-            mbar_arrive(bar(B_SFREE + box));
-          }
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) break;
-        }
-        ++ep;
+        warp_arrive(bar(B_OST + 2 * which + box));
       }
-      if (!ok) break;
+      if (box_leader) {
+        // one thread per box stores each accumulator's box; the resident
+        // buffer is freed once the stores have read it
+        release();
+        for (int which = 0; which < kNacc; ++which) {
+          ok = mbar_wait(bar(B_OST + 2 * which + box), an & 1, a.ws) && ok;
+          if (lane == 0 && ok && whole) {
+            tma_store_2d(which ? &tmo2 : &tmo1, sA + ab * C::ABUF + which * C::RTILE + box * C::RBLK,
+                         h * D + box * C::BOXW, s0 + t0);
+            bulk_commit_group();
+          }
+        }
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        if (whole) {
+          pend_ab = (int)ab;
+        } else {
+          if (lane == 0) mbar_arrive(bar(B_A_EMPTY + ab));
+          __syncwarp();
+        }
+      }
+      ++an;
       warp_arrive(bar(B_U_EMPTY + slot));
     }
     // stores still in flight must complete before the CTA exits
+    if (ok) release();
     if (box_leader && lane == 0) bulk_wait_all();
   }
 
