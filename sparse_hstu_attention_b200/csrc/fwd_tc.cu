@@ -334,7 +334,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (mbar_test_wait(b, parity)) return true;
         const uint64_t t0 = globaltimer();
         for (uint32_t it = 1;; ++it) {
-          if (mbar_test_wait(b, parity)) return true;
+          // try_wait may suspend this lane in hardware until the phase
+          // completes, leaving the issue slots of its sub-partition to the
+          // pointwise warps there; deferred P V readiness is polled between
+          if (mbar_try_wait(b, parity)) return true;
           if (pvc != tc && pv_ready()) {
             pv_issue();
             continue;
@@ -415,7 +418,91 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int box_c0 = ((chunk * 32) % C::BOXW) / 8;  // its first 16-byte chunk in a box row
     const bool box_leader = has_o && quarter == 0 && (chunk * 32) % C::BOXW == 0;
     const uint32_t swz = C::SW == 128 ? (uint32_t)(row & 7) : (uint32_t)((row >> 1) & 3);
+    // A unit's epilogue is deferred until this warp has done its first key
+    // tile of the next unit (whose scores are ready by then), so the P of a
+    // unit's first tiles does not wait for the previous unit's last P V and
+    // epilogue.  The deferred unit keeps its ring slot until then.  Every
+    // epilogue and Q-buffer release completes before the warp waits on a
+    // tile of the unit after next, whose Q load depends on them.
     uint32_t tc = 0, on = 0, qn = 0;
+    bool ep_pend = false;
+    int e_h = 0, e_s0 = 0, e_t0 = 0, e_t1 = 0, e_slot = 0;
+    uint32_t e_qn = 0;
+    int rel_qb = -1;  // box leaders: Q buffer whose O stores are issued, not yet released
+    auto release = [&]() {
+      if (rel_qb >= 0) {
+        if (lane == 0) {
+          bulk_wait_read_all();
+          mbar_arrive(bar(BAR_Q_EMPTY + rel_qb));
+        }
+        __syncwarp();
+        rel_qb = -1;
+      }
+    };
+    auto epilogue = [&]() -> bool {
+      ep_pend = false;
+      if (!warp_wait(bar(BAR_O_FULL), on & 1, a.ws)) return false;
+      tc_fence_after();
+      const uint32_t qb = e_qn & 1;
+      const bool whole = e_t1 - e_t0 == kBM;
+      const int i = e_t0 + row;
+      uint32_t o[16];
+      if (has_o) {
+        uint32_t r0[16], r1[16];
+        tmem_ld16(lane_base + kColO + chunk * 32, r0);
+        tmem_ld16(lane_base + kColO + chunk * 32 + 16, r1);
+        tmem_ld_wait2(r0, r1);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          o[e] = pack_bf16x2(__uint_as_float(r0[2 * e]) * a.inv_n,
+                             __uint_as_float(r0[2 * e + 1]) * a.inv_n);
+          o[8 + e] = pack_bf16x2(__uint_as_float(r1[2 * e]) * a.inv_n,
+                                 __uint_as_float(r1[2 * e + 1]) * a.inv_n);
+        }
+      }
+      // O is in registers: the next unit's P V may overwrite it
+      tc_fence_before();
+      warp_arrive(bar(BAR_O_EMPTY));
+      ++on;
+      bool good = true;
+      if (has_o) {
+        if (whole) {
+          const uint32_t rowaddr = sQ + qb * C::TILE + box * C::BLK + row * C::SW;
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            st_shared_v4(rowaddr + ((((uint32_t)(box_c0 + v)) ^ swz) << 4), o[4 * v],
+                         o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+          fence_proxy_async_smem();  // staged rows visible to the TMA store
+        } else if (i < e_t1) {
+          uint4* dst = reinterpret_cast<uint4*>(a.out + (int64_t)(e_s0 + i) * a.o_rs + e_h * D +
+                                                chunk * 32);
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            dst[v] = make_uint4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+        }
+        warp_arrive(bar(BAR_OST + box));
+        if (box_leader) {
+          release();
+          good = mbar_wait(bar(BAR_OST + box), e_qn & 1, a.ws);
+          if (lane == 0 && good && whole) {
+            tma_store_2d(&tmo, sQ + qb * C::TILE + box * C::BLK, e_h * D + box * C::BOXW,
+                         e_s0 + e_t0);
+            bulk_commit_group();
+          }
+          good = __all_sync(0xffffffffu, good);
+          if (good) {
+            if (whole) {
+              rel_qb = (int)qb;  // released after this warp's next tile
+            } else {
+              if (lane == 0) mbar_arrive(bar(BAR_Q_EMPTY + qb));
+              __syncwarp();
+            }
+          }
+        }
+      }
+      warp_arrive(bar(BAR_U_EMPTY + e_slot));
+      return good;
+    };
     bool ok = true;
     for (int kk = 0; ok; ++kk) {
       const int slot = kk % kUSlots;
@@ -423,22 +510,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       const UnitRec* r = &ring[slot];
       const int nt = r->nsteps;
-      if (nt < 0) {
-        warp_arrive(bar(BAR_U_EMPTY + slot));
-        break;
-      }
-      const int h = r->h, s0 = r->s0, Lh = r->Lh, t0 = r->t0, t1 = r->t1;
-      const int i = t0 + row;  // row within the sequence
-      bf16* orow = a.out + (int64_t)(s0 + i) * a.o_rs + h * D + chunk * 32;
-      if (nt == 0) {  // no visible key anywhere in the tile
-        if (has_o && i < t1) {
+      if (nt <= 0) {
+        if (ep_pend) {
+          ok = epilogue();
+          if (!ok) break;
+        }
+        release();
+        if (nt < 0) {
+          warp_arrive(bar(BAR_U_EMPTY + slot));
+          break;
+        }
+        // no visible key anywhere in the tile
+        const int i = r->t0 + row;
+        if (has_o && i < r->t1) {
+          uint4* dst = reinterpret_cast<uint4*>(a.out + (int64_t)(r->s0 + i) * a.o_rs +
+                                                r->h * D + chunk * 32);
           const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
-          for (int v = 0; v < 4; ++v) reinterpret_cast<uint4*>(orow)[v] = z;
+          for (int v = 0; v < 4; ++v) dst[v] = z;
         }
         warp_arrive(bar(BAR_U_EMPTY + slot));
         continue;
       }
+      const int h = r->h, s0 = r->s0, Lh = r->Lh, t0 = r->t0, t1 = r->t1;
+      const int i = t0 + row;  // row within the sequence
       const RowMask m = row_mask(i, r->L, Lh, a.K1, a.K2e);
       SpanCursor c;
       c.begin(r);
@@ -477,64 +572,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_st_wait();
         tc_fence_before();
         warp_arrive(bar(BAR_P_FULL + b));
-      }
-      if (!ok) break;
-      // epilogue
-      ok = warp_wait(bar(BAR_O_FULL), on & 1, a.ws);
-      if (!ok) break;
-      tc_fence_after();
-      const uint32_t qb = qn & 1;
-      const bool whole = t1 - t0 == kBM;
-      uint32_t o[16];
-      if (has_o) {
-        uint32_t r0[16], r1[16];
-        tmem_ld16(lane_base + kColO + chunk * 32, r0);
-        tmem_ld16(lane_base + kColO + chunk * 32 + 16, r1);
-        tmem_ld_wait2(r0, r1);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          o[e] = pack_bf16x2(__uint_as_float(r0[2 * e]) * a.inv_n,
-                             __uint_as_float(r0[2 * e + 1]) * a.inv_n);
-          o[8 + e] = pack_bf16x2(__uint_as_float(r1[2 * e]) * a.inv_n,
-                                 __uint_as_float(r1[2 * e + 1]) * a.inv_n);
-        }
-      }
-      // O is in registers: the next unit's P V may overwrite it
-      tc_fence_before();
-      warp_arrive(bar(BAR_O_EMPTY));
-      if (has_o) {
-        if (whole) {
-          const uint32_t rowaddr = sQ + qb * C::TILE + box * C::BLK + row * C::SW;
-#pragma unroll
-          for (int v = 0; v < 4; ++v)
-            st_shared_v4(rowaddr + ((((uint32_t)(box_c0 + v)) ^ swz) << 4), o[4 * v],
-                         o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
-          fence_proxy_async_smem();  // staged rows visible to the TMA store
-        } else if (i < t1) {
-          uint4* dst = reinterpret_cast<uint4*>(orow);
-#pragma unroll
-          for (int v = 0; v < 4; ++v)
-            dst[v] = make_uint4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
-        }
-        warp_arrive(bar(BAR_OST + box));
-        if (box_leader) {
-          ok = mbar_wait(bar(BAR_OST + box), qn & 1, a.ws) && ok;
-          if (lane == 0 && ok) {
-            if (whole) {
-              tma_store_2d(&tmo, sQ + qb * C::TILE + box * C::BLK, h * D + box * C::BOXW,
-                           s0 + t0);
-              bulk_commit_group();
-              bulk_wait_read_all();
-            }
-            mbar_arrive(bar(BAR_Q_EMPTY + qb));
-          }
-          ok = __all_sync(0xffffffffu, ok);
+        if (ep_pend) {
+          ok = epilogue();
           if (!ok) break;
+        } else {
+          release();
         }
       }
-      ++on;
+      if (!ok) break;
+      if (ep_pend) {  // no tile of this unit for this warp's group
+        ok = epilogue();
+        if (!ok) break;
+      }
+      release();
+      ep_pend = true;
+      e_h = h; e_s0 = s0; e_t0 = t0; e_t1 = t1; e_slot = slot; e_qn = qn;
       ++qn;
-      warp_arrive(bar(BAR_U_EMPTY + slot));
     }
     // stores still in flight must complete before the CTA exits
     if (box_leader && lane == 0) bulk_wait_all();
