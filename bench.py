@@ -37,8 +37,10 @@ from workloads import WORKLOADS, make_batch  # noqa: E402
 
 METRIC = "SLA HSTU attn fwd+bwd TFLOP/s (unmasked pairs), % of B200 BF16 peak"
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0}
-KERNEL_SOURCES = {"fwd": "sparse_hstu_attention_b200/csrc/fwd_tc.cu",
-                  "bwd": "sparse_hstu_attention_b200/csrc/bwd_tc.cu"}
+# sources a kernel's device code is compiled from (its .cu and the shared headers)
+_HDRS = ("sparse_hstu_attention_b200/csrc/sm100.cuh", "sparse_hstu_attention_b200/csrc/sla_common.cuh")
+KERNEL_SOURCES = {"fwd": ("sparse_hstu_attention_b200/csrc/fwd_tc.cu",) + _HDRS,
+                  "bwd": ("sparse_hstu_attention_b200/csrc/bwd_tc.cu",) + _HDRS}
 KERNEL_NAMES = {"fwd": "fwd_tc_kernel", "bwd": "bwd_tc_kernel (KV pass + Q pass)"}
 LAUNCHES_PER_STEP = {"fwd": 2, "bwd": 4}  # work list(s) + attention kernel(s)
 
@@ -52,12 +54,16 @@ def _peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def _sha1(path):
-    p = os.path.join(ROOT, path)
-    if not os.path.exists(p):
-        return None
-    with open(p, "rb") as f:
-        return hashlib.sha1(f.read()).hexdigest()
+def _sha1(paths):
+    """SHA-1 over the concatenated contents of `paths` (None if one is missing)."""
+    h = hashlib.sha1()
+    for path in paths:
+        p = os.path.join(ROOT, path)
+        if not os.path.exists(p):
+            return None
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
 
 
 def _traffic(which, workload):
@@ -75,7 +81,7 @@ def _traffic(which, workload):
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms while active."""
+    """nvidia-smi clocks / throttle reasons sampled every 50 ms while active."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -90,7 +96,7 @@ class ClockSampler:
             self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200", "-i", str(self.dev)], stdout=self.file,
+                 "-lms", "50", "-i", str(self.dev)], stdout=self.file,
                 stderr=subprocess.DEVNULL)
             time.sleep(0.3)
         except (OSError, FileNotFoundError):
@@ -175,8 +181,15 @@ def cpu_baseline(batch, target_s=15.0):
     """The oracle, as it stands, on a bounded random sample of the workload's tokens."""
     w = batch.workload
     rp, kp = _pair_tables(batch)
-    n = 64
-    t, _ = _oracle_sample(batch, n, seed=7)
+    # The oracle runs its loops on all host cores, so a small sample costs
+    # more per token than a large one: grow the sample geometrically until a
+    # run takes a second or more, then scale it to the target time.
+    n, t = 64, 0.0
+    while n < batch.T:
+        t, _ = _oracle_sample(batch, n, seed=7)
+        if t >= 1.0:
+            break
+        n = min(batch.T, n * 4)
     n = int(min(batch.T, max(64, n * target_s / max(t, 1e-3))))
     t, rows = _oracle_sample(batch, n, seed=8)
     fl, _ = _sample_cost_flops(None, rows, w.d, w.H, rp, kp)
@@ -234,7 +247,7 @@ def _config(w, batch):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="hist16k", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
