@@ -1,7 +1,7 @@
 // Host-side check of the library's tile enumeration (sla_common.cuh), built
 // and run on the CPU by tests/test_enumeration_host.py.  For random sequence
-// geometries it brute-forces the mask predicate and verifies, for both tile
-// sizes the kernels use, that
+// geometries it brute-forces the mask predicate and verifies, for every tile
+// shape the kernels use (256-row units on CTA pairs included), that
 //   - every visible (row, key) pair lies in an enumerated (query tile, key tile)
 //     pair, from the query side (forward) and from the key side (backward);
 //   - no enumerated (query tile, key tile) pair is empty, from either side;
@@ -89,7 +89,7 @@ int main(int argc, char** argv) {
   int n = argc > 1 ? atoi(argv[1]) : 3000;
   std::mt19937 rng(12345);
   int cases = 0;
-  const int tiles[][2] = {{64, 64}, {128, 128}, {128, 64}, {64, 128}};
+  const int tiles[][2] = {{64, 64}, {128, 128}, {128, 64}, {64, 128}, {256, 64}, {64, 256}};
   for (int c = 0; c < n; ++c) {
     int L = 1 + rng() % 700;
     if (rng() % 6 == 0) L = 64 * (1 + rng() % 8) + (rng() % 2 ? 1 : 0);
