@@ -39,10 +39,15 @@ METRIC = "SLA HSTU attn fwd+bwd TFLOP/s (unmasked pairs), % of B200 BF16 peak"
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0}
 # sources a kernel's device code is compiled from (its .cu and the shared headers)
 _HDRS = ("sparse_hstu_attention_b200/csrc/sm100.cuh", "sparse_hstu_attention_b200/csrc/sla_common.cuh")
+# (head_dim 128 kernels: the workloads this bench times all have d = 128)
 KERNEL_SOURCES = {"fwd": ("sparse_hstu_attention_b200/csrc/fwd_tc.cu",) + _HDRS,
-                  "bwd": ("sparse_hstu_attention_b200/csrc/bwd_tc.cu",) + _HDRS}
-KERNEL_NAMES = {"fwd": "fwd_tc_kernel", "bwd": "bwd_tc_kernel (KV pass + Q pass)"}
-LAUNCHES_PER_STEP = {"fwd": 2, "bwd": 4}  # work list(s) + attention kernel(s)
+                  "bwd": ("sparse_hstu_attention_b200/csrc/bwd_fused.cu",) + _HDRS}
+KERNEL_NAMES = {"fwd": "fwd_tc_kernel",
+                "bwd": "bwd_kvq_kernel (one pass, dQ via fp32 workspace) + dq_convert_kernel"}
+# kernels of this library per call: forward = work list + attention; backward
+# (d = 128) = work list + one-pass kernel + dq conversion (the workspace
+# zeroing is a cudaMemsetAsync, not counted)
+LAUNCHES_PER_STEP = {"fwd": 2, "bwd": 3}
 
 
 def _peaks():

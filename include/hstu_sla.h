@@ -109,8 +109,10 @@ typedef struct {
 /* Bytes of device workspace hstu_sla_fwd (which = HSTU_SLA_WS_FWD) or
  * hstu_sla_bwd (HSTU_SLA_WS_BWD) needs for a batch of total_tokens tokens in
  * B sequences: a status word and the device-built work lists, about
- * 16 * (total_tokens / 64 + B) bytes (H and d do not change it).  The
- * workspace must be 256-byte aligned.  Returns 0 on invalid arguments. */
+ * 16 * (total_tokens / 64 + B) bytes, plus, for the backward at d = 128, an
+ * fp32 dQ accumulator of total_tokens * H * d * 4 bytes.  The workspace must
+ * be 256-byte aligned; its contents need not be initialised.  Returns 0 on
+ * invalid arguments. */
 size_t hstu_sla_workspace_bytes(int which, int64_t total_tokens, int32_t B, int32_t H,
                                 int32_t d);
 
@@ -120,9 +122,16 @@ size_t hstu_sla_workspace_bytes(int which, int64_t total_tokens, int32_t B, int3
 int hstu_sla_fwd(const hstu_sla_fwd_params* p, void* workspace, size_t workspace_bytes,
                  hstu_stream_t stream);
 
-/* Backward: writes p->dq, p->dk, p->dv (bf16).  Two passes, no atomics, a
- * deterministic result: a key-tile pass accumulates dk/dv on chip, a
- * query-tile pass recomputes the scores and accumulates dq on chip. */
+/* Backward: writes p->dq, p->dk, p->dv (bf16).  No atomics on dk/dv: each
+ * key tile's dk/dv rows are accumulated on chip by one CTA.
+ *  d = 128: one pass over key tiles.  Each (key tile, query tile) step also
+ *           forms its dQ contribution on the tensor cores and adds it to the
+ *           workspace's fp32 accumulator with fp32 atomic additions; a final
+ *           kernel converts it to bf16 dq.  dk/dv are bitwise reproducible;
+ *           dq is reproducible up to the order of fp32 additions.
+ *  d = 32, 64: two passes, no atomics at all, bitwise reproducible: a
+ *           key-tile pass for dk/dv and a query-tile pass that recomputes the
+ *           scores for dq. */
 int hstu_sla_bwd(const hstu_sla_bwd_params* p, void* workspace, size_t workspace_bytes,
                  hstu_stream_t stream);
 

@@ -81,7 +81,8 @@ extern "C" {
 size_t hstu_sla_workspace_bytes(int which, int64_t total_tokens, int32_t B, int32_t H,
                                 int32_t d) {
   if (total_tokens < 0 || B < 1 || H < 1 || d < 1) return 0;
-  if (which == HSTU_SLA_WS_FWD || which == HSTU_SLA_WS_BWD) return ws_bytes(total_tokens, B);
+  if (which == HSTU_SLA_WS_FWD) return ws_bytes(total_tokens, B);
+  if (which == HSTU_SLA_WS_BWD) return ws_bwd_bytes(total_tokens, B, H, d);
   return 0;
 }
 
@@ -97,7 +98,7 @@ int hstu_sla_fwd(const hstu_sla_fwd_params* p, void* workspace, size_t workspace
   AttnArgs a = make_args(p, workspace);
   a.out = static_cast<bf16*>(p->out);
   a.o_rs = p->out_row_stride;
-  cudaError_t ce = launch_worklist(a, kFwdBM, 0, st);
+  cudaError_t ce = launch_worklist(a, kFwdBM, 0, true, st);
   if (ce == cudaSuccess) ce = record(p->event_begin, st);
   if (ce == cudaSuccess) ce = launch_fwd_tc(a, p->d, st);
   if (ce == cudaSuccess) ce = record(p->event_end, st);
@@ -127,12 +128,23 @@ int hstu_sla_bwd(const hstu_sla_bwd_params* p, void* workspace, size_t workspace
   a.dq_rs = p->dq_row_stride;
   a.dk_rs = p->dk_row_stride;
   a.dv_rs = p->dv_row_stride;
-  cudaError_t ce = launch_worklist(a, kQpBM, 0, st);
-  if (ce == cudaSuccess) ce = launch_worklist(a, kKvBN, 1, st);
-  if (ce == cudaSuccess) ce = record(f->event_begin, st);
-  if (ce == cudaSuccess) ce = launch_bwd_tc(a, f->d, /*kv_pass=*/true, st);
-  if (ce == cudaSuccess) ce = launch_bwd_tc(a, f->d, /*kv_pass=*/false, st);
-  if (ce == cudaSuccess) ce = record(f->event_end, st);
+  cudaError_t ce;
+  if (f->d == kFusedBwdD) {
+    // one pass over key tiles; dQ through the fp32 workspace after the lists
+    a.dqacc = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                       ws_bytes(f->total_tokens, f->B));
+    ce = launch_worklist(a, kKvBN, 1, true, st);
+    if (ce == cudaSuccess) ce = record(f->event_begin, st);
+    if (ce == cudaSuccess) ce = launch_bwd_fused(a, st);
+    if (ce == cudaSuccess) ce = record(f->event_end, st);
+  } else {
+    ce = launch_worklist(a, kQpBM, 0, true, st);
+    if (ce == cudaSuccess) ce = launch_worklist(a, kKvBN, 1, false, st);
+    if (ce == cudaSuccess) ce = record(f->event_begin, st);
+    if (ce == cudaSuccess) ce = launch_bwd_tc(a, f->d, /*kv_pass=*/true, st);
+    if (ce == cudaSuccess) ce = launch_bwd_tc(a, f->d, /*kv_pass=*/false, st);
+    if (ce == cudaSuccess) ce = record(f->event_end, st);
+  }
   return cuda_status(ce);
 }
 
@@ -145,7 +157,7 @@ int hstu_sla_count_pairs(const hstu_sla_fwd_params* p, int64_t* row_counts, int6
     return e;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   AttnArgs a = make_args(p, workspace);
-  cudaError_t ce = launch_worklist(a, kFwdBM, 0, st);
+  cudaError_t ce = launch_worklist(a, kFwdBM, 0, true, st);
   if (ce == cudaSuccess)
     ce = launch_count_pairs(a, kFwdBM, kFwdBN, kKvBM, kKvBN, row_counts, key_counts, st);
   return cuda_status(ce);

@@ -1,0 +1,570 @@
+// SLA HSTU attention backward for head_dim 128 in ONE pass over key tiles, on
+// the 5th-generation tensor cores (tcgen05 / TMEM / TMA).
+//
+// With x_ij = alpha q_i.k_j, P_ij = M SiLU(x)/N and dP_ij = dO_i.v_j:
+//   dV_j = sum_i P_ij dO_i,   dK_j = sum_i dS_ij q_i,   dQ_i = sum_j dS_ij k_j,
+//   dS_ij = M dP_ij SiLU'(x_ij) alpha/N
+// (the chain rule through "Bending the Scaling Law Curve in Large-Scale
+// Recommendation Systems", section 3, Eq. 3, under the SLA mask of section
+// 4.2.1, Eq. 7).
+//
+// A resident 128-key tile (K, V) meets streamed 64-row query tiles (Q, dO):
+//   S^T = K Q^T, dP^T = V dO^T            (tensor cores, fp32 in TMEM)
+//   P^T, dS^T                              (pointwise warps, bf16)
+//   dV += P^T dO, dK += dS^T Q            (TMEM accumulators: each key tile has
+//                                          one owner, so no atomics on dK, dV)
+//   dQ^T(step) = K^T dS^T                 (128 x 64 fp32 in TMEM)
+//   dQ workspace += dQ(step)               (fp32 reductions in L2, by the
+//                                          pointwise warps that drained it)
+// and a second kernel turns the fp32 dQ workspace into bf16 dq, applying
+// alpha / (2N).  Against a separate query-major pass that recomputes S and dP
+// this saves two of the seven tile contractions per (key tile, query tile)
+// pair; the price is the fp32 workspace and the order of the dQ additions,
+// which is not fixed (dq is reproducible to fp32 rounding, not bitwise).
+//
+// Roles (persistent CTAs, one per SM; units handed out by an atomic counter,
+// prefix-key units first):
+//   warp 0      scheduler + TMA producer (K double-buffered, V single,
+//               3-stage Q / dO ring)
+//   warp 1      TMEM allocation; one lane issues every UMMA and commit
+//   warps 2..17 pointwise, two groups of eight on alternate steps; then the
+//               dQ drain of their step; at the end of a unit, all sixteen
+//               store dK and dV
+// TMEM columns:
+//   X1(b) = [64b, 64b+64)       S^T (fp32); after the pointwise: per 32-column
+//                               chunk c, P^T bf16 in [32c, 32c+16) and dS^T
+//                               bf16 in [32c+16, 32c+32)
+//   X2(b) = [128+64b, 192+64b)  dP^T (fp32); then the step's dQ^T (lanes =
+//                               head-dim index, columns = query rows)
+//   ACC1 = [256, 384) dV,  ACC2 = [384, 512) dK
+// Shared memory (227 KB): K 2 x 32 KB, V 32 KB, Q and dO 3 x 16 KB each, dS^T
+// 2 x 16 KB (the B operand of the dQ MMA), barriers and the unit ring.
+#include <cudaTypedefs.h>
+
+#include "sm100.cuh"
+
+namespace hstu {
+
+bool make_tma_2d(CUtensorMap* m, const void* ptr, int64_t T, int HD, int64_t rs, int box_w,
+                 int box_h, bool sw128);
+int device_sm_count();
+
+namespace {
+
+using namespace sm100;
+
+constexpr int D = 128;
+constexpr int kRes = 128, kStr = 64, kSt = 3, kPwWarps = 16, kUSlots = 4, kPwWarp0 = 2;
+constexpr int kThreads = 32 * (kPwWarp0 + kPwWarps);
+constexpr uint32_t kColX1 = 0, kColX2 = 128, kColAcc1 = 256, kColAcc2 = 384, kTmemCols = 512;
+constexpr int SW = 128, BOXW = 64, NB = D / BOXW;
+constexpr int RTILE = kRes * D * 2;     // resident tile, two 64-column boxes
+constexpr int STILE = kStr * D * 2;     // streamed tile, two boxes
+constexpr int RBLK = kRes * SW;         // one box of a resident tile
+constexpr int SBLK = kStr * SW;         // one box of a streamed tile
+constexpr int DSTILE = kRes * kStr * 2;  // dS^T: [128 keys][64 rows] bf16, one box
+constexpr int OFF_K = 0;
+constexpr int OFF_V = OFF_K + 2 * RTILE;
+constexpr int OFF_B1 = OFF_V + RTILE;
+constexpr int OFF_B2 = OFF_B1 + kSt * STILE;
+constexpr int OFF_DS = OFF_B2 + kSt * STILE;
+constexpr int OFF_BAR = OFF_DS + 2 * DSTILE;
+constexpr int OFF_UNIT = OFF_BAR + 512;
+constexpr int OFF_SLOT = OFF_UNIT + kUSlots * (int)sizeof(UnitRec);
+constexpr int SMEM = OFF_SLOT + 16 + 1024;
+static_assert(SMEM <= 232448, "shared memory budget");
+constexpr uint32_t SBO = 8 * SW;
+// 128 x 64 scores, both operands K-major
+constexpr uint32_t IDESC_X = idesc_bf16(kRes, kStr, false, false);
+// 128 x 128 accumulators: A = P^T / dS^T from TMEM, B = dO / Q MN-major
+constexpr uint32_t IDESC_ACC = idesc_bf16(kRes, D, false, true);
+// 128 x 64 dQ^T: A = K^T and B = dS^T, both read MN-major from their tiles
+constexpr uint32_t IDESC_DQ = idesc_bf16(D, kStr, true, true);
+
+enum {
+  F_K_FULL = 0, F_K_EMPTY = 2, F_V_FULL = 4, F_V_EMPTY, F_B_FULL,
+  F_B_EMPTY = F_B_FULL + kSt, F_X_FULL = F_B_EMPTY + kSt, F_OP_FULL = F_X_FULL + 2,
+  F_DQ_FULL = F_OP_FULL + 2, F_DQ_EMPTY = F_DQ_FULL + 2, F_ACC_FULL = F_DQ_EMPTY + 2,
+  F_ACC_EMPTY, F_U_FULL, F_U_EMPTY = F_U_FULL + kUSlots, F_DRAIN = F_U_EMPTY + kUSlots,
+  F_COUNT
+};
+static_assert(8 * F_COUNT <= 512, "barrier area");
+
+// Unit u: key-tile work-list entry u / H, head u % H, and the query tiles
+// that see its keys.  u < 0 ends the schedule.
+__device__ void decode_kv_unit(const AttnArgs& a, int u, UnitRec* r) {
+  if (u < 0) {
+    r->nsteps = -1;
+    return;
+  }
+  const int idx = u / a.H;
+  const int h = u - idx * a.H;
+  const int2 it = a.items2[idx];
+  const SeqGeom g = seq_geom(a, it.x);
+  const int t0 = it.y * kRes;
+  const int t1 = imin(t0 + kRes, g.L);
+  unit_rec_fill(r, h, g.s0, g.L, g.Lh, t0, t1, k_tile_q_tiles(t0, t1, g.L, g.Lh, a.K1, a.K2e, kStr));
+}
+
+// Fire-and-forget fp32 addition in L2 (the result is unused, so this is a
+// reduction, not a round trip).
+__device__ __forceinline__ void red_add_f32(float* p, uint32_t v) { atomicAdd(p, __uint_as_float(v)); }
+
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_kvq_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+                   const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmdo,
+                   const AttnArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* base_ptr = smem_raw + (base - raw);
+  const uint32_t sK = base + OFF_K, sV = base + OFF_V, sB1 = base + OFF_B1, sB2 = base + OFF_B2;
+  const uint32_t sDS = base + OFF_DS;
+  const uint32_t bar0 = base + OFF_BAR;
+  auto bar = [&](int i) { return bar0 + 8u * i; };
+  UnitRec* ring = reinterpret_cast<UnitRec*>(base_ptr + OFF_UNIT);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + OFF_SLOT);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (load_status(a.ws) != 0) return;
+  const int total = a.ws->n_items2 * a.H;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(F_K_FULL + i), 1);
+      mbar_init(bar(F_K_EMPTY + i), 1);                // commit after the unit's last dQ MMA
+      mbar_init(bar(F_X_FULL + i), 1);
+      mbar_init(bar(F_OP_FULL + i), kPwWarps / 2);     // one arrive per warp of group i
+      mbar_init(bar(F_DQ_FULL + i), 1);
+      mbar_init(bar(F_DQ_EMPTY + i), kPwWarps / 2);
+    }
+    mbar_init(bar(F_V_FULL), 1);
+    mbar_init(bar(F_V_EMPTY), 1);                      // commit after the unit's last X MMA
+    for (int s = 0; s < kSt; ++s) {
+      mbar_init(bar(F_B_FULL + s), 1);
+      mbar_init(bar(F_B_EMPTY + s), 1);
+    }
+    mbar_init(bar(F_ACC_FULL), 1);
+    mbar_init(bar(F_ACC_EMPTY), kPwWarps);
+    for (int s = 0; s < kUSlots; ++s) {
+      mbar_init(bar(F_U_FULL + s), 1);
+      mbar_init(bar(F_U_EMPTY + s), 1 + kPwWarps);     // MMA lane + pointwise warps
+    }
+    mbar_init(bar(F_DRAIN), 1);
+    fence_barrier_init();
+    prefetch_tmap(&tmk);
+    prefetch_tmap(&tmv);
+    prefetch_tmap(&tmq);
+    prefetch_tmap(&tmdo);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------- scheduler + producer
+    // The whole warp walks the schedule (warp-uniform values); lane 0 takes
+    // units from the counter, decodes them, arms barriers and issues copies.
+    uint32_t kn = 0, vn = 0, bn = 0;  // K, V and streamed loads issued
+    bool ok = true;
+    for (int kk = 0; ok; ++kk) {
+      const int slot = kk % kUSlots;
+      ok = warp_wait(bar(F_U_EMPTY + slot), ((kk / kUSlots) & 1) ^ 1, a.ws);
+      if (!ok) break;
+      if (lane == 0) {
+        const int u = atomicAdd(&a.ws->sched2, 1);
+        decode_kv_unit(a, u < total ? u : -1, &ring[slot]);
+        mbar_arrive(bar(F_U_FULL + slot));
+      }
+      __syncwarp();
+      const UnitRec* r = &ring[slot];
+      const int nt = r->nsteps;
+      if (nt < 0) break;
+      if (nt == 0) continue;
+      const int h = r->h, y0 = r->s0 + r->t0;
+      // K buffer kn % 2: free once the unit two back issued its last dQ MMA
+      const uint32_t kb = kn & 1;
+      ok = warp_wait(bar(F_K_EMPTY + kb), ((kn >> 1) & 1) ^ 1, a.ws);
+      if (!ok) break;
+      if (lane == 0) {
+        const uint32_t fb = bar(F_K_FULL + kb);
+        mbar_expect_tx(fb, RTILE);
+        for (int b = 0; b < NB; ++b)
+          tma_load_2d(sK + kb * RTILE + b * RBLK, &tmk, fb, h * D + b * BOXW, y0);
+      }
+      ++kn;
+      // V: free once the previous unit's last score MMA is done
+      ok = warp_wait(bar(F_V_EMPTY), (vn & 1) ^ 1, a.ws);
+      if (!ok) break;
+      if (lane == 0) {
+        const uint32_t fb = bar(F_V_FULL);
+        mbar_expect_tx(fb, RTILE);
+        for (int b = 0; b < NB; ++b) tma_load_2d(sV + b * RBLK, &tmv, fb, h * D + b * BOXW, y0);
+      }
+      ++vn;
+      SpanCursor c;
+      c.begin(r);
+      for (int n = 0; n < nt && ok; ++n, c.next(r)) {
+        const int s = bn % kSt;
+        ok = warp_wait(bar(F_B_EMPTY + s), ((bn / kSt) & 1) ^ 1, a.ws);
+        if (!ok) break;
+        if (lane == 0) {
+          const uint32_t fb = bar(F_B_FULL + s);
+          mbar_expect_tx(fb, 2 * STILE);
+          const int y = r->s0 + c.j * kStr;
+          for (int b = 0; b < NB; ++b) {
+            tma_load_2d(sB1 + s * STILE + b * SBLK, &tmq, fb, h * D + b * BOXW, y);
+            tma_load_2d(sB2 + s * STILE + b * SBLK, &tmdo, fb, h * D + b * BOXW, y);
+          }
+        }
+        ++bn;
+      }
+    }
+    if (lane == 0 && load_status(a.ws) != 0) {  // drain copies in flight before exiting
+      for (uint32_t kb = 0; kb < 2; ++kb) {
+        const uint32_t armed = kn / 2 + (kb < (kn & 1) ? 1u : 0u);
+        if (armed > 0) drain_wait(bar(F_K_FULL + kb), (armed - 1) & 1);
+      }
+      if (vn > 0) drain_wait(bar(F_V_FULL), (vn - 1) & 1);
+      for (int s = 0; s < kSt; ++s) {
+        const uint32_t armed = bn / kSt + (s < (int)(bn % kSt) ? 1u : 0u);
+        if (armed > 0) drain_wait(bar(F_B_FULL + s), (armed - 1) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // --------------------------------------------------------- MMA issuer
+    // One lane.  Step n: the S^T MMAs into X1, then (once the dQ^T two steps
+    // back has been read out of X2) the dP^T MMAs into X2; then the MMAs of
+    // step n - 1 that consume its bf16 P^T / dS^T: dQ^T first (its drain
+    // overlaps the rest), then dV and dK.
+    if (lane == 0) {
+      uint32_t an = 0, bn = 0, xc = 0, accn = 0;
+      bool ok = true;
+      // Descriptor bases; offsets only add to the start-address field.
+      const uint64_t dK0 = smem_desc(sK, 16, SBO, kSwizzle128B);      // K, K-major
+      const uint64_t dKt0 = smem_desc(sK, RBLK, SBO, kSwizzle128B);   // K^T, MN-major
+      const uint64_t dV = smem_desc(sV, 16, SBO, kSwizzle128B);
+      const uint64_t dB1 = smem_desc(sB1, 16, SBO, kSwizzle128B);
+      const uint64_t dB2 = smem_desc(sB2, 16, SBO, kSwizzle128B);
+      const uint64_t mB1 = smem_desc(sB1, SBLK, SBO, kSwizzle128B);  // MN-major views
+      const uint64_t mB2 = smem_desc(sB2, SBLK, SBO, kSwizzle128B);
+      // dS^T is one 128-byte-wide box: the leading byte offset is never used
+      const uint64_t dDS = smem_desc(sDS, DSTILE, SBO, kSwizzle128B);
+      auto koff = [](int ks, int blk) -> uint32_t {  // k-step ks of a K-major tile, 16-byte units
+        return (uint32_t)((((ks * 32) / SW) * blk + (ks * 32) % SW) >> 4);
+      };
+      constexpr uint32_t kRows16 = (16 * SW) >> 4;  // 16 rows of an MN-major tile, 16-byte units
+      // MMAs of the step with ring counter bm / X counter xm, K buffer kb
+      auto acc = [&](uint32_t bm, uint32_t xm, uint32_t kb, bool first, bool last) -> bool {
+        const uint32_t b = xm & 1;
+        if (!mbar_wait(bar(F_OP_FULL + b), (xm >> 1) & 1, a.ws)) return false;
+        if (first && !mbar_wait(bar(F_ACC_EMPTY), (accn & 1) ^ 1, a.ws)) return false;
+        tc_fence_after();
+        const uint64_t dKt = dKt0 + ((kb * RTILE) >> 4);
+        const uint64_t dS = dDS + ((b * DSTILE) >> 4);
+#pragma unroll
+        for (int ks = 0; ks < kRes / 16; ++ks)  // dQ^T = K^T dS^T over the read-out dP^T
+          mma_ss(tmem + kColX2 + b * 64, dKt + ks * kRows16, dS + ks * kRows16, IDESC_DQ,
+                 ks > 0 ? 1u : 0u);
+        tc_commit(bar(F_DQ_FULL + b));
+        if (last) tc_commit(bar(F_K_EMPTY + kb));  // last use of this K buffer
+        const int s = bm % kSt;
+        const uint32_t so = (uint32_t)(s * STILE) >> 4;
+#pragma unroll
+        for (int ks = 0; ks < kStr / 16; ++ks) {
+          const uint32_t accum = (!first || ks > 0) ? 1u : 0u;
+          const uint32_t ko = so + ks * kRows16;
+          const uint32_t xo = b * 64 + (ks >> 1) * 32 + (ks & 1) * 8;
+          mma_ts(tmem + kColAcc1, tmem + kColX1 + xo, mB2 + ko, IDESC_ACC, accum);       // dV += P^T dO
+          mma_ts(tmem + kColAcc2, tmem + kColX1 + xo + 16, mB1 + ko, IDESC_ACC, accum);  // dK += dS^T Q
+        }
+        tc_commit(bar(F_B_EMPTY + s));
+        return true;
+      };
+      for (int kk = 0; ok; ++kk) {
+        const int slot = kk % kUSlots;
+        ok = mbar_wait(bar(F_U_FULL + slot), (kk / kUSlots) & 1, a.ws);
+        if (!ok) break;
+        const int nt = ring[slot].nsteps;
+        mbar_arrive(bar(F_U_EMPTY + slot));
+        if (nt < 0) break;
+        if (nt == 0) continue;
+        const uint32_t kb = an & 1;
+        ok = mbar_wait(bar(F_K_FULL + kb), (an >> 1) & 1, a.ws) &&
+             mbar_wait(bar(F_V_FULL), an & 1, a.ws);
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t dK = dK0 + ((kb * RTILE) >> 4);
+        const uint32_t bn0 = bn, xc0 = xc;
+        for (int n = 0; n < nt; ++n) {
+          const int s = bn % kSt;
+          ok = mbar_wait(bar(F_B_FULL + s), (bn / kSt) & 1, a.ws);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t b = xc & 1;
+          const uint32_t so = (uint32_t)(s * STILE) >> 4;
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks)  // S^T = K Q^T
+            mma_ss(tmem + kColX1 + b * 64, dK + koff(ks, RBLK), dB1 + so + koff(ks, SBLK), IDESC_X,
+                   ks > 0 ? 1u : 0u);
+          // X2(b) still holds the dQ^T of step xc - 2 until its drain is done
+          ok = mbar_wait(bar(F_DQ_EMPTY + b), ((xc >> 1) & 1) ^ 1, a.ws);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks)  // dP^T = V dO^T
+            mma_ss(tmem + kColX2 + b * 64, dV + koff(ks, RBLK), dB2 + so + koff(ks, SBLK), IDESC_X,
+                   ks > 0 ? 1u : 0u);
+          tc_commit(bar(F_X_FULL + b));
+          if (n + 1 == nt) tc_commit(bar(F_V_EMPTY));  // last use of V
+          if (n > 0) {
+            ok = acc(bn - 1, xc - 1, kb, n == 1, false);
+            if (!ok) break;
+          }
+          ++bn;
+          ++xc;
+        }
+        if (!ok) break;
+        ok = acc(bn0 + nt - 1, xc0 + nt - 1, kb, nt == 1, true);
+        if (!ok) break;
+        tc_commit(bar(F_ACC_FULL));
+        ++an;
+        ++accn;
+      }
+      tc_commit(bar(F_DRAIN));
+      drain_wait(bar(F_DRAIN), 0);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ pointwise + drains
+    // Two groups of eight warps take alternate steps (group g owns X buffer
+    // g); the two warps of a group on one 32-lane TMEM quarter split the
+    // step's 64 query columns in halves.  Per step a warp turns its 32 scores
+    // per key into P^T and dS^T (bf16, TMEM), copies dS^T into shared memory
+    // for the dQ MMA, and once that MMA is done reads its 32 dQ^T columns
+    // (query rows) for the 32 head-dim lanes of its quarter and adds them to
+    // the fp32 workspace.  Unit epilogue: warp `chunk` of a quarter stores
+    // accumulator columns [32 chunk, +32) of dV and dK.
+    const int pw = warp - kPwWarp0;
+    const int grp = pw >> 3;              // X buffer / step parity of this warp
+    const int quarter = warp & 3;
+    const int chunk = pw >> 2;            // 0..3
+    const int half = chunk & 1;           // query-column half within the group
+    const int row = quarter * 32 + lane;  // key row (and head-dim lane of dQ^T)
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    const uint64_t half_alpha2 = f2s(0.5f * a.alpha);
+    // dS is produced as 2 dP SiLU'(x): its consumers take alpha / (2N)
+    const float sc_dv = a.inv_n, sc_dk = 0.5f * a.alpha * a.inv_n;
+    const int col = half * 32;
+    const uint32_t ds_row = sDS + (uint32_t)row * SW;
+    const uint32_t swz = (uint32_t)(row & 7);
+    uint32_t xc = 0, accn = 0;
+    bool ok = true;
+    for (int kk = 0; ok; ++kk) {
+      const int slot = kk % kUSlots;
+      ok = warp_wait(bar(F_U_FULL + slot), (kk / kUSlots) & 1, a.ws);
+      if (!ok) break;
+      const UnitRec* r = &ring[slot];
+      const int nt = r->nsteps;
+      if (nt < 0) {
+        warp_arrive(bar(F_U_EMPTY + slot));
+        break;
+      }
+      const int h = r->h, s0 = r->s0, L = r->L, Lh = r->Lh, t0 = r->t0, t1 = r->t1;
+      const int rr = t0 + row;  // this thread's key position in the sequence
+      bf16* o1 = a.dv + (int64_t)(s0 + rr) * a.dv_rs + h * D + chunk * 32;
+      bf16* o2 = a.dk + (int64_t)(s0 + rr) * a.dk_rs + h * D + chunk * 32;
+      if (nt == 0) {  // keys no row sees
+        if (rr < t1) {
+          const uint4 z = make_uint4(0, 0, 0, 0);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            reinterpret_cast<uint4*>(o1)[v] = z;
+            reinterpret_cast<uint4*>(o2)[v] = z;
+          }
+        }
+        warp_arrive(bar(F_U_EMPTY + slot));
+        continue;
+      }
+      const KeyMask km = key_mask(rr, L, Lh, a.K1, a.K2e);
+      // dQ workspace ([H][T][D]) column of this lane (head-dim index `row`)
+      // at the sequence start
+      float* dqa = a.dqacc + ((int64_t)h * a.T + s0) * D + row;
+      SpanCursor c;
+      c.begin(r);
+      for (int n = 0; n < nt; ++n, ++xc, c.next(r)) {
+        const uint32_t b = xc & 1;
+        if ((int)b != grp) continue;  // the other group's step
+        ok = warp_wait(bar(F_X_FULL + b), (xc >> 1) & 1, a.ws);
+        if (!ok) break;
+        tc_fence_after();
+        const int c0 = c.j * kStr;  // first query row of this step
+        const bool full = tile_full(c0, c0 + kStr, t0, t0 + kRes, Lh, a.K1, a.K2e);
+        const uint32_t xs_addr = lane_base + kColX1 + b * 64 + col;
+        const uint32_t xd_addr = lane_base + kColX2 + b * 64 + col;
+        uint32_t xs0[16], xs1[16], xd0[16], xd1[16];
+        tmem_ld16(xs_addr, xs0);
+        tmem_ld16(xs_addr + 16, xs1);
+        tmem_ld16(xd_addr, xd0);
+        tmem_ld16(xd_addr + 16, xd1);
+        tmem_ld_wait2(xs0, xs1);
+        tmem_ld_wait2(xd0, xd1);
+        // Fully visible tiles skip the mask; others clear invisible entries by
+        // one bit test against this key's 32-row visibility mask.
+        const uint32_t bits = full ? 0xFFFFFFFFu : key_mask_bits(km, c0 + col);
+        uint32_t pp[16], dd[16];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          bwd_pair(xs0[2 * e], xs0[2 * e + 1], xd0[2 * e], xd0[2 * e + 1], half_alpha2, pp[e], dd[e]);
+          bwd_pair(xs1[2 * e], xs1[2 * e + 1], xd1[2 * e], xd1[2 * e + 1], half_alpha2, pp[8 + e],
+                   dd[8 + e]);
+        }
+        if (!full) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            pp[e] = mask_pair(pp[e], bits, e);
+            dd[e] = mask_pair(dd[e], bits, e);
+          }
+        }
+        // P^T and dS^T over the score columns this warp just read
+        tmem_st16(xs_addr, pp);
+        tmem_st16(xs_addr + 16, dd);
+        // dS^T row of this key, query columns [col, col + 32): 16-byte chunks
+        // half * 4 + q of the 128-byte row, 128-byte swizzled
+        const uint32_t dsr = ds_row + b * DSTILE;
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          st_shared_v4(dsr + ((((uint32_t)(half * 4 + q)) ^ swz) << 4), dd[4 * q], dd[4 * q + 1],
+                       dd[4 * q + 2], dd[4 * q + 3]);
+        fence_proxy_async_smem();  // visible to the dQ MMA
+        tmem_st_wait();
+        tc_fence_before();
+        warp_arrive(bar(F_OP_FULL + b));
+        // ------------------------------------------- dQ^T of this step
+        ok = warp_wait(bar(F_DQ_FULL + b), (xc >> 1) & 1, a.ws);
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t g0[16], g1[16];
+        tmem_ld16(xd_addr, g0);
+        tmem_ld16(xd_addr + 16, g1);
+        tmem_ld_wait2(g0, g1);
+        tc_fence_before();
+        warp_arrive(bar(F_DQ_EMPTY + b));
+        // column e is query row c0 + col + e; rows past the sequence end are skipped
+        const int q0 = c0 + col;
+        const int nv = L - q0;
+        float* p = dqa + q0 * D;
+        if (nv >= 32) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) red_add_f32(p + e * D, g0[e]);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) red_add_f32(p + (16 + e) * D, g1[e]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            if (e < nv) red_add_f32(p + e * D, g0[e]);
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            if (16 + e < nv) red_add_f32(p + (16 + e) * D, g1[e]);
+        }
+      }
+      if (!ok) break;
+      // ---------------------------------------------------------- epilogue
+      ok = warp_wait(bar(F_ACC_FULL), accn & 1, a.ws);
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll 1
+      for (int which = 0; which < 2; ++which) {
+        uint32_t x0[16], x1[16], o[16];
+        const uint32_t cbase = lane_base + (which ? kColAcc2 : kColAcc1) + chunk * 32;
+        tmem_ld16(cbase, x0);
+        tmem_ld16(cbase + 16, x1);
+        tmem_ld_wait2(x0, x1);
+        const float sc = which ? sc_dk : sc_dv;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          o[e] = pack_bf16x2(__uint_as_float(x0[2 * e]) * sc, __uint_as_float(x0[2 * e + 1]) * sc);
+          o[8 + e] =
+              pack_bf16x2(__uint_as_float(x1[2 * e]) * sc, __uint_as_float(x1[2 * e + 1]) * sc);
+        }
+        if (which == 1) {  // both accumulators read: the next unit may start
+          tc_fence_before();
+          warp_arrive(bar(F_ACC_EMPTY));
+          ++accn;
+        }
+        if (rr < t1) {
+          uint4* dst = reinterpret_cast<uint4*>(which ? o2 : o1);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            dst[q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+        }
+      }
+      warp_arrive(bar(F_U_EMPTY + slot));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// dq[t, h, :] = bf16(scale * workspace[h, t, :]), eight head-dim values per
+// thread and step.
+__global__ void __launch_bounds__(256) dq_convert_kernel(const float* __restrict__ acc,
+                                                         bf16* __restrict__ dq, int64_t dq_rs,
+                                                         int64_t T, int H, float scale) {
+  constexpr int kChunks = D / 8;
+  const int64_t n = T * H * kChunks;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t th = i / kChunks;  // t * H + h
+    const int c = (int)(i - th * kChunks) * 8;
+    const int64_t t = th / H;
+    const int h = (int)(th - t * H);
+    const float4* src = reinterpret_cast<const float4*>(acc + ((int64_t)h * T + t) * D + c);
+    const float4 x0 = __ldcs(src), x1 = __ldcs(src + 1);
+    uint4 o;
+    o.x = pack_bf16x2(x0.x * scale, x0.y * scale);
+    o.y = pack_bf16x2(x0.z * scale, x0.w * scale);
+    o.z = pack_bf16x2(x1.x * scale, x1.y * scale);
+    o.w = pack_bf16x2(x1.z * scale, x1.w * scale);
+    *reinterpret_cast<uint4*>(dq + t * dq_rs + h * D + c) = o;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_fused(const AttnArgs& a, cudaStream_t st) {
+  if (a.T == 0) return cudaSuccess;
+  const int HD = a.H * D;
+  CUtensorMap mk, mv, mq, mdo;
+  if (!make_tma_2d(&mk, a.k, a.T, HD, a.k_rs, BOXW, kRes, true) ||
+      !make_tma_2d(&mv, a.v, a.T, HD, a.v_rs, BOXW, kRes, true) ||
+      !make_tma_2d(&mq, a.q, a.T, HD, a.q_rs, BOXW, kStr, true) ||
+      !make_tma_2d(&mdo, a.dout, a.T, HD, a.do_rs, BOXW, kStr, true))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaMemsetAsync(a.dqacc, 0, dq_workspace_bytes(a.T, a.H, D), st);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(bwd_kvq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+  if (e != cudaSuccess) return e;
+  const int64_t units = max_items(a.T, a.B) * a.H;
+  const int sms = device_sm_count();
+  const int grid = (int)(units < sms ? units : sms);
+  bwd_kvq_kernel<<<grid, kThreads, SMEM, st>>>(mk, mv, mq, mdo, a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  dq_convert_kernel<<<sms * 8, 256, 0, st>>>(a.dqacc, a.dq, a.dq_rs, a.T, a.H,
+                                             0.5f * a.alpha * a.inv_n);
+  return cudaGetLastError();
+}
+
+}  // namespace hstu

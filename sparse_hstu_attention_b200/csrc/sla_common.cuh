@@ -58,6 +58,16 @@ __host__ __device__ inline size_t ws_bytes(int64_t T, int B) {
   return align256(ws_items2_offset(T, B) + sizeof(int2) * size_t(max_items(T, B)));
 }
 
+// The one-pass backward (head_dim kFusedBwdD) accumulates dQ in fp32 [H, T, d]
+// after the work lists; other head dims need no such buffer.
+constexpr int kFusedBwdD = 128;
+__host__ __device__ inline size_t dq_workspace_bytes(int64_t T, int H, int d) {
+  return d == kFusedBwdD ? size_t(T) * size_t(H) * size_t(d) * sizeof(float) : 0;
+}
+__host__ __device__ inline size_t ws_bwd_bytes(int64_t T, int B, int H, int d) {
+  return ws_bytes(T, B) + dq_workspace_bytes(T, H, d);
+}
+
 // ------------------------------------------------------------ kernel args
 struct AttnArgs {
   const int32_t* offs;   // [B+1]
@@ -65,6 +75,7 @@ struct AttnArgs {
   const int2* items;     // work list 0 (query tiles)
   const int2* items2;    // work list 1 (key tiles)
   WsHeader* ws;          // status / counts
+  float* dqacc;          // fp32 dQ accumulator [H, T, d] (one-pass backward only)
   int B, H, K1, K2e, max_seq_len;
   int64_t T;
   float alpha, inv_n;
@@ -335,10 +346,13 @@ __device__ __forceinline__ int load_status(const WsHeader* ws) {
 // (defined in the .cu files; return cudaError_t of the launch)
 // list 0: (sequence, query tile of `tile` rows); list 1: (sequence, key tile
 // of `tile` keys), prefix key tiles first.
-cudaError_t launch_worklist(const AttnArgs& a, int tile, int list, cudaStream_t st);
+// `first`: the call's first work list, which also resets the status word.
+cudaError_t launch_worklist(const AttnArgs& a, int tile, int list, bool first, cudaStream_t st);
 cudaError_t launch_count_pairs(const AttnArgs& a, int BMf, int BNf, int BMb, int BNb,
                                int64_t* row_counts, int64_t* key_counts, cudaStream_t st);
 cudaError_t launch_fwd_tc(const AttnArgs& a, int d, cudaStream_t st);
 cudaError_t launch_bwd_tc(const AttnArgs& a, int d, bool kv_pass, cudaStream_t st);
+// head_dim kFusedBwdD: zeroes a.dqacc, runs the one-pass backward, converts dq
+cudaError_t launch_bwd_fused(const AttnArgs& a, cudaStream_t st);
 
 }  // namespace hstu

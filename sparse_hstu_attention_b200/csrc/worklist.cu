@@ -45,7 +45,8 @@ __device__ int block_exclusive_scan(int v, int* out, int* smem) {
 // One block.  list 0: items (b, query tile) in sequence order.  list 1:
 // first every (b, key tile) whose key tile starts inside the history prefix
 // [0, min(K2eff, Lh)), then all other key tiles.
-__global__ void __launch_bounds__(kWlThreads) worklist_kernel(AttnArgs a, int tile, int list) {
+__global__ void __launch_bounds__(kWlThreads) worklist_kernel(AttnArgs a, int tile, int list,
+                                                             int first) {
   __shared__ int s_scan[32];
   __shared__ int s_bad;
   const int backward = list;
@@ -104,12 +105,12 @@ __global__ void __launch_bounds__(kWlThreads) worklist_kernel(AttnArgs a, int ti
     if (pass == 0) n_pre = written;
   }
   if (threadIdx.x == 0) {
+    if (first) a.ws->status = HSTU_SLA_OK;
     if (list) {
       a.ws->n_items2 = written;
       a.ws->n_items2_pre = n_pre;
       a.ws->sched2 = 0;
     } else {
-      a.ws->status = HSTU_SLA_OK;  // list 0 is always built first
       a.ws->n_items = written;
       a.ws->sched = 0;
     }
@@ -157,8 +158,8 @@ __global__ void count_pairs_kernel(AttnArgs a, int BMf, int BNf, int BMb, int BN
 
 }  // namespace
 
-cudaError_t launch_worklist(const AttnArgs& a, int tile, int list, cudaStream_t st) {
-  worklist_kernel<<<1, kWlThreads, 0, st>>>(a, tile, list);
+cudaError_t launch_worklist(const AttnArgs& a, int tile, int list, bool first, cudaStream_t st) {
+  worklist_kernel<<<1, kWlThreads, 0, st>>>(a, tile, list, first ? 1 : 0);
   return cudaGetLastError();
 }
 

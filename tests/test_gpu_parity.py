@@ -85,15 +85,26 @@ def test_strided_fused_projection_views():
     _full_check(b, strided=True)
 
 
-def test_repeat_calls_are_bitwise_identical():
-    """No atomics anywhere: forward and backward are deterministic."""
-    b = _edge_batch(lengths=[300, 200, 1000], nt=10)
+@pytest.mark.parametrize("d", [128, 64])
+def test_repeat_calls_reproducible(d):
+    """The forward, dk and dv have no atomics: bitwise identical across calls.
+    dq at d = 128 sums fp32 partials with atomic additions in no fixed order,
+    so two calls agree only to within the bf16 rounding of the same fp32
+    sum; at d = 64 (query-tile pass, no atomics) dq is bitwise identical."""
+    b = _edge_batch(lengths=[300, 200, 1000], nt=10, d=d)
     g = to_gpu(b)
     o1, o2 = gpu_fwd(b, g), gpu_fwd(b, g)
     assert torch.equal(o1, o2)
-    d1, d2 = gpu_bwd(b, g), gpu_bwd(b, g)
-    for x, y in zip(d1, d2):
-        assert torch.equal(x, y)
+    (q1, k1, v1), (q2, k2, v2) = gpu_bwd(b, g), gpu_bwd(b, g)
+    assert torch.equal(k1, k2) and torch.equal(v1, v2)
+    if d == 128:
+        # one bf16 ulp of the larger magnitude (2^-7 relative) bounds the gap,
+        # plus a floor for sums that cancel to near zero
+        a1, a2 = q1.float(), q2.float()
+        bound = 2.0 ** -7 * torch.maximum(a1.abs(), a2.abs()) + 1e-4 * a1.abs().max()
+        assert ((a1 - a2).abs() <= bound).all()
+    else:
+        assert torch.equal(q1, q2)
 
 
 @pytest.mark.parametrize("wname", ["mid", "hist16k"])
