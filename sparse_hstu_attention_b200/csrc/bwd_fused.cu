@@ -31,9 +31,9 @@
 //               dQ drain of their step; at the end of a unit, all sixteen
 //               store dK and dV
 // TMEM columns:
-//   X1(b) = [64b, 64b+64)       S^T (fp32); after the pointwise: per 32-column
-//                               chunk c, P^T bf16 in [32c, 32c+16) and dS^T
-//                               bf16 in [32c+16, 32c+32)
+//   X1(b) = [64b, 64b+64)       S^T (fp32); after the pointwise: per 16-column
+//                               group g, P^T bf16 in [16g, 16g+8) and dS^T
+//                               bf16 in [16g+8, 16g+16)
 //   X2(b) = [128+64b, 192+64b)  dP^T (fp32); then the step's dQ^T (lanes =
 //                               head-dim index, columns = query rows)
 //   ACC1 = [256, 384) dV,  ACC2 = [384, 512) dK
@@ -279,9 +279,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int ks = 0; ks < kStr / 16; ++ks) {
           const uint32_t accum = (!first || ks > 0) ? 1u : 0u;
           const uint32_t ko = so + ks * kRows16;
-          const uint32_t xo = b * 64 + (ks >> 1) * 32 + (ks & 1) * 8;
-          mma_ts(tmem + kColAcc1, tmem + kColX1 + xo, mB2 + ko, IDESC_ACC, accum);       // dV += P^T dO
-          mma_ts(tmem + kColAcc2, tmem + kColX1 + xo + 16, mB1 + ko, IDESC_ACC, accum);  // dK += dS^T Q
+          // queries [16 ks, +16): P^T at columns 32 (ks / 2) + 16 (ks % 2), dS^T 8 further
+          const uint32_t xo = b * 64 + (ks >> 1) * 32 + (ks & 1) * 16;
+          mma_ts(tmem + kColAcc1, tmem + kColX1 + xo, mB2 + ko, IDESC_ACC, accum);      // dV += P^T dO
+          mma_ts(tmem + kColAcc2, tmem + kColX1 + xo + 8, mB1 + ko, IDESC_ACC, accum);  // dK += dS^T Q
         }
         tc_commit(bar(F_B_EMPTY + s));
         return true;
@@ -407,40 +408,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool full = tile_full(c0, c0 + kStr, t0, t0 + kRes, Lh, a.K1, a.K2e);
         const uint32_t xs_addr = lane_base + kColX1 + b * 64 + col;
         const uint32_t xd_addr = lane_base + kColX2 + b * 64 + col;
-        uint32_t xs0[16], xs1[16], xd0[16], xd1[16];
-        tmem_ld16(xs_addr, xs0);
-        tmem_ld16(xs_addr + 16, xs1);
-        tmem_ld16(xd_addr, xd0);
-        tmem_ld16(xd_addr + 16, xd1);
-        tmem_ld_wait2(xs0, xs1);
-        tmem_ld_wait2(xd0, xd1);
+        const uint32_t dsr = ds_row + b * DSTILE;
         // Fully visible tiles skip the mask; others clear invisible entries by
         // one bit test against this key's 32-row visibility mask.
         const uint32_t bits = full ? 0xFFFFFFFFu : key_mask_bits(km, c0 + col);
-        uint32_t pp[16], dd[16];
+        // Two rounds of 16 query columns each (fewer live registers).  Round r
+        // writes P^T (8 packed columns) then dS^T (8) over the 16 score
+        // columns it read, and copies dS^T to 16-byte chunks half*4 + 2r,
+        // +1 of this key's 128-byte swizzled row of the dS^T tile.
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          bwd_pair(xs0[2 * e], xs0[2 * e + 1], xd0[2 * e], xd0[2 * e + 1], half_alpha2, pp[e], dd[e]);
-          bwd_pair(xs1[2 * e], xs1[2 * e + 1], xd1[2 * e], xd1[2 * e + 1], half_alpha2, pp[8 + e],
-                   dd[8 + e]);
-        }
-        if (!full) {
+        for (int r = 0; r < 2; ++r) {
+          uint32_t xs[16], xd[16], pp[8], dd[8];
+          tmem_ld16(xs_addr + 16 * r, xs);
+          tmem_ld16(xd_addr + 16 * r, xd);
+          tmem_ld_wait2(xs, xd);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            pp[e] = mask_pair(pp[e], bits, e);
-            dd[e] = mask_pair(dd[e], bits, e);
+          for (int e = 0; e < 8; ++e)
+            bwd_pair(xs[2 * e], xs[2 * e + 1], xd[2 * e], xd[2 * e + 1], half_alpha2, pp[e], dd[e]);
+          if (!full) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              pp[e] = mask_pair(pp[e], bits, 8 * r + e);
+              dd[e] = mask_pair(dd[e], bits, 8 * r + e);
+            }
           }
-        }
-        // P^T and dS^T over the score columns this warp just read
-        tmem_st16(xs_addr, pp);
-        tmem_st16(xs_addr + 16, dd);
-        // dS^T row of this key, query columns [col, col + 32): 16-byte chunks
-        // half * 4 + q of the 128-byte row, 128-byte swizzled
-        const uint32_t dsr = ds_row + b * DSTILE;
+          tmem_st8(xs_addr + 16 * r, pp);
+          tmem_st8(xs_addr + 16 * r + 8, dd);
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          st_shared_v4(dsr + ((((uint32_t)(half * 4 + q)) ^ swz) << 4), dd[4 * q], dd[4 * q + 1],
-                       dd[4 * q + 2], dd[4 * q + 3]);
+          for (int q = 0; q < 2; ++q)
+            st_shared_v4(dsr + ((((uint32_t)(half * 4 + 2 * r + q)) ^ swz) << 4), dd[4 * q],
+                         dd[4 * q + 1], dd[4 * q + 2], dd[4 * q + 3]);
+        }
         fence_proxy_async_smem();  // visible to the dQ MMA
         tmem_st_wait();
         tc_fence_before();
