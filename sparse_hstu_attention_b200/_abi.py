@@ -8,6 +8,7 @@ import re
 PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libhstu_sla.so")
 HEADER = os.path.join(os.path.dirname(PKG), "include", "hstu_sla.h")
+HEADERS = [HEADER, os.path.join(os.path.dirname(PKG), "include", "hstu_stu.h")]
 
 OK = 0
 ERR_INVALID_ARG = -1
@@ -46,6 +47,50 @@ class BwdParams(ctypes.Structure):
     ]
 
 
+class StuLayerParams(ctypes.Structure):
+    _fields_ = [
+        ("B", ctypes.c_int32), ("H", ctypes.c_int32), ("d", ctypes.c_int32),
+        ("total_tokens", ctypes.c_int64), ("max_seq_len", ctypes.c_int32),
+        ("seq_offsets", ctypes.c_void_p), ("num_targets", ctypes.c_void_p),
+        ("contextual_len", ctypes.c_int32), ("K1", ctypes.c_int32), ("K2", ctypes.c_int32),
+        ("alpha", ctypes.c_float), ("N", ctypes.c_float), ("ln_eps", ctypes.c_float),
+        ("ln1_w", ctypes.c_void_p), ("ln1_b", ctypes.c_void_p), ("w1", ctypes.c_void_p),
+        ("b1", ctypes.c_void_p), ("ln2_w", ctypes.c_void_p), ("ln2_b", ctypes.c_void_p),
+        ("w2", ctypes.c_void_p), ("b2", ctypes.c_void_p),
+        ("x", ctypes.c_void_p), ("out", ctypes.c_void_p),
+        ("xn", ctypes.c_void_p), ("pre", ctypes.c_void_p), ("uvqk", ctypes.c_void_p),
+        ("av", ctypes.c_void_p), ("y", ctypes.c_void_p), ("stats", ctypes.c_void_p),
+    ]
+
+
+class StuLayerBwdParams(ctypes.Structure):
+    _fields_ = [
+        ("fwd", StuLayerParams),
+        ("dout", ctypes.c_void_p), ("dx", ctypes.c_void_p),
+        ("dy", ctypes.c_void_p), ("dav", ctypes.c_void_p), ("dpre", ctypes.c_void_p),
+        ("dxn", ctypes.c_void_p),
+        ("d_ln1_w", ctypes.c_void_p), ("d_ln1_b", ctypes.c_void_p), ("d_w1", ctypes.c_void_p),
+        ("d_b1", ctypes.c_void_p), ("d_ln2_w", ctypes.c_void_p), ("d_ln2_b", ctypes.c_void_p),
+        ("d_w2", ctypes.c_void_p), ("d_b2", ctypes.c_void_p),
+    ]
+
+
+GEMM_STORE, GEMM_BIAS_SILU, GEMM_BIAS_RESID, GEMM_RED_F32 = 0, 1, 2, 3
+
+
+class GemmParams(ctypes.Structure):
+    _fields_ = [
+        ("M", ctypes.c_int32), ("N", ctypes.c_int32), ("K", ctypes.c_int32),
+        ("a", ctypes.c_void_p), ("lda", ctypes.c_int64), ("a_mn_major", ctypes.c_int32),
+        ("b", ctypes.c_void_p), ("ldb", ctypes.c_int64), ("b_mn_major", ctypes.c_int32),
+        ("epilogue", ctypes.c_int32), ("splits", ctypes.c_int32),
+        ("bias", ctypes.c_void_p), ("resid", ctypes.c_void_p), ("ldr", ctypes.c_int64),
+        ("out", ctypes.c_void_p), ("ldo", ctypes.c_int64),
+        ("out2", ctypes.c_void_p), ("ldo2", ctypes.c_int64),
+        ("outf", ctypes.c_void_p), ("ldf", ctypes.c_int64),
+    ]
+
+
 _lib = None
 
 
@@ -80,15 +125,33 @@ def load():
     lib.hstu_sla_strerror.restype = ctypes.c_char_p
     lib.hstu_sla_version.argtypes = []
     lib.hstu_sla_version.restype = ctypes.c_int
+    i32, i64 = ctypes.c_int32, ctypes.c_int64
+    lib.hstu_stu_workspace_bytes.argtypes = [ctypes.c_int, i64, i32, i32, i32]
+    lib.hstu_stu_workspace_bytes.restype = sz
+    lib.hstu_stu_layer_fwd.argtypes = [ctypes.POINTER(StuLayerParams), vp, sz, vp]
+    lib.hstu_stu_layer_fwd.restype = ctypes.c_int
+    lib.hstu_stu_layer_bwd.argtypes = [ctypes.POINTER(StuLayerBwdParams), vp, sz, vp]
+    lib.hstu_stu_layer_bwd.restype = ctypes.c_int
+    lib.hstu_stu_get_error.argtypes = [vp, vp]
+    lib.hstu_stu_get_error.restype = ctypes.c_int
+    lib.hstu_jagged_truncate_offsets.argtypes = [vp, vp, i32, i32, i32, vp, vp]
+    lib.hstu_jagged_truncate_offsets.restype = ctypes.c_int
+    lib.hstu_jagged_truncate.argtypes = [vp, i64, vp, vp, vp, i32, i32, i32, i32, vp, i64, i64,
+                                         i32, vp]
+    lib.hstu_jagged_truncate.restype = ctypes.c_int
+    lib.hstu_gemm.argtypes = [ctypes.POINTER(GemmParams), vp, vp]
+    lib.hstu_gemm.restype = ctypes.c_int
     _lib = lib
     return lib
 
 
 def declared_functions():
-    """Names of the functions include/hstu_sla.h declares."""
-    text = open(HEADER).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(hstu_\w+)\s*\(", text)))
+    """Names of the functions include/hstu_sla.h and include/hstu_stu.h declare."""
+    names = set()
+    for h in HEADERS:
+        text = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        names.update(re.findall(r"\b(hstu_\w+)\s*\(", text))
+    return sorted(names)
 
 
 def strerror(code: int) -> str:

@@ -1,0 +1,334 @@
+// Dense bf16 GEMM on the 5th-generation tensor cores (tcgen05 / TMEM / TMA)
+// for the STU layer's projections: f1 of Eq. 2 (the UVQK projection), f2 of
+// Eq. 4 (the output projection) and their backward contractions, of "Bending
+// the Scaling Law Curve in Large-Scale Recommendation Systems", section 3
+// (and the addmm steps of its Listing 1, section 4.2.2).
+//
+//   D[m, n] = sum_k A[m, k] B[n, k]      (bf16 operands, fp32 accumulation)
+//
+// Each operand is read either K-major (row m of A / row n of B holds its K
+// values contiguously: activations x [T, d_in] as A, or a weight W [N, K]
+// as B) or MN-major (row k holds the M / N values contiguously: a weight
+// W [K, N] as B, or activations read transposed for a weight gradient).
+// Epilogues, fused on the TMEM read-out:
+//   kEpiStore      out  = bf16(D)
+//   kEpiBiasSilu   out2 = bf16(D + bias),  out = bf16(SiLU(D + bias))
+//   kEpiBiasResid  out  = bf16(D + bias + resid)
+//   kEpiRedF32     outf += D              (fp32 reductions: split-K partial
+//                                          sums of a weight gradient)
+//
+// Tiles of 128 x 256 (one 128x256x16 UMMA per 16 of K, the full-rate shape),
+// K in blocks of 64 (one 128-byte swizzle atom), 4-stage TMA ring, two TMEM
+// accumulators so a tile's epilogue overlaps the next tile's main loop.
+// Persistent CTAs walk tiles (split, m block, n block) with n fastest, so
+// consecutive tiles share their A rows in L2.
+// Roles: warp 0 TMA producer, warp 1 TMEM allocation + one MMA-issuing lane,
+// warps 2..5 epilogue (warp w reads TMEM lanes 32 (w % 4) .. +32).
+#include <cudaTypedefs.h>
+
+#include "sm100.cuh"
+#include "stu_common.cuh"
+
+namespace hstu {
+
+bool make_tma_2d(CUtensorMap* m, const void* ptr, int64_t T, int HD, int64_t rs, int box_w,
+                 int box_h, bool sw128);
+int device_sm_count();
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kBM = 128, kBN = 256, kBK = 64, kStages = 4;
+constexpr int kThreads = 192;
+constexpr int A_TILE = kBM * kBK * 2;  // 16 KB
+constexpr int B_TILE = kBN * kBK * 2;  // 32 KB
+constexpr int MN_BOX = 64 * kBK * 2;   // one 64 (M or N) x 64 (K) box of an MN-major tile
+constexpr int OFF_A = 0;
+constexpr int OFF_B = OFF_A + kStages * A_TILE;
+constexpr int OFF_BAR = OFF_B + kStages * B_TILE;
+constexpr int OFF_SLOT = OFF_BAR + 128;
+constexpr int SMEM = OFF_SLOT + 16 + 1024;
+static_assert(SMEM <= 232448, "shared memory budget");
+constexpr uint32_t kTmemCols = 2 * kBN;
+
+enum { G_FULL = 0, G_EMPTY = kStages, G_ACC_FULL = 2 * kStages, G_ACC_EMPTY = G_ACC_FULL + 2,
+       G_COUNT = G_ACC_EMPTY + 2 };
+static_assert(8 * G_COUNT <= 128, "barrier area");
+
+struct TileInfo {
+  int m0, n0, k0, nkb;  // first row / column / k, number of 64-wide k blocks
+};
+
+__device__ __forceinline__ TileInfo tile_info(const GemmArgs& g, int t, int tiles_m,
+                                              int tiles_n) {
+  TileInfo ti;
+  const int nb = t % tiles_n;
+  const int rest = t / tiles_n;
+  const int mb = rest % tiles_m;
+  const int split = rest / tiles_m;
+  ti.m0 = mb * kBM;
+  ti.n0 = nb * kBN;
+  ti.k0 = split * g.k_split;
+  const int k1 = min(g.K, ti.k0 + g.k_split);
+  ti.nkb = k1 > ti.k0 ? (k1 - ti.k0 + kBK - 1) / kBK : 0;
+  return ti;
+}
+
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+  asm volatile(
+      "{\n .reg .u64 g;\n cvta.to.global.u64 g, %0;\n"
+      " red.relaxed.gpu.global.add.v4.f32 [g], {%1, %2, %3, %4};\n}\n" ::"l"(p),
+      "f"(a), "f"(b), "f"(c), "f"(d)
+      : "memory");
+}
+
+__device__ __forceinline__ float silu_f(float v) { return v / (1.0f + __expf(-v)); }
+
+template <bool A_MN, bool B_MN, int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmb,
+                   const GemmArgs g) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* base_ptr = smem_raw + (base - raw);
+  const uint32_t sA = base + OFF_A, sB = base + OFF_B;
+  const uint32_t bar0 = base + OFF_BAR;
+  auto bar = [&](int i) { return bar0 + 8u * i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + OFF_SLOT);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tiles_m = (g.M + kBM - 1) / kBM, tiles_n = g.N / kBN;
+  const int ntiles = tiles_m * tiles_n * g.splits;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar(G_FULL + s), 1);
+      mbar_init(bar(G_EMPTY + s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(G_ACC_FULL + b), 1);
+      mbar_init(bar(G_ACC_EMPTY + b), 4);  // the four epilogue warps
+    }
+    fence_barrier_init();
+    prefetch_tmap(&tma);
+    prefetch_tmap(&tmb);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        const TileInfo ti = tile_info(g, t, tiles_m, tiles_n);
+        for (int kb = 0; kb < ti.nkb; ++kb, ++it) {
+          const int s = it % kStages;
+          ok = mbar_wait(bar(G_EMPTY + s), ((it / kStages) & 1) ^ 1, g.ws);
+          if (!ok) break;
+          const uint32_t fb = bar(G_FULL + s);
+          mbar_expect_tx(fb, A_TILE + B_TILE);
+          const int k = ti.k0 + kb * kBK;
+          const uint32_t a = sA + s * A_TILE, b = sB + s * B_TILE;
+          if (A_MN) {  // [K][M]: two 64-wide column boxes
+            tma_load_2d(a, &tma, fb, ti.m0, k);
+            tma_load_2d(a + MN_BOX, &tma, fb, ti.m0 + 64, k);
+          } else {     // [M][K]: 128 rows x 64 k
+            tma_load_2d(a, &tma, fb, k, ti.m0);
+          }
+          if (B_MN) {  // [K][N]: four 64-wide column boxes
+            for (int j = 0; j < kBN / 64; ++j) tma_load_2d(b + j * MN_BOX, &tmb, fb, ti.n0 + 64 * j, k);
+          } else {     // [N][K]: 256 rows x 64 k
+            tma_load_2d(b, &tmb, fb, k, ti.n0);
+          }
+        }
+      }
+      if (load_status(g.ws) != 0) {  // drain copies in flight before exiting
+        for (int s = 0; s < kStages; ++s) {
+          const uint32_t armed = it / kStages + (s < (int)(it % kStages) ? 1u : 0u);
+          if (armed > 0) drain_wait(bar(G_FULL + s), (armed - 1) & 1);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // --------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC = idesc_bf16(kBM, kBN, A_MN, B_MN);
+      // K-major: a 16-wide k step moves 32 bytes inside the 128-byte row;
+      // MN-major: it moves 16 rows of 128 bytes.  Units of 16 bytes.
+      constexpr uint32_t kStepA = A_MN ? 128u : 2u, kStepB = B_MN ? 128u : 2u;
+      const uint64_t dA = A_MN ? smem_desc(sA, MN_BOX, 1024, kSwizzle128B)
+                               : smem_desc(sA, 16, 1024, kSwizzle128B);
+      const uint64_t dB = B_MN ? smem_desc(sB, MN_BOX, 1024, kSwizzle128B)
+                               : smem_desc(sB, 16, 1024, kSwizzle128B);
+      uint32_t it = 0, tc = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        const TileInfo ti = tile_info(g, t, tiles_m, tiles_n);
+        if (ti.nkb == 0) continue;
+        const uint32_t buf = tc & 1;
+        ok = mbar_wait(bar(G_ACC_EMPTY + buf), ((tc >> 1) & 1) ^ 1, g.ws);
+        if (!ok) break;
+        tc_fence_after();
+        for (int kb = 0; kb < ti.nkb; ++kb, ++it) {
+          const int s = it % kStages;
+          ok = mbar_wait(bar(G_FULL + s), (it / kStages) & 1, g.ws);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t ao = (uint32_t)(s * A_TILE) >> 4, bo = (uint32_t)(s * B_TILE) >> 4;
+#pragma unroll
+          for (int ks = 0; ks < kBK / 16; ++ks)
+            mma_ss(tmem + buf * kBN, dA + ao + ks * kStepA, dB + bo + ks * kStepB, IDESC,
+                   (kb > 0 || ks > 0) ? 1u : 0u);
+          tc_commit(bar(G_EMPTY + s));
+        }
+        if (!ok) break;
+        tc_commit(bar(G_ACC_FULL + buf));
+        ++tc;
+      }
+    }
+    __syncwarp();
+  } else {
+    // ----------------------------------------------------------- epilogue
+    const int quarter = warp & 3;
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    uint32_t tc = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+      const TileInfo ti = tile_info(g, t, tiles_m, tiles_n);
+      if (ti.nkb == 0) continue;
+      const uint32_t buf = tc & 1;
+      ok = warp_wait(bar(G_ACC_FULL + buf), (tc >> 1) & 1, g.ws);
+      if (!ok) break;
+      tc_fence_after();
+      const int m = ti.m0 + quarter * 32 + lane;
+      const bool live = m < g.M;
+#pragma unroll 1
+      for (int c = 0; c < kBN; c += 32) {
+        uint32_t v[32];
+        tmem_ld32(lane_base + buf * kBN + c, v);
+        tmem_ld_wait(v);
+        if (c + 32 == kBN) {  // accumulator read out: the next tile may start
+          tc_fence_before();
+          warp_arrive(bar(G_ACC_EMPTY + buf));
+        }
+        if (!live) continue;
+        const int n = ti.n0 + c;
+        if (EPI == kEpiRedF32) {
+          float* dst = g.outf + (int64_t)m * g.ldf + n;
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            red_add_v4(dst + e, __uint_as_float(v[e]), __uint_as_float(v[e + 1]),
+                       __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+          continue;
+        }
+        float f[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(v[e]);
+        if (EPI == kEpiBiasSilu || EPI == kEpiBiasResid) {
+          const float4* bp = reinterpret_cast<const float4*>(g.bias + n);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float4 b4 = __ldg(bp + e);
+            f[4 * e] += b4.x;
+            f[4 * e + 1] += b4.y;
+            f[4 * e + 2] += b4.z;
+            f[4 * e + 3] += b4.w;
+          }
+        }
+        if (EPI == kEpiBiasResid) {
+          const uint4* rp = reinterpret_cast<const uint4*>(g.resid + (int64_t)m * g.ldr + n);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint4 r4 = rp[q];
+            const uint32_t w[4] = {r4.x, r4.y, r4.z, r4.w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              f[8 * q + 2 * h] += __uint_as_float(w[h] << 16);
+              f[8 * q + 2 * h + 1] += __uint_as_float(w[h] & 0xFFFF0000u);
+            }
+          }
+        }
+        uint32_t o[16];
+        if (EPI == kEpiBiasSilu) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) o[e] = pack_bf16x2(f[2 * e], f[2 * e + 1]);
+          uint4* pp = reinterpret_cast<uint4*>(g.out2 + (int64_t)m * g.ldo2 + n);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) pp[q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) o[e] = pack_bf16x2(silu_f(f[2 * e]), silu_f(f[2 * e + 1]));
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) o[e] = pack_bf16x2(f[2 * e], f[2 * e + 1]);
+        }
+        uint4* op = reinterpret_cast<uint4*>(g.out + (int64_t)m * g.ldo + n);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) op[q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+      }
+      ++tc;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <bool A_MN, bool B_MN, int EPI>
+cudaError_t launch_t(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g,
+                     int ntiles, cudaStream_t st) {
+  cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<A_MN, B_MN, EPI>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+  if (e != cudaSuccess) return e;
+  const int sms = device_sm_count();
+  gemm_tc_kernel<A_MN, B_MN, EPI><<<ntiles < sms ? ntiles : sms, kThreads, SMEM, st>>>(ma, mb, g);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm(const GemmOperand& A, const GemmOperand& B, GemmArgs g, int epi,
+                        cudaStream_t st) {
+  if (g.M == 0 || g.N == 0) return cudaSuccess;
+  // split-K only for the reducing epilogue; each split covers whole k blocks
+  if (epi != kEpiRedF32) g.splits = 1;
+  if (g.splits < 1) g.splits = 1;
+  const int kb_total = (g.K + kBK - 1) / kBK;
+  const int kb_per = (kb_total + g.splits - 1) / g.splits;
+  g.k_split = kb_per * kBK;
+  g.splits = kb_per > 0 ? (kb_total + kb_per - 1) / kb_per : 1;
+  CUtensorMap ma, mb;
+  // K-major operand: rows = M (or N), columns = K.  MN-major: rows = K.
+  if (!(A.mn_major ? make_tma_2d(&ma, A.ptr, g.K, g.M, A.ld, 64, kBK, true)
+                   : make_tma_2d(&ma, A.ptr, g.M, g.K, A.ld, kBK, kBM, true)) ||
+      !(B.mn_major ? make_tma_2d(&mb, B.ptr, g.K, g.N, B.ld, 64, kBK, true)
+                   : make_tma_2d(&mb, B.ptr, g.N, g.K, B.ld, kBK, kBN, true)))
+    return cudaErrorInvalidValue;
+  const int ntiles = ((g.M + kBM - 1) / kBM) * (g.N / kBN) * g.splits;
+#define HSTU_GEMM_CASE(AM, BM_, E) \
+  if (A.mn_major == AM && B.mn_major == BM_ && epi == E) return launch_t<AM, BM_, E>(ma, mb, g, ntiles, st);
+  HSTU_GEMM_CASE(false, true, kEpiBiasSilu)    // x^ W1 + b1 -> SiLU      (W1 stored [K][N])
+  HSTU_GEMM_CASE(false, true, kEpiBiasResid)   // y W2 + b2 + x           (W2 stored [K][N])
+  HSTU_GEMM_CASE(false, false, kEpiStore)      // dOut W2^T, dPre W1^T     (W read [N][K])
+  HSTU_GEMM_CASE(false, true, kEpiStore)
+  HSTU_GEMM_CASE(true, true, kEpiRedF32)       // x^T dPre, y^T dOut       (both [K][*])
+  HSTU_GEMM_CASE(false, false, kEpiRedF32)
+#undef HSTU_GEMM_CASE
+  return cudaErrorNotSupported;
+}
+
+}  // namespace hstu

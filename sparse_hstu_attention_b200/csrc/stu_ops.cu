@@ -1,0 +1,311 @@
+// Row- and column-wise kernels of the STU layer ("Bending the Scaling Law
+// Curve in Large-Scale Recommendation Systems", section 3, Eq. 1-5; HSTU's
+// "Actions Speak Louder than Words", section 3.1):
+//   LayerNorm before the UVQK projection (Eq. 1), the gated norm
+//   y = LayerNorm(A V) * U after the attention (Eq. 4), their backward with
+//   the affine-parameter gradients, SiLU' on the projection's gradient with
+//   the bias gradient, and the attention truncation of section 4.3 (keep the
+//   contextual prefix, the last `tail` history tokens and the candidates, as
+//   TorchEasyRec's "Mid-stack Attention Truncation" bullet states).
+// Rows are d_model wide (W = 256, 512 or 1024); one warp per row, lane l
+// owning the 16-byte chunks l, l + 32, ... of the row.
+#include "stu_common.cuh"
+
+namespace hstu {
+namespace {
+
+constexpr int kRowWarps = 8;  // rows per 256-thread block
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ void load8(const bf16* p, float* f) {
+  const uint4 r = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+  for (int h = 0; h < 4; ++h) {
+    f[2 * h] = __uint_as_float(w[h] << 16);
+    f[2 * h + 1] = __uint_as_float(w[h] & 0xFFFF0000u);
+  }
+}
+
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ void store8(bf16* p, const float* f) {
+  *reinterpret_cast<uint4*>(p) =
+      make_uint4(pack2(f[0], f[1]), pack2(f[2], f[3]), pack2(f[4], f[5]), pack2(f[6], f[7]));
+}
+
+__device__ __forceinline__ float silu_grad(float v) {
+  const float s = 1.0f / (1.0f + __expf(-v));
+  return s * (1.0f + v * (1.0f - s));
+}
+
+// LayerNorm (biased variance) of each row, then the affine map; GATED also
+// multiplies by the gate row u.  Saves the row mean and 1/sqrt(var + eps).
+template <int NV, bool GATED>
+__global__ void __launch_bounds__(32 * kRowWarps) ln_fwd_kernel(const LnArgs a) {
+  const int64_t row = (int64_t)blockIdx.x * kRowWarps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= a.T) return;
+  constexpr int W = NV * 256;
+  float x[NV][8];
+#pragma unroll
+  for (int v = 0; v < NV; ++v) load8(a.x + row * a.ldx + 8 * (lane + 32 * v), x[v]);
+  float s = 0.f;
+#pragma unroll
+  for (int v = 0; v < NV; ++v)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) s += x[v][e];
+  const float mean = warp_sum(s) * (1.0f / W);
+  float q = 0.f;
+#pragma unroll
+  for (int v = 0; v < NV; ++v)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) q += (x[v][e] - mean) * (x[v][e] - mean);
+  const float rstd = rsqrtf(warp_sum(q) * (1.0f / W) + a.eps);
+#pragma unroll
+  for (int v = 0; v < NV; ++v) {
+    const int c = 8 * (lane + 32 * v);
+    float z[8], u[8];
+    if (GATED) load8(a.u + row * a.ldu + c, u);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      z[e] = (x[v][e] - mean) * rstd * a.gamma[c + e] + a.beta[c + e];
+      if (GATED) z[e] *= u[e];
+    }
+    store8(a.y + row * a.ldy + c, z);
+  }
+  if (lane == 0) {
+    a.mean[row] = mean;
+    a.rstd[row] = rstd;
+  }
+}
+
+// Backward of the above.  Plain: dx = resid_grad + LN'(dy * gamma).
+// Gated: dz = dy * u, du = dy * z (times SiLU'(pre_u), since the gate is a
+// SiLU output), dx = LN'(dz * gamma).  dgamma / dbeta accumulate per lane
+// over the rows a warp visits, then once into global memory.
+template <int NV, bool GATED>
+__global__ void __launch_bounds__(32 * kRowWarps) ln_bwd_kernel(const LnArgs a) {
+  constexpr int W = NV * 256;
+  const int lane = threadIdx.x & 31;
+  float dg[NV][8], db[NV][8];
+#pragma unroll
+  for (int v = 0; v < NV; ++v)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) dg[v][e] = db[v][e] = 0.f;
+  const int64_t nwarps = (int64_t)gridDim.x * kRowWarps;
+  for (int64_t row = (int64_t)blockIdx.x * kRowWarps + (threadIdx.x >> 5); row < a.T;
+       row += nwarps) {
+    const float mean = a.mean[row], rstd = a.rstd[row];
+    float xh[NV][8], g[NV][8];
+    float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+    for (int v = 0; v < NV; ++v) {
+      const int c = 8 * (lane + 32 * v);
+      float x[8], dy[8];
+      load8(a.x + row * a.ldx + c, x);
+      load8(a.dy + row * a.lddy + c, dy);
+      float u[8], pu[8], du[8];
+      if (GATED) {
+        load8(a.u + row * a.ldu + c, u);
+        load8(a.pre_u + row * a.ldpu + c, pu);
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        xh[v][e] = (x[e] - mean) * rstd;
+        float dz = dy[e];
+        if (GATED) {
+          const float z = a.gamma[c + e] * xh[v][e] + a.beta[c + e];
+          du[e] = dy[e] * z * silu_grad(pu[e]);
+          dz = dy[e] * u[e];
+        }
+        dg[v][e] += dz * xh[v][e];
+        db[v][e] += dz;
+        g[v][e] = dz * a.gamma[c + e];
+        s1 += g[v][e];
+        s2 += g[v][e] * xh[v][e];
+      }
+      if (GATED) store8(a.du + row * a.lddu + c, du);
+    }
+    const float m1 = warp_sum(s1) * (1.0f / W), m2 = warp_sum(s2) * (1.0f / W);
+#pragma unroll
+    for (int v = 0; v < NV; ++v) {
+      const int c = 8 * (lane + 32 * v);
+      float dx[8], r[8];
+      if (a.resid_grad) load8(a.resid_grad + row * a.ldr + c, r);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        dx[e] = rstd * (g[v][e] - m1 - xh[v][e] * m2);
+        if (a.resid_grad) dx[e] += r[e];
+      }
+      store8(a.dx + row * a.lddx + c, dx);
+    }
+  }
+#pragma unroll
+  for (int v = 0; v < NV; ++v) {
+    const int c = 8 * (lane + 32 * v);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      atomicAdd(a.dgamma + c + e, dg[v][e]);
+      atomicAdd(a.dbeta + c + e, db[v][e]);
+    }
+  }
+}
+
+// Column-parallel pass over [T][W]: thread t owns columns [8t, 8t + 8) of the
+// rows of its block's chunk.  SCALE multiplies columns >= c0 by SiLU'(pre) in
+// place; every column's (scaled) values are summed into dbias.
+constexpr int kColRows = 64;
+template <bool SCALE>
+__global__ void colsum_kernel(bf16* g, int64_t ldg, const bf16* pre, int64_t ldp, int64_t T,
+                              int W, int c0, float* dbias) {
+  const int c = 8 * threadIdx.x;
+  if (c >= W) return;
+  const int64_t r0 = (int64_t)blockIdx.x * kColRows;
+  const int64_t r1 = r0 + kColRows < T ? r0 + kColRows : T;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int64_t r = r0; r < r1; ++r) {
+    float v[8];
+    load8(g + r * ldg + c, v);
+    if (SCALE && c >= c0) {
+      float p[8];
+      load8(pre + r * ldp + c, p);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] *= silu_grad(p[e]);
+      store8(g + r * ldg + c, v);
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] += v[e];
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) atomicAdd(dbias + c + e, acc[e]);
+}
+
+// New offsets after truncation (one thread; B is small).
+__global__ void trunc_offsets_kernel(const int32_t* offs, const int32_t* nts, int B, int c,
+                                     int tail, int32_t* new_offs) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  int32_t o = 0;
+  new_offs[0] = 0;
+  for (int b = 0; b < B; ++b) {
+    const int L = offs[b + 1] - offs[b];
+    const int Lh = L - (nts ? nts[b] : 0);
+    const int drop = Lh - c - tail > 0 ? Lh - c - tail : 0;
+    o += L - drop;
+    new_offs[b + 1] = o;
+  }
+}
+
+__device__ __forceinline__ int find_seq(const int32_t* offs, int B, int64_t r) {
+  int lo = 0, hi = B;  // offs[lo] <= r < offs[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (offs[mid] <= r) lo = mid; else hi = mid;
+  }
+  return lo;
+}
+
+// Gather (rows of the truncated layout from the full one) or scatter (rows of
+// the full layout from the truncated one; dropped rows become zero).  One warp
+// per output row.
+__global__ void __launch_bounds__(256) trunc_rows_kernel(const bf16* src, int64_t lds,
+                                                         const int32_t* offs,
+                                                         const int32_t* new_offs,
+                                                         const int32_t* nts, int B, int c,
+                                                         int tail, int W, bf16* dst, int64_t ldd,
+                                                         int64_t T_out, int scatter) {
+  const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (r >= T_out) return;
+  const int32_t* out_offs = scatter ? offs : new_offs;
+  const int32_t* in_offs = scatter ? new_offs : offs;
+  const int b = find_seq(out_offs, B, r);
+  const int L = offs[b + 1] - offs[b];
+  const int Lh = L - (nts ? nts[b] : 0);
+  const int drop = Lh - c - tail > 0 ? Lh - c - tail : 0;
+  const int p = (int)(r - out_offs[b]);
+  int64_t s;  // source row, or -1 for a dropped row (scatter)
+  if (scatter) s = (p < c || p >= c + drop) ? in_offs[b] + p - (p >= c ? drop : 0) : -1;
+  else s = in_offs[b] + p + (p >= c ? drop : 0);
+  uint4* d = reinterpret_cast<uint4*>(dst + r * ldd);
+  const uint4* q = s >= 0 ? reinterpret_cast<const uint4*>(src + s * lds) : nullptr;
+  for (int j = lane; j < W / 8; j += 32) d[j] = q ? q[j] : make_uint4(0, 0, 0, 0);
+}
+
+}  // namespace
+
+cudaError_t launch_ln_fwd(const LnArgs& a, bool gated, cudaStream_t st) {
+  if (a.T == 0) return cudaSuccess;
+  const int grid = (int)((a.T + kRowWarps - 1) / kRowWarps);
+#define HSTU_LN(NV)                                                                     \
+  if (a.W == NV * 256) {                                                                \
+    if (gated) ln_fwd_kernel<NV, true><<<grid, 32 * kRowWarps, 0, st>>>(a);             \
+    else ln_fwd_kernel<NV, false><<<grid, 32 * kRowWarps, 0, st>>>(a);                  \
+    return cudaGetLastError();                                                          \
+  }
+  HSTU_LN(1) HSTU_LN(2) HSTU_LN(4)
+#undef HSTU_LN
+  return cudaErrorNotSupported;
+}
+
+cudaError_t launch_ln_bwd(const LnArgs& a, bool gated, cudaStream_t st) {
+  if (a.T == 0) return cudaSuccess;
+  const int64_t need = (a.T + kRowWarps - 1) / kRowWarps;
+  const int cap = device_sm_count() * 8;  // rows per warp grow past this
+  const int grid = (int)(need < cap ? need : cap);
+#define HSTU_LNB(NV)                                                                    \
+  if (a.W == NV * 256) {                                                                \
+    if (gated) ln_bwd_kernel<NV, true><<<grid, 32 * kRowWarps, 0, st>>>(a);             \
+    else ln_bwd_kernel<NV, false><<<grid, 32 * kRowWarps, 0, st>>>(a);                  \
+    return cudaGetLastError();                                                          \
+  }
+  HSTU_LNB(1) HSTU_LNB(2) HSTU_LNB(4)
+#undef HSTU_LNB
+  return cudaErrorNotSupported;
+}
+
+cudaError_t launch_silu_bwd_colsum(bf16* g, int64_t ldg, const bf16* pre, int64_t ldp, int64_t T,
+                                   int W, int c0, float* dbias, cudaStream_t st) {
+  if (T == 0) return cudaSuccess;
+  if (W % 8 != 0 || W / 8 > 1024) return cudaErrorNotSupported;
+  const int grid = (int)((T + kColRows - 1) / kColRows);
+  colsum_kernel<true><<<grid, W / 8, 0, st>>>(g, ldg, pre, ldp, T, W, c0, dbias);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_colsum(const bf16* g, int64_t ldg, int64_t T, int W, float* dbias,
+                          cudaStream_t st) {
+  if (T == 0) return cudaSuccess;
+  if (W % 8 != 0 || W / 8 > 1024) return cudaErrorNotSupported;
+  const int grid = (int)((T + kColRows - 1) / kColRows);
+  colsum_kernel<false><<<grid, W / 8, 0, st>>>(const_cast<bf16*>(g), ldg, nullptr, 0, T, W, W,
+                                               dbias);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_trunc_offsets(const int32_t* offs, const int32_t* nts, int B, int c, int tail,
+                                 int32_t* new_offs, cudaStream_t st) {
+  trunc_offsets_kernel<<<1, 32, 0, st>>>(offs, nts, B, c, tail, new_offs);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_trunc_rows(const bf16* src, int64_t lds, const int32_t* offs,
+                              const int32_t* new_offs, const int32_t* nts, int B, int c, int tail,
+                              int W, bf16* dst, int64_t ldd, int64_t T_out, bool scatter,
+                              cudaStream_t st) {
+  if (T_out == 0) return cudaSuccess;
+  const int grid = (int)((T_out + 7) / 8);
+  trunc_rows_kernel<<<grid, 256, 0, st>>>(src, lds, offs, new_offs, nts, B, c, tail, W, dst, ldd,
+                                          T_out, scatter ? 1 : 0);
+  return cudaGetLastError();
+}
+
+}  // namespace hstu

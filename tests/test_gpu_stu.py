@@ -1,0 +1,149 @@
+"""GPU parity of the STU layer around the SLA attention: the tcgen05 GEMM in
+every operand layout / epilogue the layer uses, one full layer forward +
+backward, the truncation gather / scatter, and the 6-layer truncated stack,
+each against oracle/stu.py (fp64) on the same seeded bf16 inputs."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import stu as S
+from parity import assert_close
+from sparse_hstu_attention_b200 import _abi, stu
+from workloads import STU_LAYERS, STU_TRUNC_AFTER, draw_stu, offsets_from_lengths
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda")
+FIELDS = ("ln1_w", "ln1_b", "w1", "b1", "ln2_w", "ln2_b", "w2", "b2")
+
+
+def f64(t):
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+GEMM_CASES = [  # (a_mn, b_mn, epilogue, M, N, K, splits)
+    (False, True, _abi.GEMM_BIAS_SILU, 300, 512, 512, 1),
+    (False, True, _abi.GEMM_BIAS_RESID, 300, 512, 512, 1),
+    (False, True, _abi.GEMM_STORE, 129, 1024, 256, 1),
+    (False, False, _abi.GEMM_STORE, 300, 512, 2048, 1),
+    (True, True, _abi.GEMM_RED_F32, 512, 2048, 1000, 4),
+    (True, True, _abi.GEMM_RED_F32, 256, 512, 77, 3),
+    (False, False, _abi.GEMM_RED_F32, 300, 256, 640, 2),
+]
+
+
+@pytest.mark.parametrize("a_mn,b_mn,epi,M,N,K,splits", GEMM_CASES)
+def test_gemm_layouts_and_epilogues(a_mn, b_mn, epi, M, N, K, splits):
+    g = torch.Generator().manual_seed(M * 7 + N + K)
+    A = torch.randn((K, M) if a_mn else (M, K), generator=g).to(torch.bfloat16)
+    B = torch.randn((K, N) if b_mn else (N, K), generator=g).to(torch.bfloat16)
+    bias = torch.randn(N, generator=g)
+    resid = torch.randn((M, N), generator=g).to(torch.bfloat16)
+    acc0 = torch.randn((M, N), generator=g)
+    a64 = f64(A).T if a_mn else f64(A)
+    b64 = f64(B).T if b_mn else f64(B)
+    ref = a64 @ b64.T                       # D[m][n] = sum_k A[m][k] B[n][k]
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=DEV)
+    out2 = torch.empty((M, N), dtype=torch.bfloat16, device=DEV)
+    outf = acc0.to(DEV)
+    stu.gemm(A.to(DEV), B.to(DEV), M=M, N=N, K=K, a_mn_major=a_mn, b_mn_major=b_mn,
+             epilogue=epi, splits=splits, bias=bias.to(DEV), resid=resid.to(DEV), out=out,
+             out2=out2, outf=outf)
+    torch.cuda.synchronize()
+    pre = ref + f64(bias)
+    if epi == _abi.GEMM_STORE:
+        assert_close("D", out, ref)
+    elif epi == _abi.GEMM_BIAS_SILU:
+        assert_close("D + bias", out2, pre)
+        assert_close("SiLU(D + bias)", out, S.silu(pre))
+    elif epi == _abi.GEMM_BIAS_RESID:
+        assert_close("D + bias + resid", out, pre + f64(resid))
+    else:
+        assert_close("acc + D", outf, f64(acc0) + ref, tol=1e-4)
+
+
+def _cfgs(lengths, nts, c, K1, K2, tail, trunc=True):
+    H, d = 4, 128
+    alpha = 1.0 / math.sqrt(d)
+    tl = stu.truncated_lengths(lengths, nts, c, tail)
+    full = stu.StuConfig(H, d, c, K1, K2, alpha, float(max(lengths)))
+    cut = stu.StuConfig(H, d, c, K1, K2, alpha, float(max(tl)))
+    return full, cut, tl
+
+
+def _oracle_cfg(c: stu.StuConfig):
+    return S.AttnCfg(c.H, c.d, c.contextual_len, c.K1, c.K2, c.alpha, c.N, c.ln_eps)
+
+
+def _oracle_weights(lw):
+    return S.Weights.of(**{k: f64(lw[k]) for k in FIELDS})
+
+
+def test_stu_layer_matches_oracle():
+    lengths, nts = np.array([300, 520, 180]), np.array([16, 10, 5])
+    full, _, _ = _cfgs(lengths, nts, c=8, K1=128, K2=32, tail=64)
+    offs = offsets_from_lengths(lengths)
+    T = int(offs[-1])
+    dr = draw_stu(T, T, full.d_model, 1, seed=2024, perturb=True)
+    w = stu.StuWeights.from_host(dr.layers[0], DEV)
+    offs_d = torch.tensor(offs, dtype=torch.int32, device=DEV)
+    nts_d = torch.tensor(nts, dtype=torch.int32, device=DEV)
+    out, st = stu.layer_fwd(dr.x.to(DEV), offs_d, nts_d, w, full, int(lengths.max()))
+    dx, g = stu.layer_bwd(dr.dout.to(DEV), st, w, full)
+    torch.cuda.synchronize()
+    wo = _oracle_weights(dr.layers[0])
+    ref, cache = S.layer_fwd(f64(dr.x), wo, offs, nts, _oracle_cfg(full))
+    rdx, rg = S.layer_bwd(f64(dr.dout), wo, cache)
+    assert_close("out", out, ref)
+    assert_close("dx", dx, rdx)
+    for name in FIELDS:
+        assert_close("d_" + name, getattr(g, name), getattr(rg, name))
+
+
+def test_truncation_gather_and_scatter_are_exact():
+    lengths, nts = np.array([300, 40, 1200, 77]), np.array([16, 3, 64, 0])
+    c, tail = 8, 100
+    offs = offsets_from_lengths(lengths)
+    T = int(offs[-1])
+    x = torch.randn((T, 512), generator=torch.Generator().manual_seed(1)).to(torch.bfloat16)
+    idx, new = S.truncation_index(offs, nts, c, tail)
+    offs_d = torch.tensor(offs, dtype=torch.int32, device=DEV)
+    nts_d = torch.tensor(nts, dtype=torch.int32, device=DEV)
+    new_d = stu.truncate_offsets(offs_d, nts_d, c, tail)
+    y = stu.jagged_truncate(x.to(DEV), offs_d, new_d, nts_d, c, tail, len(idx))
+    torch.cuda.synchronize()
+    assert np.array_equal(new_d.cpu().numpy(), new)
+    assert torch.equal(y.cpu(), x[torch.from_numpy(idx)])
+    z = stu.jagged_truncate(y, offs_d, new_d, nts_d, c, tail, T, scatter=True)
+    ref = torch.zeros_like(x)
+    ref[torch.from_numpy(idx)] = x[torch.from_numpy(idx)]
+    assert torch.equal(z.cpu(), ref)
+
+
+def test_stu_stack_matches_oracle():
+    """Six layers, truncation after the third to contextual + the last `tail`
+    history tokens + candidates, every gradient compared."""
+    lengths, nts = np.array([700, 400, 1100]), np.array([20, 8, 30])
+    c, tail = 16, 128
+    full, cut, tl = _cfgs(lengths, nts, c=c, K1=128, K2=32, tail=tail)
+    offs = offsets_from_lengths(lengths)
+    T, T_out = int(offs[-1]), int(tl.sum())
+    dr = draw_stu(T, T_out, full.d_model, STU_LAYERS, seed=77, perturb=True)
+    ws = [stu.StuWeights.from_host(lw, DEV) for lw in dr.layers]
+    stack = stu.StuStack(ws, full, cut, STU_TRUNC_AFTER, tail)
+    offs_d = torch.tensor(offs, dtype=torch.int32, device=DEV)
+    nts_d = torch.tensor(nts, dtype=torch.int32, device=DEV)
+    out, ctx = stack.forward(dr.x.to(DEV), offs_d, nts_d, lengths, nts)
+    dx, gs = stack.backward(dr.dout.to(DEV), ctx)
+    torch.cuda.synchronize()
+    wo = [_oracle_weights(lw) for lw in dr.layers]
+    ref, cache = S.stack_fwd(f64(dr.x), wo, offs, nts, _oracle_cfg(full), _oracle_cfg(cut),
+                             STU_TRUNC_AFTER, tail)
+    rdx, rgs = S.stack_bwd(f64(dr.dout), wo, cache)
+    assert out.shape[0] == T_out
+    assert_close("out", out, ref)
+    assert_close("dx", dx, rdx)
+    for i in range(STU_LAYERS):
+        for name in FIELDS:
+            assert_close(f"layer {i} d_{name}", getattr(gs[i], name), getattr(rgs[i], name))

@@ -139,3 +139,55 @@ def make_batch(w: Workload, lengths=None, num_targets=None, seed: Optional[int] 
 def with_params(w: Workload, **kw) -> Workload:
     """A copy of a workload with some fields changed (edge cases)."""
     return dataclasses.replace(w, **kw)
+
+
+# ----------------------------------------------------------------- STU stack
+# The 6-layer STU stack workload: d_model = H * d = 512, truncation after
+# layer 3 to contextual + the last 1024 history tokens + the candidates
+# (TorchEasyRec "ULTRA HSTU" docs: attn_truncation_tail_len), N = the longest
+# sequence of each stage.
+STU_LAYERS = 6
+STU_TRUNC_AFTER = 3
+STU_TAIL = 1024
+
+
+@dataclasses.dataclass
+class StuDraw:
+    """Seeded inputs of an STU stack: x, the upstream gradient of the stack
+    output, and each layer's parameters as CPU tensors (projections bf16 in
+    the x W convention, the rest fp32)."""
+    x: torch.Tensor                 # bf16 [T, d_model]
+    dout: torch.Tensor              # bf16 [T_out, d_model]
+    layers: list                    # per layer: dict of CPU tensors
+
+
+def draw_stu(T: int, T_out: int, d_model: int, n_layers: int, seed: int,
+             perturb: bool = False) -> StuDraw:
+    """x, dout ~ N(0, 1); W1 [d_model, 4 d_model] and W2 [d_model, d_model]
+    Xavier-uniform (bound sqrt(6 / (fan_in + fan_out))); biases 0 and
+    LayerNorm weight 1 / bias 0, or (perturb=True, to exercise those terms)
+    biases ~ 0.1 N(0, 1) and LayerNorm weight 1 + 0.1 N(0, 1), bias 0.1 N(0, 1).
+    Draw order: x, dout, then per layer W1, W2, then the perturbations."""
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    x = torch.randn((T, d_model), generator=g).to(torch.bfloat16)
+    dout = torch.randn((T_out, d_model), generator=g).to(torch.bfloat16)
+
+    def xavier(fi, fo):
+        a = math.sqrt(6.0 / (fi + fo))
+        return ((torch.rand((fi, fo), generator=g) * 2 - 1) * a).to(torch.bfloat16)
+
+    layers = []
+    for _ in range(n_layers):
+        lw = dict(w1=xavier(d_model, 4 * d_model), w2=xavier(d_model, d_model),
+                  ln1_w=torch.ones(d_model), ln1_b=torch.zeros(d_model),
+                  b1=torch.zeros(4 * d_model), ln2_w=torch.ones(d_model),
+                  ln2_b=torch.zeros(d_model), b2=torch.zeros(d_model))
+        layers.append(lw)
+    if perturb:
+        for lw in layers:
+            for k in ("ln1_w", "ln2_w"):
+                lw[k] = 1.0 + 0.1 * torch.randn(d_model, generator=g)
+            for k in ("ln1_b", "ln2_b", "b2"):
+                lw[k] = 0.1 * torch.randn(d_model, generator=g)
+            lw["b1"] = 0.1 * torch.randn(4 * d_model, generator=g)
+    return StuDraw(x, dout, layers)
