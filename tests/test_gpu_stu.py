@@ -147,3 +147,56 @@ def test_stu_stack_matches_oracle():
     for i in range(STU_LAYERS):
         for name in FIELDS:
             assert_close(f"layer {i} d_{name}", getattr(gs[i], name), getattr(rgs[i], name))
+
+
+def test_stu_stack_full_size_sampled():
+    """The 6-layer STU stack workload at full size (16 sequences of
+    U{4096..16384} tokens, truncation to 32 + 1024 + 64 after layer 3), forward
+    and backward on the GPU.  The oracle checks, teacher-forced with the GPU's
+    own layer inputs, layer 1 on the shortest sequence and layer 6 (forward
+    and its dx) on the longest truncated one; every output and gradient must
+    be finite."""
+    from workloads import STU_TAIL, WORKLOADS, draw_lengths
+    w = WORKLOADS["stu"]
+    lengths = draw_lengths(w)
+    nts = np.minimum(np.full(len(lengths), w.num_targets), lengths)
+    c, tail = w.contextual_len, STU_TAIL
+    tl = stu.truncated_lengths(lengths, nts, c, tail)
+    full = stu.StuConfig(w.H, w.d, c, w.K1, w.K2, w.alpha, w.N)
+    cut = stu.StuConfig(w.H, w.d, c, w.K1, w.K2, w.alpha, float(c + tail + w.num_targets))
+    offs = offsets_from_lengths(lengths)
+    T, T_out = int(offs[-1]), int(tl.sum())
+    dr = draw_stu(T, T_out, full.d_model, STU_LAYERS, seed=w.seed)
+    ws = [stu.StuWeights.from_host(lw, DEV) for lw in dr.layers]
+    stack = stu.StuStack(ws, full, cut, STU_TRUNC_AFTER, tail)
+    offs_d = torch.tensor(offs, dtype=torch.int32, device=DEV)
+    nts_d = torch.tensor(nts, dtype=torch.int32, device=DEV)
+    out, ctx = stack.forward(dr.x.to(DEV), offs_d, nts_d, lengths, nts)
+    dx, gs = stack.backward(dr.dout.to(DEV), ctx)
+    torch.cuda.synchronize()
+    states = ctx[0]
+    for t in [out, dx] + [getattr(g, f) for g in gs for f in FIELDS]:
+        assert torch.isfinite(t.float()).all()
+    wo = [_oracle_weights(lw) for lw in dr.layers]
+    # layer 1 on the shortest sequence
+    b = int(np.argmin(lengths))
+    s0, s1 = int(offs[b]), int(offs[b + 1])
+    one = np.array([0, s1 - s0])
+    ref1, _ = S.layer_fwd(f64(dr.x[s0:s1]), wo[0], one, nts[b:b + 1], _oracle_cfg(full))
+    assert_close("layer 1 out", states[1].x[s0:s1], ref1)
+    # layer 6 on the longest truncated sequence, fed the GPU's layer-6 input
+    new = offsets_from_lengths(tl)
+    b = int(np.argmax(tl))
+    s0, s1 = int(new[b]), int(new[b + 1])
+    one = np.array([0, s1 - s0])
+    x6 = f64(states[5].x[s0:s1])
+    ref6, cache6 = S.layer_fwd(x6, wo[5], one, nts[b:b + 1], _oracle_cfg(cut))
+    assert_close("layer 6 out", out[s0:s1], ref6)
+    rdx6, _ = S.layer_bwd(f64(dr.dout[s0:s1]), wo[5], cache6)
+    gdx6, _ = stu.layer_bwd(dr.dout[s0:s1].to(DEV).contiguous(), stu.LayerState(
+        states[5].x[s0:s1], torch.tensor(one, dtype=torch.int32, device=DEV),
+        nts_d[b:b + 1], int(tl[b]), *(t[s0:s1].contiguous() for t in (
+            states[5].xn, states[5].pre, states[5].uvqk, states[5].av, states[5].y)),
+        states[5].stats[:, s0:s1].contiguous()), ws[5], cut)
+    torch.cuda.synchronize()
+    assert_close("layer 6 dx", gdx6, rdx6)
