@@ -8,8 +8,8 @@ import torch
 import sparse_hstu_attention_b200 as sla
 from workloads import WORKLOADS, make_batch, with_params
 
-from parity import (TOL, assert_close, gpu_bwd, gpu_fwd, oracle_problem, sample_tokens,
-                    to_gpu)
+from parity import (TOL, assert_close, gpu_bwd, gpu_fwd, kwargs_of, oracle_problem,
+                    sample_tokens, to_gpu)
 
 pytestmark = pytest.mark.gpu
 
@@ -105,6 +105,25 @@ def test_repeat_calls_reproducible(d):
         assert ((a1 - a2).abs() <= bound).all()
     else:
         assert torch.equal(q1, q2)
+
+
+def test_backward_reuses_a_workspace():
+    """One workspace reused across backward calls (same batch, a larger one,
+    the first again) gives the oracle's results every time."""
+    b1 = _edge_batch(lengths=[300, 200, 1000], nt=10)
+    b2 = _edge_batch(lengths=[700, 64, 1500, 90], nt=5, seed=9)
+    need = max(sla.hstu_sla_workspace_bytes(1, b.T, len(b.lengths), 2, 128) for b in (b1, b2))
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    for b in (b1, b1, b2, b1):
+        g = to_gpu(b)
+        dq, dk, dv = sla.hstu_sla_bwd(g["dout"], g["q"], g["k"], g["v"], g["offs"], g["nts"],
+                                      workspace=ws, **kwargs_of(b))
+        assert sla.hstu_sla_get_error(ws) == 0
+        p = oracle_problem(b)
+        rq, rk, rv = p.bwd(b.q, b.k, b.v, b.dout)
+        assert_close("dq", dq, rq)
+        assert_close("dk", dk, rk)
+        assert_close("dv", dv, rv)
 
 
 @pytest.mark.parametrize("wname", ["mid", "hist16k"])
