@@ -249,6 +249,87 @@ def _config(w, batch):
             "l2": f"inputs {in_bytes / 1e6:.0f} MB > 126 MB L2; no flush"}
 
 
+def run_stu(args, world, rank, local):
+    """The 6-layer STU stack workload (truncation after layer 3): one step is
+    the stack's forward and backward, every parameter gradient included."""
+    from sparse_hstu_attention_b200 import stu
+    from workloads import (STU_LAYERS, STU_TAIL, STU_TRUNC_AFTER, draw_lengths, draw_stu,
+                           offsets_from_lengths)
+    dev = torch.device("cuda", local)
+    w = WORKLOADS["stu"]
+    lengths = draw_lengths(w)
+    nts = np.minimum(np.full(len(lengths), w.num_targets), lengths)
+    c, tail = w.contextual_len, STU_TAIL
+    tl = stu.truncated_lengths(lengths, nts, c, tail)
+    full = stu.StuConfig(w.H, w.d, c, w.K1, w.K2, w.alpha, w.N)
+    cut = stu.StuConfig(w.H, w.d, c, w.K1, w.K2, w.alpha, float(c + tail + w.num_targets))
+    offs = offsets_from_lengths(lengths)
+    T, T_out, dm = int(offs[-1]), int(tl.sum()), full.d_model
+    dr = draw_stu(T, T_out, dm, STU_LAYERS, seed=w.seed + 7919 * rank)
+    ws = [stu.StuWeights.from_host(lw, dev) for lw in dr.layers]
+    stack = stu.StuStack(ws, full, cut, STU_TRUNC_AFTER, tail)
+    offs_d = torch.tensor(offs, dtype=torch.int32, device=dev)
+    nts_d = torch.tensor(nts, dtype=torch.int32, device=dev)
+    x, dout = dr.x.to(dev), dr.dout.to(dev)
+    # FLOPs: per layer the two projections (2 T dm (4 dm + dm)) forward and
+    # twice that backward (input and weight gradients); attention 4d / 10d
+    # per unmasked pair per head
+    p_full = F.total_pairs(lengths, nts, c, w.K1, w.K2)
+    p_cut = F.total_pairs(tl, nts, c, w.K1, w.K2)
+    n_full, n_cut = STU_TRUNC_AFTER, STU_LAYERS - STU_TRUNC_AFTER
+    gemm = 3 * 2 * dm * 5 * dm * (n_full * T + n_cut * T_out)
+    attn = (F.fwd_flops(p_full, w.H, w.d) + F.bwd_flops(p_full, w.H, w.d)) * n_full + \
+           (F.fwd_flops(p_cut, w.H, w.d) + F.bwd_flops(p_cut, w.H, w.d)) * n_cut
+
+    def step():
+        out, ctx = stack.forward(x, offs_d, nts_d, lengths, nts)
+        stack.backward(dout, ctx)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    K = args.steps
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        t0.record()
+        for _ in range(K):
+            step()
+        t1.record()
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+    ms = t0.elapsed_time(t1) / K
+    if world > 1:
+        tt = torch.tensor([ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        ms = float(tt.item())
+    if rank == 0:
+        peaks, src = _peaks()
+        peak = float(peaks.get("bf16_tflops_sustained") or peaks.get("bf16_tflops"))
+        value = world * (gemm + attn) / (ms * 1e-3) / 1e12
+        print(json.dumps({
+            "metric": "STU stack fwd+bwd TFLOP/s (projections + SLA attention over unmasked pairs)",
+            "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) inputs, Xavier-uniform weights)",
+            "config": {"workload": "stu", "layers": STU_LAYERS, "trunc_after": STU_TRUNC_AFTER,
+                       "tail": tail, "B": int(len(lengths)), "T": T, "T_truncated": T_out,
+                       "d_model": dm, "H": w.H, "d": w.d, "K1": w.K1, "K2": w.K2,
+                       "contextual_len": c, "num_targets": w.num_targets,
+                       "N": [w.N, cut.N]},
+            "flops_per_step": {"projections": gemm, "attention": attn},
+            "frac_of_sustained_peak": value / world / peak,
+            "gpu_launches": K * (STU_LAYERS * (6 + 11) + 3),
+            "clocks": clocks.summary()}), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -267,6 +348,8 @@ def main():
 
     world, rank, local = _setup_dist(args)
     torch.cuda.set_device(local)
+    if args.workload == "stu":
+        return run_stu(args, world, rank, local)
     dev = torch.device("cuda", local)
     w = WORKLOADS[args.workload]
     batch = make_batch(w, seed=w.seed + 7919 * rank)

@@ -23,7 +23,8 @@
 // Persistent CTAs walk tiles (split, m block, n block) with n fastest, so
 // consecutive tiles share their A rows in L2.
 // Roles: warp 0 TMA producer, warp 1 TMEM allocation + one MMA-issuing lane,
-// warps 2..5 epilogue (warp w reads TMEM lanes 32 (w % 4) .. +32).
+// warps 2..9 epilogue (warp w reads TMEM lanes 32 (w % 4) .. +32 and half of
+// the tile's columns).
 #include <cudaTypedefs.h>
 
 #include "sm100.cuh"
@@ -40,7 +41,8 @@ namespace {
 using namespace sm100;
 
 constexpr int kBM = 128, kBN = 256, kBK = 64, kStages = 4;
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;  // two per TMEM lane quarter, each half of the tile's columns
+constexpr int kThreads = 32 * (2 + kEpiWarps);
 constexpr int A_TILE = kBM * kBK * 2;  // 16 KB
 constexpr int B_TILE = kBN * kBK * 2;  // 32 KB
 constexpr int MN_BOX = 64 * kBK * 2;   // one 64 (M or N) x 64 (K) box of an MN-major tile
@@ -83,7 +85,13 @@ __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, 
       : "memory");
 }
 
-__device__ __forceinline__ float silu_f(float v) { return v / (1.0f + __expf(-v)); }
+// SiLU(v) = h + h tanh(h) with h = v / 2 (one MUFU op)
+__device__ __forceinline__ float silu_f(float v) {
+  float t;
+  const float h = 0.5f * v;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(h));
+  return fmaf(h, t, h);
+}
 
 template <bool A_MN, bool B_MN, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -108,7 +116,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(G_ACC_FULL + b), 1);
-      mbar_init(bar(G_ACC_EMPTY + b), 4);  // the four epilogue warps
+      mbar_init(bar(G_ACC_EMPTY + b), kEpiWarps);
     }
     fence_barrier_init();
     prefetch_tmap(&tma);
@@ -200,6 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ----------------------------------------------------------- epilogue
     const int quarter = warp & 3;
+    const int col0 = ((warp - 2) >> 2) * (kBN / 2);  // this warp's half of the columns
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     uint32_t tc = 0;
     bool ok = true;
@@ -213,11 +222,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int m = ti.m0 + quarter * 32 + lane;
       const bool live = m < g.M;
 #pragma unroll 1
-      for (int c = 0; c < kBN; c += 32) {
+      for (int c = col0; c < col0 + kBN / 2; c += 32) {
         uint32_t v[32];
         tmem_ld32(lane_base + buf * kBN + c, v);
         tmem_ld_wait(v);
-        if (c + 32 == kBN) {  // accumulator read out: the next tile may start
+        if (c + 32 == col0 + kBN / 2) {  // this warp's share read out
           tc_fence_before();
           warp_arrive(bar(G_ACC_EMPTY + buf));
         }

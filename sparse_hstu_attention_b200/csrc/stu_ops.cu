@@ -90,103 +90,155 @@ __global__ void __launch_bounds__(32 * kRowWarps) ln_fwd_kernel(const LnArgs a) 
 
 // Backward of the above.  Plain: dx = resid_grad + LN'(dy * gamma).
 // Gated: dz = dy * u, du = dy * z (times SiLU'(pre_u), since the gate is a
-// SiLU output), dx = LN'(dz * gamma).  dgamma / dbeta accumulate per lane
-// over the rows a warp visits, then once into global memory.
+// SiLU output), dx = LN'(dz * gamma).  Two passes over each row (the second
+// re-reads x, dy, u from L1 instead of keeping them in registers, so many
+// warps fit per SM); dgamma / dbeta accumulate in shared memory over the
+// rows a block visits (per warp, each lane updating only its own columns, for
+// W <= 512; shared atomics beyond), then once per block and column in global
+// memory.
 template <int NV, bool GATED>
-__global__ void __launch_bounds__(32 * kRowWarps) ln_bwd_kernel(const LnArgs a) {
+__global__ void __launch_bounds__(32 * kRowWarps, 2) ln_bwd_kernel(const LnArgs a) {
   constexpr int W = NV * 256;
+  constexpr bool kPerWarp = NV <= 2;
+  constexpr int kAcc = kPerWarp ? kRowWarps : 1;
+  __shared__ __align__(16) float s_g[W], s_b[W], s_dg[kAcc][W], s_db[kAcc][W];
+  for (int c = threadIdx.x; c < W; c += blockDim.x) {
+    s_g[c] = a.gamma[c];
+    s_b[c] = a.beta[c];
+    for (int w = 0; w < kAcc; ++w) s_dg[w][c] = s_db[w][c] = 0.f;
+  }
+  __syncthreads();
   const int lane = threadIdx.x & 31;
-  float dg[NV][8], db[NV][8];
-#pragma unroll
-  for (int v = 0; v < NV; ++v)
-#pragma unroll
-    for (int e = 0; e < 8; ++e) dg[v][e] = db[v][e] = 0.f;
+  float* my_dg = s_dg[kPerWarp ? (threadIdx.x >> 5) : 0];
+  float* my_db = s_db[kPerWarp ? (threadIdx.x >> 5) : 0];
   const int64_t nwarps = (int64_t)gridDim.x * kRowWarps;
   for (int64_t row = (int64_t)blockIdx.x * kRowWarps + (threadIdx.x >> 5); row < a.T;
        row += nwarps) {
     const float mean = a.mean[row], rstd = a.rstd[row];
-    float xh[NV][8], g[NV][8];
     float s1 = 0.f, s2 = 0.f;
-#pragma unroll
+#pragma unroll 1
     for (int v = 0; v < NV; ++v) {
       const int c = 8 * (lane + 32 * v);
-      float x[8], dy[8];
+      float x[8], dy[8], u[8], pu[8], du[8], tg[8], tb[8];
       load8(a.x + row * a.ldx + c, x);
       load8(a.dy + row * a.lddy + c, dy);
-      float u[8], pu[8], du[8];
       if (GATED) {
         load8(a.u + row * a.ldu + c, u);
         load8(a.pre_u + row * a.ldpu + c, pu);
       }
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        xh[v][e] = (x[e] - mean) * rstd;
+        const float xh = (x[e] - mean) * rstd;
         float dz = dy[e];
         if (GATED) {
-          const float z = a.gamma[c + e] * xh[v][e] + a.beta[c + e];
-          du[e] = dy[e] * z * silu_grad(pu[e]);
+          du[e] = dy[e] * (s_g[c + e] * xh + s_b[c + e]) * silu_grad(pu[e]);
           dz = dy[e] * u[e];
         }
-        dg[v][e] += dz * xh[v][e];
-        db[v][e] += dz;
-        g[v][e] = dz * a.gamma[c + e];
-        s1 += g[v][e];
-        s2 += g[v][e] * xh[v][e];
+        tg[e] = dz * xh;
+        tb[e] = dz;
+        const float g = dz * s_g[c + e];
+        s1 += g;
+        s2 += g * xh;
+      }
+      if (kPerWarp) {  // this lane's own 8 columns of its warp's row
+        float4* pg = reinterpret_cast<float4*>(my_dg + c);
+        float4* pb = reinterpret_cast<float4*>(my_db + c);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          float4 g4 = pg[h], b4 = pb[h];
+          g4.x += tg[4 * h]; g4.y += tg[4 * h + 1]; g4.z += tg[4 * h + 2]; g4.w += tg[4 * h + 3];
+          b4.x += tb[4 * h]; b4.y += tb[4 * h + 1]; b4.z += tb[4 * h + 2]; b4.w += tb[4 * h + 3];
+          pg[h] = g4;
+          pb[h] = b4;
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          atomicAdd(my_dg + c + e, tg[e]);
+          atomicAdd(my_db + c + e, tb[e]);
+        }
       }
       if (GATED) store8(a.du + row * a.lddu + c, du);
     }
     const float m1 = warp_sum(s1) * (1.0f / W), m2 = warp_sum(s2) * (1.0f / W);
-#pragma unroll
+#pragma unroll 1
     for (int v = 0; v < NV; ++v) {
       const int c = 8 * (lane + 32 * v);
-      float dx[8], r[8];
+      float x[8], dy[8], u[8], dx[8], r[8];
+      load8(a.x + row * a.ldx + c, x);
+      load8(a.dy + row * a.lddy + c, dy);
+      if (GATED) load8(a.u + row * a.ldu + c, u);
       if (a.resid_grad) load8(a.resid_grad + row * a.ldr + c, r);
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        dx[e] = rstd * (g[v][e] - m1 - xh[v][e] * m2);
+        const float xh = (x[e] - mean) * rstd;
+        const float g = (GATED ? dy[e] * u[e] : dy[e]) * s_g[c + e];
+        dx[e] = rstd * (g - m1 - xh * m2);
         if (a.resid_grad) dx[e] += r[e];
       }
       store8(a.dx + row * a.lddx + c, dx);
     }
   }
-#pragma unroll
-  for (int v = 0; v < NV; ++v) {
-    const int c = 8 * (lane + 32 * v);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      atomicAdd(a.dgamma + c + e, dg[v][e]);
-      atomicAdd(a.dbeta + c + e, db[v][e]);
+  __syncthreads();
+  for (int c = threadIdx.x; c < W; c += blockDim.x) {
+    float g = 0.f, b = 0.f;
+    for (int w = 0; w < kAcc; ++w) {
+      g += s_dg[w][c];
+      b += s_db[w][c];
     }
+    atomicAdd(a.dgamma + c, g);
+    atomicAdd(a.dbeta + c, b);
   }
 }
 
-// Column-parallel pass over [T][W]: thread t owns columns [8t, 8t + 8) of the
-// rows of its block's chunk.  SCALE multiplies columns >= c0 by SiLU'(pre) in
-// place; every column's (scaled) values are summed into dbias.
-constexpr int kColRows = 64;
+// Column-parallel pass over [T][W] in 256-thread blocks: W / 8 threads own
+// columns [8t, 8t + 8) of a row; 256 / (W / 8) such groups take interleaved
+// rows of the block's chunk.  SCALE multiplies columns >= c0 by SiLU'(pre)
+// in place; every column's (scaled) values are summed, per block in shared
+// memory, then into dbias.
+constexpr int kColThreads = 256;
 template <bool SCALE>
-__global__ void colsum_kernel(bf16* g, int64_t ldg, const bf16* pre, int64_t ldp, int64_t T,
-                              int W, int c0, float* dbias) {
-  const int c = 8 * threadIdx.x;
-  if (c >= W) return;
-  const int64_t r0 = (int64_t)blockIdx.x * kColRows;
-  const int64_t r1 = r0 + kColRows < T ? r0 + kColRows : T;
+__global__ void __launch_bounds__(kColThreads) colsum_kernel(bf16* g, int64_t ldg, const bf16* pre,
+                                                             int64_t ldp, int64_t T, int W,
+                                                             int c0, float* dbias, int rows) {
+  const int ncol = W / 8, groups = kColThreads / ncol;
+  const int t = threadIdx.x % ncol, grp = threadIdx.x / ncol;
+  const int c = 8 * t;
+  const int64_t r0 = (int64_t)blockIdx.x * rows;
+  const int64_t r1 = r0 + rows < T ? r0 + rows : T;
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  for (int64_t r = r0; r < r1; ++r) {
-    float v[8];
-    load8(g + r * ldg + c, v);
-    if (SCALE && c >= c0) {
-      float p[8];
-      load8(pre + r * ldp + c, p);
+  if (grp < groups) {
+    const bool scale = SCALE && c >= c0;
+    for (int64_t r = r0 + grp; r < r1; r += groups) {
+      float v[8];
+      load8(g + r * ldg + c, v);
+      if (scale) {
+        float p[8];
+        load8(pre + r * ldp + c, p);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) v[e] *= silu_grad(p[e]);
-      store8(g + r * ldg + c, v);
+        for (int e = 0; e < 8; ++e) v[e] *= silu_grad(p[e]);
+        store8(g + r * ldg + c, v);
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] += v[e];
     }
-#pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] += v[e];
   }
+  if (groups == 1) {
 #pragma unroll
-  for (int e = 0; e < 8; ++e) atomicAdd(dbias + c + e, acc[e]);
+    for (int e = 0; e < 8; ++e) atomicAdd(dbias + c + e, acc[e]);
+    return;
+  }
+  // several row groups: sum them through shared memory, column by column
+  __shared__ float s_sum[kColThreads * 8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) s_sum[threadIdx.x * 8 + e] = acc[e];
+  __syncthreads();
+  for (int col = threadIdx.x; col < W; col += kColThreads) {
+    const int tt = col / 8, e = col % 8;
+    float sum = 0.f;
+    for (int q = 0; q < groups; ++q) sum += s_sum[(q * ncol + tt) * 8 + e];
+    atomicAdd(dbias + col, sum);
+  }
 }
 
 // New offsets after truncation (one thread; B is small).
@@ -259,7 +311,7 @@ cudaError_t launch_ln_fwd(const LnArgs& a, bool gated, cudaStream_t st) {
 cudaError_t launch_ln_bwd(const LnArgs& a, bool gated, cudaStream_t st) {
   if (a.T == 0) return cudaSuccess;
   const int64_t need = (a.T + kRowWarps - 1) / kRowWarps;
-  const int cap = device_sm_count() * 8;  // rows per warp grow past this
+  const int cap = device_sm_count() * 4;  // rows per warp grow past this
   const int grid = (int)(need < cap ? need : cap);
 #define HSTU_LNB(NV)                                                                    \
   if (a.W == NV * 256) {                                                                \
@@ -272,22 +324,31 @@ cudaError_t launch_ln_bwd(const LnArgs& a, bool gated, cudaStream_t st) {
   return cudaErrorNotSupported;
 }
 
+// Rows per block: about 64 rows' worth of 16-byte loads per thread.
+int colsum_rows(int W) { return 64 * (kColThreads / (W / 8)); }
+
+bool colsum_width_ok(int W) {
+  return W % 8 == 0 && W / 8 <= kColThreads && kColThreads % (W / 8) == 0;
+}
+
 cudaError_t launch_silu_bwd_colsum(bf16* g, int64_t ldg, const bf16* pre, int64_t ldp, int64_t T,
                                    int W, int c0, float* dbias, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
-  if (W % 8 != 0 || W / 8 > 1024) return cudaErrorNotSupported;
-  const int grid = (int)((T + kColRows - 1) / kColRows);
-  colsum_kernel<true><<<grid, W / 8, 0, st>>>(g, ldg, pre, ldp, T, W, c0, dbias);
+  if (!colsum_width_ok(W)) return cudaErrorNotSupported;
+  const int rows = colsum_rows(W);
+  const int grid = (int)((T + rows - 1) / rows);
+  colsum_kernel<true><<<grid, kColThreads, 0, st>>>(g, ldg, pre, ldp, T, W, c0, dbias, rows);
   return cudaGetLastError();
 }
 
 cudaError_t launch_colsum(const bf16* g, int64_t ldg, int64_t T, int W, float* dbias,
                           cudaStream_t st) {
   if (T == 0) return cudaSuccess;
-  if (W % 8 != 0 || W / 8 > 1024) return cudaErrorNotSupported;
-  const int grid = (int)((T + kColRows - 1) / kColRows);
-  colsum_kernel<false><<<grid, W / 8, 0, st>>>(const_cast<bf16*>(g), ldg, nullptr, 0, T, W, W,
-                                               dbias);
+  if (!colsum_width_ok(W)) return cudaErrorNotSupported;
+  const int rows = colsum_rows(W);
+  const int grid = (int)((T + rows - 1) / rows);
+  colsum_kernel<false><<<grid, kColThreads, 0, st>>>(const_cast<bf16*>(g), ldg, nullptr, 0, T, W,
+                                                     W, dbias, rows);
   return cudaGetLastError();
 }
 
