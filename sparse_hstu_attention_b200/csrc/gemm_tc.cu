@@ -26,6 +26,7 @@
 // warps 2..9 epilogue (warp w reads TMEM lanes 32 (w % 4) .. +32 and half of
 // the tile's columns).
 #include <cudaTypedefs.h>
+#include <string.h>
 
 #include "sm100.cuh"
 #include "stu_common.cuh"
@@ -40,21 +41,33 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kBM = 128, kBN = 256, kBK = 64, kStages = 4;
+constexpr int kBM = 128, kBN = 256, kBK = 64;
 constexpr int kEpiWarps = 8;  // two per TMEM lane quarter, each half of the tile's columns
-constexpr int kThreads = 32 * (2 + kEpiWarps);
+constexpr int kThreads = 32 * (2 + 8);
 constexpr int A_TILE = kBM * kBK * 2;  // 16 KB
 constexpr int B_TILE = kBN * kBK * 2;  // 32 KB
 constexpr int MN_BOX = 64 * kBK * 2;   // one 64 (M or N) x 64 (K) box of an MN-major tile
-constexpr int OFF_A = 0;
-constexpr int OFF_B = OFF_A + kStages * A_TILE;
-constexpr int OFF_BAR = OFF_B + kStages * B_TILE;
-constexpr int OFF_SLOT = OFF_BAR + 128;
-constexpr int SMEM = OFF_SLOT + 16 + 1024;
-static_assert(SMEM <= 232448, "shared memory budget");
+// bf16 outputs leave through shared memory and TMA: each epilogue warp stages
+// a 32-row x 64-column box (128-byte rows, 128B-swizzled) of each output
+constexpr int STG_BOX = 32 * 128;
+constexpr int STG_WARP = 2 * STG_BOX;  // out, out2
+// Shared-memory plan per epilogue: bf16 outputs take 3 ring stages and the
+// staging boxes, the fp32 reductions 4 stages and no staging.
+template <int EPI>
+struct GLayout {
+  static constexpr int kStages = EPI == kEpiRedF32 ? 4 : 3;
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_B = OFF_A + kStages * A_TILE;
+  static constexpr int OFF_STG = OFF_B + kStages * B_TILE;
+  static constexpr int OFF_BAR = OFF_STG + (EPI == kEpiRedF32 ? 0 : kEpiWarps * STG_WARP);
+  static constexpr int OFF_SLOT = OFF_BAR + 128;
+  static constexpr int SMEM = OFF_SLOT + 16 + 1024;
+  static_assert(SMEM <= 232448, "shared memory budget");
+};
+constexpr int kMaxStages = 4;
 constexpr uint32_t kTmemCols = 2 * kBN;
 
-enum { G_FULL = 0, G_EMPTY = kStages, G_ACC_FULL = 2 * kStages, G_ACC_EMPTY = G_ACC_FULL + 2,
+enum { G_FULL = 0, G_EMPTY = kMaxStages, G_ACC_FULL = 2 * kMaxStages, G_ACC_EMPTY = G_ACC_FULL + 2,
        G_COUNT = G_ACC_EMPTY + 2 };
 static_assert(8 * G_COUNT <= 128, "barrier area");
 
@@ -96,7 +109,11 @@ __device__ __forceinline__ float silu_f(float v) {
 template <bool A_MN, bool B_MN, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmb,
+                   const __grid_constant__ CUtensorMap tmo, const __grid_constant__ CUtensorMap tmo2,
                    const GemmArgs g) {
+  using Lay = GLayout<EPI>;
+  constexpr int kStages = Lay::kStages, OFF_A = Lay::OFF_A, OFF_B = Lay::OFF_B;
+  constexpr int OFF_STG = Lay::OFF_STG, OFF_BAR = Lay::OFF_BAR, OFF_SLOT = Lay::OFF_SLOT;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -121,6 +138,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_barrier_init();
     prefetch_tmap(&tma);
     prefetch_tmap(&tmb);
+    if (EPI != kEpiRedF32) prefetch_tmap(&tmo);
+    if (EPI == kEpiBiasSilu) prefetch_tmap(&tmo2);
   }
   if (warp == 1) {
     tmem_alloc(smem_addr(tmem_slot), kTmemCols);
@@ -210,6 +229,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;
     const int col0 = ((warp - 2) >> 2) * (kBN / 2);  // this warp's half of the columns
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t stg = base + OFF_STG + (uint32_t)(warp - 2) * STG_WARP;
+    const uint32_t stg_row = (uint32_t)lane * 128;
+    const uint32_t swz = (uint32_t)(lane & 7);
+    bool stores_pending = false;
     uint32_t tc = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
@@ -230,16 +253,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_before();
           warp_arrive(bar(G_ACC_EMPTY + buf));
         }
-        if (!live) continue;
         const int n = ti.n0 + c;
-        if (EPI == kEpiRedF32) {
-          float* dst = g.outf + (int64_t)m * g.ldf + n;
+        if constexpr (EPI == kEpiRedF32) {
+          if (live) {
+            float* dst = g.outf + (int64_t)m * g.ldf + n;
 #pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            red_add_v4(dst + e, __uint_as_float(v[e]), __uint_as_float(v[e + 1]),
-                       __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
-          continue;
-        }
+            for (int e = 0; e < 32; e += 4)
+              red_add_v4(dst + e, __uint_as_float(v[e]), __uint_as_float(v[e + 1]),
+                         __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+          }
+        } else {
         float f[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(v[e]);
@@ -254,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             f[4 * e + 3] += b4.w;
           }
         }
-        if (EPI == kEpiBiasResid) {
+        if (EPI == kEpiBiasResid && live) {
           const uint4* rp = reinterpret_cast<const uint4*>(g.resid + (int64_t)m * g.ldr + n);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -267,25 +290,49 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
+        // a 64-column box: its first 32 columns go to 16-byte chunks 0..3 of
+        // this lane's staged row, the next 32 to chunks 4..7
+        const int half = (c >> 5) & 1;
+        if (half == 0 && stores_pending) {  // the box staged before must be read out
+          if (lane == 0) bulk_wait_read_all();
+          __syncwarp();
+          stores_pending = false;
+        }
         uint32_t o[16];
         if (EPI == kEpiBiasSilu) {
 #pragma unroll
           for (int e = 0; e < 16; ++e) o[e] = pack_bf16x2(f[2 * e], f[2 * e + 1]);
-          uint4* pp = reinterpret_cast<uint4*>(g.out2 + (int64_t)m * g.ldo2 + n);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) pp[q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+          for (int q = 0; q < 4; ++q)
+            st_shared_v4(stg + STG_BOX + stg_row + ((((uint32_t)(half * 4 + q)) ^ swz) << 4),
+                         o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
 #pragma unroll
           for (int e = 0; e < 16; ++e) o[e] = pack_bf16x2(silu_f(f[2 * e]), silu_f(f[2 * e + 1]));
         } else {
 #pragma unroll
           for (int e = 0; e < 16; ++e) o[e] = pack_bf16x2(f[2 * e], f[2 * e + 1]);
         }
-        uint4* op = reinterpret_cast<uint4*>(g.out + (int64_t)m * g.ldo + n);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) op[q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+        for (int q = 0; q < 4; ++q)
+          st_shared_v4(stg + stg_row + ((((uint32_t)(half * 4 + q)) ^ swz) << 4), o[4 * q],
+                       o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+        if (half == 1) {  // box complete: one TMA store per output (rows past M are clipped)
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            const int x = n - 32, y = ti.m0 + quarter * 32;
+            tma_store_2d(&tmo, stg, x, y);
+            if (EPI == kEpiBiasSilu) tma_store_2d(&tmo2, stg + STG_BOX, x, y);
+            bulk_commit_group();
+          }
+          stores_pending = true;
+        }
+        }  // bf16 outputs
       }
       ++tc;
     }
+    if (lane == 0) bulk_wait_all();  // every store complete before the CTA exits
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -298,13 +345,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <bool A_MN, bool B_MN, int EPI>
-cudaError_t launch_t(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g,
-                     int ntiles, cudaStream_t st) {
+cudaError_t launch_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mo,
+                     const CUtensorMap& mo2, const GemmArgs& g, int ntiles, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<A_MN, B_MN, EPI>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       GLayout<EPI>::SMEM);
   if (e != cudaSuccess) return e;
   const int sms = device_sm_count();
-  gemm_tc_kernel<A_MN, B_MN, EPI><<<ntiles < sms ? ntiles : sms, kThreads, SMEM, st>>>(ma, mb, g);
+  gemm_tc_kernel<A_MN, B_MN, EPI>
+      <<<ntiles < sms ? ntiles : sms, kThreads, GLayout<EPI>::SMEM, st>>>(ma, mb, mo, mo2, g);
   return cudaGetLastError();
 }
 
@@ -327,9 +376,18 @@ cudaError_t launch_gemm(const GemmOperand& A, const GemmOperand& B, GemmArgs g, 
       !(B.mn_major ? make_tma_2d(&mb, B.ptr, g.K, g.N, B.ld, 64, kBK, true)
                    : make_tma_2d(&mb, B.ptr, g.N, g.K, B.ld, kBK, kBN, true)))
     return cudaErrorInvalidValue;
+  // bf16 outputs: 64-column x 32-row boxes, 128B-swizzled like the staging
+  CUtensorMap mo, mo2;
+  memset(&mo, 0, sizeof(mo));
+  memset(&mo2, 0, sizeof(mo2));
+  if (epi != kEpiRedF32 && !make_tma_2d(&mo, g.out, g.M, g.N, g.ldo, 64, 32, true))
+    return cudaErrorInvalidValue;
+  if (epi == kEpiBiasSilu && !make_tma_2d(&mo2, g.out2, g.M, g.N, g.ldo2, 64, 32, true))
+    return cudaErrorInvalidValue;
   const int ntiles = ((g.M + kBM - 1) / kBM) * (g.N / kBN) * g.splits;
 #define HSTU_GEMM_CASE(AM, BM_, E) \
-  if (A.mn_major == AM && B.mn_major == BM_ && epi == E) return launch_t<AM, BM_, E>(ma, mb, g, ntiles, st);
+  if (A.mn_major == AM && B.mn_major == BM_ && epi == E) \
+    return launch_t<AM, BM_, E>(ma, mb, mo, mo2, g, ntiles, st);
   HSTU_GEMM_CASE(false, true, kEpiBiasSilu)    // x^ W1 + b1 -> SiLU      (W1 stored [K][N])
   HSTU_GEMM_CASE(false, true, kEpiBiasResid)   // y W2 + b2 + x           (W2 stored [K][N])
   HSTU_GEMM_CASE(false, false, kEpiStore)      // dOut W2^T, dPre W1^T     (W read [N][K])
