@@ -491,6 +491,25 @@ def main():
                              (0 if w.fwd_only else LAUNCHES_PER_STEP["bwd"])),
         "clocks": clocks.summary(),
     }
+    if w.fwd_only:
+        # M-FALCON candidate scoring on the same batch: only the query tiles that
+        # hold candidates (history K/V as the cache); FLOPs over candidate pairs
+        cp = F.candidate_pairs(batch.lengths, batch.num_targets, w.contextual_len, w.K1, w.K2)
+        cev = new_events(2)
+        for _ in range(3):
+            sla.hstu_sla_fwd(q, k, v, offs, nts, out=out, workspace=ws_f, candidates_only=True, **kw)
+        torch.cuda.synchronize()
+        cev[0].record(stream)
+        for _ in range(K):
+            sla.hstu_sla_fwd(q, k, v, offs, nts, out=out, workspace=ws_f, candidates_only=True, **kw)
+        cev[1].record(stream)
+        torch.cuda.synchronize()
+        c_ms = cev[0].elapsed_time(cev[1]) / K
+        line["candidate_scoring"] = {
+            "ms_per_call": c_ms, "candidate_rows": int(batch.num_targets.sum()),
+            "candidate_pairs_per_head": cp,
+            "tflops": F.fwd_flops(cp, H, d) / (c_ms * 1e-3) / 1e12,
+            "speedup_vs_full_forward": ms_step / c_ms}
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(batch)
     print(json.dumps(line), flush=True)

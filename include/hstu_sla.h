@@ -88,6 +88,14 @@ typedef struct {
    * conversion kernels).  NULL = not recorded. */
   void* event_begin;
   void* event_end;
+  /* M-FALCON candidate scoring (HSTU notes, section 2.6): non-zero computes
+   * only the query tiles that hold candidates (rows >= L - num_targets of
+   * each sequence), reading every key's k and v (the cached history and the
+   * candidates); out rows of other tiles are left untouched.  The rows of
+   * the first candidate tile that precede the candidates are history rows
+   * and are written too (with their correct values).  Ignored by the
+   * backward. */
+  int32_t candidates_only;
 } hstu_sla_fwd_params;
 
 /* Backward problem: the forward problem plus dout and the three gradients. */

@@ -64,7 +64,7 @@ def hstu_sla_workspace_bytes(which: int, total_tokens: int, B: int, H: int, d: i
 
 
 def _fwd_params(q, k, v, seq_offsets, num_targets, contextual_len, K1, K2, alpha, N,
-                max_seq_len, events=None) -> _abi.FwdParams:
+                max_seq_len, events=None, candidates_only=False) -> _abi.FwdParams:
     T, H, d = q.shape
     if seq_offsets.dtype != torch.int32 or not seq_offsets.is_cuda:
         raise TypeError("seq_offsets must be a CUDA int32 tensor [B+1]")
@@ -88,6 +88,7 @@ def _fwd_params(q, k, v, seq_offsets, num_targets, contextual_len, K1, K2, alpha
     if events is not None:
         p.event_begin = events[0].cuda_event
         p.event_end = events[1].cuda_event
+    p.candidates_only = int(bool(candidates_only))
     return p
 
 
@@ -104,12 +105,14 @@ def hstu_sla_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, seq_offsets:
                  num_targets: Optional[torch.Tensor], *, contextual_len: int, K1: int, K2: int,
                  alpha: float, N: float, max_seq_len: Optional[int] = None,
                  out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
-                 stream=None, events=None) -> torch.Tensor:
+                 stream=None, events=None, candidates_only: bool = False) -> torch.Tensor:
     """SLA HSTU attention forward; returns out [T, H, d] (bf16).  `events`: an
-    optional pair of torch.cuda.Event recorded around the attention kernel."""
+    optional pair of torch.cuda.Event recorded around the attention kernel.
+    candidates_only: M-FALCON scoring, only the query tiles that hold
+    candidates are computed (other rows of `out` are left as they were)."""
     lib = _abi.load()
     p = _fwd_params(q, k, v, seq_offsets, num_targets, contextual_len, K1, K2, alpha, N,
-                    max_seq_len, events)
+                    max_seq_len, events, candidates_only)
     if out is None:
         out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
     p.out = out.data_ptr()

@@ -34,6 +34,7 @@ class FwdParams(ctypes.Structure):
         ("v_row_stride", ctypes.c_int64),
         ("out", ctypes.c_void_p), ("out_row_stride", ctypes.c_int64),
         ("event_begin", ctypes.c_void_p), ("event_end", ctypes.c_void_p),
+        ("candidates_only", ctypes.c_int32),
     ]
 
 

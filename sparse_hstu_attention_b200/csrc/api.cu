@@ -65,6 +65,7 @@ AttnArgs make_args(const hstu_sla_fwd_params* f, void* ws) {
   a.q_rs = f->q_row_stride;
   a.k_rs = f->k_row_stride;
   a.v_rs = f->v_row_stride;
+  a.cand_only = f->candidates_only != 0;
   return a;
 }
 
@@ -120,6 +121,7 @@ int hstu_sla_bwd(const hstu_sla_bwd_params* p, void* workspace, size_t workspace
     return e;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   AttnArgs a = make_args(f, workspace);
+  a.cand_only = 0;  // the backward covers every row
   a.dout = static_cast<const bf16*>(p->dout);
   a.dq = static_cast<bf16*>(p->dq);
   a.dk = static_cast<bf16*>(p->dk);

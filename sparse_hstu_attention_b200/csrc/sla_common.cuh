@@ -77,6 +77,7 @@ struct AttnArgs {
   WsHeader* ws;          // status / counts
   float* dqacc;          // fp32 dQ accumulator [H, T, d] (one-pass backward only)
   int B, H, K1, K2e, max_seq_len;
+  int cand_only;         // forward work list: only query tiles holding candidates
   int64_t T;
   float alpha, inv_n;
   const bf16* q;

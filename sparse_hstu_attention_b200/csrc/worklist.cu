@@ -96,6 +96,10 @@ __global__ void __launch_bounds__(kWlThreads) worklist_kernel(AttnArgs a, int ti
         }
         if (pass == 0) { cnt = npre; first = 0; }
         else { cnt = ntile - npre; first = npre; }
+        if (!backward && a.cand_only) {  // from the tile of the first candidate on
+          first = Lh < L ? Lh / tile : ntile;
+          cnt = ntile - first;
+        }
       }
       int off;
       int total = block_exclusive_scan(cnt, &off, s_scan);

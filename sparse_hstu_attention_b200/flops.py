@@ -31,6 +31,15 @@ def pairs_per_sequence(lengths, num_targets, contextual_len: int, K1: int, K2: i
     return history_pairs(Lh, K1 + K2e) + tgt
 
 
+def candidate_pairs(lengths, num_targets, contextual_len: int, K1: int, K2: int) -> int:
+    """Unmasked pairs of the candidate rows alone (one head): what M-FALCON
+    scoring computes per candidate."""
+    lengths = np.asarray(lengths, dtype=np.int64)
+    nt = np.asarray(num_targets, dtype=np.int64)
+    K2e = max(K2, contextual_len)
+    return int((nt * (np.minimum(lengths - nt, K2e + max(K1 - 1, 0)) + 1)).sum())
+
+
 def total_pairs(lengths, num_targets, contextual_len, K1, K2) -> int:
     """Unmasked (row, key) pairs of one head over the batch."""
     return int(pairs_per_sequence(lengths, num_targets, contextual_len, K1, K2).sum())

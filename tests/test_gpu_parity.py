@@ -146,6 +146,29 @@ def test_full_size_sampled(wname):
         assert torch.isfinite(t.float()).all()
 
 
+def test_candidate_scoring_computes_only_candidate_tiles():
+    """M-FALCON scoring (candidates_only): rows of the query tiles that hold
+    candidates equal the full forward bit for bit (and the oracle); rows of
+    the other tiles keep what the output buffer held."""
+    lengths, nts = [700, 1300, 260, 90], [64, 100, 260, 0]
+    b = _edge_batch(lengths=lengths, nt=np.array(nts), K1=128, K2=32, ctx=8)
+    g = to_gpu(b)
+    full = gpu_fwd(b, g)
+    out = torch.full_like(g["q"], 7.0)
+    sla.hstu_sla_fwd(g["q"], g["k"], g["v"], g["offs"], g["nts"], out=out, candidates_only=True,
+                     **kwargs_of(b))
+    torch.cuda.synchronize()
+    p = oracle_problem(b)
+    for i, (L, nt) in enumerate(zip(lengths, nts)):
+        s0 = int(b.seq_offsets[i])
+        first = ((L - nt) // 128) * 128 if nt > 0 else L
+        assert bool((out[s0:s0 + first] == 7.0).all())
+        assert torch.equal(out[s0 + first:s0 + L], full[s0 + first:s0 + L])
+        if nt:
+            rows = np.arange(s0 + L - nt, s0 + L)
+            assert_close("candidates", out[rows], p.fwd(b.q, b.k, b.v, rows=rows))
+
+
 def test_inference_workload_sampled():
     b = make_batch(WORKLOADS["infer"], with_dout=False)
     g = to_gpu(b)
@@ -153,6 +176,14 @@ def test_inference_workload_sampled():
     p = oracle_problem(b)
     rows = sample_tokens(b, 96, seed=3)
     assert_close("out", out[rows], p.fwd(b.q, b.k, b.v, rows=rows))
+    # candidate scoring on the same batch: every candidate row as in the full pass
+    cand = sla.hstu_sla_fwd(g["q"], g["k"], g["v"], g["offs"], g["nts"], candidates_only=True,
+                            out=torch.zeros_like(out), **kwargs_of(b))
+    torch.cuda.synchronize()
+    for i in range(len(b.lengths)):
+        s0, s1 = int(b.seq_offsets[i]), int(b.seq_offsets[i + 1])
+        lo = s1 - int(b.num_targets[i])
+        assert torch.equal(cand[lo:s1], out[lo:s1])
     assert torch.isfinite(out.float()).all()
 
 

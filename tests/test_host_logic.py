@@ -48,3 +48,17 @@ def test_partition_covers_every_sequence_once(world):
     for o in owned:
         offs, toks = shard_offsets(lengths, o)
         assert offs[-1] == len(toks) == lengths[o].sum()
+
+
+def test_candidate_pairs_match_oracle_row_counts():
+    """The M-FALCON scoring work (pairs of candidate rows) equals the oracle's
+    per-row counts summed over the candidate rows."""
+    import oracle
+    from sparse_hstu_attention_b200 import flops as F
+    lengths, nts = np.array([40, 17, 90, 5]), np.array([6, 0, 30, 5])
+    offs = np.concatenate([[0], np.cumsum(lengths)])
+    for c, K1, K2 in [(2, 8, 3), (0, 0, 4), (5, 100, 0)]:
+        p = oracle.Problem(offs, nts, 1, 4, c, K1, K2, 1.0, 1.0)
+        rc = p.row_counts()
+        want = sum(int(rc[offs[b + 1] - nts[b]:offs[b + 1]].sum()) for b in range(len(lengths)))
+        assert F.candidate_pairs(lengths, nts, c, K1, K2) == want
