@@ -89,8 +89,9 @@ enum {
 };
 static_assert(8 * BAR_COUNT <= 512, "barrier area");
 
-// Unit u of the static schedule: head u / n_items, query tile
-// items[u % n_items]; the key tiles it meets.  u >= total ends the schedule.
+// Unit u of the schedule (units are taken from an atomic counter in order, so
+// a CTA that drew short units takes more of them): head u / n_items, query
+// tile items[u % n_items]; the key tiles it meets.  u >= total ends it.
 __device__ void decode_unit(const AttnArgs& a, int n_items, int total, int u, UnitRec* r) {
   if (u >= total) {
     r->nsteps = -1;
@@ -177,7 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int slot = kk % kUSlots;
       if (!warp_wait(bar(BAR_U_EMPTY + slot), ((kk / kUSlots) & 1) ^ 1, a.ws)) return false;
       if (lane == 0) {
-        decode_unit(a, n_items, total, blockIdx.x + kk * gridDim.x, &ring[slot]);
+        decode_unit(a, n_items, total, atomicAdd(&a.ws->sched, 1), &ring[slot]);
         mbar_arrive(bar(BAR_U_FULL + slot));
       }
       __syncwarp();
