@@ -251,7 +251,9 @@ def _config(w, batch):
 
 def run_stu(args, world, rank, local):
     """The 6-layer STU stack workload (truncation after layer 3): one step is
-    the stack's forward and backward, every parameter gradient included."""
+    the stack's forward and backward, every parameter gradient included.
+    --fp8: the forward projections in E4M3, the weights' E4M3 copies redone
+    inside every step (as after each optimizer update)."""
     from sparse_hstu_attention_b200 import stu
     from workloads import (STU_LAYERS, STU_TAIL, STU_TRUNC_AFTER, draw_lengths, draw_stu,
                            offsets_from_lengths)
@@ -267,7 +269,7 @@ def run_stu(args, world, rank, local):
     T, T_out, dm = int(offs[-1]), int(tl.sum()), full.d_model
     dr = draw_stu(T, T_out, dm, STU_LAYERS, seed=w.seed + 7919 * rank)
     ws = [stu.StuWeights.from_host(lw, dev) for lw in dr.layers]
-    stack = stu.StuStack(ws, full, cut, STU_TRUNC_AFTER, tail)
+    stack = stu.StuStack(ws, full, cut, STU_TRUNC_AFTER, tail, fp8=args.fp8)
     offs_d = torch.tensor(offs, dtype=torch.int32, device=dev)
     nts_d = torch.tensor(nts, dtype=torch.int32, device=dev)
     x, dout = dr.x.to(dev), dr.dout.to(dev)
@@ -282,6 +284,8 @@ def run_stu(args, world, rank, local):
            (F.fwd_flops(p_cut, w.H, w.d) + F.bwd_flops(p_cut, w.H, w.d)) * n_cut
 
     def step():
+        if args.fp8:
+            stack.requantize()
         out, ctx = stack.forward(x, offs_d, nts_d, lengths, nts)
         stack.backward(dout, ctx)
 
@@ -314,16 +318,17 @@ def run_stu(args, world, rank, local):
             "metric": "STU stack fwd+bwd TFLOP/s (projections + SLA attention over unmasked pairs)",
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16, forward projections e4m3" if args.fp8 else "bf16",
             "data": "synthetic (seeded N(0,1) inputs, Xavier-uniform weights)",
-            "config": {"workload": "stu", "layers": STU_LAYERS, "trunc_after": STU_TRUNC_AFTER,
+            "config": {"workload": "stu", "fp8_forward_projections": bool(args.fp8), "layers": STU_LAYERS, "trunc_after": STU_TRUNC_AFTER,
                        "tail": tail, "B": int(len(lengths)), "T": T, "T_truncated": T_out,
                        "d_model": dm, "H": w.H, "d": w.d, "K1": w.K1, "K2": w.K2,
                        "contextual_len": c, "num_targets": w.num_targets,
                        "N": [w.N, cut.N]},
             "flops_per_step": {"projections": gemm, "attention": attn},
             "frac_of_sustained_peak": value / world / peak,
-            "gpu_launches": K * (STU_LAYERS * (6 + 11) + 3),
+            "gpu_launches": K * (STU_LAYERS * (6 + 11 + (2 if args.fp8 else 0)) + 3),
             "clocks": clocks.summary()}), flush=True)
     if world > 1:
         torch.distributed.barrier()
@@ -339,6 +344,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--fp8", action="store_true",
+                    help="stu workload: E4M3 forward projections (weights requantized every step)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":

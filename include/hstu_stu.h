@@ -62,6 +62,19 @@ typedef struct {
   void* av;                    /* [T][d_model]    attention output */
   void* y;                     /* [T][d_model]    gated norm output */
   float* stats;                /* [4][T]          mean / rstd of both norms */
+  /* FP8 forward projections (section 4.2.2, mixed-precision training and
+   * inference; appendix E.1, Tables 7 and 10): with fp8 = 1 the forward computes x^ W1 and y W2 with E4M3
+   * operands and fp32 accumulation.  Each LayerNorm also writes its output
+   * row in E4M3 with one scale per row (max |row| / 448, into the workspace),
+   * and the weights come pre-quantized by hstu_quant_weight_e4m3 (one scale
+   * per output column).  Everything saved for the backward stays bf16 and the
+   * backward itself is unchanged (bf16 GEMMs against w1 / w2).  fp8 = 0 reads
+   * none of the four fields below. */
+  int32_t fp8;
+  const void* w1q;             /* E4M3 [4 d_model][d_model]: W1 transposed */
+  const float* w1s;            /* [4 d_model] column scales of W1 */
+  const void* w2q;             /* E4M3 [d_model][d_model]:   W2 transposed */
+  const float* w2s;            /* [d_model] */
 } hstu_stu_layer_params;
 
 typedef struct {
@@ -84,15 +97,25 @@ typedef struct {
   float* d_b2;
 } hstu_stu_layer_bwd_params;
 
-/* Workspace bytes for hstu_stu_layer_fwd (which = HSTU_SLA_WS_FWD) or
+/* Workspace bytes for hstu_stu_layer_fwd (which = HSTU_SLA_WS_FWD, or
+ * HSTU_STU_WS_FWD_FP8 when fp8 = 1: the E4M3 activation rows on top) or
  * hstu_stu_layer_bwd (HSTU_SLA_WS_BWD); 256-byte aligned, contents need not
  * be initialised.  0 on invalid arguments. */
+#define HSTU_STU_WS_FWD_FP8 2
 size_t hstu_stu_workspace_bytes(int which, int64_t total_tokens, int32_t B, int32_t H, int32_t d);
 
 int hstu_stu_layer_fwd(const hstu_stu_layer_params* p, void* workspace, size_t workspace_bytes,
                        hstu_stream_t stream);
 int hstu_stu_layer_bwd(const hstu_stu_layer_bwd_params* p, void* workspace,
                        size_t workspace_bytes, hstu_stream_t stream);
+
+/* E4M3 copy of a weight W (bf16 [K][N], row stride ldw elements, the x W
+ * convention of the layer) for the FP8 forward: wq[n][k] (row stride ldq
+ * bytes, a multiple of 16) and scale[n] = max_k |W[k][n]| / 448 (1 for an
+ * all-zero column), so that wq[n][k] * scale[n] ~ W[k][n] (round to nearest
+ * even, saturating).  K and N multiples of 64.  Call it whenever W changes. */
+int hstu_quant_weight_e4m3(const void* w, int64_t ldw, int32_t K, int32_t N, void* wq,
+                           int64_t ldq, float* scale, hstu_stream_t stream);
 
 /* Status of the last layer call that used `workspace` (syncs the stream). */
 int hstu_stu_get_error(const void* workspace, hstu_stream_t stream);
@@ -118,7 +141,9 @@ int hstu_jagged_truncate(const void* src, int64_t src_row_stride, const int32_t*
  * bf16 operands and fp32 accumulation.  An operand with *_mn_major = 0 is
  * stored K-major (row m of A / row n of B, K values contiguous); with 1, it
  * is stored with row k holding its M (or N) values.  N must be a multiple of
- * 256.  Epilogues: */
+ * 256.  With fp8 = 1 both operands are E4M3, K-major, leading dimensions in
+ * bytes (multiples of 16), and D[m][n] = a_scale[m] * b_scale[n] *
+ * sum_k A[m][k] B[n][k] (not with HSTU_GEMM_RED_F32).  Epilogues: */
 enum {
   HSTU_GEMM_STORE = 0,       /* out  = bf16(D) */
   HSTU_GEMM_BIAS_SILU = 1,   /* out2 = bf16(D + bias), out = bf16(SiLU(D + bias)) */
@@ -144,6 +169,9 @@ typedef struct {
   int64_t ldo2;
   float* outf;         /* fp32 [M][N] */
   int64_t ldf;
+  int32_t fp8;
+  const float* a_scale;  /* [M], fp8 = 1 only */
+  const float* b_scale;  /* [N] */
 } hstu_gemm_params;
 
 /* workspace: >= 256 bytes, 256-byte aligned (a status word; read it with

@@ -36,6 +36,7 @@ from typing import List, Optional
 import numpy as np
 
 from . import Problem
+from . import fp8 as _fp8
 
 
 def silu(x):
@@ -95,12 +96,15 @@ def _problem(offsets, num_targets, cfg: AttnCfg) -> Problem:
                    cfg.alpha, cfg.N)
 
 
-def layer_fwd(x, w: Weights, offsets, num_targets, cfg: AttnCfg):
-    """One STU layer; returns (out, cache)."""
+def layer_fwd(x, w: Weights, offsets, num_targets, cfg: AttnCfg, fp8: bool = False):
+    """One STU layer; returns (out, cache).  fp8: both projections take E4M3
+    operands (oracle.fp8: the bf16 value of x^ and of y quantized per row,
+    W1 and W2 per column); the cache, and so the backward, keeps the
+    unquantized values."""
     x = np.asarray(x, dtype=np.float64)
     T, dm = x.shape
     xn, xh1, r1 = layer_norm(x, w.ln1_w, w.ln1_b, cfg.eps)
-    pre = xn @ w.w1 + w.b1
+    pre = (_fp8.fp8_matmul(_fp8.bf16_round(xn), w.w1) if fp8 else xn @ w.w1) + w.b1
     uvqk = silu(pre)
     u, v, q, k = (uvqk[:, i * dm:(i + 1) * dm] for i in range(4))
     prob = _problem(offsets, num_targets, cfg)
@@ -108,7 +112,7 @@ def layer_fwd(x, w: Weights, offsets, num_targets, cfg: AttnCfg):
     av = prob.fwd(q.reshape(shp), k.reshape(shp), v.reshape(shp)).reshape(T, dm)
     z, xh2, r2 = layer_norm(av, w.ln2_w, w.ln2_b, cfg.eps)
     y = z * u
-    out = y @ w.w2 + w.b2 + x
+    out = (_fp8.fp8_matmul(_fp8.bf16_round(y), w.w2) if fp8 else y @ w.w2) + w.b2 + x
     cache = dict(x=x, xn=xn, xh1=xh1, r1=r1, pre=pre, u=u, v=v, q=q, k=k, av=av, z=z, xh2=xh2,
                  r2=r2, y=y, prob=prob, shp=shp)
     return out, cache
@@ -163,8 +167,8 @@ def truncation_index(offsets, num_targets, contextual_len: int, tail: int):
 
 
 def stack_fwd(x, weights: List[Weights], offsets, num_targets, cfg_full: AttnCfg,
-              cfg_trunc: AttnCfg, trunc_after: int, tail: int):
-    """The truncated STU stack; returns (out, cache)."""
+              cfg_trunc: AttnCfg, trunc_after: int, tail: int, fp8: bool = False):
+    """The truncated STU stack; returns (out, cache).  fp8 as in layer_fwd."""
     h = np.asarray(x, dtype=np.float64)
     caches, offs, idx, new_offs = [], offsets, None, None
     for i, w in enumerate(weights):
@@ -173,7 +177,7 @@ def stack_fwd(x, weights: List[Weights], offsets, num_targets, cfg_full: AttnCfg
             h = h[idx]
             offs = new_offs
         cfg = cfg_full if i < trunc_after else cfg_trunc
-        h, c = layer_fwd(h, w, offs, num_targets, cfg)
+        h, c = layer_fwd(h, w, offs, num_targets, cfg, fp8)
         caches.append(c)
     return h, dict(caches=caches, idx=idx, T=np.asarray(x).shape[0], trunc_after=trunc_after)
 

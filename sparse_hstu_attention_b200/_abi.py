@@ -8,7 +8,8 @@ import re
 PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libhstu_sla.so")
 HEADER = os.path.join(os.path.dirname(PKG), "include", "hstu_sla.h")
-HEADERS = [HEADER, os.path.join(os.path.dirname(PKG), "include", "hstu_stu.h")]
+INCLUDE_DIR = os.path.join(os.path.dirname(PKG), "include")
+HEADERS = [HEADER, os.path.join(INCLUDE_DIR, "hstu_stu.h")]
 
 OK = 0
 ERR_INVALID_ARG = -1
@@ -20,6 +21,7 @@ ERR_TIMEOUT = -6
 
 WS_FWD = 0
 WS_BWD = 1
+WS_FWD_FP8 = 2   # hstu_stu_workspace_bytes only: the layer forward with fp8 = 1
 
 
 class FwdParams(ctypes.Structure):
@@ -61,6 +63,8 @@ class StuLayerParams(ctypes.Structure):
         ("x", ctypes.c_void_p), ("out", ctypes.c_void_p),
         ("xn", ctypes.c_void_p), ("pre", ctypes.c_void_p), ("uvqk", ctypes.c_void_p),
         ("av", ctypes.c_void_p), ("y", ctypes.c_void_p), ("stats", ctypes.c_void_p),
+        ("fp8", ctypes.c_int32), ("w1q", ctypes.c_void_p), ("w1s", ctypes.c_void_p),
+        ("w2q", ctypes.c_void_p), ("w2s", ctypes.c_void_p),
     ]
 
 
@@ -89,6 +93,7 @@ class GemmParams(ctypes.Structure):
         ("out", ctypes.c_void_p), ("ldo", ctypes.c_int64),
         ("out2", ctypes.c_void_p), ("ldo2", ctypes.c_int64),
         ("outf", ctypes.c_void_p), ("ldf", ctypes.c_int64),
+        ("fp8", ctypes.c_int32), ("a_scale", ctypes.c_void_p), ("b_scale", ctypes.c_void_p),
     ]
 
 
@@ -142,6 +147,8 @@ def load():
     lib.hstu_jagged_truncate.restype = ctypes.c_int
     lib.hstu_gemm.argtypes = [ctypes.POINTER(GemmParams), vp, vp]
     lib.hstu_gemm.restype = ctypes.c_int
+    lib.hstu_quant_weight_e4m3.argtypes = [vp, i64, i32, i32, vp, i64, vp, vp]
+    lib.hstu_quant_weight_e4m3.restype = ctypes.c_int
     _lib = lib
     return lib
 

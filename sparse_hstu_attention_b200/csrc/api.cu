@@ -9,7 +9,7 @@ using namespace hstu;
 
 namespace {
 
-constexpr int kAbiVersion = 101;  // 101: hstu_sla_fwd_params.candidates_only
+constexpr int kAbiVersion = 102;  // 101: hstu_sla_fwd_params.candidates_only; 102: FP8 forward
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 

@@ -26,6 +26,9 @@ int check_layer(const hstu_stu_layer_params* p, bool need_out) {
                         p->x,     p->out,   p->xn, p->pre, p->uvqk, p->av,   p->y,  p->stats};
   for (const void* q : ptrs)
     if (!al16(q) && !(q == p->out && !need_out)) return HSTU_SLA_ERR_INVALID_ARG;
+  if (p->fp8 != 0 && p->fp8 != 1) return HSTU_SLA_ERR_INVALID_ARG;
+  if (p->fp8 && need_out && (!al16(p->w1q) || !al16(p->w1s) || !al16(p->w2q) || !al16(p->w2s)))
+    return HSTU_SLA_ERR_INVALID_ARG;
   return HSTU_SLA_OK;
 }
 
@@ -74,27 +77,42 @@ int wgrad_splits(int M, int N, int64_t T) {
 
 int status_of(cudaError_t e) { return e == cudaSuccess ? HSTU_SLA_OK : HSTU_SLA_ERR_CUDA; }
 
+size_t round256(size_t n) { return (n + 255) & ~size_t(255); }
+
+// FP8 forward scratch after the attention's workspace: E4M3 rows [T][d_model]
+// (x^, then y) and their per-row scales [T].
+size_t fp8_scratch_bytes(int64_t T, int dm) {
+  return round256((size_t)T * dm) + round256((size_t)T * sizeof(float));
+}
+
 }  // namespace
 
 extern "C" {
 
 size_t hstu_stu_workspace_bytes(int which, int64_t total_tokens, int32_t B, int32_t H, int32_t d) {
-  const size_t a = hstu_sla_workspace_bytes(which, total_tokens, B, H, d);
-  return a ? kHdr + a : 0;
+  const bool f8 = which == HSTU_STU_WS_FWD_FP8;
+  const size_t a = hstu_sla_workspace_bytes(f8 ? HSTU_SLA_WS_FWD : which, total_tokens, B, H, d);
+  if (a == 0) return 0;
+  return kHdr + a + (f8 ? fp8_scratch_bytes(total_tokens, H * d) : 0);
 }
 
 int hstu_stu_layer_fwd(const hstu_stu_layer_params* p, void* workspace, size_t workspace_bytes,
                        hstu_stream_t stream) {
   int e = check_layer(p, true);
   if (e) return e;
+  const bool f8 = p->fp8 != 0;
   if ((e = check_ws(workspace, workspace_bytes,
-                    hstu_stu_workspace_bytes(HSTU_SLA_WS_FWD, p->total_tokens, p->B, p->H, p->d))))
+                    hstu_stu_workspace_bytes(f8 ? HSTU_STU_WS_FWD_FP8 : HSTU_SLA_WS_FWD,
+                                             p->total_tokens, p->B, p->H, p->d))))
     return e;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   WsHeader* gh = static_cast<WsHeader*>(workspace);
   void* aws = static_cast<char*>(workspace) + kHdr;
   const int64_t T = p->total_tokens;
   const int dm = p->H * p->d;
+  const size_t aws_bytes = hstu_sla_workspace_bytes(HSTU_SLA_WS_FWD, T, p->B, p->H, p->d);
+  uint8_t* q8 = f8 ? static_cast<uint8_t*>(aws) + aws_bytes : nullptr;  // E4M3 rows
+  float* q8s = f8 ? reinterpret_cast<float*>(q8 + round256((size_t)T * dm)) : nullptr;
   cudaError_t ce = cudaMemsetAsync(gh, 0, sizeof(WsHeader), st);
   if (ce != cudaSuccess) return HSTU_SLA_ERR_CUDA;
   // x^ = LayerNorm(x)
@@ -111,6 +129,9 @@ int hstu_stu_layer_fwd(const hstu_stu_layer_params* p, void* workspace, size_t w
   l1.ldy = dm;
   l1.mean = p->stats;
   l1.rstd = p->stats + T;
+  l1.yq = q8;
+  l1.ldyq = dm;
+  l1.yscale = q8s;
   if ((ce = launch_ln_fwd(l1, false, st)) != cudaSuccess) return status_of(ce);
   // pre = x^ W1 + b1, UVQK = SiLU(pre)
   GemmArgs g;
@@ -124,9 +145,14 @@ int hstu_stu_layer_fwd(const hstu_stu_layer_params* p, void* workspace, size_t w
   g.out2 = static_cast<bf16*>(p->pre);
   g.ldo2 = 4 * dm;
   g.ws = gh;
-  if ((ce = launch_gemm({p->xn, dm, false}, {p->w1, 4 * dm, true}, g, kEpiBiasSilu, st)) !=
-      cudaSuccess)
-    return status_of(ce);
+  if (f8) {
+    g.sa = q8s;
+    g.sb = p->w1s;
+    ce = launch_gemm({q8, dm, false, true}, {p->w1q, dm, false, true}, g, kEpiBiasSilu, st);
+  } else {
+    ce = launch_gemm({p->xn, dm, false}, {p->w1, 4 * dm, true}, g, kEpiBiasSilu, st);
+  }
+  if (ce != cudaSuccess) return status_of(ce);
   // A = SLA attention (Q, K, V)
   hstu_sla_fwd_params f = attn_params(p);
   if ((e = hstu_sla_fwd(&f, aws, workspace_bytes - kHdr, stream))) return e;
@@ -153,7 +179,13 @@ int hstu_stu_layer_fwd(const hstu_stu_layer_params* p, void* workspace, size_t w
   g2.out = static_cast<bf16*>(p->out);
   g2.ldo = dm;
   g2.ws = gh;
-  ce = launch_gemm({p->y, dm, false}, {p->w2, dm, true}, g2, kEpiBiasResid, st);
+  if (f8) {
+    g2.sa = q8s;
+    g2.sb = p->w2s;
+    ce = launch_gemm({q8, dm, false, true}, {p->w2q, dm, false, true}, g2, kEpiBiasResid, st);
+  } else {
+    ce = launch_gemm({p->y, dm, false}, {p->w2, dm, true}, g2, kEpiBiasResid, st);
+  }
   return status_of(ce);
 }
 
@@ -329,8 +361,13 @@ int hstu_gemm(const hstu_gemm_params* p, void* workspace, hstu_stream_t stream) 
     return HSTU_SLA_ERR_INVALID_ARG;
   if (p->M < 0 || p->N < 0 || p->K < 1 || p->N % 256 != 0 || p->epilogue < 0 ||
       p->epilogue > HSTU_GEMM_RED_F32 || !al16(p->a) || !al16(p->b) || p->lda % 8 != 0 ||
-      p->ldb % 8 != 0)
+      p->ldb % 8 != 0 || (p->fp8 != 0 && p->fp8 != 1))
     return HSTU_SLA_ERR_INVALID_ARG;
+  const bool f8 = p->fp8 != 0;
+  if (f8 && (p->lda % 16 != 0 || p->ldb % 16 != 0 || !al16(p->a_scale) || !al16(p->b_scale)))
+    return HSTU_SLA_ERR_INVALID_ARG;
+  if (f8 && (p->a_mn_major || p->b_mn_major || p->epilogue == HSTU_GEMM_RED_F32))
+    return HSTU_SLA_ERR_UNSUPPORTED;
   const bool red = p->epilogue == HSTU_GEMM_RED_F32;
   if (red ? !al16(p->outf) || p->ldf % 4 != 0 : !al16(p->out) || p->ldo % 8 != 0)
     return HSTU_SLA_ERR_INVALID_ARG;
@@ -357,11 +394,24 @@ int hstu_gemm(const hstu_gemm_params* p, void* workspace, hstu_stream_t stream) 
   g.outf = p->outf;
   g.ldf = p->ldf;
   g.ws = static_cast<WsHeader*>(workspace);
+  g.sa = p->a_scale;
+  g.sb = p->b_scale;
   cudaError_t ce = cudaMemsetAsync(workspace, 0, sizeof(WsHeader), st);
   if (ce == cudaSuccess)
-    ce = launch_gemm({p->a, p->lda, p->a_mn_major != 0}, {p->b, p->ldb, p->b_mn_major != 0}, g,
-                     p->epilogue, st);
+    ce = launch_gemm({p->a, p->lda, p->a_mn_major != 0, f8},
+                     {p->b, p->ldb, p->b_mn_major != 0, f8}, g, p->epilogue, st);
   if (ce == cudaErrorNotSupported) return HSTU_SLA_ERR_UNSUPPORTED;
+  return status_of(ce);
+}
+
+int hstu_quant_weight_e4m3(const void* w, int64_t ldw, int32_t K, int32_t N, void* wq,
+                           int64_t ldq, float* scale, hstu_stream_t stream) {
+  if (!al16(w) || !al16(wq) || !al16(scale) || K < 0 || N < 0 || ldw < N || ldq < K)
+    return HSTU_SLA_ERR_INVALID_ARG;
+  if (K % 64 != 0 || N % 64 != 0 || ldq % 16 != 0) return HSTU_SLA_ERR_UNSUPPORTED;
+  cudaError_t ce = launch_quant_wt(static_cast<const bf16*>(w), ldw, K, N,
+                                   static_cast<uint8_t*>(wq), ldq, scale,
+                                   reinterpret_cast<cudaStream_t>(stream));
   return status_of(ce);
 }
 

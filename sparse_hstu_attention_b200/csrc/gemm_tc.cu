@@ -35,6 +35,8 @@ namespace hstu {
 
 bool make_tma_2d(CUtensorMap* m, const void* ptr, int64_t T, int HD, int64_t rs, int box_w,
                  int box_h, bool sw128);
+bool make_tma_2d_u8(CUtensorMap* m, const void* ptr, int64_t T, int W, int64_t rs, int box_w,
+                    int box_h);
 int device_sm_count();
 
 namespace {
@@ -75,8 +77,9 @@ struct TileInfo {
   int m0, n0, k0, nkb;  // first row / column / k, number of 64-wide k blocks
 };
 
-__device__ __forceinline__ TileInfo tile_info(const GemmArgs& g, int t, int tiles_m,
-                                              int tiles_n) {
+// bk: elements per k block (64 bf16 or 128 8-bit values: 128 bytes either way)
+__device__ __forceinline__ TileInfo tile_info(const GemmArgs& g, int t, int tiles_m, int tiles_n,
+                                              int bk) {
   TileInfo ti;
   const int nb = t % tiles_n;
   const int rest = t / tiles_n;
@@ -86,7 +89,7 @@ __device__ __forceinline__ TileInfo tile_info(const GemmArgs& g, int t, int tile
   ti.n0 = nb * kBN;
   ti.k0 = split * g.k_split;
   const int k1 = min(g.K, ti.k0 + g.k_split);
-  ti.nkb = k1 > ti.k0 ? (k1 - ti.k0 + kBK - 1) / kBK : 0;
+  ti.nkb = k1 > ti.k0 ? (k1 - ti.k0 + bk - 1) / bk : 0;
   return ti;
 }
 
@@ -106,11 +109,13 @@ __device__ __forceinline__ float silu_f(float v) {
   return fmaf(h, t, h);
 }
 
-template <bool A_MN, bool B_MN, int EPI>
+template <bool A_MN, bool B_MN, int EPI, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmb,
                    const __grid_constant__ CUtensorMap tmo, const __grid_constant__ CUtensorMap tmo2,
                    const GemmArgs g) {
+  static_assert(!F8 || (!A_MN && !B_MN), "8-bit operands are read K-major");
+  constexpr int kBKe = F8 ? 2 * kBK : kBK;  // elements per 128-byte k block
   using Lay = GLayout<EPI>;
   constexpr int kStages = Lay::kStages, OFF_A = Lay::OFF_A, OFF_B = Lay::OFF_B;
   constexpr int OFF_STG = Lay::OFF_STG, OFF_BAR = Lay::OFF_BAR, OFF_SLOT = Lay::OFF_SLOT;
@@ -156,14 +161,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t it = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        const TileInfo ti = tile_info(g, t, tiles_m, tiles_n);
+        const TileInfo ti = tile_info(g, t, tiles_m, tiles_n, kBKe);
         for (int kb = 0; kb < ti.nkb; ++kb, ++it) {
           const int s = it % kStages;
           ok = mbar_wait(bar(G_EMPTY + s), ((it / kStages) & 1) ^ 1, g.ws);
           if (!ok) break;
           const uint32_t fb = bar(G_FULL + s);
           mbar_expect_tx(fb, A_TILE + B_TILE);
-          const int k = ti.k0 + kb * kBK;
+          const int k = ti.k0 + kb * kBKe;
           const uint32_t a = sA + s * A_TILE, b = sB + s * B_TILE;
           if (A_MN) {  // [K][M]: two 64-wide column boxes
             tma_load_2d(a, &tma, fb, ti.m0, k);
@@ -189,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // --------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t IDESC = idesc_bf16(kBM, kBN, A_MN, B_MN);
+      constexpr uint32_t IDESC = F8 ? idesc_e4m3(kBM, kBN) : idesc_bf16(kBM, kBN, A_MN, B_MN);
       // K-major: a 16-wide k step moves 32 bytes inside the 128-byte row;
       // MN-major: it moves 16 rows of 128 bytes.  Units of 16 bytes.
       constexpr uint32_t kStepA = A_MN ? 128u : 2u, kStepB = B_MN ? 128u : 2u;
@@ -200,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t it = 0, tc = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        const TileInfo ti = tile_info(g, t, tiles_m, tiles_n);
+        const TileInfo ti = tile_info(g, t, tiles_m, tiles_n, kBKe);
         if (ti.nkb == 0) continue;
         const uint32_t buf = tc & 1;
         ok = mbar_wait(bar(G_ACC_EMPTY + buf), ((tc >> 1) & 1) ^ 1, g.ws);
@@ -212,10 +217,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
           tc_fence_after();
           const uint32_t ao = (uint32_t)(s * A_TILE) >> 4, bo = (uint32_t)(s * B_TILE) >> 4;
+          // four 32-byte k steps per 128-byte block (16 bf16 or 32 8-bit values each)
 #pragma unroll
-          for (int ks = 0; ks < kBK / 16; ++ks)
-            mma_ss(tmem + buf * kBN, dA + ao + ks * kStepA, dB + bo + ks * kStepB, IDESC,
-                   (kb > 0 || ks > 0) ? 1u : 0u);
+          for (int ks = 0; ks < 4; ++ks) {
+            if constexpr (F8)
+              mma_ss_f8(tmem + buf * kBN, dA + ao + ks * kStepA, dB + bo + ks * kStepB, IDESC,
+                        (kb > 0 || ks > 0) ? 1u : 0u);
+            else
+              mma_ss(tmem + buf * kBN, dA + ao + ks * kStepA, dB + bo + ks * kStepB, IDESC,
+                     (kb > 0 || ks > 0) ? 1u : 0u);
+          }
           tc_commit(bar(G_EMPTY + s));
         }
         if (!ok) break;
@@ -236,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t tc = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-      const TileInfo ti = tile_info(g, t, tiles_m, tiles_n);
+      const TileInfo ti = tile_info(g, t, tiles_m, tiles_n, kBKe);
       if (ti.nkb == 0) continue;
       const uint32_t buf = tc & 1;
       ok = warp_wait(bar(G_ACC_FULL + buf), (tc >> 1) & 1, g.ws);
@@ -266,6 +277,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         float f[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(v[e]);
+        if constexpr (F8) {  // row scale of A times column scale of B
+          const float sm = live ? g.sa[m] : 0.f;
+          const float4* sp = reinterpret_cast<const float4*>(g.sb + n);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float4 s4 = __ldg(sp + e);
+            f[4 * e] *= sm * s4.x;
+            f[4 * e + 1] *= sm * s4.y;
+            f[4 * e + 2] *= sm * s4.z;
+            f[4 * e + 3] *= sm * s4.w;
+          }
+        }
         if (EPI == kEpiBiasSilu || EPI == kEpiBiasResid) {
           const float4* bp = reinterpret_cast<const float4*>(g.bias + n);
 #pragma unroll
@@ -344,15 +367,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <bool A_MN, bool B_MN, int EPI>
+template <bool A_MN, bool B_MN, int EPI, bool F8 = false>
 cudaError_t launch_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mo,
                      const CUtensorMap& mo2, const GemmArgs& g, int ntiles, cudaStream_t st) {
-  cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<A_MN, B_MN, EPI>,
+  cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<A_MN, B_MN, EPI, F8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        GLayout<EPI>::SMEM);
   if (e != cudaSuccess) return e;
   const int sms = device_sm_count();
-  gemm_tc_kernel<A_MN, B_MN, EPI>
+  gemm_tc_kernel<A_MN, B_MN, EPI, F8>
       <<<ntiles < sms ? ntiles : sms, kThreads, GLayout<EPI>::SMEM, st>>>(ma, mb, mo, mo2, g);
   return cudaGetLastError();
 }
@@ -365,17 +388,27 @@ cudaError_t launch_gemm(const GemmOperand& A, const GemmOperand& B, GemmArgs g, 
   // split-K only for the reducing epilogue; each split covers whole k blocks
   if (epi != kEpiRedF32) g.splits = 1;
   if (g.splits < 1) g.splits = 1;
-  const int kb_total = (g.K + kBK - 1) / kBK;
+  const bool f8 = A.fp8 || B.fp8;
+  if (f8 && (!A.fp8 || !B.fp8 || A.mn_major || B.mn_major || epi == kEpiRedF32 ||
+             g.sa == nullptr || g.sb == nullptr))
+    return cudaErrorNotSupported;
+  const int bke = f8 ? 2 * kBK : kBK;
+  const int kb_total = (g.K + bke - 1) / bke;
   const int kb_per = (kb_total + g.splits - 1) / g.splits;
-  g.k_split = kb_per * kBK;
+  g.k_split = kb_per * bke;
   g.splits = kb_per > 0 ? (kb_total + kb_per - 1) / kb_per : 1;
   CUtensorMap ma, mb;
   // K-major operand: rows = M (or N), columns = K.  MN-major: rows = K.
-  if (!(A.mn_major ? make_tma_2d(&ma, A.ptr, g.K, g.M, A.ld, 64, kBK, true)
-                   : make_tma_2d(&ma, A.ptr, g.M, g.K, A.ld, kBK, kBM, true)) ||
-      !(B.mn_major ? make_tma_2d(&mb, B.ptr, g.K, g.N, B.ld, 64, kBK, true)
-                   : make_tma_2d(&mb, B.ptr, g.N, g.K, B.ld, kBK, kBN, true)))
+  if (f8) {
+    if (!make_tma_2d_u8(&ma, A.ptr, g.M, g.K, A.ld, 128, kBM) ||
+        !make_tma_2d_u8(&mb, B.ptr, g.N, g.K, B.ld, 128, kBN))
+      return cudaErrorInvalidValue;
+  } else if (!(A.mn_major ? make_tma_2d(&ma, A.ptr, g.K, g.M, A.ld, 64, kBK, true)
+                          : make_tma_2d(&ma, A.ptr, g.M, g.K, A.ld, kBK, kBM, true)) ||
+             !(B.mn_major ? make_tma_2d(&mb, B.ptr, g.K, g.N, B.ld, 64, kBK, true)
+                          : make_tma_2d(&mb, B.ptr, g.N, g.K, B.ld, kBK, kBN, true))) {
     return cudaErrorInvalidValue;
+  }
   // bf16 outputs: 64-column x 32-row boxes, 128B-swizzled like the staging
   CUtensorMap mo, mo2;
   memset(&mo, 0, sizeof(mo));
@@ -385,6 +418,12 @@ cudaError_t launch_gemm(const GemmOperand& A, const GemmOperand& B, GemmArgs g, 
   if (epi == kEpiBiasSilu && !make_tma_2d(&mo2, g.out2, g.M, g.N, g.ldo2, 64, 32, true))
     return cudaErrorInvalidValue;
   const int ntiles = ((g.M + kBM - 1) / kBM) * (g.N / kBN) * g.splits;
+  if (f8) {  // the forward projections in E4M3
+    if (epi == kEpiBiasSilu) return launch_t<false, false, kEpiBiasSilu, true>(ma, mb, mo, mo2, g, ntiles, st);
+    if (epi == kEpiBiasResid) return launch_t<false, false, kEpiBiasResid, true>(ma, mb, mo, mo2, g, ntiles, st);
+    if (epi == kEpiStore) return launch_t<false, false, kEpiStore, true>(ma, mb, mo, mo2, g, ntiles, st);
+    return cudaErrorNotSupported;
+  }
 #define HSTU_GEMM_CASE(AM, BM_, E) \
   if (A.mn_major == AM && B.mn_major == BM_ && epi == E) \
     return launch_t<AM, BM_, E>(ma, mb, mo, mo2, g, ntiles, st);

@@ -16,8 +16,9 @@ enum { kEpiStore = 0, kEpiBiasSilu = 1, kEpiBiasResid = 2, kEpiRedF32 = 3 };
 // the M (or N) index; MN-major: rows are the K index.
 struct GemmOperand {
   const void* ptr;
-  int64_t ld;
+  int64_t ld;      // elements (bytes for 8-bit operands)
   bool mn_major;
+  bool fp8 = false;  // E4M3 bytes (K-major only)
 };
 
 struct GemmArgs {
@@ -34,6 +35,8 @@ struct GemmArgs {
   float* outf;        // kEpiRedF32: [M][N] fp32 accumulated into, row stride ldf
   int64_t ldf;
   WsHeader* ws;       // status word for the bounded waits
+  const float* sa;    // 8-bit operands: D[m][n] is scaled by sa[m] * sb[n]
+  const float* sb;
 };
 
 cudaError_t launch_gemm(const GemmOperand& A, const GemmOperand& B, GemmArgs g, int epi,
@@ -55,6 +58,9 @@ struct LnArgs {
   int64_t ldy;
   float* mean;         // [T]
   float* rstd;         // [T]
+  uint8_t* yq;         // optional E4M3 copy of y [T][W] (row stride ldyq bytes), with
+  int64_t ldyq;        //   yq[t] * yscale[t] ~ y[t] (per-row scale, max |y[t]| / 448)
+  float* yscale;
   // backward
   const bf16* dy;      // gradient of y [T][W], row stride lddy
   int64_t lddy;
@@ -70,6 +76,10 @@ struct LnArgs {
   float* dbeta;        // [W], accumulated into
 };
 cudaError_t launch_ln_fwd(const LnArgs& a, bool gated, cudaStream_t st);
+// E4M3 copy of a weight W [K][N] (x W convention) transposed to [N][K] (row
+// stride ldq bytes) with one scale per output column: Wq[n][k] * scale[n] ~ W[k][n].
+cudaError_t launch_quant_wt(const bf16* W, int64_t ldw, int K, int N, uint8_t* Wq, int64_t ldq,
+                            float* scale, cudaStream_t st);
 cudaError_t launch_ln_bwd(const LnArgs& a, bool gated, cudaStream_t st);
 
 // g[t][c] *= SiLU'(pre[t][c]) for columns [c0, W) and dbias[c] += sum_t of the

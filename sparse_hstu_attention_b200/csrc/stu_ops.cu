@@ -9,6 +9,7 @@
 //   TorchEasyRec's "Mid-stack Attention Truncation" bullet states).
 // Rows are d_model wide (W = 256, 512 or 1024); one warp per row, lane l
 // owning the 16-byte chunks l, l + 32, ... of the row.
+#include "sm100.cuh"
 #include "stu_common.cuh"
 
 namespace hstu {
@@ -49,6 +50,10 @@ __device__ __forceinline__ float silu_grad(float v) {
 
 // LayerNorm (biased variance) of each row, then the affine map; GATED also
 // multiplies by the gate row u.  Saves the row mean and 1/sqrt(var + eps).
+// With yq set, also writes the row in E4M3 with a per-row scale: the FP8
+// quantization fused into the norm that precedes each projection ("Bending
+// the Scaling Law Curve...", section 4.2.2, mixed-precision training and
+// inference; Figure 4).
 template <int NV, bool GATED>
 __global__ void __launch_bounds__(32 * kRowWarps) ln_fwd_kernel(const LnArgs a) {
   const int64_t row = (int64_t)blockIdx.x * kRowWarps + (threadIdx.x >> 5);
@@ -70,21 +75,81 @@ __global__ void __launch_bounds__(32 * kRowWarps) ln_fwd_kernel(const LnArgs a) 
 #pragma unroll
     for (int e = 0; e < 8; ++e) q += (x[v][e] - mean) * (x[v][e] - mean);
   const float rstd = rsqrtf(warp_sum(q) * (1.0f / W) + a.eps);
+  float amax = 0.f;
 #pragma unroll
   for (int v = 0; v < NV; ++v) {
     const int c = 8 * (lane + 32 * v);
-    float z[8], u[8];
+    float u[8];
     if (GATED) load8(a.u + row * a.ldu + c, u);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      z[e] = (x[v][e] - mean) * rstd * a.gamma[c + e] + a.beta[c + e];
-      if (GATED) z[e] *= u[e];
+      x[v][e] = (x[v][e] - mean) * rstd * a.gamma[c + e] + a.beta[c + e];  // x now holds y
+      if (GATED) x[v][e] *= u[e];
     }
-    store8(a.y + row * a.ldy + c, z);
+    store8(a.y + row * a.ldy + c, x[v]);
+    if (a.yq) {  // quantize what the bf16 output holds
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        x[v][e] = __bfloat162float(__float2bfloat16(x[v][e]));
+        amax = fmaxf(amax, fabsf(x[v][e]));
+      }
+    }
+  }
+  if (a.yq) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float scale = amax > 0.f ? amax * (1.0f / 448.0f) : 1.0f;
+    const float inv = 1.0f / scale;
+#pragma unroll
+    for (int v = 0; v < NV; ++v) {
+      const int c = 8 * (lane + 32 * v);
+      uint2 w;
+      w.x = sm100::pack_e4m3x2(x[v][0] * inv, x[v][1] * inv) |
+            (sm100::pack_e4m3x2(x[v][2] * inv, x[v][3] * inv) << 16);
+      w.y = sm100::pack_e4m3x2(x[v][4] * inv, x[v][5] * inv) |
+            (sm100::pack_e4m3x2(x[v][6] * inv, x[v][7] * inv) << 16);
+      *reinterpret_cast<uint2*>(a.yq + row * a.ldyq + c) = w;
+    }
+    if (lane == 0) a.yscale[row] = scale;
   }
   if (lane == 0) {
     a.mean[row] = mean;
     a.rstd[row] = rstd;
+  }
+}
+
+// Weight quantizer: a block owns 64 output columns.  It first takes each
+// column's max |W[k][n]| over all K (4 row phases x 64 columns, one reduce),
+// then converts 64 x 64 chunks through shared memory so that the transposed
+// rows of Wq are written 16 bytes at a time.
+__global__ void __launch_bounds__(256) quant_wt_kernel(const bf16* W, int64_t ldw, int K,
+                                                       uint8_t* Wq, int64_t ldq, float* scale) {
+  __shared__ float s_amax[4][64];
+  __shared__ __align__(16) uint8_t s_q[64][80];  // [n][k], rows padded to 80 bytes
+  const int c = threadIdx.x & 63, r = threadIdx.x >> 6;
+  const int n0 = blockIdx.x * 64;
+  const bf16* col = W + n0 + c;
+  float amax = 0.f;
+#pragma unroll 4
+  for (int k = r; k < K; k += 4) amax = fmaxf(amax, fabsf(__bfloat162float(col[(int64_t)k * ldw])));
+  s_amax[r][c] = amax;
+  __syncthreads();
+  amax = fmaxf(fmaxf(s_amax[0][c], s_amax[1][c]), fmaxf(s_amax[2][c], s_amax[3][c]));
+  const float sc = amax > 0.f ? amax * (1.0f / 448.0f) : 1.0f;
+  const float inv = 1.0f / sc;
+  if (r == 0) scale[n0 + c] = sc;
+  const int orow = threadIdx.x >> 2, ochunk = (threadIdx.x & 3) * 16;
+  for (int k0 = 0; k0 < K; k0 += 64) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int kk = r + 4 * i;
+      const float f = __bfloat162float(col[(int64_t)(k0 + kk) * ldw]) * inv;
+      s_q[c][kk] = (uint8_t)sm100::pack_e4m3x2(f, 0.f);
+    }
+    __syncthreads();
+    *reinterpret_cast<uint4*>(Wq + (int64_t)(n0 + orow) * ldq + k0 + ochunk) =
+        *reinterpret_cast<const uint4*>(&s_q[orow][ochunk]);
+    __syncthreads();
   }
 }
 
@@ -306,6 +371,14 @@ cudaError_t launch_ln_fwd(const LnArgs& a, bool gated, cudaStream_t st) {
   HSTU_LN(1) HSTU_LN(2) HSTU_LN(4)
 #undef HSTU_LN
   return cudaErrorNotSupported;
+}
+
+cudaError_t launch_quant_wt(const bf16* W, int64_t ldw, int K, int N, uint8_t* Wq, int64_t ldq,
+                            float* scale, cudaStream_t st) {
+  if (K % 64 != 0 || N % 64 != 0 || ldq % 16 != 0) return cudaErrorNotSupported;
+  if (N == 0) return cudaSuccess;
+  quant_wt_kernel<<<N / 64, 256, 0, st>>>(W, ldw, K, Wq, ldq, scale);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_ln_bwd(const LnArgs& a, bool gated, cudaStream_t st) {

@@ -42,6 +42,21 @@ bool make_tma_2d(CUtensorMap* m, const void* ptr, int64_t T, int HD, int64_t rs,
   return r == CUDA_SUCCESS;
 }
 
+// The same over a [T, W] byte matrix (8-bit floats), row stride rs bytes.
+bool make_tma_2d_u8(CUtensorMap* m, const void* ptr, int64_t T, int W, int64_t rs, int box_w,
+                    int box_h) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)W, (cuuint64_t)T};
+  cuuint64_t strides[1] = {(cuuint64_t)rs};
+  cuuint32_t box[2] = {(cuuint32_t)box_w, (cuuint32_t)box_h};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 int device_sm_count() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;

@@ -90,6 +90,36 @@ class StuWeights:
 
 
 @dataclasses.dataclass
+class Fp8Weights:
+    """E4M3 copies of a layer's projections for the FP8 forward: W1 and W2
+    transposed to [out][in] bytes, with one fp32 scale per output column
+    (wq[n][k] * scale[n] ~ W[k][n])."""
+    w1q: torch.Tensor  # uint8 [4 d_model, d_model]
+    w1s: torch.Tensor  # [4 d_model]
+    w2q: torch.Tensor  # uint8 [d_model, d_model]
+    w2s: torch.Tensor  # [d_model]
+
+
+def quantize_weight_e4m3(w: torch.Tensor, stream=None):
+    """(wq, scale) for a bf16 [K, N] weight: wq uint8 [N, K] holding E4M3
+    bytes, scale [N] = max_k |w[k, n]| / 448 (1 for a zero column)."""
+    if w.dtype != torch.bfloat16 or not w.is_cuda or w.dim() != 2 or w.stride(1) != 1:
+        raise ValueError("w must be a CUDA bf16 matrix with contiguous rows")
+    K, N = w.shape
+    wq = torch.empty((N, K), dtype=torch.uint8, device=w.device)
+    sc = torch.empty(N, dtype=torch.float32, device=w.device)
+    _check(_abi.load().hstu_quant_weight_e4m3(w.data_ptr(), w.stride(0), K, N, wq.data_ptr(), K,
+                                              sc.data_ptr(), _stream(stream)),
+           "hstu_quant_weight_e4m3")
+    return wq, sc
+
+
+def quantize_weights(w: StuWeights, stream=None) -> Fp8Weights:
+    """The E4M3 projections of one layer (redo after every weight update)."""
+    return Fp8Weights(*quantize_weight_e4m3(w.w1, stream), *quantize_weight_e4m3(w.w2, stream))
+
+
+@dataclasses.dataclass
 class LayerState:
     """What one layer's forward saves for its backward."""
     x: torch.Tensor
@@ -104,7 +134,8 @@ class LayerState:
     stats: torch.Tensor
 
 
-def _layer_params(cfg: StuConfig, w: StuWeights, st: LayerState, out) -> _abi.StuLayerParams:
+def _layer_params(cfg: StuConfig, w: StuWeights, st: LayerState, out,
+                  fp8: Optional[Fp8Weights] = None) -> _abi.StuLayerParams:
     p = _abi.StuLayerParams()
     T = st.x.shape[0]
     p.B, p.H, p.d = st.seq_offsets.numel() - 1, cfg.H, cfg.d
@@ -117,6 +148,10 @@ def _layer_params(cfg: StuConfig, w: StuWeights, st: LayerState, out) -> _abi.St
     p.x, p.out = st.x.data_ptr(), _ptr(out)
     p.xn, p.pre, p.uvqk = st.xn.data_ptr(), st.pre.data_ptr(), st.uvqk.data_ptr()
     p.av, p.y, p.stats = st.av.data_ptr(), st.y.data_ptr(), st.stats.data_ptr()
+    if fp8 is not None:
+        p.fp8 = 1
+        p.w1q, p.w1s, p.w2q, p.w2s = (fp8.w1q.data_ptr(), fp8.w1s.data_ptr(), fp8.w2q.data_ptr(),
+                                      fp8.w2s.data_ptr())
     return p
 
 
@@ -132,8 +167,10 @@ def workspace_bytes(which: int, T: int, B: int, cfg: StuConfig) -> int:
 
 
 def layer_fwd(x: torch.Tensor, seq_offsets: torch.Tensor, num_targets: Optional[torch.Tensor],
-              w: StuWeights, cfg: StuConfig, max_seq_len: int, workspace=None, stream=None):
-    """One STU layer forward; returns (out, state for the backward)."""
+              w: StuWeights, cfg: StuConfig, max_seq_len: int, workspace=None, stream=None,
+              fp8: Optional[Fp8Weights] = None):
+    """One STU layer forward; returns (out, state for the backward).  With
+    fp8 (from quantize_weights) the two projections run in E4M3."""
     _check_x(x, cfg)
     T, dm, dev = x.shape[0], cfg.d_model, x.device
     bf = dict(dtype=torch.bfloat16, device=dev)
@@ -142,8 +179,8 @@ def layer_fwd(x: torch.Tensor, seq_offsets: torch.Tensor, num_targets: Optional[
                     torch.empty((T, 4 * dm), **bf), torch.empty((T, dm), **bf),
                     torch.empty((T, dm), **bf), torch.empty((4, T), dtype=torch.float32, device=dev))
     out = torch.empty((T, dm), **bf)
-    p = _layer_params(cfg, w, st, out)
-    need = workspace_bytes(_abi.WS_FWD, T, p.B, cfg)
+    p = _layer_params(cfg, w, st, out, fp8)
+    need = workspace_bytes(_abi.WS_FWD if fp8 is None else _abi.WS_FWD_FP8, T, p.B, cfg)
     ws = torch.empty(need, dtype=torch.uint8, device=dev) if workspace is None else workspace
     _check(_abi.load().hstu_stu_layer_fwd(ctypes.byref(p), ws.data_ptr(), ws.numel(),
                                           _stream(stream)), "hstu_stu_layer_fwd")
@@ -211,8 +248,10 @@ def jagged_truncate(x, seq_offsets, new_offsets, num_targets, contextual_len: in
 
 
 def gemm(a, b, *, M, N, K, a_mn_major, b_mn_major, epilogue, splits=1, bias=None, resid=None,
-         out=None, out2=None, outf=None, stream=None):
-    """The layer GEMM D[m][n] = sum_k A[m][k] B[n][k] (test hook)."""
+         out=None, out2=None, outf=None, a_scale=None, b_scale=None, stream=None):
+    """The layer GEMM D[m][n] = sum_k A[m][k] B[n][k] (test hook).  With
+    a_scale / b_scale, a and b are E4M3 bytes and D is scaled by
+    a_scale[m] * b_scale[n]."""
     p = _abi.GemmParams()
     p.M, p.N, p.K = M, N, K
     p.a, p.lda, p.a_mn_major = a.data_ptr(), a.stride(0), int(a_mn_major)
@@ -223,6 +262,8 @@ def gemm(a, b, *, M, N, K, a_mn_major, b_mn_major, epilogue, splits=1, bias=None
     p.out, p.ldo = _ptr(out), (out.stride(0) if out is not None else 0)
     p.out2, p.ldo2 = _ptr(out2), (out2.stride(0) if out2 is not None else 0)
     p.outf, p.ldf = _ptr(outf), (outf.stride(0) if outf is not None else 0)
+    if a_scale is not None or b_scale is not None:
+        p.fp8, p.a_scale, p.b_scale = 1, _ptr(a_scale), _ptr(b_scale)
     ws = torch.empty(256, dtype=torch.uint8, device=a.device)
     lib = _abi.load()
     _check(lib.hstu_gemm(ctypes.byref(p), ws.data_ptr(), _stream(stream)), "hstu_gemm")
@@ -233,12 +274,20 @@ class StuStack:
     """`len(weights)` STU layers, truncation after the first `trunc_after`.
 
     cfg_full / cfg_trunc: attention settings before / after truncation (their
-    N differ: the longest sequence of each stage)."""
+    N differ: the longest sequence of each stage).  fp8=True runs the forward
+    projections in E4M3; call requantize() after every weight update."""
 
     def __init__(self, weights: List[StuWeights], cfg_full: StuConfig, cfg_trunc: StuConfig,
-                 trunc_after: int, tail: int):
+                 trunc_after: int, tail: int, fp8: bool = False):
         self.weights, self.cfg_full, self.cfg_trunc = weights, cfg_full, cfg_trunc
         self.trunc_after, self.tail = trunc_after, tail
+        self.fp8 = None
+        if fp8:
+            self.requantize()
+
+    def requantize(self, stream=None):
+        """E4M3 copies of every layer's projections (the FP8 forward's weights)."""
+        self.fp8 = [quantize_weights(w, stream) for w in self.weights]
 
     def forward(self, x, seq_offsets, num_targets, lengths, host_num_targets, stream=None):
         """x: [T, d_model] bf16; lengths / host_num_targets: host copies of the
@@ -256,7 +305,8 @@ class StuStack:
                                     stream=stream)
                 offs = new_offs
             cfg = self.cfg_full if i < self.trunc_after else self.cfg_trunc
-            h, st = layer_fwd(h, offs, num_targets, w, cfg, msl, stream=stream)
+            h, st = layer_fwd(h, offs, num_targets, w, cfg, msl, stream=stream,
+                              fp8=None if self.fp8 is None else self.fp8[i])
             states.append(st)
         return h, (states, seq_offsets, new_offs, num_targets, x.shape[0])
 

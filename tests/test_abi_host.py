@@ -109,3 +109,32 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(_abi, "LIB_PATH", str(tmp_path / "absent.so"))
     with pytest.raises(_abi.LibraryMissing):
         _abi.load()
+
+
+def _c_layout(struct_name, fields, tmp_path):
+    """sizeof and every field's offsetof as gcc lays the header's struct out."""
+    import subprocess
+    src = tmp_path / "layout.c"
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "hstu_stu.h"',
+             'int main(void) {', f'  printf("%zu\\n", sizeof({struct_name}));']
+    lines += [f'  printf("%zu\\n", offsetof({struct_name}, {f}));' for f in fields]
+    lines += ['  return 0;', '}']
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-std=c99", "-I", _abi.INCLUDE_DIR, str(src), "-o", str(exe)],
+                   check=True)
+    return [int(v) for v in subprocess.run([str(exe)], check=True, capture_output=True,
+                                           text=True).stdout.split()]
+
+
+@pytest.mark.parametrize("py,c", [
+    (_abi.FwdParams, "hstu_sla_fwd_params"), (_abi.BwdParams, "hstu_sla_bwd_params"),
+    (_abi.StuLayerParams, "hstu_stu_layer_params"),
+    (_abi.StuLayerBwdParams, "hstu_stu_layer_bwd_params"), (_abi.GemmParams, "hstu_gemm_params"),
+])
+def test_binding_structs_match_the_headers(py, c, tmp_path):
+    """The binding's ctypes structs have the C compiler's size and offsets."""
+    names = [f[0] for f in py._fields_]
+    got = _c_layout(c, names, tmp_path)
+    assert got[0] == ctypes.sizeof(py)
+    assert got[1:] == [getattr(py, n).offset for n in names]

@@ -1,13 +1,24 @@
 """GPU parity of the STU layer around the SLA attention: the tcgen05 GEMM in
 every operand layout / epilogue the layer uses, one full layer forward +
 backward, the truncation gather / scatter, and the 6-layer truncated stack,
-each against oracle/stu.py (fp64) on the same seeded bf16 inputs."""
+each against oracle/stu.py (fp64) on the same seeded bf16 inputs; and the
+FP8 forward projections (E4M3 GEMM, weight quantizer, layer and stack with
+fp8) against oracle/fp8.py.
+
+Tolerances: TOL (2e-2 of max|ref|) wherever both sides compute the same
+values; TOL_FP8 = 6e-2 for the gradients and the stack under the FP8
+forward.  There the two sides quantize activations that already differ by
+the bf16 path's rounding (about 2^-8 relative), so a share of the E4M3 codes
+differs by one step (2^-3 relative); the oracle alone, with its quantizer's
+inputs perturbed by 2^-7 relative noise, moves its parameter gradients by up
+to 3.9% and its layer output by 0.9% of their maxima."""
 import math
 
 import numpy as np
 import pytest
 import torch
 
+from oracle import fp8 as F
 from oracle import stu as S
 from parity import assert_close
 from sparse_hstu_attention_b200 import _abi, stu
@@ -15,6 +26,7 @@ from workloads import STU_LAYERS, STU_TRUNC_AFTER, draw_stu, offsets_from_length
 
 pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda")
+TOL_FP8 = 6e-2
 FIELDS = ("ln1_w", "ln1_b", "w1", "b1", "ln2_w", "ln2_b", "w2", "b2")
 
 
@@ -63,6 +75,70 @@ def test_gemm_layouts_and_epilogues(a_mn, b_mn, epi, M, N, K, splits):
         assert_close("acc + D", outf, f64(acc0) + ref, tol=1e-4)
 
 
+def _e4m3_bytes(x: torch.Tensor) -> torch.Tensor:
+    """Seeded E4M3 operands: torch's conversion of fp32 values, as bytes."""
+    return x.to(torch.float8_e4m3fn).view(torch.uint8)
+
+
+def _decode(b: torch.Tensor) -> np.ndarray:
+    table = np.array([F.e4m3_decode(c) for c in range(256)])
+    return table[b.cpu().numpy().astype(np.int64)]
+
+
+F8_GEMM_CASES = [  # (epilogue, M, N, K)
+    (_abi.GEMM_STORE, 300, 512, 256),
+    (_abi.GEMM_STORE, 129, 1024, 208),      # K tail inside a 128-byte k block
+    (_abi.GEMM_BIAS_SILU, 300, 2048, 512),
+    (_abi.GEMM_BIAS_RESID, 257, 512, 1024),
+]
+
+
+@pytest.mark.parametrize("epi,M,N,K", F8_GEMM_CASES)
+def test_fp8_gemm(epi, M, N, K):
+    """E4M3 x E4M3 -> fp32 with the row / column scales in the epilogue,
+    against fp64 products of the bytes as the format's fields decode them."""
+    g = torch.Generator().manual_seed(M + 3 * N + 5 * K)
+    A = _e4m3_bytes(torch.randn((M, K), generator=g) * 40)
+    B = _e4m3_bytes(torch.randn((N, K), generator=g) * 40)
+    sa = torch.rand(M, generator=g) * 2 ** -5 + 2 ** -6
+    sb = torch.rand(N, generator=g) * 2 ** -5 + 2 ** -6
+    bias = torch.randn(N, generator=g)
+    resid = torch.randn((M, N), generator=g).to(torch.bfloat16)
+    ref = (_decode(A) @ _decode(B).T) * f64(sa)[:, None] * f64(sb)[None, :]
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=DEV)
+    out2 = torch.empty((M, N), dtype=torch.bfloat16, device=DEV)
+    stu.gemm(A.to(DEV), B.to(DEV), M=M, N=N, K=K, a_mn_major=False, b_mn_major=False,
+             epilogue=epi, bias=bias.to(DEV), resid=resid.to(DEV), out=out, out2=out2,
+             a_scale=sa.to(DEV), b_scale=sb.to(DEV))
+    torch.cuda.synchronize()
+    pre = ref + f64(bias)
+    if epi == _abi.GEMM_STORE:
+        assert_close("D", out, ref, tol=1e-2)
+    elif epi == _abi.GEMM_BIAS_SILU:
+        assert_close("D + bias", out2, pre, tol=1e-2)
+        assert_close("SiLU(D + bias)", out, S.silu(pre), tol=1e-2)
+    else:
+        assert_close("D + bias + resid", out, pre + f64(resid), tol=1e-2)
+
+
+def test_fp8_weight_quantizer_is_bit_exact():
+    """Codes and scales of hstu_quant_weight_e4m3 equal the oracle's per-column
+    quantization byte for byte (same bf16 inputs, decisions in fp32 on both
+    sides), including an all-zero column and a column with one outlier."""
+    g = torch.Generator().manual_seed(11)
+    K, N = 512, 2048
+    W = torch.randn((K, N), generator=g) * torch.exp2(
+        torch.randint(-12, 6, (1, N), generator=g).float())
+    W[:, 7] = 0.0
+    W[3, 9] = 3e4
+    W = W.to(torch.bfloat16)
+    wq, ws = stu.quantize_weight_e4m3(W.to(DEV))
+    torch.cuda.synchronize()
+    q, sc = F.quantize_cols(f64(W))
+    assert np.array_equal(ws.cpu().numpy().astype(np.float64), sc)
+    assert np.array_equal(wq.cpu().numpy(), F.e4m3_code(q).T)
+
+
 def _cfgs(lengths, nts, c, K1, K2, tail, trunc=True):
     H, d = 4, 128
     alpha = 1.0 / math.sqrt(d)
@@ -101,6 +177,36 @@ def test_stu_layer_matches_oracle():
         assert_close("d_" + name, getattr(g, name), getattr(rg, name))
 
 
+def test_stu_layer_fp8_forward_matches_oracle():
+    """The layer with E4M3 projections against the oracle's FP8 layer (the
+    same quantization rules), forward and the unchanged backward; and it does
+    differ from the bf16 layer."""
+    lengths, nts = np.array([300, 520, 180]), np.array([16, 10, 5])
+    full, _, _ = _cfgs(lengths, nts, c=8, K1=128, K2=32, tail=64)
+    offs = offsets_from_lengths(lengths)
+    T = int(offs[-1])
+    dr = draw_stu(T, T, full.d_model, 1, seed=2024, perturb=True)
+    w = stu.StuWeights.from_host(dr.layers[0], DEV)
+    q8 = stu.quantize_weights(w)
+    offs_d = torch.tensor(offs, dtype=torch.int32, device=DEV)
+    nts_d = torch.tensor(nts, dtype=torch.int32, device=DEV)
+    x = dr.x.to(DEV)
+    out, st = stu.layer_fwd(x, offs_d, nts_d, w, full, int(lengths.max()), fp8=q8)
+    dx, g = stu.layer_bwd(dr.dout.to(DEV), st, w, full)
+    out_bf, _ = stu.layer_fwd(x, offs_d, nts_d, w, full, int(lengths.max()))
+    torch.cuda.synchronize()
+    wo = _oracle_weights(dr.layers[0])
+    ref, cache = S.layer_fwd(f64(dr.x), wo, offs, nts, _oracle_cfg(full), fp8=True)
+    rdx, rg = S.layer_bwd(f64(dr.dout), wo, cache)
+    assert_close("out", out, ref)
+    assert_close("pre", st.pre, cache["pre"], tol=TOL_FP8)
+    assert_close("dx", dx, rdx)
+    for name in FIELDS:
+        assert_close("d_" + name, getattr(g, name), getattr(rg, name), tol=TOL_FP8)
+    diff = (out.float() - out_bf.float()).abs().max().item()
+    assert diff > 1e-3 * out_bf.float().abs().max().item()
+
+
 def test_truncation_gather_and_scatter_are_exact():
     lengths, nts = np.array([300, 40, 1200, 77]), np.array([16, 3, 64, 0])
     c, tail = 8, 100
@@ -121,9 +227,11 @@ def test_truncation_gather_and_scatter_are_exact():
     assert torch.equal(z.cpu(), ref)
 
 
-def test_stu_stack_matches_oracle():
+@pytest.mark.parametrize("fp8", [False, True])
+def test_stu_stack_matches_oracle(fp8):
     """Six layers, truncation after the third to contextual + the last `tail`
-    history tokens + candidates, every gradient compared."""
+    history tokens + candidates, every gradient compared; fp8: the forward
+    projections in E4M3."""
     lengths, nts = np.array([700, 400, 1100]), np.array([20, 8, 30])
     c, tail = 16, 128
     full, cut, tl = _cfgs(lengths, nts, c=c, K1=128, K2=32, tail=tail)
@@ -131,7 +239,7 @@ def test_stu_stack_matches_oracle():
     T, T_out = int(offs[-1]), int(tl.sum())
     dr = draw_stu(T, T_out, full.d_model, STU_LAYERS, seed=77, perturb=True)
     ws = [stu.StuWeights.from_host(lw, DEV) for lw in dr.layers]
-    stack = stu.StuStack(ws, full, cut, STU_TRUNC_AFTER, tail)
+    stack = stu.StuStack(ws, full, cut, STU_TRUNC_AFTER, tail, fp8=fp8)
     offs_d = torch.tensor(offs, dtype=torch.int32, device=DEV)
     nts_d = torch.tensor(nts, dtype=torch.int32, device=DEV)
     out, ctx = stack.forward(dr.x.to(DEV), offs_d, nts_d, lengths, nts)
@@ -139,23 +247,26 @@ def test_stu_stack_matches_oracle():
     torch.cuda.synchronize()
     wo = [_oracle_weights(lw) for lw in dr.layers]
     ref, cache = S.stack_fwd(f64(dr.x), wo, offs, nts, _oracle_cfg(full), _oracle_cfg(cut),
-                             STU_TRUNC_AFTER, tail)
+                             STU_TRUNC_AFTER, tail, fp8=fp8)
     rdx, rgs = S.stack_bwd(f64(dr.dout), wo, cache)
+    tol = TOL_FP8 if fp8 else 2e-2
     assert out.shape[0] == T_out
-    assert_close("out", out, ref)
-    assert_close("dx", dx, rdx)
+    assert_close("out", out, ref, tol=tol)
+    assert_close("dx", dx, rdx, tol=tol)
     for i in range(STU_LAYERS):
         for name in FIELDS:
-            assert_close(f"layer {i} d_{name}", getattr(gs[i], name), getattr(rgs[i], name))
+            assert_close(f"layer {i} d_{name}", getattr(gs[i], name), getattr(rgs[i], name),
+                         tol=tol)
 
 
 def test_stu_stack_full_size_sampled():
     """The 6-layer STU stack workload at full size (16 sequences of
     U{4096..16384} tokens, truncation to 32 + 1024 + 64 after layer 3), forward
-    and backward on the GPU.  The oracle checks, teacher-forced with the GPU's
-    own layer inputs, layer 1 on the shortest sequence and layer 6 (forward
-    and its dx) on the longest truncated one; every output and gradient must
-    be finite."""
+    and backward on the GPU.  Sequences are independent, so the oracle runs the
+    whole stack, forward and backward, on the shortest sequence alone (same
+    attention settings) and its output rows and dx rows must match; every
+    output and gradient must be finite.  The weight gradients sum over all
+    sequences and are compared at the smaller sizes above."""
     from workloads import STU_TAIL, WORKLOADS, draw_lengths
     w = WORKLOADS["stu"]
     lengths = draw_lengths(w)
@@ -174,29 +285,15 @@ def test_stu_stack_full_size_sampled():
     out, ctx = stack.forward(dr.x.to(DEV), offs_d, nts_d, lengths, nts)
     dx, gs = stack.backward(dr.dout.to(DEV), ctx)
     torch.cuda.synchronize()
-    states = ctx[0]
     for t in [out, dx] + [getattr(g, f) for g in gs for f in FIELDS]:
         assert torch.isfinite(t.float()).all()
     wo = [_oracle_weights(lw) for lw in dr.layers]
-    # layer 1 on the shortest sequence
-    b = int(np.argmin(lengths))
-    s0, s1 = int(offs[b]), int(offs[b + 1])
-    one = np.array([0, s1 - s0])
-    ref1, _ = S.layer_fwd(f64(dr.x[s0:s1]), wo[0], one, nts[b:b + 1], _oracle_cfg(full))
-    assert_close("layer 1 out", states[1].x[s0:s1], ref1)
-    # layer 6 on the longest truncated sequence, fed the GPU's layer-6 input
     new = offsets_from_lengths(tl)
-    b = int(np.argmax(tl))
-    s0, s1 = int(new[b]), int(new[b + 1])
+    b = int(np.argmin(lengths))
+    s0, s1, n0, n1 = int(offs[b]), int(offs[b + 1]), int(new[b]), int(new[b + 1])
     one = np.array([0, s1 - s0])
-    x6 = f64(states[5].x[s0:s1])
-    ref6, cache6 = S.layer_fwd(x6, wo[5], one, nts[b:b + 1], _oracle_cfg(cut))
-    assert_close("layer 6 out", out[s0:s1], ref6)
-    rdx6, _ = S.layer_bwd(f64(dr.dout[s0:s1]), wo[5], cache6)
-    gdx6, _ = stu.layer_bwd(dr.dout[s0:s1].to(DEV).contiguous(), stu.LayerState(
-        states[5].x[s0:s1], torch.tensor(one, dtype=torch.int32, device=DEV),
-        nts_d[b:b + 1], int(tl[b]), *(t[s0:s1].contiguous() for t in (
-            states[5].xn, states[5].pre, states[5].uvqk, states[5].av, states[5].y)),
-        states[5].stats[:, s0:s1].contiguous()), ws[5], cut)
-    torch.cuda.synchronize()
-    assert_close("layer 6 dx", gdx6, rdx6)
+    ref, cache = S.stack_fwd(f64(dr.x[s0:s1]), wo, one, nts[b:b + 1], _oracle_cfg(full),
+                             _oracle_cfg(cut), STU_TRUNC_AFTER, tail)
+    assert_close("out rows of the shortest sequence", out[n0:n1], ref)
+    rdx, _ = S.stack_bwd(f64(dr.dout[n0:n1]), wo, cache)
+    assert_close("dx rows of the shortest sequence", dx[s0:s1], rdx)
