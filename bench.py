@@ -211,6 +211,11 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
+    if args.workload == "mot":
+        print(json.dumps({"impl": "reference",
+                          "unavailable": "the oracle arm times single workloads; "
+                                         "run it on mot_long's shape via the default workloads"}))
+        return
     w = WORKLOADS[args.workload]
     batch = make_batch(w)
     rp, kp = _pair_tables(batch)
@@ -335,12 +340,108 @@ def run_stu(args, world, rank, local):
         torch.distributed.destroy_process_group()
 
 
+def run_mot(args, world, rank, local):
+    """Mixture of Transducers: the SLA attention of three channels (each its own
+    sequences, heads and SLA window) forward and backward, as one grouped
+    launch per pass; the same work as three separate calls per pass is timed
+    beside it."""
+    import sparse_hstu_attention_b200 as sla
+    from workloads import MOT_CHANNELS
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    chans, groups, fl = [], [], 0.0
+    for name, w in MOT_CHANNELS.items():
+        b = make_batch(w, seed=w.seed + 7919 * rank)
+        pairs = F.total_pairs(b.lengths, b.num_targets, w.contextual_len, w.K1, w.K2)
+        fl += F.fwd_flops(pairs, w.H, w.d) + F.bwd_flops(pairs, w.H, w.d)
+        q, k, v, dout = (t.to(dev) for t in (b.q, b.k, b.v, b.dout))
+        g = dict(q=q, k=k, v=v, dout=dout,
+                 seq_offsets=torch.tensor(b.seq_offsets, dtype=torch.int32, device=dev),
+                 num_targets=torch.tensor(b.num_targets, dtype=torch.int32, device=dev),
+                 contextual_len=w.contextual_len, K1=w.K1, K2=w.K2, alpha=w.alpha, N=w.N,
+                 max_seq_len=int(b.lengths.max()), out=torch.empty_like(q))
+        groups.append(g)
+        chans.append({"name": name, "B": int(len(b.lengths)), "T": b.T, "H": w.H, "d": w.d,
+                      "K1": w.K1, "K2": w.K2, "contextual_len": w.contextual_len,
+                      "num_targets": w.num_targets, "N": w.N, "unmasked_pairs_per_head": pairs})
+    sizes = [(g["q"].shape[0], g["seq_offsets"].numel() - 1, g["q"].shape[1], 128)
+             for g in groups]
+    ws_f = torch.empty(sla.hstu_sla_grouped_workspace_bytes(0, sizes), dtype=torch.uint8,
+                       device=dev)
+    ws_b = torch.empty(sla.hstu_sla_grouped_workspace_bytes(1, sizes), dtype=torch.uint8,
+                       device=dev)
+    sep_ws = [(torch.empty(sla.hstu_sla_workspace_bytes(0, *sz), dtype=torch.uint8, device=dev),
+               torch.empty(sla.hstu_sla_workspace_bytes(1, *sz), dtype=torch.uint8, device=dev))
+              for sz in sizes]
+    fwd_keys = ("contextual_len", "K1", "K2", "alpha", "N", "max_seq_len")
+
+    def grouped_step():
+        sla.hstu_sla_fwd_grouped(groups, workspace=ws_f)
+        sla.hstu_sla_bwd_grouped(groups, workspace=ws_b)
+
+    def separate_step():
+        for g, (wf, wb) in zip(groups, sep_ws):
+            kw = {k: g[k] for k in fwd_keys}
+            sla.hstu_sla_fwd(g["q"], g["k"], g["v"], g["seq_offsets"], g["num_targets"],
+                             out=g["out"], workspace=wf, **kw)
+            sla.hstu_sla_bwd(g["dout"], g["q"], g["k"], g["v"], g["seq_offsets"],
+                             g["num_targets"], workspace=wb, **kw)
+
+    def timed(fn, K):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            torch.distributed.barrier()
+        e0.record(stream)
+        for _ in range(K):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / K
+        if world > 1:
+            tt = torch.tensor([ms], device=dev, dtype=torch.float64)
+            torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+            ms = float(tt.item())
+        return ms
+
+    K = args.steps
+    with ClockSampler(local) as clocks:
+        ms = timed(grouped_step, K)
+    status = max(sla.hstu_sla_get_error(ws_f), sla.hstu_sla_get_error(ws_b))
+    if status != 0:
+        raise RuntimeError(f"device status {status}")
+    ms_sep = timed(separate_step, K)
+    if rank == 0:
+        peaks, src = _peaks()
+        peak = float(peaks.get("bf16_tflops_sustained") or peaks.get("bf16_tflops"))
+        value = world * fl / (ms * 1e-3) / 1e12
+        print(json.dumps({
+            "metric": "MoT channels SLA attn fwd+bwd TFLOP/s (unmasked pairs), grouped launch",
+            "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) bf16, jagged lengths per channel recipe)",
+            "config": {"workload": "mot", "channels": chans,
+                       "l2": "inputs > 126 MB L2; no flush"},
+            "separate_calls_ms_per_step": ms_sep, "grouped_speedup": ms_sep / ms,
+            "frac_of_sustained_peak": value / world / peak,
+            # forward: 3 work lists + 1 kernel; backward: 3 work lists + 1 kernel
+            # + 3 dq conversions (memsets not counted)
+            "gpu_launches": K * (3 + 1 + 3 + 1 + 3),
+            "clocks": clocks.summary()}), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="hist16k", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="hist16k", choices=sorted(WORKLOADS) + ["mot"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
@@ -357,6 +458,8 @@ def main():
     torch.cuda.set_device(local)
     if args.workload == "stu":
         return run_stu(args, world, rank, local)
+    if args.workload == "mot":
+        return run_mot(args, world, rank, local)
     dev = torch.device("cuda", local)
     w = WORKLOADS[args.workload]
     batch = make_batch(w, seed=w.seed + 7919 * rank)

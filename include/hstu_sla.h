@@ -75,7 +75,7 @@ typedef struct {
   int32_t K2;                   /* global prefix, >= 0 */
   float alpha;                  /* scale inside SiLU */
   float N;                      /* normaliser, > 0 */
-  const void* q;                /* device bf16 [T, H, d] */
+  const void* q;                /* device bf16 [T, H, d]; the tensors may be NULL when T = 0 */
   const void* k;
   const void* v;
   int64_t q_row_stride;         /* elements between consecutive tokens (>= H*d) */
@@ -142,6 +142,33 @@ int hstu_sla_fwd(const hstu_sla_fwd_params* p, void* workspace, size_t workspace
  *           scores for dq. */
 int hstu_sla_bwd(const hstu_sla_bwd_params* p, void* workspace, size_t workspace_bytes,
                  hstu_stream_t stream);
+
+/* Grouped calls: up to HSTU_SLA_MAX_GROUPS independent problems in ONE
+ * launch of the attention kernel.  The use is the Mixture of Transducers
+ * ("Bending the Scaling Law Curve in Large-Scale Recommendation Systems",
+ * section 4.3; TorchEasyRec "ULTRA HSTU" docs, MoT): one transducer per
+ * user-signal channel, each with its own sequences, SLA window (K1, K2,
+ * contextual_len), N, alpha, heads and tensors.  The kernel's scheduler hands
+ * out the units of all problems from one counter (the backward's prefix key
+ * tiles of every problem first), so short channels fill the tail of long
+ * ones.  Results equal G separate calls: the forward and dk / dv bitwise, dq
+ * to fp32 summation order (as for one call).
+ *   - groups[g] is read as for hstu_sla_fwd / hstu_sla_bwd; every group has
+ *     the same d (the backward: d = 128).  candidates_only is per group.
+ *   - workspace: hstu_sla_grouped_workspace_bytes(which, G, ...) bytes, 256-byte
+ *     aligned: a 256-byte status header (read by hstu_sla_get_error; a
+ *     device-side input error of any group is reported there), then each
+ *     group's own workspace in the order given.
+ *   - groups[0].event_begin / event_end (if set) bracket the attention kernel.
+ * Returns HSTU_SLA_ERR_INVALID_ARG for G outside [1, HSTU_SLA_MAX_GROUPS] or a
+ * bad group, HSTU_SLA_ERR_UNSUPPORTED for mixed d (or d != 128 backward). */
+#define HSTU_SLA_MAX_GROUPS 4
+size_t hstu_sla_grouped_workspace_bytes(int which, int32_t G, const int64_t* total_tokens,
+                                        const int32_t* B, const int32_t* H, const int32_t* d);
+int hstu_sla_fwd_grouped(const hstu_sla_fwd_params* groups, int32_t G, void* workspace,
+                         size_t workspace_bytes, hstu_stream_t stream);
+int hstu_sla_bwd_grouped(const hstu_sla_bwd_params* groups, int32_t G, void* workspace,
+                         size_t workspace_bytes, hstu_stream_t stream);
 
 /* Forward without a caller-provided workspace, for callers that may not
  * allocate device memory: inference engines and plugin hosts that plan all

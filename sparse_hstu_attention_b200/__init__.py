@@ -19,14 +19,16 @@ from __future__ import annotations
 import ctypes
 from typing import Optional
 
+import numpy as np
 import torch
 
 from . import _abi
 from ._abi import LibraryMissing  # noqa: F401
 
-__all__ = ["hstu_sla_fwd", "hstu_sla_fwd_noalloc", "hstu_sla_bwd", "hstu_sla_workspace_bytes", "hstu_sla_count_pairs",
-           "hstu_sla_get_error", "hstu_sla_strerror", "SLAError", "SLAAttention",
-           "sla_attention"]
+__all__ = ["hstu_sla_fwd", "hstu_sla_fwd_noalloc", "hstu_sla_bwd", "hstu_sla_workspace_bytes",
+           "hstu_sla_count_pairs", "hstu_sla_fwd_grouped", "hstu_sla_bwd_grouped",
+           "hstu_sla_grouped_workspace_bytes", "hstu_sla_get_error", "hstu_sla_strerror",
+           "SLAError", "SLAAttention", "sla_attention"]
 
 
 class SLAError(RuntimeError):
@@ -165,6 +167,82 @@ def hstu_sla_bwd(dout: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: torch.
     _check(lib.hstu_sla_bwd(ctypes.byref(p), ws.data_ptr(), ws.numel(), _stream_ptr(stream)),
            "hstu_sla_bwd")
     return dq, dk, dv
+
+
+def hstu_sla_grouped_workspace_bytes(which: int, problems) -> int:
+    """Workspace of a grouped call; problems: (total_tokens, B, H, d) per group."""
+    G = len(problems)
+    arr = [np.asarray([p[i] for p in problems], dtype=dt)
+           for i, dt in enumerate((np.int64, np.int32, np.int32, np.int32))]
+    ptrs = [a.ctypes.data for a in arr]
+    return int(_abi.load().hstu_sla_grouped_workspace_bytes(which, G, *ptrs))
+
+
+def _group_params(g: dict, events=None) -> _abi.FwdParams:
+    return _fwd_params(g["q"], g["k"], g["v"], g["seq_offsets"], g.get("num_targets"),
+                       g["contextual_len"], g["K1"], g["K2"], g["alpha"], g["N"],
+                       g.get("max_seq_len"), events, g.get("candidates_only", False))
+
+
+def _grouped_ws(which, params, device, workspace):
+    need = hstu_sla_grouped_workspace_bytes(
+        which, [(p.total_tokens, p.B, p.H, p.d) for p in params])
+    if need == 0:
+        raise ValueError("invalid grouped problem sizes")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=device)
+    if workspace.numel() < need:
+        raise ValueError(f"workspace too small: {workspace.numel()} < {need} bytes")
+    return workspace
+
+
+def hstu_sla_fwd_grouped(groups, *, workspace=None, stream=None, events=None):
+    """Several independent SLA forwards (e.g. the channels of a Mixture of
+    Transducers) in one launch.  groups: list of dicts with the keyword
+    arguments of hstu_sla_fwd plus q, k, v, seq_offsets (num_targets,
+    max_seq_len, out, candidates_only optional).  Returns the outputs."""
+    lib = _abi.load()
+    G = len(groups)
+    arr = (_abi.FwdParams * G)()
+    outs = []
+    for i, g in enumerate(groups):
+        p = _group_params(g, events if i == 0 else None)
+        out = g.get("out")
+        if out is None:
+            out = torch.empty(g["q"].shape, dtype=torch.bfloat16, device=g["q"].device)
+        p.out = out.data_ptr()
+        p.out_row_stride = _row_stride(out, "out", p.H, p.d)
+        arr[i] = p
+        outs.append(out)
+    ws = _grouped_ws(_abi.WS_FWD, list(arr), groups[0]["q"].device, workspace)
+    _check(lib.hstu_sla_fwd_grouped(arr, G, ws.data_ptr(), ws.numel(), _stream_ptr(stream)),
+           "hstu_sla_fwd_grouped")
+    return outs
+
+
+def hstu_sla_bwd_grouped(groups, *, workspace=None, stream=None, events=None):
+    """Several independent SLA backwards in one launch (head_dim 128).  groups:
+    as for hstu_sla_fwd_grouped plus dout.  Returns [(dq, dk, dv)] per group."""
+    lib = _abi.load()
+    G = len(groups)
+    arr = (_abi.BwdParams * G)()
+    grads = []
+    for i, g in enumerate(groups):
+        b = _abi.BwdParams()
+        b.fwd = _group_params(g, events if i == 0 else None)
+        q, H, d = g["q"], b.fwd.H, b.fwd.d
+        dq, dk, dv = (torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
+                      for _ in range(3))
+        b.dout, b.dout_row_stride = g["dout"].data_ptr(), _row_stride(g["dout"], "dout", H, d)
+        b.dq, b.dq_row_stride = dq.data_ptr(), _row_stride(dq, "dq", H, d)
+        b.dk, b.dk_row_stride = dk.data_ptr(), _row_stride(dk, "dk", H, d)
+        b.dv, b.dv_row_stride = dv.data_ptr(), _row_stride(dv, "dv", H, d)
+        arr[i] = b
+        grads.append((dq, dk, dv))
+    ws = _grouped_ws(_abi.WS_BWD, [b.fwd for b in arr], groups[0]["q"].device, workspace)
+    _check(lib.hstu_sla_bwd_grouped(arr, G, ws.data_ptr(), ws.numel(), _stream_ptr(stream)),
+           "hstu_sla_bwd_grouped")
+    return grads
 
 
 def hstu_sla_count_pairs(q, k, v, seq_offsets, num_targets, *, contextual_len, K1, K2,

@@ -21,6 +21,7 @@ ERR_TIMEOUT = -6
 
 WS_FWD = 0
 WS_BWD = 1
+MAX_GROUPS = 4   # HSTU_SLA_MAX_GROUPS
 WS_FWD_FP8 = 2   # hstu_stu_workspace_bytes only: the layer forward with fp8 = 1
 
 
@@ -125,6 +126,13 @@ def load():
     lib.hstu_sla_fwd_noalloc.restype = ctypes.c_int
     lib.hstu_sla_count_pairs.argtypes = [ctypes.POINTER(FwdParams), vp, vp, vp, sz, vp]
     lib.hstu_sla_count_pairs.restype = ctypes.c_int
+    lib.hstu_sla_grouped_workspace_bytes.argtypes = [ctypes.c_int, ctypes.c_int32, vp, vp, vp,
+                                                     vp]
+    lib.hstu_sla_grouped_workspace_bytes.restype = sz
+    lib.hstu_sla_fwd_grouped.argtypes = [ctypes.POINTER(FwdParams), ctypes.c_int32, vp, sz, vp]
+    lib.hstu_sla_fwd_grouped.restype = ctypes.c_int
+    lib.hstu_sla_bwd_grouped.argtypes = [ctypes.POINTER(BwdParams), ctypes.c_int32, vp, sz, vp]
+    lib.hstu_sla_bwd_grouped.restype = ctypes.c_int
     lib.hstu_sla_get_error.argtypes = [vp, vp]
     lib.hstu_sla_get_error.restype = ctypes.c_int
     lib.hstu_sla_strerror.argtypes = [ctypes.c_int]

@@ -9,11 +9,14 @@ using namespace hstu;
 
 namespace {
 
-constexpr int kAbiVersion = 102;  // 101: hstu_sla_fwd_params.candidates_only; 102: FP8 forward
+// 101: hstu_sla_fwd_params.candidates_only; 102: FP8 forward; 103: grouped calls
+constexpr int kAbiVersion = 103;
+static_assert(HSTU_SLA_MAX_GROUPS == kMaxGroups, "one grouped launch holds every group");
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 int check_tensor(const void* p, int64_t rs, const hstu_sla_fwd_params* f) {
+  if (p == nullptr && f->total_tokens == 0) return HSTU_SLA_OK;  // nothing is read or written
   if (p == nullptr) return HSTU_SLA_ERR_INVALID_ARG;
   if (!aligned16(p)) return HSTU_SLA_ERR_INVALID_ARG;
   if (rs < (int64_t)f->H * f->d || (rs % 8) != 0) return HSTU_SLA_ERR_INVALID_ARG;
@@ -73,6 +76,24 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? HSTU_SLA_OK : HSTU_SL
 
 cudaError_t record(void* ev, cudaStream_t st) {
   return ev ? cudaEventRecord(reinterpret_cast<cudaEvent_t>(ev), st) : cudaSuccess;
+}
+
+size_t round256(size_t n) { return (n + 255) & ~size_t(255); }
+
+// Launch order of a group's problems: larger windows (longer units) first.
+void order_by_window(const hstu_sla_fwd_params* const* f, int G, int* order) {
+  auto cost = [&](int g) {
+    const int64_t m = f[g]->max_seq_len;
+    const int64_t k2e = f[g]->K2 > f[g]->contextual_len ? f[g]->K2 : f[g]->contextual_len;
+    return (f[g]->K1 < m ? f[g]->K1 : m) + (k2e < m ? k2e : m);
+  };
+  for (int g = 0; g < G; ++g) order[g] = g;
+  for (int i = 1; i < G; ++i)  // insertion sort, stable
+    for (int j = i; j > 0 && cost(order[j]) > cost(order[j - 1]); --j) {
+      const int t = order[j];
+      order[j] = order[j - 1];
+      order[j - 1] = t;
+    }
 }
 
 }  // namespace
@@ -147,6 +168,119 @@ int hstu_sla_bwd(const hstu_sla_bwd_params* p, void* workspace, size_t workspace
     if (ce == cudaSuccess) ce = launch_bwd_tc(a, f->d, /*kv_pass=*/false, st);
     if (ce == cudaSuccess) ce = record(f->event_end, st);
   }
+  return cuda_status(ce);
+}
+
+size_t hstu_sla_grouped_workspace_bytes(int which, int32_t G, const int64_t* total_tokens,
+                                        const int32_t* B, const int32_t* H, const int32_t* d) {
+  if (G < 1 || G > HSTU_SLA_MAX_GROUPS || !total_tokens || !B || !H || !d) return 0;
+  size_t n = sizeof(WsHeader);
+  for (int g = 0; g < G; ++g) {
+    const size_t b = hstu_sla_workspace_bytes(which, total_tokens[g], B[g], H[g], d[g]);
+    if (b == 0) return 0;
+    n += round256(b);
+  }
+  return n;
+}
+
+int hstu_sla_fwd_grouped(const hstu_sla_fwd_params* groups, int32_t G, void* workspace,
+                         size_t workspace_bytes, hstu_stream_t stream) {
+  if (groups == nullptr || G < 1 || G > HSTU_SLA_MAX_GROUPS) return HSTU_SLA_ERR_INVALID_ARG;
+  int64_t T[HSTU_SLA_MAX_GROUPS];
+  int32_t Bs[HSTU_SLA_MAX_GROUPS], Hs[HSTU_SLA_MAX_GROUPS], ds[HSTU_SLA_MAX_GROUPS];
+  const hstu_sla_fwd_params* f[HSTU_SLA_MAX_GROUPS];
+  int e;
+  for (int g = 0; g < G; ++g) {
+    f[g] = &groups[g];
+    if ((e = check_common(f[g]))) return e;
+    if ((e = check_tensor(f[g]->out, f[g]->out_row_stride, f[g]))) return e;
+    if (f[g]->d != f[0]->d) return HSTU_SLA_ERR_UNSUPPORTED;
+    T[g] = f[g]->total_tokens;
+    Bs[g] = f[g]->B;
+    Hs[g] = f[g]->H;
+    ds[g] = f[g]->d;
+  }
+  if ((e = check_ws(workspace, workspace_bytes,
+                    hstu_sla_grouped_workspace_bytes(HSTU_SLA_WS_FWD, G, T, Bs, Hs, ds))))
+    return e;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t ce = cudaMemsetAsync(workspace, 0, sizeof(WsHeader), st);
+  AttnArgs a[HSTU_SLA_MAX_GROUPS];
+  char* w = static_cast<char*>(workspace) + sizeof(WsHeader);
+  for (int g = 0; g < G && ce == cudaSuccess; ++g) {
+    a[g] = make_args(f[g], w);
+    a[g].out = static_cast<bf16*>(f[g]->out);
+    a[g].o_rs = f[g]->out_row_stride;
+    ce = launch_worklist(a[g], kFwdBM, 0, true, st);
+    w += round256(hstu_sla_workspace_bytes(HSTU_SLA_WS_FWD, T[g], Bs[g], Hs[g], ds[g]));
+  }
+  int order[HSTU_SLA_MAX_GROUPS];
+  order_by_window(f, G, order);
+  GroupSet gs;
+  memset(&gs, 0, sizeof(gs));
+  for (int k = 0; k < G; ++k) gs.g[k] = a[order[k]];
+  gs.common = static_cast<WsHeader*>(workspace);
+  gs.G = G;
+  if (ce == cudaSuccess) ce = record(f[0]->event_begin, st);
+  if (ce == cudaSuccess) ce = launch_fwd_grouped(gs, f[0]->d, st);
+  if (ce == cudaSuccess) ce = record(f[0]->event_end, st);
+  return cuda_status(ce);
+}
+
+int hstu_sla_bwd_grouped(const hstu_sla_bwd_params* groups, int32_t G, void* workspace,
+                         size_t workspace_bytes, hstu_stream_t stream) {
+  if (groups == nullptr || G < 1 || G > HSTU_SLA_MAX_GROUPS) return HSTU_SLA_ERR_INVALID_ARG;
+  int64_t T[HSTU_SLA_MAX_GROUPS];
+  int32_t Bs[HSTU_SLA_MAX_GROUPS], Hs[HSTU_SLA_MAX_GROUPS], ds[HSTU_SLA_MAX_GROUPS];
+  const hstu_sla_fwd_params* f[HSTU_SLA_MAX_GROUPS];
+  int e;
+  for (int g = 0; g < G; ++g) {
+    const hstu_sla_bwd_params* p = &groups[g];
+    f[g] = &p->fwd;
+    if ((e = check_common(f[g]))) return e;
+    if ((e = check_tensor(p->dout, p->dout_row_stride, f[g]))) return e;
+    if ((e = check_tensor(p->dq, p->dq_row_stride, f[g]))) return e;
+    if ((e = check_tensor(p->dk, p->dk_row_stride, f[g]))) return e;
+    if ((e = check_tensor(p->dv, p->dv_row_stride, f[g]))) return e;
+    if (f[g]->d != kFusedBwdD) return HSTU_SLA_ERR_UNSUPPORTED;
+    T[g] = f[g]->total_tokens;
+    Bs[g] = f[g]->B;
+    Hs[g] = f[g]->H;
+    ds[g] = f[g]->d;
+  }
+  if ((e = check_ws(workspace, workspace_bytes,
+                    hstu_sla_grouped_workspace_bytes(HSTU_SLA_WS_BWD, G, T, Bs, Hs, ds))))
+    return e;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t ce = cudaMemsetAsync(workspace, 0, sizeof(WsHeader), st);
+  AttnArgs a[HSTU_SLA_MAX_GROUPS];
+  char* w = static_cast<char*>(workspace) + sizeof(WsHeader);
+  for (int g = 0; g < G && ce == cudaSuccess; ++g) {
+    const hstu_sla_bwd_params* p = &groups[g];
+    a[g] = make_args(f[g], w);
+    a[g].cand_only = 0;
+    a[g].dout = static_cast<const bf16*>(p->dout);
+    a[g].dq = static_cast<bf16*>(p->dq);
+    a[g].dk = static_cast<bf16*>(p->dk);
+    a[g].dv = static_cast<bf16*>(p->dv);
+    a[g].do_rs = p->dout_row_stride;
+    a[g].dq_rs = p->dq_row_stride;
+    a[g].dk_rs = p->dk_row_stride;
+    a[g].dv_rs = p->dv_row_stride;
+    a[g].dqacc = reinterpret_cast<float*>(w + ws_bytes(T[g], Bs[g]));
+    ce = launch_worklist(a[g], kKvBN, 1, true, st);
+    w += round256(hstu_sla_workspace_bytes(HSTU_SLA_WS_BWD, T[g], Bs[g], Hs[g], ds[g]));
+  }
+  int order[HSTU_SLA_MAX_GROUPS];
+  order_by_window(f, G, order);
+  GroupSet gs;
+  memset(&gs, 0, sizeof(gs));
+  for (int k = 0; k < G; ++k) gs.g[k] = a[order[k]];
+  gs.common = static_cast<WsHeader*>(workspace);
+  gs.G = G;
+  if (ce == cudaSuccess) ce = record(f[0]->event_begin, st);
+  if (ce == cudaSuccess) ce = launch_bwd_fused_grouped(gs, st);
+  if (ce == cudaSuccess) ce = record(f[0]->event_end, st);
   return cuda_status(ce);
 }
 

@@ -90,30 +90,45 @@ enum {
 };
 static_assert(8 * F_COUNT <= 512, "barrier area");
 
-// Unit u: key-tile work-list entry u / H, head u % H, and the query tiles
-// that see its keys.  u < 0 ends the schedule.
-__device__ void decode_kv_unit(const AttnArgs& a, int u, UnitRec* r) {
-  if (u < 0) {
-    r->nsteps = -1;
-    return;
+// Unit u of the schedule: the prefix key tiles of every problem first (the
+// longest units: every later row sees a prefix key), then the other key
+// tiles, problem after problem; within a problem's part, item u / H, head
+// u % H.  Past the last unit the record ends the schedule.
+__device__ void decode_kv_unit(const GroupSet& gs, int u, UnitRec* r) {
+  for (int part = 0; part < 2 && u >= 0; ++part) {
+    for (int p = 0; p < kMaxGroups && p < gs.G; ++p) {
+      const AttnArgs& a = gs.g[p];
+      const int n_pre = a.ws->n_items2_pre;
+      const int units = (part == 0 ? n_pre : a.ws->n_items2 - n_pre) * a.H;
+      if (u < units) {
+        const int idx = u / a.H;
+        const int h = u - idx * a.H;
+        const int2 it = a.items2[(part == 0 ? 0 : n_pre) + idx];
+        const SeqGeom g = seq_geom(a, it.x);
+        const int t0 = it.y * kRes;
+        const int t1 = imin(t0 + kRes, g.L);
+        unit_rec_fill(r, h, g.s0, g.L, g.Lh, t0, t1,
+                      k_tile_q_tiles(t0, t1, g.L, g.Lh, a.K1, a.K2e, kStr));
+        r->grp = p;
+        return;
+      }
+      u -= units;
+    }
   }
-  const int idx = u / a.H;
-  const int h = u - idx * a.H;
-  const int2 it = a.items2[idx];
-  const SeqGeom g = seq_geom(a, it.x);
-  const int t0 = it.y * kRes;
-  const int t1 = imin(t0 + kRes, g.L);
-  unit_rec_fill(r, h, g.s0, g.L, g.Lh, t0, t1, k_tile_q_tiles(t0, t1, g.L, g.Lh, a.K1, a.K2e, kStr));
+  r->nsteps = -1;
 }
+
+// k, v, q, dout maps of every problem of a launch.
+struct BwdMaps {
+  CUtensorMap k[kMaxGroups], v[kMaxGroups], q[kMaxGroups], dout[kMaxGroups];
+};
 
 // Fire-and-forget fp32 addition in L2 (the result is unused, so this is a
 // reduction, not a round trip).
 __device__ __forceinline__ void red_add_f32(float* p, uint32_t v) { atomicAdd(p, __uint_as_float(v)); }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    bwd_kvq_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
-                   const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmdo,
-                   const AttnArgs a) {
+    bwd_kvq_kernel(const __grid_constant__ BwdMaps maps, const __grid_constant__ GroupSet gs) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -126,8 +141,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + OFF_SLOT);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (load_status(a.ws) != 0) return;
-  const int total = a.ws->n_items2 * a.H;
+  WsHeader* const ws = gs.common;  // status word and scheduler of the launch
+  // a problem's device-side input check failed: report it for the launch
+  for (int p = 0; p < kMaxGroups && p < gs.G; ++p) {
+    const int st = load_status(gs.g[p].ws);
+    if (st != 0) {
+      if (threadIdx.x == 0) set_status(ws, st);
+      return;
+    }
+  }
+  if (load_status(ws) != 0) return;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -152,10 +175,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(bar(F_DRAIN), 1);
     fence_barrier_init();
-    prefetch_tmap(&tmk);
-    prefetch_tmap(&tmv);
-    prefetch_tmap(&tmq);
-    prefetch_tmap(&tmdo);
+    for (int p = 0; p < kMaxGroups && p < gs.G; ++p) {
+      if (gs.g[p].T == 0) continue;  // no map was built
+      prefetch_tmap(&maps.k[p]);
+      prefetch_tmap(&maps.v[p]);
+      prefetch_tmap(&maps.q[p]);
+      prefetch_tmap(&maps.dout[p]);
+    }
   }
   if (warp == 1) {
     tmem_alloc(smem_addr(tmem_slot), kTmemCols);
@@ -174,11 +200,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int kk = 0; ok; ++kk) {
       const int slot = kk % kUSlots;
-      ok = warp_wait(bar(F_U_EMPTY + slot), ((kk / kUSlots) & 1) ^ 1, a.ws);
+      ok = warp_wait(bar(F_U_EMPTY + slot), ((kk / kUSlots) & 1) ^ 1, ws);
       if (!ok) break;
       if (lane == 0) {
-        const int u = atomicAdd(&a.ws->sched2, 1);
-        decode_kv_unit(a, u < total ? u : -1, &ring[slot]);
+        decode_kv_unit(gs, atomicAdd(&ws->sched2, 1), &ring[slot]);
         mbar_arrive(bar(F_U_FULL + slot));
       }
       __syncwarp();
@@ -187,45 +212,47 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (nt < 0) break;
       if (nt == 0) continue;
       const int h = r->h, y0 = r->s0 + r->t0;
+      const int p = r->grp;
       // K buffer kn % 2: free once the unit two back issued its last dQ MMA
       const uint32_t kb = kn & 1;
-      ok = warp_wait(bar(F_K_EMPTY + kb), ((kn >> 1) & 1) ^ 1, a.ws);
+      ok = warp_wait(bar(F_K_EMPTY + kb), ((kn >> 1) & 1) ^ 1, ws);
       if (!ok) break;
       if (lane == 0) {
         const uint32_t fb = bar(F_K_FULL + kb);
         mbar_expect_tx(fb, RTILE);
         for (int b = 0; b < NB; ++b)
-          tma_load_2d(sK + kb * RTILE + b * RBLK, &tmk, fb, h * D + b * BOXW, y0);
+          tma_load_2d(sK + kb * RTILE + b * RBLK, &maps.k[p], fb, h * D + b * BOXW, y0);
       }
       ++kn;
       // V: free once the previous unit's last score MMA is done
-      ok = warp_wait(bar(F_V_EMPTY), (vn & 1) ^ 1, a.ws);
+      ok = warp_wait(bar(F_V_EMPTY), (vn & 1) ^ 1, ws);
       if (!ok) break;
       if (lane == 0) {
         const uint32_t fb = bar(F_V_FULL);
         mbar_expect_tx(fb, RTILE);
-        for (int b = 0; b < NB; ++b) tma_load_2d(sV + b * RBLK, &tmv, fb, h * D + b * BOXW, y0);
+        for (int b = 0; b < NB; ++b)
+          tma_load_2d(sV + b * RBLK, &maps.v[p], fb, h * D + b * BOXW, y0);
       }
       ++vn;
       SpanCursor c;
       c.begin(r);
       for (int n = 0; n < nt && ok; ++n, c.next(r)) {
         const int s = bn % kSt;
-        ok = warp_wait(bar(F_B_EMPTY + s), ((bn / kSt) & 1) ^ 1, a.ws);
+        ok = warp_wait(bar(F_B_EMPTY + s), ((bn / kSt) & 1) ^ 1, ws);
         if (!ok) break;
         if (lane == 0) {
           const uint32_t fb = bar(F_B_FULL + s);
           mbar_expect_tx(fb, 2 * STILE);
           const int y = r->s0 + c.j * kStr;
           for (int b = 0; b < NB; ++b) {
-            tma_load_2d(sB1 + s * STILE + b * SBLK, &tmq, fb, h * D + b * BOXW, y);
-            tma_load_2d(sB2 + s * STILE + b * SBLK, &tmdo, fb, h * D + b * BOXW, y);
+            tma_load_2d(sB1 + s * STILE + b * SBLK, &maps.q[p], fb, h * D + b * BOXW, y);
+            tma_load_2d(sB2 + s * STILE + b * SBLK, &maps.dout[p], fb, h * D + b * BOXW, y);
           }
         }
         ++bn;
       }
     }
-    if (lane == 0 && load_status(a.ws) != 0) {  // drain copies in flight before exiting
+    if (lane == 0 && load_status(ws) != 0) {  // drain copies in flight before exiting
       for (uint32_t kb = 0; kb < 2; ++kb) {
         const uint32_t armed = kn / 2 + (kb < (kn & 1) ? 1u : 0u);
         if (armed > 0) drain_wait(bar(F_K_FULL + kb), (armed - 1) & 1);
@@ -262,8 +289,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // MMAs of the step with ring counter bm / X counter xm, K buffer kb
       auto acc = [&](uint32_t bm, uint32_t xm, uint32_t kb, bool first, bool last) -> bool {
         const uint32_t b = xm & 1;
-        if (!mbar_wait(bar(F_OP_FULL + b), (xm >> 1) & 1, a.ws)) return false;
-        if (first && !mbar_wait(bar(F_ACC_EMPTY), (accn & 1) ^ 1, a.ws)) return false;
+        if (!mbar_wait(bar(F_OP_FULL + b), (xm >> 1) & 1, ws)) return false;
+        if (first && !mbar_wait(bar(F_ACC_EMPTY), (accn & 1) ^ 1, ws)) return false;
         tc_fence_after();
         const uint64_t dKt = dKt0 + ((kb * RTILE) >> 4);
         const uint64_t dS = dDS + ((b * DSTILE) >> 4);
@@ -289,22 +316,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       for (int kk = 0; ok; ++kk) {
         const int slot = kk % kUSlots;
-        ok = mbar_wait(bar(F_U_FULL + slot), (kk / kUSlots) & 1, a.ws);
+        ok = mbar_wait(bar(F_U_FULL + slot), (kk / kUSlots) & 1, ws);
         if (!ok) break;
         const int nt = ring[slot].nsteps;
         mbar_arrive(bar(F_U_EMPTY + slot));
         if (nt < 0) break;
         if (nt == 0) continue;
         const uint32_t kb = an & 1;
-        ok = mbar_wait(bar(F_K_FULL + kb), (an >> 1) & 1, a.ws) &&
-             mbar_wait(bar(F_V_FULL), an & 1, a.ws);
+        ok = mbar_wait(bar(F_K_FULL + kb), (an >> 1) & 1, ws) &&
+             mbar_wait(bar(F_V_FULL), an & 1, ws);
         if (!ok) break;
         tc_fence_after();
         const uint64_t dK = dK0 + ((kb * RTILE) >> 4);
         const uint32_t bn0 = bn, xc0 = xc;
         for (int n = 0; n < nt; ++n) {
           const int s = bn % kSt;
-          ok = mbar_wait(bar(F_B_FULL + s), (bn / kSt) & 1, a.ws);
+          ok = mbar_wait(bar(F_B_FULL + s), (bn / kSt) & 1, ws);
           if (!ok) break;
           tc_fence_after();
           const uint32_t b = xc & 1;
@@ -314,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_ss(tmem + kColX1 + b * 64, dK + koff(ks, RBLK), dB1 + so + koff(ks, SBLK), IDESC_X,
                    ks > 0 ? 1u : 0u);
           // X2(b) still holds the dQ^T of step xc - 2 until its drain is done
-          ok = mbar_wait(bar(F_DQ_EMPTY + b), ((xc >> 1) & 1) ^ 1, a.ws);
+          ok = mbar_wait(bar(F_DQ_EMPTY + b), ((xc >> 1) & 1) ^ 1, ws);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
@@ -358,9 +385,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int half = chunk & 1;           // query-column half within the group
     const int row = quarter * 32 + lane;  // key row (and head-dim lane of dQ^T)
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-    const uint64_t half_alpha2 = f2s(0.5f * a.alpha);
-    // dS is produced as 2 dP SiLU'(x): its consumers take alpha / (2N)
-    const float sc_dv = a.inv_n, sc_dk = 0.5f * a.alpha * a.inv_n;
     const int col = half * 32;
     const uint32_t ds_row = sDS + (uint32_t)row * SW;
     const uint32_t swz = (uint32_t)(row & 7);
@@ -368,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int kk = 0; ok; ++kk) {
       const int slot = kk % kUSlots;
-      ok = warp_wait(bar(F_U_FULL + slot), (kk / kUSlots) & 1, a.ws);
+      ok = warp_wait(bar(F_U_FULL + slot), (kk / kUSlots) & 1, ws);
       if (!ok) break;
       const UnitRec* r = &ring[slot];
       const int nt = r->nsteps;
@@ -377,9 +401,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       const int h = r->h, s0 = r->s0, L = r->L, Lh = r->Lh, t0 = r->t0, t1 = r->t1;
+      const AttnArgs& A = gs.g[r->grp];
+      const int K1 = A.K1, K2e = A.K2e;
+      const uint64_t half_alpha2 = f2s(0.5f * A.alpha);
+      // dS is produced as 2 dP SiLU'(x): its consumers take alpha / (2N)
+      const float sc_dv = A.inv_n, sc_dk = 0.5f * A.alpha * A.inv_n;
       const int rr = t0 + row;  // this thread's key position in the sequence
-      bf16* o1 = a.dv + (int64_t)(s0 + rr) * a.dv_rs + h * D + chunk * 32;
-      bf16* o2 = a.dk + (int64_t)(s0 + rr) * a.dk_rs + h * D + chunk * 32;
+      bf16* o1 = A.dv + (int64_t)(s0 + rr) * A.dv_rs + h * D + chunk * 32;
+      bf16* o2 = A.dk + (int64_t)(s0 + rr) * A.dk_rs + h * D + chunk * 32;
       if (nt == 0) {  // keys no row sees
         if (rr < t1) {
           const uint4 z = make_uint4(0, 0, 0, 0);
@@ -392,20 +421,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         warp_arrive(bar(F_U_EMPTY + slot));
         continue;
       }
-      const KeyMask km = key_mask(rr, L, Lh, a.K1, a.K2e);
+      const KeyMask km = key_mask(rr, L, Lh, K1, K2e);
       // dQ workspace ([H][T][D]) column of this lane (head-dim index `row`)
       // at the sequence start
-      float* dqa = a.dqacc + ((int64_t)h * a.T + s0) * D + row;
+      float* dqa = A.dqacc + ((int64_t)h * A.T + s0) * D + row;
       SpanCursor c;
       c.begin(r);
       for (int n = 0; n < nt; ++n, ++xc, c.next(r)) {
         const uint32_t b = xc & 1;
         if ((int)b != grp) continue;  // the other group's step
-        ok = warp_wait(bar(F_X_FULL + b), (xc >> 1) & 1, a.ws);
+        ok = warp_wait(bar(F_X_FULL + b), (xc >> 1) & 1, ws);
         if (!ok) break;
         tc_fence_after();
         const int c0 = c.j * kStr;  // first query row of this step
-        const bool full = tile_full(c0, c0 + kStr, t0, t0 + kRes, Lh, a.K1, a.K2e);
+        const bool full = tile_full(c0, c0 + kStr, t0, t0 + kRes, Lh, K1, K2e);
         const uint32_t xs_addr = lane_base + kColX1 + b * 64 + col;
         const uint32_t xd_addr = lane_base + kColX2 + b * 64 + col;
         const uint32_t dsr = ds_row + b * DSTILE;
@@ -444,7 +473,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         warp_arrive(bar(F_OP_FULL + b));
         // ------------------------------------------- dQ^T of this step
-        ok = warp_wait(bar(F_DQ_FULL + b), (xc >> 1) & 1, a.ws);
+        ok = warp_wait(bar(F_DQ_FULL + b), (xc >> 1) & 1, ws);
         if (!ok) break;
         tc_fence_after();
         uint32_t g0[16], g1[16];
@@ -473,7 +502,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
       // ---------------------------------------------------------- epilogue
-      ok = warp_wait(bar(F_ACC_FULL), accn & 1, a.ws);
+      ok = warp_wait(bar(F_ACC_FULL), accn & 1, ws);
       if (!ok) break;
       tc_fence_after();
 #pragma unroll 1
@@ -541,28 +570,50 @@ __global__ void __launch_bounds__(256) dq_convert_kernel(const float* __restrict
 
 }  // namespace
 
-cudaError_t launch_bwd_fused(const AttnArgs& a, cudaStream_t st) {
-  if (a.T == 0) return cudaSuccess;
-  const int HD = a.H * D;
-  CUtensorMap mk, mv, mq, mdo;
-  if (!make_tma_2d(&mk, a.k, a.T, HD, a.k_rs, BOXW, kRes, true) ||
-      !make_tma_2d(&mv, a.v, a.T, HD, a.v_rs, BOXW, kRes, true) ||
-      !make_tma_2d(&mq, a.q, a.T, HD, a.q_rs, BOXW, kStr, true) ||
-      !make_tma_2d(&mdo, a.dout, a.T, HD, a.do_rs, BOXW, kStr, true))
-    return cudaErrorInvalidValue;
-  cudaError_t e = cudaMemsetAsync(a.dqacc, 0, dq_workspace_bytes(a.T, a.H, D), st);
-  if (e != cudaSuccess) return e;
+cudaError_t launch_bwd_fused_grouped(const GroupSet& gs, cudaStream_t st) {
+  if (gs.G < 1 || gs.G > kMaxGroups) return cudaErrorInvalidValue;
+  BwdMaps m;
+  memset(&m, 0, sizeof(m));
+  int64_t units = 0;
+  cudaError_t e;
+  for (int p = 0; p < gs.G; ++p) {
+    const AttnArgs& a = gs.g[p];
+    if (a.T == 0) continue;  // no units; its maps stay unused
+    const int HD = a.H * D;
+    if (!make_tma_2d(&m.k[p], a.k, a.T, HD, a.k_rs, BOXW, kRes, true) ||
+        !make_tma_2d(&m.v[p], a.v, a.T, HD, a.v_rs, BOXW, kRes, true) ||
+        !make_tma_2d(&m.q[p], a.q, a.T, HD, a.q_rs, BOXW, kStr, true) ||
+        !make_tma_2d(&m.dout[p], a.dout, a.T, HD, a.do_rs, BOXW, kStr, true))
+      return cudaErrorInvalidValue;
+    if ((e = cudaMemsetAsync(a.dqacc, 0, dq_workspace_bytes(a.T, a.H, D), st)) != cudaSuccess)
+      return e;
+    units += max_items(a.T, a.B) * a.H;
+  }
+  if (units == 0) return cudaSuccess;
   e = cudaFuncSetAttribute(bwd_kvq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
   if (e != cudaSuccess) return e;
-  const int64_t units = max_items(a.T, a.B) * a.H;
   const int sms = device_sm_count();
   const int grid = (int)(units < sms ? units : sms);
-  bwd_kvq_kernel<<<grid, kThreads, SMEM, st>>>(mk, mv, mq, mdo, a);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  dq_convert_kernel<<<sms * 8, 256, 0, st>>>(a.dqacc, a.dq, a.dq_rs, a.T, a.H,
-                                             0.5f * a.alpha * a.inv_n);
-  return cudaGetLastError();
+  bwd_kvq_kernel<<<grid, kThreads, SMEM, st>>>(m, gs);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  for (int p = 0; p < gs.G; ++p) {
+    const AttnArgs& a = gs.g[p];
+    if (a.T == 0) continue;
+    dq_convert_kernel<<<sms * 8, 256, 0, st>>>(a.dqacc, a.dq, a.dq_rs, a.T, a.H,
+                                               0.5f * a.alpha * a.inv_n);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+cudaError_t launch_bwd_fused(const AttnArgs& a, cudaStream_t st) {
+  if (a.T == 0) return cudaSuccess;
+  GroupSet gs;
+  memset(&gs, 0, sizeof(gs));
+  gs.g[0] = a;
+  gs.common = a.ws;
+  gs.G = 1;
+  return launch_bwd_fused_grouped(gs, st);
 }
 
 }  // namespace hstu

@@ -90,26 +90,39 @@ enum {
 static_assert(8 * BAR_COUNT <= 512, "barrier area");
 
 // Unit u of the schedule (units are taken from an atomic counter in order, so
-// a CTA that drew short units takes more of them): head u / n_items, query
-// tile items[u % n_items]; the key tiles it meets.  u >= total ends it.
-__device__ void decode_unit(const AttnArgs& a, int n_items, int total, int u, UnitRec* r) {
-  if (u >= total) {
-    r->nsteps = -1;
-    return;
+// a CTA that drew short units takes more of them).  The problems' units follow
+// one another; within problem p, unit u is head u / n_items, query tile
+// items[u % n_items]; the record gets the key tiles it meets.  Past the last
+// unit the record ends the schedule.
+__device__ void decode_unit(const GroupSet& gs, int u, UnitRec* r) {
+  for (int p = 0; p < kMaxGroups && p < gs.G; ++p) {
+    const AttnArgs& a = gs.g[p];
+    const int n_items = a.ws->n_items;
+    const int units = n_items * a.H;
+    if (u < units) {
+      const int h = u / n_items;
+      const int2 it = a.items[u - h * n_items];
+      const SeqGeom g = seq_geom(a, it.x);
+      const int t0 = it.y * kBM;
+      const int t1 = imin(t0 + kBM, g.L);
+      unit_rec_fill(r, h, g.s0, g.L, g.Lh, t0, t1,
+                    q_tile_key_tiles(t0, t1, g.Lh, a.K1, a.K2e, kBN));
+      r->grp = p;
+      return;
+    }
+    u -= units;
   }
-  const int h = u / n_items;
-  const int2 it = a.items[u - h * n_items];
-  const SeqGeom g = seq_geom(a, it.x);
-  const int t0 = it.y * kBM;
-  const int t1 = imin(t0 + kBM, g.L);
-  unit_rec_fill(r, h, g.s0, g.L, g.Lh, t0, t1, q_tile_key_tiles(t0, t1, g.Lh, a.K1, a.K2e, kBN));
+  r->nsteps = -1;
 }
+
+// q, k, v, out maps of every problem of a launch.
+struct FwdMaps {
+  CUtensorMap q[kMaxGroups], k[kMaxGroups], v[kMaxGroups], o[kMaxGroups];
+};
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
-    fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
-                  const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
-                  const AttnArgs a) {
+    fwd_tc_kernel(const __grid_constant__ FwdMaps maps, const __grid_constant__ GroupSet gs) {
   using C = Cfg<D>;
   constexpr int kKSt = C::kKSt, kVSt = C::kVSt;
   extern __shared__ uint8_t smem_raw[];
@@ -123,9 +136,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + C::OFF_SLOT);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (load_status(a.ws) != 0) return;  // device-side input check failed
-  const int n_items = a.ws->n_items;
-  const int total = n_items * a.H;
+  WsHeader* const ws = gs.common;  // status word and scheduler of the launch
+  // a problem's device-side input check failed: report it for the launch
+  for (int p = 0; p < kMaxGroups && p < gs.G; ++p) {
+    const int st = load_status(gs.g[p].ws);
+    if (st != 0) {
+      if (threadIdx.x == 0) set_status(ws, st);
+      return;
+    }
+  }
+  if (load_status(ws) != 0) return;
 
   if (threadIdx.x == 0) {
     for (int qb = 0; qb < 2; ++qb) {
@@ -152,10 +172,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(BAR_DRAIN), 1);
     for (int b = 0; b < C::NB; ++b) mbar_init(bar(BAR_OST + b), 4 * (C::BOXW / 32));
     fence_barrier_init();
-    prefetch_tmap(&tmq);
-    prefetch_tmap(&tmk);
-    prefetch_tmap(&tmv);
-    prefetch_tmap(&tmo);
+    for (int p = 0; p < kMaxGroups && p < gs.G; ++p) {
+      if (gs.g[p].T == 0) continue;  // no map was built
+      prefetch_tmap(&maps.q[p]);
+      prefetch_tmap(&maps.k[p]);
+      prefetch_tmap(&maps.v[p]);
+      prefetch_tmap(&maps.o[p]);
+    }
   }
   if (warp == 1) {
     tmem_alloc(smem_addr(tmem_slot), kTmemCols);
@@ -176,9 +199,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     auto publish = [&](int kk) -> bool {
       const int slot = kk % kUSlots;
-      if (!warp_wait(bar(BAR_U_EMPTY + slot), ((kk / kUSlots) & 1) ^ 1, a.ws)) return false;
+      if (!warp_wait(bar(BAR_U_EMPTY + slot), ((kk / kUSlots) & 1) ^ 1, ws)) return false;
       if (lane == 0) {
-        decode_unit(a, n_items, total, atomicAdd(&a.ws->sched, 1), &ring[slot]);
+        decode_unit(gs, atomicAdd(&ws->sched, 1), &ring[slot]);
         mbar_arrive(bar(BAR_U_FULL + slot));
       }
       __syncwarp();
@@ -194,15 +217,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         continue;
       }
       const int h = r->h, s0 = r->s0;
+      const CUtensorMap* tmq = &maps.q[r->grp];
+      const CUtensorMap* tmk = &maps.k[r->grp];
       // Q tiles alternate between two buffers, so the next unit's Q is loaded
       // while the current unit still runs.
       const uint32_t qb = qn & 1;
-      ok = warp_wait(bar(BAR_Q_EMPTY + qb), ((qn >> 1) & 1) ^ 1, a.ws);
+      ok = warp_wait(bar(BAR_Q_EMPTY + qb), ((qn >> 1) & 1) ^ 1, ws);
       if (!ok) break;
       if (lane == 0) {
         mbar_expect_tx(bar(BAR_Q_FULL + qb), C::TILE);
         for (int b = 0; b < C::NB; ++b)
-          tma_load_2d(sQ + qb * C::TILE + b * C::BLK, &tmq, bar(BAR_Q_FULL + qb),
+          tma_load_2d(sQ + qb * C::TILE + b * C::BLK, tmq, bar(BAR_Q_FULL + qb),
                       h * D + b * C::BOXW, s0 + r->t0);
       }
       ++qn;
@@ -213,13 +238,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = kn % kKSt;
         if (kn >= (uint32_t)kKSt) {
           const uint32_t prev = kn - kKSt;
-          ok = warp_wait(bar(BAR_S_FULL + prev % kSBufs), (prev / kSBufs) & 1, a.ws);
+          ok = warp_wait(bar(BAR_S_FULL + prev % kSBufs), (prev / kSBufs) & 1, ws);
           if (!ok) break;
         }
         if (lane == 0) {
           mbar_expect_tx(bar(BAR_K_FULL + s), C::TILE);
           for (int b = 0; b < C::NB; ++b)
-            tma_load_2d(sK + s * C::TILE + b * C::BLK, &tmk, bar(BAR_K_FULL + s),
+            tma_load_2d(sK + s * C::TILE + b * C::BLK, tmk, bar(BAR_K_FULL + s),
                         h * D + b * C::BOXW, s0 + c.j * kBN);
         }
         ++kn;
@@ -228,7 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // If any role gave up, every load issued must still land before the CTA
     // exits (each barrier has at most its last armed phase outstanding).
-    if (lane == 0 && load_status(a.ws) != 0) {
+    if (lane == 0 && load_status(ws) != 0) {
       for (uint32_t qb = 0; qb < 2; ++qb) {
         const uint32_t armed = qn / 2 + (qb < (qn & 1) ? 1u : 0u);
         if (armed > 0) drain_wait(bar(BAR_Q_FULL + qb), (armed - 1) & 1);
@@ -244,20 +269,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int kk = 0; ok; ++kk) {
       const int slot = kk % kUSlots;
-      ok = warp_wait(bar(BAR_U_FULL + slot), (kk / kUSlots) & 1, a.ws);
+      ok = warp_wait(bar(BAR_U_FULL + slot), (kk / kUSlots) & 1, ws);
       if (!ok) break;
       const UnitRec* r = &ring[slot];
       const int nt = r->nsteps, h = r->h, s0 = r->s0;
+      const CUtensorMap* tmv = &maps.v[nt > 0 ? r->grp : 0];
       SpanCursor c;
       c.begin(r);
       for (int n = 0; n < nt && ok; ++n, c.next(r)) {
         const int s = vn % kVSt;
-        ok = warp_wait(bar(BAR_V_EMPTY + s), ((vn / kVSt) & 1) ^ 1, a.ws);
+        ok = warp_wait(bar(BAR_V_EMPTY + s), ((vn / kVSt) & 1) ^ 1, ws);
         if (!ok) break;
         if (lane == 0) {
           mbar_expect_tx(bar(BAR_V_FULL + s), C::TILE);
           for (int b = 0; b < C::NB; ++b)
-            tma_load_2d(sV + s * C::TILE + b * C::BLK, &tmv, bar(BAR_V_FULL + s),
+            tma_load_2d(sV + s * C::TILE + b * C::BLK, tmv, bar(BAR_V_FULL + s),
                         h * D + b * C::BOXW, s0 + c.j * kBN);
         }
         ++vn;
@@ -265,7 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       warp_arrive(bar(BAR_U_EMPTY + slot));
       if (nt < 0) break;
     }
-    if (lane == 0 && load_status(a.ws) != 0) {
+    if (lane == 0 && load_status(ws) != 0) {
       for (int s = 0; s < kVSt; ++s) {
         const uint32_t armed = vn / kVSt + (s < (int)(vn % kVSt) ? 1u : 0u);
         if (armed > 0) drain_wait(bar(BAR_V_FULL + s), (armed - 1) & 1);
@@ -320,9 +346,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                ((pend & 1u) == 0 || mbar_test_wait(bar(BAR_O_EMPTY), (on & 1) ^ 1));
       };
       auto pv = [&]() -> bool {  // blocking form
-        if (!mbar_wait(bar(BAR_P_FULL + pvc % kSBufs), (pvc / kSBufs) & 1, a.ws)) return false;
-        if (!mbar_wait(bar(BAR_V_FULL + pvc % kVSt), (pvc / kVSt) & 1, a.ws)) return false;
-        if ((pend & 1u) && !mbar_wait(bar(BAR_O_EMPTY), (on & 1) ^ 1, a.ws)) return false;
+        if (!mbar_wait(bar(BAR_P_FULL + pvc % kSBufs), (pvc / kSBufs) & 1, ws)) return false;
+        if (!mbar_wait(bar(BAR_V_FULL + pvc % kVSt), (pvc / kVSt) & 1, ws)) return false;
+        if ((pend & 1u) && !mbar_wait(bar(BAR_O_EMPTY), (on & 1) ^ 1, ws)) return false;
         pv_issue();
         return true;
       };
@@ -344,9 +370,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             continue;
           }
           if ((it & 255u) == 0) {
-            if (load_status(a.ws) != 0) return false;
+            if (load_status(ws) != 0) return false;
             if (globaltimer() - t0 > kWaitLimitNs) {
-              set_status(a.ws, HSTU_SLA_ERR_TIMEOUT);
+              set_status(ws, HSTU_SLA_ERR_TIMEOUT);
               return false;
             }
           }
@@ -408,7 +434,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int half = chunk & 1;            // column half within the group
     const int row = quarter * 32 + lane;   // row of the 128-row tile
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-    const uint64_t half_alpha2 = f2s(0.5f * a.alpha);
     const bool has_o = chunk < D / 32;     // this warp writes an O chunk
     // Epilogue store: a tile that lies inside its sequence is staged as bf16
     // in the unit's Q buffer (no S MMA reads it any more) in the swizzled
@@ -427,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // tile of the unit after next, whose Q load depends on them.
     uint32_t tc = 0, on = 0, qn = 0;
     bool ep_pend = false;
-    int e_h = 0, e_s0 = 0, e_t0 = 0, e_t1 = 0, e_slot = 0;
+    int e_h = 0, e_s0 = 0, e_t0 = 0, e_t1 = 0, e_slot = 0, e_grp = 0;
     uint32_t e_qn = 0;
     int rel_qb = -1;  // box leaders: Q buffer whose O stores are issued, not yet released
     auto release = [&]() {
@@ -442,11 +467,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     auto epilogue = [&]() -> bool {
       ep_pend = false;
-      if (!warp_wait(bar(BAR_O_FULL), on & 1, a.ws)) return false;
+      if (!warp_wait(bar(BAR_O_FULL), on & 1, ws)) return false;
       tc_fence_after();
       const uint32_t qb = e_qn & 1;
       const bool whole = e_t1 - e_t0 == kBM;
       const int i = e_t0 + row;
+      const AttnArgs& E = gs.g[e_grp];
+      const float inv_n = E.inv_n;
       uint32_t o[16];
       if (has_o) {
         uint32_t r0[16], r1[16];
@@ -455,10 +482,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_wait2(r0, r1);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          o[e] = pack_bf16x2(__uint_as_float(r0[2 * e]) * a.inv_n,
-                             __uint_as_float(r0[2 * e + 1]) * a.inv_n);
-          o[8 + e] = pack_bf16x2(__uint_as_float(r1[2 * e]) * a.inv_n,
-                                 __uint_as_float(r1[2 * e + 1]) * a.inv_n);
+          o[e] = pack_bf16x2(__uint_as_float(r0[2 * e]) * inv_n,
+                             __uint_as_float(r0[2 * e + 1]) * inv_n);
+          o[8 + e] = pack_bf16x2(__uint_as_float(r1[2 * e]) * inv_n,
+                                 __uint_as_float(r1[2 * e + 1]) * inv_n);
         }
       }
       // O is in registers: the next unit's P V may overwrite it
@@ -475,7 +502,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                          o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
           fence_proxy_async_smem();  // staged rows visible to the TMA store
         } else if (i < e_t1) {
-          uint4* dst = reinterpret_cast<uint4*>(a.out + (int64_t)(e_s0 + i) * a.o_rs + e_h * D +
+          uint4* dst = reinterpret_cast<uint4*>(E.out + (int64_t)(e_s0 + i) * E.o_rs + e_h * D +
                                                 chunk * 32);
 #pragma unroll
           for (int v = 0; v < 4; ++v)
@@ -484,9 +511,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         warp_arrive(bar(BAR_OST + box));
         if (box_leader) {
           release();
-          good = mbar_wait(bar(BAR_OST + box), e_qn & 1, a.ws);
+          good = mbar_wait(bar(BAR_OST + box), e_qn & 1, ws);
           if (lane == 0 && good && whole) {
-            tma_store_2d(&tmo, sQ + qb * C::TILE + box * C::BLK, e_h * D + box * C::BOXW,
+            tma_store_2d(&maps.o[e_grp], sQ + qb * C::TILE + box * C::BLK, e_h * D + box * C::BOXW,
                          e_s0 + e_t0);
             bulk_commit_group();
           }
@@ -507,7 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int kk = 0; ok; ++kk) {
       const int slot = kk % kUSlots;
-      ok = warp_wait(bar(BAR_U_FULL + slot), (kk / kUSlots) & 1, a.ws);
+      ok = warp_wait(bar(BAR_U_FULL + slot), (kk / kUSlots) & 1, ws);
       if (!ok) break;
       const UnitRec* r = &ring[slot];
       const int nt = r->nsteps;
@@ -524,7 +551,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // no visible key anywhere in the tile
         const int i = r->t0 + row;
         if (has_o && i < r->t1) {
-          uint4* dst = reinterpret_cast<uint4*>(a.out + (int64_t)(r->s0 + i) * a.o_rs +
+          const AttnArgs& A = gs.g[r->grp];
+          uint4* dst = reinterpret_cast<uint4*>(A.out + (int64_t)(r->s0 + i) * A.o_rs +
                                                 r->h * D + chunk * 32);
           const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
@@ -535,17 +563,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const int h = r->h, s0 = r->s0, Lh = r->Lh, t0 = r->t0, t1 = r->t1;
       const int i = t0 + row;  // row within the sequence
-      const RowMask m = row_mask(i, r->L, Lh, a.K1, a.K2e);
+      const AttnArgs& A = gs.g[r->grp];
+      const int K1 = A.K1, K2e = A.K2e;
+      const uint64_t half_alpha2 = f2s(0.5f * A.alpha);
+      const RowMask m = row_mask(i, r->L, Lh, K1, K2e);
       SpanCursor c;
       c.begin(r);
       for (int n = 0; n < nt; ++n, ++tc, c.next(r)) {
         if ((int)(tc & 1) != grp) continue;  // the other group's tile
         const uint32_t b = tc % kSBufs;
-        ok = warp_wait(bar(BAR_S_FULL + b), (tc / kSBufs) & 1, a.ws);
+        ok = warp_wait(bar(BAR_S_FULL + b), (tc / kSBufs) & 1, ws);
         if (!ok) break;
         tc_fence_after();
         const int j0 = c.j * kBN;
-        const bool full = tile_full(t0, t0 + kBM, j0, j0 + kBN, Lh, a.K1, a.K2e);
+        const bool full = tile_full(t0, t0 + kBM, j0, j0 + kBN, Lh, K1, K2e);
         // P = SiLU(alpha S) = h + h tanh(h) with h = alpha S / 2.  Tiles that
         // are entirely visible skip the mask; the others clear invisible
         // entries with one bit test each against this row's 32-key bitmask.
@@ -587,7 +618,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       release();
       ep_pend = true;
-      e_h = h; e_s0 = s0; e_t0 = t0; e_t1 = t1; e_slot = slot; e_qn = qn;
+      e_h = h; e_s0 = s0; e_t0 = t0; e_t1 = t1; e_slot = slot; e_qn = qn; e_grp = r->grp;
       ++qn;
     }
     // stores still in flight must complete before the CTA exits
@@ -604,32 +635,49 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int D>
-cudaError_t launch_d(const AttnArgs& a, cudaStream_t st) {
+cudaError_t launch_d(const GroupSet& gs, cudaStream_t st) {
   using C = Cfg<D>;
-  CUtensorMap mq, mk, mv, mo;
-  const int HD = a.H * D;
-  if (!make_tma_2d(&mq, a.q, a.T, HD, a.q_rs, C::BOXW, kBM, C::SW == 128) ||
-      !make_tma_2d(&mk, a.k, a.T, HD, a.k_rs, C::BOXW, kBN, C::SW == 128) ||
-      !make_tma_2d(&mv, a.v, a.T, HD, a.v_rs, C::BOXW, kBN, C::SW == 128) ||
-      !make_tma_2d(&mo, a.out, a.T, HD, a.o_rs, C::BOXW, kBM, C::SW == 128))
-    return cudaErrorInvalidValue;
+  FwdMaps m;
+  memset(&m, 0, sizeof(m));
+  int64_t units = 0;
+  for (int p = 0; p < gs.G; ++p) {
+    const AttnArgs& a = gs.g[p];
+    if (a.T == 0) continue;  // no units; its maps stay unused
+    const int HD = a.H * D;
+    if (!make_tma_2d(&m.q[p], a.q, a.T, HD, a.q_rs, C::BOXW, kBM, C::SW == 128) ||
+        !make_tma_2d(&m.k[p], a.k, a.T, HD, a.k_rs, C::BOXW, kBN, C::SW == 128) ||
+        !make_tma_2d(&m.v[p], a.v, a.T, HD, a.v_rs, C::BOXW, kBN, C::SW == 128) ||
+        !make_tma_2d(&m.o[p], a.out, a.T, HD, a.o_rs, C::BOXW, kBM, C::SW == 128))
+      return cudaErrorInvalidValue;
+    units += max_items(a.T, a.B) * a.H;
+  }
+  if (units == 0) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  const int64_t units = max_items(a.T, a.B) * a.H;
   const int sms = device_sm_count();
   const int grid = (int)(units < sms ? units : sms);
-  fwd_tc_kernel<D><<<grid, kThreads, C::SMEM, st>>>(mq, mk, mv, mo, a);
+  fwd_tc_kernel<D><<<grid, kThreads, C::SMEM, st>>>(m, gs);
   return cudaGetLastError();
 }
 
 }  // namespace
 
+cudaError_t launch_fwd_grouped(const GroupSet& gs, int d, cudaStream_t st) {
+  if (gs.G < 1 || gs.G > kMaxGroups) return cudaErrorInvalidValue;
+  if (d == 32) return launch_d<32>(gs, st);
+  if (d == 64) return launch_d<64>(gs, st);
+  return launch_d<128>(gs, st);
+}
+
 cudaError_t launch_fwd_tc(const AttnArgs& a, int d, cudaStream_t st) {
   if (a.T == 0) return cudaSuccess;
-  if (d == 32) return launch_d<32>(a, st);
-  if (d == 64) return launch_d<64>(a, st);
-  return launch_d<128>(a, st);
+  GroupSet gs;
+  memset(&gs, 0, sizeof(gs));
+  gs.g[0] = a;
+  gs.common = a.ws;
+  gs.G = 1;
+  return launch_fwd_grouped(gs, d, st);
 }
 
 }  // namespace hstu

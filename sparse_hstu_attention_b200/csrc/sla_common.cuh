@@ -69,6 +69,8 @@ __host__ __device__ inline size_t ws_bwd_bytes(int64_t T, int B, int H, int d) {
 }
 
 // ------------------------------------------------------------ kernel args
+constexpr int kMaxGroups = 4;  // problems per grouped launch
+
 struct AttnArgs {
   const int32_t* offs;   // [B+1]
   const int32_t* nts;    // [B] or null
@@ -303,13 +305,15 @@ __host__ __device__ __forceinline__ uint32_t key_mask_bits(const KeyMask& m, int
 struct UnitRec {
   int h, s0, L, Lh, t0, t1, nsteps, nsp;
   int lo[3], hi[3];
-  int pad[2];
+  int grp;  // problem of the unit within its launch (0 unless grouped)
+  int pad;
 };
 static_assert(sizeof(UnitRec) == 64, "unit record size");
 
 __device__ __forceinline__ void unit_rec_fill(UnitRec* r, int h, int s0, int L, int Lh, int t0,
                                               int t1, const Spans& sp) {
   r->h = h; r->s0 = s0; r->L = L; r->Lh = Lh; r->t0 = t0; r->t1 = t1;
+  r->grp = 0;
   r->nsteps = sp.count();
   r->nsp = sp.n;
   for (int s = 0; s < 3; ++s) {
@@ -352,6 +356,17 @@ cudaError_t launch_worklist(const AttnArgs& a, int tile, int list, bool first, c
 cudaError_t launch_count_pairs(const AttnArgs& a, int BMf, int BNf, int BMb, int BNb,
                                int64_t* row_counts, int64_t* key_counts, cudaStream_t st);
 cudaError_t launch_fwd_tc(const AttnArgs& a, int d, cudaStream_t st);
+// Several problems (same head_dim) in one launch of the forward / one-pass
+// backward kernel: one schedule over every problem's units.  `common` holds
+// the launch's status word and scheduler counters; each problem's work lists
+// were built into its own workspace beforehand.
+struct GroupSet {
+  AttnArgs g[kMaxGroups];
+  WsHeader* common;
+  int G;
+};
+cudaError_t launch_fwd_grouped(const GroupSet& gs, int d, cudaStream_t st);
+cudaError_t launch_bwd_fused_grouped(const GroupSet& gs, cudaStream_t st);
 cudaError_t launch_bwd_tc(const AttnArgs& a, int d, bool kv_pass, cudaStream_t st);
 // head_dim kFusedBwdD: zeroes a.dqacc, runs the one-pass backward, converts dq
 cudaError_t launch_bwd_fused(const AttnArgs& a, cudaStream_t st);

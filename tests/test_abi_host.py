@@ -138,3 +138,32 @@ def test_binding_structs_match_the_headers(py, c, tmp_path):
     got = _c_layout(c, names, tmp_path)
     assert got[0] == ctypes.sizeof(py)
     assert got[1:] == [getattr(py, n).offset for n in names]
+
+
+def test_grouped_calls_reject_bad_groups_on_the_host(lib):
+    """Host-side checks of the grouped entry points (no CUDA call is reached)."""
+    import numpy as np
+    G = 2
+    arr = (_abi.FwdParams * G)(_params(), _params())
+    for p in arr:
+        p.out, p.out_row_stride = FAKE, 512
+    ws = 0x100000  # 256-byte aligned, never dereferenced
+    assert lib.hstu_sla_fwd_grouped(arr, 0, ws, 1 << 30, None) == _abi.ERR_INVALID_ARG
+    assert lib.hstu_sla_fwd_grouped(arr, _abi.MAX_GROUPS + 1, ws, 1 << 30, None) == \
+        _abi.ERR_INVALID_ARG
+    assert lib.hstu_sla_fwd_grouped(arr, G, ws, 255, None) == _abi.ERR_WORKSPACE
+    arr[1].d = 64
+    assert lib.hstu_sla_fwd_grouped(arr, G, ws, 1 << 30, None) == _abi.ERR_UNSUPPORTED
+    b = (_abi.BwdParams * 1)()
+    b[0].fwd = _params(d=64, q_row_stride=256, k_row_stride=256, v_row_stride=256)
+    b[0].dout = b[0].dq = b[0].dk = b[0].dv = FAKE
+    b[0].dout_row_stride = b[0].dq_row_stride = b[0].dk_row_stride = b[0].dv_row_stride = 256
+    assert lib.hstu_sla_bwd_grouped(b, 1, ws, 1 << 30, None) == _abi.ERR_UNSUPPORTED
+    # the grouped workspace: a 256-byte header, then each group's own workspace
+    T = np.array([1000, 500], np.int64)
+    B, H, d = np.array([3, 2], np.int32), np.array([4, 2], np.int32), np.array([128, 128], np.int32)
+    f = lib.hstu_sla_grouped_workspace_bytes
+    want = 256 + sum(lib.hstu_sla_workspace_bytes(_abi.WS_BWD, int(T[i]), int(B[i]), int(H[i]), 128)
+                     for i in range(2))
+    assert f(_abi.WS_BWD, 2, T.ctypes.data, B.ctypes.data, H.ctypes.data, d.ctypes.data) == want
+    assert f(_abi.WS_BWD, 0, T.ctypes.data, B.ctypes.data, H.ctypes.data, d.ctypes.data) == 0

@@ -72,6 +72,25 @@ WORKLOADS = {
 
 HIST16K_TOKEN_BUDGET = 96 * 1024
 
+# Mixture of Transducers: one transducer per user-signal channel, each with its
+# own sequences and SLA settings ("Bending the Scaling Law Curve...", section
+# 4.3 and appendix A; TorchEasyRec "ULTRA HSTU" docs, MoT: per-channel STU
+# stack and SLA / truncation configuration).  The pages give no channel mix;
+# this one pairs a long dense channel (16K-class histories, as hist16k), a
+# medium one and a short one with full causal attention.  The three
+# channels' attentions run as one grouped launch.
+MOT_CHANNELS = {
+    "mot_long": Workload(6, "mot_long", B=8, H=4, d=128, K1=1024, K2=128, contextual_len=32,
+                         num_targets=64, alpha=1.0 / math.sqrt(128), N=16384.0,
+                         description="8 seqs, L~U{8192..16384}"),
+    "mot_mid": Workload(7, "mot_mid", B=32, H=4, d=128, K1=256, K2=64, contextual_len=16,
+                        num_targets=16, alpha=1.0 / math.sqrt(128), N=4096.0,
+                        description="32 seqs, L~U{1024..4096}"),
+    "mot_short": Workload(8, "mot_short", B=128, H=4, d=128, K1=1024, K2=0, contextual_len=0,
+                          num_targets=8, alpha=1.0 / math.sqrt(128), N=1024.0,
+                          description="128 seqs, L~U{128..1024}, full causal"),
+}
+
 
 def draw_lengths(w: Workload) -> np.ndarray:
     """Total per-sequence lengths (contextual prefix and candidates included)."""
@@ -90,6 +109,12 @@ def draw_lengths(w: Workload) -> np.ndarray:
         return np.full(w.B, 8192 + 512, dtype=np.int64)
     if w.name == "stu":
         return rng.integers(4096, 16384, size=w.B, endpoint=True).astype(np.int64)
+    if w.name == "mot_long":
+        return rng.integers(8192, 16384, size=w.B, endpoint=True).astype(np.int64)
+    if w.name == "mot_mid":
+        return rng.integers(1024, 4096, size=w.B, endpoint=True).astype(np.int64)
+    if w.name == "mot_short":
+        return rng.integers(128, 1024, size=w.B, endpoint=True).astype(np.int64)
     raise KeyError(w.name)
 
 
