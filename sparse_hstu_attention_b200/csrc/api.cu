@@ -129,46 +129,7 @@ int hstu_sla_fwd(const hstu_sla_fwd_params* p, void* workspace, size_t workspace
 
 int hstu_sla_bwd(const hstu_sla_bwd_params* p, void* workspace, size_t workspace_bytes,
                  hstu_stream_t stream) {
-  if (p == nullptr) return HSTU_SLA_ERR_INVALID_ARG;
-  const hstu_sla_fwd_params* f = &p->fwd;
-  int e = check_common(f);
-  if (e) return e;
-  if ((e = check_tensor(p->dout, p->dout_row_stride, f))) return e;
-  if ((e = check_tensor(p->dq, p->dq_row_stride, f))) return e;
-  if ((e = check_tensor(p->dk, p->dk_row_stride, f))) return e;
-  if ((e = check_tensor(p->dv, p->dv_row_stride, f))) return e;
-  if ((e = check_ws(workspace, workspace_bytes,
-                    hstu_sla_workspace_bytes(HSTU_SLA_WS_BWD, f->total_tokens, f->B, f->H, f->d))))
-    return e;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  AttnArgs a = make_args(f, workspace);
-  a.cand_only = 0;  // the backward covers every row
-  a.dout = static_cast<const bf16*>(p->dout);
-  a.dq = static_cast<bf16*>(p->dq);
-  a.dk = static_cast<bf16*>(p->dk);
-  a.dv = static_cast<bf16*>(p->dv);
-  a.do_rs = p->dout_row_stride;
-  a.dq_rs = p->dq_row_stride;
-  a.dk_rs = p->dk_row_stride;
-  a.dv_rs = p->dv_row_stride;
-  cudaError_t ce;
-  if (f->d == kFusedBwdD) {
-    // one pass over key tiles; dQ through the fp32 workspace after the lists
-    a.dqacc = reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                       ws_bytes(f->total_tokens, f->B));
-    ce = launch_worklist(a, kKvBN, 1, true, st);
-    if (ce == cudaSuccess) ce = record(f->event_begin, st);
-    if (ce == cudaSuccess) ce = launch_bwd_fused(a, st);
-    if (ce == cudaSuccess) ce = record(f->event_end, st);
-  } else {
-    ce = launch_worklist(a, kQpBM, 0, true, st);
-    if (ce == cudaSuccess) ce = launch_worklist(a, kKvBN, 1, false, st);
-    if (ce == cudaSuccess) ce = record(f->event_begin, st);
-    if (ce == cudaSuccess) ce = launch_bwd_tc(a, f->d, /*kv_pass=*/true, st);
-    if (ce == cudaSuccess) ce = launch_bwd_tc(a, f->d, /*kv_pass=*/false, st);
-    if (ce == cudaSuccess) ce = record(f->event_end, st);
-  }
-  return cuda_status(ce);
+  return sla_bwd(p, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream), nullptr);
 }
 
 size_t hstu_sla_grouped_workspace_bytes(int which, int32_t G, const int64_t* total_tokens,
@@ -325,3 +286,65 @@ const char* hstu_sla_strerror(int code) {
 int hstu_sla_version(void) { return kAbiVersion; }
 
 }  // extern "C"
+
+namespace hstu {
+
+int sla_bwd(const hstu_sla_bwd_params* p, void* workspace, size_t workspace_bytes,
+            cudaStream_t st, const SiluFusion* fz) {
+  if (p == nullptr) return HSTU_SLA_ERR_INVALID_ARG;
+  const hstu_sla_fwd_params* f = &p->fwd;
+  int e = check_common(f);
+  if (e) return e;
+  if ((e = check_tensor(p->dout, p->dout_row_stride, f))) return e;
+  if ((e = check_tensor(p->dq, p->dq_row_stride, f))) return e;
+  if ((e = check_tensor(p->dk, p->dk_row_stride, f))) return e;
+  if ((e = check_tensor(p->dv, p->dv_row_stride, f))) return e;
+  if ((e = check_ws(workspace, workspace_bytes,
+                    hstu_sla_workspace_bytes(HSTU_SLA_WS_BWD, f->total_tokens, f->B, f->H, f->d))))
+    return e;
+  AttnArgs a = make_args(f, workspace);
+  a.cand_only = 0;  // the backward covers every row
+  a.dout = static_cast<const bf16*>(p->dout);
+  a.dq = static_cast<bf16*>(p->dq);
+  a.dk = static_cast<bf16*>(p->dk);
+  a.dv = static_cast<bf16*>(p->dv);
+  a.do_rs = p->dout_row_stride;
+  a.dq_rs = p->dq_row_stride;
+  a.dk_rs = p->dk_row_stride;
+  a.dv_rs = p->dv_row_stride;
+  cudaError_t ce;
+  if (fz != nullptr) {  // the STU layer's SiLU' and bias-gradient fusion
+    // silu_qkv_kernel: 3 H d / 8 threads, whole warps per block part
+    const int ch = f->H * (f->d / 8);
+    if (f->d != kFusedBwdD || ch % 32 != 0 || 3 * ch > 384) return HSTU_SLA_ERR_UNSUPPORTED;
+    a.pre_q = fz->pre_q;
+    a.pre_k = fz->pre_k;
+    a.pre_v = fz->pre_v;
+    a.pre_rs = fz->pre_rs;
+    a.db_q = fz->db_q;
+    a.db_k = fz->db_k;
+    a.db_v = fz->db_v;
+    a.db_part = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                         ws_bytes(f->total_tokens, f->B) +
+                                         dq_workspace_bytes(f->total_tokens, f->H, f->d));
+  }
+  if (f->d == kFusedBwdD) {
+    // one pass over key tiles; dQ through the fp32 workspace after the lists
+    a.dqacc = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                       ws_bytes(f->total_tokens, f->B));
+    ce = launch_worklist(a, kKvBN, 1, true, st);
+    if (ce == cudaSuccess) ce = record(f->event_begin, st);
+    if (ce == cudaSuccess) ce = launch_bwd_fused(a, st);
+    if (ce == cudaSuccess) ce = record(f->event_end, st);
+  } else {
+    ce = launch_worklist(a, kQpBM, 0, true, st);
+    if (ce == cudaSuccess) ce = launch_worklist(a, kKvBN, 1, false, st);
+    if (ce == cudaSuccess) ce = record(f->event_begin, st);
+    if (ce == cudaSuccess) ce = launch_bwd_tc(a, f->d, /*kv_pass=*/true, st);
+    if (ce == cudaSuccess) ce = launch_bwd_tc(a, f->d, /*kv_pass=*/false, st);
+    if (ce == cudaSuccess) ce = record(f->event_end, st);
+  }
+  return cuda_status(ce);
+}
+
+}  // namespace hstu

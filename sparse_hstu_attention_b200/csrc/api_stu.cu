@@ -268,6 +268,11 @@ int hstu_stu_layer_bwd(const hstu_stu_layer_bwd_params* p, void* workspace,
   l2.ldpu = 4 * dm;
   l2.dgamma = p->d_ln2_w;
   l2.dbeta = p->d_ln2_b;
+  // d = 128 with an even number of heads up to 8: the attention backward's
+  // last pass applies SiLU' to dQ, dK, dV and sums their bias gradients, the
+  // gated norm sums dU's; no separate pass over dpre
+  const bool fused = f->d == 128 && (f->H * 16) % 32 == 0 && 3 * f->H * 16 <= 384;
+  if (fused) l2.dbias_u = p->d_b1;
   if ((ce = launch_ln_bwd(l2, true, st)) != cudaSuccess) return status_of(ce);
   // attention backward: dQ, dK, dV into blocks 2, 3, 1 of dpre
   hstu_sla_bwd_params ab;
@@ -279,11 +284,18 @@ int hstu_stu_layer_bwd(const hstu_stu_layer_bwd_params* p, void* workspace,
   ab.dk = dpre + 3 * dm;
   ab.dv = dpre + dm;
   ab.dq_row_stride = ab.dk_row_stride = ab.dv_row_stride = 4 * dm;
-  if ((e = hstu_sla_bwd(&ab, aws, workspace_bytes - kHdr, stream))) return e;
-  // SiLU' on the V, Q, K blocks (U is done), d b1 = colsum(dpre)
-  if ((ce = launch_silu_bwd_colsum(dpre, 4 * dm, static_cast<const bf16*>(f->pre), 4 * dm, T,
-                                   4 * dm, dm, p->d_b1, st)) != cudaSuccess)
-    return status_of(ce);
+  const bf16* pre = static_cast<const bf16*>(f->pre);
+  if (fused) {
+    const SiluFusion fz = {pre + 2 * dm, pre + 3 * dm, pre + dm, 4 * dm,
+                           p->d_b1 + 2 * dm, p->d_b1 + 3 * dm, p->d_b1 + dm};
+    if ((e = sla_bwd(&ab, aws, workspace_bytes - kHdr, st, &fz))) return e;
+  } else {
+    if ((e = hstu_sla_bwd(&ab, aws, workspace_bytes - kHdr, stream))) return e;
+    // SiLU' on the V, Q, K blocks (U is done), d b1 = colsum(dpre)
+    if ((ce = launch_silu_bwd_colsum(dpre, 4 * dm, pre, 4 * dm, T, 4 * dm, dm, p->d_b1, st)) !=
+        cudaSuccess)
+      return status_of(ce);
+  }
   // d W1 = x^T dpre
   GemmArgs gw1 = gw;
   gw1.N = 4 * dm;

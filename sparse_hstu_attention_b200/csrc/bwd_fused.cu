@@ -544,6 +544,89 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// The STU layer's form of the step after the one-pass backward: the
+// pre-activation gradients of the Q, K, V blocks, in one pass over the rows,
+//   dq = bf16(scale * workspace * SiLU'(pre_q))
+//   dk = bf16(dk * SiLU'(pre_k)),  dv likewise      (in place)
+// and per block the column sums of the three (the bias gradient), stored
+// to db_part[block] for silu_db_reduce_kernel.  Thread j: block part j / ch
+// (0 Q, 1 K, 2 V; ch = H * D / 8 threads each, a multiple of 32, so parts are
+// warp-uniform), columns [8 (j % ch), +8); a block takes a contiguous range
+// of rows.
+__global__ void __launch_bounds__(384) silu_qkv_kernel(const AttnArgs a, float scale) {
+  const int HD = a.H * D, ch = HD / 8;
+  const int j = threadIdx.x;
+  const int part = j / ch;
+  const int cj = (j - part * ch) * 8;
+  const int h = cj / D, cd = cj - h * D;
+  const int64_t T = a.T;
+  const int64_t per = (T + gridDim.x - 1) / gridDim.x;
+  const int64_t r0 = blockIdx.x * per, r1 = r0 + per < T ? r0 + per : T;
+  const bf16* pre = (part == 0 ? a.pre_q : part == 1 ? a.pre_k : a.pre_v) + cj;
+  bf16* g = part == 0 ? a.dq : part == 1 ? a.dk : a.dv;
+  const int64_t g_rs = part == 0 ? a.dq_rs : part == 1 ? a.dk_rs : a.dv_rs;
+  float sum[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+  for (int64_t t = r0; t < r1; ++t) {
+    float x[8];
+    if (part == 0) {
+      const float4* src = reinterpret_cast<const float4*>(a.dqacc + ((int64_t)h * T + t) * D + cd);
+      const float4 x0 = __ldcs(src), x1 = __ldcs(src + 1);
+      x[0] = x0.x * scale; x[1] = x0.y * scale; x[2] = x0.z * scale; x[3] = x0.w * scale;
+      x[4] = x1.x * scale; x[5] = x1.y * scale; x[6] = x1.z * scale; x[7] = x1.w * scale;
+    } else {
+      const uint4 w = *reinterpret_cast<const uint4*>(g + t * g_rs + cj);
+      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        x[2 * e] = __uint_as_float(ww[e] << 16);
+        x[2 * e + 1] = __uint_as_float(ww[e] & 0xFFFF0000u);
+      }
+    }
+    const uint4 pw = __ldg(reinterpret_cast<const uint4*>(pre + t * a.pre_rs));
+    const uint32_t pp[4] = {pw.x, pw.y, pw.z, pw.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      x[2 * e] *= silu_grad(__uint_as_float(pp[e] << 16));
+      x[2 * e + 1] *= silu_grad(__uint_as_float(pp[e] & 0xFFFF0000u));
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) sum[e] += x[e];
+    uint4 o;
+    o.x = pack_bf16x2(x[0], x[1]);
+    o.y = pack_bf16x2(x[2], x[3]);
+    o.z = pack_bf16x2(x[4], x[5]);
+    o.w = pack_bf16x2(x[6], x[7]);
+    *reinterpret_cast<uint4*>(g + t * g_rs + cj) = o;
+  }
+  float4* dst = reinterpret_cast<float4*>(a.db_part + ((int64_t)blockIdx.x * 3 + part) * HD + cj);
+  dst[0] = make_float4(sum[0], sum[1], sum[2], sum[3]);
+  dst[1] = make_float4(sum[4], sum[5], sum[6], sum[7]);
+}
+
+// db_{q,k,v}[c] += the blocks' partial sums.  A block owns 32 consecutive
+// columns of the 3 * H * D; its warp w adds the partials of blocks w, w + 8,
+// ... (lane = column, so each read is 128 contiguous bytes), then the eight
+// warps' totals are added.
+__global__ void __launch_bounds__(256) silu_db_reduce_kernel(const AttnArgs a, int nblk) {
+  __shared__ float s_part[8][32];
+  const int HD = a.H * D;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int col = blockIdx.x * 32 + lane;  // in [0, 3 HD)
+  const int part = col / HD, c = col - part * HD;
+  float v = 0.f;
+#pragma unroll 4
+  for (int b = w; b < nblk; b += 8) v += a.db_part[((int64_t)b * 3 + part) * HD + c];
+  s_part[w][lane] = v;
+  __syncthreads();
+  if (w == 0) {
+    float t = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) t += s_part[k][lane];
+    atomicAdd((part == 0 ? a.db_q : part == 1 ? a.db_k : a.db_v) + c, t);
+  }
+}
+
 // dq[t, h, :] = bf16(scale * workspace[h, t, :]), eight head-dim values per
 // thread and step.
 __global__ void __launch_bounds__(256) dq_convert_kernel(const float* __restrict__ acc,
@@ -599,8 +682,15 @@ cudaError_t launch_bwd_fused_grouped(const GroupSet& gs, cudaStream_t st) {
   for (int p = 0; p < gs.G; ++p) {
     const AttnArgs& a = gs.g[p];
     if (a.T == 0) continue;
-    dq_convert_kernel<<<sms * 8, 256, 0, st>>>(a.dqacc, a.dq, a.dq_rs, a.T, a.H,
-                                               0.5f * a.alpha * a.inv_n);
+    if (a.pre_q != nullptr) {  // STU layer: SiLU' of Q, K, V and the bias gradient
+      const int HD = a.H * D;
+      silu_qkv_kernel<<<kSiluBlocks, 3 * HD / 8, 0, st>>>(a, 0.5f * a.alpha * a.inv_n);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+      silu_db_reduce_kernel<<<3 * HD / 32, 256, 0, st>>>(a, kSiluBlocks);
+    } else {
+      dq_convert_kernel<<<sms * 8, 256, 0, st>>>(a.dqacc, a.dq, a.dq_rs, a.T, a.H,
+                                                 0.5f * a.alpha * a.inv_n);
+    }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   return cudaSuccess;

@@ -64,8 +64,15 @@ constexpr int kFusedBwdD = 128;
 __host__ __device__ inline size_t dq_workspace_bytes(int64_t T, int H, int d) {
   return d == kFusedBwdD ? size_t(T) * size_t(H) * size_t(d) * sizeof(float) : 0;
 }
+// The STU layer's SiLU' pass after the one-pass backward (silu_qkv_kernel)
+// runs kSiluBlocks blocks; each leaves its column sums of the Q, K, V blocks
+// (the bias gradient's partial sums) after the dQ accumulator.
+constexpr int kSiluBlocks = 1024;
+__host__ __device__ inline size_t db_parts_bytes(int H, int d) {
+  return d == kFusedBwdD ? size_t(kSiluBlocks) * 3 * size_t(H) * size_t(d) * sizeof(float) : 0;
+}
 __host__ __device__ inline size_t ws_bwd_bytes(int64_t T, int B, int H, int d) {
-  return ws_bytes(T, B) + dq_workspace_bytes(T, H, d);
+  return ws_bytes(T, B) + dq_workspace_bytes(T, H, d) + db_parts_bytes(H, d);
 }
 
 // ------------------------------------------------------------ kernel args
@@ -91,6 +98,19 @@ struct AttnArgs {
   bf16* dk;
   bf16* dv;
   int64_t q_rs, k_rs, v_rs, do_rs, o_rs, dq_rs, dk_rs, dv_rs;
+  // Optional (one-pass backward, set by the STU layer): q, k, v are SiLU
+  // outputs of the pre-activations pre_q / pre_k / pre_v (row stride pre_rs);
+  // the backward then leaves the pre-activation gradients dq * SiLU'(pre_q),
+  // ... in dq, dk, dv and adds their column sums (the bias gradient) into
+  // db_q / db_k / db_v ([H * d] each).  Null pre_q: plain dq, dk, dv.
+  const bf16* pre_q;
+  const bf16* pre_k;
+  const bf16* pre_v;
+  int64_t pre_rs;
+  float* db_q;
+  float* db_k;
+  float* db_v;
+  float* db_part;  // [kSiluBlocks][3 (q, k, v)][H * d] partial sums (workspace)
 };
 
 __host__ __device__ inline int cdiv(int a, int b) { return (a + b - 1) / b; }
@@ -366,6 +386,20 @@ struct GroupSet {
   int G;
 };
 cudaError_t launch_fwd_grouped(const GroupSet& gs, int d, cudaStream_t st);
+// The backward entry point with the STU layer's SiLU' / bias-gradient fusion
+// (AttnArgs::pre_q ...); fz = nullptr is hstu_sla_bwd.  Fusion needs
+// d = kFusedBwdD and H * d / 8 dividing 256.
+struct SiluFusion {
+  const bf16* pre_q;
+  const bf16* pre_k;
+  const bf16* pre_v;
+  int64_t pre_rs;
+  float* db_q;
+  float* db_k;
+  float* db_v;
+};
+int sla_bwd(const hstu_sla_bwd_params* p, void* workspace, size_t workspace_bytes,
+            cudaStream_t st, const SiluFusion* fz);
 cudaError_t launch_bwd_fused_grouped(const GroupSet& gs, cudaStream_t st);
 cudaError_t launch_bwd_tc(const AttnArgs& a, int d, bool kv_pass, cudaStream_t st);
 // head_dim kFusedBwdD: zeroes a.dqacc, runs the one-pass backward, converts dq

@@ -74,6 +74,7 @@ struct LnArgs {
   int64_t ldpu;
   float* dgamma;       // [W], accumulated into
   float* dbeta;        // [W], accumulated into
+  float* dbias_u;      // gated norm, optional: column sums of du accumulated into [W]
 };
 cudaError_t launch_ln_fwd(const LnArgs& a, bool gated, cudaStream_t st);
 // E4M3 copy of a weight W [K][N] (x W convention) transposed to [N][K] (row

@@ -43,10 +43,7 @@ __device__ __forceinline__ void store8(bf16* p, const float* f) {
       make_uint4(pack2(f[0], f[1]), pack2(f[2], f[3]), pack2(f[4], f[5]), pack2(f[6], f[7]));
 }
 
-__device__ __forceinline__ float silu_grad(float v) {
-  const float s = 1.0f / (1.0f + __expf(-v));
-  return s * (1.0f + v * (1.0f - s));
-}
+using sm100::silu_grad;
 
 // LayerNorm (biased variance) of each row, then the affine map; GATED also
 // multiplies by the gate row u.  Saves the row mean and 1/sqrt(var + eps).
@@ -157,25 +154,45 @@ __global__ void __launch_bounds__(256) quant_wt_kernel(const bf16* W, int64_t ld
 // Gated: dz = dy * u, du = dy * z (times SiLU'(pre_u), since the gate is a
 // SiLU output), dx = LN'(dz * gamma).  Two passes over each row (the second
 // re-reads x, dy, u from L1 instead of keeping them in registers, so many
-// warps fit per SM); dgamma / dbeta accumulate in shared memory over the
-// rows a block visits (per warp, each lane updating only its own columns, for
-// W <= 512; shared atomics beyond), then once per block and column in global
-// memory.
+// warps fit per SM); dgamma / dbeta (and, gated, the column sums of du: the
+// gate's bias gradient) accumulate in shared memory over the rows a block
+// visits (per warp, each lane updating only its own columns, for W <= 512;
+// shared atomics beyond), then once per block and column in global memory.
 template <int NV, bool GATED>
-__global__ void __launch_bounds__(32 * kRowWarps, 2) ln_bwd_kernel(const LnArgs a) {
+__global__ void __launch_bounds__(32 * kRowWarps, GATED ? 2 : 4) ln_bwd_kernel(const LnArgs a) {
   constexpr int W = NV * 256;
   constexpr bool kPerWarp = NV <= 2;
   constexpr int kAcc = kPerWarp ? kRowWarps : 1;
-  __shared__ __align__(16) float s_g[W], s_b[W], s_dg[kAcc][W], s_db[kAcc][W];
+  // shared memory: gamma, beta, then the dgamma, dbeta (and, gated, du)
+  // accumulators, kAcc rows of W each; dynamic for the gated form (past the
+  // 48 KB of static shared memory at W = 512)
+  float* ln_smem;
+  if constexpr (GATED) {
+    extern __shared__ __align__(16) float ln_dyn[];
+    ln_smem = ln_dyn;
+  } else {
+    __shared__ __align__(16) float ln_static[(2 + 2 * kAcc) * W];
+    ln_smem = ln_static;
+  }
+  float* s_g = ln_smem;
+  float* s_b = s_g + W;
+  float* s_dg = s_b + W;
+  float* s_db = s_dg + kAcc * W;
+  float* s_du = s_db + kAcc * W;
   for (int c = threadIdx.x; c < W; c += blockDim.x) {
     s_g[c] = a.gamma[c];
     s_b[c] = a.beta[c];
-    for (int w = 0; w < kAcc; ++w) s_dg[w][c] = s_db[w][c] = 0.f;
+    for (int w = 0; w < kAcc; ++w) {
+      s_dg[w * W + c] = s_db[w * W + c] = 0.f;
+      if (GATED) s_du[w * W + c] = 0.f;
+    }
   }
   __syncthreads();
   const int lane = threadIdx.x & 31;
-  float* my_dg = s_dg[kPerWarp ? (threadIdx.x >> 5) : 0];
-  float* my_db = s_db[kPerWarp ? (threadIdx.x >> 5) : 0];
+  const int acc_row = kPerWarp ? (threadIdx.x >> 5) : 0;
+  float* my_dg = s_dg + acc_row * W;
+  float* my_db = s_db + acc_row * W;
+  float* my_du = s_du + acc_row * W;
   const int64_t nwarps = (int64_t)gridDim.x * kRowWarps;
   for (int64_t row = (int64_t)blockIdx.x * kRowWarps + (threadIdx.x >> 5); row < a.T;
        row += nwarps) {
@@ -223,7 +240,24 @@ __global__ void __launch_bounds__(32 * kRowWarps, 2) ln_bwd_kernel(const LnArgs 
           atomicAdd(my_db + c + e, tb[e]);
         }
       }
-      if (GATED) store8(a.du + row * a.lddu + c, du);
+      if (GATED) {
+        store8(a.du + row * a.lddu + c, du);
+        if (a.dbias_u) {
+          if (kPerWarp) {
+            float4* pu4 = reinterpret_cast<float4*>(my_du + c);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              float4 u4 = pu4[h];
+              u4.x += du[4 * h]; u4.y += du[4 * h + 1]; u4.z += du[4 * h + 2];
+              u4.w += du[4 * h + 3];
+              pu4[h] = u4;
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) atomicAdd(my_du + c + e, du[e]);
+          }
+        }
+      }
     }
     const float m1 = warp_sum(s1) * (1.0f / W), m2 = warp_sum(s2) * (1.0f / W);
 #pragma unroll 1
@@ -247,12 +281,15 @@ __global__ void __launch_bounds__(32 * kRowWarps, 2) ln_bwd_kernel(const LnArgs 
   __syncthreads();
   for (int c = threadIdx.x; c < W; c += blockDim.x) {
     float g = 0.f, b = 0.f;
+    float u = 0.f;
     for (int w = 0; w < kAcc; ++w) {
-      g += s_dg[w][c];
-      b += s_db[w][c];
+      g += s_dg[w * W + c];
+      b += s_db[w * W + c];
+      if (GATED) u += s_du[w * W + c];
     }
     atomicAdd(a.dgamma + c, g);
     atomicAdd(a.dbeta + c, b);
+    if (GATED && a.dbias_u) atomicAdd(a.dbias_u + c, u);
   }
 }
 
@@ -381,16 +418,41 @@ cudaError_t launch_quant_wt(const bf16* W, int64_t ldw, int K, int N, uint8_t* W
   return cudaGetLastError();
 }
 
+template <int NV, bool GATED>
+cudaError_t launch_ln_bwd_t(const LnArgs& a, cudaStream_t st) {
+  constexpr int W = NV * 256;
+  constexpr int kAcc = NV <= 2 ? kRowWarps : 1;
+  // dynamic shared memory for the gated form only; its carveout keeps the
+  // rest of the SM's 256 KB as L1, which the second pass over a row reads
+  constexpr int bytes = GATED ? (2 + 3 * kAcc) * W * (int)sizeof(float) : 0;
+  if (GATED) {
+    cudaError_t e = cudaFuncSetAttribute(ln_bwd_kernel<NV, GATED>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(ln_bwd_kernel<NV, GATED>,
+                               cudaFuncAttributePreferredSharedMemoryCarveout,
+                               (2 * (bytes + 1024) * 100 + 228 * 1024 - 1) / (228 * 1024));
+    if (e != cudaSuccess) return e;
+  }
+  // whole waves: as many blocks as fit on every SM at once (rows are strided
+  // over the grid), fewer for short batches
+  int per_sm = 0;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+      &per_sm, ln_bwd_kernel<NV, GATED>, 32 * kRowWarps, bytes);
+  if (e != cudaSuccess) return e;
+  const int64_t need = (a.T + kRowWarps - 1) / kRowWarps;
+  const int64_t cap = (int64_t)device_sm_count() * (per_sm > 0 ? per_sm : 1);
+  const int grid = (int)(need < cap ? need : cap);
+  ln_bwd_kernel<NV, GATED><<<grid, 32 * kRowWarps, bytes, st>>>(a);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_ln_bwd(const LnArgs& a, bool gated, cudaStream_t st) {
   if (a.T == 0) return cudaSuccess;
-  const int64_t need = (a.T + kRowWarps - 1) / kRowWarps;
-  const int cap = device_sm_count() * 4;  // rows per warp grow past this
-  const int grid = (int)(need < cap ? need : cap);
 #define HSTU_LNB(NV)                                                                    \
   if (a.W == NV * 256) {                                                                \
-    if (gated) ln_bwd_kernel<NV, true><<<grid, 32 * kRowWarps, 0, st>>>(a);             \
-    else ln_bwd_kernel<NV, false><<<grid, 32 * kRowWarps, 0, st>>>(a);                  \
-    return cudaGetLastError();                                                          \
+    if (gated) return launch_ln_bwd_t<NV, true>(a, st);                                 \
+    return launch_ln_bwd_t<NV, false>(a, st);                                           \
   }
   HSTU_LNB(1) HSTU_LNB(2) HSTU_LNB(4)
 #undef HSTU_LNB

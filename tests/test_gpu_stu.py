@@ -177,6 +177,31 @@ def test_stu_layer_matches_oracle():
         assert_close("d_" + name, getattr(g, name), getattr(rg, name))
 
 
+def test_stu_layer_head_dim_64_matches_oracle():
+    """d = 64 heads (8 x 64): the attention's two-pass backward and the
+    separate SiLU' / bias-gradient pass (d = 128 fuses them into the
+    attention backward)."""
+    lengths, nts = np.array([260, 400, 90]), np.array([12, 7, 3])
+    H, d = 8, 64
+    cfg = stu.StuConfig(H, d, 8, 128, 32, 1.0 / math.sqrt(d), float(lengths.max()))
+    offs = offsets_from_lengths(lengths)
+    T = int(offs[-1])
+    dr = draw_stu(T, T, cfg.d_model, 1, seed=64, perturb=True)
+    w = stu.StuWeights.from_host(dr.layers[0], DEV)
+    offs_d = torch.tensor(offs, dtype=torch.int32, device=DEV)
+    nts_d = torch.tensor(nts, dtype=torch.int32, device=DEV)
+    out, st = stu.layer_fwd(dr.x.to(DEV), offs_d, nts_d, w, cfg, int(lengths.max()))
+    dx, g = stu.layer_bwd(dr.dout.to(DEV), st, w, cfg)
+    torch.cuda.synchronize()
+    wo = _oracle_weights(dr.layers[0])
+    ref, cache = S.layer_fwd(f64(dr.x), wo, offs, nts, _oracle_cfg(cfg))
+    rdx, rg = S.layer_bwd(f64(dr.dout), wo, cache)
+    assert_close("out", out, ref)
+    assert_close("dx", dx, rdx)
+    for name in FIELDS:
+        assert_close("d_" + name, getattr(g, name), getattr(rg, name))
+
+
 def test_stu_layer_fp8_forward_matches_oracle():
     """The layer with E4M3 projections against the oracle's FP8 layer (the
     same quantization rules), forward and the unchanged backward; and it does
