@@ -50,68 +50,110 @@ using sm100::silu_grad;
 // With yq set, also writes the row in E4M3 with a per-row scale: the FP8
 // quantization fused into the norm that precedes each projection ("Bending
 // the Scaling Law Curve...", section 4.2.2, mixed-precision training and
-// inference; Figure 4).
+// inference; Figure 4).  A warp takes kLnRows rows; every load (x, the gate,
+// gamma, beta) is issued before the first reduction, so their latencies
+// overlap instead of following one another.
+constexpr int kLnRows = 1;
+
 template <int NV, bool GATED>
 __global__ void __launch_bounds__(32 * kRowWarps) ln_fwd_kernel(const LnArgs a) {
-  const int64_t row = (int64_t)blockIdx.x * kRowWarps + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= a.T) return;
   constexpr int W = NV * 256;
-  float x[NV][8];
+  const int lane = threadIdx.x & 31;
+  const int64_t row0 = ((int64_t)blockIdx.x * kRowWarps + (threadIdx.x >> 5)) * kLnRows;
+  if (row0 >= a.T) return;
+  float x[kLnRows][NV][8], u[GATED ? kLnRows : 1][NV][8];
 #pragma unroll
-  for (int v = 0; v < NV; ++v) load8(a.x + row * a.ldx + 8 * (lane + 32 * v), x[v]);
-  float s = 0.f;
+  for (int r = 0; r < kLnRows; ++r) {
+    const int64_t row = row0 + r < a.T ? row0 + r : row0;  // a missing second row repeats the first
 #pragma unroll
-  for (int v = 0; v < NV; ++v)
-#pragma unroll
-    for (int e = 0; e < 8; ++e) s += x[v][e];
-  const float mean = warp_sum(s) * (1.0f / W);
-  float q = 0.f;
-#pragma unroll
-  for (int v = 0; v < NV; ++v)
-#pragma unroll
-    for (int e = 0; e < 8; ++e) q += (x[v][e] - mean) * (x[v][e] - mean);
-  const float rstd = rsqrtf(warp_sum(q) * (1.0f / W) + a.eps);
-  float amax = 0.f;
-#pragma unroll
-  for (int v = 0; v < NV; ++v) {
-    const int c = 8 * (lane + 32 * v);
-    float u[8];
-    if (GATED) load8(a.u + row * a.ldu + c, u);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      x[v][e] = (x[v][e] - mean) * rstd * a.gamma[c + e] + a.beta[c + e];  // x now holds y
-      if (GATED) x[v][e] *= u[e];
-    }
-    store8(a.y + row * a.ldy + c, x[v]);
-    if (a.yq) {  // quantize what the bf16 output holds
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        x[v][e] = __bfloat162float(__float2bfloat16(x[v][e]));
-        amax = fmaxf(amax, fabsf(x[v][e]));
-      }
+    for (int v = 0; v < NV; ++v) {
+      load8(a.x + row * a.ldx + 8 * (lane + 32 * v), x[r][v]);
+      if (GATED) load8(a.u + row * a.ldu + 8 * (lane + 32 * v), u[GATED ? r : 0][v]);
     }
   }
-  if (a.yq) {
+  float gm[NV][8], bt[NV][8];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    const float scale = amax > 0.f ? amax * (1.0f / 448.0f) : 1.0f;
-    const float inv = 1.0f / scale;
+  for (int v = 0; v < NV; ++v) {
+    const float4* g4 = reinterpret_cast<const float4*>(a.gamma + 8 * (lane + 32 * v));
+    const float4* b4 = reinterpret_cast<const float4*>(a.beta + 8 * (lane + 32 * v));
+    const float4 ga = __ldg(g4), gb = __ldg(g4 + 1), ba = __ldg(b4), bb = __ldg(b4 + 1);
+    gm[v][0] = ga.x; gm[v][1] = ga.y; gm[v][2] = ga.z; gm[v][3] = ga.w;
+    gm[v][4] = gb.x; gm[v][5] = gb.y; gm[v][6] = gb.z; gm[v][7] = gb.w;
+    bt[v][0] = ba.x; bt[v][1] = ba.y; bt[v][2] = ba.z; bt[v][3] = ba.w;
+    bt[v][4] = bb.x; bt[v][5] = bb.y; bt[v][6] = bb.z; bt[v][7] = bb.w;
+  }
+  float mean[kLnRows], rstd[kLnRows];
+#pragma unroll
+  for (int r = 0; r < kLnRows; ++r) {
+    float s = 0.f;
+#pragma unroll
+    for (int v = 0; v < NV; ++v)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s += x[r][v][e];
+    mean[r] = s;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+    for (int r = 0; r < kLnRows; ++r) mean[r] += __shfl_xor_sync(0xffffffffu, mean[r], o);
+#pragma unroll
+  for (int r = 0; r < kLnRows; ++r) {
+    mean[r] *= 1.0f / W;
+    float q = 0.f;
+#pragma unroll
+    for (int v = 0; v < NV; ++v)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) q += (x[r][v][e] - mean[r]) * (x[r][v][e] - mean[r]);
+    rstd[r] = q;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+    for (int r = 0; r < kLnRows; ++r) rstd[r] += __shfl_xor_sync(0xffffffffu, rstd[r], o);
+#pragma unroll
+  for (int r = 0; r < kLnRows; ++r) {
+    const int64_t row = row0 + r;
+    if (row >= a.T) break;
+    rstd[r] = rsqrtf(rstd[r] * (1.0f / W) + a.eps);
+    float amax = 0.f;
 #pragma unroll
     for (int v = 0; v < NV; ++v) {
       const int c = 8 * (lane + 32 * v);
-      uint2 w;
-      w.x = sm100::pack_e4m3x2(x[v][0] * inv, x[v][1] * inv) |
-            (sm100::pack_e4m3x2(x[v][2] * inv, x[v][3] * inv) << 16);
-      w.y = sm100::pack_e4m3x2(x[v][4] * inv, x[v][5] * inv) |
-            (sm100::pack_e4m3x2(x[v][6] * inv, x[v][7] * inv) << 16);
-      *reinterpret_cast<uint2*>(a.yq + row * a.ldyq + c) = w;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        x[r][v][e] = (x[r][v][e] - mean[r]) * rstd[r] * gm[v][e] + bt[v][e];  // x now holds y
+        if (GATED) x[r][v][e] *= u[GATED ? r : 0][v][e];
+      }
+      store8(a.y + row * a.ldy + c, x[r][v]);
+      if (a.yq) {  // quantize what the bf16 output holds
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          x[r][v][e] = __bfloat162float(__float2bfloat16(x[r][v][e]));
+          amax = fmaxf(amax, fabsf(x[r][v][e]));
+        }
+      }
     }
-    if (lane == 0) a.yscale[row] = scale;
-  }
-  if (lane == 0) {
-    a.mean[row] = mean;
-    a.rstd[row] = rstd;
+    if (a.yq) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      const float scale = amax > 0.f ? amax * (1.0f / 448.0f) : 1.0f;
+      const float inv = 1.0f / scale;
+#pragma unroll
+      for (int v = 0; v < NV; ++v) {
+        const int c = 8 * (lane + 32 * v);
+        uint2 w;
+        w.x = sm100::pack_e4m3x2(x[r][v][0] * inv, x[r][v][1] * inv) |
+              (sm100::pack_e4m3x2(x[r][v][2] * inv, x[r][v][3] * inv) << 16);
+        w.y = sm100::pack_e4m3x2(x[r][v][4] * inv, x[r][v][5] * inv) |
+              (sm100::pack_e4m3x2(x[r][v][6] * inv, x[r][v][7] * inv) << 16);
+        *reinterpret_cast<uint2*>(a.yq + row * a.ldyq + c) = w;
+      }
+      if (lane == 0) a.yscale[row] = scale;
+    }
+    if (lane == 0) {
+      a.mean[row] = mean[r];
+      a.rstd[row] = rstd[r];
+    }
   }
 }
 
@@ -398,7 +440,7 @@ __global__ void __launch_bounds__(256) trunc_rows_kernel(const bf16* src, int64_
 
 cudaError_t launch_ln_fwd(const LnArgs& a, bool gated, cudaStream_t st) {
   if (a.T == 0) return cudaSuccess;
-  const int grid = (int)((a.T + kRowWarps - 1) / kRowWarps);
+  const int grid = (int)((a.T + kRowWarps * kLnRows - 1) / (kRowWarps * kLnRows));
 #define HSTU_LN(NV)                                                                     \
   if (a.W == NV * 256) {                                                                \
     if (gated) ln_fwd_kernel<NV, true><<<grid, 32 * kRowWarps, 0, st>>>(a);             \
