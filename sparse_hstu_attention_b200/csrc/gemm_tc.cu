@@ -49,15 +49,21 @@ constexpr int kThreads = 32 * (2 + 8);
 constexpr int A_TILE = kBM * kBK * 2;  // 16 KB
 constexpr int B_TILE = kBN * kBK * 2;  // 32 KB
 constexpr int MN_BOX = 64 * kBK * 2;   // one 64 (M or N) x 64 (K) box of an MN-major tile
-// bf16 outputs leave through shared memory and TMA: each epilogue warp stages
-// a 32-row x 64-column box (128-byte rows, 128B-swizzled) of each output
-constexpr int STG_BOX = 32 * 128;
-constexpr int STG_WARP = 2 * STG_BOX;  // out, out2
-// Shared-memory plan per epilogue: bf16 outputs take 3 ring stages and the
-// staging boxes, the fp32 reductions 4 stages and no staging.
-template <int EPI>
+// bf16 outputs leave through shared memory and TMA: each epilogue warp
+// stages 32-row x 32-column boxes (64-byte rows, 64B-swizzled) of each
+// output; with two buffers the store of one chunk reads shared memory while
+// the next chunk is computed.
+constexpr int STG_BOX = 32 * 64;
+constexpr int STG_BUF = 2 * STG_BOX;  // out, out2
+// Shared-memory plan: the fp32 reductions take 4 ring stages and no staging;
+// bf16 operands with bf16 outputs 4 stages (the main loop is the longer side)
+// and one staging buffer; 8-bit operands (half the ring stages per tile) 3
+// stages and two staging buffers (the epilogue is the longer side).
+template <int EPI, bool F8>
 struct GLayout {
-  static constexpr int kStages = EPI == kEpiRedF32 ? 4 : 3;
+  static constexpr int kStages = EPI == kEpiRedF32 ? 4 : (F8 ? 3 : 4);
+  static constexpr int kStgBufs = F8 ? 2 : 1;
+  static constexpr int STG_WARP = kStgBufs * STG_BUF;
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + kStages * A_TILE;
   static constexpr int OFF_STG = OFF_B + kStages * B_TILE;
@@ -116,7 +122,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const GemmArgs g) {
   static_assert(!F8 || (!A_MN && !B_MN), "8-bit operands are read K-major");
   constexpr int kBKe = F8 ? 2 * kBK : kBK;  // elements per 128-byte k block
-  using Lay = GLayout<EPI>;
+  using Lay = GLayout<EPI, F8>;
+  constexpr int kStgBufs = Lay::kStgBufs, STG_WARP = Lay::STG_WARP;
   constexpr int kStages = Lay::kStages, OFF_A = Lay::OFF_A, OFF_B = Lay::OFF_B;
   constexpr int OFF_STG = Lay::OFF_STG, OFF_BAR = Lay::OFF_BAR, OFF_SLOT = Lay::OFF_SLOT;
   extern __shared__ uint8_t smem_raw[];
@@ -241,9 +248,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int col0 = ((warp - 2) >> 2) * (kBN / 2);  // this warp's half of the columns
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     const uint32_t stg = base + OFF_STG + (uint32_t)(warp - 2) * STG_WARP;
-    const uint32_t stg_row = (uint32_t)lane * 128;
-    const uint32_t swz = (uint32_t)(lane & 7);
-    bool stores_pending = false;
+    const uint32_t stg_row = (uint32_t)lane * 64;          // 64-byte staged rows
+    const uint32_t swz = (uint32_t)((lane >> 1) & 3);     // 64B swizzle of row `lane`
+    uint32_t ec = 0;  // chunks this warp has staged
     uint32_t tc = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
@@ -255,102 +262,120 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const int m = ti.m0 + quarter * 32 + lane;
       const bool live = m < g.M;
+      if constexpr (EPI == kEpiRedF32) {
 #pragma unroll 1
-      for (int c = col0; c < col0 + kBN / 2; c += 32) {
-        uint32_t v[32];
-        tmem_ld32(lane_base + buf * kBN + c, v);
-        tmem_ld_wait(v);
-        if (c + 32 == col0 + kBN / 2) {  // this warp's share read out
-          tc_fence_before();
-          warp_arrive(bar(G_ACC_EMPTY + buf));
-        }
-        const int n = ti.n0 + c;
-        if constexpr (EPI == kEpiRedF32) {
+        for (int c = col0; c < col0 + kBN / 2; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(lane_base + buf * kBN + c, v);
+          tmem_ld_wait(v);
+          if (c + 32 == col0 + kBN / 2) {  // this warp's share read out
+            tc_fence_before();
+            warp_arrive(bar(G_ACC_EMPTY + buf));
+          }
           if (live) {
-            float* dst = g.outf + (int64_t)m * g.ldf + n;
+            float* dst = g.outf + (int64_t)m * g.ldf + ti.n0 + c;
 #pragma unroll
             for (int e = 0; e < 32; e += 4)
               red_add_v4(dst + e, __uint_as_float(v[e]), __uint_as_float(v[e + 1]),
                          __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
           }
-        } else {
-        float f[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(v[e]);
-        if constexpr (F8) {  // row scale of A times column scale of B
-          const float sm = live ? g.sa[m] : 0.f;
-          const float4* sp = reinterpret_cast<const float4*>(g.sb + n);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float4 s4 = __ldg(sp + e);
-            f[4 * e] *= sm * s4.x;
-            f[4 * e + 1] *= sm * s4.y;
-            f[4 * e + 2] *= sm * s4.z;
-            f[4 * e + 3] *= sm * s4.w;
-          }
         }
-        if (EPI == kEpiBiasSilu || EPI == kEpiBiasResid) {
-          const float4* bp = reinterpret_cast<const float4*>(g.bias + n);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float4 b4 = __ldg(bp + e);
-            f[4 * e] += b4.x;
-            f[4 * e + 1] += b4.y;
-            f[4 * e + 2] += b4.z;
-            f[4 * e + 3] += b4.w;
+      } else {
+        // 32-column chunks; the next chunk's TMEM load is in flight while this
+        // one is converted and staged
+        uint32_t va[32], vb[32];
+        tmem_ld32(lane_base + buf * kBN + col0, va);
+        tmem_ld_wait(va);
+        auto chunk = [&](int i, uint32_t(&v)[32], uint32_t(&vn)[32]) {
+          constexpr int kChunks = kBN / 2 / 32;
+          if (i + 1 < kChunks) {
+            tmem_ld32(lane_base + buf * kBN + col0 + 32 * (i + 1), vn);
+          } else {  // this warp's share of the accumulator is in registers
+            tc_fence_before();
+            warp_arrive(bar(G_ACC_EMPTY + buf));
           }
-        }
-        if (EPI == kEpiBiasResid && live) {
-          const uint4* rp = reinterpret_cast<const uint4*>(g.resid + (int64_t)m * g.ldr + n);
+          const int n = ti.n0 + col0 + 32 * i;
+          float f[32];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint4 r4 = rp[q];
-            const uint32_t w[4] = {r4.x, r4.y, r4.z, r4.w};
+          for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(v[e]);
+          if constexpr (F8) {  // row scale of A times column scale of B
+            const float sm = live ? g.sa[m] : 0.f;
+            const float4* sp = reinterpret_cast<const float4*>(g.sb + n);
 #pragma unroll
-            for (int h = 0; h < 4; ++h) {
-              f[8 * q + 2 * h] += __uint_as_float(w[h] << 16);
-              f[8 * q + 2 * h + 1] += __uint_as_float(w[h] & 0xFFFF0000u);
+            for (int e = 0; e < 8; ++e) {
+              const float4 s4 = __ldg(sp + e);
+              f[4 * e] *= sm * s4.x;
+              f[4 * e + 1] *= sm * s4.y;
+              f[4 * e + 2] *= sm * s4.z;
+              f[4 * e + 3] *= sm * s4.w;
             }
           }
-        }
-        // a 64-column box: its first 32 columns go to 16-byte chunks 0..3 of
-        // this lane's staged row, the next 32 to chunks 4..7
-        const int half = (c >> 5) & 1;
-        if (half == 0 && stores_pending) {  // the box staged before must be read out
-          if (lane == 0) bulk_wait_read_all();
-          __syncwarp();
-          stores_pending = false;
-        }
-        uint32_t o[16];
-        if (EPI == kEpiBiasSilu) {
+          if (EPI == kEpiBiasSilu || EPI == kEpiBiasResid) {
+            const float4* bp = reinterpret_cast<const float4*>(g.bias + n);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float4 b4 = __ldg(bp + e);
+              f[4 * e] += b4.x;
+              f[4 * e + 1] += b4.y;
+              f[4 * e + 2] += b4.z;
+              f[4 * e + 3] += b4.w;
+            }
+          }
+          if (EPI == kEpiBiasResid && live) {
+            const uint4* rp = reinterpret_cast<const uint4*>(g.resid + (int64_t)m * g.ldr + n);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint4 r4 = rp[q];
+              const uint32_t w[4] = {r4.x, r4.y, r4.z, r4.w};
+#pragma unroll
+              for (int h = 0; h < 4; ++h) {
+                f[8 * q + 2 * h] += __uint_as_float(w[h] << 16);
+                f[8 * q + 2 * h + 1] += __uint_as_float(w[h] & 0xFFFF0000u);
+              }
+            }
+          }
+          uint32_t o[16], o2[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) o[e] = pack_bf16x2(f[2 * e], f[2 * e + 1]);
+          if (EPI == kEpiBiasSilu) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            st_shared_v4(stg + STG_BOX + stg_row + ((((uint32_t)(half * 4 + q)) ^ swz) << 4),
-                         o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+            for (int e = 0; e < 16; ++e) {
+              o2[e] = o[e];  // pre-activation
+              o[e] = pack_bf16x2(silu_f(f[2 * e]), silu_f(f[2 * e + 1]));
+            }
+          }
+          // the buffer's previous store (two chunks back) must have read it
+          const uint32_t sb = stg + (uint32_t)(ec % kStgBufs) * STG_BUF;
+          if (ec >= (uint32_t)kStgBufs) {
+            if (lane == 0) {
+              if (kStgBufs == 2) bulk_wait_read_1();
+              else bulk_wait_read_all();
+            }
+            __syncwarp();
+          }
 #pragma unroll
-          for (int e = 0; e < 16; ++e) o[e] = pack_bf16x2(silu_f(f[2 * e]), silu_f(f[2 * e + 1]));
-        } else {
-#pragma unroll
-          for (int e = 0; e < 16; ++e) o[e] = pack_bf16x2(f[2 * e], f[2 * e + 1]);
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          st_shared_v4(stg + stg_row + ((((uint32_t)(half * 4 + q)) ^ swz) << 4), o[4 * q],
-                       o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
-        if (half == 1) {  // box complete: one TMA store per output (rows past M are clipped)
+          for (int q = 0; q < 4; ++q) {
+            const uint32_t off = stg_row + ((((uint32_t)q) ^ swz) << 4);
+            st_shared_v4(sb + off, o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+            if (EPI == kEpiBiasSilu)
+              st_shared_v4(sb + STG_BOX + off, o2[4 * q], o2[4 * q + 1], o2[4 * q + 2],
+                           o2[4 * q + 3]);
+          }
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) {
-            const int x = n - 32, y = ti.m0 + quarter * 32;
-            tma_store_2d(&tmo, stg, x, y);
-            if (EPI == kEpiBiasSilu) tma_store_2d(&tmo2, stg + STG_BOX, x, y);
+          if (lane == 0) {  // rows past M are clipped by the store
+            const int y = ti.m0 + quarter * 32;
+            tma_store_2d(&tmo, sb, n, y);
+            if (EPI == kEpiBiasSilu) tma_store_2d(&tmo2, sb + STG_BOX, n, y);
             bulk_commit_group();
           }
-          stores_pending = true;
-        }
-        }  // bf16 outputs
+          ++ec;
+          if (i + 1 < kChunks) tmem_ld_wait(vn);
+        };
+        chunk(0, va, vb);
+        chunk(1, vb, va);
+        chunk(2, va, vb);
+        chunk(3, vb, va);
       }
       ++tc;
     }
@@ -372,11 +397,11 @@ cudaError_t launch_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtenso
                      const CUtensorMap& mo2, const GemmArgs& g, int ntiles, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<A_MN, B_MN, EPI, F8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       GLayout<EPI>::SMEM);
+                                       GLayout<EPI, F8>::SMEM);
   if (e != cudaSuccess) return e;
   const int sms = device_sm_count();
   gemm_tc_kernel<A_MN, B_MN, EPI, F8>
-      <<<ntiles < sms ? ntiles : sms, kThreads, GLayout<EPI>::SMEM, st>>>(ma, mb, mo, mo2, g);
+      <<<ntiles < sms ? ntiles : sms, kThreads, GLayout<EPI, F8>::SMEM, st>>>(ma, mb, mo, mo2, g);
   return cudaGetLastError();
 }
 
@@ -413,9 +438,9 @@ cudaError_t launch_gemm(const GemmOperand& A, const GemmOperand& B, GemmArgs g, 
   CUtensorMap mo, mo2;
   memset(&mo, 0, sizeof(mo));
   memset(&mo2, 0, sizeof(mo2));
-  if (epi != kEpiRedF32 && !make_tma_2d(&mo, g.out, g.M, g.N, g.ldo, 64, 32, true))
+  if (epi != kEpiRedF32 && !make_tma_2d(&mo, g.out, g.M, g.N, g.ldo, 32, 32, false))
     return cudaErrorInvalidValue;
-  if (epi == kEpiBiasSilu && !make_tma_2d(&mo2, g.out2, g.M, g.N, g.ldo2, 64, 32, true))
+  if (epi == kEpiBiasSilu && !make_tma_2d(&mo2, g.out2, g.M, g.N, g.ldo2, 32, 32, false))
     return cudaErrorInvalidValue;
   const int ntiles = ((g.M + kBM - 1) / kBM) * (g.N / kBN) * g.splits;
   if (f8) {  // the forward projections in E4M3
