@@ -284,14 +284,17 @@ def test_stu_stack_matches_oracle(fp8):
                          tol=tol)
 
 
-def test_stu_stack_full_size_sampled():
+@pytest.mark.parametrize("fp8", [False, True])
+def test_stu_stack_full_size_sampled(fp8):
     """The 6-layer STU stack workload at full size (16 sequences of
     U{4096..16384} tokens, truncation to 32 + 1024 + 64 after layer 3), forward
-    and backward on the GPU.  Sequences are independent, so the oracle runs the
-    whole stack, forward and backward, on the shortest sequence alone (same
-    attention settings) and its output rows and dx rows must match; every
-    output and gradient must be finite.  The weight gradients sum over all
-    sequences and are compared at the smaller sizes above."""
+    and backward on the GPU, with bf16 or E4M3 forward projections.  Sequences
+    are independent, so the oracle runs the whole stack, forward and backward,
+    on the shortest sequence alone (same attention settings; per-row and
+    per-column quantization make that exact for FP8 too) and its output rows
+    and dx rows must match; every output and gradient must be finite.  The
+    weight gradients sum over all sequences and are compared at the smaller
+    sizes above."""
     from workloads import STU_TAIL, WORKLOADS, draw_lengths
     w = WORKLOADS["stu"]
     lengths = draw_lengths(w)
@@ -304,7 +307,7 @@ def test_stu_stack_full_size_sampled():
     T, T_out = int(offs[-1]), int(tl.sum())
     dr = draw_stu(T, T_out, full.d_model, STU_LAYERS, seed=w.seed)
     ws = [stu.StuWeights.from_host(lw, DEV) for lw in dr.layers]
-    stack = stu.StuStack(ws, full, cut, STU_TRUNC_AFTER, tail)
+    stack = stu.StuStack(ws, full, cut, STU_TRUNC_AFTER, tail, fp8=fp8)
     offs_d = torch.tensor(offs, dtype=torch.int32, device=DEV)
     nts_d = torch.tensor(nts, dtype=torch.int32, device=DEV)
     out, ctx = stack.forward(dr.x.to(DEV), offs_d, nts_d, lengths, nts)
@@ -312,13 +315,14 @@ def test_stu_stack_full_size_sampled():
     torch.cuda.synchronize()
     for t in [out, dx] + [getattr(g, f) for g in gs for f in FIELDS]:
         assert torch.isfinite(t.float()).all()
+    tol = TOL_FP8 if fp8 else 2e-2
     wo = [_oracle_weights(lw) for lw in dr.layers]
     new = offsets_from_lengths(tl)
     b = int(np.argmin(lengths))
     s0, s1, n0, n1 = int(offs[b]), int(offs[b + 1]), int(new[b]), int(new[b + 1])
     one = np.array([0, s1 - s0])
     ref, cache = S.stack_fwd(f64(dr.x[s0:s1]), wo, one, nts[b:b + 1], _oracle_cfg(full),
-                             _oracle_cfg(cut), STU_TRUNC_AFTER, tail)
-    assert_close("out rows of the shortest sequence", out[n0:n1], ref)
+                             _oracle_cfg(cut), STU_TRUNC_AFTER, tail, fp8=fp8)
+    assert_close("out rows of the shortest sequence", out[n0:n1], ref, tol=tol)
     rdx, _ = S.stack_bwd(f64(dr.dout[n0:n1]), wo, cache)
-    assert_close("dx rows of the shortest sequence", dx[s0:s1], rdx)
+    assert_close("dx rows of the shortest sequence", dx[s0:s1], rdx, tol=tol)
