@@ -49,7 +49,9 @@ class _Cfg(ctypes.Structure):
                 ("offsets", ctypes.c_void_p), ("num_targets", ctypes.c_void_p),
                 ("contextual_len", ctypes.c_int64), ("K1", ctypes.c_int64),
                 ("K2", ctypes.c_int64), ("alpha", ctypes.c_double), ("N", ctypes.c_double),
-                ("flags", ctypes.c_int)]
+                ("flags", ctypes.c_int), ("ts", ctypes.c_void_p),
+                ("rab_pos", ctypes.c_void_p), ("n_pos", ctypes.c_int64),
+                ("rab_time", ctypes.c_void_p), ("n_time", ctypes.c_int64)]
 
 
 def _load():
@@ -65,8 +67,11 @@ def _load():
             lib.oracle_sla_fwd_rows.argtypes = [vp, vp, vp, vp, vp, i64, vp]
             lib.oracle_sla_bwd_dq_rows.argtypes = [vp, vp, vp, vp, vp, vp, i64, vp]
             lib.oracle_sla_bwd_dkv_keys.argtypes = [vp, vp, vp, vp, vp, vp, i64, vp, vp]
+            lib.oracle_sla_bwd_drab.argtypes = [vp, vp, vp, vp, vp, vp, vp]
+            lib.oracle_rab_bucket.argtypes = [i64, i64]
+            lib.oracle_rab_bucket.restype = i64
             for f in ("oracle_sla_row_counts", "oracle_sla_key_counts", "oracle_sla_fwd_rows",
-                      "oracle_sla_bwd_dq_rows", "oracle_sla_bwd_dkv_keys"):
+                      "oracle_sla_bwd_dq_rows", "oracle_sla_bwd_dkv_keys", "oracle_sla_bwd_drab"):
                 getattr(lib, f).restype = None
             _lib = lib
     return _lib
@@ -86,13 +91,24 @@ class Problem:
     """One jagged SLA attention problem: offsets, targets, window sizes, scales."""
 
     def __init__(self, seq_offsets, num_targets, H, d, contextual_len, K1, K2,
-                 alpha, N, flags=0):
+                 alpha, N, flags=0, timestamps=None, rab_pos=None, rab_time=None):
+        """rab_pos [H][n_pos], rab_time [H][n_time] and timestamps [T]: the
+        optional relative attention bias (rab_time needs timestamps)."""
         self.offsets = np.ascontiguousarray(np.asarray(seq_offsets, dtype=np.int64))
         B = len(self.offsets) - 1
         nt = np.zeros(B, np.int64) if num_targets is None else num_targets
         self.num_targets = np.ascontiguousarray(np.asarray(nt, dtype=np.int64))
+        keep = lambda a, dt: None if a is None else np.ascontiguousarray(np.asarray(a, dtype=dt))
+        self.ts = keep(timestamps, np.int64)
+        self.rab_pos = keep(rab_pos, np.float64)
+        self.rab_time = keep(rab_time, np.float64)
+        ptr = lambda a: None if a is None else a.ctypes.data
         self._cfg = _Cfg(B, H, d, self.offsets.ctypes.data, self.num_targets.ctypes.data,
-                         contextual_len, K1, K2, float(alpha), float(N), flags)
+                         contextual_len, K1, K2, float(alpha), float(N), flags,
+                         ptr(self.ts), ptr(self.rab_pos),
+                         0 if self.rab_pos is None else self.rab_pos.shape[1],
+                         ptr(self.rab_time),
+                         0 if self.rab_time is None else self.rab_time.shape[1])
         self.B, self.H, self.d = B, H, d
         self.T = int(self.offsets[-1])
 
@@ -151,6 +167,22 @@ class Problem:
         dq = self.bwd_dq(q, k, v, dout)
         dk, dv = self.bwd_dkv(q, k, v, dout)
         return dq, dk, dv
+
+    def bwd_rab(self, q, k, v, dout):
+        """Gradients of the bias tables (None for an absent table)."""
+        q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+        dp = None if self.rab_pos is None else np.zeros_like(self.rab_pos)
+        dt = None if self.rab_time is None else np.zeros_like(self.rab_time)
+        _load().oracle_sla_bwd_drab(ctypes.byref(self._cfg), q.ctypes.data, k.ctypes.data,
+                                    v.ctypes.data, dout.ctypes.data,
+                                    None if dp is None else dp.ctypes.data,
+                                    None if dt is None else dt.ctypes.data)
+        return dp, dt
+
+
+def rab_bucket(n: int, nb: int) -> int:
+    """The oracle's bucket of a non-negative distance n (tables of nb rows)."""
+    return int(_load().oracle_rab_bucket(int(n), int(nb)))
 
 
 def visible(L, nt, contextual_len, K1, K2, i, j, flags=0) -> int:

@@ -39,8 +39,25 @@
  * alpha/N;  dQ_i = sum_j dS_ij k_j;  dK_j = sum_i dS_ij q_i   (the chain rule
  * on the forward above; Listing 1's attention_backward(dattn, q, k, v)).
  *
+ * Relative attention bias (optional; HSTU notes "Actions Speak Louder than
+ * Words", section 2.4, Eq. 2: phi2(Q K^T + rab^{p,t}) with a positional and a
+ * temporal part; the relative time encoding as the talk notes
+ * "基于昇腾 NPU 的生成式推荐 Scaling Law 落地实践" describe its usual
+ * implementation, Fuxi section: difference of the two timestamps, bucketed,
+ * looked up, added into the attention scores).  With it
+ *   x_ij = alpha q_i.k_j + rab_pos[h][bucket(dpos)] + rab_time[h][bucket(dt)]
+ * and everything above uses that x.  Readings (the pages fix none of them):
+ *   - dpos = i - j for history rows; a candidate row measures from Lh, the
+ *     position its window is applied at (Lh - j), and 0 to itself;
+ *   - dt = |ts_i - ts_j| (integer timestamps);
+ *   - bucket(n) = floor(log2(n + 1)), capped at the table size - 1;
+ *   - one table row per head; a NULL table adds nothing.
+ * Its gradient: d rab_*[h][b] = sum over visible pairs in bucket b of
+ * dP_ij SiLU'(x_ij) / N (oracle_sla_bwd_drab).
+ *
  * Layout: q, k, v, dout and all outputs are [T, H, d] row-major doubles;
- * seq_offsets is [B+1] with seq_offsets[0] = 0; num_targets is [B] or NULL.
+ * seq_offsets is [B+1] with seq_offsets[0] = 0; num_targets is [B] or NULL;
+ * timestamps [T]; rab tables [H][buckets].
  */
 #include <math.h>
 #include <stdint.h>
@@ -99,9 +116,52 @@ typedef struct {
   int64_t contextual_len, K1, K2;
   double alpha, N;
   int flags;
+  const int64_t* ts;      /* [T] timestamps, or NULL */
+  const double* rab_pos;  /* [H][n_pos], or NULL */
+  int64_t n_pos;
+  const double* rab_time; /* [H][n_time], or NULL */
+  int64_t n_time;
 } oracle_cfg;
 
 static int64_t nt_of(const oracle_cfg* c, int b) { return c->num_targets ? c->num_targets[b] : 0; }
+
+/* floor(log2(n + 1)) for n >= 0, at most nb - 1: the number of times n + 1
+ * can be halved before it reaches 1. */
+int64_t oracle_rab_bucket(int64_t n, int64_t nb) {
+  if (n < 0) n = 0;
+  uint64_t x = (uint64_t)n + 1;
+  int64_t b = 0;
+  while (x > 1) {
+    x >>= 1;
+    ++b;
+  }
+  return b < nb - 1 ? b : nb - 1;
+}
+
+/* Position and time buckets of the pair (i, j) of the sequence starting at
+ * token s0 (history length Lh). */
+static void rab_buckets(const oracle_cfg* c, int64_t s0, int64_t Lh, int64_t i, int64_t j,
+                        int64_t* bp, int64_t* bt) {
+  int64_t dpos = i < Lh ? i - j : (j == i ? 0 : Lh - j);
+  *bp = oracle_rab_bucket(dpos, c->n_pos);
+  int64_t dt = 0;
+  if (c->ts) {
+    dt = c->ts[s0 + i] - c->ts[s0 + j];
+    if (dt < 0) dt = -dt;
+  }
+  *bt = oracle_rab_bucket(dt, c->n_time);
+}
+
+/* The bias rab(i, j) of head h (0 without tables). */
+static double rab_of(const oracle_cfg* c, int64_t s0, int64_t Lh, int h, int64_t i, int64_t j) {
+  if (!c->rab_pos && !c->rab_time) return 0.0;
+  int64_t bp, bt;
+  rab_buckets(c, s0, Lh, i, j, &bp, &bt);
+  double r = 0.0;
+  if (c->rab_pos) r += c->rab_pos[h * c->n_pos + bp];
+  if (c->rab_time) r += c->rab_time[h * c->n_time + bt];
+  return r;
+}
 
 /* Number of visible keys of every token (the same for every head): [T]. */
 void oracle_sla_row_counts(const oracle_cfg* c, int64_t* counts) {
@@ -148,7 +208,8 @@ void oracle_sla_fwd_rows(const oracle_cfg* c, const double* q, const double* k,
           continue;
         const double* kj = k + ((s0 + j) * H + h) * d;
         const double* vj = v + ((s0 + j) * H + h) * d;
-        double p = silu(c->alpha * dot(qi, kj, d)) / c->N;
+        double x = c->alpha * dot(qi, kj, d) + rab_of(c, s0, L - nt_of(c, b), h, i, j);
+        double p = silu(x) / c->N;
         for (int e = 0; e < d; ++e) o[e] += p * vj[e];
       }
     }
@@ -175,7 +236,7 @@ void oracle_sla_bwd_dq_rows(const oracle_cfg* c, const double* q, const double* 
           continue;
         const double* kj = k + ((s0 + j) * H + h) * d;
         const double* vj = v + ((s0 + j) * H + h) * d;
-        double x = c->alpha * dot(qi, kj, d);
+        double x = c->alpha * dot(qi, kj, d) + rab_of(c, s0, L - nt_of(c, b), h, i, j);
         double ds = dot(doi, vj, d) * dsilu(x) * c->alpha / c->N;
         for (int e = 0; e < d; ++e) g[e] += ds * kj[e];
       }
@@ -206,10 +267,43 @@ void oracle_sla_bwd_dkv_keys(const oracle_cfg* c, const double* q, const double*
           continue;
         const double* qi = q + ((s0 + i) * H + h) * d;
         const double* doi = dout + ((s0 + i) * H + h) * d;
-        double x = c->alpha * dot(qi, kj, d);
+        double x = c->alpha * dot(qi, kj, d) + rab_of(c, s0, L - nt_of(c, b), h, i, j);
         double p = silu(x) / c->N;
         double ds = dot(doi, vj, d) * dsilu(x) * c->alpha / c->N;
         for (int e = 0; e < d; ++e) { gv[e] += p * doi[e]; gk[e] += ds * qi[e]; }
+      }
+    }
+  }
+}
+
+/* Gradients of the bias tables (either may be NULL):
+ *   d_pos[h][b]  = sum over visible (i, j) with position bucket b of
+ *                  dP_ij SiLU'(x_ij) / N,   d_time likewise. */
+void oracle_sla_bwd_drab(const oracle_cfg* c, const double* q, const double* k, const double* v,
+                         const double* dout, double* d_pos, double* d_time) {
+  const int H = c->H, d = c->d;
+  if (d_pos) memset(d_pos, 0, sizeof(double) * H * c->n_pos);
+  if (d_time) memset(d_time, 0, sizeof(double) * H * c->n_time);
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int h = 0; h < H; ++h) {  /* each head owns its table rows */
+    for (int b = 0; b < c->B; ++b) {
+      int64_t s0 = c->offsets[b], L = c->offsets[b + 1] - s0, Lh = L - nt_of(c, b);
+      for (int64_t i = 0; i < L; ++i) {
+        const double* qi = q + ((s0 + i) * H + h) * d;
+        const double* doi = dout + ((s0 + i) * H + h) * d;
+        for (int64_t j = 0; j < L; ++j) {
+          if (!oracle_sla_visible(L, nt_of(c, b), c->contextual_len, c->K1, c->K2, i, j,
+                                  c->flags))
+            continue;
+          const double* kj = k + ((s0 + j) * H + h) * d;
+          const double* vj = v + ((s0 + j) * H + h) * d;
+          double x = c->alpha * dot(qi, kj, d) + rab_of(c, s0, Lh, h, i, j);
+          double g = dot(doi, vj, d) * dsilu(x) / c->N;
+          int64_t bp, bt;
+          rab_buckets(c, s0, Lh, i, j, &bp, &bt);
+          if (d_pos) d_pos[h * c->n_pos + bp] += g;
+          if (d_time) d_time[h * c->n_time + bt] += g;
+        }
       }
     }
   }
