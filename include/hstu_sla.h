@@ -96,6 +96,19 @@ typedef struct {
    * and are written too (with their correct values).  Ignored by the
    * backward. */
   int32_t candidates_only;
+  /* Relative attention bias (optional; HSTU notes "Actions Speak Louder than
+   * Words", section 2.4, Eq. 2, phi2(Q K^T + rab^{p,t})):
+   *   x_ij = alpha q_i.k_j + rab_pos[h][bucket(dpos)] + rab_time[h][bucket(dt)]
+   * with bucket(n) = min(floor(log2(n + 1)), buckets - 1), dpos = i - j for
+   * a history row, Lh - j for a candidate row (0 to itself), and
+   * dt = |timestamps[i] - timestamps[j]|.  A NULL table adds nothing;
+   * rab_time needs timestamps.  Each table has 1..32 buckets per head.  Not
+   * available with the grouped calls; the backward needs d = 128. */
+  const int32_t* timestamps;    /* device [T], any integer time unit, or NULL */
+  const float* rab_pos;         /* device [H][rab_pos_buckets], or NULL */
+  const float* rab_time;        /* device [H][rab_time_buckets], or NULL */
+  int32_t rab_pos_buckets;
+  int32_t rab_time_buckets;
 } hstu_sla_fwd_params;
 
 /* Backward problem: the forward problem plus dout and the three gradients. */
@@ -109,6 +122,11 @@ typedef struct {
   int64_t dq_row_stride;
   int64_t dk_row_stride;
   int64_t dv_row_stride;
+  /* With fwd.rab_pos / fwd.rab_time set: their gradients (device [H][buckets],
+   * overwritten): d rab[h][b] = sum over visible pairs in bucket b of
+   * dP_ij SiLU'(x_ij) / N.  Required for every table that is set. */
+  float* d_rab_pos;
+  float* d_rab_time;
 } hstu_sla_bwd_params;
 
 #define HSTU_SLA_WS_FWD 0

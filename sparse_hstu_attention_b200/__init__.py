@@ -65,6 +65,22 @@ def hstu_sla_workspace_bytes(which: int, total_tokens: int, B: int, H: int, d: i
     return int(_abi.load().hstu_sla_workspace_bytes(which, total_tokens, B, H, d))
 
 
+def _set_rab(p, H, timestamps, rab_pos, rab_time):
+    """Relative attention bias fields: timestamps CUDA int32 [T]; rab_pos /
+    rab_time CUDA float32 [H, buckets] (1..32 buckets), either may be None."""
+    for name, t in (("rab_pos", rab_pos), ("rab_time", rab_time)):
+        if t is not None and (t.dtype != torch.float32 or not t.is_cuda or t.dim() != 2 or
+                              t.shape[0] != H or not t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous CUDA float32 [{H}, buckets] tensor")
+    if timestamps is not None and (timestamps.dtype != torch.int32 or not timestamps.is_cuda):
+        raise TypeError("timestamps must be a CUDA int32 tensor [T]")
+    p.timestamps = timestamps.data_ptr() if timestamps is not None else None
+    if rab_pos is not None:
+        p.rab_pos, p.rab_pos_buckets = rab_pos.data_ptr(), rab_pos.shape[1]
+    if rab_time is not None:
+        p.rab_time, p.rab_time_buckets = rab_time.data_ptr(), rab_time.shape[1]
+
+
 def _fwd_params(q, k, v, seq_offsets, num_targets, contextual_len, K1, K2, alpha, N,
                 max_seq_len, events=None, candidates_only=False) -> _abi.FwdParams:
     T, H, d = q.shape
@@ -107,14 +123,18 @@ def hstu_sla_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, seq_offsets:
                  num_targets: Optional[torch.Tensor], *, contextual_len: int, K1: int, K2: int,
                  alpha: float, N: float, max_seq_len: Optional[int] = None,
                  out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
-                 stream=None, events=None, candidates_only: bool = False) -> torch.Tensor:
+                 stream=None, events=None, candidates_only: bool = False,
+                 timestamps=None, rab_pos=None, rab_time=None) -> torch.Tensor:
     """SLA HSTU attention forward; returns out [T, H, d] (bf16).  `events`: an
     optional pair of torch.cuda.Event recorded around the attention kernel.
     candidates_only: M-FALCON scoring, only the query tiles that hold
-    candidates are computed (other rows of `out` are left as they were)."""
+    candidates are computed (other rows of `out` are left as they were).
+    timestamps / rab_pos / rab_time: the optional relative attention bias
+    (include/hstu_sla.h)."""
     lib = _abi.load()
     p = _fwd_params(q, k, v, seq_offsets, num_targets, contextual_len, K1, K2, alpha, N,
                     max_seq_len, events, candidates_only)
+    _set_rab(p, q.shape[1], timestamps, rab_pos, rab_time)
     if out is None:
         out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
     p.out = out.data_ptr()
@@ -149,12 +169,20 @@ def hstu_sla_bwd(dout: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: torch.
                  contextual_len: int, K1: int, K2: int, alpha: float, N: float,
                  max_seq_len: Optional[int] = None, dq: Optional[torch.Tensor] = None,
                  dk: Optional[torch.Tensor] = None, dv: Optional[torch.Tensor] = None,
-                 workspace: Optional[torch.Tensor] = None, stream=None, events=None):
-    """SLA HSTU attention backward; returns (dq, dk, dv) [T, H, d] (bf16)."""
+                 workspace: Optional[torch.Tensor] = None, stream=None, events=None,
+                 timestamps=None, rab_pos=None, rab_time=None):
+    """SLA HSTU attention backward; returns (dq, dk, dv) [T, H, d] (bf16), and
+    with a relative attention bias (dq, dk, dv, (d_rab_pos, d_rab_time)),
+    fp32, None for an absent table."""
     lib = _abi.load()
     p = _abi.BwdParams()
     p.fwd = _fwd_params(q, k, v, seq_offsets, num_targets, contextual_len, K1, K2, alpha, N,
                         max_seq_len, events)
+    _set_rab(p.fwd, q.shape[1], timestamps, rab_pos, rab_time)
+    d_rab = (torch.empty_like(rab_pos) if rab_pos is not None else None,
+             torch.empty_like(rab_time) if rab_time is not None else None)
+    p.d_rab_pos = d_rab[0].data_ptr() if d_rab[0] is not None else None
+    p.d_rab_time = d_rab[1].data_ptr() if d_rab[1] is not None else None
     H, d = p.fwd.H, p.fwd.d
     dq = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device) if dq is None else dq
     dk = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device) if dk is None else dk
@@ -166,6 +194,8 @@ def hstu_sla_bwd(dout: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: torch.
     ws = _workspace(_abi.WS_BWD, p.fwd.total_tokens, p.fwd.B, H, d, q.device, workspace)
     _check(lib.hstu_sla_bwd(ctypes.byref(p), ws.data_ptr(), ws.numel(), _stream_ptr(stream)),
            "hstu_sla_bwd")
+    if rab_pos is not None or rab_time is not None:
+        return dq, dk, dv, d_rab
     return dq, dk, dv
 
 

@@ -38,6 +38,9 @@ class FwdParams(ctypes.Structure):
         ("out", ctypes.c_void_p), ("out_row_stride", ctypes.c_int64),
         ("event_begin", ctypes.c_void_p), ("event_end", ctypes.c_void_p),
         ("candidates_only", ctypes.c_int32),
+        ("timestamps", ctypes.c_void_p), ("rab_pos", ctypes.c_void_p),
+        ("rab_time", ctypes.c_void_p), ("rab_pos_buckets", ctypes.c_int32),
+        ("rab_time_buckets", ctypes.c_int32),
     ]
 
 
@@ -48,6 +51,7 @@ class BwdParams(ctypes.Structure):
         ("dq", ctypes.c_void_p), ("dk", ctypes.c_void_p), ("dv", ctypes.c_void_p),
         ("dq_row_stride", ctypes.c_int64), ("dk_row_stride", ctypes.c_int64),
         ("dv_row_stride", ctypes.c_int64),
+        ("d_rab_pos", ctypes.c_void_p), ("d_rab_time", ctypes.c_void_p),
     ]
 
 

@@ -9,8 +9,9 @@ using namespace hstu;
 
 namespace {
 
-// 101: hstu_sla_fwd_params.candidates_only; 102: FP8 forward; 103: grouped calls
-constexpr int kAbiVersion = 103;
+// 101: hstu_sla_fwd_params.candidates_only; 102: FP8 forward; 103: grouped calls;
+// 104: relative attention bias
+constexpr int kAbiVersion = 104;
 static_assert(HSTU_SLA_MAX_GROUPS == kMaxGroups, "one grouped launch holds every group");
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
@@ -32,6 +33,10 @@ int check_common(const hstu_sla_fwd_params* f) {
   if (f->K1 < 0 || f->K2 < 0 || f->contextual_len < 0) return HSTU_SLA_ERR_INVALID_ARG;
   if (!(f->N > 0.f) || !isfinite(f->N) || !isfinite(f->alpha)) return HSTU_SLA_ERR_INVALID_ARG;
   if (f->seq_offsets == nullptr) return HSTU_SLA_ERR_INVALID_ARG;
+  if (f->rab_pos && (f->rab_pos_buckets < 1 || f->rab_pos_buckets > 32))
+    return HSTU_SLA_ERR_INVALID_ARG;
+  if (f->rab_time && (f->rab_time_buckets < 1 || f->rab_time_buckets > 32 || !f->timestamps))
+    return HSTU_SLA_ERR_INVALID_ARG;
   int e;
   if ((e = check_tensor(f->q, f->q_row_stride, f))) return e;
   if ((e = check_tensor(f->k, f->k_row_stride, f))) return e;
@@ -69,6 +74,11 @@ AttnArgs make_args(const hstu_sla_fwd_params* f, void* ws) {
   a.k_rs = f->k_row_stride;
   a.v_rs = f->v_row_stride;
   a.cand_only = f->candidates_only != 0;
+  a.ts = f->timestamps;
+  a.rab_pos = f->rab_pos;
+  a.rab_time = f->rab_time;
+  a.nbp = f->rab_pos ? f->rab_pos_buckets : 1;
+  a.nbt = f->rab_time ? f->rab_time_buckets : 1;
   return a;
 }
 
@@ -155,6 +165,7 @@ int hstu_sla_fwd_grouped(const hstu_sla_fwd_params* groups, int32_t G, void* wor
     f[g] = &groups[g];
     if ((e = check_common(f[g]))) return e;
     if ((e = check_tensor(f[g]->out, f[g]->out_row_stride, f[g]))) return e;
+    if (f[g]->rab_pos || f[g]->rab_time) return HSTU_SLA_ERR_UNSUPPORTED;
     if (f[g]->d != f[0]->d) return HSTU_SLA_ERR_UNSUPPORTED;
     T[g] = f[g]->total_tokens;
     Bs[g] = f[g]->B;
@@ -199,6 +210,7 @@ int hstu_sla_bwd_grouped(const hstu_sla_bwd_params* groups, int32_t G, void* wor
     const hstu_sla_bwd_params* p = &groups[g];
     f[g] = &p->fwd;
     if ((e = check_common(f[g]))) return e;
+    if (f[g]->rab_pos || f[g]->rab_time) return HSTU_SLA_ERR_UNSUPPORTED;
     if ((e = check_tensor(p->dout, p->dout_row_stride, f[g]))) return e;
     if ((e = check_tensor(p->dq, p->dq_row_stride, f[g]))) return e;
     if ((e = check_tensor(p->dk, p->dk_row_stride, f[g]))) return e;
@@ -312,6 +324,13 @@ int sla_bwd(const hstu_sla_bwd_params* p, void* workspace, size_t workspace_byte
   a.dq_rs = p->dq_row_stride;
   a.dk_rs = p->dk_row_stride;
   a.dv_rs = p->dv_row_stride;
+  if (f->rab_pos || f->rab_time) {  // relative attention bias: one-pass kernel only
+    if (f->d != kFusedBwdD) return HSTU_SLA_ERR_UNSUPPORTED;
+    if ((f->rab_pos && !p->d_rab_pos) || (f->rab_time && !p->d_rab_time))
+      return HSTU_SLA_ERR_INVALID_ARG;
+    a.d_rab_pos = f->rab_pos ? p->d_rab_pos : nullptr;
+    a.d_rab_time = f->rab_time ? p->d_rab_time : nullptr;
+  }
   cudaError_t ce;
   if (fz != nullptr) {  // the STU layer's SiLU' and bias-gradient fusion
     // silu_qkv_kernel: 3 H d / 8 threads, whole warps per block part

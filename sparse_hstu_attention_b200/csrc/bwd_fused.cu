@@ -71,7 +71,11 @@ constexpr int OFF_DS = OFF_B2 + kSt * STILE;
 constexpr int OFF_BAR = OFF_DS + 2 * DSTILE;
 constexpr int OFF_UNIT = OFF_BAR + 512;
 constexpr int OFF_SLOT = OFF_UNIT + kUSlots * (int)sizeof(UnitRec);
-constexpr int SMEM = OFF_SLOT + 16 + 1024;
+// relative attention bias: per-unit histograms of the bias gradient, two
+// (alternating units), 32 position then 32 time buckets each
+constexpr int kHistBins = 64;
+constexpr int OFF_HIST = OFF_SLOT + 16;
+constexpr int SMEM = OFF_HIST + 2 * kHistBins * 4 + 1024;
 static_assert(SMEM <= 232448, "shared memory budget");
 constexpr uint32_t SBO = 8 * SW;
 // 128 x 64 scores, both operands K-major
@@ -86,7 +90,7 @@ enum {
   F_B_EMPTY = F_B_FULL + kSt, F_X_FULL = F_B_EMPTY + kSt, F_OP_FULL = F_X_FULL + 2,
   F_DQ_FULL = F_OP_FULL + 2, F_DQ_EMPTY = F_DQ_FULL + 2, F_ACC_FULL = F_DQ_EMPTY + 2,
   F_ACC_EMPTY, F_U_FULL, F_U_EMPTY = F_U_FULL + kUSlots, F_DRAIN = F_U_EMPTY + kUSlots,
-  F_COUNT
+  F_H_DONE, F_H_ZERO = F_H_DONE + 2, F_COUNT = F_H_ZERO + 2
 };
 static_assert(8 * F_COUNT <= 512, "barrier area");
 
@@ -127,6 +131,11 @@ struct BwdMaps {
 // reduction, not a round trip).
 __device__ __forceinline__ void red_add_f32(float* p, uint32_t v) { atomicAdd(p, __uint_as_float(v)); }
 
+// RAB: the relative attention bias is added to every recomputed score and
+// its gradient is accumulated per unit in a shared-memory histogram (each
+// thread adds runs of equal buckets along its query columns; one pointwise
+// warp flushes the unit's sums into this head's table gradients).
+template <bool RAB>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_kvq_kernel(const __grid_constant__ BwdMaps maps, const __grid_constant__ GroupSet gs) {
   extern __shared__ uint8_t smem_raw[];
@@ -139,6 +148,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar = [&](int i) { return bar0 + 8u * i; };
   UnitRec* ring = reinterpret_cast<UnitRec*>(base_ptr + OFF_UNIT);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + OFF_SLOT);
+  float* hist = reinterpret_cast<float*>(base_ptr + OFF_HIST);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   WsHeader* const ws = gs.common;  // status word and scheduler of the launch
@@ -174,6 +184,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(F_U_EMPTY + s), 1 + kPwWarps);     // MMA lane + pointwise warps
     }
     mbar_init(bar(F_DRAIN), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(F_H_DONE + i), kPwWarps);  // every pointwise warp's sums are in
+      mbar_init(bar(F_H_ZERO + i), 1);         // flushed and cleared
+    }
     fence_barrier_init();
     for (int p = 0; p < kMaxGroups && p < gs.G; ++p) {
       if (gs.g[p].T == 0) continue;  // no map was built
@@ -187,6 +201,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(smem_addr(tmem_slot), kTmemCols);
     tmem_relinquish();
   }
+  if (RAB)
+    for (int i = threadIdx.x; i < 2 * kHistBins; i += blockDim.x) hist[i] = 0.f;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -389,6 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t ds_row = sDS + (uint32_t)row * SW;
     const uint32_t swz = (uint32_t)(row & 7);
     uint32_t xc = 0, accn = 0;
+    uint32_t hu = 0;  // units with steps so far (histogram buffer hu & 1)
     bool ok = true;
     for (int kk = 0; ok; ++kk) {
       const int slot = kk % kUSlots;
@@ -425,6 +442,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       // dQ workspace ([H][T][D]) column of this lane (head-dim index `row`)
       // at the sequence start
       float* dqa = A.dqacc + ((int64_t)h * A.T + s0) * D + row;
+      // relative attention bias: this head's tables, this key's timestamp and
+      // the unit's histogram buffer (free once the unit two back was flushed)
+      const float* rab_p = nullptr;
+      const float* rab_t = nullptr;
+      int32_t tj = 0;
+      float* hst = hist + (hu & 1) * kHistBins;
+      if constexpr (RAB) {
+        rab_p = A.rab_pos ? A.rab_pos + h * A.nbp : nullptr;
+        rab_t = A.rab_time ? A.rab_time + h * A.nbt : nullptr;
+        tj = (A.ts && rr < L) ? __ldg(A.ts + s0 + rr) : 0;
+        ok = warp_wait(bar(F_H_ZERO + (hu & 1)), ((hu >> 1) & 1) ^ 1, ws);
+        if (!ok) break;
+      }
       SpanCursor c;
       c.begin(r);
       for (int n = 0; n < nt; ++n, ++xc, c.next(r)) {
@@ -441,6 +471,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Fully visible tiles skip the mask; others clear invisible entries by
         // one bit test against this key's 32-row visibility mask.
         const uint32_t bits = full ? 0xFFFFFFFFu : key_mask_bits(km, c0 + col);
+        // relative attention bias: the 32 queries' timestamps (one per lane)
+        // and this step's runs of equal buckets (position, time)
+        int32_t tql = 0;
+        int run_p = -1, run_t = -1;
+        float sum_p = 0.f, sum_t = 0.f;
+        if constexpr (RAB) {
+          const int ql = c0 + col + lane;
+          tql = (A.ts && ql < L) ? __ldg(A.ts + s0 + ql) : 0;
+        }
+        auto run_add = [&](int& run, float& sum, int bin, float g) {
+          if (bin != run) {
+            if (run >= 0) atomicAdd(hst + run, sum);
+            run = bin;
+            sum = g;
+          } else {
+            sum += g;
+          }
+        };
         // Two rounds of 16 query columns each (fewer live registers).  Round r
         // writes P^T (8 packed columns) then dS^T (8) over the 16 score
         // columns it read, and copies dS^T to 16-byte chunks half*4 + 2r,
@@ -451,9 +499,35 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld16(xs_addr + 16 * r, xs);
           tmem_ld16(xd_addr + 16 * r, xd);
           tmem_ld_wait2(xs, xd);
+          if constexpr (RAB) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            bwd_pair(xs[2 * e], xs[2 * e + 1], xd[2 * e], xd[2 * e + 1], half_alpha2, pp[e], dd[e]);
+            for (int e = 0; e < 8; ++e) {
+              const int k = 16 * r + 2 * e;  // column within this half
+              const int32_t tqa = __shfl_sync(0xffffffffu, tql, k);
+              const int32_t tqb = __shfl_sync(0xffffffffu, tql, k + 1);
+              int bpa, bta, bpb, btb;
+              rab_buckets(A.nbp, A.nbt, c0 + col + k, rr, Lh, tqa, tj, bpa, bta);
+              rab_buckets(A.nbp, A.nbt, c0 + col + k + 1, rr, Lh, tqb, tj, bpb, btb);
+              const float ba = (rab_p ? __ldg(rab_p + bpa) : 0.f) + (rab_t ? __ldg(rab_t + bta) : 0.f);
+              const float bb = (rab_p ? __ldg(rab_p + bpb) : 0.f) + (rab_t ? __ldg(rab_t + btb) : 0.f);
+              float ga, gb;
+              bwd_pair_bias(xs[2 * e], xs[2 * e + 1], xd[2 * e], xd[2 * e + 1], half_alpha2, ba, bb,
+                            pp[e], dd[e], ga, gb);
+              if ((bits >> k) & 1u) {
+                run_add(run_p, sum_p, bpa, ga);
+                run_add(run_t, sum_t, 32 + bta, ga);
+              }
+              if ((bits >> (k + 1)) & 1u) {
+                run_add(run_p, sum_p, bpb, gb);
+                run_add(run_t, sum_t, 32 + btb, gb);
+              }
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              bwd_pair(xs[2 * e], xs[2 * e + 1], xd[2 * e], xd[2 * e + 1], half_alpha2, pp[e],
+                       dd[e]);
+          }
           if (!full) {
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
@@ -467,6 +541,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int q = 0; q < 2; ++q)
             st_shared_v4(dsr + ((((uint32_t)(half * 4 + 2 * r + q)) ^ swz) << 4), dd[4 * q],
                          dd[4 * q + 1], dd[4 * q + 2], dd[4 * q + 3]);
+        }
+        if constexpr (RAB) {  // this step's last runs
+          if (run_p >= 0) atomicAdd(hst + run_p, sum_p);
+          if (run_t >= 0) atomicAdd(hst + run_t, sum_t);
         }
         fence_proxy_async_smem();  // visible to the dQ MMA
         tmem_st_wait();
@@ -530,6 +608,30 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int q = 0; q < 4; ++q)
             dst[q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
         }
+      }
+      if constexpr (RAB) {
+        // this warp's sums of the unit are in; the first pointwise warp adds
+        // the unit's histogram into this head's table gradients (dS2 is
+        // 2 dP SiLU'(x); the gradient takes dP SiLU'(x) / N) and clears it
+        warp_arrive(bar(F_H_DONE + (hu & 1)));
+        if (pw == 0) {
+          ok = warp_wait(bar(F_H_DONE + (hu & 1)), (hu >> 1) & 1, ws);
+          if (!ok) break;
+          const float sc = 0.5f * A.inv_n;
+          for (int bin = lane; bin < kHistBins; bin += 32) {
+            const float v = hst[bin];
+            if (bin < 32) {
+              if (bin < A.nbp && A.d_rab_pos) atomicAdd(A.d_rab_pos + h * A.nbp + bin, v * sc);
+            } else if (bin - 32 < A.nbt && A.d_rab_time) {
+              atomicAdd(A.d_rab_time + h * A.nbt + (bin - 32), v * sc);
+            }
+            hst[bin] = 0.f;
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(F_H_ZERO + (hu & 1)));
+          __syncwarp();
+        }
+        ++hu;
       }
       warp_arrive(bar(F_U_EMPTY + slot));
     }
@@ -673,11 +775,22 @@ cudaError_t launch_bwd_fused_grouped(const GroupSet& gs, cudaStream_t st) {
     units += max_items(a.T, a.B) * a.H;
   }
   if (units == 0) return cudaSuccess;
-  e = cudaFuncSetAttribute(bwd_kvq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+  const bool rab = gs.G == 1 && (gs.g[0].rab_pos != nullptr || gs.g[0].rab_time != nullptr);
+  if (rab) {  // the table gradients are overwritten
+    const AttnArgs& a = gs.g[0];
+    if (a.d_rab_pos &&
+        (e = cudaMemsetAsync(a.d_rab_pos, 0, sizeof(float) * a.H * a.nbp, st)) != cudaSuccess)
+      return e;
+    if (a.d_rab_time &&
+        (e = cudaMemsetAsync(a.d_rab_time, 0, sizeof(float) * a.H * a.nbt, st)) != cudaSuccess)
+      return e;
+  }
+  const auto kern = rab ? bwd_kvq_kernel<true> : bwd_kvq_kernel<false>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
   if (e != cudaSuccess) return e;
   const int sms = device_sm_count();
   const int grid = (int)(units < sms ? units : sms);
-  bwd_kvq_kernel<<<grid, kThreads, SMEM, st>>>(m, gs);
+  kern<<<grid, kThreads, SMEM, st>>>(m, gs);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   for (int p = 0; p < gs.G; ++p) {
     const AttnArgs& a = gs.g[p];

@@ -120,7 +120,8 @@ struct FwdMaps {
   CUtensorMap q[kMaxGroups], k[kMaxGroups], v[kMaxGroups], o[kMaxGroups];
 };
 
-template <int D>
+// RAB: add the relative attention bias to every score (AttnArgs::rab_*).
+template <int D, bool RAB>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_tc_kernel(const __grid_constant__ FwdMaps maps, const __grid_constant__ GroupSet gs) {
   using C = Cfg<D>;
@@ -567,6 +568,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int K1 = A.K1, K2e = A.K2e;
       const uint64_t half_alpha2 = f2s(0.5f * A.alpha);
       const RowMask m = row_mask(i, r->L, Lh, K1, K2e);
+      // relative attention bias: this head's tables and this row's timestamp
+      const float* rab_p = nullptr;
+      const float* rab_t = nullptr;
+      int32_t ti = 0;
+      if constexpr (RAB) {
+        rab_p = A.rab_pos ? A.rab_pos + h * A.nbp : nullptr;
+        rab_t = A.rab_time ? A.rab_time + h * A.nbt : nullptr;
+        ti = (A.ts && i < r->L) ? __ldg(A.ts + s0 + i) : 0;
+      }
       SpanCursor c;
       c.begin(r);
       for (int n = 0; n < nt; ++n, ++tc, c.next(r)) {
@@ -589,10 +599,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld16(taddr + 16, c1);
           tmem_ld_wait2(c0, c1);
           uint32_t p[16];
+          if constexpr (RAB) {
+            // the 32 keys' timestamps, one per lane, then each score's bias
+            const int jl = j0 + col + lane;
+            const int32_t tjl = (A.ts && jl < r->L) ? __ldg(A.ts + s0 + jl) : 0;
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            p[e] = silu_pair(c0[2 * e], c0[2 * e + 1], half_alpha2);
-            p[8 + e] = silu_pair(c1[2 * e], c1[2 * e + 1], half_alpha2);
+            for (int e = 0; e < 16; ++e) {
+              const int ja = j0 + col + 2 * e, jb = ja + 1;
+              const float ba = rab_value(rab_p, A.nbp, rab_t, A.nbt, i, ja, Lh, ti,
+                                         __shfl_sync(0xffffffffu, tjl, 2 * e));
+              const float bb = rab_value(rab_p, A.nbp, rab_t, A.nbt, i, jb, Lh, ti,
+                                         __shfl_sync(0xffffffffu, tjl, 2 * e + 1));
+              p[e] = silu_pair_bias(e < 8 ? c0[2 * e] : c1[2 * e - 16],
+                                    e < 8 ? c0[2 * e + 1] : c1[2 * e - 15], half_alpha2, ba, bb);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              p[e] = silu_pair(c0[2 * e], c0[2 * e + 1], half_alpha2);
+              p[8 + e] = silu_pair(c1[2 * e], c1[2 * e + 1], half_alpha2);
+            }
           }
           if (!full) {
             const uint32_t bits = row_mask_bits(m, j0 + col);
@@ -652,12 +678,13 @@ cudaError_t launch_d(const GroupSet& gs, cudaStream_t st) {
     units += max_items(a.T, a.B) * a.H;
   }
   if (units == 0) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel<D>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  const bool rab = gs.G == 1 && (gs.g[0].rab_pos != nullptr || gs.g[0].rab_time != nullptr);
+  const auto kern = rab ? fwd_tc_kernel<D, true> : fwd_tc_kernel<D, false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   const int sms = device_sm_count();
   const int grid = (int)(units < sms ? units : sms);
-  fwd_tc_kernel<D><<<grid, kThreads, C::SMEM, st>>>(m, gs);
+  kern<<<grid, kThreads, C::SMEM, st>>>(m, gs);
   return cudaGetLastError();
 }
 

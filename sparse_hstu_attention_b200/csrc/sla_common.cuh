@@ -111,7 +111,46 @@ struct AttnArgs {
   float* db_k;
   float* db_v;
   float* db_part;  // [kSiluBlocks][3 (q, k, v)][H * d] partial sums (workspace)
+  // Relative attention bias (optional): per-head tables of nbp / nbt log2
+  // buckets of the position and timestamp differences; their gradients.
+  const int32_t* ts;
+  const float* rab_pos;
+  const float* rab_time;
+  int nbp, nbt;
+  float* d_rab_pos;
+  float* d_rab_time;
 };
+
+// floor(log2(n + 1)) for n >= 0, at most nb - 1.
+__host__ __device__ __forceinline__ int rab_bucket(uint32_t n, int nb) {
+#ifdef __CUDA_ARCH__
+  const int b = 31 - __clz(n + 1u);
+#else
+  int b = 0;
+  for (uint32_t x = n + 1u; x > 1u; x >>= 1) ++b;
+#endif
+  return b < nb - 1 ? b : nb - 1;
+}
+
+// Buckets of the pair (query i, key j) in a sequence with Lh history rows
+// (ti, tj the timestamps): the position difference measures a candidate row
+// from Lh (0 to itself).
+__device__ __forceinline__ void rab_buckets(int nbp, int nbt, int i, int j, int Lh, int32_t ti,
+                                            int32_t tj, int& bp, int& bt) {
+  int dpos = i < Lh ? i - j : (j == i ? 0 : Lh - j);
+  bp = rab_bucket((uint32_t)(dpos > 0 ? dpos : 0), nbp);
+  const int64_t dt = (int64_t)ti - (int64_t)tj;
+  const int64_t adt = dt < 0 ? -dt : dt;
+  bt = rab_bucket(adt > 0x7FFFFFFF ? 0x7FFFFFFFu : (uint32_t)adt, nbt);
+}
+
+// The bias of a pair from one head's tables (tp, tt; NULL adds nothing).
+__device__ __forceinline__ float rab_value(const float* tp, int nbp, const float* tt, int nbt,
+                                           int i, int j, int Lh, int32_t ti, int32_t tj) {
+  int bp, bt;
+  rab_buckets(nbp, nbt, i, j, Lh, ti, tj, bp, bt);
+  return (tp ? __ldg(tp + bp) : 0.f) + (tt ? __ldg(tt + bt) : 0.f);
+}
 
 __host__ __device__ inline int cdiv(int a, int b) { return (a + b - 1) / b; }
 __host__ __device__ __forceinline__ int imin(int a, int b) { return a < b ? a : b; }

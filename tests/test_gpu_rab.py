@@ -1,0 +1,119 @@
+"""GPU parity of the relative attention bias (HSTU notes, section 2.4, Eq. 2:
+phi2(Q K^T + rab^{p,t})): forward, dq, dk, dv and both tables' gradients
+against the oracle on seeded inputs (TOL of max|ref| per tensor), each table
+alone, all-zero tables equal to the bias-free kernels, the forward at
+head_dim 64, and the host-side refusals (backward at head_dim 64, grouped)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sparse_hstu_attention_b200 as sla
+from sparse_hstu_attention_b200 import _abi
+from workloads import WORKLOADS, draw_rab_tables, draw_timestamps, make_batch, with_params
+
+from parity import TOL, assert_close, kwargs_of, to_gpu
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda")
+NP, NT = 12, 24
+
+
+def _case(lengths=(300, 1200, 77, 640, 129), nt=16, H=4, d=128, K1=256, K2=64, ctx=16, seed=21):
+    w = with_params(WORKLOADS["tiny"], H=H, d=d, K1=K1, K2=K2, contextual_len=ctx,
+                    num_targets=nt, alpha=d ** -0.5, N=float(max(lengths)))
+    lengths = np.array(lengths, dtype=np.int64)
+    b = make_batch(w, lengths=lengths, num_targets=np.minimum(nt, lengths), seed=seed)
+    ts = draw_timestamps(b.lengths, b.num_targets, seed)
+    rp, rt = draw_rab_tables(H, NP, NT, seed)
+    return b, ts, rp, rt
+
+
+def _run(b, ts, rp, rt, bwd=True):
+    g = to_gpu(b)
+    rab = dict(timestamps=torch.from_numpy(ts).to(DEV),
+               rab_pos=None if rp is None else rp.to(DEV),
+               rab_time=None if rt is None else rt.to(DEV))
+    out = sla.hstu_sla_fwd(g["q"], g["k"], g["v"], g["offs"], g["nts"], **kwargs_of(b), **rab)
+    res = [out]
+    if bwd:
+        res += list(sla.hstu_sla_bwd(g["dout"], g["q"], g["k"], g["v"], g["offs"], g["nts"],
+                                     **kwargs_of(b), **rab))
+    torch.cuda.synchronize()
+    return res
+
+
+def _oracle(b, ts, rp, rt):
+    w = b.workload
+    return oracle.Problem(b.seq_offsets, b.num_targets, w.H, w.d, w.contextual_len, w.K1, w.K2,
+                          w.alpha, w.N, timestamps=ts,
+                          rab_pos=None if rp is None else rp.numpy(),
+                          rab_time=None if rt is None else rt.numpy())
+
+
+@pytest.mark.parametrize("tables", ["both", "pos", "time"])
+def test_rab_forward_backward_and_table_gradients(tables):
+    b, ts, rp, rt = _case()
+    rp = rp if tables in ("both", "pos") else None
+    rt = rt if tables in ("both", "time") else None
+    out, dq, dk, dv, (drp, drt) = _run(b, ts, rp, rt)
+    p = _oracle(b, ts, rp, rt)
+    assert_close("out", out, p.fwd(b.q, b.k, b.v))
+    rq, rk, rv = p.bwd(b.q, b.k, b.v, b.dout)
+    assert_close("dq", dq, rq)
+    assert_close("dk", dk, rk)
+    assert_close("dv", dv, rv)
+    rdp, rdt = p.bwd_rab(b.q, b.k, b.v, b.dout)
+    if rp is not None:
+        assert_close("d rab_pos", drp, rdp)
+    if rt is not None:
+        assert_close("d rab_time", drt, rdt)
+
+
+def test_rab_edge_batch():
+    """Ragged tiles, a sequence of candidates only, K1 = 0 (prefix only) and
+    candidate self-pairs in their own bucket."""
+    b, ts, rp, rt = _case(lengths=(1, 130, 64, 65, 257, 9), nt=9, K1=0, K2=40, ctx=8, seed=5)
+    out, dq, dk, dv, (drp, drt) = _run(b, ts, rp, rt)
+    p = _oracle(b, ts, rp, rt)
+    assert_close("out", out, p.fwd(b.q, b.k, b.v))
+    rq, rk, rv = p.bwd(b.q, b.k, b.v, b.dout)
+    for name, got, ref in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
+        assert_close(name, got, ref)
+    rdp, rdt = p.bwd_rab(b.q, b.k, b.v, b.dout)
+    assert_close("d rab_pos", drp, rdp)
+    assert_close("d rab_time", drt, rdt)
+
+
+def test_zero_tables_equal_the_bias_free_kernels():
+    b, ts, rp, rt = _case(seed=8)
+    out, dq, dk, dv, _ = _run(b, ts, torch.zeros_like(rp), torch.zeros_like(rt))
+    g = to_gpu(b)
+    out0 = sla.hstu_sla_fwd(g["q"], g["k"], g["v"], g["offs"], g["nts"], **kwargs_of(b))
+    dq0, dk0, dv0 = sla.hstu_sla_bwd(g["dout"], g["q"], g["k"], g["v"], g["offs"], g["nts"],
+                                     **kwargs_of(b))
+    torch.cuda.synchronize()
+    assert torch.equal(out, out0)
+    assert torch.equal(dk, dk0) and torch.equal(dv, dv0)
+    assert_close("dq", dq, dq0.float().cpu().numpy().astype(np.float64), tol=1e-2)
+
+
+def test_rab_forward_head_dim_64_and_refusals():
+    b, ts, rp, rt = _case(lengths=(200, 77), H=3, d=64, K1=50, K2=8, ctx=4, seed=9)
+    (out,) = _run(b, ts, rp, rt, bwd=False)
+    assert_close("out d64", out, _oracle(b, ts, rp, rt).fwd(b.q, b.k, b.v))
+    with pytest.raises(sla.SLAError) as ex:
+        _run(b, ts, rp, rt)
+    assert ex.value.code == _abi.ERR_UNSUPPORTED
+    b2, ts2, rp2, rt2 = _case(seed=10)
+    g = to_gpu(b2)
+    grp = dict(q=g["q"], k=g["k"], v=g["v"], seq_offsets=g["offs"], num_targets=g["nts"],
+               **kwargs_of(b2))
+    p = sla._group_params(grp)
+    sla._set_rab(p, 4, torch.from_numpy(ts2).to(DEV), rp2.to(DEV), None)
+    out = torch.empty_like(g["q"])
+    p.out, p.out_row_stride = out.data_ptr(), out.stride(0)
+    arr = (_abi.FwdParams * 1)(p)
+    ws = torch.empty(1 << 20, dtype=torch.uint8, device=DEV)
+    assert _abi.load().hstu_sla_fwd_grouped(arr, 1, ws.data_ptr(), ws.numel(), None) == \
+        _abi.ERR_UNSUPPORTED

@@ -118,6 +118,31 @@ def draw_lengths(w: Workload) -> np.ndarray:
     raise KeyError(w.name)
 
 
+def draw_timestamps(lengths, num_targets, seed: int) -> np.ndarray:
+    """Seeded int32 event times (seconds) for the relative attention bias:
+    per sequence a start in [1.6e9, 1.61e9), exponential gaps of mean 600 s
+    between history events, and every candidate at the request time (an
+    exponential gap after the last history event)."""
+    rng = np.random.default_rng(seed)
+    out = []
+    for L, nt in zip(np.asarray(lengths, np.int64), np.asarray(num_targets, np.int64)):
+        Lh = int(L - nt)
+        start = 1_600_000_000 + int(rng.integers(0, 10_000_000))
+        hist = start + np.cumsum(rng.exponential(600.0, size=Lh).astype(np.int64))
+        req = (hist[-1] if Lh else start) + int(rng.exponential(600.0))
+        out.append(np.concatenate([hist, np.full(int(nt), req, np.int64)]))
+    ts = np.concatenate(out) if out else np.zeros(0, np.int64)
+    assert ts.size == 0 or ts.max() < 2 ** 31
+    return ts.astype(np.int32)
+
+
+def draw_rab_tables(H: int, n_pos: int, n_time: int, seed: int):
+    """Seeded relative-attention-bias tables [H][buckets], N(0, 0.5^2)."""
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    return (torch.randn((H, n_pos), generator=g) * 0.5,
+            torch.randn((H, n_time), generator=g) * 0.5)
+
+
 def offsets_from_lengths(lengths) -> np.ndarray:
     lengths = np.asarray(lengths, dtype=np.int64)
     return np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64)
