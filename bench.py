@@ -445,6 +445,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--rab", action="store_true",
+                    help="attention workloads: with the relative attention bias (32 position and "
+                         "32 time buckets per head, seeded tables and timestamps)")
     ap.add_argument("--fp8", action="store_true",
                     help="stu workload: E4M3 forward projections (weights requantized every step)")
     args = ap.parse_args()
@@ -479,6 +482,12 @@ def main():
                        dtype=torch.uint8, device=dev)
     kw = dict(contextual_len=w.contextual_len, K1=w.K1, K2=w.K2, alpha=w.alpha, N=w.N,
               max_seq_len=int(batch.lengths.max()))
+    if args.rab:
+        from workloads import draw_rab_tables, draw_timestamps
+        rp, rt = draw_rab_tables(H, 32, 32, w.seed)
+        kw.update(timestamps=torch.from_numpy(
+            draw_timestamps(batch.lengths, batch.num_targets, w.seed)).to(dev),
+            rab_pos=rp.to(dev), rab_time=rt.to(dev))
     stream = torch.cuda.current_stream()
 
     def new_events(n):
@@ -585,7 +594,9 @@ def main():
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16, jagged lengths drawn per workload recipe)",
-        "config": _config(w, batch),
+        "config": dict(_config(w, batch), **(
+            {"relative_attention_bias": {"pos_buckets": 32, "time_buckets": 32}}
+            if args.rab else {})),
         "pct_of_peak": 100.0 * value / world / peak,
         "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
         "fwd_tflops": fl_f / (fwd_ms * 1e-3) / 1e12 if fwd_ms else None,
@@ -620,7 +631,7 @@ def main():
             "candidate_pairs_per_head": cp,
             "tflops": F.fwd_flops(cp, H, d) / (c_ms * 1e-3) / 1e12,
             "speedup_vs_full_forward": ms_step / c_ms}
-    if world == 1 and not args.no_cpu_baseline:
+    if world == 1 and not args.no_cpu_baseline and not args.rab:
         line["cpu_baseline"] = cpu_baseline(batch)
     print(json.dumps(line), flush=True)
     if world > 1:

@@ -127,6 +127,22 @@ struct BwdMaps {
   CUtensorMap k[kMaxGroups], v[kMaxGroups], q[kMaxGroups], dout[kMaxGroups];
 };
 
+// Adds each lane's (bin, sum) into the shared histogram, lanes of equal bins
+// first summed with shuffles (one shared atomic per distinct bin instead of
+// up to 32 on one address).  bin < 0: nothing.  Called by the whole warp.
+__device__ __forceinline__ void warp_flush_bins(float* hst, int bin, float sum, int lane) {
+  uint32_t todo = __ballot_sync(0xffffffffu, bin >= 0);
+  while (todo) {
+    const int b = __shfl_sync(0xffffffffu, bin, __ffs(todo) - 1);
+    const bool mine = bin == b;
+    float v = mine ? sum : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == __ffs(todo) - 1) atomicAdd(hst + b, v);
+    todo &= ~__ballot_sync(0xffffffffu, mine);
+  }
+}
+
 // Fire-and-forget fp32 addition in L2 (the result is unused, so this is a
 // reduction, not a round trip).
 __device__ __forceinline__ void red_add_f32(float* p, uint32_t v) { atomicAdd(p, __uint_as_float(v)); }
@@ -444,17 +460,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       float* dqa = A.dqacc + ((int64_t)h * A.T + s0) * D + row;
       // relative attention bias: this head's tables, this key's timestamp and
       // the unit's histogram buffer (free once the unit two back was flushed)
-      const float* rab_p = nullptr;
-      const float* rab_t = nullptr;
+      float tabp = 0.f, tabt = 0.f;  // bucket `lane` of this head's tables
       int32_t tj = 0;
       float* hst = hist + (hu & 1) * kHistBins;
       if constexpr (RAB) {
-        rab_p = A.rab_pos ? A.rab_pos + h * A.nbp : nullptr;
-        rab_t = A.rab_time ? A.rab_time + h * A.nbt : nullptr;
+        if (A.rab_pos && lane < A.nbp) tabp = __ldg(A.rab_pos + h * A.nbp + lane);
+        if (A.rab_time && lane < A.nbt) tabt = __ldg(A.rab_time + h * A.nbt + lane);
         tj = (A.ts && rr < L) ? __ldg(A.ts + s0 + rr) : 0;
         ok = warp_wait(bar(F_H_ZERO + (hu & 1)), ((hu >> 1) & 1) ^ 1, ws);
         if (!ok) break;
       }
+      // runs of equal buckets (position, time) along this key's query
+      // columns, which only grow through the unit's steps
+      int run_p = -1, run_t = -1;
+      float sum_p = 0.f, sum_t = 0.f;
+      auto run_add = [&](int& run, float& sum, int bin, float g) {
+        if (bin != run) {
+          if (run >= 0) atomicAdd(hst + run, sum);
+          run = bin;
+          sum = g;
+        } else {
+          sum += g;
+        }
+      };
       SpanCursor c;
       c.begin(r);
       for (int n = 0; n < nt; ++n, ++xc, c.next(r)) {
@@ -472,23 +500,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         // one bit test against this key's 32-row visibility mask.
         const uint32_t bits = full ? 0xFFFFFFFFu : key_mask_bits(km, c0 + col);
         // relative attention bias: the 32 queries' timestamps (one per lane)
-        // and this step's runs of equal buckets (position, time)
         int32_t tql = 0;
-        int run_p = -1, run_t = -1;
-        float sum_p = 0.f, sum_t = 0.f;
         if constexpr (RAB) {
           const int ql = c0 + col + lane;
           tql = (A.ts && ql < L) ? __ldg(A.ts + s0 + ql) : 0;
         }
-        auto run_add = [&](int& run, float& sum, int bin, float g) {
-          if (bin != run) {
-            if (run >= 0) atomicAdd(hst + run, sum);
-            run = bin;
-            sum = g;
-          } else {
-            sum += g;
-          }
-        };
         // Two rounds of 16 query columns each (fewer live registers).  Round r
         // writes P^T (8 packed columns) then dS^T (8) over the 16 score
         // columns it read, and copies dS^T to 16-byte chunks half*4 + 2r,
@@ -508,8 +524,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               int bpa, bta, bpb, btb;
               rab_buckets(A.nbp, A.nbt, c0 + col + k, rr, Lh, tqa, tj, bpa, bta);
               rab_buckets(A.nbp, A.nbt, c0 + col + k + 1, rr, Lh, tqb, tj, bpb, btb);
-              const float ba = (rab_p ? __ldg(rab_p + bpa) : 0.f) + (rab_t ? __ldg(rab_t + bta) : 0.f);
-              const float bb = (rab_p ? __ldg(rab_p + bpb) : 0.f) + (rab_t ? __ldg(rab_t + btb) : 0.f);
+              const float ba = rab_bias(tabp, tabt, bpa, bta);
+              const float bb = rab_bias(tabp, tabt, bpb, btb);
               float ga, gb;
               bwd_pair_bias(xs[2 * e], xs[2 * e + 1], xd[2 * e], xd[2 * e + 1], half_alpha2, ba, bb,
                             pp[e], dd[e], ga, gb);
@@ -541,10 +557,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int q = 0; q < 2; ++q)
             st_shared_v4(dsr + ((((uint32_t)(half * 4 + 2 * r + q)) ^ swz) << 4), dd[4 * q],
                          dd[4 * q + 1], dd[4 * q + 2], dd[4 * q + 3]);
-        }
-        if constexpr (RAB) {  // this step's last runs
-          if (run_p >= 0) atomicAdd(hst + run_p, sum_p);
-          if (run_t >= 0) atomicAdd(hst + run_t, sum_t);
         }
         fence_proxy_async_smem();  // visible to the dQ MMA
         tmem_st_wait();
@@ -610,6 +622,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if constexpr (RAB) {
+        // the unit's last runs, lanes with equal buckets added up first
+        warp_flush_bins(hst, run_p, sum_p, lane);
+        warp_flush_bins(hst, run_t, sum_t, lane);
         // this warp's sums of the unit are in; the first pointwise warp adds
         // the unit's histogram into this head's table gradients (dS2 is
         // 2 dP SiLU'(x); the gradient takes dP SiLU'(x) / N) and clears it

@@ -568,13 +568,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int K1 = A.K1, K2e = A.K2e;
       const uint64_t half_alpha2 = f2s(0.5f * A.alpha);
       const RowMask m = row_mask(i, r->L, Lh, K1, K2e);
-      // relative attention bias: this head's tables and this row's timestamp
-      const float* rab_p = nullptr;
-      const float* rab_t = nullptr;
+      // relative attention bias: bucket `lane` of this head's tables in
+      // this lane, and this row's timestamp
+      float tabp = 0.f, tabt = 0.f;
       int32_t ti = 0;
       if constexpr (RAB) {
-        rab_p = A.rab_pos ? A.rab_pos + h * A.nbp : nullptr;
-        rab_t = A.rab_time ? A.rab_time + h * A.nbt : nullptr;
+        if (A.rab_pos && lane < A.nbp) tabp = __ldg(A.rab_pos + h * A.nbp + lane);
+        if (A.rab_time && lane < A.nbt) tabt = __ldg(A.rab_time + h * A.nbt + lane);
         ti = (A.ts && i < r->L) ? __ldg(A.ts + s0 + i) : 0;
       }
       SpanCursor c;
@@ -606,10 +606,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
               const int ja = j0 + col + 2 * e, jb = ja + 1;
-              const float ba = rab_value(rab_p, A.nbp, rab_t, A.nbt, i, ja, Lh, ti,
-                                         __shfl_sync(0xffffffffu, tjl, 2 * e));
-              const float bb = rab_value(rab_p, A.nbp, rab_t, A.nbt, i, jb, Lh, ti,
-                                         __shfl_sync(0xffffffffu, tjl, 2 * e + 1));
+              int bpa, bta, bpb, btb;
+              rab_buckets(A.nbp, A.nbt, i, ja, Lh, ti, __shfl_sync(0xffffffffu, tjl, 2 * e), bpa,
+                          bta);
+              rab_buckets(A.nbp, A.nbt, i, jb, Lh, ti, __shfl_sync(0xffffffffu, tjl, 2 * e + 1),
+                          bpb, btb);
+              const float ba = rab_bias(tabp, tabt, bpa, bta);
+              const float bb = rab_bias(tabp, tabt, bpb, btb);
               p[e] = silu_pair_bias(e < 8 ? c0[2 * e] : c1[2 * e - 16],
                                     e < 8 ? c0[2 * e + 1] : c1[2 * e - 15], half_alpha2, ba, bb);
             }

@@ -134,22 +134,21 @@ __host__ __device__ __forceinline__ int rab_bucket(uint32_t n, int nb) {
 
 // Buckets of the pair (query i, key j) in a sequence with Lh history rows
 // (ti, tj the timestamps): the position difference measures a candidate row
-// from Lh (0 to itself).
+// from Lh (0 to itself); the time difference is exact for any two int32
+// values (unsigned) and capped at 2^31 - 1 (bucket 31).
 __device__ __forceinline__ void rab_buckets(int nbp, int nbt, int i, int j, int Lh, int32_t ti,
                                             int32_t tj, int& bp, int& bt) {
-  int dpos = i < Lh ? i - j : (j == i ? 0 : Lh - j);
+  const int dpos = i < Lh ? i - j : (j == i ? 0 : Lh - j);
   bp = rab_bucket((uint32_t)(dpos > 0 ? dpos : 0), nbp);
-  const int64_t dt = (int64_t)ti - (int64_t)tj;
-  const int64_t adt = dt < 0 ? -dt : dt;
-  bt = rab_bucket(adt > 0x7FFFFFFF ? 0x7FFFFFFFu : (uint32_t)adt, nbt);
+  const uint32_t adt = ti >= tj ? (uint32_t)ti - (uint32_t)tj : (uint32_t)tj - (uint32_t)ti;
+  bt = rab_bucket(adt < 0x7FFFFFFFu ? adt : 0x7FFFFFFFu, nbt);
 }
 
-// The bias of a pair from one head's tables (tp, tt; NULL adds nothing).
-__device__ __forceinline__ float rab_value(const float* tp, int nbp, const float* tt, int nbt,
-                                           int i, int j, int Lh, int32_t ti, int32_t tj) {
-  int bp, bt;
-  rab_buckets(nbp, nbt, i, j, Lh, ti, tj, bp, bt);
-  return (tp ? __ldg(tp + bp) : 0.f) + (tt ? __ldg(tt + bt) : 0.f);
+// The bias of a pair when lane b of the warp holds bucket b of this head's
+// position table (tabp) and time table (tabt), 0 beyond a table or without
+// one: two shuffles instead of two memory loads.  Every lane must call it.
+__device__ __forceinline__ float rab_bias(float tabp, float tabt, int bp, int bt) {
+  return __shfl_sync(0xffffffffu, tabp, bp) + __shfl_sync(0xffffffffu, tabt, bt);
 }
 
 __host__ __device__ inline int cdiv(int a, int b) { return (a + b - 1) / b; }
