@@ -117,3 +117,39 @@ def test_rab_forward_head_dim_64_and_refusals():
     ws = torch.empty(1 << 20, dtype=torch.uint8, device=DEV)
     assert _abi.load().hstu_sla_fwd_grouped(arr, 1, ws.data_ptr(), ws.numel(), None) == \
         _abi.ERR_UNSUPPORTED
+
+
+def _table_totals_agree(drp, drt):
+    """Both tables partition the same unmasked pairs into buckets, so per
+    head their gradients have the same total (up to fp32 summation)."""
+    sp, st = drp.double().sum(dim=1), drt.double().sum(dim=1)
+    scale = float(drp.double().abs().sum()) + float(drt.double().abs().sum())
+    assert torch.allclose(sp, st, atol=1e-4 * scale, rtol=0), (sp, st)
+
+
+def test_rab_full_size_sampled():
+    """hist16k at full size with both tables: forward and dq on sampled rows,
+    dk and dv on sampled keys against the oracle one by one; the tables'
+    gradients are checked by the equal-totals invariant and for finiteness."""
+    from parity import sample_tokens
+    b = make_batch(WORKLOADS["hist16k"])
+    ts = draw_timestamps(b.lengths, b.num_targets, b.workload.seed)
+    rp, rt = draw_rab_tables(b.workload.H, 32, 32, b.workload.seed)
+    out, dq, dk, dv, (drp, drt) = _run(b, ts, rp, rt)
+    p = _oracle(b, ts, rp, rt)
+    rows = sample_tokens(b, 120, seed=11)
+    keys = sample_tokens(b, 120, seed=12)
+    assert_close("out", out[rows], p.fwd(b.q, b.k, b.v, rows=rows))
+    assert_close("dq", dq[rows], p.bwd_dq(b.q, b.k, b.v, b.dout, rows=rows))
+    rk, rv = p.bwd_dkv(b.q, b.k, b.v, b.dout, keys=keys)
+    assert_close("dk", dk[keys], rk)
+    assert_close("dv", dv[keys], rv)
+    for t in (out, dq, dk, dv, drp, drt):
+        assert torch.isfinite(t.float()).all()
+    _table_totals_agree(drp, drt)
+
+
+def test_rab_table_totals_small():
+    b, ts, rp, rt = _case(seed=31)
+    *_, (drp, drt) = _run(b, ts, rp, rt)
+    _table_totals_agree(drp, drt)

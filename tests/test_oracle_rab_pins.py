@@ -134,3 +134,12 @@ def test_table_gradient_by_finite_differences(table, h, b):
         minus_t[h, b] -= eps
     fd = (loss(plus_p, plus_t) - loss(minus_p, minus_t)) / (2 * eps)
     assert math.isclose(g, fd, rel_tol=1e-6, abs_tol=1e-9), (g, fd)
+
+
+def test_both_tables_sum_the_same_pairs():
+    """Each unmasked pair adds its gradient to one position bucket and one
+    time bucket, so per head the two tables' gradients have equal totals."""
+    offs, nts, q, k, v, do, ts, rp, rt, cfg = _case(11)
+    p = oracle.Problem(offs, nts, timestamps=ts, rab_pos=rp, rab_time=rt, **cfg)
+    dp, dt = p.bwd_rab(q, k, v, do)
+    np.testing.assert_allclose(dp.sum(axis=1), dt.sum(axis=1), rtol=1e-12, atol=1e-12)
