@@ -192,7 +192,7 @@ int hstu_sla_bwd_grouped(const hstu_sla_bwd_params* groups, int32_t G, void* wor
  * allocate device memory: inference engines and plugin hosts that plan all
  * device memory before running and forbid allocation inside their launch
  * path, and latency-critical loops that cannot afford cudaMalloc/cudaFree
- * (which may synchronise the device).  The pages have no counterpart: this is
+ * (which may synchronise the device).  The cited papers have no counterpart: this is
  * an interface convenience, not part of the method.
  *
  * Same arguments, outputs and kernels as hstu_sla_fwd; the work lists and

@@ -9,7 +9,7 @@ key of every sequence, gated by the SLA mask predicate); this module only
 compiles it with gcc and marshals numpy arrays.  ``stu.py`` holds the STU-layer
 oracle (LayerNorm, linear, SiLU, gated norm, truncation) in plain numpy.
 
-Parity pins (tests/test_oracle_pins.py) tie it to the pages: a dense
+Parity pins (tests/test_oracle_pins.py) tie it to the cited definitions: a dense
 brute-force masked attention built from the mask's definition, the full-causal
 special case, the closed-form per-row pair counts, the K1 = 0 and K2 = 0
 cases, the M-FALCON mask figure, finite differences and invariants.

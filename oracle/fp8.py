@@ -5,7 +5,7 @@ INFRASTRUCTURE ONLY (tests and the benchmark's CPU-baseline leg).
 section 4.2.2 (mixed-precision training and inference) and Figure 4: both
 projections of a layer take FP8 operands, everything else stays BF16, and the
 row-wise scale and the quantization of the activations are computed inside
-the LayerNorm that precedes each projection.  The pages fix neither the FP8
+the LayerNorm that precedes each projection.  Those sources fix neither the FP8
 format nor the weights' scaling; the readings taken here:
 
   * the format is E4M3 as the OCP 8-bit floating-point specification defines

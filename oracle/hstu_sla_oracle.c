@@ -23,7 +23,7 @@
  *     themselves, never each other (HSTU notes, section 2.6 and the M-FALCON
  *     mask figure of Q8).
  *
- * Readings taken where the pages are garbled or silent (flags select the
+ * Readings taken where the cited sources are garbled or silent (flags select the
  * alternatives, for tests only):
  *   - Eq. 7's index form is garbled; the window is read as i - j < K1
  *     (K1 tokens including self).  ORACLE_INCLUSIVE_WINDOW selects the
@@ -46,7 +46,7 @@
  * implementation, Fuxi section: difference of the two timestamps, bucketed,
  * looked up, added into the attention scores).  With it
  *   x_ij = alpha q_i.k_j + rab_pos[h][bucket(dpos)] + rab_time[h][bucket(dt)]
- * and everything above uses that x.  Readings (the pages fix none of them):
+ * and everything above uses that x.  Readings (the sources fix none of them):
  *   - dpos = i - j for history rows; a candidate row measures from Lh, the
  *     position its window is applied at (Lh - j), and 0 to itself;
  *   - dt = |ts_i - ts_j| (integer timestamps);

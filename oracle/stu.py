@@ -1,7 +1,7 @@
 """STU-layer and STU-stack oracle -- TEST INFRASTRUCTURE ONLY.
 
 Plain numpy in fp64 (matrix products through numpy's matmul, the attention
-through this package's C loops), step by step as the pages define them; no
+through this package's C loops), step by step as the cited papers define them; no
 fusion, no blocking.  Only the tests and the benchmark's CPU-baseline leg may
 import it; the CUDA library shares nothing with it.
 

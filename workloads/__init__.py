@@ -11,7 +11,7 @@ Systems", section 5.1.1; 16K production sequences, section 1), a contextual
 prefix at the start and candidate targets at the end (section 3, "Input";
 TorchEasyRec "ULTRA HSTU" docs), 4 heads of 128 (TorchEasyRec example config,
 embedding_dim 512 / num_heads 4 / attention_dim 128).  The industrial logs and
-KuaiRand the pages measure on are not available; these draws stand in for
+KuaiRand those papers measure on are not available; these draws stand in for
 them.
 
 Recipe (fixed): lengths from ``numpy.random.default_rng(1000 + index)``;
@@ -75,7 +75,7 @@ HIST16K_TOKEN_BUDGET = 96 * 1024
 # Mixture of Transducers: one transducer per user-signal channel, each with its
 # own sequences and SLA settings ("Bending the Scaling Law Curve...", section
 # 4.3 and appendix A; TorchEasyRec "ULTRA HSTU" docs, MoT: per-channel STU
-# stack and SLA / truncation configuration).  The pages give no channel mix;
+# stack and SLA / truncation configuration).  The sources give no channel mix;
 # this one pairs a long dense channel (16K-class histories, as hist16k), a
 # medium one and a short one with full causal attention.  The three
 # channels' attentions run as one grouped launch.
