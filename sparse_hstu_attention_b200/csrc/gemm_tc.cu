@@ -257,11 +257,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       const TileInfo ti = tile_info(g, t, tiles_m, tiles_n, kBKe);
       if (ti.nkb == 0) continue;
       const uint32_t buf = tc & 1;
+      const int m = ti.m0 + quarter * 32 + lane;
+      const bool live = m < g.M;
+      // residual epilogue: the first chunk's residual row segment is read
+      // before the accumulator wait, each later one a chunk ahead
+      uint4 res_a[4], res_b[4];
+      auto load_res = [&](int i, uint4(&r)[4]) {
+        if (EPI == kEpiBiasResid && live) {
+          const uint4* rp = reinterpret_cast<const uint4*>(g.resid + (int64_t)m * g.ldr + ti.n0 +
+                                                           col0 + 32 * i);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) r[q] = rp[q];
+        }
+      };
+      load_res(0, res_a);
       ok = warp_wait(bar(G_ACC_FULL + buf), (tc >> 1) & 1, g.ws);
       if (!ok) break;
       tc_fence_after();
-      const int m = ti.m0 + quarter * 32 + lane;
-      const bool live = m < g.M;
       if constexpr (EPI == kEpiRedF32) {
 #pragma unroll 1
         for (int c = col0; c < col0 + kBN / 2; c += 32) {
@@ -286,10 +298,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t va[32], vb[32];
         tmem_ld32(lane_base + buf * kBN + col0, va);
         tmem_ld_wait(va);
-        auto chunk = [&](int i, uint32_t(&v)[32], uint32_t(&vn)[32]) {
+        auto chunk = [&](int i, uint32_t(&v)[32], uint32_t(&vn)[32], uint4(&res)[4],
+                         uint4(&res_n)[4]) {
           constexpr int kChunks = kBN / 2 / 32;
           if (i + 1 < kChunks) {
             tmem_ld32(lane_base + buf * kBN + col0 + 32 * (i + 1), vn);
+            load_res(i + 1, res_n);
           } else {  // this warp's share of the accumulator is in registers
             tc_fence_before();
             warp_arrive(bar(G_ACC_EMPTY + buf));
@@ -322,10 +336,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           if (EPI == kEpiBiasResid && live) {
-            const uint4* rp = reinterpret_cast<const uint4*>(g.resid + (int64_t)m * g.ldr + n);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-              const uint4 r4 = rp[q];
+              const uint4 r4 = res[q];
               const uint32_t w[4] = {r4.x, r4.y, r4.z, r4.w};
 #pragma unroll
               for (int h = 0; h < 4; ++h) {
@@ -372,10 +385,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++ec;
           if (i + 1 < kChunks) tmem_ld_wait(vn);
         };
-        chunk(0, va, vb);
-        chunk(1, vb, va);
-        chunk(2, va, vb);
-        chunk(3, vb, va);
+        chunk(0, va, vb, res_a, res_b);
+        chunk(1, vb, va, res_b, res_a);
+        chunk(2, va, vb, res_a, res_b);
+        chunk(3, vb, va, res_b, res_a);
       }
       ++tc;
     }
