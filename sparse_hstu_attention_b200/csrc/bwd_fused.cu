@@ -721,10 +721,11 @@ __global__ void __launch_bounds__(384) silu_qkv_kernel(const AttnArgs a, float s
   dst[1] = make_float4(sum[4], sum[5], sum[6], sum[7]);
 }
 
-// db_{q,k,v}[c] += the blocks' partial sums.  A block owns 32 consecutive
-// columns of the 3 * H * D; its warp w adds the partials of blocks w, w + 8,
-// ... (lane = column, so each read is 128 contiguous bytes), then the eight
-// warps' totals are added.
+// db_{q,k,v}[c] += the blocks' partial sums.  Block (x, y) owns 32
+// consecutive columns of the 3 * H * D and the partials of blocks y, y +
+// gridDim.y, ...; its warp w takes every eighth of those (lane = column, so
+// each read is 128 contiguous bytes), then the eight warps' totals are added
+// and one atomic per column and block row goes out.
 __global__ void __launch_bounds__(256) silu_db_reduce_kernel(const AttnArgs a, int nblk) {
   __shared__ float s_part[8][32];
   const int HD = a.H * D;
@@ -733,7 +734,8 @@ __global__ void __launch_bounds__(256) silu_db_reduce_kernel(const AttnArgs a, i
   const int part = col / HD, c = col - part * HD;
   float v = 0.f;
 #pragma unroll 4
-  for (int b = w; b < nblk; b += 8) v += a.db_part[((int64_t)b * 3 + part) * HD + c];
+  for (int b = blockIdx.y + gridDim.y * w; b < nblk; b += 8 * gridDim.y)
+    v += a.db_part[((int64_t)b * 3 + part) * HD + c];
   s_part[w][lane] = v;
   __syncthreads();
   if (w == 0) {
@@ -812,9 +814,20 @@ cudaError_t launch_bwd_fused_grouped(const GroupSet& gs, cudaStream_t st) {
     if (a.T == 0) continue;
     if (a.pre_q != nullptr) {  // STU layer: SiLU' of Q, K, V and the bias gradient
       const int HD = a.H * D;
-      silu_qkv_kernel<<<kSiluBlocks, 3 * HD / 8, 0, st>>>(a, 0.5f * a.alpha * a.inv_n);
+      // one wave of blocks (as many as fit on every SM), at least ~128 rows
+      // each, at most kSiluBlocks
+      int per_sm = 1;
+      if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, silu_qkv_kernel,
+                                                             3 * HD / 8, 0)) != cudaSuccess)
+        return e;
+      const int64_t wave = (int64_t)sms * (per_sm > 0 ? per_sm : 1);
+      const int64_t want = (a.T + 127) / 128;
+      int64_t nb = want < wave ? want : wave;
+      nb = nb < kSiluBlocks ? nb : kSiluBlocks;
+      const int nblk = (int)(nb > 0 ? nb : 1);
+      silu_qkv_kernel<<<nblk, 3 * HD / 8, 0, st>>>(a, 0.5f * a.alpha * a.inv_n);
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
-      silu_db_reduce_kernel<<<3 * HD / 32, 256, 0, st>>>(a, kSiluBlocks);
+      silu_db_reduce_kernel<<<dim3(3 * HD / 32, 8), 256, 0, st>>>(a, nblk);
     } else {
       dq_convert_kernel<<<sms * 8, 256, 0, st>>>(a.dqacc, a.dq, a.dq_rs, a.T, a.H,
                                                  0.5f * a.alpha * a.inv_n);
