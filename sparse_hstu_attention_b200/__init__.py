@@ -13,6 +13,13 @@ missing, the calls raise.
 q, k, v, dout: CUDA bf16 tensors [T, H, d] whose last two dims are dense
 (row stride free, so views into a fused [T, 4*H*d] projection work);
 seq_offsets: CUDA int32 [B+1]; num_targets: CUDA int32 [B] or None.
+
+Options of the same calls: candidates_only=True (M-FALCON candidate scoring,
+forward); timestamps / rab_pos / rab_time (relative attention bias; the
+backward then also returns the tables' gradients).  Several problems (e.g.
+Mixture-of-Transducers channels) run in one launch through
+hstu_sla_fwd_grouped / hstu_sla_bwd_grouped.  The STU layer, the truncated
+stack and the FP8 projections are in the ``stu`` module.
 """
 from __future__ import annotations
 
