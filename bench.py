@@ -165,9 +165,9 @@ def _sample_cost_flops(p, rows, d, H, row_pairs, key_pairs):
     return H * d * (4.0 * rp + 10.0 * 0.5 * (rp + kp)), rp
 
 
-def _oracle_sample(batch, n_tokens, seed):
+def _oracle_sample(batch, n_tokens, seed, rab=None):
     import oracle
-    p = oracle.Problem.from_batch(batch)
+    p = oracle.Problem.from_batch(batch, **(rab or {}))
     rng = np.random.default_rng(seed)
     rows = np.sort(rng.choice(batch.T, size=min(n_tokens, batch.T), replace=False))
     t0 = time.perf_counter()
@@ -182,8 +182,9 @@ def _pair_tables(batch):
     return F.pairs_per_token(batch.lengths, batch.num_targets, w.contextual_len, w.K1, w.K2)
 
 
-def cpu_baseline(batch, target_s=15.0):
-    """The oracle, as it stands, on a bounded random sample of the workload's tokens."""
+def cpu_baseline(batch, target_s=15.0, rab=None):
+    """The oracle, as it stands, on a bounded random sample of the workload's
+    tokens (rab: the oracle's relative-attention-bias arguments, or None)."""
     w = batch.workload
     rp, kp = _pair_tables(batch)
     # The oracle runs its loops on all host cores, so a small sample costs
@@ -191,18 +192,20 @@ def cpu_baseline(batch, target_s=15.0):
     # run takes a second or more, then scale it to the target time.
     n, t = 64, 0.0
     while n < batch.T:
-        t, _ = _oracle_sample(batch, n, seed=7)
+        t, _ = _oracle_sample(batch, n, seed=7, rab=rab)
         if t >= 1.0:
             break
         n = min(batch.T, n * 4)
     n = int(min(batch.T, max(64, n * target_s / max(t, 1e-3))))
-    t, rows = _oracle_sample(batch, n, seed=8)
+    t, rows = _oracle_sample(batch, n, seed=8, rab=rab)
     fl, _ = _sample_cost_flops(None, rows, w.d, w.H, rp, kp)
     cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
     cores = int(os.environ.get("OMP_NUM_THREADS", cores))
     return {"value": fl / t / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
             "sample": f"{len(rows)} random tokens of the {w.name} batch: forward and dq for them "
-                      f"as rows, dk/dv for them as keys; fp64 C loops; {t:.1f} s",
+                      f"as rows, dk/dv for them as keys"
+                      f"{' (with the relative attention bias)' if rab else ''}; fp64 C loops; "
+                      f"{t:.1f} s",
             "seconds": t}
 
 
@@ -252,6 +255,35 @@ def _config(w, batch):
             "num_targets": w.num_targets, "N": w.N, "alpha": w.alpha,
             "lengths": [int(x) for x in batch.lengths], "pairs_per_head": pairs,
             "l2": f"inputs {in_bytes / 1e6:.0f} MB > 126 MB L2; no flush"}
+
+
+def stu_cpu_baseline(w, lengths, nts, dr, cfg_full, fp8=False):
+    """The STU oracle, as it stands (fp64 numpy around the C attention), on a
+    bounded sample: layer 1 forward and backward over the batch's shortest
+    sequence; FLOPs counted as the GPU line counts them."""
+    from oracle import stu as S
+    b = int(np.argmin(lengths))
+    offs = np.concatenate([[0], np.cumsum(lengths)])
+    s0, s1 = int(offs[b]), int(offs[b + 1])
+    L, dm = s1 - s0, cfg_full.d_model
+    wo = S.Weights.of(**{k: dr.layers[0][k].float().numpy() for k in
+                         ("ln1_w", "ln1_b", "w1", "b1", "ln2_w", "ln2_b", "w2", "b2")})
+    cfg = S.AttnCfg(cfg_full.H, cfg_full.d, cfg_full.contextual_len, cfg_full.K1, cfg_full.K2,
+                    cfg_full.alpha, cfg_full.N, cfg_full.ln_eps)
+    x = dr.x[s0:s1].float().numpy().astype(np.float64)
+    g = np.random.default_rng(0).standard_normal((L, dm))
+    t0 = time.perf_counter()
+    _, cache = S.layer_fwd(x, wo, np.array([0, L]), nts[b:b + 1], cfg, fp8=fp8)
+    S.layer_bwd(g, wo, cache)
+    t = time.perf_counter() - t0
+    pairs = F.total_pairs(np.array([L]), nts[b:b + 1], w.contextual_len, w.K1, w.K2)
+    fl = 3 * 2 * dm * 5 * dm * L + F.fwd_flops(pairs, w.H, w.d) + F.bwd_flops(pairs, w.H, w.d)
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    cores = int(os.environ.get("OMP_NUM_THREADS", cores))
+    return {"value": fl / t / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"layer 1 forward and backward on the shortest sequence ({L} tokens)"
+                      f"{', E4M3 forward projections' if fp8 else ''}; fp64; {t:.1f} s",
+            "seconds": t}
 
 
 def run_stu(args, world, rank, local):
@@ -334,7 +366,10 @@ def run_stu(args, world, rank, local):
             "flops_per_step": {"projections": gemm, "attention": attn},
             "frac_of_sustained_peak": value / world / peak,
             "gpu_launches": K * (STU_LAYERS * (6 + 11 + (2 if args.fp8 else 0)) + 3),
-            "clocks": clocks.summary()}), flush=True)
+            "clocks": clocks.summary(),
+            **({} if (world > 1 or args.no_cpu_baseline) else
+               {"cpu_baseline": stu_cpu_baseline(w, lengths, nts, dr, full, args.fp8)})}),
+            flush=True)
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
@@ -631,8 +666,13 @@ def main():
             "candidate_pairs_per_head": cp,
             "tflops": F.fwd_flops(cp, H, d) / (c_ms * 1e-3) / 1e12,
             "speedup_vs_full_forward": ms_step / c_ms}
-    if world == 1 and not args.no_cpu_baseline and not args.rab:
-        line["cpu_baseline"] = cpu_baseline(batch)
+    if world == 1 and not args.no_cpu_baseline:
+        rab_o = None
+        if args.rab:  # the same tables and timestamps, in the oracle's types
+            rab_o = dict(timestamps=kw["timestamps"].cpu().numpy().astype(np.int64),
+                         rab_pos=kw["rab_pos"].cpu().numpy().astype(np.float64),
+                         rab_time=kw["rab_time"].cpu().numpy().astype(np.float64))
+        line["cpu_baseline"] = cpu_baseline(batch, rab=rab_o)
     print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.barrier()
