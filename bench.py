@@ -257,32 +257,41 @@ def _config(w, batch):
             "l2": f"inputs {in_bytes / 1e6:.0f} MB > 126 MB L2; no flush"}
 
 
-def stu_cpu_baseline(w, lengths, nts, dr, cfg_full, fp8=False):
+def stu_cpu_baseline(w, lengths, nts, dr, cfg_full, fp8=False, budget_s=10.0):
     """The STU oracle, as it stands (fp64 numpy around the C attention), on a
-    bounded sample: layer 1 forward and backward over the batch's shortest
-    sequence; FLOPs counted as the GPU line counts them."""
+    bounded sample: layer 1 forward and backward, one sequence at a time from
+    the shortest up, until about budget_s seconds of CPU work are done; FLOPs
+    counted as the GPU line counts them."""
     from oracle import stu as S
-    b = int(np.argmin(lengths))
     offs = np.concatenate([[0], np.cumsum(lengths)])
-    s0, s1 = int(offs[b]), int(offs[b + 1])
-    L, dm = s1 - s0, cfg_full.d_model
+    dm = cfg_full.d_model
     wo = S.Weights.of(**{k: dr.layers[0][k].float().numpy() for k in
                          ("ln1_w", "ln1_b", "w1", "b1", "ln2_w", "ln2_b", "w2", "b2")})
     cfg = S.AttnCfg(cfg_full.H, cfg_full.d, cfg_full.contextual_len, cfg_full.K1, cfg_full.K2,
                     cfg_full.alpha, cfg_full.N, cfg_full.ln_eps)
-    x = dr.x[s0:s1].float().numpy().astype(np.float64)
-    g = np.random.default_rng(0).standard_normal((L, dm))
-    t0 = time.perf_counter()
-    _, cache = S.layer_fwd(x, wo, np.array([0, L]), nts[b:b + 1], cfg, fp8=fp8)
-    S.layer_bwd(g, wo, cache)
-    t = time.perf_counter() - t0
-    pairs = F.total_pairs(np.array([L]), nts[b:b + 1], w.contextual_len, w.K1, w.K2)
-    fl = 3 * 2 * dm * 5 * dm * L + F.fwd_flops(pairs, w.H, w.d) + F.bwd_flops(pairs, w.H, w.d)
+    rng = np.random.default_rng(0)
+    t, fl, toks, nseq = 0.0, 0.0, 0, 0
+    for b in np.argsort(lengths, kind="stable"):
+        s0, s1 = int(offs[b]), int(offs[b + 1])
+        L = s1 - s0
+        x = dr.x[s0:s1].float().numpy().astype(np.float64)
+        g = rng.standard_normal((L, dm))
+        t0 = time.perf_counter()
+        _, cache = S.layer_fwd(x, wo, np.array([0, L]), nts[b:b + 1], cfg, fp8=fp8)
+        S.layer_bwd(g, wo, cache)
+        t += time.perf_counter() - t0
+        pairs = F.total_pairs(np.array([L]), nts[b:b + 1], w.contextual_len, w.K1, w.K2)
+        fl += 3 * 2 * dm * 5 * dm * L + F.fwd_flops(pairs, w.H, w.d) + \
+            F.bwd_flops(pairs, w.H, w.d)
+        toks, nseq = toks + L, nseq + 1
+        if t >= budget_s:
+            break
     cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
     cores = int(os.environ.get("OMP_NUM_THREADS", cores))
     return {"value": fl / t / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-            "sample": f"layer 1 forward and backward on the shortest sequence ({L} tokens)"
-                      f"{', E4M3 forward projections' if fp8 else ''}; fp64; {t:.1f} s",
+            "sample": f"layer 1 forward and backward on the {nseq} shortest sequences "
+                      f"({toks} tokens){', E4M3 forward projections' if fp8 else ''}; "
+                      f"fp64; {t:.1f} s",
             "seconds": t}
 
 
