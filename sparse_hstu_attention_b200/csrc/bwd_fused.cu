@@ -40,6 +40,7 @@
 // Shared memory (227 KB): K 2 x 32 KB, V 32 KB, Q and dO 3 x 16 KB each, dS^T
 // 2 x 16 KB (the B operand of the dQ MMA), barriers and the unit ring.
 #include <cudaTypedefs.h>
+#include <type_traits>
 
 #include "sm100.cuh"
 
@@ -148,9 +149,16 @@ __device__ __forceinline__ void warp_flush_bins(float* hst, int bin, float sum, 
 __device__ __forceinline__ void red_add_f32(float* p, uint32_t v) { atomicAdd(p, __uint_as_float(v)); }
 
 // RAB: the relative attention bias is added to every recomputed score and
-// its gradient is accumulated per unit in a shared-memory histogram (each
-// thread adds runs of equal buckets along its query columns; one pointwise
-// warp flushes the unit's sums into this head's table gradients).
+// its gradient is accumulated per unit in a shared-memory histogram.  Each
+// thread keeps runs of equal buckets along its key's query columns: in a
+// 16-column round where every lane's buckets span at most two neighbouring
+// values (the position bucket only grows along the columns; the time bucket
+// is bounded by the round's earliest and latest query) a score adds its
+// gradient to two or three register totals; finished runs wait in one slot
+// per table and are added into the histogram once per step, lanes with
+// equal buckets summed by shuffles first (same-address shared atomics from
+// many lanes were the cost).  One pointwise warp flushes the unit's sums
+// into this head's table gradients.
 template <bool RAB>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_kvq_kernel(const __grid_constant__ BwdMaps maps, const __grid_constant__ GroupSet gs) {
@@ -460,28 +468,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       float* dqa = A.dqacc + ((int64_t)h * A.T + s0) * D + row;
       // relative attention bias: this head's tables, this key's timestamp and
       // the unit's histogram buffer (free once the unit two back was flushed)
-      float tabp = 0.f, tabt = 0.f;  // bucket `lane` of this head's tables
+      float tabp = 0.f, tabt = 0.f;  // half of bucket min(lane, nb - 1)
       int32_t tj = 0;
       float* hst = hist + (hu & 1) * kHistBins;
       if constexpr (RAB) {
-        if (A.rab_pos && lane < A.nbp) tabp = __ldg(A.rab_pos + h * A.nbp + lane);
-        if (A.rab_time && lane < A.nbt) tabt = __ldg(A.rab_time + h * A.nbt + lane);
+        tabp = rab_lane_table(A.rab_pos, A.nbp, h, lane);
+        tabt = rab_lane_table(A.rab_time, A.nbt, h, lane);
         tj = (A.ts && rr < L) ? __ldg(A.ts + s0 + rr) : 0;
         ok = warp_wait(bar(F_H_ZERO + (hu & 1)), ((hu >> 1) & 1) ^ 1, ws);
         if (!ok) break;
       }
       // runs of equal buckets (position, time) along this key's query
-      // columns, which only grow through the unit's steps
+      // columns, which only grow through the unit's steps.  Bins hold the
+      // buckets before the tables' clamp (0..31 each); the flush folds bins
+      // past a table's last bucket into it.
       int run_p = -1, run_t = -1;
       float sum_p = 0.f, sum_t = 0.f;
-      auto run_add = [&](int& run, float& sum, int bin, float g) {
-        if (bin != run) {
-          if (run >= 0) atomicAdd(hst + run, sum);
-          run = bin;
-          sum = g;
-        } else {
-          sum += g;
+      // a finished run waits in one pending slot per table until the end of
+      // the step, when the warp adds the slots up bin by bin; a second one in
+      // the same step goes straight into the histogram
+      int pend_p = -1, pend_t = -1;
+      float psum_p = 0.f, psum_t = 0.f;
+      auto run_add = [&](int& run, float& sum, int& pend, float& psum, int bin, float g) {
+        const bool c = bin != run;
+        if (c && pend >= 0) {  // a second finished run in this step
+          atomicAdd(hst + run, sum);
+          sum = 0.f;
+          run = -1;
         }
+        const bool mv = c && run >= 0;
+        pend = mv ? run : pend;
+        psum = mv ? sum : psum;
+        sum = c ? g : sum + g;
+        run = bin;
       };
       SpanCursor c;
       c.begin(r);
@@ -501,9 +520,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t bits = full ? 0xFFFFFFFFu : key_mask_bits(km, c0 + col);
         // relative attention bias: the 32 queries' timestamps (one per lane)
         int32_t tql = 0;
+        bool tq_ok = false;  // this lane's query column is in the sequence
         if constexpr (RAB) {
           const int ql = c0 + col + lane;
-          tql = (A.ts && ql < L) ? __ldg(A.ts + s0 + ql) : 0;
+          tq_ok = ql < L;
+          tql = (A.ts && tq_ok) ? __ldg(A.ts + s0 + ql) : 0;
         }
         // Two rounds of 16 query columns each (fewer live registers).  Round r
         // writes P^T (8 packed columns) then dS^T (8) over the 16 score
@@ -516,28 +537,87 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld16(xd_addr + 16 * r, xd);
           tmem_ld_wait2(xs, xd);
           if constexpr (RAB) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const int k = 16 * r + 2 * e;  // column within this half
-              const int32_t tqa = __shfl_sync(0xffffffffu, tql, k);
-              const int32_t tqb = __shfl_sync(0xffffffffu, tql, k + 1);
-              int bpa, bta, bpb, btb;
-              rab_buckets(A.nbp, A.nbt, c0 + col + k, rr, Lh, tqa, tj, bpa, bta);
-              rab_buckets(A.nbp, A.nbt, c0 + col + k + 1, rr, Lh, tqb, tj, bpb, btb);
-              const float ba = rab_bias(tabp, tabt, bpa, bta);
-              const float bb = rab_bias(tabp, tabt, bpb, btb);
-              float ga, gb;
-              bwd_pair_bias(xs[2 * e], xs[2 * e + 1], xd[2 * e], xd[2 * e + 1], half_alpha2, ba, bb,
-                            pp[e], dd[e], ga, gb);
-              if ((bits >> k) & 1u) {
-                run_add(run_p, sum_p, bpa, ga);
-                run_add(run_t, sum_t, 32 + bta, ga);
-              }
-              if ((bits >> (k + 1)) & 1u) {
-                run_add(run_p, sum_p, bpb, gb);
-                run_add(run_t, sum_t, 32 + btb, gb);
-              }
+            // Bounds of the round's buckets for this key: the position bucket
+            // only grows along the columns (first and last column), the time
+            // difference lies between those to the round's earliest and latest
+            // query.  When every lane's buckets take at most two neighbouring
+            // values, each score only adds its gradient to the round's total
+            // and to the upper buckets' totals; else each score extends its
+            // runs one by one.
+            const int b0p = rab_log_bucket(rab_pos_u(__viaddmin_s32(c0 + col, 16 * r, Lh), 1 - rr));
+            const int b1p =
+                rab_log_bucket(rab_pos_u(__viaddmin_s32(c0 + col, 16 * r + 15, Lh), 1 - rr));
+            const bool in_round = tq_ok && (lane >> 4) == r;
+            const int32_t tmin = __reduce_min_sync(0xffffffffu, in_round ? tql : INT32_MAX);
+            const int32_t tmax = __reduce_max_sync(0xffffffffu, in_round ? tql : INT32_MIN);
+            uint32_t dlo, dhi;
+            if (tj <= tmin) {
+              dlo = (uint32_t)tmin - (uint32_t)tj;
+              dhi = (uint32_t)tmax - (uint32_t)tj;
+            } else if (tj >= tmax) {
+              dlo = (uint32_t)tj - (uint32_t)tmax;
+              dhi = (uint32_t)tj - (uint32_t)tmin;
+            } else {
+              dlo = 0u;
+              dhi = max((uint32_t)tmax - (uint32_t)tj, (uint32_t)tj - (uint32_t)tmin);
             }
+            const int b0t = rab_log_bucket(dlo + 1u) & 31;
+            const int b1t = rab_log_bucket(dhi + 1u) & 31;
+            const bool two = (uint32_t)(b1p - b0p) <= 1u && (uint32_t)(b1t - b0t) <= 1u;
+            auto rab_round = [&](auto all_c, auto two_c) {
+              constexpr bool kAll = decltype(all_c)::value;
+              constexpr bool kTwo = decltype(two_c)::value;
+              float acc = 0.f, ahp = 0.f, aht = 0.f;  // round total, upper buckets
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const int k = 16 * r + 2 * e;
+                const int bpa = rab_log_bucket(rab_pos_u(__viaddmin_s32(c0 + col, k, Lh), 1 - rr));
+                const int bpb =
+                    rab_log_bucket(rab_pos_u(__viaddmin_s32(c0 + col, k + 1, Lh), 1 - rr));
+                const int bta =
+                    rab_log_bucket(rab_time_u(__shfl_sync(0xffffffffu, tql, k), tj)) & 31;
+                const int btb =
+                    rab_log_bucket(rab_time_u(__shfl_sync(0xffffffffu, tql, k + 1), tj)) & 31;
+                const float ba = rab_half_bias(tabp, tabt, bpa, bta);
+                const float bb = rab_half_bias(tabp, tabt, bpb, btb);
+                float ga, gb;
+                bwd_pair_bias(xs[2 * e], xs[2 * e + 1], xd[2 * e], xd[2 * e + 1], half_alpha2, ba,
+                              bb, pp[e], dd[e], ga, gb);
+                if constexpr (kTwo) {
+                  if (!kAll && !((bits >> k) & 1u)) ga = 0.f;
+                  if (!kAll && !((bits >> (k + 1)) & 1u)) gb = 0.f;
+                  acc += ga;
+                  ahp += bpa != b0p ? ga : 0.f;
+                  aht += bta != b0t ? ga : 0.f;
+                  acc += gb;
+                  ahp += bpb != b0p ? gb : 0.f;
+                  aht += btb != b0t ? gb : 0.f;
+                } else {
+                  if (kAll || ((bits >> k) & 1u)) {
+                    run_add(run_p, sum_p, pend_p, psum_p, bpa, ga);
+                    run_add(run_t, sum_t, pend_t, psum_t, 32 + bta, ga);
+                  }
+                  if (kAll || ((bits >> (k + 1)) & 1u)) {
+                    run_add(run_p, sum_p, pend_p, psum_p, bpb, gb);
+                    run_add(run_t, sum_t, pend_t, psum_t, 32 + btb, gb);
+                  }
+                }
+              }
+              if constexpr (kTwo) {
+                // lower then upper bucket (an exact zero adds nothing)
+                const float lop = acc - ahp, lot = acc - aht;
+                if (lop != 0.f) run_add(run_p, sum_p, pend_p, psum_p, b0p, lop);
+                if (ahp != 0.f) run_add(run_p, sum_p, pend_p, psum_p, b0p + 1, ahp);
+                if (lot != 0.f) run_add(run_t, sum_t, pend_t, psum_t, 32 + b0t, lot);
+                if (aht != 0.f) run_add(run_t, sum_t, pend_t, psum_t, 33 + b0t, aht);
+              }
+            };
+            if (!__all_sync(0xffffffffu, two))
+              rab_round(std::false_type{}, std::false_type{});
+            else if (full)
+              rab_round(std::true_type{}, std::true_type{});
+            else
+              rab_round(std::false_type{}, std::true_type{});
           } else {
 #pragma unroll
             for (int e = 0; e < 8; ++e)
@@ -557,6 +637,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int q = 0; q < 2; ++q)
             st_shared_v4(dsr + ((((uint32_t)(half * 4 + 2 * r + q)) ^ swz) << 4), dd[4 * q],
                          dd[4 * q + 1], dd[4 * q + 2], dd[4 * q + 3]);
+        }
+        if constexpr (RAB) {  // the step's finished runs, equal bins added up first
+          if (__any_sync(0xffffffffu, (pend_p >= 0) | (pend_t >= 0))) {
+            warp_flush_bins(hst, pend_p, psum_p, lane);
+            warp_flush_bins(hst, pend_t, psum_t, lane);
+            pend_p = pend_t = -1;
+          }
         }
         fence_proxy_async_smem();  // visible to the dQ MMA
         tmem_st_wait();
@@ -635,10 +722,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float sc = 0.5f * A.inv_n;
           for (int bin = lane; bin < kHistBins; bin += 32) {
             const float v = hst[bin];
-            if (bin < 32) {
-              if (bin < A.nbp && A.d_rab_pos) atomicAdd(A.d_rab_pos + h * A.nbp + bin, v * sc);
-            } else if (bin - 32 < A.nbt && A.d_rab_time) {
-              atomicAdd(A.d_rab_time + h * A.nbt + (bin - 32), v * sc);
+            if (v != 0.f) {
+              if (bin < 32) {
+                if (A.d_rab_pos) atomicAdd(A.d_rab_pos + h * A.nbp + imin(bin, A.nbp - 1), v * sc);
+              } else if (A.d_rab_time) {
+                atomicAdd(A.d_rab_time + h * A.nbt + imin(bin - 32, A.nbt - 1), v * sc);
+              }
             }
             hst[bin] = 0.f;
           }

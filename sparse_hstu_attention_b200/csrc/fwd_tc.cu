@@ -568,13 +568,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int K1 = A.K1, K2e = A.K2e;
       const uint64_t half_alpha2 = f2s(0.5f * A.alpha);
       const RowMask m = row_mask(i, r->L, Lh, K1, K2e);
-      // relative attention bias: bucket `lane` of this head's tables in
-      // this lane, and this row's timestamp
+      // relative attention bias: half of this head's tables' bucket
+      // min(lane, nb - 1) in this lane, and this row's timestamp
       float tabp = 0.f, tabt = 0.f;
       int32_t ti = 0;
       if constexpr (RAB) {
-        if (A.rab_pos && lane < A.nbp) tabp = __ldg(A.rab_pos + h * A.nbp + lane);
-        if (A.rab_time && lane < A.nbt) tabt = __ldg(A.rab_time + h * A.nbt + lane);
+        tabp = rab_lane_table(A.rab_pos, A.nbp, h, lane);
+        tabt = rab_lane_table(A.rab_time, A.nbt, h, lane);
         ti = (A.ts && i < r->L) ? __ldg(A.ts + s0 + i) : 0;
       }
       SpanCursor c;
@@ -600,19 +600,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld_wait2(c0, c1);
           uint32_t p[16];
           if constexpr (RAB) {
-            // the 32 keys' timestamps, one per lane, then each score's bias
+            // the 32 keys' timestamps, one per lane, then each score's bias:
+            // key j = j0 + col + k has u_pos = max(pb - k, 1)
             const int jl = j0 + col + lane;
             const int32_t tjl = (A.ts && jl < r->L) ? __ldg(A.ts + s0 + jl) : 0;
+            const int pb = imin(i, Lh) + 1 - (j0 + col);
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
-              const int ja = j0 + col + 2 * e, jb = ja + 1;
-              int bpa, bta, bpb, btb;
-              rab_buckets(A.nbp, A.nbt, i, ja, Lh, ti, __shfl_sync(0xffffffffu, tjl, 2 * e), bpa,
-                          bta);
-              rab_buckets(A.nbp, A.nbt, i, jb, Lh, ti, __shfl_sync(0xffffffffu, tjl, 2 * e + 1),
-                          bpb, btb);
-              const float ba = rab_bias(tabp, tabt, bpa, bta);
-              const float bb = rab_bias(tabp, tabt, bpb, btb);
+              const float ba = rab_half_bias(
+                  tabp, tabt, rab_log_bucket(rab_pos_u(pb, -2 * e)),
+                  rab_log_bucket(rab_time_u(ti, __shfl_sync(0xffffffffu, tjl, 2 * e))));
+              const float bb = rab_half_bias(
+                  tabp, tabt, rab_log_bucket(rab_pos_u(pb, -2 * e - 1)),
+                  rab_log_bucket(rab_time_u(ti, __shfl_sync(0xffffffffu, tjl, 2 * e + 1))));
               p[e] = silu_pair_bias(e < 8 ? c0[2 * e] : c1[2 * e - 16],
                                     e < 8 ? c0[2 * e + 1] : c1[2 * e - 15], half_alpha2, ba, bb);
             }

@@ -121,33 +121,39 @@ struct AttnArgs {
   float* d_rab_time;
 };
 
-// floor(log2(n + 1)) for n >= 0, at most nb - 1.
-__host__ __device__ __forceinline__ int rab_bucket(uint32_t n, int nb) {
-#ifdef __CUDA_ARCH__
-  const int b = 31 - __clz(n + 1u);
-#else
-  int b = 0;
-  for (uint32_t x = n + 1u; x > 1u; x >>= 1) ++b;
-#endif
-  return b < nb - 1 ? b : nb - 1;
+// Relative attention bias, with the tables held in registers: lane b of a
+// warp holds half of bucket min(b, nb - 1) of this head's table (0 without
+// one), so a bucket index needs no clamp to nb - 1 and the value goes
+// straight into x / 2 = (alpha s + bias) / 2.  Every lane must take part.
+__device__ __forceinline__ float rab_lane_table(const float* tab, int nb, int h, int lane) {
+  return tab ? 0.5f * __ldg(tab + h * nb + (lane < nb ? lane : nb - 1)) : 0.f;
 }
 
-// Buckets of the pair (query i, key j) in a sequence with Lh history rows
-// (ti, tj the timestamps): the position difference measures a candidate row
-// from Lh (0 to itself); the time difference is exact for any two int32
-// values (unsigned) and capped at 2^31 - 1 (bucket 31).
-__device__ __forceinline__ void rab_buckets(int nbp, int nbt, int i, int j, int Lh, int32_t ti,
-                                            int32_t tj, int& bp, int& bt) {
-  const int dpos = i < Lh ? i - j : (j == i ? 0 : Lh - j);
-  bp = rab_bucket((uint32_t)(dpos > 0 ? dpos : 0), nbp);
-  const uint32_t adt = ti >= tj ? (uint32_t)ti - (uint32_t)tj : (uint32_t)tj - (uint32_t)ti;
-  bt = rab_bucket(adt < 0x7FFFFFFFu ? adt : 0x7FFFFFFFu, nbt);
+// The log bucket floor(log2(n + 1)) of a difference n >= 0, from u = n + 1
+// modulo 2^32: the index of u's top bit, and -1 for u = 0 (n = 2^32 - 1).
+// As a shuffle lane (low 5 bits) or after `& 31`, every n >= 2^31 - 1 lands
+// in bucket 31, so the result equals the bucket of n capped at 2^31 - 1.
+__device__ __forceinline__ int rab_log_bucket(uint32_t u) { return 31 - __clz(u); }
+
+// u = |ti - tj| + 1 for two int32 timestamps: the exact difference as an
+// unsigned 32-bit value.
+__device__ __forceinline__ uint32_t rab_time_u(int32_t ti, int32_t tj) {
+  return __sad(ti, tj, 1u);
 }
 
-// The bias of a pair when lane b of the warp holds bucket b of this head's
-// position table (tabp) and time table (tabt), 0 beyond a table or without
-// one: two shuffles instead of two memory loads.  Every lane must call it.
-__device__ __forceinline__ float rab_bias(float tabp, float tabt, int bp, int bt) {
+// u = dpos + 1 of the pair (query i, key j) in a sequence with Lh history
+// rows, where dpos = i - j for a history row and Lh - j for a candidate row
+// (0 to itself), clamped below at 0.  Every visible pair has dpos >= 0, so
+// one form serves both kinds of row: u = max(min(i, Lh) - j + 1, 1), which
+// also gives a candidate's self pair dpos = 0 (invisible pairs' buckets are
+// never used).  Callers split min(i, Lh) + 1 - j into a + b, one of them
+// constant along their loop, for one fused add-max per pair.
+__device__ __forceinline__ uint32_t rab_pos_u(int a, int b) {
+  return (uint32_t)__viaddmax_s32(a, b, 1);
+}
+
+// Half the bias of a pair from its two buckets (shuffle lanes).
+__device__ __forceinline__ float rab_half_bias(float tabp, float tabt, int bp, int bt) {
   return __shfl_sync(0xffffffffu, tabp, bp) + __shfl_sync(0xffffffffu, tabt, bt);
 }
 

@@ -391,21 +391,21 @@ __device__ __forceinline__ uint32_t silu_pair(uint32_t s0, uint32_t s1, uint64_t
   return f2_bf16(f2_fma(h, f2_tanh(h), h));
 }
 
-// silu_pair with an additive bias per score: SiLU(alpha s + b).
+// silu_pair with an additive bias per score, given as half biases
+// hb = b / 2: SiLU(alpha s + b), h = alpha s / 2 + hb.
 __device__ __forceinline__ uint32_t silu_pair_bias(uint32_t s0, uint32_t s1, uint64_t half_alpha2,
-                                                   float b0, float b1) {
-  const uint64_t h = f2_fma(f2(s0, s1), half_alpha2,
-                            f2(__float_as_uint(0.5f * b0), __float_as_uint(0.5f * b1)));
+                                                   float hb0, float hb1) {
+  const uint64_t h = f2_fma(f2(s0, s1), half_alpha2, f2(__float_as_uint(hb0), __float_as_uint(hb1)));
   return f2_bf16(f2_fma(h, f2_tanh(h), h));
 }
 
-// bwd_pair with an additive bias per score (x = alpha s + b), also returning
-// the fp32 dS2 pair (for the bias gradient).
+// bwd_pair with an additive bias per score (x = alpha s + b, given as half
+// biases hb = b / 2), also returning the fp32 dS2 pair (for the bias
+// gradient).
 __device__ __forceinline__ void bwd_pair_bias(uint32_t s0, uint32_t s1, uint32_t d0, uint32_t d1,
-                                              uint64_t half_alpha2, float b0, float b1,
+                                              uint64_t half_alpha2, float hb0, float hb1,
                                               uint32_t& p2, uint32_t& ds2, float& g0, float& g1) {
-  const uint64_t h = f2_fma(f2(s0, s1), half_alpha2,
-                            f2(__float_as_uint(0.5f * b0), __float_as_uint(0.5f * b1)));
+  const uint64_t h = f2_fma(f2(s0, s1), half_alpha2, f2(__float_as_uint(hb0), __float_as_uint(hb1)));
   const uint64_t u = f2_add(f2_tanh(h), f2s(1.f));
   const uint64_t p = f2_mul(h, u);
   const uint64_t w = f2_fma(p, f2s(-1.f), f2_fma(h, f2s(2.f), f2s(1.f)));  // 1 + 2h - P

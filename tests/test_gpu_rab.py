@@ -85,6 +85,32 @@ def test_rab_edge_batch():
     assert_close("d rab_time", drt, rdt)
 
 
+def test_rab_timestamps_over_the_whole_int32_range():
+    """Unsorted timestamps drawn over all of int32 (both ends included) next
+    to small ones: differences up to 2^32 - 1, the cap at 2^31 - 1 and every
+    time bucket up to 31 of a 32-bucket table, plus a 5-bucket position
+    table (most pairs past its last bucket)."""
+    b, _, _, _ = _case(lengths=(190, 333, 64, 9), seed=13)
+    rng = np.random.default_rng(13)
+    T = int(b.seq_offsets[-1])
+    wide = rng.integers(-2 ** 31, 2 ** 31, size=T, dtype=np.int64)
+    small = rng.integers(-5000, 5000, size=T, dtype=np.int64)
+    ts = np.where(rng.random(T) < 0.5, wide, small)
+    ts[:6] = [-2 ** 31, 2 ** 31 - 1, 0, -1, 2 ** 31 - 2, -2 ** 31 + 1]
+    ts = ts.astype(np.int32)
+    rp, rt = draw_rab_tables(b.workload.H, 5, 32, 13)
+    out, dq, dk, dv, (drp, drt) = _run(b, ts, rp, rt)
+    p = _oracle(b, ts, rp, rt)
+    assert_close("out", out, p.fwd(b.q, b.k, b.v))
+    rq, rk, rv = p.bwd(b.q, b.k, b.v, b.dout)
+    for name, got, ref in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
+        assert_close(name, got, ref)
+    rdp, rdt = p.bwd_rab(b.q, b.k, b.v, b.dout)
+    assert_close("d rab_pos", drp, rdp)
+    assert_close("d rab_time", drt, rdt)
+    assert (np.abs(rdt[:, 30:]) > 0).all()  # the top buckets were reached
+
+
 def test_zero_tables_equal_the_bias_free_kernels():
     b, ts, rp, rt = _case(seed=8)
     out, dq, dk, dv, _ = _run(b, ts, torch.zeros_like(rp), torch.zeros_like(rt))
