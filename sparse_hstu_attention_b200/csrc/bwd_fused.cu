@@ -73,10 +73,13 @@ constexpr int OFF_BAR = OFF_DS + 2 * DSTILE;
 constexpr int OFF_UNIT = OFF_BAR + 512;
 constexpr int OFF_SLOT = OFF_UNIT + kUSlots * (int)sizeof(UnitRec);
 // relative attention bias: per-unit histograms of the bias gradient, two
-// (alternating units), 32 position then 32 time buckets each
+// (alternating units), each in two copies (warps of even and odd index add
+// into separate copies, halving same-address atomics), 32 position then 32
+// time buckets each
 constexpr int kHistBins = 64;
 constexpr int OFF_HIST = OFF_SLOT + 16;
-constexpr int SMEM = OFF_HIST + 2 * kHistBins * 4 + 1024;
+constexpr int kHistCopies = 2;
+constexpr int SMEM = OFF_HIST + 2 * kHistCopies * kHistBins * 4 + 1024;
 static_assert(SMEM <= 232448, "shared memory budget");
 constexpr uint32_t SBO = 8 * SW;
 // 128 x 64 scores, both operands K-major
@@ -128,20 +131,28 @@ struct BwdMaps {
   CUtensorMap k[kMaxGroups], v[kMaxGroups], q[kMaxGroups], dout[kMaxGroups];
 };
 
-// Adds each lane's (bin, sum) into the shared histogram, lanes of equal bins
-// first summed with shuffles (one shared atomic per distinct bin instead of
-// up to 32 on one address).  bin < 0: nothing.  Called by the whole warp.
-__device__ __forceinline__ void warp_flush_bins(float* hst, int bin, float sum, int lane) {
-  uint32_t todo = __ballot_sync(0xffffffffu, bin >= 0);
-  while (todo) {
-    const int b = __shfl_sync(0xffffffffu, bin, __ffs(todo) - 1);
-    const bool mine = bin == b;
-    float v = mine ? sum : 0.f;
+// Adds two (bin, value) pairs per lane (one per table; bin < 0: nothing)
+// into the shared histogram: a segmented sum over runs of consecutive lanes
+// with equal bins (five shuffle steps for every run at once), then one
+// shared atomic from each run's last lane.  Equal bins in separate runs
+// stay correct (one atomic per run).  Called by the whole warp.
+__device__ __forceinline__ void warp_flush_runs(float* hst, int bp, float vp, int bt, float vt,
+                                                int lane) {
+  const uint32_t full = 0xffffffffu;
+  const int bp_prev = __shfl_up_sync(full, bp, 1), bt_prev = __shfl_up_sync(full, bt, 1);
+  const int bp_next = __shfl_down_sync(full, bp, 1), bt_next = __shfl_down_sync(full, bt, 1);
+  const uint32_t below = (2u << lane) - 1u;  // lanes 0..lane
+  const uint32_t hp = __ballot_sync(full, lane == 0 || bp != bp_prev) & below;
+  const uint32_t ht = __ballot_sync(full, lane == 0 || bt != bt_prev) & below;
+  const int sp = 31 - __clz(hp), st = 31 - __clz(ht);  // first lane of my run
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (lane == __ffs(todo) - 1) atomicAdd(hst + b, v);
-    todo &= ~__ballot_sync(0xffffffffu, mine);
+  for (int o = 1; o < 32; o <<= 1) {
+    const float up = __shfl_up_sync(full, vp, o), ut = __shfl_up_sync(full, vt, o);
+    if (lane - o >= sp) vp += up;
+    if (lane - o >= st) vt += ut;
   }
+  if (bp >= 0 && (lane == 31 || bp_next != bp)) atomicAdd(hst + bp, vp);
+  if (bt >= 0 && (lane == 31 || bt_next != bt)) atomicAdd(hst + bt, vt);
 }
 
 // Fire-and-forget fp32 addition in L2 (the result is unused, so this is a
@@ -155,10 +166,10 @@ __device__ __forceinline__ void red_add_f32(float* p, uint32_t v) { atomicAdd(p,
 // values (the position bucket only grows along the columns; the time bucket
 // is bounded by the round's earliest and latest query) a score adds its
 // gradient to two or three register totals; finished runs wait in one slot
-// per table and are added into the histogram once per step, lanes with
-// equal buckets summed by shuffles first (same-address shared atomics from
-// many lanes were the cost).  One pointwise warp flushes the unit's sums
-// into this head's table gradients.
+// per table and are added into the histogram once per step, runs of lanes
+// with equal buckets summed by a segmented shuffle scan first
+// (same-address shared atomics from many lanes were the cost).  One
+// pointwise warp flushes the unit's sums into this head's table gradients.
 template <bool RAB>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_kvq_kernel(const __grid_constant__ BwdMaps maps, const __grid_constant__ GroupSet gs) {
@@ -226,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   if (RAB)
-    for (int i = threadIdx.x; i < 2 * kHistBins; i += blockDim.x) hist[i] = 0.f;
+    for (int i = threadIdx.x; i < 2 * kHistCopies * kHistBins; i += blockDim.x) hist[i] = 0.f;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -470,7 +481,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the unit's histogram buffer (free once the unit two back was flushed)
       float tabp = 0.f, tabt = 0.f;  // half of bucket min(lane, nb - 1)
       int32_t tj = 0;
-      float* hst = hist + (hu & 1) * kHistBins;
+      float* const hst0 = hist + (hu & 1) * kHistCopies * kHistBins;  // the unit's copies
+      float* hst = hst0 + (pw % kHistCopies) * kHistBins;
       if constexpr (RAB) {
         tabp = rab_lane_table(A.rab_pos, A.nbp, h, lane);
         tabt = rab_lane_table(A.rab_time, A.nbt, h, lane);
@@ -485,8 +497,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int run_p = -1, run_t = -1;
       float sum_p = 0.f, sum_t = 0.f;
       // a finished run waits in one pending slot per table until the end of
-      // the step, when the warp adds the slots up bin by bin; a second one in
-      // the same step goes straight into the histogram
+      // the step, when the warp sums runs of lanes with equal bins; a second
+      // one in the same step goes straight into the histogram
       int pend_p = -1, pend_t = -1;
       float psum_p = 0.f, psum_t = 0.f;
       auto run_add = [&](int& run, float& sum, int& pend, float& psum, int bin, float g) {
@@ -640,8 +652,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if constexpr (RAB) {  // the step's finished runs, equal bins added up first
           if (__any_sync(0xffffffffu, (pend_p >= 0) | (pend_t >= 0))) {
-            warp_flush_bins(hst, pend_p, psum_p, lane);
-            warp_flush_bins(hst, pend_t, psum_t, lane);
+            warp_flush_runs(hst, pend_p, psum_p, pend_t, psum_t, lane);
             pend_p = pend_t = -1;
           }
         }
@@ -710,8 +721,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if constexpr (RAB) {
         // the unit's last runs, lanes with equal buckets added up first
-        warp_flush_bins(hst, run_p, sum_p, lane);
-        warp_flush_bins(hst, run_t, sum_t, lane);
+        warp_flush_runs(hst, run_p, sum_p, run_t, sum_t, lane);
         // this warp's sums of the unit are in; the first pointwise warp adds
         // the unit's histogram into this head's table gradients (dS2 is
         // 2 dP SiLU'(x); the gradient takes dP SiLU'(x) / N) and clears it
@@ -721,7 +731,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
           const float sc = 0.5f * A.inv_n;
           for (int bin = lane; bin < kHistBins; bin += 32) {
-            const float v = hst[bin];
+            float v = 0.f;
+            for (int cp = 0; cp < kHistCopies; ++cp) v += hst0[cp * kHistBins + bin];
             if (v != 0.f) {
               if (bin < 32) {
                 if (A.d_rab_pos) atomicAdd(A.d_rab_pos + h * A.nbp + imin(bin, A.nbp - 1), v * sc);
@@ -729,7 +740,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 atomicAdd(A.d_rab_time + h * A.nbt + imin(bin - 32, A.nbt - 1), v * sc);
               }
             }
-            hst[bin] = 0.f;
+            for (int cp = 0; cp < kHistCopies; ++cp) hst0[cp * kHistBins + bin] = 0.f;
           }
           __syncwarp();
           if (lane == 0) mbar_arrive(bar(F_H_ZERO + (hu & 1)));
