@@ -543,7 +543,7 @@ def main():
     K = args.steps
     fb, fe, bb, be = new_events(K), new_events(K), new_events(K), new_events(K)
 
-    def step(i=None, e2e=None):
+    def step(i=None):
         evf = (fb[i], fe[i]) if i is not None else None
         evb = (bb[i], be[i]) if i is not None else None
         sla.hstu_sla_fwd(q, k, v, offs, nts, out=out, workspace=ws_f, events=evf, **kw)
