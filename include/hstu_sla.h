@@ -102,8 +102,9 @@ typedef struct {
    * with bucket(n) = min(floor(log2(n + 1)), buckets - 1), dpos = i - j for
    * a history row, Lh - j for a candidate row (0 to itself), and
    * dt = |timestamps[i] - timestamps[j]|.  A NULL table adds nothing;
-   * rab_time needs timestamps.  Each table has 1..32 buckets per head.  Not
-   * available with the grouped calls; the backward needs d = 128. */
+   * rab_time needs timestamps.  Each table has 1..32 buckets per head.  The
+   * backward needs d = 128.  In a grouped call each group has its own
+   * tables and timestamps, or none. */
   const int32_t* timestamps;    /* device [T], any integer time unit, or NULL */
   const float* rab_pos;         /* device [H][rab_pos_buckets], or NULL */
   const float* rab_time;        /* device [H][rab_time_buckets], or NULL */
@@ -178,8 +179,13 @@ int hstu_sla_bwd(const hstu_sla_bwd_params* p, void* workspace, size_t workspace
  *     device-side input error of any group is reported there), then each
  *     group's own workspace in the order given.
  *   - groups[0].event_begin / event_end (if set) bracket the attention kernel.
+ *   - relative attention bias: per group, as for one call (the backward
+ *     writes each group's d_rab_pos / d_rab_time).  If any group has a
+ *     table, the launch runs the bias variant of the kernel for every group
+ *     (a group without tables adds nothing but shares that kernel's cost).
  * Returns HSTU_SLA_ERR_INVALID_ARG for G outside [1, HSTU_SLA_MAX_GROUPS] or a
- * bad group, HSTU_SLA_ERR_UNSUPPORTED for mixed d (or d != 128 backward). */
+ * bad group (a backward group with a table but no gradient buffer for it),
+ * HSTU_SLA_ERR_UNSUPPORTED for mixed d (or d != 128 backward). */
 #define HSTU_SLA_MAX_GROUPS 4
 size_t hstu_sla_grouped_workspace_bytes(int which, int32_t G, const int64_t* total_tokens,
                                         const int32_t* B, const int32_t* H, const int32_t* d);

@@ -216,9 +216,11 @@ def hstu_sla_grouped_workspace_bytes(which: int, problems) -> int:
 
 
 def _group_params(g: dict, events=None) -> _abi.FwdParams:
-    return _fwd_params(g["q"], g["k"], g["v"], g["seq_offsets"], g.get("num_targets"),
-                       g["contextual_len"], g["K1"], g["K2"], g["alpha"], g["N"],
-                       g.get("max_seq_len"), events, g.get("candidates_only", False))
+    p = _fwd_params(g["q"], g["k"], g["v"], g["seq_offsets"], g.get("num_targets"),
+                    g["contextual_len"], g["K1"], g["K2"], g["alpha"], g["N"],
+                    g.get("max_seq_len"), events, g.get("candidates_only", False))
+    _set_rab(p, g["q"].shape[1], g.get("timestamps"), g.get("rab_pos"), g.get("rab_time"))
+    return p
 
 
 def _grouped_ws(which, params, device, workspace):
@@ -237,7 +239,9 @@ def hstu_sla_fwd_grouped(groups, *, workspace=None, stream=None, events=None):
     """Several independent SLA forwards (e.g. the channels of a Mixture of
     Transducers) in one launch.  groups: list of dicts with the keyword
     arguments of hstu_sla_fwd plus q, k, v, seq_offsets (num_targets,
-    max_seq_len, out, candidates_only optional).  Returns the outputs."""
+    max_seq_len, out, candidates_only, and the relative attention bias's
+    timestamps, rab_pos, rab_time optional, per group).  Returns the
+    outputs."""
     lib = _abi.load()
     G = len(groups)
     arr = (_abi.FwdParams * G)()
@@ -259,7 +263,9 @@ def hstu_sla_fwd_grouped(groups, *, workspace=None, stream=None, events=None):
 
 def hstu_sla_bwd_grouped(groups, *, workspace=None, stream=None, events=None):
     """Several independent SLA backwards in one launch (head_dim 128).  groups:
-    as for hstu_sla_fwd_grouped plus dout.  Returns [(dq, dk, dv)] per group."""
+    as for hstu_sla_fwd_grouped plus dout.  Returns (dq, dk, dv) per group, and
+    (dq, dk, dv, (d_rab_pos, d_rab_time)) for a group with a relative
+    attention bias."""
     lib = _abi.load()
     G = len(groups)
     arr = (_abi.BwdParams * G)()
@@ -274,8 +280,13 @@ def hstu_sla_bwd_grouped(groups, *, workspace=None, stream=None, events=None):
         b.dq, b.dq_row_stride = dq.data_ptr(), _row_stride(dq, "dq", H, d)
         b.dk, b.dk_row_stride = dk.data_ptr(), _row_stride(dk, "dk", H, d)
         b.dv, b.dv_row_stride = dv.data_ptr(), _row_stride(dv, "dv", H, d)
+        rp, rt = g.get("rab_pos"), g.get("rab_time")
+        d_rab = (torch.empty_like(rp) if rp is not None else None,
+                 torch.empty_like(rt) if rt is not None else None)
+        b.d_rab_pos = d_rab[0].data_ptr() if d_rab[0] is not None else None
+        b.d_rab_time = d_rab[1].data_ptr() if d_rab[1] is not None else None
         arr[i] = b
-        grads.append((dq, dk, dv))
+        grads.append((dq, dk, dv, d_rab) if rp is not None or rt is not None else (dq, dk, dv))
     ws = _grouped_ws(_abi.WS_BWD, [b.fwd for b in arr], groups[0]["q"].device, workspace)
     _check(lib.hstu_sla_bwd_grouped(arr, G, ws.data_ptr(), ws.numel(), _stream_ptr(stream)),
            "hstu_sla_bwd_grouped")

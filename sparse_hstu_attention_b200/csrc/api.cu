@@ -11,7 +11,7 @@ namespace {
 
 // 101: hstu_sla_fwd_params.candidates_only; 102: FP8 forward; 103: grouped calls;
 // 104: relative attention bias
-constexpr int kAbiVersion = 104;
+constexpr int kAbiVersion = 105;
 static_assert(HSTU_SLA_MAX_GROUPS == kMaxGroups, "one grouped launch holds every group");
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
@@ -165,7 +165,6 @@ int hstu_sla_fwd_grouped(const hstu_sla_fwd_params* groups, int32_t G, void* wor
     f[g] = &groups[g];
     if ((e = check_common(f[g]))) return e;
     if ((e = check_tensor(f[g]->out, f[g]->out_row_stride, f[g]))) return e;
-    if (f[g]->rab_pos || f[g]->rab_time) return HSTU_SLA_ERR_UNSUPPORTED;
     if (f[g]->d != f[0]->d) return HSTU_SLA_ERR_UNSUPPORTED;
     T[g] = f[g]->total_tokens;
     Bs[g] = f[g]->B;
@@ -210,7 +209,8 @@ int hstu_sla_bwd_grouped(const hstu_sla_bwd_params* groups, int32_t G, void* wor
     const hstu_sla_bwd_params* p = &groups[g];
     f[g] = &p->fwd;
     if ((e = check_common(f[g]))) return e;
-    if (f[g]->rab_pos || f[g]->rab_time) return HSTU_SLA_ERR_UNSUPPORTED;
+    if ((f[g]->rab_pos && !p->d_rab_pos) || (f[g]->rab_time && !p->d_rab_time))
+      return HSTU_SLA_ERR_INVALID_ARG;
     if ((e = check_tensor(p->dout, p->dout_row_stride, f[g]))) return e;
     if ((e = check_tensor(p->dq, p->dq_row_stride, f[g]))) return e;
     if ((e = check_tensor(p->dk, p->dk_row_stride, f[g]))) return e;
@@ -241,6 +241,8 @@ int hstu_sla_bwd_grouped(const hstu_sla_bwd_params* groups, int32_t G, void* wor
     a[g].dk_rs = p->dk_row_stride;
     a[g].dv_rs = p->dv_row_stride;
     a[g].dqacc = reinterpret_cast<float*>(w + ws_bytes(T[g], Bs[g]));
+    a[g].d_rab_pos = f[g]->rab_pos ? p->d_rab_pos : nullptr;
+    a[g].d_rab_time = f[g]->rab_time ? p->d_rab_time : nullptr;
     ce = launch_worklist(a[g], kKvBN, 1, true, st);
     w += round256(hstu_sla_workspace_bytes(HSTU_SLA_WS_BWD, T[g], Bs[g], Hs[g], ds[g]));
   }

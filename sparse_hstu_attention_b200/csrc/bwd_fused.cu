@@ -878,8 +878,17 @@ cudaError_t launch_bwd_fused_grouped(const GroupSet& gs, cudaStream_t st) {
   memset(&m, 0, sizeof(m));
   int64_t units = 0;
   cudaError_t e;
+  bool rab = false;  // a problem with a relative attention bias
   for (int p = 0; p < gs.G; ++p) {
     const AttnArgs& a = gs.g[p];
+    rab = rab || a.rab_pos != nullptr || a.rab_time != nullptr;
+    // its table gradients are overwritten (also when it has no tokens)
+    if (a.d_rab_pos &&
+        (e = cudaMemsetAsync(a.d_rab_pos, 0, sizeof(float) * a.H * a.nbp, st)) != cudaSuccess)
+      return e;
+    if (a.d_rab_time &&
+        (e = cudaMemsetAsync(a.d_rab_time, 0, sizeof(float) * a.H * a.nbt, st)) != cudaSuccess)
+      return e;
     if (a.T == 0) continue;  // no units; its maps stay unused
     const int HD = a.H * D;
     if (!make_tma_2d(&m.k[p], a.k, a.T, HD, a.k_rs, BOXW, kRes, true) ||
@@ -892,16 +901,6 @@ cudaError_t launch_bwd_fused_grouped(const GroupSet& gs, cudaStream_t st) {
     units += max_items(a.T, a.B) * a.H;
   }
   if (units == 0) return cudaSuccess;
-  const bool rab = gs.G == 1 && (gs.g[0].rab_pos != nullptr || gs.g[0].rab_time != nullptr);
-  if (rab) {  // the table gradients are overwritten
-    const AttnArgs& a = gs.g[0];
-    if (a.d_rab_pos &&
-        (e = cudaMemsetAsync(a.d_rab_pos, 0, sizeof(float) * a.H * a.nbp, st)) != cudaSuccess)
-      return e;
-    if (a.d_rab_time &&
-        (e = cudaMemsetAsync(a.d_rab_time, 0, sizeof(float) * a.H * a.nbt, st)) != cudaSuccess)
-      return e;
-  }
   const auto kern = rab ? bwd_kvq_kernel<true> : bwd_kvq_kernel<false>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
   if (e != cudaSuccess) return e;

@@ -681,7 +681,8 @@ cudaError_t launch_d(const GroupSet& gs, cudaStream_t st) {
     units += max_items(a.T, a.B) * a.H;
   }
   if (units == 0) return cudaSuccess;
-  const bool rab = gs.G == 1 && (gs.g[0].rab_pos != nullptr || gs.g[0].rab_time != nullptr);
+  bool rab = false;  // any problem with a relative attention bias takes the bias kernel
+  for (int p = 0; p < gs.G; ++p) rab = rab || gs.g[p].rab_pos != nullptr || gs.g[p].rab_time != nullptr;
   const auto kern = rab ? fwd_tc_kernel<D, true> : fwd_tc_kernel<D, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;

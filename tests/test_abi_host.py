@@ -170,8 +170,9 @@ def test_grouped_calls_reject_bad_groups_on_the_host(lib):
 
 
 def test_rab_arguments_are_checked_on_the_host(lib):
-    """Bucket counts outside 1..32 and a time table without timestamps are
-    refused before any CUDA call; so are the bias with the grouped calls."""
+    """Bucket counts outside 1..32, a time table without timestamps and a
+    table without a gradient buffer (one call or grouped) are refused before
+    any CUDA call."""
     p = _params(d=128, q_row_stride=512, k_row_stride=512, v_row_stride=512)
     p.out, p.out_row_stride = FAKE, 512
     ws = 0x100000
@@ -183,11 +184,11 @@ def test_rab_arguments_are_checked_on_the_host(lib):
     p.rab_time, p.rab_time_buckets = FAKE, 8
     assert lib.hstu_sla_fwd(ctypes.byref(p), ws, 1 << 30, None) == _abi.ERR_INVALID_ARG
     p.timestamps = FAKE
-    arr = (_abi.FwdParams * 1)(p)
-    assert lib.hstu_sla_fwd_grouped(arr, 1, ws, 1 << 30, None) == _abi.ERR_UNSUPPORTED
     b = _abi.BwdParams()
     b.fwd = p
     b.dout = b.dq = b.dk = b.dv = FAKE
     b.dout_row_stride = b.dq_row_stride = b.dk_row_stride = b.dv_row_stride = 512
     # the time table's gradient buffer is missing
     assert lib.hstu_sla_bwd(ctypes.byref(b), ws, 1 << 30, None) == _abi.ERR_INVALID_ARG
+    arr = (_abi.BwdParams * 1)(b)
+    assert lib.hstu_sla_bwd_grouped(arr, 1, ws, 1 << 30, None) == _abi.ERR_INVALID_ARG

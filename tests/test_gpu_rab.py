@@ -2,7 +2,8 @@
 phi2(Q K^T + rab^{p,t})): forward, dq, dk, dv and both tables' gradients
 against the oracle on seeded inputs (TOL of max|ref| per tensor), each table
 alone, all-zero tables equal to the bias-free kernels, the forward at
-head_dim 64, and the host-side refusals (backward at head_dim 64, grouped)."""
+head_dim 64, the refusal of the backward at head_dim 64, and grouped calls
+with a bias on some of their problems."""
 import numpy as np
 import pytest
 import torch
@@ -124,25 +125,58 @@ def test_zero_tables_equal_the_bias_free_kernels():
     assert_close("dq", dq, dq0.float().cpu().numpy().astype(np.float64), tol=1e-2)
 
 
-def test_rab_forward_head_dim_64_and_refusals():
+def test_rab_forward_head_dim_64_and_refusal():
     b, ts, rp, rt = _case(lengths=(200, 77), H=3, d=64, K1=50, K2=8, ctx=4, seed=9)
     (out,) = _run(b, ts, rp, rt, bwd=False)
     assert_close("out d64", out, _oracle(b, ts, rp, rt).fwd(b.q, b.k, b.v))
     with pytest.raises(sla.SLAError) as ex:
         _run(b, ts, rp, rt)
     assert ex.value.code == _abi.ERR_UNSUPPORTED
-    b2, ts2, rp2, rt2 = _case(seed=10)
-    g = to_gpu(b2)
-    grp = dict(q=g["q"], k=g["k"], v=g["v"], seq_offsets=g["offs"], num_targets=g["nts"],
-               **kwargs_of(b2))
-    p = sla._group_params(grp)
-    sla._set_rab(p, 4, torch.from_numpy(ts2).to(DEV), rp2.to(DEV), None)
-    out = torch.empty_like(g["q"])
-    p.out, p.out_row_stride = out.data_ptr(), out.stride(0)
-    arr = (_abi.FwdParams * 1)(p)
-    ws = torch.empty(1 << 20, dtype=torch.uint8, device=DEV)
-    assert _abi.load().hstu_sla_fwd_grouped(arr, 1, ws.data_ptr(), ws.numel(), None) == \
-        _abi.ERR_UNSUPPORTED
+
+
+def test_rab_in_grouped_calls():
+    """Three problems in one grouped launch (MoT channels): both tables, the
+    position table only, no bias.  Each against the oracle, and against its
+    own single call: forward and dk / dv bitwise, the rest to fp32 order."""
+    cases = [_case(lengths=(300, 700, 65), K1=256, K2=64, seed=41),
+             _case(lengths=(129, 40, 520, 255), nt=8, K1=100, K2=16, ctx=4, seed=42),
+             _case(lengths=(90, 333), nt=4, K1=64, K2=8, ctx=2, seed=43)]
+    tables = [(True, True), (True, False), (False, False)]
+    groups, singles = [], []
+    for (b, ts, rp, rt), (use_p, use_t) in zip(cases, tables):
+        rp, rt = (rp if use_p else None), (rt if use_t else None)
+        g = to_gpu(b)
+        rab = dict(timestamps=torch.from_numpy(ts).to(DEV),
+                   rab_pos=None if rp is None else rp.to(DEV),
+                   rab_time=None if rt is None else rt.to(DEV))
+        groups.append(dict(q=g["q"], k=g["k"], v=g["v"], dout=g["dout"], seq_offsets=g["offs"],
+                           num_targets=g["nts"], **kwargs_of(b), **rab))
+        singles.append(_run(b, ts, rp, rt))
+    outs = sla.hstu_sla_fwd_grouped(groups)
+    grads = sla.hstu_sla_bwd_grouped(groups)
+    torch.cuda.synchronize()
+    for (b, ts, rp, rt), (use_p, use_t), out, gr, one in zip(cases, tables, outs, grads, singles):
+        rp, rt = (rp if use_p else None), (rt if use_t else None)
+        assert torch.equal(out, one[0])
+        assert torch.equal(gr[1], one[2]) and torch.equal(gr[2], one[3])
+        p = _oracle(b, ts, rp, rt)
+        assert_close("out", out, p.fwd(b.q, b.k, b.v))
+        rq, rk, rv = p.bwd(b.q, b.k, b.v, b.dout)
+        for name, got, ref in (("dq", gr[0], rq), ("dk", gr[1], rk), ("dv", gr[2], rv)):
+            assert_close(name, got, ref)
+        if rp is None and rt is None:
+            assert len(gr) == 3
+            continue
+        rdp, rdt = p.bwd_rab(b.q, b.k, b.v, b.dout)
+        drp, drt = gr[3]
+        assert_close("d rab_pos", drp, rdp)
+        if rt is None:
+            assert drt is None
+        else:
+            assert_close("d rab_time", drt, rdt)
+        for mine, single in zip(gr[3], one[4]):
+            if mine is not None:
+                assert torch.allclose(mine, single, rtol=1e-5, atol=1e-6 * float(single.abs().max()))
 
 
 def _table_totals_agree(drp, drt):
