@@ -212,10 +212,21 @@ int hstu_sla_bwd_grouped(const hstu_sla_bwd_params* groups, int32_t G, void* wor
  *    GPU (other streams, other host threads) race and must be serialised by
  *    the caller.  Each call rewrites the status and work lists it reads, so
  *    nothing carries over from the previous call.
- *  - Device-detected input errors are not reported (hstu_sla_get_error needs
- *    a workspace pointer); out is then left unwritten.
+ *  - Device-detected input errors (corrupt seq_offsets / num_targets, a
+ *    timed-out wait) leave out unwritten; hstu_sla_noalloc_get_error reads
+ *    them.
+ *  - The array's address is cached per device and context; after a device
+ *    reset the next call looks it up again.
  * Allocates nothing: no cudaMalloc, no cudaFree. */
 int hstu_sla_fwd_noalloc(const hstu_sla_fwd_params* p, hstu_stream_t stream);
+
+/* Synchronises `stream` and returns the device-side status that the last
+ * hstu_sla_fwd_noalloc call on the current device recorded in the library's
+ * scratch array (HSTU_SLA_OK, HSTU_SLA_ERR_BAD_INPUT or HSTU_SLA_ERR_TIMEOUT),
+ * or HSTU_SLA_ERR_CUDA.  Like the call itself, it reads the one shared array:
+ * a call of another stream in between overwrites the status.  Allocates
+ * nothing. */
+int hstu_sla_noalloc_get_error(hstu_stream_t stream);
 
 /* Test hook: the number of visible keys of every token as the forward
  * kernels enumerate them (row_counts, device int64 [T]) and the number of

@@ -32,7 +32,7 @@ import torch
 from . import _abi
 from ._abi import LibraryMissing  # noqa: F401
 
-__all__ = ["hstu_sla_fwd", "hstu_sla_fwd_noalloc", "hstu_sla_bwd", "hstu_sla_workspace_bytes",
+__all__ = ["hstu_sla_fwd", "hstu_sla_fwd_noalloc", "hstu_sla_noalloc_get_error", "hstu_sla_bwd", "hstu_sla_workspace_bytes",
            "hstu_sla_count_pairs", "hstu_sla_fwd_grouped", "hstu_sla_bwd_grouped",
            "hstu_sla_grouped_workspace_bytes", "hstu_sla_get_error", "hstu_sla_strerror",
            "SLAError", "SLAAttention", "sla_attention"]
@@ -156,10 +156,13 @@ def hstu_sla_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                          seq_offsets: torch.Tensor, num_targets: Optional[torch.Tensor], *,
                          contextual_len: int, K1: int, K2: int, alpha: float, N: float,
                          max_seq_len: Optional[int] = None, out: Optional[torch.Tensor] = None,
-                         stream=None) -> torch.Tensor:
+                         stream=None, check: bool = True) -> torch.Tensor:
     """The forward through the C entry point that allocates no workspace (for
     callers whose runtime forbids device allocation in the launch path).  The
-    library keeps one 2 MiB scratch array per device; overlapping calls race."""
+    library keeps one 2 MiB scratch array per device; overlapping calls race.
+    check: synchronise and raise if the device recorded an input error or a
+    timed-out wait (out is then unwritten); check=False leaves that to
+    hstu_sla_noalloc_get_error."""
     lib = _abi.load()
     p = _fwd_params(q, k, v, seq_offsets, num_targets, contextual_len, K1, K2, alpha, N,
                     max_seq_len)
@@ -168,7 +171,15 @@ def hstu_sla_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     p.out = out.data_ptr()
     p.out_row_stride = _row_stride(out, "out", p.H, p.d)
     _check(lib.hstu_sla_fwd_noalloc(ctypes.byref(p), _stream_ptr(stream)), "hstu_sla_fwd_noalloc")
+    if check:
+        _check(lib.hstu_sla_noalloc_get_error(_stream_ptr(stream)), "hstu_sla_fwd_noalloc (device)")
     return out
+
+
+def hstu_sla_noalloc_get_error(stream=None) -> int:
+    """Synchronise and return the device-side status of the last
+    hstu_sla_fwd_noalloc call on the current device."""
+    return int(_abi.load().hstu_sla_noalloc_get_error(_stream_ptr(stream)))
 
 
 def hstu_sla_bwd(dout: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
@@ -263,7 +274,8 @@ def hstu_sla_fwd_grouped(groups, *, workspace=None, stream=None, events=None):
 
 def hstu_sla_bwd_grouped(groups, *, workspace=None, stream=None, events=None):
     """Several independent SLA backwards in one launch (head_dim 128).  groups:
-    as for hstu_sla_fwd_grouped plus dout.  Returns (dq, dk, dv) per group, and
+    as for hstu_sla_fwd_grouped plus dout (and optionally preallocated dq, dk,
+    dv).  Returns (dq, dk, dv) per group, and
     (dq, dk, dv, (d_rab_pos, d_rab_time)) for a group with a relative
     attention bias."""
     lib = _abi.load()
@@ -274,8 +286,9 @@ def hstu_sla_bwd_grouped(groups, *, workspace=None, stream=None, events=None):
         b = _abi.BwdParams()
         b.fwd = _group_params(g, events if i == 0 else None)
         q, H, d = g["q"], b.fwd.H, b.fwd.d
-        dq, dk, dv = (torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
-                      for _ in range(3))
+        dq, dk, dv = (g.get(n) if g.get(n) is not None else
+                      torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
+                      for n in ("dq", "dk", "dv"))
         b.dout, b.dout_row_stride = g["dout"].data_ptr(), _row_stride(g["dout"], "dout", H, d)
         b.dq, b.dq_row_stride = dq.data_ptr(), _row_stride(dq, "dq", H, d)
         b.dk, b.dk_row_stride = dk.data_ptr(), _row_stride(dk, "dk", H, d)

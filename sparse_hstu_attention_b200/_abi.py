@@ -128,6 +128,8 @@ def load():
     lib.hstu_sla_bwd.restype = ctypes.c_int
     lib.hstu_sla_fwd_noalloc.argtypes = [ctypes.POINTER(FwdParams), vp]
     lib.hstu_sla_fwd_noalloc.restype = ctypes.c_int
+    lib.hstu_sla_noalloc_get_error.argtypes = [vp]
+    lib.hstu_sla_noalloc_get_error.restype = ctypes.c_int
     lib.hstu_sla_count_pairs.argtypes = [ctypes.POINTER(FwdParams), vp, vp, vp, sz, vp]
     lib.hstu_sla_count_pairs.restype = ctypes.c_int
     lib.hstu_sla_grouped_workspace_bytes.argtypes = [ctypes.c_int, ctypes.c_int32, vp, vp, vp,
@@ -154,6 +156,8 @@ def load():
     lib.hstu_stu_get_error.restype = ctypes.c_int
     lib.hstu_jagged_truncate_offsets.argtypes = [vp, vp, i32, i32, i32, vp, vp]
     lib.hstu_jagged_truncate_offsets.restype = ctypes.c_int
+    lib.hstu_jagged_truncate_lengths.argtypes = [vp, vp, i32, i32, i32, vp]
+    lib.hstu_jagged_truncate_lengths.restype = ctypes.c_int64
     lib.hstu_jagged_truncate.argtypes = [vp, i64, vp, vp, vp, i32, i32, i32, i32, vp, i64, i64,
                                          i32, vp]
     lib.hstu_jagged_truncate.restype = ctypes.c_int

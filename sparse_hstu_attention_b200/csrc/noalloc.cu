@@ -3,7 +3,8 @@
 // tcgen05 forward kernel), with the work lists and status word placed in a
 // fixed-size array that lives in the library's own device memory instead of a
 // caller-provided workspace.
-#include <atomic>
+#include <cuda.h>
+
 #include <mutex>
 
 #include "sla_common.cuh"
@@ -18,27 +19,65 @@ constexpr size_t kNoAllocScratchBytes = size_t(2) << 20;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxDevices = 64;
-std::atomic<void*> g_scratch_addr[kMaxDevices];
+// Per device: the context the address was looked up in and the address.  A
+// device reset (or a release and re-creation of the primary context) makes
+// a new context in which the array can sit elsewhere: the address is looked
+// up again when the current context differs from the cached one.
+struct ScratchEntry {
+  unsigned long long ctx_id;
+  void* addr;
+};
+ScratchEntry g_scratch[kMaxDevices];
 std::mutex g_scratch_mutex;
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Identifier of the context current on this thread (0 if the driver entry
+// points are unavailable: the cache is then keyed by device alone).
+unsigned long long current_ctx_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  if (get_current == nullptr || get_id == nullptr) return 0;
+  CUcontext c = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&c) != CUDA_SUCCESS || c == nullptr || get_id(c, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
 
 // Device address of g_noalloc_scratch on the current device.  In host code the
 // symbol name is only a host-side handle; the device address must be looked up
-// once per device, with that device current.
+// with that device current, once per device and context.
 int scratch_address(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return HSTU_SLA_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return HSTU_SLA_ERR_UNSUPPORTED;
-  void* p = g_scratch_addr[dev].load(std::memory_order_acquire);
-  if (p == nullptr) {
-    std::lock_guard<std::mutex> lock(g_scratch_mutex);
-    p = g_scratch_addr[dev].load(std::memory_order_relaxed);
-    if (p == nullptr) {
-      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
-        return HSTU_SLA_ERR_CUDA;
-      g_scratch_addr[dev].store(p, std::memory_order_release);
-    }
+  // binds the device's primary context to this thread (creating it after a
+  // reset); allocates nothing
+  if (cudaSetDevice(dev) != cudaSuccess) return HSTU_SLA_ERR_CUDA;
+  const unsigned long long ctx = current_ctx_id();
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  ScratchEntry& e = g_scratch[dev];
+  if (e.addr == nullptr || e.ctx_id != ctx) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return HSTU_SLA_ERR_CUDA;
+    e.addr = p;
+    e.ctx_id = ctx;
   }
-  *out = p;
+  *out = e.addr;
   return HSTU_SLA_OK;
 }
 
@@ -53,4 +92,11 @@ extern "C" int hstu_sla_fwd_noalloc(const hstu_sla_fwd_params* p, hstu_stream_t 
   const int e = scratch_address(&scratch);
   if (e != HSTU_SLA_OK) return e;
   return hstu_sla_fwd(p, scratch, kNoAllocScratchBytes, stream);
+}
+
+extern "C" int hstu_sla_noalloc_get_error(hstu_stream_t stream) {
+  void* scratch = nullptr;
+  const int e = scratch_address(&scratch);
+  if (e != HSTU_SLA_OK) return e;
+  return hstu_sla_get_error(scratch, stream);
 }

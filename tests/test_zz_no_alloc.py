@@ -33,6 +33,9 @@ def _params(g, kw, out):
 
 
 def test_noalloc_matches_workspace_entry_point_on_consecutive_calls():
+    """Both entry points run the same kernels on the same work lists, and the
+    forward is deterministic: the results must be identical bit for bit, so
+    any corruption left in the shared scratch by the previous call shows."""
     lib = _abi.load()
     stream = torch.cuda.current_stream().cuda_stream
     batches = [make_batch(WORKLOADS["mid"], with_dout=False),
@@ -45,10 +48,34 @@ def test_noalloc_matches_workspace_entry_point_on_consecutive_calls():
             out = torch.full_like(ref, float("nan"))
             rc = lib.hstu_sla_fwd_noalloc(ctypes.byref(_params(g, kw, out)), stream)
             assert rc == _abi.OK, sla.hstu_sla_strerror(rc)
+            assert lib.hstu_sla_noalloc_get_error(stream) == _abi.OK
             torch.cuda.synchronize()
+            assert torch.equal(out, ref)
             scale = ref.float().abs().max().item()
             err = (out.float() - ref.float()).abs().max().item()
             assert err <= TOL * scale, (err, scale)
+
+
+def test_noalloc_python_binding_and_device_status():
+    """The binding's wrapper checks the device status; corrupted offsets are
+    reported as BAD_INPUT (out left unwritten), and the next good call
+    clears the status."""
+    b = make_batch(WORKLOADS["tiny"], with_dout=False)
+    g = to_gpu(b)
+    kw = kwargs_of(b)
+    ref = sla.hstu_sla_fwd(g["q"], g["k"], g["v"], g["offs"], g["nts"], **kw)
+    out = sla.hstu_sla_fwd_noalloc(g["q"], g["k"], g["v"], g["offs"], g["nts"], **kw)
+    assert torch.equal(out, ref)
+    bad = g["offs"].clone()
+    bad[1] = bad[2] + 1  # offsets no longer monotone
+    out = torch.full_like(ref, float("nan"))
+    with pytest.raises(sla.SLAError):
+        sla.hstu_sla_fwd_noalloc(g["q"], g["k"], g["v"], bad, g["nts"], out=out, **kw)
+    assert sla.hstu_sla_noalloc_get_error() == _abi.ERR_BAD_INPUT
+    assert torch.isnan(out.float()).all()
+    out = sla.hstu_sla_fwd_noalloc(g["q"], g["k"], g["v"], g["offs"], g["nts"], **kw)
+    assert sla.hstu_sla_noalloc_get_error() == _abi.OK
+    assert torch.equal(out, ref)
 
 
 def test_noalloc_rejects_batches_beyond_its_scratch():
