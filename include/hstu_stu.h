@@ -131,6 +131,14 @@ int hstu_stu_get_error(const void* workspace, hstu_stream_t stream);
 int hstu_jagged_truncate_offsets(const int32_t* seq_offsets, const int32_t* num_targets, int32_t B,
                                  int32_t contextual_len, int32_t tail, int32_t* new_offsets,
                                  hstu_stream_t stream);
+/* Host-side form of the same rule, for sizing the truncated buffers before
+ * any launch: host arrays lengths[B] and num_targets[B] (NULL = none) give
+ * new_lengths[B] (host, may be NULL) and the return value T_out, the total
+ * kept rows; HSTU_SLA_ERR_INVALID_ARG (negative) for a negative length or
+ * num_targets outside [0, length].  Runs on the host only (no CUDA call). */
+int64_t hstu_jagged_truncate_lengths(const int32_t* lengths, const int32_t* num_targets,
+                                     int32_t B, int32_t contextual_len, int32_t tail,
+                                     int32_t* new_lengths);
 int hstu_jagged_truncate(const void* src, int64_t src_row_stride, const int32_t* seq_offsets,
                          const int32_t* new_offsets, const int32_t* num_targets, int32_t B,
                          int32_t contextual_len, int32_t tail, int32_t width, void* dst,

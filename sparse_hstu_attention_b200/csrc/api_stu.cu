@@ -352,6 +352,25 @@ int hstu_jagged_truncate_offsets(const int32_t* seq_offsets, const int32_t* num_
                                         new_offsets, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int64_t hstu_jagged_truncate_lengths(const int32_t* lengths, const int32_t* num_targets,
+                                     int32_t B, int32_t contextual_len, int32_t tail,
+                                     int32_t* new_lengths) {
+  if (lengths == nullptr || B < 1 || contextual_len < 0 || tail < 0)
+    return HSTU_SLA_ERR_INVALID_ARG;
+  int64_t total = 0;
+  for (int b = 0; b < B; ++b) {
+    const int nt = num_targets ? num_targets[b] : 0;
+    if (lengths[b] < 0 || nt < 0 || nt > lengths[b]) return HSTU_SLA_ERR_INVALID_ARG;
+  }
+  for (int b = 0; b < B; ++b) {
+    const int nt = num_targets ? num_targets[b] : 0;
+    const int kept = lengths[b] - hstu::trunc_drop(lengths[b], nt, contextual_len, tail);
+    if (new_lengths) new_lengths[b] = kept;
+    total += kept;
+  }
+  return total;
+}
+
 int hstu_jagged_truncate(const void* src, int64_t src_row_stride, const int32_t* seq_offsets,
                          const int32_t* new_offsets, const int32_t* num_targets, int32_t B,
                          int32_t contextual_len, int32_t tail, int32_t width, void* dst,

@@ -9,6 +9,17 @@ namespace hstu {
 
 int device_sm_count();
 
+// Attention truncation ("Bending the Scaling Law Curve in Large-Scale
+// Recommendation Systems", section 4.3; TorchEasyRec's attention truncation
+// fields): a sequence of length L with nt candidates keeps its contextual
+// prefix [0, c), its last `tail` history rows and its candidates; the history
+// rows in between, max(0, L - nt - c - tail) of them, are dropped.  The one
+// definition of the rule, used by the device kernels and the host helper.
+__host__ __device__ __forceinline__ int trunc_drop(int L, int nt, int c, int tail) {
+  const int d = L - nt - c - tail;
+  return d > 0 ? d : 0;
+}
+
 // GEMM epilogues (gemm_tc.cu)
 enum { kEpiStore = 0, kEpiBiasSilu = 1, kEpiBiasResid = 2, kEpiRedF32 = 3 };
 

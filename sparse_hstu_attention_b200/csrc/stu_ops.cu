@@ -393,8 +393,7 @@ __global__ void trunc_offsets_kernel(const int32_t* offs, const int32_t* nts, in
   new_offs[0] = 0;
   for (int b = 0; b < B; ++b) {
     const int L = offs[b + 1] - offs[b];
-    const int Lh = L - (nts ? nts[b] : 0);
-    const int drop = Lh - c - tail > 0 ? Lh - c - tail : 0;
+    const int drop = trunc_drop(L, nts ? nts[b] : 0, c, tail);
     o += L - drop;
     new_offs[b + 1] = o;
   }
@@ -425,8 +424,7 @@ __global__ void __launch_bounds__(256) trunc_rows_kernel(const bf16* src, int64_
   const int32_t* in_offs = scatter ? new_offs : offs;
   const int b = find_seq(out_offs, B, r);
   const int L = offs[b + 1] - offs[b];
-  const int Lh = L - (nts ? nts[b] : 0);
-  const int drop = Lh - c - tail > 0 ? Lh - c - tail : 0;
+  const int drop = trunc_drop(L, nts ? nts[b] : 0, c, tail);
   const int p = (int)(r - out_offs[b]);
   int64_t s;  // source row, or -1 for a dropped row (scatter)
   if (scatter) s = (p < c || p >= c + drop) ? in_offs[b] + p - (p >= c ? drop : 0) : -1;

@@ -215,11 +215,17 @@ def layer_bwd(dout: torch.Tensor, st: LayerState, w: StuWeights, cfg: StuConfig,
 
 
 def truncated_lengths(lengths, num_targets, contextual_len: int, tail: int) -> np.ndarray:
-    """Host-side lengths after truncation (to size the truncated buffers)."""
-    L = np.asarray(lengths, dtype=np.int64)
-    nt = np.zeros_like(L) if num_targets is None else np.asarray(num_targets, dtype=np.int64)
-    drop = np.maximum(0, L - nt - contextual_len - tail)
-    return L - drop
+    """Per-sequence lengths after truncation, from the library's host helper
+    (the rule the truncation kernels apply), to size the truncated buffers."""
+    L = np.ascontiguousarray(lengths, dtype=np.int32)
+    nt = None if num_targets is None else np.ascontiguousarray(num_targets, dtype=np.int32)
+    out = np.empty_like(L)
+    total = _abi.load().hstu_jagged_truncate_lengths(
+        L.ctypes.data, None if nt is None else nt.ctypes.data, len(L), int(contextual_len),
+        int(tail), out.ctypes.data)
+    if total < 0:
+        _check(int(total), "hstu_jagged_truncate_lengths")
+    return out.astype(np.int64)
 
 
 def truncate_offsets(seq_offsets, num_targets, contextual_len: int, tail: int, stream=None):

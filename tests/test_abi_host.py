@@ -192,3 +192,28 @@ def test_rab_arguments_are_checked_on_the_host(lib):
     assert lib.hstu_sla_bwd(ctypes.byref(b), ws, 1 << 30, None) == _abi.ERR_INVALID_ARG
     arr = (_abi.BwdParams * 1)(b)
     assert lib.hstu_sla_bwd_grouped(arr, 1, ws, 1 << 30, None) == _abi.ERR_INVALID_ARG
+
+
+def test_truncation_lengths_follow_the_oracle_index_set():
+    """The host helper that sizes the truncated buffers keeps exactly the rows
+    the oracle's truncation keeps, sequence by sequence (no GPU needed)."""
+    import numpy as np
+    from oracle import stu as S
+    from sparse_hstu_attention_b200 import stu
+    rng = np.random.default_rng(5)
+    for c, tail in [(0, 0), (4, 16), (32, 1024), (7, 3)]:
+        lengths = rng.integers(0, 3000, size=23)
+        lengths[:3] = [0, 1, c + tail]
+        nts = np.minimum(rng.integers(0, 80, size=23), lengths)
+        got = stu.truncated_lengths(lengths, nts, c, tail)
+        for b in range(len(lengths)):
+            keep, _ = S.truncation_index(np.array([0, lengths[b]]), nts[b:b + 1], c, tail)
+            assert got[b] == len(keep), (b, lengths[b], nts[b], c, tail)
+        assert (stu.truncated_lengths(lengths, None, c, tail) ==
+                [len(S.truncation_index(np.array([0, L]), np.array([0]), c, tail)[0])
+                 for L in lengths]).all()
+    lib = _abi.load()
+    bad = np.array([10, 5], dtype=np.int32)
+    nt = np.array([2, 6], dtype=np.int32)  # more candidates than tokens
+    assert lib.hstu_jagged_truncate_lengths(bad.ctypes.data, nt.ctypes.data, 2, 0, 1, None) \
+        == _abi.ERR_INVALID_ARG
