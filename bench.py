@@ -85,6 +85,44 @@ def _traffic(which, workload):
     return e.get("dram_bytes_per_launch")
 
 
+def roofline(flops, alg_bytes, ms, peaks, peak_src, clk):
+    """The dominant kernel against the roof its arithmetic intensity puts it
+    under: the tensor roof (measured dense bf16 GEMM) when flops / bytes is at
+    or above the ridge, else the HBM roof (measured copy bandwidth).
+
+    The tensor denominator is the burst GEMM figure, measured at the maximum
+    SM clock, the clock a kernel runs at in a short timed loop.  The
+    sustained figure was measured seconds into a power-capped loop at a lower
+    clock; the fraction of it is reported beside, with both clock medians,
+    but never as `frac`."""
+    tflops = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    s = ms * 1e-3
+    ach_t = flops / s / 1e12
+    ach_b = alg_bytes / s / 1e9
+    ridge = tflops * 1e12 / (hbm * 1e9)
+    ai = flops / alg_bytes
+    tensor = ai >= ridge
+    r = {"bound": "tensor" if tensor else "hbm",
+         "achieved": ach_t if tensor else ach_b,
+         "peak": tflops if tensor else hbm,
+         "unit": "TFLOP/s" if tensor else "GB/s",
+         "frac": (ach_t / tflops) if tensor else (ach_b / hbm),
+         "peak_source": (f"bf16_tflops (burst) of {peak_src}" if tensor
+                         else f"hbm_gbs of {peak_src}"),
+         "arithmetic_intensity": ai, "ridge_flop_per_byte": ridge,
+         "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": alg_bytes,
+         "tensor_tflops": ach_t, "frac_of_tensor_peak": ach_t / tflops,
+         "hbm_gbs": ach_b, "frac_of_hbm_peak": ach_b / hbm}
+    sus = peaks.get("bf16_tflops_sustained")
+    if sus:
+        under = (peaks.get("clocks_under_load") or {}).get("sm_mhz_median")
+        r["frac_of_sustained_tensor_peak"] = ach_t / float(sus)
+        r["sustained_peak_sm_mhz"] = under
+        r["run_sm_mhz"] = clk.get("sm_mhz")
+    return r
+
+
 class ClockSampler:
     """nvidia-smi clocks / throttle reasons sampled every 50 ms while active."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -374,6 +412,7 @@ def run_stu(args, world, rank, local):
                        "N": [w.N, cut.N]},
             "flops_per_step": {"projections": gemm, "attention": attn},
             "frac_of_sustained_peak": value / world / peak,
+            "frac_of_burst_peak": value / world / float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])),
             "gpu_launches": K * (STU_LAYERS * (6 + 11 + (2 if args.fp8 else 0)) + 3),
             "clocks": clocks.summary(),
             **({} if (world > 1 or args.no_cpu_baseline) else
@@ -471,6 +510,7 @@ def run_mot(args, world, rank, local):
                        "l2": "inputs > 126 MB L2; no flush"},
             "separate_calls_ms_per_step": ms_sep, "grouped_speedup": ms_sep / ms,
             "frac_of_sustained_peak": value / world / peak,
+            "frac_of_burst_peak": value / world / float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])),
             # forward: 3 work lists + 1 kernel; backward: 3 work lists + 1 kernel
             # + 3 dq conversions (memsets not counted)
             "gpu_launches": K * (3 + 1 + 3 + 1 + 3),
@@ -675,15 +715,13 @@ def main():
 
     peaks, peak_src = _peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    # the roofline kernel runs inside a long timed loop (power-capped clocks):
-    # its denominator is the sustained GEMM figure when one was measured
-    peak_sus = peaks.get("bf16_tflops_sustained")
-    roof_peak = float(peak_sus) if peak_sus else peak
-    roof_src = ("bf16_tflops_sustained of " if peak_sus else "bf16_tflops (burst) of ") + peak_src
+    clk = clocks.summary()
     dom = "bwd" if bwd_ms > fwd_ms else "fwd"
     dom_ms = bwd_ms if dom == "bwd" else fwd_ms
     dom_fl = fl_b if dom == "bwd" else fl_f
-    achieved = dom_fl / (dom_ms * 1e-3) / 1e12
+    dom_bytes = (F.bwd_bytes if dom == "bwd" else F.fwd_bytes)(T, H, d)
+    roof = roofline(dom_fl, dom_bytes, dom_ms, peaks, peak_src, clk)
+    roof.update(kernel=KERNEL_NAMES[dom], traffic=_traffic(dom, w.name))
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
@@ -696,16 +734,12 @@ def main():
         "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
         "fwd_tflops": fl_f / (fwd_ms * 1e-3) / 1e12 if fwd_ms else None,
         "bwd_tflops": fl_b / (bwd_ms * 1e-3) / 1e12 if bwd_ms else None,
-        "roofline": {"bound": "tensor", "kernel": KERNEL_NAMES[dom], "achieved": achieved,
-                     "peak": roof_peak, "unit": "TFLOP/s", "frac": achieved / roof_peak,
-                     "peak_source": roof_src, "frac_of_burst_peak": achieved / peak,
-                     "traffic": _traffic(dom, w.name),
-                     "algorithmic_flops_per_launch": dom_fl},
+        "roofline": roof,
         "e2e": {"value": world * (fl_f + fl_b) / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": K * (LAUNCHES_PER_STEP["fwd"] +
                              (0 if w.fwd_only else LAUNCHES_PER_STEP["bwd"])),
-        "clocks": clocks.summary(),
+        "clocks": clk,
     }
     if w.fwd_only:
         # M-FALCON candidate scoring on the same batch: only the query tiles that

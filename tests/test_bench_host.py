@@ -60,3 +60,20 @@ def test_source_hash_covers_every_listed_file(tmp_path):
     b.write_text("z")
     assert bench._sha1([str(a), str(b)]) != h1
     assert bench._sha1([str(a), str(tmp_path / "missing.cuh")]) is None
+
+
+def test_roofline_picks_the_bound_and_the_burst_denominator():
+    bench = _bench_module()
+    peaks = {"bf16_tflops": 1600.0, "hbm_gbs": 6400.0, "bf16_tflops_sustained": 1400.0,
+             "clocks_under_load": {"sm_mhz_median": 1300.0}}
+    clk = {"sm_mhz": 1965.0}
+    # ridge = 1600e12 / 6400e9 = 250 FLOP/B
+    t = bench.roofline(800e9, 1e9, 1.0, peaks, "measured", clk)  # AI 800: tensor roof
+    assert t["bound"] == "tensor" and t["unit"] == "TFLOP/s"
+    assert abs(t["achieved"] - 800.0) < 1e-9 and abs(t["frac"] - 0.5) < 1e-12
+    assert t["peak"] == 1600.0 and abs(t["frac_of_sustained_tensor_peak"] - 800 / 1400) < 1e-12
+    assert t["sustained_peak_sm_mhz"] == 1300.0 and t["run_sm_mhz"] == 1965.0
+    h = bench.roofline(100e9, 1e9, 0.5, peaks, "measured", clk)  # AI 100: HBM roof
+    assert h["bound"] == "hbm" and h["unit"] == "GB/s" and h["peak"] == 6400.0
+    assert abs(h["achieved"] - 2000.0) < 1e-9 and abs(h["frac"] - 2000 / 6400) < 1e-12
+    assert abs(h["tensor_tflops"] - 200.0) < 1e-9
