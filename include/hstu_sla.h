@@ -243,6 +243,23 @@ int hstu_sla_count_pairs(const hstu_sla_fwd_params* p, int64_t* row_counts,
  * next hstu_sla_fwd / hstu_sla_bwd / hstu_sla_count_pairs call. */
 int hstu_sla_get_error(const void* workspace, hstu_stream_t stream);
 
+/* Test hook for the bounded-wait failure path (no counterpart in the cited
+ * papers: it exists to show that a stalled kernel gives up instead of
+ * hanging).  Runs the head_dim-128 forward (which = 0; p->fwd.out written) or
+ * one-pass backward (which = 1) on the given inputs with a kernel
+ * instantiation whose pointwise warps each withhold one hand-over arrive, so
+ * the warp waiting for it runs into the limit: after wait_limit_ns (> 0)
+ * the kernel records HSTU_SLA_ERR_TIMEOUT, every role stops, copies and
+ * MMAs in flight drain, TMEM is released and the kernel returns.
+ * hstu_sla_get_error(workspace) then reads HSTU_SLA_ERR_TIMEOUT; the outputs
+ * are unspecified.  The production calls never take this instantiation, and
+ * their limit stays 2 s.  Needs head_dim 128, no relative attention bias,
+ * total_tokens > 0 (else HSTU_SLA_ERR_UNSUPPORTED); workspace as for the
+ * chosen pass. */
+int hstu_sla_test_wait_timeout(const hstu_sla_bwd_params* p, int32_t which,
+                               int64_t wait_limit_ns, void* workspace, size_t workspace_bytes,
+                               hstu_stream_t stream);
+
 /* Static message for a status code. */
 const char* hstu_sla_strerror(int code);
 

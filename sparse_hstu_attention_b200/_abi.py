@@ -23,6 +23,8 @@ WS_FWD = 0
 WS_BWD = 1
 MAX_GROUPS = 4   # HSTU_SLA_MAX_GROUPS
 WS_FWD_FP8 = 2   # hstu_stu_workspace_bytes only: the layer forward with fp8 = 1
+WS_FWD_REMAT = 3  # hstu_stu_workspace_bytes only: the layer forward with remat = 1
+WS_BWD_REMAT = 4  # hstu_stu_workspace_bytes only: the layer backward with remat = 1
 
 
 class FwdParams(ctypes.Structure):
@@ -70,6 +72,7 @@ class StuLayerParams(ctypes.Structure):
         ("av", ctypes.c_void_p), ("y", ctypes.c_void_p), ("stats", ctypes.c_void_p),
         ("fp8", ctypes.c_int32), ("w1q", ctypes.c_void_p), ("w1s", ctypes.c_void_p),
         ("w2q", ctypes.c_void_p), ("w2s", ctypes.c_void_p),
+        ("remat", ctypes.c_int32), ("u", ctypes.c_void_p),
     ]
 
 
@@ -139,6 +142,9 @@ def load():
     lib.hstu_sla_fwd_grouped.restype = ctypes.c_int
     lib.hstu_sla_bwd_grouped.argtypes = [ctypes.POINTER(BwdParams), ctypes.c_int32, vp, sz, vp]
     lib.hstu_sla_bwd_grouped.restype = ctypes.c_int
+    lib.hstu_sla_test_wait_timeout.argtypes = [ctypes.POINTER(BwdParams), ctypes.c_int32,
+                                               ctypes.c_int64, vp, sz, vp]
+    lib.hstu_sla_test_wait_timeout.restype = ctypes.c_int
     lib.hstu_sla_get_error.argtypes = [vp, vp]
     lib.hstu_sla_get_error.restype = ctypes.c_int
     lib.hstu_sla_strerror.argtypes = [ctypes.c_int]

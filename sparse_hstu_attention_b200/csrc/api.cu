@@ -284,6 +284,62 @@ int hstu_sla_get_error(const void* workspace, hstu_stream_t stream) {
   return status;
 }
 
+int hstu_sla_test_wait_timeout(const hstu_sla_bwd_params* p, int32_t which,
+                               int64_t wait_limit_ns, void* workspace, size_t workspace_bytes,
+                               hstu_stream_t stream) {
+  if (p == nullptr || (which != 0 && which != 1) || wait_limit_ns <= 0)
+    return HSTU_SLA_ERR_INVALID_ARG;
+  const hstu_sla_fwd_params* f = &p->fwd;
+  int e = check_common(f);
+  if (e) return e;
+  if (f->d != kFusedBwdD || f->rab_pos || f->rab_time || f->total_tokens == 0)
+    return HSTU_SLA_ERR_UNSUPPORTED;
+  if (which == 0) {
+    if ((e = check_tensor(f->out, f->out_row_stride, f))) return e;
+  } else {
+    if ((e = check_tensor(p->dout, p->dout_row_stride, f))) return e;
+    if ((e = check_tensor(p->dq, p->dq_row_stride, f))) return e;
+    if ((e = check_tensor(p->dk, p->dk_row_stride, f))) return e;
+    if ((e = check_tensor(p->dv, p->dv_row_stride, f))) return e;
+  }
+  if ((e = check_ws(workspace, workspace_bytes,
+                    hstu_sla_workspace_bytes(which ? HSTU_SLA_WS_BWD : HSTU_SLA_WS_FWD,
+                                             f->total_tokens, f->B, f->H, f->d))))
+    return e;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  AttnArgs a = make_args(f, workspace);
+  a.wait_limit_ns = wait_limit_ns;
+  GroupSet gs;
+  memset(&gs, 0, sizeof(gs));
+  gs.common = a.ws;
+  gs.G = 1;
+  gs.stall = 1;
+  cudaError_t ce;
+  if (which == 0) {
+    a.out = static_cast<bf16*>(f->out);
+    a.o_rs = f->out_row_stride;
+    ce = launch_worklist(a, kFwdBM, 0, true, st);
+    gs.g[0] = a;
+    if (ce == cudaSuccess) ce = launch_fwd_grouped(gs, f->d, st);
+  } else {
+    a.cand_only = 0;
+    a.dout = static_cast<const bf16*>(p->dout);
+    a.dq = static_cast<bf16*>(p->dq);
+    a.dk = static_cast<bf16*>(p->dk);
+    a.dv = static_cast<bf16*>(p->dv);
+    a.do_rs = p->dout_row_stride;
+    a.dq_rs = p->dq_row_stride;
+    a.dk_rs = p->dk_row_stride;
+    a.dv_rs = p->dv_row_stride;
+    a.dqacc = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                       ws_bytes(f->total_tokens, f->B));
+    ce = launch_worklist(a, kKvBN, 1, true, st);
+    gs.g[0] = a;
+    if (ce == cudaSuccess) ce = launch_bwd_fused_grouped(gs, st);
+  }
+  return cuda_status(ce);
+}
+
 const char* hstu_sla_strerror(int code) {
   switch (code) {
     case HSTU_SLA_OK: return "ok";

@@ -26,10 +26,11 @@
 // prefix-key units first):
 //   warp 0      scheduler + TMA producer (K double-buffered, V single,
 //               3-stage Q / dO ring)
-//   warp 1      TMEM allocation; one lane issues every UMMA and commit
-//   warps 2..17 pointwise, two groups of eight on alternate steps; then the
-//               dQ drain of their step; at the end of a unit, all sixteen
-//               store dK and dV
+//   warp 1      TMEM allocation; the warp computes every MMA operand, one
+//               elected lane issues each batch of UMMAs and its commits
+//   warps 2..17 pointwise, all sixteen on every step (16 query columns
+//               each); then the dQ drain of the step before; at the end of
+//               a unit, they store dK and dV
 // TMEM columns:
 //   X1(b) = [64b, 64b+64)       S^T (fp32); after the pointwise: per 16-column
 //                               group g, P^T bf16 in [16g, 16g+8) and dS^T
@@ -126,6 +127,12 @@ __device__ void decode_kv_unit(const GroupSet& gs, int u, UnitRec* r) {
   r->nsteps = -1;
 }
 
+// k-step ks of a K-major 128B-swizzled tile whose 64-column boxes are `blk`
+// bytes apart, in the 16-byte units of a descriptor's start address.
+__host__ __device__ constexpr uint32_t koff_k(int ks, int blk) {
+  return (uint32_t)((((ks * 32) / SW) * blk + (ks * 32) % SW) >> 4);
+}
+
 // k, v, q, dout maps of every problem of a launch.
 struct BwdMaps {
   CUtensorMap k[kMaxGroups], v[kMaxGroups], q[kMaxGroups], dout[kMaxGroups];
@@ -170,7 +177,10 @@ __device__ __forceinline__ void red_add_f32(float* p, uint32_t v) { atomicAdd(p,
 // with equal buckets summed by a segmented shuffle scan first
 // (same-address shared atomics from many lanes were the cost).  One
 // pointwise warp flushes the unit's sums into this head's table gradients.
-template <bool RAB>
+// STALL (the wait-timeout test hook only): each pointwise warp withholds its
+// OP_FULL arrive of the first step it processes, so the MMA warp's wait for
+// those operands runs into the launch's wait limit.
+template <bool RAB, bool STALL = false>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_kvq_kernel(const __grid_constant__ BwdMaps maps, const __grid_constant__ GroupSet gs) {
   extern __shared__ uint8_t smem_raw[];
@@ -202,9 +212,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(F_K_FULL + i), 1);
       mbar_init(bar(F_K_EMPTY + i), 1);                // commit after the unit's last dQ MMA
       mbar_init(bar(F_X_FULL + i), 1);
-      mbar_init(bar(F_OP_FULL + i), kPwWarps / 2);     // one arrive per warp of group i
+      mbar_init(bar(F_OP_FULL + i), kPwWarps);         // one arrive per pointwise warp
       mbar_init(bar(F_DQ_FULL + i), 1);
-      mbar_init(bar(F_DQ_EMPTY + i), kPwWarps / 2);
+      mbar_init(bar(F_DQ_EMPTY + i), kPwWarps);
     }
     mbar_init(bar(F_V_FULL), 1);
     mbar_init(bar(F_V_EMPTY), 1);                      // commit after the unit's last X MMA
@@ -316,11 +326,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // --------------------------------------------------------- MMA issuer
-    // One lane.  Step n: the S^T MMAs into X1, then (once the dQ^T two steps
-    // back has been read out of X2) the dP^T MMAs into X2; then the MMAs of
-    // step n - 1 that consume its bf16 P^T / dS^T: dQ^T first (its drain
-    // overlaps the rest), then dV and dK.
-    if (lane == 0) {
+    // The whole warp walks the schedule and computes every operand (TMEM
+    // addresses, descriptor bases, barrier addresses) together, so they are
+    // warp-uniform; one elected lane then issues each batch of UMMAs with
+    // only immediate offsets added, and the commits that close it.  A lone
+    // lane (a divergent branch) pays ~60 clk per tcgen05.mma against ~10 here.
+    // Step n: the S^T MMAs into X1, then (once the dQ^T two steps back has
+    // been read out of X2) the dP^T MMAs into X2; then the MMAs of step n - 1
+    // that consume its bf16 P^T / dS^T: dQ^T first (its drain overlaps the
+    // rest), then dV and dK.
+    {
       uint32_t an = 0, bn = 0, xc = 0, accn = 0;
       bool ok = true;
       // Descriptor bases; offsets only add to the start-address field.
@@ -333,74 +348,85 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t mB2 = smem_desc(sB2, SBLK, SBO, kSwizzle128B);
       // dS^T is one 128-byte-wide box: the leading byte offset is never used
       const uint64_t dDS = smem_desc(sDS, DSTILE, SBO, kSwizzle128B);
-      auto koff = [](int ks, int blk) -> uint32_t {  // k-step ks of a K-major tile, 16-byte units
-        return (uint32_t)((((ks * 32) / SW) * blk + (ks * 32) % SW) >> 4);
-      };
       constexpr uint32_t kRows16 = (16 * SW) >> 4;  // 16 rows of an MN-major tile, 16-byte units
       // MMAs of the step with ring counter bm / X counter xm, K buffer kb
       auto acc = [&](uint32_t bm, uint32_t xm, uint32_t kb, bool first, bool last) -> bool {
         const uint32_t b = xm & 1;
-        if (!mbar_wait(bar(F_OP_FULL + b), (xm >> 1) & 1, ws)) return false;
-        if (first && !mbar_wait(bar(F_ACC_EMPTY), (accn & 1) ^ 1, ws)) return false;
+        if (!warp_wait(bar(F_OP_FULL + b), (xm >> 1) & 1, ws)) return false;
+        if (first && !warp_wait(bar(F_ACC_EMPTY), (accn & 1) ^ 1, ws)) return false;
         tc_fence_after();
-        const uint64_t dKt = dKt0 + ((kb * RTILE) >> 4);
-        const uint64_t dS = dDS + ((b * DSTILE) >> 4);
-#pragma unroll
-        for (int ks = 0; ks < kRes / 16; ++ks)  // dQ^T = K^T dS^T over the read-out dP^T
-          mma_ss(tmem + kColX2 + b * 64, dKt + ks * kRows16, dS + ks * kRows16, IDESC_DQ,
-                 ks > 0 ? 1u : 0u);
-        tc_commit(bar(F_DQ_FULL + b));
-        if (last) tc_commit(bar(F_K_EMPTY + kb));  // last use of this K buffer
         const int s = bm % kSt;
         const uint32_t so = (uint32_t)(s * STILE) >> 4;
+        const uint64_t aq = dKt0 + ((kb * RTILE) >> 4), bq = dDS + ((b * DSTILE) >> 4);
+        const uint64_t b1 = mB1 + so, b2 = mB2 + so;
+        const uint32_t dq_t = tmem + kColX2 + b * 64, x1 = tmem + kColX1 + b * 64;
+        const uint32_t bar_dq = bar(F_DQ_FULL + b), bar_k = bar(F_K_EMPTY + kb);
+        const uint32_t bar_b = bar(F_B_EMPTY + s);
+        const uint32_t acc0 = first ? 0u : 1u;
+        if (elect_one()) {
 #pragma unroll
-        for (int ks = 0; ks < kStr / 16; ++ks) {
-          const uint32_t accum = (!first || ks > 0) ? 1u : 0u;
-          const uint32_t ko = so + ks * kRows16;
-          // queries [16 ks, +16): P^T at columns 32 (ks / 2) + 16 (ks % 2), dS^T 8 further
-          const uint32_t xo = b * 64 + (ks >> 1) * 32 + (ks & 1) * 16;
-          mma_ts(tmem + kColAcc1, tmem + kColX1 + xo, mB2 + ko, IDESC_ACC, accum);      // dV += P^T dO
-          mma_ts(tmem + kColAcc2, tmem + kColX1 + xo + 8, mB1 + ko, IDESC_ACC, accum);  // dK += dS^T Q
+          for (int ks = 0; ks < kRes / 16; ++ks)  // dQ^T = K^T dS^T over the read-out dP^T
+            mma_ss(dq_t, aq + ks * kRows16, bq + ks * kRows16, IDESC_DQ, ks > 0 ? 1u : 0u);
+          tc_commit(bar_dq);
+          if (last) tc_commit(bar_k);  // last use of this K buffer
+#pragma unroll
+          for (int ks = 0; ks < kStr / 16; ++ks) {
+            // queries [16 ks, +16): P^T at columns 32 (ks / 2) + 16 (ks % 2), dS^T 8 further
+            const uint32_t xo = (ks >> 1) * 32 + (ks & 1) * 16;
+            mma_ts(tmem + kColAcc1, x1 + xo, b2 + ks * kRows16, IDESC_ACC,
+                   ks > 0 ? 1u : acc0);  // dV += P^T dO
+            mma_ts(tmem + kColAcc2, x1 + xo + 8, b1 + ks * kRows16, IDESC_ACC,
+                   ks > 0 ? 1u : acc0);  // dK += dS^T Q
+          }
+          tc_commit(bar_b);
         }
-        tc_commit(bar(F_B_EMPTY + s));
+        __syncwarp();
         return true;
       };
       for (int kk = 0; ok; ++kk) {
         const int slot = kk % kUSlots;
-        ok = mbar_wait(bar(F_U_FULL + slot), (kk / kUSlots) & 1, ws);
+        ok = warp_wait(bar(F_U_FULL + slot), (kk / kUSlots) & 1, ws);
         if (!ok) break;
-        const int nt = ring[slot].nsteps;
-        mbar_arrive(bar(F_U_EMPTY + slot));
+        const int nt = __shfl_sync(0xffffffffu, ring[slot].nsteps, 0);
+        warp_arrive(bar(F_U_EMPTY + slot));
         if (nt < 0) break;
         if (nt == 0) continue;
         const uint32_t kb = an & 1;
-        ok = mbar_wait(bar(F_K_FULL + kb), (an >> 1) & 1, ws) &&
-             mbar_wait(bar(F_V_FULL), an & 1, ws);
+        ok = warp_wait(bar(F_K_FULL + kb), (an >> 1) & 1, ws) &&
+             warp_wait(bar(F_V_FULL), an & 1, ws);
         if (!ok) break;
         tc_fence_after();
         const uint64_t dK = dK0 + ((kb * RTILE) >> 4);
         const uint32_t bn0 = bn, xc0 = xc;
         for (int n = 0; n < nt; ++n) {
           const int s = bn % kSt;
-          ok = mbar_wait(bar(F_B_FULL + s), (bn / kSt) & 1, ws);
+          ok = warp_wait(bar(F_B_FULL + s), (bn / kSt) & 1, ws);
           if (!ok) break;
           tc_fence_after();
           const uint32_t b = xc & 1;
           const uint32_t so = (uint32_t)(s * STILE) >> 4;
+          const uint64_t bq = dB1 + so, bo = dB2 + so;
+          const uint32_t x1 = tmem + kColX1 + b * 64, x2 = tmem + kColX2 + b * 64;
+          if (elect_one()) {
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks)  // S^T = K Q^T
-            mma_ss(tmem + kColX1 + b * 64, dK + koff(ks, RBLK), dB1 + so + koff(ks, SBLK), IDESC_X,
-                   ks > 0 ? 1u : 0u);
+            for (int ks = 0; ks < D / 16; ++ks)  // S^T = K Q^T
+              mma_ss(x1, dK + koff_k(ks, RBLK), bq + koff_k(ks, SBLK), IDESC_X, ks > 0 ? 1u : 0u);
+          }
+          __syncwarp();
           // X2(b) still holds the dQ^T of step xc - 2 until its drain is done
-          ok = mbar_wait(bar(F_DQ_EMPTY + b), ((xc >> 1) & 1) ^ 1, ws);
+          ok = warp_wait(bar(F_DQ_EMPTY + b), ((xc >> 1) & 1) ^ 1, ws);
           if (!ok) break;
           tc_fence_after();
+          const uint32_t bar_x = bar(F_X_FULL + b), bar_v = bar(F_V_EMPTY);
+          const bool last_v = n + 1 == nt;
+          if (elect_one()) {
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks)  // dP^T = V dO^T
-            mma_ss(tmem + kColX2 + b * 64, dV + koff(ks, RBLK), dB2 + so + koff(ks, SBLK), IDESC_X,
-                   ks > 0 ? 1u : 0u);
-          tc_commit(bar(F_X_FULL + b));
-          if (n + 1 == nt) tc_commit(bar(F_V_EMPTY));  // last use of V
+            for (int ks = 0; ks < D / 16; ++ks)  // dP^T = V dO^T
+              mma_ss(x2, dV + koff_k(ks, RBLK), bo + koff_k(ks, SBLK), IDESC_X, ks > 0 ? 1u : 0u);
+            tc_commit(bar_x);
+            if (last_v) tc_commit(bar_v);  // last use of V
+          }
+          __syncwarp();
           if (n > 0) {
             ok = acc(bn - 1, xc - 1, kb, n == 1, false);
             if (!ok) break;
@@ -411,35 +437,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         ok = acc(bn0 + nt - 1, xc0 + nt - 1, kb, nt == 1, true);
         if (!ok) break;
-        tc_commit(bar(F_ACC_FULL));
+        if (elect_one()) tc_commit(bar(F_ACC_FULL));
+        __syncwarp();
         ++an;
         ++accn;
       }
-      tc_commit(bar(F_DRAIN));
+      if (elect_one()) tc_commit(bar(F_DRAIN));
+      __syncwarp();
       drain_wait(bar(F_DRAIN), 0);
     }
     __syncwarp();
   } else {
     // ------------------------------------------------ pointwise + drains
-    // Two groups of eight warps take alternate steps (group g owns X buffer
-    // g); the two warps of a group on one 32-lane TMEM quarter split the
-    // step's 64 query columns in halves.  Per step a warp turns its 32 scores
-    // per key into P^T and dS^T (bf16, TMEM), copies dS^T into shared memory
-    // for the dQ MMA, and once that MMA is done reads its 32 dQ^T columns
-    // (query rows) for the 32 head-dim lanes of its quarter and adds them to
-    // the fp32 workspace.  Unit epilogue: warp `chunk` of a quarter stores
-    // accumulator columns [32 chunk, +32) of dV and dK.
+    // All sixteen warps work on every step: the four warps on one 32-lane
+    // TMEM quarter split the step's 64 query columns in chunks of 16 (the
+    // step's pointwise latency, which the MMA of the step after next waits
+    // for, is that of one 16-column round).  Per step a warp turns its 16
+    // scores per key into P^T and dS^T (bf16, TMEM) and copies dS^T into
+    // shared memory for the dQ MMA; then it drains the PREVIOUS step's dQ^T
+    // (done by now: the MMA lane issued it right after this step's dP^T),
+    // reading its 16 columns (query rows) for the 32 head-dim lanes of its
+    // quarter and adding them to the fp32 workspace, so no warp ever waits
+    // for a dQ^T.  A unit's last dQ^T is drained before its epilogue.  Unit
+    // epilogue: warp `chunk` of a quarter stores accumulator columns
+    // [32 chunk, +32) of dV and dK.
     const int pw = warp - kPwWarp0;
-    const int grp = pw >> 3;              // X buffer / step parity of this warp
     const int quarter = warp & 3;
     const int chunk = pw >> 2;            // 0..3
-    const int half = chunk & 1;           // query-column half within the group
     const int row = quarter * 32 + lane;  // key row (and head-dim lane of dQ^T)
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-    const int col = half * 32;
+    const int col = chunk * 16;           // this warp's query columns of a step
     const uint32_t ds_row = sDS + (uint32_t)row * SW;
     const uint32_t swz = (uint32_t)(row & 7);
     uint32_t xc = 0, accn = 0;
+    bool withhold = STALL;  // the test hook's one withheld arrive
     uint32_t hu = 0;  // units with steps so far (histogram buffer hu & 1)
     bool ok = true;
     for (int kk = 0; ok; ++kk) {
@@ -514,11 +545,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         sum = c ? g : sum + g;
         run = bin;
       };
+      // Reads step xd's dQ^T (first query row q0) out of X2 and adds this
+      // warp's 16 rows of it to the workspace; rows past the sequence end are
+      // skipped.
+      auto drain = [&](uint32_t xd, int q0) -> bool {
+        const uint32_t bb = xd & 1;
+        if (!warp_wait(bar(F_DQ_FULL + bb), (xd >> 1) & 1, ws)) return false;
+        tc_fence_after();
+        uint32_t g[16];
+        tmem_ld16(lane_base + kColX2 + bb * 64 + col, g);
+        tmem_ld_wait(g);
+        tc_fence_before();
+        warp_arrive(bar(F_DQ_EMPTY + bb));
+        const int qq = q0 + col;
+        const int nv = L - qq;
+        float* p = dqa + (int64_t)qq * D;
+        if (nv >= 16) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) red_add_f32(p + e * D, g[e]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            if (e < nv) red_add_f32(p + e * D, g[e]);
+        }
+        return true;
+      };
+      int prev_c0 = 0;  // first query row of the previous step of this unit
       SpanCursor c;
       c.begin(r);
       for (int n = 0; n < nt; ++n, ++xc, c.next(r)) {
         const uint32_t b = xc & 1;
-        if ((int)b != grp) continue;  // the other group's step
         ok = warp_wait(bar(F_X_FULL + b), (xc >> 1) & 1, ws);
         if (!ok) break;
         tc_fence_after();
@@ -528,22 +584,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t xd_addr = lane_base + kColX2 + b * 64 + col;
         const uint32_t dsr = ds_row + b * DSTILE;
         // Fully visible tiles skip the mask; others clear invisible entries by
-        // one bit test against this key's 32-row visibility mask.
+        // one bit test against this key's visibility mask of the chunk's rows.
         const uint32_t bits = full ? 0xFFFFFFFFu : key_mask_bits(km, c0 + col);
-        // relative attention bias: the 32 queries' timestamps (one per lane)
+        // relative attention bias: the 16 queries' timestamps (lanes 0..15)
         int32_t tql = 0;
         bool tq_ok = false;  // this lane's query column is in the sequence
         if constexpr (RAB) {
           const int ql = c0 + col + lane;
-          tq_ok = ql < L;
+          tq_ok = lane < 16 && ql < L;
           tql = (A.ts && tq_ok) ? __ldg(A.ts + s0 + ql) : 0;
         }
-        // Two rounds of 16 query columns each (fewer live registers).  Round r
-        // writes P^T (8 packed columns) then dS^T (8) over the 16 score
-        // columns it read, and copies dS^T to 16-byte chunks half*4 + 2r,
-        // +1 of this key's 128-byte swizzled row of the dS^T tile.
+        // One round of the chunk's 16 query columns: P^T (8 packed columns)
+        // then dS^T (8) over the 16 score columns it read, and dS^T copied to
+        // 16-byte chunks 2 chunk, +1 of this key's 128-byte swizzled row of
+        // the dS^T tile.
 #pragma unroll
-        for (int r = 0; r < 2; ++r) {
+        for (int r = 0; r < 1; ++r) {
           uint32_t xs[16], xd[16], pp[8], dd[8];
           tmem_ld16(xs_addr + 16 * r, xs);
           tmem_ld16(xd_addr + 16 * r, xd);
@@ -639,15 +695,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!full) {
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-              pp[e] = mask_pair(pp[e], bits, 8 * r + e);
-              dd[e] = mask_pair(dd[e], bits, 8 * r + e);
+              pp[e] = mask_pair(pp[e], bits, e);
+              dd[e] = mask_pair(dd[e], bits, e);
             }
           }
           tmem_st8(xs_addr + 16 * r, pp);
           tmem_st8(xs_addr + 16 * r + 8, dd);
 #pragma unroll
           for (int q = 0; q < 2; ++q)
-            st_shared_v4(dsr + ((((uint32_t)(half * 4 + 2 * r + q)) ^ swz) << 4), dd[4 * q],
+            st_shared_v4(dsr + ((((uint32_t)(2 * chunk + q)) ^ swz) << 4), dd[4 * q],
                          dd[4 * q + 1], dd[4 * q + 2], dd[4 * q + 3]);
         }
         if constexpr (RAB) {  // the step's finished runs, equal bins added up first
@@ -659,35 +715,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();  // visible to the dQ MMA
         tmem_st_wait();
         tc_fence_before();
-        warp_arrive(bar(F_OP_FULL + b));
-        // ------------------------------------------- dQ^T of this step
-        ok = warp_wait(bar(F_DQ_FULL + b), (xc >> 1) & 1, ws);
-        if (!ok) break;
-        tc_fence_after();
-        uint32_t g0[16], g1[16];
-        tmem_ld16(xd_addr, g0);
-        tmem_ld16(xd_addr + 16, g1);
-        tmem_ld_wait2(g0, g1);
-        tc_fence_before();
-        warp_arrive(bar(F_DQ_EMPTY + b));
-        // column e is query row c0 + col + e; rows past the sequence end are skipped
-        const int q0 = c0 + col;
-        const int nv = L - q0;
-        float* p = dqa + q0 * D;
-        if (nv >= 32) {
-#pragma unroll
-          for (int e = 0; e < 16; ++e) red_add_f32(p + e * D, g0[e]);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) red_add_f32(p + (16 + e) * D, g1[e]);
-        } else {
-#pragma unroll
-          for (int e = 0; e < 16; ++e)
-            if (e < nv) red_add_f32(p + e * D, g0[e]);
-#pragma unroll
-          for (int e = 0; e < 16; ++e)
-            if (16 + e < nv) red_add_f32(p + (16 + e) * D, g1[e]);
+        if (!withhold) warp_arrive(bar(F_OP_FULL + b));
+        withhold = false;
+        // the previous step's dQ^T, issued right after this step's dP^T
+        if (n > 0) {
+          ok = drain(xc - 1, prev_c0);
+          if (!ok) break;
         }
+        prev_c0 = c0;
       }
+      if (!ok) break;
+      ok = drain(xc - 1, prev_c0);  // the unit's last step
       if (!ok) break;
       // ---------------------------------------------------------- epilogue
       ok = warp_wait(bar(F_ACC_FULL), accn & 1, ws);
@@ -901,7 +939,8 @@ cudaError_t launch_bwd_fused_grouped(const GroupSet& gs, cudaStream_t st) {
     units += max_items(a.T, a.B) * a.H;
   }
   if (units == 0) return cudaSuccess;
-  const auto kern = rab ? bwd_kvq_kernel<true> : bwd_kvq_kernel<false>;
+  auto kern = rab ? bwd_kvq_kernel<true> : bwd_kvq_kernel<false>;
+  if (gs.stall) kern = bwd_kvq_kernel<false, true>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
   if (e != cudaSuccess) return e;
   const int sms = device_sm_count();

@@ -121,7 +121,10 @@ struct FwdMaps {
 };
 
 // RAB: add the relative attention bias to every score (AttnArgs::rab_*).
-template <int D, bool RAB>
+// STALL (the wait-timeout test hook only): each pointwise warp withholds
+// its P_FULL arrive of the first tile it processes, so the MMA warp's wait
+// for that P runs into the launch's wait limit.
+template <int D, bool RAB, bool STALL = false>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_tc_kernel(const __grid_constant__ FwdMaps maps, const __grid_constant__ GroupSet gs) {
   using C = Cfg<D>;
@@ -300,15 +303,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------- MMA issuer
-    // One lane runs this role alone: a tcgen05.mma costs its issuing thread
-    // about as long as the tensor pipe takes to execute it, so every wait and
-    // commit here is kept single-threaded and per tile there are only two
-    // commits (S_FULL, which also frees the K slot, and V_EMPTY).
+    // The whole warp runs this role converged and computes every descriptor
+    // together (warp-uniform values); one elected lane issues each UMMA and
+    // commit.  Per tile there are only two commits (S_FULL, which also frees
+    // the K slot, and V_EMPTY).
     // Tiles are numbered across units: tile t uses score buffer t % 3, K slot
     // t % kKSt and V slot t % kVSt; its P V is issued once S of tile t + 2 is
-    // issued, or earlier while the lane waits for a copy, so P V of a unit's
+    // issued, or earlier while the warp waits for a copy, so P V of a unit's
     // last tiles overlaps S of the next unit's first.
-    if (lane == 0) {
+    {
+      constexpr uint32_t kAll = 0xffffffffu;
       uint32_t qn = 0, tc = 0, pvc = 0, on = 0;
       uint32_t pend = 0;  // 2 bits per tile in [pvc, tc): first / last of its unit
       bool ok = true;
@@ -320,7 +324,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto kstep = [](int ks) -> uint32_t {  // byte offset of k-step ks in a K-major tile
         return (uint32_t)(((ks * 32) / C::SW) * C::BLK + (ks * 32) % C::SW);
       };
-      // O += P V for tile pvc, its operands known to be ready.
+      auto commit = [&](uint32_t b) {
+        if (elect_one()) tc_commit(b);
+        __syncwarp();
+      };
+      // O += P V for tile pvc, its operands known to be ready.  Every operand
+      // is computed by the whole warp (warp-uniform); one elected lane issues
+      // the batch with immediate offsets only (a lone lane in a divergent
+      // branch pays ~60 clk per tcgen05.mma against ~10 here).
       auto pv_issue = [&]() {
         const uint32_t f = pend & 3u;
         pend >>= 2;
@@ -329,27 +340,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = pvc % kVSt;
         tc_fence_after();
         const uint64_t dv = dV + ((uint32_t)(s * C::TILE) >> 4);
+        const uint32_t pa = tmem + kColS + b * 128;
+        const uint32_t acc0 = first ? 0u : 1u;
+        const uint32_t bar_v = bar(BAR_V_EMPTY + s), bar_o = bar(BAR_O_FULL);
+        if (elect_one()) {
 #pragma unroll
-        for (int ks = 0; ks < kBN / 16; ++ks)
-          mma_ts(tmem + kColO, tmem + kColS + b * 128 + (ks >> 1) * 32 + (ks & 1) * 8,
-                 dv + ((uint32_t)(ks * 16 * C::SW) >> 4), C::IDESC_O,
-                 (first && ks == 0) ? 0u : 1u);
-        tc_commit(bar(BAR_V_EMPTY + s));
-        if (last) {
-          tc_commit(bar(BAR_O_FULL));
-          ++on;
+          for (int ks = 0; ks < kBN / 16; ++ks)
+            mma_ts(tmem + kColO, pa + (ks >> 1) * 32 + (ks & 1) * 8,
+                   dv + ((uint32_t)(ks * 16 * C::SW) >> 4), C::IDESC_O, ks > 0 ? 1u : acc0);
+          tc_commit(bar_v);
+          if (last) tc_commit(bar_o);
         }
+        __syncwarp();
+        if (last) ++on;
         ++pvc;
       };
       auto pv_ready = [&]() -> bool {  // P, V (and O, for a unit's first) of tile pvc
-        return mbar_test_wait(bar(BAR_P_FULL + pvc % kSBufs), (pvc / kSBufs) & 1) &&
-               mbar_test_wait(bar(BAR_V_FULL + pvc % kVSt), (pvc / kVSt) & 1) &&
-               ((pend & 1u) == 0 || mbar_test_wait(bar(BAR_O_EMPTY), (on & 1) ^ 1));
+        return __all_sync(
+            kAll, mbar_test_wait(bar(BAR_P_FULL + pvc % kSBufs), (pvc / kSBufs) & 1) &&
+                      mbar_test_wait(bar(BAR_V_FULL + pvc % kVSt), (pvc / kVSt) & 1) &&
+                      ((pend & 1u) == 0 || mbar_test_wait(bar(BAR_O_EMPTY), (on & 1) ^ 1)));
       };
       auto pv = [&]() -> bool {  // blocking form
-        if (!mbar_wait(bar(BAR_P_FULL + pvc % kSBufs), (pvc / kSBufs) & 1, ws)) return false;
-        if (!mbar_wait(bar(BAR_V_FULL + pvc % kVSt), (pvc / kVSt) & 1, ws)) return false;
-        if ((pend & 1u) && !mbar_wait(bar(BAR_O_EMPTY), (on & 1) ^ 1, ws)) return false;
+        if (!warp_wait(bar(BAR_P_FULL + pvc % kSBufs), (pvc / kSBufs) & 1, ws)) return false;
+        if (!warp_wait(bar(BAR_V_FULL + pvc % kVSt), (pvc / kVSt) & 1, ws)) return false;
+        if ((pend & 1u) && !warp_wait(bar(BAR_O_EMPTY), (on & 1) ^ 1, ws)) return false;
         pv_issue();
         return true;
       };
@@ -359,21 +374,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       // its Q buffer or ring slot) can depend on deferred P V, so they must
       // never sit behind such a wait.
       auto wait_issuing = [&](uint32_t b, uint32_t parity) -> bool {
-        if (mbar_test_wait(b, parity)) return true;
+        if (__all_sync(kAll, mbar_test_wait(b, parity))) return true;
         const uint64_t t0 = globaltimer();
         for (uint32_t it = 1;; ++it) {
-          // try_wait may suspend this lane in hardware until the phase
+          // try_wait may suspend the warp in hardware until the phase
           // completes, leaving the issue slots of its sub-partition to the
           // pointwise warps there; deferred P V readiness is polled between
-          if (mbar_try_wait(b, parity)) return true;
+          if (__all_sync(kAll, mbar_try_wait(b, parity))) return true;
           if (pvc != tc && pv_ready()) {
             pv_issue();
             continue;
           }
           if ((it & 255u) == 0) {
-            if (load_status(ws) != 0) return false;
-            if (globaltimer() - t0 > kWaitLimitNs) {
-              set_status(ws, HSTU_SLA_ERR_TIMEOUT);
+            if (__any_sync(kAll, load_status(ws) != 0)) return false;
+            if (__any_sync(kAll, globaltimer() - t0 > wait_limit(ws, kWaitLimitNs))) {
+              if (lane == 0) set_status(ws, HSTU_SLA_ERR_TIMEOUT);
               return false;
             }
           }
@@ -383,8 +398,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int slot = kk % kUSlots;
         ok = wait_issuing(bar(BAR_U_FULL + slot), (kk / kUSlots) & 1);
         if (!ok) break;
-        const int nt = ring[slot].nsteps;
-        mbar_arrive(bar(BAR_U_EMPTY + slot));
+        const int nt = __shfl_sync(kAll, ring[slot].nsteps, 0);
+        warp_arrive(bar(BAR_U_EMPTY + slot));
         if (nt < 0) break;
         if (nt == 0) continue;
         const uint32_t qb = qn & 1;
@@ -398,12 +413,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint32_t b = tc % kSBufs;
           const uint64_t dk = dK + ((uint32_t)(s * C::TILE) >> 4);
+          const uint64_t dq = dQ + ((uint32_t)(qb * C::TILE) >> 4);
+          const uint32_t sd = tmem + kColS + b * 128;
+          const uint32_t bar_s = bar(BAR_S_FULL + b), bar_q = bar(BAR_Q_EMPTY + qb);
+          const bool last_q = n + 1 == nt;
+          if (elect_one()) {
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks)
-            mma_ss(tmem + kColS + b * 128, dQ + ((qb * C::TILE + kstep(ks)) >> 4),
-                   dk + (kstep(ks) >> 4), C::IDESC_S, ks > 0 ? 1u : 0u);
-          tc_commit(bar(BAR_S_FULL + b));
-          if (n + 1 == nt) tc_commit(bar(BAR_Q_EMPTY + qb));  // last S read of this Q tile
+            for (int ks = 0; ks < D / 16; ++ks)
+              mma_ss(sd, dq + (kstep(ks) >> 4), dk + (kstep(ks) >> 4), C::IDESC_S,
+                     ks > 0 ? 1u : 0u);
+            tc_commit(bar_s);
+            if (last_q) tc_commit(bar_q);  // last S read of this Q tile
+          }
+          __syncwarp();
           pend |= ((n == 0 ? 1u : 0u) | (n + 1 == nt ? 2u : 0u)) << (2 * (tc - pvc));
           ++tc;
           // the score buffer of tile tc (next S) is free once P V of tc - 3
@@ -417,7 +439,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       while (ok && pvc != tc) ok = pv();
       // Every MMA issued must finish before TMEM is released.
-      tc_commit(bar(BAR_DRAIN));
+      commit(bar(BAR_DRAIN));
       drain_wait(bar(BAR_DRAIN), 0);
     }
     __syncwarp();
@@ -452,6 +474,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // epilogue and Q-buffer release completes before the warp waits on a
     // tile of the unit after next, whose Q load depends on them.
     uint32_t tc = 0, on = 0, qn = 0;
+    bool withhold = STALL;  // the test hook's one withheld arrive
     bool ep_pend = false;
     int e_h = 0, e_s0 = 0, e_t0 = 0, e_t1 = 0, e_slot = 0, e_grp = 0;
     uint32_t e_qn = 0;
@@ -632,7 +655,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_st_wait();
         tc_fence_before();
-        warp_arrive(bar(BAR_P_FULL + b));
+        if (!withhold) warp_arrive(bar(BAR_P_FULL + b));
+        withhold = false;
         if (ep_pend) {
           ok = epilogue();
           if (!ok) break;
@@ -683,7 +707,11 @@ cudaError_t launch_d(const GroupSet& gs, cudaStream_t st) {
   if (units == 0) return cudaSuccess;
   bool rab = false;  // any problem with a relative attention bias takes the bias kernel
   for (int p = 0; p < gs.G; ++p) rab = rab || gs.g[p].rab_pos != nullptr || gs.g[p].rab_time != nullptr;
-  const auto kern = rab ? fwd_tc_kernel<D, true> : fwd_tc_kernel<D, false>;
+  auto kern = rab ? fwd_tc_kernel<D, true> : fwd_tc_kernel<D, false>;
+  if (gs.stall) {
+    if constexpr (D == 128) kern = fwd_tc_kernel<D, false, true>;
+    else return cudaErrorInvalidValue;
+  }
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   const int sms = device_sm_count();

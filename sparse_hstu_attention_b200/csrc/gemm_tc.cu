@@ -200,7 +200,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == 1) {
     // --------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    // The whole warp computes every operand (warp-uniform); one elected lane
+    // issues each k block's UMMAs with immediate offsets and its commit.
+    {
       constexpr uint32_t IDESC = F8 ? idesc_e4m3(kBM, kBN) : idesc_bf16(kBM, kBN, A_MN, B_MN);
       // K-major: a 16-wide k step moves 32 bytes inside the 128-byte row;
       // MN-major: it moves 16 rows of 128 bytes.  Units of 16 bytes.
@@ -215,29 +217,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         const TileInfo ti = tile_info(g, t, tiles_m, tiles_n, kBKe);
         if (ti.nkb == 0) continue;
         const uint32_t buf = tc & 1;
-        ok = mbar_wait(bar(G_ACC_EMPTY + buf), ((tc >> 1) & 1) ^ 1, g.ws);
+        ok = warp_wait(bar(G_ACC_EMPTY + buf), ((tc >> 1) & 1) ^ 1, g.ws);
         if (!ok) break;
         tc_fence_after();
+        const uint32_t acc_t = tmem + buf * kBN;
         for (int kb = 0; kb < ti.nkb; ++kb, ++it) {
           const int s = it % kStages;
-          ok = mbar_wait(bar(G_FULL + s), (it / kStages) & 1, g.ws);
+          ok = warp_wait(bar(G_FULL + s), (it / kStages) & 1, g.ws);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t ao = (uint32_t)(s * A_TILE) >> 4, bo = (uint32_t)(s * B_TILE) >> 4;
-          // four 32-byte k steps per 128-byte block (16 bf16 or 32 8-bit values each)
+          const uint64_t a = dA + ((uint32_t)(s * A_TILE) >> 4);
+          const uint64_t b = dB + ((uint32_t)(s * B_TILE) >> 4);
+          const uint32_t acc0 = kb > 0 ? 1u : 0u;
+          const uint32_t bar_e = bar(G_EMPTY + s);
+          if (elect_one()) {
+            // four 32-byte k steps per 128-byte block (16 bf16 or 32 8-bit values each)
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            if constexpr (F8)
-              mma_ss_f8(tmem + buf * kBN, dA + ao + ks * kStepA, dB + bo + ks * kStepB, IDESC,
-                        (kb > 0 || ks > 0) ? 1u : 0u);
-            else
-              mma_ss(tmem + buf * kBN, dA + ao + ks * kStepA, dB + bo + ks * kStepB, IDESC,
-                     (kb > 0 || ks > 0) ? 1u : 0u);
+            for (int ks = 0; ks < 4; ++ks) {
+              if constexpr (F8)
+                mma_ss_f8(acc_t, a + ks * kStepA, b + ks * kStepB, IDESC, ks > 0 ? 1u : acc0);
+              else
+                mma_ss(acc_t, a + ks * kStepA, b + ks * kStepB, IDESC, ks > 0 ? 1u : acc0);
+            }
+            tc_commit(bar_e);
           }
-          tc_commit(bar(G_EMPTY + s));
+          __syncwarp();
         }
         if (!ok) break;
-        tc_commit(bar(G_ACC_FULL + buf));
+        if (elect_one()) tc_commit(bar(G_ACC_FULL + buf));
+        __syncwarp();
         ++tc;
       }
     }

@@ -34,7 +34,9 @@ struct WsHeader {
   int32_t n_items2_pre;  // leading entries of list 1 that hold prefix key tiles
   int32_t sched;         // dynamic scheduler counter over list 0 units
   int32_t sched2;        // dynamic scheduler counter over list 1 units
-  int32_t pad[58];
+  int32_t pad0[2];
+  int64_t wait_limit_ns; // bounded-wait limit of the launch's kernels (0: the default)
+  int32_t pad[54];
 };
 static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 
@@ -119,6 +121,9 @@ struct AttnArgs {
   int nbp, nbt;
   float* d_rab_pos;
   float* d_rab_time;
+  // Bounded-wait limit the work-list kernel records for the launch (0: the
+  // kernels' default); only the wait-timeout test hook sets it.
+  int64_t wait_limit_ns;
 };
 
 // Relative attention bias, with the tables held in registers: lane b of a
@@ -411,6 +416,12 @@ __device__ __forceinline__ int load_status(const WsHeader* ws) {
   return *((volatile const int32_t*)&ws->status);
 }
 
+// The launch's bounded-wait limit in ns (`dflt` unless the header sets one).
+__device__ __forceinline__ uint64_t wait_limit(const WsHeader* ws, uint64_t dflt) {
+  const int64_t v = *((volatile const int64_t*)&ws->wait_limit_ns);
+  return v > 0 ? (uint64_t)v : dflt;
+}
+
 // ------------------------------------------------------------ host launchers
 // (defined in the .cu files; return cudaError_t of the launch)
 // list 0: (sequence, query tile of `tile` rows); list 1: (sequence, key tile
@@ -428,6 +439,10 @@ struct GroupSet {
   AttnArgs g[kMaxGroups];
   WsHeader* common;
   int G;
+  // Wait-timeout test hook only: the launch takes the kernel instantiation
+  // whose pointwise warps withhold their first hand-over arrive, so that the
+  // role waiting for it runs into the bounded-wait limit.
+  int stall;
 };
 cudaError_t launch_fwd_grouped(const GroupSet& gs, int d, cudaStream_t st);
 // The backward entry point with the STU layer's SiLU' / bias-gradient fusion

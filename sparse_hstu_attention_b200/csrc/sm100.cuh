@@ -65,8 +65,9 @@ __device__ __forceinline__ uint64_t globaltimer() {
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far beyond any legitimate wait
 
 // Waits for the phase of parity `parity` of barrier `bar` to complete.  Gives
-// up (returns false) if another role already reported an error, or after
-// kWaitLimitNs, in which case it records HSTU_SLA_ERR_TIMEOUT.
+// up (returns false) if another role already reported an error, or after the
+// launch's wait limit (kWaitLimitNs unless the header sets a shorter one), in
+// which case it records HSTU_SLA_ERR_TIMEOUT.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, WsHeader* ws) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
@@ -74,7 +75,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, WsHeade
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 255u) == 0) {
       if (load_status(ws) != 0) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) {
+      if (globaltimer() - t0 > wait_limit(ws, kWaitLimitNs)) {
         set_status(ws, HSTU_SLA_ERR_TIMEOUT);
         return false;
       }
@@ -92,6 +93,18 @@ __device__ __forceinline__ void warp_arrive(uint32_t bar) {
 // mbar_wait by every lane of a warp, with a warp-uniform result.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, WsHeader* ws) {
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, ws));
+}
+
+// One lane of a converged warp (the same lane every time the whole warp
+// executes it): the issuer of tcgen05.mma / commit in warp-converged MMA
+// roles, whose descriptors the warp computes together.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t p;
+  asm volatile(
+      "{\n .reg .b32 r;\n .reg .pred q;\n elect.sync r|q, 0xffffffff;\n"
+      " selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(p));
+  return p != 0;
 }
 
 // Bounded wait that ignores the error status: used only to drain copies

@@ -109,7 +109,10 @@ __global__ void __launch_bounds__(kWlThreads) worklist_kernel(AttnArgs a, int ti
     if (pass == 0) n_pre = written;
   }
   if (threadIdx.x == 0) {
-    if (first) a.ws->status = HSTU_SLA_OK;
+    if (first) {
+      a.ws->status = HSTU_SLA_OK;
+      a.ws->wait_limit_ns = a.wait_limit_ns;
+    }
     if (list) {
       a.ws->n_items2 = written;
       a.ws->n_items2_pre = n_pre;

@@ -146,6 +146,22 @@ def test_full_size_sampled(wname):
         assert torch.isfinite(t.float()).all()
 
 
+def test_mid_full_tensor():
+    """The mid-length training batch (32 sequences of 1K-4K tokens, 4 x 128
+    heads, K1 256, K2 64) compared element by element over the whole jagged
+    tensor: out, dq, dk, dv against the oracle's full forward and backward."""
+    b = make_batch(WORKLOADS["mid"])
+    g = to_gpu(b)
+    out = gpu_fwd(b, g)
+    dq, dk, dv = gpu_bwd(b, g)
+    p = oracle_problem(b)
+    assert_close("out", out, p.fwd(b.q, b.k, b.v))
+    rq, rk, rv = p.bwd(b.q, b.k, b.v, b.dout)
+    assert_close("dq", dq, rq)
+    assert_close("dk", dk, rk)
+    assert_close("dv", dv, rv)
+
+
 def test_candidate_scoring_computes_only_candidate_tiles():
     """M-FALCON scoring (candidates_only): rows of the query tiles that hold
     candidates equal the full forward bit for bit (and the oracle); rows of
