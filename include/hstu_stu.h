@@ -75,6 +75,17 @@ typedef struct {
   const float* w1s;            /* [4 d_model] column scales of W1 */
   const void* w2q;             /* E4M3 [d_model][d_model]:   W2 transposed */
   const float* w2s;            /* [d_model] */
+  /* Selective activation rematerialisation (section 4.2.2 and its code
+   * Listing 1): with remat = 1 the forward keeps for the backward only what
+   * the listing saves, x (the caller's input), u (the U block of SiLU(pre),
+   * [T][d_model], written here), av and stats; xn, pre, uvqk and y are
+   * scratch in the workspace (their pointers are not read and may be NULL).
+   * The backward recomputes x^ = LayerNorm(x) and pre, U | V | Q | K with the
+   * same kernels (so the same bits), and y = LayerNorm(av) * u, then runs the
+   * usual backward.  Workspaces: HSTU_STU_WS_FWD_REMAT / HSTU_STU_WS_BWD_REMAT.
+   * Not with fp8 = 1 (HSTU_SLA_ERR_UNSUPPORTED). */
+  int32_t remat;
+  void* u;                     /* bf16 [T][d_model]; read only with remat = 1 */
 } hstu_stu_layer_params;
 
 typedef struct {
@@ -98,10 +109,13 @@ typedef struct {
 } hstu_stu_layer_bwd_params;
 
 /* Workspace bytes for hstu_stu_layer_fwd (which = HSTU_SLA_WS_FWD, or
- * HSTU_STU_WS_FWD_FP8 when fp8 = 1: the E4M3 activation rows on top) or
- * hstu_stu_layer_bwd (HSTU_SLA_WS_BWD); 256-byte aligned, contents need not
- * be initialised.  0 on invalid arguments. */
+ * HSTU_STU_WS_FWD_FP8 when fp8 = 1: the E4M3 activation rows on top, or
+ * HSTU_STU_WS_FWD_REMAT when remat = 1) or hstu_stu_layer_bwd
+ * (HSTU_SLA_WS_BWD, or HSTU_STU_WS_BWD_REMAT when remat = 1); 256-byte
+ * aligned, contents need not be initialised.  0 on invalid arguments. */
 #define HSTU_STU_WS_FWD_FP8 2
+#define HSTU_STU_WS_FWD_REMAT 3  /* forward with remat = 1: + x^, pre, U|V|Q|K, y scratch */
+#define HSTU_STU_WS_BWD_REMAT 4  /* backward with remat = 1: + the recomputed tensors */
 size_t hstu_stu_workspace_bytes(int which, int64_t total_tokens, int32_t B, int32_t H, int32_t d);
 
 int hstu_stu_layer_fwd(const hstu_stu_layer_params* p, void* workspace, size_t workspace_bytes,

@@ -23,9 +23,19 @@ int check_layer(const hstu_stu_layer_params* p, bool need_out) {
   if (dm != 256 && dm != 512 && dm != 1024) return HSTU_SLA_ERR_UNSUPPORTED;
   if (!(p->ln_eps >= 0.f)) return HSTU_SLA_ERR_INVALID_ARG;
   const void* ptrs[] = {p->ln1_w, p->ln1_b, p->w1, p->b1, p->ln2_w, p->ln2_b, p->w2, p->b2,
-                        p->x,     p->out,   p->xn, p->pre, p->uvqk, p->av,   p->y,  p->stats};
+                        p->x,     p->av,    p->stats};
   for (const void* q : ptrs)
-    if (!al16(q) && !(q == p->out && !need_out)) return HSTU_SLA_ERR_INVALID_ARG;
+    if (!al16(q)) return HSTU_SLA_ERR_INVALID_ARG;
+  if (need_out && !al16(p->out)) return HSTU_SLA_ERR_INVALID_ARG;
+  if (p->remat != 0 && p->remat != 1) return HSTU_SLA_ERR_INVALID_ARG;
+  if (p->remat) {  // Listing 1's save set: x, u, av, stats; the rest is scratch
+    if (!al16(p->u)) return HSTU_SLA_ERR_INVALID_ARG;
+    if (p->fp8) return HSTU_SLA_ERR_UNSUPPORTED;
+  } else {
+    const void* saved[] = {p->xn, p->pre, p->uvqk, p->y};
+    for (const void* q : saved)
+      if (!al16(q)) return HSTU_SLA_ERR_INVALID_ARG;
+  }
   if (p->fp8 != 0 && p->fp8 != 1) return HSTU_SLA_ERR_INVALID_ARG;
   if (p->fp8 && need_out && (!al16(p->w1q) || !al16(p->w1s) || !al16(p->w2q) || !al16(p->w2s)))
     return HSTU_SLA_ERR_INVALID_ARG;
@@ -85,15 +95,45 @@ size_t fp8_scratch_bytes(int64_t T, int dm) {
   return round256((size_t)T * dm) + round256((size_t)T * sizeof(float));
 }
 
+// Rematerialisation scratch after the attention's workspace: x^ [T][dm],
+// pre and U|V|Q|K [T][4 dm] (bf16), y [T][dm], and the recomputed norms'
+// statistics [4][T] (fp32; equal to the saved ones).
+size_t remat_scratch_bytes(int64_t T, int dm) {
+  const size_t r = (size_t)T * dm * sizeof(bf16);
+  return 2 * round256(r) + 2 * round256(4 * r) + round256((size_t)4 * T * sizeof(float));
+}
+
+// Points x^, pre, uvqk, y and stats of `r` at the scratch.  `stats` stays
+// the caller's unless `own_stats` (the backward's recomputation writes its
+// statistics to the scratch, the saved ones are what the gradients read).
+void carve_remat(hstu_stu_layer_params* r, void* scratch, float** recomputed_stats) {
+  const int64_t T = r->total_tokens;
+  const int dm = r->H * r->d;
+  const size_t row = (size_t)T * dm * sizeof(bf16);
+  char* c = static_cast<char*>(scratch);
+  r->xn = c;
+  c += round256(row);
+  r->pre = c;
+  c += round256(4 * row);
+  r->uvqk = c;
+  c += round256(4 * row);
+  r->y = c;
+  c += round256(row);
+  *recomputed_stats = reinterpret_cast<float*>(c);
+}
+
 }  // namespace
 
 extern "C" {
 
 size_t hstu_stu_workspace_bytes(int which, int64_t total_tokens, int32_t B, int32_t H, int32_t d) {
   const bool f8 = which == HSTU_STU_WS_FWD_FP8;
-  const size_t a = hstu_sla_workspace_bytes(f8 ? HSTU_SLA_WS_FWD : which, total_tokens, B, H, d);
+  const bool rf = which == HSTU_STU_WS_FWD_REMAT, rb = which == HSTU_STU_WS_BWD_REMAT;
+  const int attn = (f8 || rf) ? HSTU_SLA_WS_FWD : rb ? HSTU_SLA_WS_BWD : which;
+  const size_t a = hstu_sla_workspace_bytes(attn, total_tokens, B, H, d);
   if (a == 0) return 0;
-  return kHdr + a + (f8 ? fp8_scratch_bytes(total_tokens, H * d) : 0);
+  return kHdr + round256(a) + (f8 ? fp8_scratch_bytes(total_tokens, H * d) : 0) +
+         ((rf || rb) ? remat_scratch_bytes(total_tokens, H * d) : 0);
 }
 
 int hstu_stu_layer_fwd(const hstu_stu_layer_params* p, void* workspace, size_t workspace_bytes,
@@ -102,9 +142,24 @@ int hstu_stu_layer_fwd(const hstu_stu_layer_params* p, void* workspace, size_t w
   if (e) return e;
   const bool f8 = p->fp8 != 0;
   if ((e = check_ws(workspace, workspace_bytes,
-                    hstu_stu_workspace_bytes(f8 ? HSTU_STU_WS_FWD_FP8 : HSTU_SLA_WS_FWD,
+                    hstu_stu_workspace_bytes(f8 ? HSTU_STU_WS_FWD_FP8
+                                                : p->remat ? HSTU_STU_WS_FWD_REMAT
+                                                           : HSTU_SLA_WS_FWD,
                                              p->total_tokens, p->B, p->H, p->d))))
     return e;
+  // Listing 1's save set: x^, pre, U|V|Q|K and y go to scratch; U is copied
+  // out for the backward at the end
+  hstu_stu_layer_params remat_p;
+  const hstu_stu_layer_params* caller = p;
+  if (p->remat) {
+    remat_p = *p;
+    float* unused_stats = nullptr;
+    carve_remat(&remat_p, static_cast<char*>(workspace) + kHdr +
+                              round256(hstu_sla_workspace_bytes(HSTU_SLA_WS_FWD, p->total_tokens,
+                                                                p->B, p->H, p->d)),
+                &unused_stats);
+    p = &remat_p;
+  }
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   WsHeader* gh = static_cast<WsHeader*>(workspace);
   void* aws = static_cast<char*>(workspace) + kHdr;
@@ -186,6 +241,10 @@ int hstu_stu_layer_fwd(const hstu_stu_layer_params* p, void* workspace, size_t w
   } else {
     ce = launch_gemm({p->y, dm, false}, {p->w2, dm, true}, g2, kEpiBiasResid, st);
   }
+  if (ce == cudaSuccess && caller->remat && T > 0)  // the saved u: block 0 of U|V|Q|K
+    ce = cudaMemcpy2DAsync(caller->u, (size_t)dm * sizeof(bf16), p->uvqk,
+                           (size_t)4 * dm * sizeof(bf16), (size_t)dm * sizeof(bf16), (size_t)T,
+                           cudaMemcpyDeviceToDevice, st);
   return status_of(ce);
 }
 
@@ -201,7 +260,8 @@ int hstu_stu_layer_bwd(const hstu_stu_layer_bwd_params* p, void* workspace,
   for (const void* q : ptrs)
     if (!al16(q)) return HSTU_SLA_ERR_INVALID_ARG;
   if ((e = check_ws(workspace, workspace_bytes,
-                    hstu_stu_workspace_bytes(HSTU_SLA_WS_BWD, f->total_tokens, f->B, f->H, f->d))))
+                    hstu_stu_workspace_bytes(f->remat ? HSTU_STU_WS_BWD_REMAT : HSTU_SLA_WS_BWD,
+                                             f->total_tokens, f->B, f->H, f->d))))
     return e;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   WsHeader* gh = static_cast<WsHeader*>(workspace);
@@ -211,6 +271,57 @@ int hstu_stu_layer_bwd(const hstu_stu_layer_bwd_params* p, void* workspace,
   const bf16* dout = static_cast<const bf16*>(p->dout);
   bf16* dpre = static_cast<bf16*>(p->dpre);
   cudaError_t ce = cudaMemsetAsync(gh, 0, sizeof(WsHeader), st);
+  hstu_stu_layer_params remat_f;
+  if (f->remat && ce == cudaSuccess) {
+    // Listing 1: recompute x^ = LayerNorm(x), pre and U|V|Q|K = SiLU(x^ W1 +
+    // b1) by the forward's own kernels (the same bits), and y = LayerNorm(av)
+    // * u, into the scratch; the gradients below then read them as saved.
+    // The recomputed statistics go to the scratch too (equal to the saved).
+    remat_f = *f;
+    float* rstats = nullptr;
+    carve_remat(&remat_f, static_cast<char*>(workspace) + kHdr +
+                              round256(hstu_sla_workspace_bytes(HSTU_SLA_WS_BWD, T, f->B, f->H,
+                                                                f->d)),
+                &rstats);
+    LnArgs r1;
+    memset(&r1, 0, sizeof(r1));
+    r1.T = T;
+    r1.W = dm;
+    r1.eps = f->ln_eps;
+    r1.x = static_cast<const bf16*>(f->x);
+    r1.ldx = dm;
+    r1.gamma = f->ln1_w;
+    r1.beta = f->ln1_b;
+    r1.y = static_cast<bf16*>(remat_f.xn);
+    r1.ldy = dm;
+    r1.mean = rstats;
+    r1.rstd = rstats + T;
+    ce = launch_ln_fwd(r1, false, st);
+    GemmArgs rg;
+    memset(&rg, 0, sizeof(rg));
+    rg.M = (int)T;
+    rg.N = 4 * dm;
+    rg.K = dm;
+    rg.bias = f->b1;
+    rg.out = static_cast<bf16*>(remat_f.uvqk);
+    rg.ldo = 4 * dm;
+    rg.out2 = static_cast<bf16*>(remat_f.pre);
+    rg.ldo2 = 4 * dm;
+    rg.ws = gh;
+    if (ce == cudaSuccess)
+      ce = launch_gemm({remat_f.xn, dm, false}, {f->w1, 4 * dm, true}, rg, kEpiBiasSilu, st);
+    LnArgs r2 = r1;
+    r2.x = static_cast<const bf16*>(f->av);
+    r2.u = static_cast<const bf16*>(f->u);
+    r2.ldu = dm;
+    r2.gamma = f->ln2_w;
+    r2.beta = f->ln2_b;
+    r2.y = static_cast<bf16*>(remat_f.y);
+    r2.mean = rstats + 2 * T;
+    r2.rstd = rstats + 3 * T;
+    if (ce == cudaSuccess) ce = launch_ln_fwd(r2, true, st);
+    f = &remat_f;
+  }
   const struct { float* p; size_t n; } grads[] = {
       {p->d_ln1_w, (size_t)dm}, {p->d_ln1_b, (size_t)dm}, {p->d_w1, (size_t)dm * 4 * dm},
       {p->d_b1, (size_t)4 * dm}, {p->d_ln2_w, (size_t)dm}, {p->d_ln2_b, (size_t)dm},

@@ -121,17 +121,28 @@ def quantize_weights(w: StuWeights, stream=None) -> Fp8Weights:
 
 @dataclasses.dataclass
 class LayerState:
-    """What one layer's forward saves for its backward."""
+    """What one layer's forward saves for its backward.  Without remat: x^,
+    pre, U|V|Q|K, A, y and both norms' statistics.  With remat (the save set
+    of Listing 1 in ULTRA-HSTU section 4.2.2): only u (the U block), A and
+    the statistics; xn, pre, uvqk, y are None and the backward recomputes
+    them."""
     x: torch.Tensor
     seq_offsets: torch.Tensor
     num_targets: Optional[torch.Tensor]
     max_seq_len: int
-    xn: torch.Tensor
-    pre: torch.Tensor
-    uvqk: torch.Tensor
+    xn: Optional[torch.Tensor]
+    pre: Optional[torch.Tensor]
+    uvqk: Optional[torch.Tensor]
     av: torch.Tensor
-    y: torch.Tensor
+    y: Optional[torch.Tensor]
     stats: torch.Tensor
+    u: Optional[torch.Tensor] = None
+    remat: bool = False
+
+    def saved_bytes(self) -> int:
+        """Bytes this state holds beyond the layer input x."""
+        ts = (self.xn, self.pre, self.uvqk, self.av, self.y, self.stats, self.u)
+        return sum(t.numel() * t.element_size() for t in ts if t is not None)
 
 
 def _layer_params(cfg: StuConfig, w: StuWeights, st: LayerState, out,
@@ -146,8 +157,9 @@ def _layer_params(cfg: StuConfig, w: StuWeights, st: LayerState, out,
     (p.ln1_w, p.ln1_b, p.w1, p.b1, p.ln2_w, p.ln2_b, p.w2, p.b2) = (t.data_ptr()
                                                                      for t in w.tensors())
     p.x, p.out = st.x.data_ptr(), _ptr(out)
-    p.xn, p.pre, p.uvqk = st.xn.data_ptr(), st.pre.data_ptr(), st.uvqk.data_ptr()
-    p.av, p.y, p.stats = st.av.data_ptr(), st.y.data_ptr(), st.stats.data_ptr()
+    p.xn, p.pre, p.uvqk = _ptr(st.xn), _ptr(st.pre), _ptr(st.uvqk)
+    p.av, p.y, p.stats = st.av.data_ptr(), _ptr(st.y), st.stats.data_ptr()
+    p.remat, p.u = int(st.remat), _ptr(st.u)
     if fp8 is not None:
         p.fp8 = 1
         p.w1q, p.w1s, p.w2q, p.w2s = (fp8.w1q.data_ptr(), fp8.w1s.data_ptr(), fp8.w2q.data_ptr(),
@@ -168,19 +180,26 @@ def workspace_bytes(which: int, T: int, B: int, cfg: StuConfig) -> int:
 
 def layer_fwd(x: torch.Tensor, seq_offsets: torch.Tensor, num_targets: Optional[torch.Tensor],
               w: StuWeights, cfg: StuConfig, max_seq_len: int, workspace=None, stream=None,
-              fp8: Optional[Fp8Weights] = None):
+              fp8: Optional[Fp8Weights] = None, remat: bool = False):
     """One STU layer forward; returns (out, state for the backward).  With
-    fp8 (from quantize_weights) the two projections run in E4M3."""
+    fp8 (from quantize_weights) the two projections run in E4M3.  remat:
+    keep only Listing 1's save set (u, A, statistics) for the backward."""
     _check_x(x, cfg)
     T, dm, dev = x.shape[0], cfg.d_model, x.device
     bf = dict(dtype=torch.bfloat16, device=dev)
-    st = LayerState(x, seq_offsets, num_targets, int(max_seq_len),
-                    torch.empty((T, dm), **bf), torch.empty((T, 4 * dm), **bf),
-                    torch.empty((T, 4 * dm), **bf), torch.empty((T, dm), **bf),
-                    torch.empty((T, dm), **bf), torch.empty((4, T), dtype=torch.float32, device=dev))
+    stats = torch.empty((4, T), dtype=torch.float32, device=dev)
+    if remat:
+        st = LayerState(x, seq_offsets, num_targets, int(max_seq_len), None, None, None,
+                        torch.empty((T, dm), **bf), None, stats, torch.empty((T, dm), **bf), True)
+    else:
+        st = LayerState(x, seq_offsets, num_targets, int(max_seq_len),
+                        torch.empty((T, dm), **bf), torch.empty((T, 4 * dm), **bf),
+                        torch.empty((T, 4 * dm), **bf), torch.empty((T, dm), **bf),
+                        torch.empty((T, dm), **bf), stats)
     out = torch.empty((T, dm), **bf)
     p = _layer_params(cfg, w, st, out, fp8)
-    need = workspace_bytes(_abi.WS_FWD if fp8 is None else _abi.WS_FWD_FP8, T, p.B, cfg)
+    kind = _abi.WS_FWD_REMAT if remat else (_abi.WS_FWD if fp8 is None else _abi.WS_FWD_FP8)
+    need = workspace_bytes(kind, T, p.B, cfg)
     ws = torch.empty(need, dtype=torch.uint8, device=dev) if workspace is None else workspace
     _check(_abi.load().hstu_stu_layer_fwd(ctypes.byref(p), ws.data_ptr(), ws.numel(),
                                           _stream(stream)), "hstu_stu_layer_fwd")
@@ -207,7 +226,7 @@ def layer_bwd(dout: torch.Tensor, st: LayerState, w: StuWeights, cfg: StuConfig,
     q.dy, q.dav, q.dpre, q.dxn = (t.data_ptr() for t in scratch)
     (q.d_ln1_w, q.d_ln1_b, q.d_w1, q.d_b1, q.d_ln2_w, q.d_ln2_b, q.d_w2,
      q.d_b2) = (t.data_ptr() for t in g.tensors())
-    need = workspace_bytes(_abi.WS_BWD, T, q.fwd.B, cfg)
+    need = workspace_bytes(_abi.WS_BWD_REMAT if st.remat else _abi.WS_BWD, T, q.fwd.B, cfg)
     ws = torch.empty(need, dtype=torch.uint8, device=dev) if workspace is None else workspace
     _check(_abi.load().hstu_stu_layer_bwd(ctypes.byref(q), ws.data_ptr(), ws.numel(),
                                           _stream(stream)), "hstu_stu_layer_bwd")
@@ -281,12 +300,15 @@ class StuStack:
 
     cfg_full / cfg_trunc: attention settings before / after truncation (their
     N differ: the longest sequence of each stage).  fp8=True runs the forward
-    projections in E4M3; call requantize() after every weight update."""
+    projections in E4M3; call requantize() after every weight update.
+    remat=True keeps only Listing 1's save set per layer and recomputes the
+    rest in the backward."""
 
     def __init__(self, weights: List[StuWeights], cfg_full: StuConfig, cfg_trunc: StuConfig,
-                 trunc_after: int, tail: int, fp8: bool = False):
+                 trunc_after: int, tail: int, fp8: bool = False, remat: bool = False):
         self.weights, self.cfg_full, self.cfg_trunc = weights, cfg_full, cfg_trunc
         self.trunc_after, self.tail = trunc_after, tail
+        self.remat = remat
         self.fp8 = None
         if fp8:
             self.requantize()
@@ -312,7 +334,7 @@ class StuStack:
                 offs = new_offs
             cfg = self.cfg_full if i < self.trunc_after else self.cfg_trunc
             h, st = layer_fwd(h, offs, num_targets, w, cfg, msl, stream=stream,
-                              fp8=None if self.fp8 is None else self.fp8[i])
+                              fp8=None if self.fp8 is None else self.fp8[i], remat=self.remat)
             states.append(st)
         return h, (states, seq_offsets, new_offs, num_targets, x.shape[0])
 
