@@ -285,6 +285,32 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def rank_batch(w, world, rank, strong=False):
+    """This rank's batch.  N = 1: the workload's batch.  N > 1: a global batch
+    split by whole sequences (sharding.partition_sequences: longest first on
+    the closed-form pair count), no exchange on the data path.  strong: the
+    global batch is the workload's one batch (total work fixed as N grows);
+    else it is N batches of the recipe (one per rank's seed), so the work per
+    GPU stays fixed (weak scaling) while the sequences still go to the ranks
+    by the balancer, not one draw per rank."""
+    from sparse_hstu_attention_b200 import sharding
+    from workloads import draw_lengths
+    if world == 1:
+        return make_batch(w), None
+    if strong:
+        lengths = draw_lengths(w)
+    else:
+        lengths = np.concatenate([draw_lengths(w, seed=w.seed + 7919 * r) for r in range(world)])
+    nts = np.minimum(np.full(len(lengths), w.num_targets), lengths)
+    owned = sharding.partition_sequences(lengths, nts, world, w.contextual_len, w.K1, w.K2)
+    mine = owned[rank]
+    info = {"global_sequences": int(len(lengths)), "global_tokens": int(lengths.sum()),
+            "rank0_sequences": [int(lengths[b]) for b in owned[0]],
+            "balancer": "longest-first on closed-form unmasked pairs"}
+    return make_batch(w, lengths=lengths[mine], num_targets=nts[mine],
+                      seed=w.seed + 7919 * rank), info
+
+
 def _config(w, batch):
     pairs = F.total_pairs(batch.lengths, batch.num_targets, w.contextual_len, w.K1, w.K2)
     in_bytes = 4 * batch.T * w.H * w.d * 2
@@ -353,7 +379,7 @@ def run_stu(args, world, rank, local):
     T, T_out, dm = int(offs[-1]), int(tl.sum()), full.d_model
     dr = draw_stu(T, T_out, dm, STU_LAYERS, seed=w.seed + 7919 * rank)
     ws = [stu.StuWeights.from_host(lw, dev) for lw in dr.layers]
-    stack = stu.StuStack(ws, full, cut, STU_TRUNC_AFTER, tail, fp8=args.fp8)
+    stack = stu.StuStack(ws, full, cut, STU_TRUNC_AFTER, tail, fp8=args.fp8, remat=args.remat)
     offs_d = torch.tensor(offs, dtype=torch.int32, device=dev)
     nts_d = torch.tensor(nts, dtype=torch.int32, device=dev)
     x, dout = dr.x.to(dev), dr.dout.to(dev)
@@ -373,6 +399,10 @@ def run_stu(args, world, rank, local):
         out, ctx = stack.forward(x, offs_d, nts_d, lengths, nts)
         stack.backward(dout, ctx)
 
+    # bytes each layer's forward keeps for its backward (beyond its input)
+    _, ctx0 = stack.forward(x, offs_d, nts_d, lengths, nts)
+    saved = [st.saved_bytes() for st in ctx0[0]]
+    del ctx0
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -405,15 +435,19 @@ def run_stu(args, world, rank, local):
             "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16, forward projections e4m3" if args.fp8 else "bf16",
             "data": "synthetic (seeded N(0,1) inputs, Xavier-uniform weights)",
-            "config": {"workload": "stu", "fp8_forward_projections": bool(args.fp8), "layers": STU_LAYERS, "trunc_after": STU_TRUNC_AFTER,
+            "config": {"workload": "stu", "fp8_forward_projections": bool(args.fp8),
+                       "remat": bool(args.remat), "layers": STU_LAYERS,
+                       "trunc_after": STU_TRUNC_AFTER,
                        "tail": tail, "B": int(len(lengths)), "T": T, "T_truncated": T_out,
                        "d_model": dm, "H": w.H, "d": w.d, "K1": w.K1, "K2": w.K2,
                        "contextual_len": c, "num_targets": w.num_targets,
                        "N": [w.N, cut.N]},
             "flops_per_step": {"projections": gemm, "attention": attn},
+            "saved_activation_bytes_per_layer": saved,
             "frac_of_sustained_peak": value / world / peak,
             "frac_of_burst_peak": value / world / float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])),
-            "gpu_launches": K * (STU_LAYERS * (6 + 11 + (2 if args.fp8 else 0)) + 3),
+            "gpu_launches": K * (STU_LAYERS * (6 + 11 + (2 if args.fp8 else 0) +
+                                              (3 if args.remat else 0)) + 3),
             "clocks": clocks.summary(),
             **({} if (world > 1 or args.no_cpu_baseline) else
                {"cpu_baseline": stu_cpu_baseline(w, lengths, nts, dr, full, args.fp8)})}),
@@ -528,12 +562,18 @@ def main():
     ap.add_argument("--workload", default="hist16k", choices=sorted(WORKLOADS) + ["mot"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--strong", action="store_true",
+                    help="N > 1: shard the workload's one batch across the GPUs (strong "
+                         "scaling); by default N batches of the recipe are sharded (weak)")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--rab", action="store_true",
                     help="attention workloads: with the relative attention bias (32 position and "
                          "32 time buckets per head, seeded tables and timestamps)")
     ap.add_argument("--fp8", action="store_true",
                     help="stu workload: E4M3 forward projections (weights requantized every step)")
+    ap.add_argument("--remat", action="store_true",
+                    help="stu workload: keep only the rematerialisation save set per layer "
+                         "(u, attention output, norm statistics); the backward recomputes the rest")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":
@@ -549,7 +589,7 @@ def main():
         return run_mot(args, world, rank, local)
     dev = torch.device("cuda", local)
     w = WORKLOADS[args.workload]
-    batch = make_batch(w, seed=w.seed + 7919 * rank)
+    batch, shard_info = rank_batch(w, world, rank, strong=args.strong)
     T, H, d = batch.T, w.H, w.d
     pairs = F.total_pairs(batch.lengths, batch.num_targets, w.contextual_len, w.K1, w.K2)
     fl_f, fl_b = F.fwd_flops(pairs, H, d), (0.0 if w.fwd_only else F.bwd_flops(pairs, H, d))
@@ -611,12 +651,16 @@ def main():
         if world > 1:
             torch.distributed.barrier()
     ms = t_start.elapsed_time(t_end)
+    job_fl = fl_f + fl_b  # every rank's FLOPs (the sharded ranks' work differs)
     if world > 1:
         tt = torch.tensor([ms], device=dev, dtype=torch.float64)
         torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
         ms = float(tt.item())
+        ff = torch.tensor([job_fl], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(ff, op=torch.distributed.ReduceOp.SUM)
+        job_fl = float(ff.item())
     ms_step = ms / K
-    value = world * (fl_f + fl_b) / (ms_step * 1e-3) / 1e12
+    value = job_fl / (ms_step * 1e-3) / 1e12
     fwd_ms = sum(fb[i].elapsed_time(fe[i]) for i in range(K)) / K
     bwd_ms = 0.0 if w.fwd_only else sum(bb[i].elapsed_time(be[i]) for i in range(K)) / K
 
@@ -725,17 +769,17 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "scaling": "strong" if args.strong else "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16, jagged lengths drawn per workload recipe)",
         "config": dict(_config(w, batch), **(
             {"relative_attention_bias": {"pos_buckets": 32, "time_buckets": 32}}
-            if args.rab else {})),
+            if args.rab else {}), **({"sharding": shard_info} if shard_info else {})),
         "pct_of_peak": 100.0 * value / world / peak,
         "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
         "fwd_tflops": fl_f / (fwd_ms * 1e-3) / 1e12 if fwd_ms else None,
         "bwd_tflops": fl_b / (bwd_ms * 1e-3) / 1e12 if bwd_ms else None,
         "roofline": roof,
-        "e2e": {"value": world * (fl_f + fl_b) / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "e2e": {"value": job_fl / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": K * (LAUNCHES_PER_STEP["fwd"] +
                              (0 if w.fwd_only else LAUNCHES_PER_STEP["bwd"])),

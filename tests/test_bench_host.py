@@ -77,3 +77,24 @@ def test_roofline_picks_the_bound_and_the_burst_denominator():
     assert h["bound"] == "hbm" and h["unit"] == "GB/s" and h["peak"] == 6400.0
     assert abs(h["achieved"] - 2000.0) < 1e-9 and abs(h["frac"] - 2000 / 6400) < 1e-12
     assert abs(h["tensor_tflops"] - 200.0) < 1e-9
+
+
+def test_rank_batches_shard_a_global_batch():
+    """N > 1: every sequence of the global batch lands on exactly one rank (by
+    length, for the strong split of the workload's one batch), N = 1 is the
+    workload's own batch, and the weak split's global batch has N batches'
+    sequences."""
+    import numpy as np
+    from workloads import WORKLOADS, draw_lengths, make_batch
+    bench = _bench_module()
+    w = WORKLOADS["tiny"]
+    b1, info = bench.rank_batch(w, 1, 0)
+    assert info is None and np.array_equal(b1.lengths, make_batch(w).lengths)
+    for world in (2, 3):
+        strong = [bench.rank_batch(w, world, r, strong=True) for r in range(world)]
+        got = np.sort(np.concatenate([b.lengths for b, _ in strong]))
+        assert np.array_equal(got, np.sort(draw_lengths(w)))
+        assert strong[0][1]["global_sequences"] == w.B
+        weak = [bench.rank_batch(w, world, r) for r in range(world)]
+        assert weak[0][1]["global_sequences"] == world * w.B
+        assert sum(len(b.lengths) for b, _ in weak) == world * w.B

@@ -92,9 +92,10 @@ MOT_CHANNELS = {
 }
 
 
-def draw_lengths(w: Workload) -> np.ndarray:
-    """Total per-sequence lengths (contextual prefix and candidates included)."""
-    rng = np.random.default_rng(w.seed)
+def draw_lengths(w: Workload, seed: Optional[int] = None) -> np.ndarray:
+    """Total per-sequence lengths (contextual prefix and candidates included);
+    `seed` overrides the workload's own (another batch of the same recipe)."""
+    rng = np.random.default_rng(w.seed if seed is None else seed)
     if w.name == "tiny":
         return rng.integers(32, 256, size=w.B, endpoint=True).astype(np.int64)
     if w.name == "mid":
