@@ -24,8 +24,8 @@
 //
 // Roles (persistent CTAs, one per SM; units handed out by an atomic counter,
 // prefix-key units first):
-//   warp 0      scheduler + TMA producer (K double-buffered, V single,
-//               3-stage Q / dO ring)
+//   warp 0      scheduler + TMA producer of the 3-stage Q / dO ring
+//   warp 18     TMA loads of K (double-buffered) and V (single)
 //   warp 1      TMEM allocation; the warp computes every MMA operand, one
 //               elected lane issues each batch of UMMAs and its commits
 //   warps 2..17 pointwise, all sixteen on every step (16 query columns
@@ -57,7 +57,8 @@ using namespace sm100;
 
 constexpr int D = 128;
 constexpr int kRes = 128, kStr = 64, kSt = 3, kPwWarps = 16, kUSlots = 4, kPwWarp0 = 2;
-constexpr int kThreads = 32 * (kPwWarp0 + kPwWarps);
+constexpr int kKvWarp = kPwWarp0 + kPwWarps;  // the K / V loader
+constexpr int kThreads = 32 * (kKvWarp + 1);
 constexpr uint32_t kColX1 = 0, kColX2 = 128, kColAcc1 = 256, kColAcc2 = 384, kTmemCols = 512;
 constexpr int SW = 128, BOXW = 64, NB = D / BOXW;
 constexpr int RTILE = kRes * D * 2;     // resident tile, two 64-column boxes
@@ -226,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(F_ACC_EMPTY), kPwWarps);
     for (int s = 0; s < kUSlots; ++s) {
       mbar_init(bar(F_U_FULL + s), 1);
-      mbar_init(bar(F_U_EMPTY + s), 1 + kPwWarps);     // MMA lane + pointwise warps
+      mbar_init(bar(F_U_EMPTY + s), 2 + kPwWarps);  // MMA, K / V loader, pointwise warps
     }
     mbar_init(bar(F_DRAIN), 1);
     for (int i = 0; i < 2; ++i) {
@@ -257,7 +258,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------- scheduler + producer
     // The whole warp walks the schedule (warp-uniform values); lane 0 takes
     // units from the counter, decodes them, arms barriers and issues copies.
-    uint32_t kn = 0, vn = 0, bn = 0;  // K, V and streamed loads issued
+    // The K / V tiles come from their own warp (kKvWarp), so this stream of
+    // Q / dO tiles runs into the next unit while its V still waits for the
+    // current unit's last score MMA.
+    uint32_t bn = 0;  // streamed loads issued
     bool ok = true;
     for (int kk = 0; ok; ++kk) {
       const int slot = kk % kUSlots;
@@ -272,29 +276,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int nt = r->nsteps;
       if (nt < 0) break;
       if (nt == 0) continue;
-      const int h = r->h, y0 = r->s0 + r->t0;
+      const int h = r->h;
       const int p = r->grp;
-      // K buffer kn % 2: free once the unit two back issued its last dQ MMA
-      const uint32_t kb = kn & 1;
-      ok = warp_wait(bar(F_K_EMPTY + kb), ((kn >> 1) & 1) ^ 1, ws);
-      if (!ok) break;
-      if (lane == 0) {
-        const uint32_t fb = bar(F_K_FULL + kb);
-        mbar_expect_tx(fb, RTILE);
-        for (int b = 0; b < NB; ++b)
-          tma_load_2d(sK + kb * RTILE + b * RBLK, &maps.k[p], fb, h * D + b * BOXW, y0);
-      }
-      ++kn;
-      // V: free once the previous unit's last score MMA is done
-      ok = warp_wait(bar(F_V_EMPTY), (vn & 1) ^ 1, ws);
-      if (!ok) break;
-      if (lane == 0) {
-        const uint32_t fb = bar(F_V_FULL);
-        mbar_expect_tx(fb, RTILE);
-        for (int b = 0; b < NB; ++b)
-          tma_load_2d(sV + b * RBLK, &maps.v[p], fb, h * D + b * BOXW, y0);
-      }
-      ++vn;
       SpanCursor c;
       c.begin(r);
       for (int n = 0; n < nt && ok; ++n, c.next(r)) {
@@ -314,11 +297,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     if (lane == 0 && load_status(ws) != 0) {  // drain copies in flight before exiting
-      for (uint32_t kb = 0; kb < 2; ++kb) {
-        const uint32_t armed = kn / 2 + (kb < (kn & 1) ? 1u : 0u);
-        if (armed > 0) drain_wait(bar(F_K_FULL + kb), (armed - 1) & 1);
-      }
-      if (vn > 0) drain_wait(bar(F_V_FULL), (vn - 1) & 1);
       for (int s = 0; s < kSt; ++s) {
         const uint32_t armed = bn / kSt + (s < (int)(bn % kSt) ? 1u : 0u);
         if (armed > 0) drain_wait(bar(F_B_FULL + s), (armed - 1) & 1);
@@ -445,6 +423,52 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (elect_one()) tc_commit(bar(F_DRAIN));
       __syncwarp();
       drain_wait(bar(F_DRAIN), 0);
+    }
+    __syncwarp();
+  } else if (warp == kKvWarp) {
+    // -------------------------------------------------------- K / V loader
+    // Per unit with steps: K into buffer kn % 2 once the unit two back
+    // issued its last dQ MMA, then V once the previous unit's last score MMA
+    // is done.
+    uint32_t kn = 0, vn = 0;  // K, V loads issued
+    bool ok = true;
+    for (int kk = 0; ok; ++kk) {
+      const int slot = kk % kUSlots;
+      ok = warp_wait(bar(F_U_FULL + slot), (kk / kUSlots) & 1, ws);
+      if (!ok) break;
+      const UnitRec* r = &ring[slot];
+      const int nt = r->nsteps;
+      if (nt > 0) {
+        const int h = r->h, y0 = r->s0 + r->t0, p = r->grp;
+        const uint32_t kb = kn & 1;
+        ok = warp_wait(bar(F_K_EMPTY + kb), ((kn >> 1) & 1) ^ 1, ws);
+        if (!ok) break;
+        if (lane == 0) {
+          const uint32_t fb = bar(F_K_FULL + kb);
+          mbar_expect_tx(fb, RTILE);
+          for (int b = 0; b < NB; ++b)
+            tma_load_2d(sK + kb * RTILE + b * RBLK, &maps.k[p], fb, h * D + b * BOXW, y0);
+        }
+        ++kn;
+        ok = warp_wait(bar(F_V_EMPTY), (vn & 1) ^ 1, ws);
+        if (!ok) break;
+        if (lane == 0) {
+          const uint32_t fb = bar(F_V_FULL);
+          mbar_expect_tx(fb, RTILE);
+          for (int b = 0; b < NB; ++b)
+            tma_load_2d(sV + b * RBLK, &maps.v[p], fb, h * D + b * BOXW, y0);
+        }
+        ++vn;
+      }
+      warp_arrive(bar(F_U_EMPTY + slot));
+      if (nt < 0) break;
+    }
+    if (lane == 0 && load_status(ws) != 0) {  // drain copies in flight before exiting
+      for (uint32_t kb = 0; kb < 2; ++kb) {
+        const uint32_t armed = kn / 2 + (kb < (kn & 1) ? 1u : 0u);
+        if (armed > 0) drain_wait(bar(F_K_FULL + kb), (armed - 1) & 1);
+      }
+      if (vn > 0) drain_wait(bar(F_V_FULL), (vn - 1) & 1);
     }
     __syncwarp();
   } else {
