@@ -562,6 +562,9 @@ def main():
     ap.add_argument("--workload", default="hist16k", choices=sorted(WORKLOADS) + ["mot"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-overlap", action="store_true",
+                    help="run the backward's preparation inside the backward call instead of "
+                         "beside the forward on a side stream")
     ap.add_argument("--strong", action="store_true",
                     help="N > 1: shard the workload's one batch across the GPUs (strong "
                          "scaling); by default N batches of the recipe are sharded (weak)")
@@ -622,14 +625,29 @@ def main():
 
     K = args.steps
     fb, fe, bb, be = new_events(K), new_events(K), new_events(K), new_events(K)
+    # The backward's preparation (its work list and the clear of its fp32 dQ
+    # accumulator) reads only the batch geometry: it runs on a side stream
+    # beside the forward, from the start of the step (the previous backward
+    # is done with the workspace by then), and the backward waits for it.
+    overlap = not w.fwd_only and not args.no_overlap
+    prep_stream = torch.cuda.Stream(dev)
+    ev_step, ev_prep = torch.cuda.Event(), torch.cuda.Event()
+    kw_prep = {n: x for n, x in kw.items() if n not in ("timestamps", "rab_pos", "rab_time")}
 
     def step(i=None):
         evf = (fb[i], fe[i]) if i is not None else None
         evb = (bb[i], be[i]) if i is not None else None
+        if overlap:
+            ev_step.record(stream)
+            prep_stream.wait_event(ev_step)
+            sla.hstu_sla_bwd_prepare(q, offs, nts, workspace=ws_b, stream=prep_stream, **kw_prep)
+            ev_prep.record(prep_stream)
         sla.hstu_sla_fwd(q, k, v, offs, nts, out=out, workspace=ws_f, events=evf, **kw)
         if not w.fwd_only:
+            if overlap:
+                stream.wait_event(ev_prep)
             sla.hstu_sla_bwd(dout, q, k, v, offs, nts, dq=dq, dk=dk, dv=dv, workspace=ws_b,
-                             events=evb, **kw)
+                             events=evb, prepared=overlap, **kw)
 
     for _ in range(args.warmup):
         step()
@@ -774,6 +792,8 @@ def main():
         "config": dict(_config(w, batch), **(
             {"relative_attention_bias": {"pos_buckets": 32, "time_buckets": 32}}
             if args.rab else {}), **({"sharding": shard_info} if shard_info else {})),
+        "bwd_prepare": ("side stream, beside the forward" if overlap else
+                        "inside the backward call") if not w.fwd_only else None,
         "pct_of_peak": 100.0 * value / world / peak,
         "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
         "fwd_tflops": fl_f / (fwd_ms * 1e-3) / 1e12 if fwd_ms else None,

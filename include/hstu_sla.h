@@ -128,6 +128,11 @@ typedef struct {
    * dP_ij SiLU'(x_ij) / N.  Required for every table that is set. */
   float* d_rab_pos;
   float* d_rab_time;
+  /* 1: hstu_sla_bwd_prepare already ran for this batch on this workspace
+   * (work lists built, dQ accumulator cleared) and was ordered before this
+   * call by the caller; the call then skips that work.  0: the call does it
+   * itself. */
+  int32_t prepared;
 } hstu_sla_bwd_params;
 
 #define HSTU_SLA_WS_FWD 0
@@ -161,6 +166,17 @@ int hstu_sla_fwd(const hstu_sla_fwd_params* p, void* workspace, size_t workspace
  *           scores for dq. */
 int hstu_sla_bwd(const hstu_sla_bwd_params* p, void* workspace, size_t workspace_bytes,
                  hstu_stream_t stream);
+
+/* The part of hstu_sla_bwd that reads neither dout nor the forward's inputs:
+ * the work lists of the batch (seq_offsets, num_targets, windows) and, for
+ * head_dim 128, the clear of the fp32 dQ accumulator in `workspace`.  A
+ * caller can issue it early on another stream, e.g. while the forward runs,
+ * then call hstu_sla_bwd with p->prepared = 1 on its stream after an event
+ * orders the two; the arguments and workspace must be the same, and nothing
+ * may use the workspace in between.  Same validation and return codes as
+ * hstu_sla_bwd; gradients and dout are not read. */
+int hstu_sla_bwd_prepare(const hstu_sla_bwd_params* p, void* workspace, size_t workspace_bytes,
+                         hstu_stream_t stream);
 
 /* Grouped calls: up to HSTU_SLA_MAX_GROUPS independent problems in ONE
  * launch of the attention kernel.  The use is the Mixture of Transducers

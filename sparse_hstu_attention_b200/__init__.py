@@ -32,7 +32,7 @@ import torch
 from . import _abi
 from ._abi import LibraryMissing  # noqa: F401
 
-__all__ = ["hstu_sla_fwd", "hstu_sla_fwd_noalloc", "hstu_sla_noalloc_get_error", "hstu_sla_bwd", "hstu_sla_workspace_bytes",
+__all__ = ["hstu_sla_fwd", "hstu_sla_bwd_prepare", "hstu_sla_fwd_noalloc", "hstu_sla_noalloc_get_error", "hstu_sla_bwd", "hstu_sla_workspace_bytes",
            "hstu_sla_count_pairs", "hstu_sla_fwd_grouped", "hstu_sla_bwd_grouped",
            "hstu_sla_grouped_workspace_bytes", "hstu_sla_get_error", "hstu_sla_strerror",
            "SLAError", "SLAAttention", "sla_attention"]
@@ -188,12 +188,14 @@ def hstu_sla_bwd(dout: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: torch.
                  max_seq_len: Optional[int] = None, dq: Optional[torch.Tensor] = None,
                  dk: Optional[torch.Tensor] = None, dv: Optional[torch.Tensor] = None,
                  workspace: Optional[torch.Tensor] = None, stream=None, events=None,
-                 timestamps=None, rab_pos=None, rab_time=None):
+                 timestamps=None, rab_pos=None, rab_time=None, prepared: bool = False):
     """SLA HSTU attention backward; returns (dq, dk, dv) [T, H, d] (bf16), and
     with a relative attention bias (dq, dk, dv, (d_rab_pos, d_rab_time)),
-    fp32, None for an absent table."""
+    fp32, None for an absent table.  prepared: hstu_sla_bwd_prepare already
+    ran on `workspace` for this batch, ordered before this call."""
     lib = _abi.load()
     p = _abi.BwdParams()
+    p.prepared = int(bool(prepared))
     p.fwd = _fwd_params(q, k, v, seq_offsets, num_targets, contextual_len, K1, K2, alpha, N,
                         max_seq_len, events)
     _set_rab(p.fwd, q.shape[1], timestamps, rab_pos, rab_time)
@@ -215,6 +217,27 @@ def hstu_sla_bwd(dout: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: torch.
     if rab_pos is not None or rab_time is not None:
         return dq, dk, dv, d_rab
     return dq, dk, dv
+
+
+def hstu_sla_bwd_prepare(q: torch.Tensor, seq_offsets: torch.Tensor,
+                         num_targets: Optional[torch.Tensor], *, contextual_len: int, K1: int,
+                         K2: int, alpha: float, N: float, workspace: torch.Tensor,
+                         max_seq_len: Optional[int] = None, stream=None) -> None:
+    """The backward's preparation (work lists; the clear of the dQ
+    accumulator for head_dim 128) into `workspace`, on `stream`: it reads only
+    the batch geometry, so it can run early (e.g. beside the forward).  The
+    backward then takes prepared=True and the same workspace."""
+    lib = _abi.load()
+    p = _abi.BwdParams()
+    p.fwd = _fwd_params(q, q, q, seq_offsets, num_targets, contextual_len, K1, K2, alpha, N,
+                        max_seq_len)
+    H, d = p.fwd.H, p.fwd.d
+    rs = _row_stride(q, "q", H, d)
+    p.dout = p.dq = p.dk = p.dv = q.data_ptr()  # validated, never read or written
+    p.dout_row_stride = p.dq_row_stride = p.dk_row_stride = p.dv_row_stride = rs
+    ws = _workspace(_abi.WS_BWD, p.fwd.total_tokens, p.fwd.B, H, d, q.device, workspace)
+    _check(lib.hstu_sla_bwd_prepare(ctypes.byref(p), ws.data_ptr(), ws.numel(),
+                                    _stream_ptr(stream)), "hstu_sla_bwd_prepare")
 
 
 def hstu_sla_grouped_workspace_bytes(which: int, problems) -> int:

@@ -54,6 +54,7 @@ class BwdParams(ctypes.Structure):
         ("dq_row_stride", ctypes.c_int64), ("dk_row_stride", ctypes.c_int64),
         ("dv_row_stride", ctypes.c_int64),
         ("d_rab_pos", ctypes.c_void_p), ("d_rab_time", ctypes.c_void_p),
+        ("prepared", ctypes.c_int32),
     ]
 
 
@@ -140,6 +141,8 @@ def load():
     lib.hstu_sla_grouped_workspace_bytes.restype = sz
     lib.hstu_sla_fwd_grouped.argtypes = [ctypes.POINTER(FwdParams), ctypes.c_int32, vp, sz, vp]
     lib.hstu_sla_fwd_grouped.restype = ctypes.c_int
+    lib.hstu_sla_bwd_prepare.argtypes = [ctypes.POINTER(BwdParams), vp, sz, vp]
+    lib.hstu_sla_bwd_prepare.restype = ctypes.c_int
     lib.hstu_sla_bwd_grouped.argtypes = [ctypes.POINTER(BwdParams), ctypes.c_int32, vp, sz, vp]
     lib.hstu_sla_bwd_grouped.restype = ctypes.c_int
     lib.hstu_sla_test_wait_timeout.argtypes = [ctypes.POINTER(BwdParams), ctypes.c_int32,

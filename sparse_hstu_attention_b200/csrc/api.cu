@@ -142,6 +142,11 @@ int hstu_sla_bwd(const hstu_sla_bwd_params* p, void* workspace, size_t workspace
   return sla_bwd(p, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream), nullptr);
 }
 
+int hstu_sla_bwd_prepare(const hstu_sla_bwd_params* p, void* workspace, size_t workspace_bytes,
+                         hstu_stream_t stream) {
+  return sla_bwd_prepare(p, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
 size_t hstu_sla_grouped_workspace_bytes(int which, int32_t G, const int64_t* total_tokens,
                                         const int32_t* B, const int32_t* H, const int32_t* d) {
   if (G < 1 || G > HSTU_SLA_MAX_GROUPS || !total_tokens || !B || !H || !d) return 0;
@@ -359,12 +364,15 @@ int hstu_sla_version(void) { return kAbiVersion; }
 
 namespace hstu {
 
-int sla_bwd(const hstu_sla_bwd_params* p, void* workspace, size_t workspace_bytes,
-            cudaStream_t st, const SiluFusion* fz) {
+// Validation and the launch arguments of a backward call (also used by its
+// prepare step).
+int bwd_args(const hstu_sla_bwd_params* p, void* workspace, size_t workspace_bytes,
+             AttnArgs* out) {
   if (p == nullptr) return HSTU_SLA_ERR_INVALID_ARG;
   const hstu_sla_fwd_params* f = &p->fwd;
   int e = check_common(f);
   if (e) return e;
+  if (p->prepared != 0 && p->prepared != 1) return HSTU_SLA_ERR_INVALID_ARG;
   if ((e = check_tensor(p->dout, p->dout_row_stride, f))) return e;
   if ((e = check_tensor(p->dq, p->dq_row_stride, f))) return e;
   if ((e = check_tensor(p->dk, p->dk_row_stride, f))) return e;
@@ -389,6 +397,41 @@ int sla_bwd(const hstu_sla_bwd_params* p, void* workspace, size_t workspace_byte
     a.d_rab_pos = f->rab_pos ? p->d_rab_pos : nullptr;
     a.d_rab_time = f->rab_time ? p->d_rab_time : nullptr;
   }
+  if (f->d == kFusedBwdD)  // the fp32 dQ workspace after the lists
+    a.dqacc = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                       ws_bytes(f->total_tokens, f->B));
+  *out = a;
+  return HSTU_SLA_OK;
+}
+
+// Work lists (both passes' for head dims 32 / 64) and the clear of the dQ
+// accumulator (head dim 128).
+cudaError_t bwd_prepare(const AttnArgs& a, int d, cudaStream_t st) {
+  if (d == kFusedBwdD) {
+    cudaError_t ce = launch_worklist(a, kKvBN, 1, true, st);
+    if (ce == cudaSuccess && a.T > 0)
+      ce = cudaMemsetAsync(a.dqacc, 0, dq_workspace_bytes(a.T, a.H, d), st);
+    return ce;
+  }
+  cudaError_t ce = launch_worklist(a, kQpBM, 0, true, st);
+  if (ce == cudaSuccess) ce = launch_worklist(a, kKvBN, 1, false, st);
+  return ce;
+}
+
+int sla_bwd_prepare(const hstu_sla_bwd_params* p, void* workspace, size_t workspace_bytes,
+                    cudaStream_t st) {
+  AttnArgs a;
+  const int e = bwd_args(p, workspace, workspace_bytes, &a);
+  if (e) return e;
+  return cuda_status(bwd_prepare(a, p->fwd.d, st));
+}
+
+int sla_bwd(const hstu_sla_bwd_params* p, void* workspace, size_t workspace_bytes,
+            cudaStream_t st, const SiluFusion* fz) {
+  AttnArgs a;
+  int e = bwd_args(p, workspace, workspace_bytes, &a);
+  if (e) return e;
+  const hstu_sla_fwd_params* f = &p->fwd;
   cudaError_t ce;
   if (fz != nullptr) {  // the STU layer's SiLU' and bias-gradient fusion
     // silu_qkv_kernel: 3 H d / 8 threads, whole warps per block part
@@ -405,17 +448,14 @@ int sla_bwd(const hstu_sla_bwd_params* p, void* workspace, size_t workspace_byte
                                          ws_bytes(f->total_tokens, f->B) +
                                          dq_workspace_bytes(f->total_tokens, f->H, f->d));
   }
+  // work lists (and the dQ clear), unless hstu_sla_bwd_prepare did them
+  ce = p->prepared ? cudaSuccess : bwd_prepare(a, f->d, st);
   if (f->d == kFusedBwdD) {
     // one pass over key tiles; dQ through the fp32 workspace after the lists
-    a.dqacc = reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                       ws_bytes(f->total_tokens, f->B));
-    ce = launch_worklist(a, kKvBN, 1, true, st);
     if (ce == cudaSuccess) ce = record(f->event_begin, st);
-    if (ce == cudaSuccess) ce = launch_bwd_fused(a, st);
+    if (ce == cudaSuccess) ce = launch_bwd_fused(a, st, /*cleared=*/true);
     if (ce == cudaSuccess) ce = record(f->event_end, st);
   } else {
-    ce = launch_worklist(a, kQpBM, 0, true, st);
-    if (ce == cudaSuccess) ce = launch_worklist(a, kKvBN, 1, false, st);
     if (ce == cudaSuccess) ce = record(f->event_begin, st);
     if (ce == cudaSuccess) ce = launch_bwd_tc(a, f->d, /*kv_pass=*/true, st);
     if (ce == cudaSuccess) ce = launch_bwd_tc(a, f->d, /*kv_pass=*/false, st);

@@ -958,7 +958,8 @@ cudaError_t launch_bwd_fused_grouped(const GroupSet& gs, cudaStream_t st) {
         !make_tma_2d(&m.q[p], a.q, a.T, HD, a.q_rs, BOXW, kStr, true) ||
         !make_tma_2d(&m.dout[p], a.dout, a.T, HD, a.do_rs, BOXW, kStr, true))
       return cudaErrorInvalidValue;
-    if ((e = cudaMemsetAsync(a.dqacc, 0, dq_workspace_bytes(a.T, a.H, D), st)) != cudaSuccess)
+    if (!gs.cleared &&
+        (e = cudaMemsetAsync(a.dqacc, 0, dq_workspace_bytes(a.T, a.H, D), st)) != cudaSuccess)
       return e;
     units += max_items(a.T, a.B) * a.H;
   }
@@ -999,13 +1000,14 @@ cudaError_t launch_bwd_fused_grouped(const GroupSet& gs, cudaStream_t st) {
   return cudaSuccess;
 }
 
-cudaError_t launch_bwd_fused(const AttnArgs& a, cudaStream_t st) {
+cudaError_t launch_bwd_fused(const AttnArgs& a, cudaStream_t st, bool cleared) {
   if (a.T == 0) return cudaSuccess;
   GroupSet gs;
   memset(&gs, 0, sizeof(gs));
   gs.g[0] = a;
   gs.common = a.ws;
   gs.G = 1;
+  gs.cleared = cleared ? 1 : 0;
   return launch_bwd_fused_grouped(gs, st);
 }
 

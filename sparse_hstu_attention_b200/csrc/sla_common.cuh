@@ -443,6 +443,8 @@ struct GroupSet {
   // whose pointwise warps withhold their first hand-over arrive, so that the
   // role waiting for it runs into the bounded-wait limit.
   int stall;
+  // The dQ accumulators were cleared beforehand (hstu_sla_bwd_prepare).
+  int cleared;
 };
 cudaError_t launch_fwd_grouped(const GroupSet& gs, int d, cudaStream_t st);
 // The backward entry point with the STU layer's SiLU' / bias-gradient fusion
@@ -459,9 +461,11 @@ struct SiluFusion {
 };
 int sla_bwd(const hstu_sla_bwd_params* p, void* workspace, size_t workspace_bytes,
             cudaStream_t st, const SiluFusion* fz);
+int sla_bwd_prepare(const hstu_sla_bwd_params* p, void* workspace, size_t workspace_bytes,
+                    cudaStream_t st);
 cudaError_t launch_bwd_fused_grouped(const GroupSet& gs, cudaStream_t st);
 cudaError_t launch_bwd_tc(const AttnArgs& a, int d, bool kv_pass, cudaStream_t st);
 // head_dim kFusedBwdD: zeroes a.dqacc, runs the one-pass backward, converts dq
-cudaError_t launch_bwd_fused(const AttnArgs& a, cudaStream_t st);
+cudaError_t launch_bwd_fused(const AttnArgs& a, cudaStream_t st, bool cleared = false);
 
 }  // namespace hstu

@@ -146,6 +146,40 @@ def test_full_size_sampled(wname):
         assert torch.isfinite(t.float()).all()
 
 
+def test_backward_prepared_on_a_side_stream():
+    """hstu_sla_bwd_prepare (work list and dQ-accumulator clear) on another
+    stream, ordered by an event, then the backward with prepared=True on the
+    same workspace: dk and dv equal the plain call's bit for bit, dq matches
+    the oracle (its fp32 additions have no fixed order), twice in a row so
+    the second prepare clears what the first backward left."""
+    b = _edge_batch(lengths=[300, 17, 201, 129], nt=12, K1=96, K2=24, ctx=8)
+    g = to_gpu(b)
+    kw = kwargs_of(b)
+    T, H, d = b.q.shape
+    ws = torch.empty(sla.hstu_sla_workspace_bytes(1, T, len(b.lengths), H, d),
+                     dtype=torch.uint8, device="cuda")
+    dq0, dk0, dv0 = sla.hstu_sla_bwd(g["dout"], g["q"], g["k"], g["v"], g["offs"], g["nts"], **kw)
+    side = torch.cuda.Stream()
+    main = torch.cuda.current_stream()
+    p = oracle_problem(b)
+    rq, rk, rv = p.bwd(b.q, b.k, b.v, b.dout)
+    for _ in range(2):
+        ev0, ev1 = torch.cuda.Event(), torch.cuda.Event()
+        ev0.record(main)
+        side.wait_event(ev0)
+        sla.hstu_sla_bwd_prepare(g["q"], g["offs"], g["nts"], workspace=ws, stream=side, **kw)
+        ev1.record(side)
+        main.wait_event(ev1)
+        dq, dk, dv = sla.hstu_sla_bwd(g["dout"], g["q"], g["k"], g["v"], g["offs"], g["nts"],
+                                      workspace=ws, prepared=True, **kw)
+        torch.cuda.synchronize()
+        assert sla.hstu_sla_get_error(ws) == 0
+        assert torch.equal(dk, dk0) and torch.equal(dv, dv0)
+        assert_close("dq", dq, rq)
+        assert_close("dk", dk, rk)
+        assert_close("dv", dv, rv)
+
+
 def test_mid_full_tensor():
     """The mid-length training batch (32 sequences of 1K-4K tokens, 4 x 128
     heads, K1 256, K2 64) compared element by element over the whole jagged
