@@ -57,6 +57,11 @@ CASES = {
     # head_dim 64 and 32 take the two-pass backward
     "ragged_d64": dict(lengths=[190, 77], nt=9, d=64),
     "ragged_d32": dict(lengths=[250, 33, 5], nt=4, d=32),
+    # long sequences whose prefix key tiles (one, two, three of them via K2)
+    # are seen by thousands of rows, last tile ragged
+    "long_prefix1_d128": dict(lengths=[8192 + 37, 5], nt=12),
+    "long_prefix2_d128": dict(lengths=[40, 10001], nt=7, K2=200),
+    "long_prefix3_d128": dict(lengths=[8200], nt=3, K2=300),
 }
 
 

@@ -107,6 +107,25 @@ def test_repeat_calls_reproducible(d):
         assert torch.equal(q1, q2)
 
 
+def test_long_prefix_units():
+    """Sequences of ~8K tokens whose prefix key tiles (one or two of them, via
+    K2) are each seen by every later row: one backward unit sweeps thousands
+    of query steps.  Every tensor against the oracle, dk / dv bitwise
+    repeatable; lengths ragged against the 64-row steps."""
+    for K2 in (100, 250):
+        b = _edge_batch(lengths=[8192 + 77, 8191, 2 * 2048 * 2 + 1], nt=20, K1=64, K2=K2, ctx=6,
+                        seed=23)
+        g = to_gpu(b)
+        dq, dk, dv = gpu_bwd(b, g)
+        p = oracle_problem(b)
+        rq, rk, rv = p.bwd(b.q, b.k, b.v, b.dout)
+        assert_close("dq", dq, rq)
+        assert_close("dk", dk, rk)
+        assert_close("dv", dv, rv)
+        _, dk2, dv2 = gpu_bwd(b, g)
+        assert torch.equal(dk, dk2) and torch.equal(dv, dv2)
+
+
 def test_backward_reuses_a_workspace():
     """One workspace reused across backward calls (same batch, a larger one,
     the first again) gives the oracle's results every time."""
