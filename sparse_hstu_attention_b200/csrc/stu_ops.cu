@@ -50,86 +50,86 @@ using sm100::silu_grad;
 // With yq set, also writes the row in E4M3 with a per-row scale: the FP8
 // quantization fused into the norm that precedes each projection ("Bending
 // the Scaling Law Curve...", section 4.2.2, mixed-precision training and
-// inference; Figure 4).  A warp takes kLnRows rows; every load (x, the gate,
-// gamma, beta) is issued before the first reduction, so their latencies
-// overlap instead of following one another.
-constexpr int kLnRows = 1;
+// inference; Figure 4).  A warp takes kLnRows rows and issues every row's
+// loads (x, the gate) before its first reduction, holding them as packed
+// bf16, so several rows' latencies overlap; gamma and beta are read where
+// they are used (the same 2 W floats for every warp: L1 hits).
+template <int NV>
+constexpr int ln_rows() { return NV >= 4 ? 2 : 4; }
+
+__device__ __forceinline__ void unpack8(const uint4 r, float* f) {
+  const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+  for (int h = 0; h < 4; ++h) {
+    f[2 * h] = __uint_as_float(w[h] << 16);
+    f[2 * h + 1] = __uint_as_float(w[h] & 0xFFFF0000u);
+  }
+}
+
+__device__ __forceinline__ void ldg8f(const float* p, float* f) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+  f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
 
 template <int NV, bool GATED>
 __global__ void __launch_bounds__(32 * kRowWarps) ln_fwd_kernel(const LnArgs a) {
   constexpr int W = NV * 256;
   const int lane = threadIdx.x & 31;
+  constexpr int kLnRows = ln_rows<NV>();
   const int64_t row0 = ((int64_t)blockIdx.x * kRowWarps + (threadIdx.x >> 5)) * kLnRows;
   if (row0 >= a.T) return;
-  float x[kLnRows][NV][8], u[GATED ? kLnRows : 1][NV][8];
+  uint4 xp[kLnRows][NV], up[GATED ? kLnRows : 1][NV];
 #pragma unroll
   for (int r = 0; r < kLnRows; ++r) {
-    const int64_t row = row0 + r < a.T ? row0 + r : row0;  // a missing second row repeats the first
+    const int64_t row = row0 + r < a.T ? row0 + r : row0;  // a missing row repeats the first
 #pragma unroll
     for (int v = 0; v < NV; ++v) {
-      load8(a.x + row * a.ldx + 8 * (lane + 32 * v), x[r][v]);
-      if (GATED) load8(a.u + row * a.ldu + 8 * (lane + 32 * v), u[GATED ? r : 0][v]);
+      xp[r][v] = *reinterpret_cast<const uint4*>(a.x + row * a.ldx + 8 * (lane + 32 * v));
+      if (GATED)
+        up[GATED ? r : 0][v] =
+            *reinterpret_cast<const uint4*>(a.u + row * a.ldu + 8 * (lane + 32 * v));
     }
   }
-  float gm[NV][8], bt[NV][8];
-#pragma unroll
-  for (int v = 0; v < NV; ++v) {
-    const float4* g4 = reinterpret_cast<const float4*>(a.gamma + 8 * (lane + 32 * v));
-    const float4* b4 = reinterpret_cast<const float4*>(a.beta + 8 * (lane + 32 * v));
-    const float4 ga = __ldg(g4), gb = __ldg(g4 + 1), ba = __ldg(b4), bb = __ldg(b4 + 1);
-    gm[v][0] = ga.x; gm[v][1] = ga.y; gm[v][2] = ga.z; gm[v][3] = ga.w;
-    gm[v][4] = gb.x; gm[v][5] = gb.y; gm[v][6] = gb.z; gm[v][7] = gb.w;
-    bt[v][0] = ba.x; bt[v][1] = ba.y; bt[v][2] = ba.z; bt[v][3] = ba.w;
-    bt[v][4] = bb.x; bt[v][5] = bb.y; bt[v][6] = bb.z; bt[v][7] = bb.w;
-  }
-  float mean[kLnRows], rstd[kLnRows];
-#pragma unroll
-  for (int r = 0; r < kLnRows; ++r) {
-    float s = 0.f;
-#pragma unroll
-    for (int v = 0; v < NV; ++v)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) s += x[r][v][e];
-    mean[r] = s;
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-    for (int r = 0; r < kLnRows; ++r) mean[r] += __shfl_xor_sync(0xffffffffu, mean[r], o);
-#pragma unroll
-  for (int r = 0; r < kLnRows; ++r) {
-    mean[r] *= 1.0f / W;
-    float q = 0.f;
-#pragma unroll
-    for (int v = 0; v < NV; ++v)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) q += (x[r][v][e] - mean[r]) * (x[r][v][e] - mean[r]);
-    rstd[r] = q;
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-    for (int r = 0; r < kLnRows; ++r) rstd[r] += __shfl_xor_sync(0xffffffffu, rstd[r], o);
 #pragma unroll
   for (int r = 0; r < kLnRows; ++r) {
     const int64_t row = row0 + r;
     if (row >= a.T) break;
-    rstd[r] = rsqrtf(rstd[r] * (1.0f / W) + a.eps);
+    float x[NV][8];
+#pragma unroll
+    for (int v = 0; v < NV; ++v) unpack8(xp[r][v], x[v]);
+    float mean = 0.f;
+#pragma unroll
+    for (int v = 0; v < NV; ++v)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) mean += x[v][e];
+    mean = warp_sum(mean) * (1.0f / W);
+    float q = 0.f;
+#pragma unroll
+    for (int v = 0; v < NV; ++v)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) q += (x[v][e] - mean) * (x[v][e] - mean);
+    const float rstd = rsqrtf(warp_sum(q) * (1.0f / W) + a.eps);
     float amax = 0.f;
 #pragma unroll
     for (int v = 0; v < NV; ++v) {
       const int c = 8 * (lane + 32 * v);
+      float gm[8], bt[8], u[8];
+      ldg8f(a.gamma + c, gm);
+      ldg8f(a.beta + c, bt);
+      if (GATED) unpack8(up[GATED ? r : 0][v], u);
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        x[r][v][e] = (x[r][v][e] - mean[r]) * rstd[r] * gm[v][e] + bt[v][e];  // x now holds y
-        if (GATED) x[r][v][e] *= u[GATED ? r : 0][v][e];
+        x[v][e] = (x[v][e] - mean) * rstd * gm[e] + bt[e];  // x now holds y
+        if (GATED) x[v][e] *= u[e];
       }
-      store8(a.y + row * a.ldy + c, x[r][v]);
+      store8(a.y + row * a.ldy + c, x[v]);
       if (a.yq) {  // quantize what the bf16 output holds
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          x[r][v][e] = __bfloat162float(__float2bfloat16(x[r][v][e]));
-          amax = fmaxf(amax, fabsf(x[r][v][e]));
+          x[v][e] = __bfloat162float(__float2bfloat16(x[v][e]));
+          amax = fmaxf(amax, fabsf(x[v][e]));
         }
       }
     }
@@ -142,17 +142,17 @@ __global__ void __launch_bounds__(32 * kRowWarps) ln_fwd_kernel(const LnArgs a) 
       for (int v = 0; v < NV; ++v) {
         const int c = 8 * (lane + 32 * v);
         uint2 w;
-        w.x = sm100::pack_e4m3x2(x[r][v][0] * inv, x[r][v][1] * inv) |
-              (sm100::pack_e4m3x2(x[r][v][2] * inv, x[r][v][3] * inv) << 16);
-        w.y = sm100::pack_e4m3x2(x[r][v][4] * inv, x[r][v][5] * inv) |
-              (sm100::pack_e4m3x2(x[r][v][6] * inv, x[r][v][7] * inv) << 16);
+        w.x = sm100::pack_e4m3x2(x[v][0] * inv, x[v][1] * inv) |
+              (sm100::pack_e4m3x2(x[v][2] * inv, x[v][3] * inv) << 16);
+        w.y = sm100::pack_e4m3x2(x[v][4] * inv, x[v][5] * inv) |
+              (sm100::pack_e4m3x2(x[v][6] * inv, x[v][7] * inv) << 16);
         *reinterpret_cast<uint2*>(a.yq + row * a.ldyq + c) = w;
       }
       if (lane == 0) a.yscale[row] = scale;
     }
     if (lane == 0) {
-      a.mean[row] = mean[r];
-      a.rstd[row] = rstd[r];
+      a.mean[row] = mean;
+      a.rstd[row] = rstd;
     }
   }
 }
@@ -194,14 +194,15 @@ __global__ void __launch_bounds__(256) quant_wt_kernel(const bf16* W, int64_t ld
 
 // Backward of the above.  Plain: dx = resid_grad + LN'(dy * gamma).
 // Gated: dz = dy * u, du = dy * z (times SiLU'(pre_u), since the gate is a
-// SiLU output), dx = LN'(dz * gamma).  Two passes over each row (the second
-// re-reads x, dy, u from L1 instead of keeping them in registers, so many
-// warps fit per SM); dgamma / dbeta (and, gated, the column sums of du: the
+// SiLU output), dx = LN'(dz * gamma).  Two passes over each row, both from
+// registers: every load of the row (x, dy, the gate and its pre-activation,
+// the residual gradient) is issued first and held as packed bf16, so a row
+// costs one memory latency; dgamma / dbeta (and, gated, the column sums of du: the
 // gate's bias gradient) accumulate in shared memory over the rows a block
 // visits (per warp, each lane updating only its own columns, for W <= 512;
 // shared atomics beyond), then once per block and column in global memory.
 template <int NV, bool GATED>
-__global__ void __launch_bounds__(32 * kRowWarps, GATED ? 2 : 4) ln_bwd_kernel(const LnArgs a) {
+__global__ void __launch_bounds__(32 * kRowWarps, GATED ? 2 : 3) ln_bwd_kernel(const LnArgs a) {
   constexpr int W = NV * 256;
   constexpr bool kPerWarp = NV <= 2;
   constexpr int kAcc = kPerWarp ? kRowWarps : 1;
@@ -238,17 +239,30 @@ __global__ void __launch_bounds__(32 * kRowWarps, GATED ? 2 : 4) ln_bwd_kernel(c
   const int64_t nwarps = (int64_t)gridDim.x * kRowWarps;
   for (int64_t row = (int64_t)blockIdx.x * kRowWarps + (threadIdx.x >> 5); row < a.T;
        row += nwarps) {
+    // every load of the row first, held as packed bf16 for both passes
+    uint4 xp[NV], dyp[NV], up[GATED ? NV : 1], pup[GATED ? NV : 1], rp[NV];
+#pragma unroll
+    for (int v = 0; v < NV; ++v) {
+      const int c = 8 * (lane + 32 * v);
+      xp[v] = *reinterpret_cast<const uint4*>(a.x + row * a.ldx + c);
+      dyp[v] = *reinterpret_cast<const uint4*>(a.dy + row * a.lddy + c);
+      if (GATED) {
+        up[GATED ? v : 0] = *reinterpret_cast<const uint4*>(a.u + row * a.ldu + c);
+        pup[GATED ? v : 0] = *reinterpret_cast<const uint4*>(a.pre_u + row * a.ldpu + c);
+      }
+      if (a.resid_grad) rp[v] = *reinterpret_cast<const uint4*>(a.resid_grad + row * a.ldr + c);
+    }
     const float mean = a.mean[row], rstd = a.rstd[row];
     float s1 = 0.f, s2 = 0.f;
-#pragma unroll 1
+#pragma unroll
     for (int v = 0; v < NV; ++v) {
       const int c = 8 * (lane + 32 * v);
       float x[8], dy[8], u[8], pu[8], du[8], tg[8], tb[8];
-      load8(a.x + row * a.ldx + c, x);
-      load8(a.dy + row * a.lddy + c, dy);
+      unpack8(xp[v], x);
+      unpack8(dyp[v], dy);
       if (GATED) {
-        load8(a.u + row * a.ldu + c, u);
-        load8(a.pre_u + row * a.ldpu + c, pu);
+        unpack8(up[GATED ? v : 0], u);
+        unpack8(pup[GATED ? v : 0], pu);
       }
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
@@ -302,14 +316,14 @@ __global__ void __launch_bounds__(32 * kRowWarps, GATED ? 2 : 4) ln_bwd_kernel(c
       }
     }
     const float m1 = warp_sum(s1) * (1.0f / W), m2 = warp_sum(s2) * (1.0f / W);
-#pragma unroll 1
+#pragma unroll
     for (int v = 0; v < NV; ++v) {
       const int c = 8 * (lane + 32 * v);
       float x[8], dy[8], u[8], dx[8], r[8];
-      load8(a.x + row * a.ldx + c, x);
-      load8(a.dy + row * a.lddy + c, dy);
-      if (GATED) load8(a.u + row * a.ldu + c, u);
-      if (a.resid_grad) load8(a.resid_grad + row * a.ldr + c, r);
+      unpack8(xp[v], x);
+      unpack8(dyp[v], dy);
+      if (GATED) unpack8(up[GATED ? v : 0], u);
+      if (a.resid_grad) unpack8(rp[v], r);
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         const float xh = (x[e] - mean) * rstd;
@@ -438,9 +452,10 @@ __global__ void __launch_bounds__(256) trunc_rows_kernel(const bf16* src, int64_
 
 cudaError_t launch_ln_fwd(const LnArgs& a, bool gated, cudaStream_t st) {
   if (a.T == 0) return cudaSuccess;
-  const int grid = (int)((a.T + kRowWarps * kLnRows - 1) / (kRowWarps * kLnRows));
 #define HSTU_LN(NV)                                                                     \
   if (a.W == NV * 256) {                                                                \
+    constexpr int rows = kRowWarps * ln_rows<NV>();                                     \
+    const int grid = (int)((a.T + rows - 1) / rows);                                    \
     if (gated) ln_fwd_kernel<NV, true><<<grid, 32 * kRowWarps, 0, st>>>(a);             \
     else ln_fwd_kernel<NV, false><<<grid, 32 * kRowWarps, 0, st>>>(a);                  \
     return cudaGetLastError();                                                          \
@@ -462,8 +477,8 @@ template <int NV, bool GATED>
 cudaError_t launch_ln_bwd_t(const LnArgs& a, cudaStream_t st) {
   constexpr int W = NV * 256;
   constexpr int kAcc = NV <= 2 ? kRowWarps : 1;
-  // dynamic shared memory for the gated form only; its carveout keeps the
-  // rest of the SM's 256 KB as L1, which the second pass over a row reads
+  // dynamic shared memory for the gated form only (its carveout: what two
+  // blocks need, the rest of the SM's 256 KB stays L1)
   constexpr int bytes = GATED ? (2 + 3 * kAcc) * W * (int)sizeof(float) : 0;
   if (GATED) {
     cudaError_t e = cudaFuncSetAttribute(ln_bwd_kernel<NV, GATED>,
