@@ -832,7 +832,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // (0 Q, 1 K, 2 V; ch = H * D / 8 threads each, a multiple of 32, so parts are
 // warp-uniform), columns [8 (j % ch), +8); a block takes a contiguous range
 // of rows.
-__global__ void __launch_bounds__(384) silu_qkv_kernel(const AttnArgs a, float scale) {
+__global__ void __launch_bounds__(384, 2) silu_qkv_kernel(const AttnArgs a, float scale) {
   const int HD = a.H * D, ch = HD / 8;
   const int j = threadIdx.x;
   const int part = j / ch;
@@ -845,38 +845,59 @@ __global__ void __launch_bounds__(384) silu_qkv_kernel(const AttnArgs a, float s
   bf16* g = part == 0 ? a.dq : part == 1 ? a.dk : a.dv;
   const int64_t g_rs = part == 0 ? a.dq_rs : part == 1 ? a.dk_rs : a.dv_rs;
   float sum[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-  for (int64_t t = r0; t < r1; ++t) {
-    float x[8];
-    if (part == 0) {
-      const float4* src = reinterpret_cast<const float4*>(a.dqacc + ((int64_t)h * T + t) * D + cd);
-      const float4 x0 = __ldcs(src), x1 = __ldcs(src + 1);
-      x[0] = x0.x * scale; x[1] = x0.y * scale; x[2] = x0.z * scale; x[3] = x0.w * scale;
-      x[4] = x1.x * scale; x[5] = x1.y * scale; x[6] = x1.z * scale; x[7] = x1.w * scale;
-    } else {
-      const uint4 w = *reinterpret_cast<const uint4*>(g + t * g_rs + cj);
-      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+  // kRows rows per round: every load of the round first (the gradient, as
+  // fp32 workspace or bf16, and the pre-activation), then the arithmetic and
+  // the stores, so that a thread keeps kRows rows of loads in flight
+  constexpr int kRows = 3;
+  for (int64_t t0 = r0; t0 < r1; t0 += kRows) {
+    // ga / gb: the two fp32 halves of a dQ row (Q part) as raw bits, or
+    // ga the bf16 dK / dV row (K, V parts)
+    uint4 ga[kRows], gb[kRows], pw[kRows];
+#pragma unroll
+    for (int k = 0; k < kRows; ++k) {
+      const int64_t t = t0 + k < r1 ? t0 + k : t0;  // a missing row repeats the first
+      if (part == 0) {
+        const uint4* src = reinterpret_cast<const uint4*>(a.dqacc + ((int64_t)h * T + t) * D + cd);
+        ga[k] = __ldcs(src);
+        gb[k] = __ldcs(src + 1);
+      } else {
+        ga[k] = *reinterpret_cast<const uint4*>(g + t * g_rs + cj);
+      }
+      pw[k] = __ldg(reinterpret_cast<const uint4*>(pre + t * a.pre_rs));
+    }
+#pragma unroll
+    for (int k = 0; k < kRows; ++k) {
+      const int64_t t = t0 + k;
+      if (t >= r1) break;
+      float x[8];
+      if (part == 0) {
+        x[0] = __uint_as_float(ga[k].x) * scale; x[1] = __uint_as_float(ga[k].y) * scale;
+        x[2] = __uint_as_float(ga[k].z) * scale; x[3] = __uint_as_float(ga[k].w) * scale;
+        x[4] = __uint_as_float(gb[k].x) * scale; x[5] = __uint_as_float(gb[k].y) * scale;
+        x[6] = __uint_as_float(gb[k].z) * scale; x[7] = __uint_as_float(gb[k].w) * scale;
+      } else {
+        const uint32_t ww[4] = {ga[k].x, ga[k].y, ga[k].z, ga[k].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          x[2 * e] = __uint_as_float(ww[e] << 16);
+          x[2 * e + 1] = __uint_as_float(ww[e] & 0xFFFF0000u);
+        }
+      }
+      const uint32_t pp[4] = {pw[k].x, pw[k].y, pw[k].z, pw[k].w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        x[2 * e] = __uint_as_float(ww[e] << 16);
-        x[2 * e + 1] = __uint_as_float(ww[e] & 0xFFFF0000u);
+        x[2 * e] *= silu_grad(__uint_as_float(pp[e] << 16));
+        x[2 * e + 1] *= silu_grad(__uint_as_float(pp[e] & 0xFFFF0000u));
       }
-    }
-    const uint4 pw = __ldg(reinterpret_cast<const uint4*>(pre + t * a.pre_rs));
-    const uint32_t pp[4] = {pw.x, pw.y, pw.z, pw.w};
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      x[2 * e] *= silu_grad(__uint_as_float(pp[e] << 16));
-      x[2 * e + 1] *= silu_grad(__uint_as_float(pp[e] & 0xFFFF0000u));
+      for (int e = 0; e < 8; ++e) sum[e] += x[e];
+      uint4 o;
+      o.x = pack_bf16x2(x[0], x[1]);
+      o.y = pack_bf16x2(x[2], x[3]);
+      o.z = pack_bf16x2(x[4], x[5]);
+      o.w = pack_bf16x2(x[6], x[7]);
+      *reinterpret_cast<uint4*>(g + t * g_rs + cj) = o;
     }
-#pragma unroll
-    for (int e = 0; e < 8; ++e) sum[e] += x[e];
-    uint4 o;
-    o.x = pack_bf16x2(x[0], x[1]);
-    o.y = pack_bf16x2(x[2], x[3]);
-    o.z = pack_bf16x2(x[4], x[5]);
-    o.w = pack_bf16x2(x[6], x[7]);
-    *reinterpret_cast<uint4*>(g + t * g_rs + cj) = o;
   }
   float4* dst = reinterpret_cast<float4*>(a.db_part + ((int64_t)blockIdx.x * 3 + part) * HD + cj);
   dst[0] = make_float4(sum[0], sum[1], sum[2], sum[3]);
