@@ -656,6 +656,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int b0t = rab_log_bucket(dlo + 1u) & 31;
             const int b1t = rab_log_bucket(dhi + 1u) & 31;
             const bool two = (uint32_t)(b1p - b0p) <= 1u && (uint32_t)(b1t - b0t) <= 1u;
+            const bool flat = b1p == b0p && b1t == b0t;
+            // every lane's buckets constant over the round: one bias for all
+            // its scores, and the round's total goes to one bin per table
+            // (the same values and order of additions as the two-bucket form)
+            auto rab_flat = [&](auto all_c) {
+              constexpr bool kAll = decltype(all_c)::value;
+              const float hb = rab_half_bias(tabp, tabt, b0p, b0t);
+              float acc = 0.f;
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const int k = 16 * r + 2 * e;
+                float ga, gb;
+                bwd_pair_bias(xs[2 * e], xs[2 * e + 1], xd[2 * e], xd[2 * e + 1], half_alpha2, hb,
+                              hb, pp[e], dd[e], ga, gb);
+                if (!kAll && !((bits >> k) & 1u)) ga = 0.f;
+                if (!kAll && !((bits >> (k + 1)) & 1u)) gb = 0.f;
+                acc += ga;
+                acc += gb;
+              }
+              if (acc != 0.f) {
+                run_add(run_p, sum_p, pend_p, psum_p, b0p, acc);
+                run_add(run_t, sum_t, pend_t, psum_t, 32 + b0t, acc);
+              }
+            };
             auto rab_round = [&](auto all_c, auto two_c) {
               constexpr bool kAll = decltype(all_c)::value;
               constexpr bool kTwo = decltype(two_c)::value;
@@ -704,7 +728,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (aht != 0.f) run_add(run_t, sum_t, pend_t, psum_t, 33 + b0t, aht);
               }
             };
-            if (!__all_sync(0xffffffffu, two))
+            if (__all_sync(0xffffffffu, flat)) {
+              if (full)
+                rab_flat(std::true_type{});
+              else
+                rab_flat(std::false_type{});
+            } else if (!__all_sync(0xffffffffu, two))
               rab_round(std::false_type{}, std::false_type{});
             else if (full)
               rab_round(std::true_type{}, std::true_type{});

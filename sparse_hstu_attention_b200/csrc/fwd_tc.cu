@@ -628,6 +628,34 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int jl = j0 + col + lane;
             const int32_t tjl = (A.ts && jl < r->L) ? __ldg(A.ts + s0 + jl) : 0;
             const int pb = imin(i, Lh) + 1 - (j0 + col);
+            // Both buckets are monotone in their difference, so the round's
+            // extreme differences bound them: the position over u_pos in
+            // [max(pb - 31, 1), max(pb, 1)], the time over the keys'
+            // timestamp range [tmin, tmax] (|ti - tj| is largest at an end
+            // and smallest at an end, or 0 inside).  When every lane's two
+            // buckets are constant over the round, one bias serves all 32
+            // scores (the same value the per-score path computes).
+            const int32_t tmin = __reduce_min_sync(0xffffffffu, tjl);
+            const int32_t tmax = __reduce_max_sync(0xffffffffu, tjl);
+            // |ti - tj| as an exact uint32; its bucket as the per-score path
+            // uses it (a shuffle lane: 2^32 - 1 lands in lane 31)
+            auto tbucket = [](uint32_t dlt) {
+              return dlt == 0xffffffffu ? 31 : rab_log_bucket(dlt + 1u);
+            };
+            const uint32_t da = __sad(ti, tmin, 0u), db = __sad(ti, tmax, 0u);
+            const uint32_t d_hi = da > db ? da : db;
+            const uint32_t d_lo = (ti >= tmin && ti <= tmax) ? 0u : (da < db ? da : db);
+            const int bp_hi = rab_log_bucket(rab_pos_u(pb, 0));
+            const int bt_hi = tbucket(d_hi);
+            const bool flat =
+                rab_log_bucket(rab_pos_u(pb, -31)) == bp_hi && tbucket(d_lo) == bt_hi;
+            if (__all_sync(0xffffffffu, flat)) {
+              const float hb = rab_half_bias(tabp, tabt, bp_hi, bt_hi);
+#pragma unroll
+              for (int e = 0; e < 16; ++e)
+                p[e] = silu_pair_bias(e < 8 ? c0[2 * e] : c1[2 * e - 16],
+                                      e < 8 ? c0[2 * e + 1] : c1[2 * e - 15], half_alpha2, hb, hb);
+            } else {
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
               const float ba = rab_half_bias(
@@ -638,6 +666,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   rab_log_bucket(rab_time_u(ti, __shfl_sync(0xffffffffu, tjl, 2 * e + 1))));
               p[e] = silu_pair_bias(e < 8 ? c0[2 * e] : c1[2 * e - 16],
                                     e < 8 ? c0[2 * e + 1] : c1[2 * e - 15], half_alpha2, ba, bb);
+            }
             }
           } else {
 #pragma unroll
