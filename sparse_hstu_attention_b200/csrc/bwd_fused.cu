@@ -599,18 +599,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       c.begin(r);
       for (int n = 0; n < nt; ++n, ++xc, c.next(r)) {
         const uint32_t b = xc & 1;
-        ok = warp_wait(bar(F_X_FULL + b), (xc >> 1) & 1, ws);
-        if (!ok) break;
-        tc_fence_after();
         const int c0 = c.j * kStr;  // first query row of this step
-        const bool full = tile_full(c0, c0 + kStr, t0, t0 + kRes, Lh, K1, K2e);
-        const uint32_t xs_addr = lane_base + kColX1 + b * 64 + col;
-        const uint32_t xd_addr = lane_base + kColX2 + b * 64 + col;
-        const uint32_t dsr = ds_row + b * DSTILE;
-        // Fully visible tiles skip the mask; others clear invisible entries by
-        // one bit test against this key's visibility mask of the chunk's rows.
-        const uint32_t bits = full ? 0xFFFFFFFFu : key_mask_bits(km, c0 + col);
-        // relative attention bias: the 16 queries' timestamps (lanes 0..15)
+        // relative attention bias: the 16 queries' timestamps (lanes 0..15),
+        // loaded before the wait for the scores
         int32_t tql = 0;
         bool tq_ok = false;  // this lane's query column is in the sequence
         if constexpr (RAB) {
@@ -618,6 +609,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           tq_ok = lane < 16 && ql < L;
           tql = (A.ts && tq_ok) ? __ldg(A.ts + s0 + ql) : 0;
         }
+        ok = warp_wait(bar(F_X_FULL + b), (xc >> 1) & 1, ws);
+        if (!ok) break;
+        tc_fence_after();
+        const bool full = tile_full(c0, c0 + kStr, t0, t0 + kRes, Lh, K1, K2e);
+        const uint32_t xs_addr = lane_base + kColX1 + b * 64 + col;
+        const uint32_t xd_addr = lane_base + kColX2 + b * 64 + col;
+        const uint32_t dsr = ds_row + b * DSTILE;
+        // Fully visible tiles skip the mask; others clear invisible entries by
+        // one bit test against this key's visibility mask of the chunk's rows.
+        const uint32_t bits = full ? 0xFFFFFFFFu : key_mask_bits(km, c0 + col);
         // One round of the chunk's 16 query columns: P^T (8 packed columns)
         // then dS^T (8) over the 16 score columns it read, and dS^T copied to
         // 16-byte chunks 2 chunk, +1 of this key's 128-byte swizzled row of

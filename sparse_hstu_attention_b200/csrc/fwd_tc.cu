@@ -605,10 +605,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int n = 0; n < nt; ++n, ++tc, c.next(r)) {
         if ((int)(tc & 1) != grp) continue;  // the other group's tile
         const uint32_t b = tc % kSBufs;
+        const int j0 = c.j * kBN;
+        // relative attention bias: this warp's 2 x 32 keys' timestamps, one
+        // per lane and round, loaded before the wait for the scores
+        int32_t tjr[2] = {0, 0};
+        if constexpr (RAB) {
+#pragma unroll
+          for (int sub = 0; sub < 2; ++sub) {
+            const int jl = j0 + half * 64 + sub * 32 + lane;
+            tjr[sub] = (A.ts && jl < r->L) ? __ldg(A.ts + s0 + jl) : 0;
+          }
+        }
         ok = warp_wait(bar(BAR_S_FULL + b), (tc / kSBufs) & 1, ws);
         if (!ok) break;
         tc_fence_after();
-        const int j0 = c.j * kBN;
         const bool full = tile_full(t0, t0 + kBM, j0, j0 + kBN, Lh, K1, K2e);
         // P = SiLU(alpha S) = h + h tanh(h) with h = alpha S / 2.  Tiles that
         // are entirely visible skip the mask; the others clear invisible
@@ -625,8 +635,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if constexpr (RAB) {
             // the 32 keys' timestamps, one per lane, then each score's bias:
             // key j = j0 + col + k has u_pos = max(pb - k, 1)
-            const int jl = j0 + col + lane;
-            const int32_t tjl = (A.ts && jl < r->L) ? __ldg(A.ts + s0 + jl) : 0;
+            const int32_t tjl = tjr[sub];
             const int pb = imin(i, Lh) + 1 - (j0 + col);
             // Both buckets are monotone in their difference, so the round's
             // extreme differences bound them: the position over u_pos in
