@@ -58,8 +58,8 @@ struct Cfg {
   // free again once the S MMA that read it has completed, which the score
   // buffer's S_FULL barrier already signals; that reuse needs kKSt <= 3 (a
   // buffer's next S cannot complete before the load that waits on it).
-  static constexpr int kKSt = D == 128 ? 2 : 3;
-  static constexpr int kVSt = D == 128 ? 3 : 4;
+  static constexpr int kKSt = 3;
+  static constexpr int kVSt = D == 128 ? 2 : 4;
   static constexpr int SW = D >= 64 ? 128 : 64;   // swizzle span (bytes) = one box row
   static constexpr int BOXW = SW / 2;             // bf16 elements per box row
   static constexpr int NB = D / BOXW;             // boxes per tile
