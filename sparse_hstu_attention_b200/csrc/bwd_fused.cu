@@ -681,6 +681,54 @@ __global__ void __launch_bounds__(kThreads, 1)
                 run_add(run_t, sum_t, pend_t, psum_t, 32 + b0t, acc);
               }
             };
+            // every lane's buckets take at most two neighbouring values: the
+            // upper position bucket starts at a column kp of the round (the
+            // position difference only grows along it), a score is in the
+            // upper time bucket from the difference thr_t on; the four table
+            // values are read once, and each score picks its bias and its
+            // upper-bucket sums by two predicates (the same values as the
+            // per-score form below)
+            auto rab_two = [&](auto all_c) {
+              constexpr bool kAll = decltype(all_c)::value;
+              const int kp =
+                  b1p != b0p
+                      ? (int)max((int64_t)0, ((int64_t)1 << (b0p + 1)) - 1 + rr - (c0 + col + 16 * r))
+                      : 16;
+              const bool two_t = b1t != b0t;
+              const uint32_t thr_t = (2u << b0t) - 1u;  // 2^(b0t + 1) - 1 (b0t <= 30 when used)
+              const float hp0 = __shfl_sync(0xffffffffu, tabp, b0p);
+              const float hp1 = __shfl_sync(0xffffffffu, tabp, b0p + 1);
+              const float ht0 = __shfl_sync(0xffffffffu, tabt, b0t);
+              const float ht1 = __shfl_sync(0xffffffffu, tabt, b0t + 1);
+              float acc = 0.f, ahp = 0.f, aht = 0.f;  // round total, upper buckets
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const int k = 16 * r + 2 * e;
+                const uint32_t da = __sad(__shfl_sync(0xffffffffu, tql, k), tj, 0u);
+                const uint32_t db = __sad(__shfl_sync(0xffffffffu, tql, k + 1), tj, 0u);
+                const bool upa = two_t && da >= thr_t, upb = two_t && db >= thr_t;
+                const bool ppa = 2 * e >= kp, ppb = 2 * e + 1 >= kp;
+                const float ba = (ppa ? hp1 : hp0) + (upa ? ht1 : ht0);
+                const float bb = (ppb ? hp1 : hp0) + (upb ? ht1 : ht0);
+                float ga, gb;
+                bwd_pair_bias(xs[2 * e], xs[2 * e + 1], xd[2 * e], xd[2 * e + 1], half_alpha2, ba,
+                              bb, pp[e], dd[e], ga, gb);
+                if (!kAll && !((bits >> k) & 1u)) ga = 0.f;
+                if (!kAll && !((bits >> (k + 1)) & 1u)) gb = 0.f;
+                acc += ga;
+                ahp += ppa ? ga : 0.f;
+                aht += upa ? ga : 0.f;
+                acc += gb;
+                ahp += ppb ? gb : 0.f;
+                aht += upb ? gb : 0.f;
+              }
+              // lower then upper bucket (an exact zero adds nothing)
+              const float lop = acc - ahp, lot = acc - aht;
+              if (lop != 0.f) run_add(run_p, sum_p, pend_p, psum_p, b0p, lop);
+              if (ahp != 0.f) run_add(run_p, sum_p, pend_p, psum_p, b0p + 1, ahp);
+              if (lot != 0.f) run_add(run_t, sum_t, pend_t, psum_t, 32 + b0t, lot);
+              if (aht != 0.f) run_add(run_t, sum_t, pend_t, psum_t, 33 + b0t, aht);
+            };
             auto rab_round = [&](auto all_c, auto two_c) {
               constexpr bool kAll = decltype(all_c)::value;
               constexpr bool kTwo = decltype(two_c)::value;
@@ -737,9 +785,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else if (!__all_sync(0xffffffffu, two))
               rab_round(std::false_type{}, std::false_type{});
             else if (full)
-              rab_round(std::true_type{}, std::true_type{});
+              rab_two(std::true_type{});
             else
-              rab_round(std::false_type{}, std::true_type{});
+              rab_two(std::false_type{});
           } else {
 #pragma unroll
             for (int e = 0; e < 8; ++e)
