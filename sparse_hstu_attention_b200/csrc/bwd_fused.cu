@@ -24,7 +24,7 @@
 //
 // Roles (persistent CTAs, one per SM; units handed out by an atomic counter,
 // prefix-key units first):
-//   warp 0      scheduler + TMA producer of the 3-stage Q / dO ring
+//   warp 0      scheduler + TMA producer of the 4-stage Q / dO ring
 //   warp 18     TMA loads of K and V (one buffer each)
 //   warp 1      TMEM allocation; the warp computes every MMA operand, one
 //               elected lane issues each batch of UMMAs and its commits
@@ -38,7 +38,7 @@
 //   X2(b) = [128+64b, 192+64b)  dP^T (fp32); then the step's dQ^T (lanes =
 //                               head-dim index, columns = query rows)
 //   ACC1 = [256, 384) dV,  ACC2 = [384, 512) dK
-// Shared memory (195 KB): K 32 KB, V 32 KB, Q and dO 3 x 16 KB each, dS^T
+// Shared memory (227 KB): K 32 KB, V 32 KB, Q and dO 4 x 16 KB each, dS^T
 // 2 x 16 KB (the B operand of the dQ MMA), barriers and the unit ring.
 #include <cudaTypedefs.h>
 #include <type_traits>
@@ -56,7 +56,7 @@ namespace {
 using namespace sm100;
 
 constexpr int D = 128;
-constexpr int kRes = 128, kStr = 64, kSt = 3, kPwWarps = 16, kUSlots = 4, kPwWarp0 = 2;
+constexpr int kRes = 128, kStr = 64, kSt = 4, kPwWarps = 16, kUSlots = 4, kPwWarp0 = 2;
 constexpr int kKvWarp = kPwWarp0 + kPwWarps;  // the K / V loader
 constexpr int kThreads = 32 * (kKvWarp + 1);
 constexpr uint32_t kColX1 = 0, kColX2 = 128, kColAcc1 = 256, kColAcc2 = 384, kTmemCols = 512;
@@ -68,8 +68,8 @@ constexpr int SBLK = kStr * SW;         // one box of a streamed tile
 constexpr int DSTILE = kRes * kStr * 2;  // dS^T: [128 keys][64 rows] bf16, one box
 constexpr int OFF_K = 0;
 // One K buffer: the next unit's K loads once the current unit's last dQ MMA
-// is done.  Measured against two buffers, the kernel ran ~1% faster (the
-// shared memory not taken is left to L1).
+// is done.  Measured against two buffers with three Q / dO stages, the
+// kernel ran ~1% faster; the 32 KB then went to a fourth Q / dO stage.
 constexpr int kKBufs = 1;
 constexpr int OFF_V = OFF_K + kKBufs * RTILE;
 constexpr int OFF_B1 = OFF_V + RTILE;
