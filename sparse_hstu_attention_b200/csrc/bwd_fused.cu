@@ -732,10 +732,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (lot != 0.f) run_add(run_t, sum_t, pend_t, psum_t, 32 + b0t, lot);
               if (aht != 0.f) run_add(run_t, sum_t, pend_t, psum_t, 33 + b0t, aht);
             };
-            auto rab_round = [&](auto all_c, auto two_c) {
-              constexpr bool kAll = decltype(all_c)::value;
-              constexpr bool kTwo = decltype(two_c)::value;
-              float acc = 0.f, ahp = 0.f, aht = 0.f;  // round total, upper buckets
+            // other rounds: each score extends its runs one by one
+            auto rab_round = [&]() {
 #pragma unroll
               for (int e = 0; e < 8; ++e) {
                 const int k = 16 * r + 2 * e;
@@ -751,33 +749,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float ga, gb;
                 bwd_pair_bias(xs[2 * e], xs[2 * e + 1], xd[2 * e], xd[2 * e + 1], half_alpha2, ba,
                               bb, pp[e], dd[e], ga, gb);
-                if constexpr (kTwo) {
-                  if (!kAll && !((bits >> k) & 1u)) ga = 0.f;
-                  if (!kAll && !((bits >> (k + 1)) & 1u)) gb = 0.f;
-                  acc += ga;
-                  ahp += bpa != b0p ? ga : 0.f;
-                  aht += bta != b0t ? ga : 0.f;
-                  acc += gb;
-                  ahp += bpb != b0p ? gb : 0.f;
-                  aht += btb != b0t ? gb : 0.f;
-                } else {
-                  if (kAll || ((bits >> k) & 1u)) {
-                    run_add(run_p, sum_p, pend_p, psum_p, bpa, ga);
-                    run_add(run_t, sum_t, pend_t, psum_t, 32 + bta, ga);
-                  }
-                  if (kAll || ((bits >> (k + 1)) & 1u)) {
-                    run_add(run_p, sum_p, pend_p, psum_p, bpb, gb);
-                    run_add(run_t, sum_t, pend_t, psum_t, 32 + btb, gb);
-                  }
+                if ((bits >> k) & 1u) {
+                  run_add(run_p, sum_p, pend_p, psum_p, bpa, ga);
+                  run_add(run_t, sum_t, pend_t, psum_t, 32 + bta, ga);
                 }
-              }
-              if constexpr (kTwo) {
-                // lower then upper bucket (an exact zero adds nothing)
-                const float lop = acc - ahp, lot = acc - aht;
-                if (lop != 0.f) run_add(run_p, sum_p, pend_p, psum_p, b0p, lop);
-                if (ahp != 0.f) run_add(run_p, sum_p, pend_p, psum_p, b0p + 1, ahp);
-                if (lot != 0.f) run_add(run_t, sum_t, pend_t, psum_t, 32 + b0t, lot);
-                if (aht != 0.f) run_add(run_t, sum_t, pend_t, psum_t, 33 + b0t, aht);
+                if ((bits >> (k + 1)) & 1u) {
+                  run_add(run_p, sum_p, pend_p, psum_p, bpb, gb);
+                  run_add(run_t, sum_t, pend_t, psum_t, 32 + btb, gb);
+                }
               }
             };
             if (__all_sync(0xffffffffu, flat)) {
@@ -786,7 +765,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               else
                 rab_flat(std::false_type{});
             } else if (!__all_sync(0xffffffffu, two))
-              rab_round(std::false_type{}, std::false_type{});
+              rab_round();
             else if (full)
               rab_two(std::true_type{});
             else
